@@ -1,0 +1,320 @@
+"""fp64 CPU oracle for Multi-Scale Retention (MSR).
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports, links or runs
+this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may call it.  It
+shares no code with the CUDA library (no kernels, headers, helpers, tables or
+constant generators); both sides only consume the same seeded inputs.
+
+Everything is plain numpy in float64, written for a reader to check against
+the pages by eye: no blocking, fusion or reordering beyond what each form
+states.  Sources (page title, section):
+
+* [RetNet-JA] abeam.tech summary of Sun et al. 2023, "Retentive Network: A
+  Successor to Transformer for Large Language Models":
+    - section 「Retentionは「内容に応じた参照」と「距離による忘却」を掛け合わせる」:
+      o_n gathers the values v_m of past positions m, weighted by the content
+      match Q_n K_m^T times the distance decay gamma^(n-m); future positions
+      are masked.
+    - section 「学習は並列、生成は状態更新」: the parallel form is Q K^T with a
+      combined causal + decay mask, applied to V; the recurrent form updates a
+      per-head state S_n = gamma S_(n-1) + K_n^T V_n and reads o_n = Q_n S_n;
+      the state shape is fixed by the head dimensions.
+    - section 「長文の学習にはチャンク再帰を使う」: chunkwise form; inside a chunk
+      the interaction is parallel, past chunks arrive through the state, which
+      is updated at the end of each chunk.
+    - section 「多時間尺度・ゲート・正規化で表現力を補う」: each head has its own
+      fixed decay rate; a Swish gate and a per-head GroupNorm follow.
+* [RetNet-abs] mlnews.online abstract page for arXiv 2307.08621, summary
+  bullets: retention outputs are normalised per head with GroupNorm before
+  the heads are concatenated; three computation modes.
+* [EulerStack] eulerwa.com EulerStack tutorial "3. RetNet 상세", sections
+  "어떻게 동작하나요?" and "장점": the three modes give the same value
+  (no error between training and inference forms).
+
+Readings taken where the pages are silent (each is pinned by a test in
+``tests/test_oracle.py``):
+
+1. No 1/sqrt(d_k) scale inside retention (the formula shows none).
+2. No normalisation of the decay mask or of the scores.
+3. The diagonal m = n is included (gamma^0 = 1); the recurrent form updates the
+   state before reading it.
+4. 0^0 = 1, so gamma = 0 leaves only the diagonal term.
+5. State orientation S in R^{d_k x d_v}: k_n is a 1 x d_k row, S = k^T v.
+6. Chunkwise form, derived from the definition by splitting the sum over m at
+   the chunk start s (row i = n - s of a chunk of length L):
+     O[i] = sum_{j<=i} gamma^(i-j) (q_i . k_j) v_j + gamma^(i+1) q_i S_prev
+     S    = gamma^L S_prev + sum_j gamma^(L-1-j) k_j^T v_j
+   since gamma^(n-m) = gamma^(i+1) * gamma^(s-1-m) for m < s.
+7. GroupNorm: groups = heads; statistics over the d_v channels of one head at
+   one token; biased variance; eps added to the variance; optional affine
+   weight/bias per channel (identity by default).
+8. Gate: swish(x) = x * sigmoid(x), applied to the already-projected gate G
+   after the GroupNorm: y = GN(o) * swish(g).
+9. Variable-length batches: every sequence starts from its own initial state
+   (zero by default) and is otherwise independent.
+
+Array conventions: per-head functions take ``q, k: [T, d_k]``, ``v: [T, d_v]``
+and a scalar ``gamma``; the ``msr_*`` wrappers take the token-major layout of
+the library boundary, ``q, k: [B, T, H, d_k]``, ``v: [B, T, H, d_v]``,
+``gamma: [H]``, and return ``o: [B, T, H, d_v]``.  States are
+``[H, d_k, d_v]`` per sequence.
+"""
+
+import numpy as np
+
+__all__ = [
+    "decay_mask",
+    "retention_brute",
+    "retention_parallel",
+    "retention_recurrent",
+    "retention_chunkwise",
+    "recurrent_step",
+    "group_norm_heads",
+    "swish",
+    "norm_gate",
+    "msr_parallel",
+    "msr_recurrent",
+    "msr_chunkwise",
+    "msr_chunkwise_varlen",
+    "msr_recurrent_step",
+]
+
+
+def _f64(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Per-head forms
+# ---------------------------------------------------------------------------
+
+def decay_mask(gamma, T):
+    """Causal decay mask D[n, m] = gamma^(n-m) for n >= m, else 0.
+
+    [RetNet-JA] 「学習は並列、生成は状態更新」: causal + decay mask of the parallel
+    form.  Built with an integer power per entry (never gamma^n * gamma^-m).
+    """
+    gamma = float(gamma)
+    idx = np.arange(T)
+    dist = idx[:, None] - idx[None, :]          # n - m
+    causal = dist >= 0
+    return np.where(causal, np.power(gamma, np.where(causal, dist, 0)), 0.0)
+
+
+def retention_brute(q, k, v, gamma):
+    """The definition, summed term by term (tiny inputs only).
+
+    o_n = sum_{m <= n} gamma^(n-m) (q_n . k_m) v_m
+    [RetNet-JA] 「Retentionは「内容に応じた参照」と「距離による忘却」を掛け合わせる」.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, dv = q.shape[0], v.shape[1]
+    gamma = float(gamma)
+    o = np.zeros((T, dv), dtype=np.float64)
+    for n in range(T):
+        for m in range(n + 1):
+            w = (gamma ** (n - m)) * float(np.dot(q[n], k[m]))
+            o[n] += w * v[m]
+    return o
+
+
+def retention_parallel(q, k, v, gamma):
+    """Parallel form O = (Q K^T * D) V.
+
+    [RetNet-JA] 「学習は並列、生成は状態更新」 (first paragraph).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    D = decay_mask(gamma, q.shape[0])
+    return ((q @ k.T) * D) @ v
+
+
+def recurrent_step(q_n, k_n, v_n, gamma, S):
+    """One step of the recurrent form: S <- gamma S + k_n^T v_n, then o_n = q_n S.
+
+    [RetNet-JA] 「学習は並列、生成は状態更新」 (second paragraph).  Returns
+    ``(o_n, S_new)``; ``S`` is not modified.
+    """
+    q_n, k_n, v_n = _f64(q_n), _f64(k_n), _f64(v_n)
+    S_new = float(gamma) * _f64(S) + np.outer(k_n, v_n)
+    return q_n @ S_new, S_new
+
+
+def retention_recurrent(q, k, v, gamma, state=None):
+    """Recurrent form over a whole sequence; returns ``(o, S_final)``."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, dk, dv = q.shape[0], q.shape[1], v.shape[1]
+    S = np.zeros((dk, dv)) if state is None else _f64(state).copy()
+    o = np.zeros((T, dv), dtype=np.float64)
+    for n in range(T):
+        o[n], S = recurrent_step(q[n], k[n], v[n], gamma, S)
+    return o, S
+
+
+def retention_chunkwise(q, k, v, gamma, chunk, state=None):
+    """Chunkwise recurrent form; returns ``(o, S_final)``.
+
+    [RetNet-JA] 「長文の学習にはチャンク再帰を使う」: parallel inside each chunk of
+    ``chunk`` tokens, past chunks through the state, state updated at the end
+    of each chunk.  Formulas: reading 6 of the module docstring.  Chunks start
+    at token 0; the last one may be shorter.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, dk, dv = q.shape[0], q.shape[1], v.shape[1]
+    if chunk < 1:
+        raise ValueError("chunk must be >= 1")
+    gamma = float(gamma)
+    S = np.zeros((dk, dv)) if state is None else _f64(state).copy()
+    o = np.zeros((T, dv), dtype=np.float64)
+    for s in range(0, T, chunk):
+        L = min(chunk, T - s)
+        Qc, Kc, Vc = q[s:s + L], k[s:s + L], v[s:s + L]
+        # inside the chunk: parallel form with its own decay mask
+        inner = ((Qc @ Kc.T) * decay_mask(gamma, L)) @ Vc
+        # past chunks: read of the carried state, decayed by gamma^(i+1)
+        read_scale = np.power(gamma, np.arange(1, L + 1))          # gamma^(i+1)
+        cross = read_scale[:, None] * (Qc @ S)
+        o[s:s + L] = inner + cross
+        # state update at the end of the chunk
+        zeta = np.power(gamma, np.arange(L - 1, -1, -1))           # gamma^(L-1-j)
+        S = (gamma ** L) * S + Kc.T @ (zeta[:, None] * Vc)
+    return o, S
+
+
+# ---------------------------------------------------------------------------
+# Per-head GroupNorm and Swish gate
+# ---------------------------------------------------------------------------
+
+def group_norm_heads(o, eps=1e-5, weight=None, bias=None):
+    """GroupNorm with one group per head, over the d_v channels of each token.
+
+    ``o: [..., H, d_v]``.  [RetNet-abs] summary bullets (per-head GroupNorm
+    before concatenation); [RetNet-JA] 「多時間尺度・ゲート・正規化で表現力を補う」.
+    Biased variance, eps added to the variance, optional per-channel affine
+    ``weight, bias: [H, d_v]``.
+    """
+    o = _f64(o)
+    mu = o.mean(axis=-1, keepdims=True)
+    var = ((o - mu) ** 2).mean(axis=-1, keepdims=True)
+    y = (o - mu) / np.sqrt(var + eps)
+    if weight is not None:
+        y = y * _f64(weight)
+    if bias is not None:
+        y = y + _f64(bias)
+    return y
+
+
+def swish(x):
+    """swish(x) = x * sigmoid(x) = x / (1 + exp(-x))."""
+    x = _f64(x)
+    return x / (1.0 + np.exp(-x))
+
+
+def norm_gate(o, g, eps=1e-5, weight=None, bias=None):
+    """y = GroupNorm_head(o) * swish(g); ``o: [..., H, d_v]``, ``g`` same shape.
+
+    [RetNet-JA] 「多時間尺度・ゲート・正規化で表現力を補う」 (Swish gate, GroupNorm).
+    """
+    g = _f64(g).reshape(np.shape(o))
+    return group_norm_heads(o, eps, weight, bias) * swish(g)
+
+
+# ---------------------------------------------------------------------------
+# Multi-head wrappers in the boundary layout [B, T, H, d]
+# ---------------------------------------------------------------------------
+
+def _heads(q, k, v, gamma):
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    gamma = np.asarray(gamma, dtype=np.float64).reshape(-1)
+    if q.ndim != 4 or k.shape != q.shape or v.shape[:3] != q.shape[:3]:
+        raise ValueError("expected q,k [B,T,H,dk] and v [B,T,H,dv]")
+    if gamma.shape[0] != q.shape[2]:
+        raise ValueError("gamma must have one entry per head")
+    return q, k, v, gamma
+
+
+def msr_parallel(q, k, v, gamma):
+    """Parallel form for every (batch, head); multi-scale: one gamma per head."""
+    q, k, v, gamma = _heads(q, k, v, gamma)
+    B, T, H, _ = q.shape
+    o = np.zeros(v.shape)
+    for b in range(B):
+        for h in range(H):
+            o[b, :, h] = retention_parallel(q[b, :, h], k[b, :, h], v[b, :, h], gamma[h])
+    return o
+
+
+def msr_recurrent(q, k, v, gamma, state=None):
+    """Recurrent form for every (batch, head); returns ``(o, S [B,H,dk,dv])``."""
+    q, k, v, gamma = _heads(q, k, v, gamma)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    o = np.zeros(v.shape)
+    S = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            s0 = None if state is None else state[b, h]
+            o[b, :, h], S[b, h] = retention_recurrent(
+                q[b, :, h], k[b, :, h], v[b, :, h], gamma[h], s0)
+    return o, S
+
+
+def msr_chunkwise(q, k, v, gamma, chunk, state=None):
+    """Chunkwise form for every (batch, head); returns ``(o, S [B,H,dk,dv])``."""
+    q, k, v, gamma = _heads(q, k, v, gamma)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    o = np.zeros(v.shape)
+    S = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            s0 = None if state is None else state[b, h]
+            o[b, :, h], S[b, h] = retention_chunkwise(
+                q[b, :, h], k[b, :, h], v[b, :, h], gamma[h], chunk, s0)
+    return o, S
+
+
+def msr_chunkwise_varlen(q, k, v, gamma, chunk, cu_seqlens, state=None, heads=None):
+    """Packed variable-length batch: ``q,k: [1, Ttot, H, dk]``, ``v: [1, Ttot, H, dv]``.
+
+    Sequence i occupies tokens ``cu_seqlens[i] : cu_seqlens[i+1]`` and is run
+    on its own from ``state[i]`` (zero if None), chunks aligned to its first
+    token (reading 9).  Returns ``(o [1,Ttot,H,dv], S [nseq,H,dk,dv])``.
+    ``heads`` optionally restricts the work to a list of head indices (other
+    heads' outputs are left at zero); used to sample large cases.
+    """
+    q, k, v, gamma = _heads(q, k, v, gamma)
+    if q.shape[0] != 1:
+        raise ValueError("packed layout has B = 1")
+    cu = [int(x) for x in cu_seqlens]
+    nseq = len(cu) - 1
+    _, T, H, dk = q.shape
+    dv = v.shape[3]
+    o = np.zeros(v.shape)
+    S = np.zeros((nseq, H, dk, dv))
+    hs = range(H) if heads is None else heads
+    for i in range(nseq):
+        a, b = cu[i], cu[i + 1]
+        for h in hs:
+            s0 = None if state is None else state[i, h]
+            if b > a:
+                o[0, a:b, h], S[i, h] = retention_chunkwise(
+                    q[0, a:b, h], k[0, a:b, h], v[0, a:b, h], gamma[h], chunk, s0)
+            else:
+                S[i, h] = 0.0 if s0 is None else _f64(s0)
+    return o, S
+
+
+def msr_recurrent_step(q, k, v, gamma, state):
+    """One decode step for a batch: ``q,k: [N,H,dk]``, ``v: [N,H,dv]``,
+    ``state: [N,H,dk,dv]``; returns ``(o [N,H,dv], state_new)``."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    gamma = np.asarray(gamma, dtype=np.float64).reshape(-1)
+    N, H, _ = q.shape
+    S = _f64(state)
+    o = np.zeros(v.shape)
+    S_new = np.zeros(S.shape)
+    for n in range(N):
+        for h in range(H):
+            o[n, h], S_new[n, h] = recurrent_step(q[n, h], k[n, h], v[n, h], gamma[h], S[n, h])
+    return o, S_new
