@@ -1,0 +1,224 @@
+/*
+ * retention.h — C ABI of libretention.so, the Multi-Scale Retention (MSR) hot
+ * path for NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  For one head with fixed decay gamma in [0, 1], queries
+ * q_n, keys k_n (rows of length d_k) and values v_n (rows of length d_v):
+ *
+ *     o_n = sum_{m <= n} gamma^(n-m) (q_n . k_m) v_m                      (R)
+ *
+ * Sources, by page title and section:
+ *   - abeam.tech summary of Sun et al. 2023, "Retentive Network: A Successor to
+ *     Transformer for Large Language Models":
+ *       「Retentionは「内容に応じた参照」と「距離による忘却」を掛け合わせる」 — (R):
+ *         values of past positions weighted by Q_n K_m^T and gamma^(n-m),
+ *         future masked;
+ *       「学習は並列、生成は状態更新」 — the parallel form (Q K^T * D) V with the
+ *         causal decay mask D_nm = gamma^(n-m) [n >= m], and the recurrent
+ *         form S_n = gamma S_(n-1) + K_n^T V_n, o_n = Q_n S_n;
+ *       「長文の学習にはチャンク再帰を使う」 — the chunkwise form: parallel inside
+ *         a chunk, past chunks through the state updated at each chunk end;
+ *       「多時間尺度・ゲート・正規化で表現力を補う」 — one fixed gamma per head,
+ *         a Swish gate and a per-head GroupNorm.
+ *   - mlnews.online abstract page for arXiv 2307.08621, summary bullets —
+ *     GroupNorm per head before the heads are concatenated.
+ *   - eulerwa.com tutorial "3. RetNet 상세", section "장점" — the three forms
+ *     give the same values.
+ *
+ * No 1/sqrt(d_k) factor is applied inside retention (the pages' formula has
+ * none); callers fold any scale into q or k.  Rotary position encoding, if
+ * used, is applied by the caller to q and k before these calls.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *   Memory:   every tensor argument is a DEVICE pointer on the current CUDA
+ *             device, owned by the caller, 16-byte aligned, densely packed in
+ *             the row-major layout stated below.  The library never frees or
+ *             keeps a caller pointer after the call returns.  `gamma` is the one
+ *             HOST array: it is read during the call and not retained.
+ *   Layout:   token-major.  q, k: [B, T, H, d_k]; v: [B, T, H, d_v];
+ *             outputs o / y: [B, T, H, d_v]; gate g: [B, T, H * d_v];
+ *             states: [B (or nseq, or N), H, d_k, d_v] float32, row = d_k index.
+ *   Dtypes:   RET_F32 (float) or RET_BF16 (bfloat16, stored as uint16).
+ *             bf16 inputs are multiplied on tensor cores with float32
+ *             accumulation; the carried state is always float32.
+ *   Gamma:    host double[H], each 0 <= gamma_h <= 1 (0^0 = 1: gamma = 0
+ *             keeps only the diagonal term q_n.k_n v_n).  H <= 64.
+ *   Streams:  every call only enqueues work on `stream` (a cudaStream_t; NULL
+ *             = the legacy default stream) and returns without synchronising.
+ *             The returned status covers argument validation and launch
+ *             errors; faults and time-outs detected on the device are
+ *             reported later by retention_check_device_error().
+ *   Errors:   on any status other than RET_OK nothing has been enqueued and no
+ *             output has been touched.  RET_ERR_UNSUPPORTED means the
+ *             arguments are valid but this build has no kernel for the shape
+ *             or dtype combination; there is no fallback path.
+ *   Aliasing: outputs must not overlap inputs, except that
+ *             retention_recurrent_step updates `state` in place by design.
+ */
+#ifndef RETENTION_H_
+#define RETENTION_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RETENTION_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define RET_API __attribute__((visibility("default")))
+#else
+#define RET_API
+#endif
+
+typedef struct CUstream_st* ret_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  RET_OK = 0,
+  RET_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, gamma out of [0,1] */
+  RET_ERR_UNSUPPORTED = 2,   /* valid request with no kernel in this build */
+  RET_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+  RET_ERR_TIMEOUT = 4,       /* a bounded device-side wait expired (from check_device_error) */
+  RET_ERR_WORKSPACE = 5,     /* workspace missing or smaller than the size query returned */
+  RET_ERR_DEVICE_DATA = 6    /* device-resident metadata (cu_seqlens) was inconsistent */
+} ret_status;
+
+typedef enum { RET_F32 = 0, RET_BF16 = 1 } ret_dtype;
+
+/*
+ * Per-head GroupNorm followed by the Swish gate (abeam.tech summary,
+ * 「多時間尺度・ゲート・正規化で表現力を補う」; mlnews.online abstract page,
+ * summary bullets).  For each token t and head h, over the d_v channels c:
+ *     mu = mean_c o[t,h,c];  var = mean_c (o[t,h,c] - mu)^2   (biased)
+ *     y[t,h,c] = ((o - mu) / sqrt(var + eps) * weight[h*d_v+c] + bias[h*d_v+c])
+ *                * g[t, h*d_v+c] * sigmoid(g[t, h*d_v+c])
+ */
+typedef struct {
+  const void*  g;        /* device gate [ntok, H*d_v], dtype g_dtype (required) */
+  ret_dtype    g_dtype;
+  const float* weight;   /* device [H*d_v] float32, or NULL for 1 */
+  const float* bias;     /* device [H*d_v] float32, or NULL for 0 */
+  float        eps;      /* added to the variance; must be >= 0 and finite */
+} ret_norm_gate;
+
+/* ABI version of the loaded library (RETENTION_ABI_VERSION at build time). */
+RET_API int retention_abi_version(void);
+
+/* Static, human-readable name of a status code. */
+RET_API const char* retention_status_string(ret_status status);
+
+/*
+ * Parallel form O = (Q K^T * D) V, D_nm = gamma_h^(n-m) for n >= m else 0
+ * (abeam.tech summary, 「学習は並列、生成は状態更新」).  Every (b, h) pair is an
+ * independent causal sequence of T tokens.
+ *   q, k:  [B,T,H,dk] in_dtype      v: [B,T,H,dv] in_dtype
+ *   o:     [B,T,H,dv] o_dtype (fully overwritten)
+ * Supported: dk, dv in 1..256; T >= 1; B*T*H*max(dk,dv) < 2^31.
+ * Returns RET_ERR_INVALID_ARG for null pointers, B,T,H,dk,dv < 1, H > 64 or
+ * gamma outside [0,1]; RET_ERR_UNSUPPORTED for larger head dims.
+ */
+RET_API ret_status retention_parallel_fwd(const void* q, const void* k, const void* v,
+                                  ret_dtype in_dtype, const double* gamma,
+                                  void* o, ret_dtype o_dtype,
+                                  int B, int T, int H, int dk, int dv,
+                                  ret_stream_t stream);
+
+/*
+ * Bytes of device workspace retention_chunkwise_fwd needs for these sizes
+ * (0 if the arguments are invalid).  The workspace holds the state entering
+ * every chunk; its contents need no initialisation and are scratch after the
+ * call.  `nseq` = 0 for the padded layout, else the number of packed
+ * sequences (then B must be 1 and T is the total token count).
+ */
+RET_API size_t retention_chunkwise_workspace_size(ret_dtype in_dtype, int chunk,
+                                          int B, int T, int H, int dk, int dv,
+                                          int nseq);
+
+/*
+ * Chunkwise recurrent form (abeam.tech summary, 「長文の学習にはチャンク再帰を
+ * 使う」), with an optional fused GroupNorm + Swish-gate epilogue.  For a
+ * chunk of L <= `chunk` tokens starting at token s (row i = n - s):
+ *     O[i] = sum_{j<=i} gamma^(i-j) (q_i . k_j) v_j + gamma^(i+1) q_i S_prev
+ *     S    = gamma^L S_prev + sum_j gamma^(L-1-j) k_j^T v_j
+ * which equals (R) exactly in real arithmetic for every chunk length.
+ *
+ *   q, k:  [B,T,H,dk] in_dtype      v: [B,T,H,dv] in_dtype
+ *   cu_seqlens: NULL for B independent sequences of T tokens each; otherwise
+ *          a DEVICE int32 [nseq+1] of packed sequence offsets (B must be 1,
+ *          cu_seqlens[0] = 0, non-decreasing, cu_seqlens[nseq] = T).  Each
+ *          sequence starts from its own state and its chunks start at its
+ *          first token; empty sequences are allowed.  If the device array
+ *          breaks these rules the kernels clamp every access to [0, T) and
+ *          raise RET_ERR_DEVICE_DATA through retention_check_device_error().
+ *   state_in:  [nseq or B, H, dk, dv] float32, or NULL for zeros.
+ *   state_out: [nseq or B, H, dk, dv] float32 final states, or NULL.  An empty
+ *          sequence's state_out equals its state_in (or zeros).
+ *   out:   [B,T,H,dv] o_dtype.  With ng == NULL it receives the retention
+ *          output o; with ng != NULL it receives y = GroupNorm(o) * swish(g).
+ *   workspace: device scratch of at least
+ *          retention_chunkwise_workspace_size(...) bytes, 256-byte aligned.
+ * Supported:
+ *   in_dtype RET_F32: dk, dv in 1..256, any chunk >= 1 (CUDA-core float32).
+ *   in_dtype RET_BF16: tensor-core kernels (tcgen05, TMEM accumulators), dk in
+ *          {64, 128, 256}, dv in {64, 128, 256, 512}, chunk in
+ *          {64, 128, 256, 512}.  Chunks shorter than 128 tokens are
+ *          evaluated as 128-token chunks, which yields the same result.
+ *   out dtype RET_F32 or RET_BF16; H <= 64; T*H*max(dk,dv) < 2^31.
+ */
+RET_API ret_status retention_chunkwise_fwd(const void* q, const void* k, const void* v,
+                                   ret_dtype in_dtype, const double* gamma,
+                                   int chunk,
+                                   const int32_t* cu_seqlens, int nseq,
+                                   const float* state_in, float* state_out,
+                                   void* out, ret_dtype out_dtype,
+                                   const ret_norm_gate* ng,
+                                   void* workspace, size_t workspace_bytes,
+                                   int B, int T, int H, int dk, int dv,
+                                   ret_stream_t stream);
+
+/*
+ * One recurrent decode step for N independent sequences (abeam.tech summary,
+ * 「学習は並列、生成は状態更新」): for every (n, h), in this order,
+ *     S <- gamma_h S + k^T v      (state updated in place)
+ *     o  = q S                     (read after the update)
+ *   q, k: [N,H,dk] in_dtype   v: [N,H,dv] in_dtype
+ *   state: [N,H,dk,dv] float32, read and overwritten
+ *   o: [N,H,dv] o_dtype
+ * Supported: dk in 1..1024, dv in 1..4096; the state streams through HBM once
+ * (read + write), the memory-bound part of generation.
+ */
+RET_API ret_status retention_recurrent_step(const void* q, const void* k, const void* v,
+                                    ret_dtype in_dtype, const double* gamma,
+                                    float* state, void* o, ret_dtype o_dtype,
+                                    int N, int H, int dk, int dv,
+                                    ret_stream_t stream);
+
+/*
+ * Standalone per-head GroupNorm + Swish gate (the epilogue that
+ * retention_chunkwise_fwd fuses when given `ng`).
+ *   o: [ntok, H, dv] o_dtype     y: [ntok, H, dv] y_dtype (may not alias o)
+ *   ng: gate, optional affine and eps as in ret_norm_gate (required).
+ * Supported: dv in 1..1024.
+ */
+RET_API ret_status msr_norm_gate(const void* o, ret_dtype o_dtype, const ret_norm_gate* ng,
+                         void* y, ret_dtype y_dtype, int ntok, int H, int dv,
+                         ret_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears this device's error word, which
+ * the kernels set instead of trapping: RET_ERR_TIMEOUT when a bounded
+ * wait inside a kernel gave up (the kernel then skipped its remaining work
+ * and released what it held), RET_ERR_DEVICE_DATA when cu_seqlens was
+ * inconsistent.  Returns RET_OK when no such event happened since the last
+ * call, RET_ERR_CUDA if the synchronisation itself failed.
+ */
+RET_API ret_status retention_check_device_error(ret_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RETENTION_H_ */

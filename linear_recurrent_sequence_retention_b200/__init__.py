@@ -2,19 +2,8 @@
 
 The compute lives in ``libretention.so`` (hand-written CUDA kernels behind a
 C ABI declared in ``include/retention.h``); ``ops`` is the thin ctypes binding
-that marshals torch tensors into those calls.  Importing this package does
-not load the library; the first call into ``ops`` does, and raises if the
-library has not been built.
+that marshals torch tensors into those calls, ``workloads`` draws the seeded
+synthetic inputs, ``build`` compiles the library.  Importing this package
+does not load the library; the first call into ``ops`` does, and raises if
+the library has not been built.
 """
-
-__all__ = ["ops", "workloads"]
-
-
-def __getattr__(name):
-    if name == "ops":
-        from . import ops
-        return ops
-    if name == "workloads":
-        from . import workloads
-        return workloads
-    raise AttributeError(name)

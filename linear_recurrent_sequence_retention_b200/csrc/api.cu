@@ -1,0 +1,263 @@
+// C ABI of libretention.so (declared in include/retention.h): argument
+// validation, per-head decay constants, the per-device error word, and
+// dispatch to the kernels.  No entry point allocates device memory: the
+// chunkwise forward takes a caller-owned workspace sized by
+// retention_chunkwise_workspace_size().
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "retention.h"
+#include "launch.h"
+
+namespace {
+
+using ret::DType;
+
+// Per-device error word; kernels atomicOr ret::kErr* bits into it instead of
+// trapping.  Host code needs the device address, resolved once per device.
+__device__ unsigned int g_error_word;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_err_mu;
+unsigned* g_err_addr[kMaxDevices] = {};
+
+unsigned* error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_err_mu);
+  if (g_err_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+    g_err_addr[dev] = static_cast<unsigned*>(p);
+  }
+  return g_err_addr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool dtype_ok(ret_dtype t) { return t == RET_F32 || t == RET_BF16; }
+DType dt(ret_dtype t) { return t == RET_F32 ? DType::F32 : DType::BF16; }
+
+bool make_decay(const double* gamma, int H, ret::HeadDecay* d) {
+  if (gamma == nullptr || H < 1 || H > ret::kMaxHeads) return false;
+  std::memset(d, 0, sizeof(*d));
+  for (int h = 0; h < H; ++h) {
+    double g = gamma[h];
+    if (!std::isfinite(g) || g < 0.0 || g > 1.0) return false;
+    d->gamma[h] = static_cast<float>(g);
+    if (g == 0.0) {
+      d->zero_mask |= 1ull << h;
+      d->log2g[h] = 0.f;
+    } else {
+      d->log2g[h] = static_cast<float>(std::log2(g));
+    }
+  }
+  return true;
+}
+
+ret_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RET_OK : RET_ERR_CUDA; }
+
+bool fits_int(long long x) { return x >= 0 && x < (1ll << 31); }
+
+struct ChunkPlan {
+  ret::SeqLayout L;
+  bool tc;
+  size_t elem;
+  size_t meta;
+  long long slots;
+  size_t bytes;
+};
+
+// Shared by the size query and the forward call.
+ret_status plan_chunkwise(ret_dtype in_dtype, int chunk, int B, int T, int H, int dk, int dv,
+                          int nseq, const int32_t* cu, ChunkPlan* p) {
+  if (!dtype_ok(in_dtype) || chunk < 1 || H < 1 || H > ret::kMaxHeads || dk < 1 || dv < 1)
+    return RET_ERR_INVALID_ARG;
+  const bool varlen = nseq > 0;
+  if (nseq < 0) return RET_ERR_INVALID_ARG;
+  if (varlen) {
+    if (B != 1 || T < 0) return RET_ERR_INVALID_ARG;
+  } else if (B < 1 || T < 1) {
+    return RET_ERR_INVALID_ARG;
+  }
+  const long long Ttot = varlen ? T : static_cast<long long>(B) * T;
+  const int dmax = dk > dv ? dk : dv;
+  if (!fits_int(Ttot * H * static_cast<long long>(dmax)) || !fits_int(Ttot + chunk))
+    return RET_ERR_INVALID_ARG;
+  int ce = chunk;
+  if (in_dtype == RET_BF16) {
+    if (!ret::chunkwise_tc_supported(dk, dv, chunk)) return RET_ERR_UNSUPPORTED;
+    ce = ret::chunkwise_tc_chunk(chunk);
+    p->tc = true;
+    p->elem = 4;   // two bf16 planes per state element (hi and lo parts)
+  } else {
+    if (dk > 256 || dv > 256) return RET_ERR_UNSUPPORTED;
+    p->tc = false;
+    p->elem = 4;
+  }
+  p->L.cu = varlen ? cu : nullptr;
+  p->L.nseq = varlen ? nseq : B;
+  p->L.T = varlen ? 0 : T;
+  p->L.Ttot = static_cast<int>(Ttot);
+  p->L.chunk = ce;
+  p->meta = ret::chunkwise_meta_bytes(p->L.nseq);
+  // one slot per chunk; a packed batch has at most ceil(Ttot/ce) + nseq chunks
+  p->slots = varlen ? (Ttot + ce - 1) / ce + nseq
+                    : static_cast<long long>(B) * ((T + ce - 1) / ce);
+  p->L.nslots = p->slots;
+  p->bytes = p->meta + static_cast<size_t>(p->slots) * H * dk * dv * p->elem;
+  return RET_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int retention_abi_version(void) { return RETENTION_ABI_VERSION; }
+
+const char* retention_status_string(ret_status s) {
+  switch (s) {
+    case RET_OK: return "RET_OK";
+    case RET_ERR_INVALID_ARG: return "RET_ERR_INVALID_ARG: invalid argument";
+    case RET_ERR_UNSUPPORTED: return "RET_ERR_UNSUPPORTED: no kernel for this shape/dtype";
+    case RET_ERR_CUDA: return "RET_ERR_CUDA: CUDA call failed";
+    case RET_ERR_TIMEOUT: return "RET_ERR_TIMEOUT: a bounded device wait expired";
+    case RET_ERR_WORKSPACE: return "RET_ERR_WORKSPACE: workspace missing or too small";
+    case RET_ERR_DEVICE_DATA: return "RET_ERR_DEVICE_DATA: inconsistent cu_seqlens";
+  }
+  return "unknown ret_status";
+}
+
+ret_status retention_parallel_fwd(const void* q, const void* k, const void* v,
+                                  ret_dtype in_dtype, const double* gamma, void* o,
+                                  ret_dtype o_dtype, int B, int T, int H, int dk, int dv,
+                                  ret_stream_t stream) {
+  if (!q || !k || !v || !o || !dtype_ok(in_dtype) || !dtype_ok(o_dtype)) return RET_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || H < 1 || dk < 1 || dv < 1) return RET_ERR_INVALID_ARG;
+  ret::HeadDecay dec;
+  if (!make_decay(gamma, H, &dec)) return RET_ERR_INVALID_ARG;
+  const int dmax = dk > dv ? dk : dv;
+  if (!fits_int(static_cast<long long>(B) * T * H * dmax)) return RET_ERR_INVALID_ARG;
+  if (dk > 256 || dv > 256) return RET_ERR_UNSUPPORTED;
+  return cuda_status(ret::launch_parallel_simt(q, k, v, dt(in_dtype), o, dt(o_dtype), B, T, H,
+                                               dk, dv, dec, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t retention_chunkwise_workspace_size(ret_dtype in_dtype, int chunk, int B, int T, int H,
+                                          int dk, int dv, int nseq) {
+  ChunkPlan p;
+  if (plan_chunkwise(in_dtype, chunk, B, T, H, dk, dv, nseq, nullptr, &p) != RET_OK) return 0;
+  return p.bytes;
+}
+
+ret_status retention_chunkwise_fwd(const void* q, const void* k, const void* v,
+                                   ret_dtype in_dtype, const double* gamma, int chunk,
+                                   const int32_t* cu_seqlens, int nseq,
+                                   const float* state_in, float* state_out,
+                                   void* out, ret_dtype out_dtype, const ret_norm_gate* ng,
+                                   void* workspace, size_t workspace_bytes,
+                                   int B, int T, int H, int dk, int dv,
+                                   ret_stream_t stream) {
+  const bool varlen = cu_seqlens != nullptr;
+  if (varlen != (nseq > 0)) return RET_ERR_INVALID_ARG;
+  ChunkPlan p;
+  ret_status st = plan_chunkwise(in_dtype, chunk, B, T, H, dk, dv, varlen ? nseq : 0,
+                                 cu_seqlens, &p);
+  if (st != RET_OK) return st;
+  const bool has_tokens = p.L.Ttot > 0;
+  if (has_tokens && (!q || !k || !v || !out)) return RET_ERR_INVALID_ARG;
+  if (!dtype_ok(out_dtype)) return RET_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, out, state_in, state_out, cu_seqlens};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return RET_ERR_INVALID_ARG;
+  ret::HeadDecay dec;
+  if (!make_decay(gamma, H, &dec)) return RET_ERR_INVALID_ARG;
+  const void* g = nullptr;
+  DType g_t = DType::F32;
+  const float* gw = nullptr;
+  const float* gb = nullptr;
+  float eps = 0.f;
+  if (ng) {
+    if (!ng->g || !dtype_ok(ng->g_dtype) || !aligned16(ng->g)) return RET_ERR_INVALID_ARG;
+    if (!std::isfinite(ng->eps) || ng->eps < 0.f) return RET_ERR_INVALID_ARG;
+    g = ng->g;
+    g_t = dt(ng->g_dtype);
+    gw = ng->weight;
+    gb = ng->bias;
+    eps = ng->eps;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < p.bytes)
+    return RET_ERR_WORKSPACE;
+  ret::ChunkWorkspace ws;
+  ws.chunk_base = static_cast<int32_t*>(workspace);
+  ws.states = static_cast<char*>(workspace) + p.meta;
+  ws.nslots = p.slots;
+  unsigned* err = error_word();
+  if (!err) return RET_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = ret::launch_chunk_prep(p.L, ws, err, s);
+  if (e != cudaSuccess) return RET_ERR_CUDA;
+  if (p.tc)
+    e = ret::launch_chunkwise_tc(q, k, v, p.L, state_in, state_out, out, dt(out_dtype), g, g_t,
+                                 gw, gb, eps, ng != nullptr, ws, H, dk, dv, dec, err, s);
+  else
+    e = ret::launch_chunkwise_simt(q, k, v, dt(in_dtype), p.L, state_in, state_out, out,
+                                   dt(out_dtype), g, g_t, gw, gb, eps, ng != nullptr, ws, H, dk,
+                                   dv, dec, err, s);
+  return cuda_status(e);
+}
+
+ret_status retention_recurrent_step(const void* q, const void* k, const void* v,
+                                    ret_dtype in_dtype, const double* gamma, float* state,
+                                    void* o, ret_dtype o_dtype, int N, int H, int dk, int dv,
+                                    ret_stream_t stream) {
+  if (!q || !k || !v || !state || !o || !dtype_ok(in_dtype) || !dtype_ok(o_dtype))
+    return RET_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(o))
+    return RET_ERR_INVALID_ARG;
+  if (N < 1 || H < 1 || dk < 1 || dv < 1) return RET_ERR_INVALID_ARG;
+  ret::HeadDecay dec;
+  if (!make_decay(gamma, H, &dec)) return RET_ERR_INVALID_ARG;
+  if (dk > 1024 || dv > 4096) return RET_ERR_UNSUPPORTED;
+  if (static_cast<long long>(N) * H > 65535ll * 65535ll || N > 65535 || H > 65535)
+    return RET_ERR_UNSUPPORTED;
+  return cuda_status(ret::launch_decode_step(q, k, v, dt(in_dtype), state, o, dt(o_dtype), N, H,
+                                             dk, dv, dec, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ret_status msr_norm_gate(const void* o, ret_dtype o_dtype, const ret_norm_gate* ng, void* y,
+                         ret_dtype y_dtype, int ntok, int H, int dv, ret_stream_t stream) {
+  if (!o || !ng || !ng->g || !y || !dtype_ok(o_dtype) || !dtype_ok(y_dtype) ||
+      !dtype_ok(ng->g_dtype))
+    return RET_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(ng->g) || !aligned16(y)) return RET_ERR_INVALID_ARG;
+  if (ntok < 1 || H < 1 || dv < 1) return RET_ERR_INVALID_ARG;
+  if (!std::isfinite(ng->eps) || ng->eps < 0.f) return RET_ERR_INVALID_ARG;
+  if (!fits_int(static_cast<long long>(ntok) * H * dv)) return RET_ERR_INVALID_ARG;
+  if (dv > 1024) return RET_ERR_UNSUPPORTED;
+  return cuda_status(ret::launch_norm_gate(o, dt(o_dtype), ng->g, dt(ng->g_dtype), ng->weight,
+                                           ng->bias, ng->eps, y, dt(y_dtype), ntok, H, dv,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ret_status retention_check_device_error(ret_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return RET_ERR_CUDA;
+  unsigned* err = error_word();
+  if (!err) return RET_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpy(&word, err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return RET_ERR_CUDA;
+  if (word != 0) {
+    const unsigned zero = 0;
+    if (cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return RET_ERR_CUDA;
+  }
+  if (word & ret::kErrTimeout) return RET_ERR_TIMEOUT;
+  if (word & ret::kErrDeviceData) return RET_ERR_DEVICE_DATA;
+  return RET_OK;
+}
+
+}  // extern "C"

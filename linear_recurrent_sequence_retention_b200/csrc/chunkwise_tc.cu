@@ -1,0 +1,923 @@
+// Chunkwise retention forward on tcgen05 tensor cores (bf16 in, f32 accumulate).
+//
+// The chunkwise form (abeam.tech summary of Sun et al. 2023, section
+// 「長文の学習にはチャンク再帰を使う」): inside a chunk of L tokens the parallel
+// form; across chunks a decayed read of the state carried from the previous
+// chunk; at the chunk end the state is updated.  Row i of chunk c:
+//     O[i] = sum_{j<=i} gamma^(i-j) (q_i.k_j) v_j  +  gamma^(i+1) q_i S_(c-1)
+//     S_c  = gamma^L S_(c-1) + sum_j gamma^(L-1-j) k_j^T v_j
+//
+// Two kernels, both warp-specialised (warp 0: TMA producer, warp 1: TMEM
+// allocation + MMA issue, warps 2-5: one warpgroup that owns the 128 TMEM
+// lanes):
+//
+//  state_kernel   one CTA per (sequence, head, 128 rows of d_k, NS columns of
+//                 d_v).  Walks the sequence's chunks in order with the state
+//                 block in TMEM (f32).  Before each chunk it stores the state
+//                 entering the chunk, rounded to bf16, in the workspace slot of
+//                 that chunk, scales TMEM by gamma^L, then accumulates
+//                 (zeta * K)^T V with the MMA (zeta_j = gamma^(L-1-j) applied to
+//                 the K rows in shared memory).  The final f32 state goes to
+//                 state_out.
+//
+//  output_kernel  one CTA per (chunk, 128-row block r of the chunk, head,
+//                 NV-wide part of d_v); the two halves of d_v = 512 form a
+//                 2-CTA cluster that exchanges the GroupNorm statistics through
+//                 distributed shared memory.  MMA order:
+//                   O  = Q S_(c-1)                 (then O *= gamma^(i+1) in TMEM)
+//                   Sc = Q K_kb^T  for kb = 0..r   (double-buffered in TMEM)
+//                   O += P_kb V_kb                 (P = decayed, masked Sc in bf16)
+//                 and the epilogue applies GroupNorm + swish gate or stores o.
+//
+// All operand tiles are loaded by TMA (no multicast) into 128-byte-swizzled
+// shared memory; every wait is bounded (see tc_ptx.cuh) and on expiry the CTA
+// drains its in-flight copies and MMAs, frees TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include "launch.h"
+#include "tc_ptx.cuh"
+
+namespace ret {
+namespace {
+
+using namespace tc;
+
+constexpr int kRowsPerTile = 128;     // MMA M, TMEM lanes, query rows per CTA
+constexpr int kKeysPerBlock = 128;    // keys per score tile
+constexpr int kThreads = 192;         // 6 warps
+constexpr int kEpiThreads = 128;      // warps 2..5
+constexpr uint32_t kBox = 8192;       // one [64 rows][128 B] box
+constexpr uint32_t kTallBox = 16384;  // one [128 rows][128 B] box
+
+struct SeqInfo {
+  int s, c, a, b, cs, len;   // sequence, chunk, sequence [a,b), chunk start, chunk length
+};
+
+// chunk slot -> (sequence, chunk); false if the slot holds no chunk
+__device__ __forceinline__ bool slot_to_chunk(const SeqLayout& L, const int32_t* chunk_base,
+                                              long long slot, SeqInfo& si) {
+  if (L.cu == nullptr) {
+    const int nch = ceil_div(L.T, L.chunk);
+    si.s = static_cast<int>(slot / nch);
+    si.c = static_cast<int>(slot % nch);
+    if (si.s >= L.nseq) return false;
+  } else {
+    if (slot >= chunk_base[L.nseq]) return false;
+    int lo = 0, hi = L.nseq - 1;               // largest s with chunk_base[s] <= slot
+    while (lo < hi) {
+      int mid = (lo + hi + 1) >> 1;
+      if (chunk_base[mid] <= slot) lo = mid; else hi = mid - 1;
+    }
+    si.s = lo;
+    si.c = static_cast<int>(slot - chunk_base[lo]);
+  }
+  seq_bounds(L, si.s, si.a, si.b);
+  si.cs = si.a + si.c * L.chunk;
+  si.len = min(L.chunk, si.b - si.cs);
+  return si.len > 0;
+}
+
+// ===========================================================================
+// State kernel
+// ===========================================================================
+constexpr int kStTok = 64;           // tokens per pipeline stage
+
+struct StateParams {
+  SeqLayout L;
+  const int32_t* chunk_base;
+  const float* state_in;
+  float* state_out;
+  __nv_bfloat16* ws;                 // [nslots][H][2 (hi, lo)][dk][dv] bf16
+  int H, dk, dv;
+  HeadDecay dec;
+  unsigned* err;
+};
+
+template <int NS>
+struct StCfg {
+  static constexpr uint32_t kKBytes = 2 * kBox;              // 64 tokens x 128 rows of d_k
+  static constexpr uint32_t kVBytes = (NS / 64) * kBox;      // 64 tokens x NS
+  static constexpr uint32_t kStage = 2 * kKBytes + kVBytes;  // K hi | K lo | V
+  static constexpr int kStages = (196608 / kStage) < 4 ? (196608 / kStage) : 4;
+  static constexpr uint32_t kSmem = kStages * kStage + 256;
+};
+
+template <int NS>
+__global__ void __launch_bounds__(kThreads, 1)
+state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+             const StateParams p) {
+  using SC = StCfg<NS>;
+  constexpr int NSTG = SC::kStages;
+  constexpr uint32_t kStage = SC::kStage;
+  constexpr uint32_t kKBytes = SC::kKBytes;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NSTG * kStage);
+  uint64_t* full = bars;
+  uint64_t* empty = full + NSTG;
+  uint64_t* kready = empty + NSTG;
+  uint64_t* acc_ready = kready + NSTG;
+  uint64_t* acc_full = acc_ready + 1;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_hold + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int s = blockIdx.x, h = blockIdx.y;
+  const int m = blockIdx.z % (p.dk / 128), part = blockIdx.z / (p.dk / 128);
+  const SeqLayout& L = p.L;
+  int a, b;
+  seq_bounds(L, s, a, b);
+  const int nch = ceil_div(b - a, L.chunk);
+  const Decay1 dec(p.dec, h);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NSTG; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+      mbar_init(&kready[i], kEpiThreads);
+    }
+    mbar_init(acc_ready, kEpiThreads);
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    if ((smem_u32(smem) & 1023u) != 0) {
+      *abort_flag = 1;
+      raise_error(p.err, kErrTimeout);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_hold, NS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_hold;
+
+  if (warp == 0) {
+    // ---------------- TMA producer: K rows (into the hi slot) and V ----------------
+    if (lane == 0 && !*abort_flag) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int it = 0;
+      bool ok = true;
+      for (int c = 0; c < nch && ok; ++c) {
+        const int tok0 = a + c * L.chunk;
+        const int Lc = min(L.chunk, b - tok0);
+        for (int sb = 0; sb * kStTok < Lc; ++sb, ++it) {
+          const int st = it % NSTG;
+          if (!mbar_wait(&empty[st], ((it / NSTG) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
+          uint8_t* base = smem + st * kStage;
+          mbar_arrive_expect_tx(&full[st], kKBytes + SC::kVBytes);
+          const int y = tok0 + sb * kStTok;
+          for (int bx = 0; bx < 2; ++bx)
+            tma_load_2d(base + bx * kBox, &tmK, &full[st], h * p.dk + 128 * m + 64 * bx, y);
+          for (int bx = 0; bx < NS / 64; ++bx)
+            tma_load_2d(base + 2 * kKBytes + bx * kBox, &tmV, &full[st],
+                        h * p.dv + NS * part + 64 * bx, y);
+        }
+      }
+      if (!ok) {   // drain: the last load issued into each stage must land before exit
+        for (int j = 1; j <= NSTG && it - j >= 0; ++j) {
+          const int i2 = it - j;
+          mbar_wait_drain(&full[i2 % NSTG], (i2 / NSTG) & 1);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer: S += (zeta K)_hi^T V + (zeta K)_lo^T V ----------------
+    if (lane == 0 && !*abort_flag) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, NS, true, true);
+      int it = 0;
+      bool ok = true, issued = false;
+      for (int c = 0; c < nch && ok; ++c) {
+        const int Lc = min(L.chunk, b - (a + c * L.chunk));
+        if (!mbar_wait(acc_ready, c & 1, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        for (int sb = 0; sb * kStTok < Lc; ++sb, ++it) {
+          const int st = it % NSTG;
+          if (!mbar_wait(&kready[st], (it / NSTG) & 1, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t khi = smem_u32(smem + st * kStage);
+          const uint32_t klo = khi + kKBytes;
+          const uint32_t vb = khi + 2 * kKBytes;
+#pragma unroll
+          for (int ks = 0; ks < kStTok / 16; ++ks) {
+            const uint64_t bd = sdesc_sw128(vb + ks * 2048, kBox, 1024);
+            mma_bf16(tmem, sdesc_sw128(khi + ks * 2048, kBox, 1024), bd, idesc, true);
+            mma_bf16(tmem, sdesc_sw128(klo + ks * 2048, kBox, 1024), bd, idesc, true);
+          }
+          issued = true;
+          mma_commit(&empty[st]);
+        }
+        if (ok) mma_commit(acc_full);
+      }
+      if (!ok && issued) {
+        mma_commit(drain);
+        mbar_wait_drain(drain, 0);
+      }
+    }
+  } else {
+    // ---------------- state warpgroup ----------------
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;            // TMEM lane = row of the state block
+    const int i = 128 * m + row;                 // d_k index
+    const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const size_t st_off = ((static_cast<size_t>(s) * p.H + h) * p.dk + i) * p.dv + NS * part;
+    int it = 0;
+    bool ok = !*abort_flag;
+    for (int c = 0; c < nch && ok; ++c) {
+      const int tok0 = a + c * L.chunk;
+      const int Lc = min(L.chunk, b - tok0);
+      const long long slot = L.cu == nullptr
+                                 ? static_cast<long long>(s) * ceil_div(L.T, L.chunk) + c
+                                 : static_cast<long long>(p.chunk_base[s]) + c;
+      const bool slot_ok = slot >= 0 && slot < L.nslots;
+      const size_t hrow = ((static_cast<size_t>(slot_ok ? slot : 0) * p.H + h) * 2) * p.dk + i;
+      __nv_bfloat16* whi = p.ws + hrow * p.dv + NS * part;
+      __nv_bfloat16* wlo = p.ws + (hrow + p.dk) * p.dv + NS * part;
+      if (c > 0) {
+        if (!mbar_wait(acc_full, (c - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+      }
+      const float gL = dec.pow(Lc);
+#pragma unroll 1
+      for (int j = 0; j < NS / 32; ++j) {
+        float r[32];
+        if (c == 0) {
+          if (p.state_in) {
+            const float4* src = reinterpret_cast<const float4*>(p.state_in + st_off + 32 * j);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              float4 x = src[e];
+              r[4 * e] = x.x; r[4 * e + 1] = x.y; r[4 * e + 2] = x.z; r[4 * e + 3] = x.w;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0.f;
+          }
+        } else {
+          tmem_ld32(trow + 32 * j, r);
+          tmem_wait_ld();
+        }
+        if (slot_ok) {   // the state entering chunk c, as a hi/lo bf16 pair
+          uint4* dh = reinterpret_cast<uint4*>(whi + 32 * j);
+          uint4* dl = reinterpret_cast<uint4*>(wlo + 32 * j);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint4 uh, ul;
+            pack_split(r[8 * e + 0], r[8 * e + 1], uh.x, ul.x);
+            pack_split(r[8 * e + 2], r[8 * e + 3], uh.y, ul.y);
+            pack_split(r[8 * e + 4], r[8 * e + 5], uh.z, ul.z);
+            pack_split(r[8 * e + 6], r[8 * e + 7], uh.w, ul.w);
+            dh[e] = uh;
+            dl[e] = ul;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] *= gL;
+        tmem_st32(trow + 32 * j, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(acc_ready);
+      // zeta_j = gamma^(Lc-1-j) times the K rows of the chunk (0 past its end),
+      // split into a hi tile (in place) and a lo tile
+      for (int sb = 0; sb * kStTok < Lc; ++sb, ++it) {
+        const int st = it % NSTG;
+        if (!mbar_wait(&full[st], (it / NSTG) & 1, abort_flag, p.err)) { ok = false; break; }
+        const int t = threadIdx.x - 64;           // 0..127: box t/64, token row t%64
+        const int jtok = sb * kStTok + (t & 63);
+        const float z = jtok < Lc ? dec.pow(Lc - 1 - jtok) : 0.f;
+        uint8_t* rowb = smem + st * kStage + (t >> 6) * kBox + (t & 63) * 128;
+        uint4* hp = reinterpret_cast<uint4*>(rowb);
+        uint4* lp = reinterpret_cast<uint4*>(rowb + kKBytes);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          uint4 u = hp[e];
+          uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          uint32_t wh[4], wl[4];
+#pragma unroll
+          for (int q2 = 0; q2 < 4; ++q2) {
+            __nv_bfloat162 hv = *reinterpret_cast<__nv_bfloat162*>(&w[q2]);
+            float2 f = __bfloat1622float2(hv);
+            pack_split(f.x * z, f.y * z, wh[q2], wl[q2]);
+          }
+          hp[e] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          lp[e] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&kready[st]);
+      }
+    }
+    // final state
+    if (ok && nch > 0) {
+      if (mbar_wait(acc_full, (nch - 1) & 1, abort_flag, p.err)) {
+        tc_fence_after();
+        if (p.state_out) {
+          for (int j = 0; j < NS / 32; ++j) {
+            float r[32];
+            tmem_ld32(trow + 32 * j, r);
+            tmem_wait_ld();
+            float4* dst = reinterpret_cast<float4*>(p.state_out + st_off + 32 * j);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]);
+          }
+        }
+      }
+    } else if (ok && p.state_out) {   // empty sequence: the state passes through
+      for (int j = 0; j < NS; j += 4) {
+        float4 x = p.state_in ? *reinterpret_cast<const float4*>(p.state_in + st_off + j)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(p.state_out + st_off + j) = x;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, NS);
+  }
+}
+
+// ===========================================================================
+// Output kernel
+// ===========================================================================
+constexpr uint32_t kOutStage = 32768;
+
+struct OutParams {
+  SeqLayout L;
+  const int32_t* chunk_base;
+  bool has_state_in;
+  void* out;
+  int out_bf16;
+  const void* g;
+  int g_bf16;
+  const float* gn_w;
+  const float* gn_b;
+  float eps;
+  int gated;
+  int H, dk, dv;
+  int rb;                      // 128-row blocks per chunk
+  int parts;                   // d_v parts (cluster size)
+  HeadDecay dec;
+  unsigned* err;
+};
+
+template <int DK, int NV>
+struct OutCfg {
+  static constexpr uint32_t kQBytes = (DK / 64) * kTallBox;
+  static constexpr uint32_t kMiscBytes = 1024 + 512 + 1024;  // barriers | gamma^d table | stats
+  static constexpr int kStages = static_cast<int>((232448 - kQBytes - kMiscBytes) / kOutStage);
+  static constexpr uint32_t kOffStages = kQBytes;
+  static constexpr uint32_t kOffMisc = kOffStages + kStages * kOutStage;
+  static constexpr uint32_t kSmem = kOffMisc + kMiscBytes;
+  // TMEM columns: O, then two score/P buffers of 128 columns
+  static constexpr uint32_t kTmemO = 0, kTmemS0 = 256, kTmemS1 = 384;
+};
+
+__device__ __forceinline__ float ld_gate(const void* g, int bf16, size_t idx) {
+  return bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(g)[idx])
+              : static_cast<const float*>(g)[idx];
+}
+
+template <int DK, int NV>
+__global__ void __launch_bounds__(kThreads, 1)
+output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
+              const OutParams p) {
+  using C = OutCfg<DK, NV>;
+  constexpr int NST = C::kStages;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffMisc);
+  uint64_t* full = bars;                 // [NST]
+  uint64_t* empty = full + NST;          // [NST]
+  uint64_t* bar_q = empty + NST;
+  uint64_t* bar_inter = bar_q + 1;
+  uint64_t* bar_s = bar_inter + 1;       // [2] scores ready in TMEM
+  uint64_t* bar_p = bar_s + 2;           // [2] P (hi/lo) written over the scores
+  uint64_t* bar_o = bar_p + 2;           // all MMAs done
+  uint64_t* drain = bar_o + 1;
+  uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_hold + 1);
+  float* pow_tab = reinterpret_cast<float*>(smem + C::kOffMisc + 1024);      // gamma^d, d<128
+  float* stats = reinterpret_cast<float*>(smem + C::kOffMisc + 1024 + 512);  // [128][2]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int part = blockIdx.x % p.parts;
+  const long long unit = blockIdx.x / p.parts;
+  const int h = blockIdx.y;
+  const long long slot = unit / p.rb;
+  const int r = p.rb - 1 - static_cast<int>(unit % p.rb);   // heaviest row blocks first
+  SeqInfo si;
+  // Identical for both CTAs of a cluster, so a skipped unit skips together.
+  if (slot >= p.L.nslots) return;
+  if (!slot_to_chunk(p.L, p.chunk_base, slot, si)) return;
+  if (r * kRowsPerTile >= si.len) return;
+  const int t0 = si.cs + r * kRowsPerTile;                  // first token of the row block
+  const int nrows = min(kRowsPerTile, si.len - r * kRowsPerTile);
+  const bool need_inter = si.c > 0 || p.has_state_in;
+  const Decay1 dec(p.dec, h);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(bar_q, 1);
+    mbar_init(bar_inter, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_s[i], 1);
+      mbar_init(&bar_p[i], kEpiThreads);
+    }
+    mbar_init(bar_o, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    if ((smem_u32(smem) & 1023u) != 0) {
+      *abort_flag = 1;
+      raise_error(p.err, kErrTimeout);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_hold, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_hold;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && !*abort_flag) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmS);
+      mbar_arrive_expect_tx(bar_q, C::kQBytes);
+      for (int u = 0; u < DK / 64; ++u)
+        tma_load_2d(smem + u * kTallBox, &tmQ, bar_q, h * DK + 64 * u, t0);
+      int it = 0;
+      bool ok = true;
+      // one stage per unit, in the MMA issue order
+      auto next = [&](uint32_t bytes) -> uint8_t* {
+        const int st = it % NST;
+        if (!mbar_wait(&empty[st], ((it / NST) & 1) ^ 1, abort_flag, p.err)) return nullptr;
+        mbar_arrive_expect_tx(&full[st], bytes);
+        return smem + C::kOffStages + st * kOutStage;
+      };
+      if (need_inter) {
+        for (int u = 0; u < DK / 64 && ok; ++u) {
+          for (int hl = 0; hl < 2 && ok; ++hl) {
+            const int srow = static_cast<int>(((slot * p.H + h) * 2 + hl) * DK) + 64 * u;
+            uint8_t* dst = next((NV / 64) * kBox);
+            if (!dst) { ok = false; break; }
+            for (int bx = 0; bx < NV / 64; ++bx)
+              tma_load_2d(dst + bx * kBox, &tmS, &full[it % NST], NV * part + 64 * bx, srow);
+            ++it;
+          }
+        }
+      }
+      auto load_k = [&](int kb) {
+        for (int ku = 0; ku < DK / 128 && ok; ++ku) {
+          uint8_t* dst = next(2 * kTallBox);
+          if (!dst) { ok = false; break; }
+          for (int bx = 0; bx < 2; ++bx)
+            tma_load_2d(dst + bx * kTallBox, &tmK, &full[it % NST], h * DK + 128 * ku + 64 * bx,
+                        si.cs + kKeysPerBlock * kb);
+          ++it;
+        }
+      };
+      auto load_v = [&](int kb) {
+        for (int vu = 0; vu < 2 && ok; ++vu) {
+          uint8_t* dst = next((NV / 64) * kBox);
+          if (!dst) { ok = false; break; }
+          for (int bx = 0; bx < NV / 64; ++bx)
+            tma_load_2d(dst + bx * kBox, &tmV, &full[it % NST], h * p.dv + NV * part + 64 * bx,
+                        si.cs + kKeysPerBlock * kb + 64 * vu);
+          ++it;
+        }
+      };
+      load_k(0);
+      for (int kb = 0; kb <= r && ok; ++kb) {
+        if (kb + 1 <= r) load_k(kb + 1);
+        load_v(kb);
+      }
+      if (!ok) {
+        mbar_wait_drain(bar_q, 0);
+        for (int j = 1; j <= NST && it - j >= 0; ++j) {
+          const int i2 = it - j;
+          mbar_wait_drain(&full[i2 % NST], (i2 / NST) & 1);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0 && !*abort_flag) {
+      constexpr uint32_t id_qs = idesc_bf16_f32(128, NV, false, true);
+      constexpr uint32_t id_qk = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t id_pv = idesc_bf16_f32(128, NV, false, true);
+      const uint32_t q_base = smem_u32(smem);
+      const uint32_t st_base = smem_u32(smem + C::kOffStages);
+      int it = 0;
+      bool ok = true, issued = false;
+      auto stage_wait = [&]() -> uint32_t {
+        const int st = it % NST;
+        if (!mbar_wait(&full[st], (it / NST) & 1, abort_flag, p.err)) return 0;
+        tc_fence_after();
+        return st_base + st * kOutStage;
+      };
+      auto stage_free = [&]() {
+        mma_commit(&empty[it % NST]);
+        ++it;
+      };
+      ok = mbar_wait(bar_q, 0, abort_flag, p.err);
+      if (ok && need_inter) {
+        // O = Q S_hi + Q S_lo  (the state entering the chunk, split in two bf16 parts)
+        for (int u = 0; u < DK / 64 && ok; ++u) {
+          for (int hl = 0; hl < 2; ++hl) {
+            const uint32_t sb = stage_wait();
+            if (!sb) { ok = false; break; }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = sdesc_sw128(q_base + u * kTallBox + kk * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(sb + kk * 2048, kBox, 1024);
+              mma_bf16(tmem + C::kTmemO, ad, bd, id_qs, (u | hl | kk) != 0);
+            }
+            issued = true;
+            stage_free();
+          }
+        }
+        if (ok) mma_commit(bar_inter);
+      }
+      auto issue_qk = [&](int kb) -> bool {
+        const uint32_t dst = tmem + ((kb & 1) ? C::kTmemS1 : C::kTmemS0);
+        for (int ku = 0; ku < DK / 128; ++ku) {
+          const uint32_t sb = stage_wait();
+          if (!sb) return false;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const int qbox = ku * 2 + kk / 4;
+            const uint64_t ad = sdesc_sw128(q_base + qbox * kTallBox + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sb + (kk / 4) * kTallBox + (kk & 3) * 32, 16, 1024);
+            mma_bf16(dst, ad, bd, id_qk, (ku | kk) != 0);
+          }
+          issued = true;
+          stage_free();
+        }
+        mma_commit(&bar_s[kb & 1]);
+        return true;
+      };
+      if (ok) ok = issue_qk(0);
+      for (int kb = 0; kb <= r && ok; ++kb) {
+        // scores for the next key block go to the other buffer while P_kb is formed
+        if (kb + 1 <= r && !issue_qk(kb + 1)) { ok = false; break; }
+        if (!mbar_wait(&bar_p[kb & 1], (kb >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t pbuf = tmem + ((kb & 1) ? C::kTmemS1 : C::kTmemS0);
+        for (int vu = 0; vu < 2; ++vu) {
+          const uint32_t sb = stage_wait();
+          if (!sb) { ok = false; break; }
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int ks = vu * 4 + kk;                      // 16 keys: 16ks .. 16ks+15
+            const uint32_t a_hi = pbuf + 32 * (ks >> 1) + 8 * (ks & 1);
+            const uint64_t bd = sdesc_sw128(sb + kk * 2048, kBox, 1024);
+            mma_bf16_ts(tmem + C::kTmemO, a_hi, bd, id_pv, need_inter || kb > 0 || ks > 0);
+            mma_bf16_ts(tmem + C::kTmemO, a_hi + 16, bd, id_pv, true);
+          }
+          stage_free();
+        }
+      }
+      if (ok) {
+        mma_commit(bar_o);
+      } else if (issued) {
+        mma_commit(drain);
+        mbar_wait_drain(drain, 0);
+      }
+    }
+  } else {
+    // ---------------- epilogue warpgroup ----------------
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;                 // query row within the block
+    const int i = r * kRowsPerTile + row;              // row within the chunk
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const int et = threadIdx.x - 64;                  // 0..127
+    pow_tab[et] = dec.pow(et);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    bool ok = !*abort_flag;
+    if (ok && need_inter) {
+      ok = mbar_wait(bar_inter, 0, abort_flag, p.err);
+      if (ok) {
+        tc_fence_after();
+        const float sc = dec.pow(i + 1);
+        for (int j = 0; j < NV / 32; ++j) {
+          float x[32];
+          tmem_ld32(tmem + lane_off + C::kTmemO + 32 * j, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] *= sc;
+          tmem_st32(tmem + lane_off + C::kTmemO + 32 * j, x);
+        }
+        tmem_wait_st();
+      }
+    }
+    for (int kb = 0; kb <= r && ok; ++kb) {
+      const int sb = kb & 1;
+      if (!mbar_wait(&bar_s[sb], (kb >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+      tc_fence_after();
+      const bool diag = kb == r;
+      // off-diagonal: gamma^(i-j) = gamma^(i - 128kb - 127) * gamma^(127 - j')
+      const float arow = diag ? 0.f : dec.pow(i - kKeysPerBlock * kb - 127);
+      const int key_lim = si.len - kKeysPerBlock * kb;   // keys j' >= key_lim are past the chunk
+      const uint32_t buf = tmem + lane_off + (sb ? C::kTmemS1 : C::kTmemS0);
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {
+        float x[32];
+        tmem_ld32(buf + 32 * j, x);
+        tmem_wait_ld();
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pv[2];
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const int jp = 32 * j + e + t;
+            float wgt;
+            if (diag) wgt = (jp <= row) ? pow_tab[row - jp] : 0.f;
+            else wgt = arow * pow_tab[127 - jp];
+            if (jp >= key_lim) wgt = 0.f;
+            pv[t] = x[e + t] * wgt;
+          }
+          // columns 32j .. 32j+15: P_hi of keys 32j .. 32j+31, two per column;
+          // columns 32j+16 .. 32j+31: P_lo of the same keys
+          pack_split(pv[0], pv[1], w[e >> 1], w[16 + (e >> 1)]);
+        }
+        tmem_st32(buf + 32 * j, *reinterpret_cast<float(*)[32]>(w));
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_p[sb]);
+    }
+    // final O
+    float mean = 0.f, m2 = 0.f;
+    if (ok) ok = mbar_wait(bar_o, 0, abort_flag, p.err);
+    if (ok) {
+      tc_fence_after();
+      if (p.gated) {
+        float sum = 0.f;
+        for (int j = 0; j < NV / 32; ++j) {
+          float x[32];
+          tmem_ld32(tmem + lane_off + C::kTmemO + 32 * j, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sum += x[e];
+        }
+        mean = sum / NV;
+        for (int j = 0; j < NV / 32; ++j) {
+          float x[32];
+          tmem_ld32(tmem + lane_off + C::kTmemO + 32 * j, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) m2 += (x[e] - mean) * (x[e] - mean);
+        }
+        stats[2 * row] = mean;
+        stats[2 * row + 1] = m2;
+      }
+    }
+  }
+  // ---------------- join: GroupNorm statistics across the d_v parts ----------------
+  tc_fence_before();
+  __syncthreads();
+  const bool ok_all = !*abort_flag;
+  float mean_all = 0.f, rstd = 0.f;
+  if (p.parts > 1 && p.gated) cluster_sync();      // partner's stats are written
+  if (warp >= 2 && ok_all && p.gated) {
+    const int row = (warp & 3) * 32 + lane;
+    float mean = stats[2 * row], m2 = stats[2 * row + 1];
+    float cnt = static_cast<float>(NV);
+    if (p.parts > 1) {
+      const uint32_t other = cluster_ctarank() ^ 1u;
+      const float mo = ld_cluster_f32(&stats[2 * row], other);
+      const float m2o = ld_cluster_f32(&stats[2 * row + 1], other);
+      const float d = mo - mean;
+      m2 = m2 + m2o + d * d * (cnt * 0.5f);
+      mean = 0.5f * (mean + mo);
+      cnt *= 2.f;
+    }
+    mean_all = mean;
+    rstd = 1.0f / sqrtf(m2 / cnt + p.eps);
+  }
+  if (p.parts > 1 && p.gated) cluster_sync();      // partner has finished reading ours
+  if (warp >= 2 && ok_all) {
+    tc_fence_after();
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const bool live = row < nrows;
+    const size_t obase = (static_cast<size_t>(t0 + row) * p.H + h) * p.dv + NV * part;
+    for (int j = 0; j < NV / 32; ++j) {
+      float x[32];
+      tmem_ld32(tmem + lane_off + C::kTmemO + 32 * j, x);
+      tmem_wait_ld();
+      if (!live) continue;
+      if (p.gated) {
+        const int c0 = h * p.dv + NV * part + 32 * j;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float y = (x[e] - mean_all) * rstd;
+          if (p.gn_w) y *= p.gn_w[c0 + e];
+          if (p.gn_b) y += p.gn_b[c0 + e];
+          const float gv = ld_gate(p.g, p.g_bf16, obase + 32 * j + e);
+          x[e] = y * (gv / (1.0f + expf(-gv)));
+        }
+      }
+      if (p.out_bf16) {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + obase + 32 * j);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint4 u;
+          u.x = pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]);
+          u.y = pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]);
+          u.z = pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]);
+          u.w = pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]);
+          dst[c4] = u;
+        }
+      } else {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + 32 * j);
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4)
+          dst[c4] = make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ===========================================================================
+// Host side
+// ===========================================================================
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map: `rows` rows of `inner` elements, row pitch `pitch`
+// elements, box = 64 elements x box_rows rows, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch,
+              uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {inner, rows};
+  cuuint64_t gstride[1] = {pitch * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int NS>
+cudaError_t launch_state(const CUtensorMap& mk, const CUtensorMap& mv, const StateParams& sp,
+                         cudaStream_t s) {
+  const size_t smem = StCfg<NS>::kSmem;
+  auto kern = state_kernel<NS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(sp.L.nseq, sp.H, (sp.dk / 128) * (sp.dv / NS));
+  kern<<<grid, kThreads, smem, s>>>(mk, mv, sp);
+  return cudaGetLastError();
+}
+
+template <int DK, int NV>
+cudaError_t launch_out(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const CUtensorMap& ms, const OutParams& op, long long units,
+                       cudaStream_t s) {
+  using C = OutCfg<DK, NV>;
+  static_assert(C::kSmem <= 232448, "shared memory budget");
+  auto kern = output_kernel<DK, NV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(C::kSmem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(units * op.parts), op.H, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = op.parts;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ms, op);
+}
+
+}  // namespace
+
+bool chunkwise_tc_supported(int dk, int dv, int chunk) {
+  const bool dk_ok = dk == 128 || dk == 256;
+  const bool dv_ok = dv == 64 || dv == 128 || dv == 256 || dv == 512;
+  const bool c_ok = chunk == 64 || chunk == 128 || chunk == 256 || chunk == 512;
+  return dk_ok && dv_ok && c_ok;
+}
+
+int chunkwise_tc_chunk(int chunk) { return chunk < 128 ? 128 : chunk; }
+
+cudaError_t launch_chunkwise_tc(const void* q, const void* k, const void* v,
+                                const SeqLayout& L, const float* state_in, float* state_out,
+                                void* out, DType out_t, const void* g, DType g_t,
+                                const float* gn_w, const float* gn_b, float eps, bool gated,
+                                ChunkWorkspace ws, int H, int dk, int dv,
+                                const HeadDecay& dec, unsigned* err, cudaStream_t s) {
+  if (!chunkwise_tc_supported(dk, dv, L.chunk)) return cudaErrorNotSupported;
+  // ---- state pass ----
+  const int NS = dv >= 256 ? 256 : dv;
+  StateParams sp;
+  sp.L = L;
+  sp.chunk_base = ws.chunk_base;
+  sp.state_in = state_in;
+  sp.state_out = state_out;
+  sp.ws = static_cast<__nv_bfloat16*>(ws.states);
+  sp.H = H;
+  sp.dk = dk;
+  sp.dv = dv;
+  sp.dec = dec;
+  sp.err = err;
+  const uint64_t Ttot = static_cast<uint64_t>(L.Ttot > 0 ? L.Ttot : 1);
+  CUtensorMap mk_st, mv_st, mq, mk, mv, ms;
+  if (!make_map(&mk_st, k, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 64) ||
+      !make_map(&mv_st, v, static_cast<uint64_t>(H) * dv, Ttot, static_cast<uint64_t>(H) * dv, 64))
+    return cudaErrorInvalidValue;
+  cudaError_t e;
+  switch (NS) {
+    case 64: e = launch_state<64>(mk_st, mv_st, sp, s); break;
+    case 128: e = launch_state<128>(mk_st, mv_st, sp, s); break;
+    default: e = launch_state<256>(mk_st, mv_st, sp, s); break;
+  }
+  if (e != cudaSuccess || L.Ttot == 0) return e;
+  // ---- output pass ----
+  const int NV = dv > 256 ? 256 : dv;
+  OutParams op;
+  op.L = L;
+  op.chunk_base = ws.chunk_base;
+  op.has_state_in = state_in != nullptr;
+  op.out = out;
+  op.out_bf16 = out_t == DType::BF16;
+  op.g = g;
+  op.g_bf16 = g_t == DType::BF16;
+  op.gn_w = gn_w;
+  op.gn_b = gn_b;
+  op.eps = eps;
+  op.gated = gated ? 1 : 0;
+  op.H = H;
+  op.dk = dk;
+  op.dv = dv;
+  op.rb = L.chunk / kRowsPerTile;
+  op.parts = dv / NV;
+  op.dec = dec;
+  op.err = err;
+  const uint64_t srows = static_cast<uint64_t>(ws.nslots) * H * 2 * dk;   // hi and lo planes
+  if (!make_map(&mq, q, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 128) ||
+      !make_map(&mk, k, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 128) ||
+      !make_map(&mv, v, static_cast<uint64_t>(H) * dv, Ttot, static_cast<uint64_t>(H) * dv, 64) ||
+      !make_map(&ms, ws.states, dv, srows, dv, 64))
+    return cudaErrorInvalidValue;
+  const long long units = ws.nslots * op.rb;
+  if (dk == 128) {
+    switch (NV) {
+      case 64: return launch_out<128, 64>(mq, mk, mv, ms, op, units, s);
+      case 128: return launch_out<128, 128>(mq, mk, mv, ms, op, units, s);
+      default: return launch_out<128, 256>(mq, mk, mv, ms, op, units, s);
+    }
+  }
+  switch (NV) {
+    case 64: return launch_out<256, 64>(mq, mk, mv, ms, op, units, s);
+    case 128: return launch_out<256, 128>(mq, mk, mv, ms, op, units, s);
+    default: return launch_out<256, 256>(mq, mk, mv, ms, op, units, s);
+  }
+}
+
+}  // namespace ret

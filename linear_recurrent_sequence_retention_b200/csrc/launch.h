@@ -1,0 +1,61 @@
+// Internal host-side launchers of libretention (not part of the C ABI).
+// Arguments are validated by the entry points in api.cu before these run.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace ret {
+
+enum class DType { F32 = 0, BF16 = 1 };
+
+// Workspace layout of the chunkwise forward:
+//   [meta: chunk_base int32[nseq+1], rounded up to 256 B][states]
+// states hold the state entering every chunk, one slot per chunk:
+//   [slot][H][dk][dv] float32 on the CUDA-core path; [slot][H][2][dk][dv]
+//   bfloat16 on the tensor-core path (the state as hi + lo bf16 parts).
+struct ChunkWorkspace {
+  int32_t* chunk_base;   // device, nseq+1 entries (varlen only; else unused)
+  void* states;          // device
+  long long nslots;      // slots available
+};
+
+size_t chunkwise_meta_bytes(int nseq);
+
+// CUDA-core (fp32 FFMA) kernels.
+cudaError_t launch_parallel_simt(const void* q, const void* k, const void* v, DType in_t,
+                                 void* o, DType o_t, int B, int T, int H, int dk, int dv,
+                                 const HeadDecay& dec, cudaStream_t s);
+
+cudaError_t launch_chunk_prep(const SeqLayout& L, ChunkWorkspace ws, unsigned* err,
+                              cudaStream_t s);
+
+cudaError_t launch_chunkwise_simt(const void* q, const void* k, const void* v, DType in_t,
+                                  const SeqLayout& L, const float* state_in, float* state_out,
+                                  void* out, DType out_t, const void* g, DType g_t,
+                                  const float* gn_w, const float* gn_b, float eps, bool gated,
+                                  ChunkWorkspace ws, int H, int dk, int dv,
+                                  const HeadDecay& dec, unsigned* err, cudaStream_t s);
+
+cudaError_t launch_decode_step(const void* q, const void* k, const void* v, DType in_t,
+                               float* state, void* o, DType o_t, int N, int H, int dk, int dv,
+                               const HeadDecay& dec, cudaStream_t s);
+
+cudaError_t launch_norm_gate(const void* o, DType o_t, const void* g, DType g_t,
+                             const float* w, const float* b, float eps, void* y, DType y_t,
+                             int ntok, int H, int dv, cudaStream_t s);
+
+// Tensor-core (tcgen05) chunkwise forward for bf16 inputs.
+bool chunkwise_tc_supported(int dk, int dv, int chunk);
+int chunkwise_tc_chunk(int chunk);  // chunk length the kernels evaluate
+cudaError_t launch_chunkwise_tc(const void* q, const void* k, const void* v,
+                                const SeqLayout& L, const float* state_in, float* state_out,
+                                void* out, DType out_t, const void* g, DType g_t,
+                                const float* gn_w, const float* gn_b, float eps, bool gated,
+                                ChunkWorkspace ws, int H, int dk, int dv,
+                                const HeadDecay& dec, unsigned* err, cudaStream_t s);
+
+}  // namespace ret

@@ -1,0 +1,268 @@
+"""Thin ctypes binding of libretention.so (C ABI in include/retention.h).
+
+Argument marshalling only: every function checks the torch tensors it is
+given, passes their device pointers, sizes and the current CUDA stream to the
+C entry point of the same name, and raises :class:`RetentionError` on a
+non-OK status.  All arithmetic happens in the library's CUDA kernels; there
+is no CPU or PyTorch fallback, and calling any function without the built
+library raises immediately.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_HERE, "libretention.so")
+
+RET_OK = 0
+RET_ERR_INVALID_ARG = 1
+RET_ERR_UNSUPPORTED = 2
+RET_ERR_CUDA = 3
+RET_ERR_TIMEOUT = 4
+RET_ERR_WORKSPACE = 5
+RET_ERR_DEVICE_DATA = 6
+
+RET_F32 = 0
+RET_BF16 = 1
+
+EXPORTED = (
+    "retention_abi_version",
+    "retention_status_string",
+    "retention_parallel_fwd",
+    "retention_chunkwise_workspace_size",
+    "retention_chunkwise_fwd",
+    "retention_recurrent_step",
+    "msr_norm_gate",
+    "retention_check_device_error",
+)
+
+
+class RetentionError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+class NormGate(ctypes.Structure):
+    _fields_ = [("g", ctypes.c_void_p), ("g_dtype", ctypes.c_int),
+                ("weight", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("eps", ctypes.c_float)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library (loads it on first use; raises if it is not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIBRARY_PATH):
+        raise RuntimeError(
+            f"{LIBRARY_PATH} is missing: build it with "
+            "`python -m linear_recurrent_sequence_retention_b200.build` (needs nvcc)")
+    L = ctypes.CDLL(LIBRARY_PATH)
+    vp, ci, cd = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_double)
+    L.retention_abi_version.restype = ci
+    L.retention_abi_version.argtypes = []
+    L.retention_status_string.restype = ctypes.c_char_p
+    L.retention_status_string.argtypes = [ci]
+    L.retention_parallel_fwd.restype = ci
+    L.retention_parallel_fwd.argtypes = [vp, vp, vp, ci, cd, vp, ci, ci, ci, ci, ci, ci, vp]
+    L.retention_chunkwise_workspace_size.restype = ctypes.c_size_t
+    L.retention_chunkwise_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci]
+    L.retention_chunkwise_fwd.restype = ci
+    L.retention_chunkwise_fwd.argtypes = [vp, vp, vp, ci, cd, ci, vp, ci, vp, vp, vp, ci,
+                                          ctypes.POINTER(NormGate), vp, ctypes.c_size_t,
+                                          ci, ci, ci, ci, ci, vp]
+    L.retention_recurrent_step.restype = ci
+    L.retention_recurrent_step.argtypes = [vp, vp, vp, ci, cd, vp, vp, ci, ci, ci, ci, ci, vp]
+    L.msr_norm_gate.restype = ci
+    L.msr_norm_gate.argtypes = [vp, ci, ctypes.POINTER(NormGate), vp, ci, ci, ci, ci, vp]
+    L.retention_check_device_error.restype = ci
+    L.retention_check_device_error.argtypes = [vp]
+    _lib = L
+    return L
+
+
+def status_string(status):
+    return lib().retention_status_string(int(status)).decode()
+
+
+def _check(status, where):
+    if status != RET_OK:
+        raise RetentionError(status, where)
+
+
+def _dt(t):
+    if t.dtype == torch.float32:
+        return RET_F32
+    if t.dtype == torch.bfloat16:
+        return RET_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(t, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _gammas(gamma, H):
+    vals = [float(x) for x in (gamma.tolist() if hasattr(gamma, "tolist") else gamma)]
+    if len(vals) != H:
+        raise ValueError(f"gamma needs {H} entries, got {len(vals)}")
+    return (ctypes.c_double * H)(*vals)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def abi_version():
+    return lib().retention_abi_version()
+
+
+def parallel_fwd(q, k, v, gamma, out_dtype=None, stream=None):
+    """Parallel form; q,k: [B,T,H,dk], v: [B,T,H,dv] -> o [B,T,H,dv]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    if k.shape != q.shape or v.shape[:3] != q.shape[:3] or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v shapes/dtypes disagree")
+    o = torch.empty(B, T, H, dv, device=q.device, dtype=out_dtype or q.dtype)
+    st = lib().retention_parallel_fwd(_ptr(q), _ptr(k), _ptr(v), _dt(q), _gammas(gamma, H),
+                                      _ptr(o), _dt(o), B, T, H, dk, dv, _stream(stream))
+    _check(st, "retention_parallel_fwd")
+    return o
+
+
+def chunkwise_workspace_size(dtype, chunk, B, T, H, dk, dv, nseq=0):
+    code = RET_F32 if dtype == torch.float32 else RET_BF16
+    return int(lib().retention_chunkwise_workspace_size(code, chunk, B, T, H, dk, dv, nseq))
+
+
+def alloc_workspace(nbytes, device):
+    """A caller-owned workspace buffer (uint8, 256-byte aligned by the allocator)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def chunkwise_fwd(q, k, v, gamma, chunk, cu_seqlens=None, state_in=None, return_state=False,
+                  g=None, gn_weight=None, gn_bias=None, eps=1e-5, out_dtype=None, out=None,
+                  state_out=None, workspace=None, stream=None):
+    """Chunkwise form (+ optional fused GroupNorm and swish gate when ``g`` is given).
+
+    q,k: [B,T,H,dk]; v: [B,T,H,dv]; packed sequences: B = 1 and ``cu_seqlens``
+    an int32 CUDA tensor [nseq+1].  Returns ``out`` ([B,T,H,dv]: o, or y when
+    gated) and, with ``return_state``, the final fp32 states.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    if k.shape != q.shape or v.shape[:3] != q.shape[:3] or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v shapes/dtypes disagree")
+    nseq = 0
+    if cu_seqlens is not None:
+        _dev(cu_seqlens, "cu_seqlens")
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be a 1-D int32 tensor")
+        nseq = cu_seqlens.numel() - 1
+        if nseq < 1:
+            raise ValueError("cu_seqlens needs at least two entries")
+    nstate = nseq if nseq else B
+    if state_in is not None:
+        _dev(state_in, "state_in")
+        if state_in.dtype != torch.float32 or tuple(state_in.shape) != (nstate, H, dk, dv):
+            raise ValueError(f"state_in must be float32 [{nstate},{H},{dk},{dv}]")
+    if return_state and state_out is None:
+        state_out = torch.empty(nstate, H, dk, dv, device=q.device, dtype=torch.float32)
+    if state_out is not None:
+        _dev(state_out, "state_out")
+        if state_out.dtype != torch.float32 or tuple(state_out.shape) != (nstate, H, dk, dv):
+            raise ValueError(f"state_out must be float32 [{nstate},{H},{dk},{dv}]")
+    if out is None:
+        out = torch.empty(B, T, H, dv, device=q.device, dtype=out_dtype or q.dtype)
+    else:
+        _dev(out, "out")
+        if tuple(out.shape) != (B, T, H, dv):
+            raise ValueError("out has the wrong shape")
+    ng = None
+    keep = []
+    if g is not None:
+        _dev(g, "g")
+        if g.numel() != B * T * H * dv:
+            raise ValueError("g must hold B*T*H*dv elements")
+        for t, n in ((gn_weight, "gn_weight"), (gn_bias, "gn_bias")):
+            if t is not None:
+                _dev(t, n)
+                if t.dtype != torch.float32 or t.numel() != H * dv:
+                    raise ValueError(f"{n} must be float32 with H*dv elements")
+        ng = NormGate(g.data_ptr(), _dt(g), gn_weight.data_ptr() if gn_weight is not None else None,
+                      gn_bias.data_ptr() if gn_bias is not None else None, float(eps))
+        keep.append(ng)
+    need = lib().retention_chunkwise_workspace_size(_dt(q), chunk, B, T, H, dk, dv, nseq)
+    if need == 0:
+        st = RET_ERR_UNSUPPORTED if _dt(q) == RET_BF16 else RET_ERR_INVALID_ARG
+        raise RetentionError(st, "retention_chunkwise_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    st = lib().retention_chunkwise_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _dt(q), _gammas(gamma, H), int(chunk),
+        _ptr(cu_seqlens), nseq, _ptr(state_in), _ptr(state_out), _ptr(out), _dt(out),
+        ctypes.byref(ng) if ng is not None else None, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), B, T, H, dk, dv, _stream(stream))
+    _check(st, "retention_chunkwise_fwd")
+    return (out, state_out) if return_state else out
+
+
+def recurrent_step(q, k, v, gamma, state, out_dtype=torch.float32, out=None, stream=None):
+    """One decode step; updates ``state`` [N,H,dk,dv] in place and returns o [N,H,dv]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (state, "state")):
+        _dev(t, n)
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    if state.dtype != torch.float32 or tuple(state.shape) != (N, H, dk, dv):
+        raise ValueError(f"state must be float32 [{N},{H},{dk},{dv}]")
+    if out is None:
+        out = torch.empty(N, H, dv, device=q.device, dtype=out_dtype)
+    st = lib().retention_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _dt(q), _gammas(gamma, H),
+                                        _ptr(state), _ptr(out), _dt(out), N, H, dk, dv,
+                                        _stream(stream))
+    _check(st, "retention_recurrent_step")
+    return out
+
+
+def norm_gate(o, g, weight=None, bias=None, eps=1e-5, out_dtype=None, stream=None):
+    """Per-head GroupNorm + swish gate; o: [ntok,H,dv] (any leading dims), g same size."""
+    _dev(o, "o")
+    _dev(g, "g")
+    H, dv = o.shape[-2], o.shape[-1]
+    ntok = o.numel() // (H * dv)
+    if g.numel() != o.numel():
+        raise ValueError("g must have as many elements as o")
+    y = torch.empty(o.shape, device=o.device, dtype=out_dtype or o.dtype)
+    ng = NormGate(g.data_ptr(), _dt(g), weight.data_ptr() if weight is not None else None,
+                  bias.data_ptr() if bias is not None else None, float(eps))
+    st = lib().msr_norm_gate(_ptr(o), _dt(o), ctypes.byref(ng), _ptr(y), _dt(y), ntok, H, dv,
+                             _stream(stream))
+    _check(st, "msr_norm_gate")
+    return y
+
+
+def check_device_error(stream=None):
+    """Synchronise the stream and raise if a kernel reported a device-side error."""
+    _check(lib().retention_check_device_error(_stream(stream)), "retention_check_device_error")

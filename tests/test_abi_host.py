@@ -1,0 +1,129 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching the GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "retention.h")
+
+
+def _lib():
+    from linear_recurrent_sequence_retention_b200 import ops
+    if not os.path.exists(ops.LIBRARY_PATH):
+        from linear_recurrent_sequence_retention_b200 import build
+        build.build()
+    return ops, ops.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^RET_API\s+[\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ("retention_parallel_fwd", "retention_chunkwise_fwd", "retention_recurrent_step",
+                 "msr_norm_gate", "retention_chunkwise_workspace_size",
+                 "retention_check_device_error", "retention_status_string",
+                 "retention_abi_version"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol():
+    ops, L = _lib()
+    for name in declared_symbols():
+        assert hasattr(L, name), f"libretention.so does not export {name}"
+    assert set(ops.EXPORTED) <= set(declared_symbols())
+
+
+def test_abi_version_and_status_strings():
+    ops, L = _lib()
+    assert L.retention_abi_version() == 1
+    for code in range(7):
+        s = ops.status_string(code)
+        assert s and "unknown" not in s
+    assert "unknown" in ops.status_string(99)
+
+
+FAKE = ctypes.c_void_p(0x10000)          # aligned, never dereferenced on these paths
+MISALIGNED = ctypes.c_void_p(0x10004)
+
+
+def _g(*vals):
+    return (ctypes.c_double * len(vals))(*vals)
+
+
+def test_parallel_rejects_bad_arguments():
+    ops, L = _lib()
+    f = L.retention_parallel_fwd
+    ok = dict(B=1, T=8, H=2, dk=16, dv=16)
+    args = lambda q=FAKE, gamma=_g(0.5, 0.9), dk=16, dv=16, T=8, H=2, o_dt=0: (
+        q, FAKE, FAKE, 0, gamma, FAKE, o_dt, 1, T, H, dk, dv, None)
+    assert f(*args(q=None)) == ops.RET_ERR_INVALID_ARG
+    assert f(*args(q=MISALIGNED)) == ops.RET_ERR_INVALID_ARG
+    assert f(*args(gamma=_g(0.5, 1.5))) == ops.RET_ERR_INVALID_ARG
+    assert f(*args(gamma=_g(-0.1, 0.5))) == ops.RET_ERR_INVALID_ARG
+    assert f(*args(gamma=_g(float("nan"), 0.5))) == ops.RET_ERR_INVALID_ARG
+    assert f(*args(T=0)) == ops.RET_ERR_INVALID_ARG
+    assert f(*args(o_dt=7)) == ops.RET_ERR_INVALID_ARG
+    assert f(*args(dk=300)) == ops.RET_ERR_UNSUPPORTED
+
+
+def test_workspace_size_query():
+    ops, L = _lib()
+    ws = L.retention_chunkwise_workspace_size
+    # float32: meta (256 B) + one fp32 state per chunk
+    assert ws(0, 16, 1, 64, 2, 16, 16, 0) == 256 + 4 * 2 * 16 * 16 * 4
+    # ragged tail: ceil(70/16) = 5 chunks per sequence
+    assert ws(0, 16, 3, 70, 2, 16, 16, 0) == 256 + 15 * 2 * 16 * 16 * 4
+    # packed: ceil(Ttot/C) + nseq slots
+    assert ws(0, 16, 1, 100, 2, 8, 8, 5) == 256 + (7 + 5) * 2 * 8 * 8 * 4
+    assert ws(0, 0, 1, 64, 2, 16, 16, 0) == 0            # chunk < 1
+    assert ws(0, 16, 1, 64, 65, 16, 16, 0) == 0          # H > 64
+    assert ws(0, 16, 2, 64, 2, 16, 16, 3) == 0           # packed needs B == 1
+    assert ws(0, 16, 1, 64, 2, 300, 16, 0) == 0          # fp32 path: dk <= 256
+
+
+def test_chunkwise_rejects_bad_arguments():
+    ops, L = _lib()
+    f = L.retention_chunkwise_fwd
+    NG = ops.NormGate
+
+    def call(ws_bytes=1 << 20, ws=FAKE, gamma=None, cu=None, nseq=0, ng=None, q=FAKE):
+        gamma = gamma or _g(0.5, 0.9)
+        return f(q, FAKE, FAKE, 0, gamma, 16, cu, nseq, None, None, FAKE, 0,
+                 ng, ws, ws_bytes, 1, 64, 2, 16, 16, None)
+    assert call(ws_bytes=10) == ops.RET_ERR_WORKSPACE
+    assert call(ws=None) == ops.RET_ERR_WORKSPACE
+    assert call(ws=ctypes.c_void_p(0x10010)) == ops.RET_ERR_WORKSPACE   # not 256-B aligned
+    assert call(gamma=_g(0.5, 2.0)) == ops.RET_ERR_INVALID_ARG
+    assert call(cu=FAKE, nseq=0) == ops.RET_ERR_INVALID_ARG              # cu without nseq
+    assert call(q=None) == ops.RET_ERR_INVALID_ARG
+    bad = NG(None, 0, None, None, 1e-5)
+    assert call(ng=ctypes.byref(bad)) == ops.RET_ERR_INVALID_ARG         # gate missing
+    bad_eps = NG(0x10000, 0, None, None, -1.0)
+    assert call(ng=ctypes.byref(bad_eps)) == ops.RET_ERR_INVALID_ARG
+
+
+def test_decode_and_norm_gate_reject_bad_arguments():
+    ops, L = _lib()
+    st = L.retention_recurrent_step(FAKE, FAKE, FAKE, 1, _g(0.5), None, FAKE, 0, 1, 1, 8, 8, None)
+    assert st == ops.RET_ERR_INVALID_ARG
+    st = L.retention_recurrent_step(FAKE, FAKE, FAKE, 1, _g(0.5), FAKE, FAKE, 0, 1, 1, 2048, 8, None)
+    assert st == ops.RET_ERR_UNSUPPORTED
+    ng = ops.NormGate(0x10000, 1, None, None, 1e-5)
+    assert L.msr_norm_gate(FAKE, 1, None, FAKE, 1, 4, 2, 8, None) == ops.RET_ERR_INVALID_ARG
+    assert L.msr_norm_gate(FAKE, 1, ctypes.byref(ng), FAKE, 1, 4, 2, 2048, None) == ops.RET_ERR_UNSUPPORTED
+    assert L.msr_norm_gate(FAKE, 1, ctypes.byref(ng), FAKE, 1, 0, 2, 8, None) == ops.RET_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    from linear_recurrent_sequence_retention_b200 import ops
+    monkeypatch.setattr(ops, "_lib", None)
+    monkeypatch.setattr(ops, "LIBRARY_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        ops.lib()
