@@ -1,0 +1,531 @@
+#!/usr/bin/env python
+"""Benchmark of the Multi-Scale Retention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+
+One JSON line on stdout (rank 0).  A step is one chunkwise forward of the
+6.7B-shaped workload (B=2 sequences of 8192 tokens, 16 heads, d_k=256,
+d_v=512, chunk 512, per-head GroupNorm + swish gate fused, final f32 state
+emitted) through the C ABI, inputs resident in HBM.  Every step reads about
+0.8 GB of inputs, far more than the 126 MB L2, so no flush is needed between
+steps.  The same run also times
+  * the two kernels of the step separately (CUDA events between the state and
+    output calls, on the launching stream) for the roofline of the dominant
+    one,
+  * the recurrent decode workload (128 sequences x 16 heads, d_k=256,
+    d_v=512, f32 state initialised by a chunkwise prefill of 8192 tokens,
+    1024 single-token steps),
+  * the end-to-end call with pinned host buffers (host->device copies of the
+    inputs and device->host copy of the output inside the timed region),
+  * the fp64 CPU oracle on a bounded sample of the same workload (rank 0, N=1).
+
+--impl reference times the oracle alone (the CPU reference arm).
+
+Multi-GPU: each rank runs its own batch of independent sequences (weak
+scaling, no collective on the data path); the step time is the maximum over
+ranks, and the value counts the tokens of all ranks.
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from linear_recurrent_sequence_retention_b200 import workloads as W  # noqa: E402
+
+METRIC = "retention fwd tokens/s & % bf16 tensor peak; decode steps/s & HBM GB/s % peak"
+HEADLINE = "msr_6p7b_b2_h16_t8192_dk256_dv512_c512"
+DECODE = "decode_6p7b_n128_h16_dk256_dv512"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TC_SOURCE = os.path.join(ROOT, "linear_recurrent_sequence_retention_b200", "csrc", "chunkwise_tc.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "chunkwise_output_kernel_6p7b_t8192_traffic.md")
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic counts (per token and head), stated with the roofline
+# ---------------------------------------------------------------------------
+
+def alg_counts(wl, chunk_exec):
+    """Per token-head: flops of the output kernel (intra-chunk causal product
+    and the decayed read of the state), of the state kernel (state update),
+    and the bytes every step must move (q, k, v, g read; y written)."""
+    C, dk, dv = chunk_exec, wl.dk, wl.dv
+    flops_out = (C + 1) * (dk + dv) + 2 * dk * dv
+    flops_state = 2 * dk * dv
+    bytes_in = 2 * (2 * dk + dv) + (2 * dv if wl.norm_gate else 0)
+    bytes_out = 2 * dv
+    return flops_out, flops_state, bytes_in, bytes_out
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for _, line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle, as it stands, on a bounded sample
+# ---------------------------------------------------------------------------
+
+def oracle_sample_step(wl, seed, chunk):
+    """One (sequence, head) of the workload through the oracle: the chunkwise
+    form over all its tokens, then GroupNorm + gate when the workload has it."""
+    import oracle
+    q, k, v, g = W.make_qkvg(1, wl.T, 1, wl.dk, wl.dv, "bf16", seed=seed, gate=wl.norm_gate)
+    f = W.to_f64
+    gam = W.head_gammas(wl.H)[seed % wl.H]
+    t0 = time.perf_counter()
+    o, _ = oracle.retention_chunkwise(f(q)[0, :, 0], f(k)[0, :, 0], f(v)[0, :, 0], gam, chunk)
+    if wl.norm_gate:
+        oracle.norm_gate(o[:, None, :], f(g)[0][:, None, :])
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        import threadpoolctl
+        n = [i["num_threads"] for i in threadpoolctl.threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(wl, budget_s=15.0):
+    """Oracle throughput in tokens/s (one token = all H heads), timed on a
+    sample of whole (sequence, head) pairs for about ``budget_s`` seconds."""
+    done, elapsed = 0, 0.0
+    while elapsed < budget_s or done == 0:
+        elapsed += oracle_sample_step(wl, done, wl.chunk)
+        done += 1
+        if done >= wl.B * wl.H:
+            break
+    token_heads = done * wl.T
+    return {"value": token_heads / wl.H / elapsed, "unit": "tokens/s",
+            "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{done} of {wl.B * wl.H} (sequence, head) pairs of {wl.name}, "
+                      f"{wl.T} tokens each, chunkwise form + GroupNorm/gate in numpy float64; "
+                      f"tokens/s counts a token once all {wl.H} heads are done"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def traffic_from_profile():
+    """DRAM bytes per launch of the output kernel from the committed ncu summary,
+    only if it was taken on the current kernel source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    text = open(TRAFFIC_FILE).read()
+    m1 = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m2 = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
+    if not (m1 and m2):
+        return None
+    sha = hashlib.sha256(open(TC_SOURCE, "rb").read()).hexdigest()
+    if sha != m1.group(1):
+        return None
+    return float(m2.group(1))
+
+
+def run_headline(args, world, rank, pk, pk_kind):
+    from linear_recurrent_sequence_retention_b200 import ops
+    wl = W.WORKLOADS[HEADLINE]
+    dev = torch.device("cuda")
+    q, k, v, g = W.make_qkvg(wl.B, wl.T, wl.H, wl.dk, wl.dv, "bf16", seed=rank, device=dev)
+    gam = W.head_gammas(wl.H)
+    y = torch.empty(wl.B, wl.T, wl.H, wl.dv, device=dev, dtype=torch.bfloat16)
+    S = torch.empty(wl.B, wl.H, wl.dk, wl.dv, device=dev, dtype=torch.float32)
+    ws = ops.alloc_workspace(ops.chunkwise_workspace_size(torch.bfloat16, wl.chunk, wl.B, wl.T,
+                                                          wl.H, wl.dk, wl.dv), dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record()
+        ops.chunkwise_states(k, v, gam, wl.chunk, state_out=S, workspace=ws)
+        if ev is not None:
+            ev[1].record()
+        ops.chunkwise_outputs(q, k, v, gam, wl.chunk, ws, g=g, out=y)
+        if ev is not None:
+            ev[2].record()
+
+    for _ in range(args.warmup):
+        step()
+    ops.check_device_error()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(K):
+        step(evs[i])
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    ops.check_device_error()
+    ms_total = start.elapsed_time(end)
+    ms_state = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    ms_out = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    ms_step = max_over_ranks(ms_total / K, world)
+    tokens = sum_over_ranks(wl.B * wl.T, world)
+    value = tokens / (ms_step / 1e3)
+
+    # roofline of the dominant (output) kernel, algorithmic counts
+    chunk_exec = max(wl.chunk, 128)
+    f_out, f_state, b_in, b_out = alg_counts(wl, chunk_exec)
+    units = wl.B * wl.T * wl.H                      # token-heads per launch
+    flops_launch = f_out * units
+    bytes_launch = (b_in + b_out) * units
+    t_out = ms_out / 1e3
+    peak_bw = pk["hbm_gbs"]
+    peak_tf = pk["bf16_tflops"]
+    t_mem, t_tc = bytes_launch / (peak_bw * 1e9), flops_launch / (peak_tf * 1e12)
+    traffic = traffic_from_profile()
+    if t_mem >= t_tc:
+        ach = bytes_launch / t_out / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peak_bw, "unit": "GB/s",
+                "frac": ach / peak_bw, "traffic": traffic}
+    else:
+        ach = flops_launch / t_out / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": ach / peak_tf, "traffic": traffic}
+    roof.update({"kernel": "output_kernel (tcgen05)", "peak_source": f"{pk_kind} (burst)",
+                 "algorithmic_flops_per_launch": flops_launch,
+                 "algorithmic_bytes_per_launch": bytes_launch, "launch_ms": ms_out})
+    step_flops = (f_out + f_state) * units
+    tensor = {"achieved_tflops": step_flops / (ms_step / 1e3) / 1e12,
+              "peak_tflops": peak_tf, "frac": step_flops / (ms_step / 1e3) / 1e12 / peak_tf,
+              "peak_source": f"{pk_kind} bf16 (burst)",
+              "spec_peak_tflops": 2250.0,
+              "frac_of_spec": step_flops / (ms_step / 1e3) / 1e12 / 2250.0,
+              "algorithmic_flops_per_step": step_flops,
+              "counting": f"per token-head (C+1)(dk+dv) + 4 dk dv, C={chunk_exec}"}
+    step_bytes = (b_in + b_out) * units + wl.B * wl.H * wl.dk * wl.dv * 4
+    hbm = {"achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9, "peak_gbs": peak_bw,
+           "frac": step_bytes / (ms_step / 1e3) / 1e9 / peak_bw,
+           "algorithmic_bytes_per_step": step_bytes}
+    kernels = {"state_kernel_ms": ms_state, "output_kernel_ms": ms_out, "step_ms": ms_total / K}
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hg = (t.to("cpu").pin_memory() for t in (q, k, v, g))
+        hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        hS = torch.empty(S.shape, dtype=S.dtype).pin_memory()
+        dq, dk_, dv_, dg = (torch.empty_like(t) for t in (q, k, v, g))
+
+        def e2e_step():
+            for d, hsrc in ((dq, hq), (dk_, hk), (dv_, hv), (dg, hg)):
+                d.copy_(hsrc, non_blocking=True)
+            ops.chunkwise_fwd(dq, dk_, dv_, gam, wl.chunk, g=dg, out=y, state_out=S,
+                              workspace=ws)
+            hy.copy_(y, non_blocking=True)
+            hS.copy_(S, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        Ke = max(3, min(K, 10))
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(Ke):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / Ke, world)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg))
+        d2h = hy.numel() * hy.element_size() + hS.numel() * hS.element_size()
+        e2e = {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "ms_per_step": ms_e2e,
+               "steps": Ke, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "api": "ops.chunkwise_fwd (C ABI retention_chunkwise_fwd) from pinned host memory"}
+        del hq, hk, hv, hg, dq, dk_, dv_, dg
+    del q, k, v, g, y, ws
+    torch.cuda.empty_cache()
+    return {"value": value, "ms_per_step": ms_step, "roofline": roof, "tensor": tensor,
+            "hbm": hbm, "kernels": kernels, "e2e": e2e, "clocks": clocks,
+            "gpu_launches": 2 * K, "wl": wl}
+
+
+def run_decode(args, world, rank, pk, pk_kind):
+    from linear_recurrent_sequence_retention_b200 import ops
+    wl = W.WORKLOADS[DECODE]
+    dev = torch.device("cuda")
+    N, H, dk, dv = wl.B, wl.H, wl.dk, wl.dv
+    gam = W.head_gammas(H)
+    S = torch.empty(N, H, dk, dv, device=dev, dtype=torch.float32)
+    # prefill: state-only chunkwise pass over 8192 tokens, in groups of sequences
+    grp = 16
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + rank)
+    sc = 1.0 / math.sqrt(dk)
+    ws = None
+    for n0 in range(0, N, grp):
+        kk = (torch.randn(grp, wl.T, H, dk, generator=gen, device=dev) * sc).to(torch.bfloat16)
+        vv = (torch.randn(grp, wl.T, H, dv, generator=gen, device=dev) * sc).to(torch.bfloat16)
+        if ws is None:
+            ws = ops.alloc_workspace(ops.chunkwise_workspace_size(torch.bfloat16, wl.chunk, grp,
+                                                                  wl.T, H, dk, dv), dev)
+        ops.chunkwise_states(kk, vv, gam, wl.chunk, state_out=S[n0:n0 + grp], workspace=ws)
+        del kk, vv
+    torch.cuda.synchronize()
+    del ws
+    steps = wl.decode_steps
+    qs = (torch.randn(steps, N, H, dk, generator=gen, device=dev) * sc).to(torch.bfloat16)
+    ks = (torch.randn(steps, N, H, dk, generator=gen, device=dev) * sc).to(torch.bfloat16)
+    vs = (torch.randn(steps, N, H, dv, generator=gen, device=dev) * sc).to(torch.bfloat16)
+    o = torch.empty(N, H, dv, device=dev, dtype=torch.float32)
+    for i in range(max(3, args.warmup)):
+        ops.recurrent_step(qs[i], ks[i], vs[i], gam, S, out=o)
+    ops.check_device_error()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        ops.recurrent_step(qs[i], ks[i], vs[i], gam, S, out=o)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ops.check_device_error()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    state_bytes = N * H * dk * dv * 4
+    step_bytes = 2 * state_bytes + N * H * (2 * dk + dv) * 2 + N * H * dv * 4
+    ach = step_bytes / (ms / 1e3) / 1e9
+    ranks_tokens = sum_over_ranks(N, world)
+    del qs, ks, vs, S, o
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "steps": steps, "ms_per_step": ms,
+            "steps_per_s": 1e3 / ms, "tokens_per_s": ranks_tokens / (ms / 1e3),
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / pk["hbm_gbs"], "peak_source": pk_kind,
+                         "frac_of_8tbs": ach / 8000.0,
+                         "algorithmic_bytes_per_launch": step_bytes,
+                         "kernel": "decode_step_kernel"},
+            "gpu_launches": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--B", type=int, default=None, help="override the headline batch (profiling)")
+    ap.add_argument("--T", type=int, default=None, help="override the headline length (profiling)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("warm-up below 3 steps is not allowed; using 3")
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    pk, pk_kind = peaks()
+    if args.B or args.T:
+        import dataclasses
+        base = W.WORKLOADS[HEADLINE]
+        B, T = args.B or base.B, args.T or base.T
+        W.WORKLOADS[HEADLINE] = dataclasses.replace(base, B=B, T=T,
+                                                    name=f"{base.name}@B{B}_T{T}")
+    wl = W.WORKLOADS[HEADLINE]
+
+    if args.impl == "reference":
+        # The CPU reference arm: the fp64 oracle, rank 0 only, bounded samples.
+        if rank == 0:
+            for i in range(args.warmup):
+                oracle_sample_step(wl, i, wl.chunk)
+            times = [oracle_sample_step(wl, i, wl.chunk) for i in range(args.steps)]
+            ms = 1e3 * float(np.sum(times)) / args.steps
+            val = wl.T / wl.H / (ms / 1e3)
+            line = {"metric": METRIC, "value": val, "unit": "tokens/s", "impl": "reference",
+                    "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                    "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                    "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                    "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H,
+                               "d_k": wl.dk, "d_v": wl.dv, "chunk": wl.chunk,
+                               "step": "one (sequence, head) pair of the workload"},
+                    "cpu_baseline": {"value": val, "unit": "tokens/s", "kind": "oracle",
+                                     "cores": blas_threads(),
+                                     "sample": f"each step: one of the {wl.B * wl.H} (sequence, "
+                                               f"head) pairs, {wl.T} tokens, numpy float64"},
+                    "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                            "d2h_bytes_per_step": 0}}
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device (use --impl reference for the CPU arm)"
+    head = run_headline(args, world, rank, pk, pk_kind)
+    dec = None if args.no_decode else run_decode(args, world, rank, pk, pk_kind)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(wl, args.cpu_seconds)
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": head["value"],
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "B_per_gpu": wl.B, "T": wl.T, "H": wl.H,
+                       "d_k": wl.dk, "d_v": wl.dv, "chunk": wl.chunk,
+                       "epilogue": "per-head GroupNorm (eps 1e-5) + swish gate, y bf16",
+                       "state_out": "f32 final state", "parallelism": f"dp{world}",
+                       "l2": f"inputs ({wl.B * wl.T * wl.H * (2 * wl.dk + 2 * wl.dv) * 2 / 1e6:.0f} MB "
+                             "per step) larger than L2; no flush"},
+            "roofline": head["roofline"],
+            "tensor": head["tensor"],
+            "hbm": head["hbm"],
+            "kernels": head["kernels"],
+            "decode": dec,
+            "e2e": head["e2e"],
+            "cpu_baseline": cpu,
+            "clocks": head["clocks"],
+            "gpu_launches": head["gpu_launches"] + (dec["gpu_launches"] if dec else 0),
+            "arithmetic": "bf16 tensor-core MMAs (tcgen05) with f32 accumulation; the "
+                          "carried state, decayed scores and zeta*K enter the MMAs as "
+                          "hi+lo bf16 pairs",
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -49,8 +49,10 @@
  *             The returned status covers argument validation and launch
  *             errors; faults and time-outs detected on the device are
  *             reported later by retention_check_device_error().
- *   Errors:   on any status other than RET_OK nothing has been enqueued and no
- *             output has been touched.  RET_ERR_UNSUPPORTED means the
+ *   Errors:   a validation status (RET_ERR_INVALID_ARG, RET_ERR_UNSUPPORTED,
+ *             RET_ERR_WORKSPACE) means nothing was enqueued and no output was
+ *             touched; RET_ERR_CUDA means a launch failed and earlier kernels
+ *             of the same call may have run.  RET_ERR_UNSUPPORTED means the
  *             arguments are valid but this build has no kernel for the shape
  *             or dtype combination; there is no fallback path.
  *   Aliasing: outputs must not overlap inputs, except that
@@ -178,6 +180,37 @@ RET_API ret_status retention_chunkwise_fwd(const void* q, const void* k, const v
                                    void* workspace, size_t workspace_bytes,
                                    int B, int T, int H, int dk, int dv,
                                    ret_stream_t stream);
+
+/*
+ * The two phases of retention_chunkwise_fwd as separate calls (same argument
+ * meanings and rules).  retention_chunkwise_states runs the chunk-to-chunk
+ * recurrence of the state (abeam.tech summary, 「長文の学習にはチャンク再帰を使う」:
+ * the state is updated at the end of every chunk): it stores the state
+ * entering every chunk in `workspace` and writes the final states to
+ * `state_out` (optional).  Alone, it is a prefill that yields the decode
+ * state without computing outputs.  retention_chunkwise_outputs then reads
+ * that workspace and writes `out` (o, or y when `ng` is given); it must
+ * follow a states call with identical q/k/v-independent arguments (dtype,
+ * gamma, chunk, cu_seqlens, sizes) on the same stream, with the workspace
+ * untouched in between.  `has_state_in` is nonzero when that states call was
+ * given a state_in.  Together they do exactly what retention_chunkwise_fwd
+ * does.
+ */
+RET_API ret_status retention_chunkwise_states(const void* k, const void* v, ret_dtype in_dtype,
+                                              const double* gamma, int chunk,
+                                              const int32_t* cu_seqlens, int nseq,
+                                              const float* state_in, float* state_out,
+                                              void* workspace, size_t workspace_bytes,
+                                              int B, int T, int H, int dk, int dv,
+                                              ret_stream_t stream);
+
+RET_API ret_status retention_chunkwise_outputs(const void* q, const void* k, const void* v,
+                                               ret_dtype in_dtype, const double* gamma,
+                                               int chunk, const int32_t* cu_seqlens, int nseq,
+                                               int has_state_in, void* out, ret_dtype out_dtype,
+                                               const ret_norm_gate* ng, const void* workspace,
+                                               size_t workspace_bytes, int B, int T, int H,
+                                               int dk, int dv, ret_stream_t stream);
 
 /*
  * One recurrent decode step for N independent sequences (abeam.tech summary,

@@ -151,6 +151,89 @@ size_t retention_chunkwise_workspace_size(ret_dtype in_dtype, int chunk, int B, 
   return p.bytes;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Validated arguments of one chunkwise call (any phase).
+struct ChunkCall {
+  ChunkPlan p;
+  ret::HeadDecay dec;
+  const void* g = nullptr;
+  DType g_t = DType::F32;
+  const float* gw = nullptr;
+  const float* gb = nullptr;
+  float eps = 0.f;
+  ret::ChunkWorkspace ws;
+  unsigned* err = nullptr;
+};
+
+constexpr int kPhaseStates = 1, kPhaseOutputs = 2;
+
+ret_status prepare_chunk_call(int phases, const void* q, const void* k, const void* v,
+                              ret_dtype in_dtype, const double* gamma, int chunk,
+                              const int32_t* cu_seqlens, int nseq, const float* state_in,
+                              const float* state_out, const void* out, ret_dtype out_dtype,
+                              const ret_norm_gate* ng, const void* workspace,
+                              size_t workspace_bytes, int B, int T, int H, int dk, int dv,
+                              ChunkCall* c) {
+  const bool varlen = cu_seqlens != nullptr;
+  if (varlen != (nseq > 0)) return RET_ERR_INVALID_ARG;
+  ret_status st = plan_chunkwise(in_dtype, chunk, B, T, H, dk, dv, varlen ? nseq : 0,
+                                 cu_seqlens, &c->p);
+  if (st != RET_OK) return st;
+  const bool has_tokens = c->p.L.Ttot > 0;
+  if (has_tokens && (!k || !v)) return RET_ERR_INVALID_ARG;
+  if ((phases & kPhaseOutputs) && has_tokens && (!q || !out)) return RET_ERR_INVALID_ARG;
+  if ((phases & kPhaseOutputs) && !dtype_ok(out_dtype)) return RET_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, out, state_in, state_out, cu_seqlens};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return RET_ERR_INVALID_ARG;
+  if (!make_decay(gamma, H, &c->dec)) return RET_ERR_INVALID_ARG;
+  if (ng && (phases & kPhaseOutputs)) {
+    if (!ng->g || !dtype_ok(ng->g_dtype) || !aligned16(ng->g)) return RET_ERR_INVALID_ARG;
+    if (!std::isfinite(ng->eps) || ng->eps < 0.f) return RET_ERR_INVALID_ARG;
+    c->g = ng->g;
+    c->g_t = dt(ng->g_dtype);
+    c->gw = ng->weight;
+    c->gb = ng->bias;
+    c->eps = ng->eps;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < c->p.bytes)
+    return RET_ERR_WORKSPACE;
+  c->ws.chunk_base = static_cast<int32_t*>(const_cast<void*>(workspace));
+  c->ws.states = static_cast<char*>(const_cast<void*>(workspace)) + c->p.meta;
+  c->ws.nslots = c->p.slots;
+  c->err = error_word();
+  if (!c->err) return RET_ERR_CUDA;
+  return RET_OK;
+}
+
+ret_status run_chunk_call(int phases, const ChunkCall& c, const void* q, const void* k,
+                          const void* v, ret_dtype in_dtype, const float* state_in,
+                          bool has_state_in, float* state_out, void* out, ret_dtype out_dtype,
+                          bool gated, int H, int dk, int dv, cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
+  if (phases & kPhaseStates) {
+    e = ret::launch_chunk_prep(c.p.L, c.ws, c.err, s);
+    if (e != cudaSuccess) return RET_ERR_CUDA;
+  }
+  if (c.p.tc)
+    e = ret::launch_chunkwise_tc(phases, q, k, v, c.p.L, state_in, has_state_in, state_out, out,
+                                 dt(out_dtype), c.g, c.g_t, c.gw, c.gb, c.eps, gated, c.ws, H, dk,
+                                 dv, c.dec, c.err, s);
+  else
+    e = ret::launch_chunkwise_simt(phases, q, k, v, dt(in_dtype), c.p.L, state_in, state_out,
+                                   out, dt(out_dtype), c.g, c.g_t, c.gw, c.gb, c.eps, gated, c.ws,
+                                   H, dk, dv, c.dec, c.err, s);
+  return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
 ret_status retention_chunkwise_fwd(const void* q, const void* k, const void* v,
                                    ret_dtype in_dtype, const double* gamma, int chunk,
                                    const int32_t* cu_seqlens, int nseq,
@@ -159,54 +242,51 @@ ret_status retention_chunkwise_fwd(const void* q, const void* k, const void* v,
                                    void* workspace, size_t workspace_bytes,
                                    int B, int T, int H, int dk, int dv,
                                    ret_stream_t stream) {
-  const bool varlen = cu_seqlens != nullptr;
-  if (varlen != (nseq > 0)) return RET_ERR_INVALID_ARG;
-  ChunkPlan p;
-  ret_status st = plan_chunkwise(in_dtype, chunk, B, T, H, dk, dv, varlen ? nseq : 0,
-                                 cu_seqlens, &p);
+  const int ph = kPhaseStates | kPhaseOutputs;
+  ChunkCall c;
+  ret_status st = prepare_chunk_call(ph, q, k, v, in_dtype, gamma, chunk, cu_seqlens, nseq,
+                                     state_in, state_out, out, out_dtype, ng, workspace,
+                                     workspace_bytes, B, T, H, dk, dv, &c);
   if (st != RET_OK) return st;
-  const bool has_tokens = p.L.Ttot > 0;
-  if (has_tokens && (!q || !k || !v || !out)) return RET_ERR_INVALID_ARG;
-  if (!dtype_ok(out_dtype)) return RET_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, out, state_in, state_out, cu_seqlens};
-  for (const void* ptr : ptrs)
-    if (ptr && !aligned16(ptr)) return RET_ERR_INVALID_ARG;
-  ret::HeadDecay dec;
-  if (!make_decay(gamma, H, &dec)) return RET_ERR_INVALID_ARG;
-  const void* g = nullptr;
-  DType g_t = DType::F32;
-  const float* gw = nullptr;
-  const float* gb = nullptr;
-  float eps = 0.f;
-  if (ng) {
-    if (!ng->g || !dtype_ok(ng->g_dtype) || !aligned16(ng->g)) return RET_ERR_INVALID_ARG;
-    if (!std::isfinite(ng->eps) || ng->eps < 0.f) return RET_ERR_INVALID_ARG;
-    g = ng->g;
-    g_t = dt(ng->g_dtype);
-    gw = ng->weight;
-    gb = ng->bias;
-    eps = ng->eps;
-  }
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
-      workspace_bytes < p.bytes)
-    return RET_ERR_WORKSPACE;
-  ret::ChunkWorkspace ws;
-  ws.chunk_base = static_cast<int32_t*>(workspace);
-  ws.states = static_cast<char*>(workspace) + p.meta;
-  ws.nslots = p.slots;
-  unsigned* err = error_word();
-  if (!err) return RET_ERR_CUDA;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = ret::launch_chunk_prep(p.L, ws, err, s);
-  if (e != cudaSuccess) return RET_ERR_CUDA;
-  if (p.tc)
-    e = ret::launch_chunkwise_tc(q, k, v, p.L, state_in, state_out, out, dt(out_dtype), g, g_t,
-                                 gw, gb, eps, ng != nullptr, ws, H, dk, dv, dec, err, s);
-  else
-    e = ret::launch_chunkwise_simt(q, k, v, dt(in_dtype), p.L, state_in, state_out, out,
-                                   dt(out_dtype), g, g_t, gw, gb, eps, ng != nullptr, ws, H, dk,
-                                   dv, dec, err, s);
-  return cuda_status(e);
+  return run_chunk_call(ph, c, q, k, v, in_dtype, state_in, state_in != nullptr, state_out, out,
+                        out_dtype, ng != nullptr, H, dk, dv,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+ret_status retention_chunkwise_states(const void* k, const void* v, ret_dtype in_dtype,
+                                      const double* gamma, int chunk,
+                                      const int32_t* cu_seqlens, int nseq,
+                                      const float* state_in, float* state_out,
+                                      void* workspace, size_t workspace_bytes,
+                                      int B, int T, int H, int dk, int dv,
+                                      ret_stream_t stream) {
+  const int ph = kPhaseStates;
+  ChunkCall c;
+  ret_status st = prepare_chunk_call(ph, nullptr, k, v, in_dtype, gamma, chunk, cu_seqlens,
+                                     nseq, state_in, state_out, nullptr, RET_F32, nullptr,
+                                     workspace, workspace_bytes, B, T, H, dk, dv, &c);
+  if (st != RET_OK) return st;
+  return run_chunk_call(ph, c, nullptr, k, v, in_dtype, state_in, state_in != nullptr,
+                        state_out, nullptr, RET_F32, false, H, dk, dv,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+ret_status retention_chunkwise_outputs(const void* q, const void* k, const void* v,
+                                       ret_dtype in_dtype, const double* gamma, int chunk,
+                                       const int32_t* cu_seqlens, int nseq, int has_state_in,
+                                       void* out, ret_dtype out_dtype, const ret_norm_gate* ng,
+                                       const void* workspace, size_t workspace_bytes,
+                                       int B, int T, int H, int dk, int dv,
+                                       ret_stream_t stream) {
+  const int ph = kPhaseOutputs;
+  ChunkCall c;
+  ret_status st = prepare_chunk_call(ph, q, k, v, in_dtype, gamma, chunk, cu_seqlens, nseq,
+                                     nullptr, nullptr, out, out_dtype, ng, workspace,
+                                     workspace_bytes, B, T, H, dk, dv, &c);
+  if (st != RET_OK) return st;
+  return run_chunk_call(ph, c, q, k, v, in_dtype, nullptr, has_state_in != 0, nullptr, out,
+                        out_dtype, ng != nullptr, H, dk, dv,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 ret_status retention_recurrent_step(const void* q, const void* k, const void* v,

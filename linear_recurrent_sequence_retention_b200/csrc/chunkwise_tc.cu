@@ -7,31 +7,38 @@
 //     O[i] = sum_{j<=i} gamma^(i-j) (q_i.k_j) v_j  +  gamma^(i+1) q_i S_(c-1)
 //     S_c  = gamma^L S_(c-1) + sum_j gamma^(L-1-j) k_j^T v_j
 //
-// Two kernels, both warp-specialised (warp 0: TMA producer, warp 1: TMEM
-// allocation + MMA issue, warps 2-5: one warpgroup that owns the 128 TMEM
+// Two warp-specialised kernels (warp 0: TMA producer, warp 1: TMEM
+// allocation + MMA issue, warps 2..9: two warpgroups that own the 128 TMEM
 // lanes):
 //
 //  state_kernel   one CTA per (sequence, head, 128 rows of d_k, NS columns of
-//                 d_v).  Walks the sequence's chunks in order with the state
-//                 block in TMEM (f32).  Before each chunk it stores the state
-//                 entering the chunk, rounded to bf16, in the workspace slot of
-//                 that chunk, scales TMEM by gamma^L, then accumulates
-//                 (zeta * K)^T V with the MMA (zeta_j = gamma^(L-1-j) applied to
-//                 the K rows in shared memory).  The final f32 state goes to
-//                 state_out.
+//                 d_v).  The state block lives in TMEM (f32) for the whole
+//                 sequence.  Warpgroup A, before each chunk, stores the state
+//                 entering it in the chunk's workspace slot (as a hi/lo bf16
+//                 pair), scales TMEM by gamma^L and releases the MMA; warpgroup
+//                 B turns every staged K tile into zeta*K hi/lo tiles
+//                 (zeta_j = gamma^(L-1-j)) ahead of the MMA, which accumulates
+//                 S += (zeta K)_hi^T V + (zeta K)_lo^T V.  The final f32 state
+//                 goes to state_out.
 //
 //  output_kernel  one CTA per (chunk, 128-row block r of the chunk, head,
-//                 NV-wide part of d_v); the two halves of d_v = 512 form a
-//                 2-CTA cluster that exchanges the GroupNorm statistics through
+//                 NV-wide part of d_v); the halves of d_v = 512 form a 2-CTA
+//                 cluster that exchanges the GroupNorm statistics through
 //                 distributed shared memory.  MMA order:
-//                   O  = Q S_(c-1)                 (then O *= gamma^(i+1) in TMEM)
+//                   O  = Q S_hi + Q S_lo           (then O *= gamma^(i+1) in TMEM)
 //                   Sc = Q K_kb^T  for kb = 0..r   (double-buffered in TMEM)
-//                   O += P_kb V_kb                 (P = decayed, masked Sc in bf16)
-//                 and the epilogue applies GroupNorm + swish gate or stores o.
+//                   O += P_hi V_kb + P_lo V_kb     (P = decayed, masked Sc, kept
+//                                                   in TMEM as the MMA's A operand)
+//                 Each epilogue warpgroup forms P for half of the keys and owns
+//                 half of the output columns in the GroupNorm + gate epilogue.
 //
-// All operand tiles are loaded by TMA (no multicast) into 128-byte-swizzled
-// shared memory; every wait is bounded (see tc_ptx.cuh) and on expiry the CTA
-// drains its in-flight copies and MMAs, frees TMEM and returns.
+// Precision: q, k, v enter the MMAs as the exact bf16 values they are; the
+// three rounded intermediates (decayed scores, carried state, zeta*K) enter as
+// hi + lo bf16 pairs (about 16 significant bits), so the result carries
+// f32-accumulation error only.  All tiles are loaded by TMA (no multicast)
+// into 128-byte-swizzled shared memory; every wait is bounded (tc_ptx.cuh)
+// and on expiry the CTA drains its in-flight copies and MMAs, frees TMEM and
+// returns.
 #include <cudaTypedefs.h>
 
 #include "launch.h"
@@ -44,8 +51,8 @@ using namespace tc;
 
 constexpr int kRowsPerTile = 128;     // MMA M, TMEM lanes, query rows per CTA
 constexpr int kKeysPerBlock = 128;    // keys per score tile
-constexpr int kThreads = 192;         // 6 warps
-constexpr int kEpiThreads = 128;      // warps 2..5
+constexpr int kThreads = 320;         // 10 warps
+constexpr int kWgThreads = 128;       // one warpgroup
 constexpr uint32_t kBox = 8192;       // one [64 rows][128 B] box
 constexpr uint32_t kTallBox = 16384;  // one [128 rows][128 B] box
 
@@ -77,6 +84,9 @@ __device__ __forceinline__ bool slot_to_chunk(const SeqLayout& L, const int32_t*
   return si.len > 0;
 }
 
+// Named barrier over the 256 threads of warps 2..9.
+__device__ __forceinline__ void wg2_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 // ===========================================================================
 // State kernel
 // ===========================================================================
@@ -98,7 +108,7 @@ struct StCfg {
   static constexpr uint32_t kKBytes = 2 * kBox;              // 64 tokens x 128 rows of d_k
   static constexpr uint32_t kVBytes = (NS / 64) * kBox;      // 64 tokens x NS
   static constexpr uint32_t kStage = 2 * kKBytes + kVBytes;  // K hi | K lo | V
-  static constexpr int kStages = (196608 / kStage) < 4 ? (196608 / kStage) : 4;
+  static constexpr int kStages = (200704 / kStage) < 6 ? (200704 / kStage) : 6;
   static constexpr uint32_t kSmem = kStages * kStage + 256;
 };
 
@@ -134,9 +144,9 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     for (int i = 0; i < NSTG; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
-      mbar_init(&kready[i], kEpiThreads);
+      mbar_init(&kready[i], kWgThreads);
     }
-    mbar_init(acc_ready, kEpiThreads);
+    mbar_init(acc_ready, kWgThreads);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -218,18 +228,16 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         mbar_wait_drain(drain, 0);
       }
     }
-  } else {
-    // ---------------- state warpgroup ----------------
+  } else if (warp < 6) {
+    // ---------------- warpgroup A: the state block in TMEM ----------------
     const int quad = warp & 3;
     const int row = quad * 32 + lane;            // TMEM lane = row of the state block
     const int i = 128 * m + row;                 // d_k index
     const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const size_t st_off = ((static_cast<size_t>(s) * p.H + h) * p.dk + i) * p.dv + NS * part;
-    int it = 0;
     bool ok = !*abort_flag;
     for (int c = 0; c < nch && ok; ++c) {
-      const int tok0 = a + c * L.chunk;
-      const int Lc = min(L.chunk, b - tok0);
+      const int Lc = min(L.chunk, b - (a + c * L.chunk));
       const long long slot = L.cu == nullptr
                                  ? static_cast<long long>(s) * ceil_div(L.T, L.chunk) + c
                                  : static_cast<long long>(p.chunk_base[s]) + c;
@@ -282,34 +290,6 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(acc_ready);
-      // zeta_j = gamma^(Lc-1-j) times the K rows of the chunk (0 past its end),
-      // split into a hi tile (in place) and a lo tile
-      for (int sb = 0; sb * kStTok < Lc; ++sb, ++it) {
-        const int st = it % NSTG;
-        if (!mbar_wait(&full[st], (it / NSTG) & 1, abort_flag, p.err)) { ok = false; break; }
-        const int t = threadIdx.x - 64;           // 0..127: box t/64, token row t%64
-        const int jtok = sb * kStTok + (t & 63);
-        const float z = jtok < Lc ? dec.pow(Lc - 1 - jtok) : 0.f;
-        uint8_t* rowb = smem + st * kStage + (t >> 6) * kBox + (t & 63) * 128;
-        uint4* hp = reinterpret_cast<uint4*>(rowb);
-        uint4* lp = reinterpret_cast<uint4*>(rowb + kKBytes);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          uint4 u = hp[e];
-          uint32_t w[4] = {u.x, u.y, u.z, u.w};
-          uint32_t wh[4], wl[4];
-#pragma unroll
-          for (int q2 = 0; q2 < 4; ++q2) {
-            __nv_bfloat162 hv = *reinterpret_cast<__nv_bfloat162*>(&w[q2]);
-            float2 f = __bfloat1622float2(hv);
-            pack_split(f.x * z, f.y * z, wh[q2], wl[q2]);
-          }
-          hp[e] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-          lp[e] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&kready[st]);
-      }
     }
     // final state
     if (ok && nch > 0) {
@@ -332,6 +312,38 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         float4 x = p.state_in ? *reinterpret_cast<const float4*>(p.state_in + st_off + j)
                               : make_float4(0.f, 0.f, 0.f, 0.f);
         *reinterpret_cast<float4*>(p.state_out + st_off + j) = x;
+      }
+    }
+  } else {
+    // ---------------- warpgroup B: zeta*K as hi/lo tiles, ahead of the MMA ----------------
+    const int t = threadIdx.x - 192;              // 0..127: box t/64, token row t%64
+    int it = 0;
+    bool ok = !*abort_flag;
+    for (int c = 0; c < nch && ok; ++c) {
+      const int Lc = min(L.chunk, b - (a + c * L.chunk));
+      for (int sb = 0; sb * kStTok < Lc; ++sb, ++it) {
+        const int st = it % NSTG;
+        if (!mbar_wait(&full[st], (it / NSTG) & 1, abort_flag, p.err)) { ok = false; break; }
+        const int jtok = sb * kStTok + (t & 63);
+        const float z = jtok < Lc ? dec.pow(Lc - 1 - jtok) : 0.f;
+        uint8_t* rowb = smem + st * kStage + (t >> 6) * kBox + (t & 63) * 128;
+        uint4* hp = reinterpret_cast<uint4*>(rowb);
+        uint4* lp = reinterpret_cast<uint4*>(rowb + kKBytes);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          uint4 u = hp[e];
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          uint32_t wh[4], wl[4];
+#pragma unroll
+          for (int q2 = 0; q2 < 4; ++q2) {
+            float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[q2]));
+            pack_split(f.x * z, f.y * z, wh[q2], wl[q2]);
+          }
+          hp[e] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          lp[e] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&kready[st]);
       }
     }
   }
@@ -370,19 +382,18 @@ struct OutParams {
 template <int DK, int NV>
 struct OutCfg {
   static constexpr uint32_t kQBytes = (DK / 64) * kTallBox;
-  static constexpr uint32_t kMiscBytes = 1024 + 512 + 1024;  // barriers | gamma^d table | stats
+  // barriers | gamma^d table | gamma^(127-d) table; the GroupNorm partials live
+  // in the Q region, which is free once every MMA has completed
+  static constexpr uint32_t kMiscBytes = 256 + 512 + 512;
   static constexpr int kStages = static_cast<int>((232448 - kQBytes - kMiscBytes) / kOutStage);
   static constexpr uint32_t kOffStages = kQBytes;
   static constexpr uint32_t kOffMisc = kOffStages + kStages * kOutStage;
   static constexpr uint32_t kSmem = kOffMisc + kMiscBytes;
-  // TMEM columns: O, then two score/P buffers of 128 columns
+  // TMEM columns: O, then two score buffers of 128 columns.  P of key piece j
+  // (keys 32j..32j+31) is written over that piece's own columns: 32j..32j+15
+  // hold P_hi (two keys per column), 32j+16..32j+31 hold P_lo.
   static constexpr uint32_t kTmemO = 0, kTmemS0 = 256, kTmemS1 = 384;
 };
-
-__device__ __forceinline__ float ld_gate(const void* g, int bf16, size_t idx) {
-  return bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(g)[idx])
-              : static_cast<const float*>(g)[idx];
-}
 
 template <int DK, int NV>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -391,6 +402,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               const OutParams p) {
   using C = OutCfg<DK, NV>;
   constexpr int NST = C::kStages;
+  constexpr int kHalf = NV / 2;                       // O columns per epilogue warpgroup
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffMisc);
   uint64_t* full = bars;                 // [NST]
@@ -398,13 +410,15 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   uint64_t* bar_q = empty + NST;
   uint64_t* bar_inter = bar_q + 1;
   uint64_t* bar_s = bar_inter + 1;       // [2] scores ready in TMEM
-  uint64_t* bar_p = bar_s + 2;           // [2] P (hi/lo) written over the scores
+  uint64_t* bar_p = bar_s + 2;           // [2] P written over the scores
   uint64_t* bar_o = bar_p + 2;           // all MMAs done
   uint64_t* drain = bar_o + 1;
   uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_hold + 1);
-  float* pow_tab = reinterpret_cast<float*>(smem + C::kOffMisc + 1024);      // gamma^d, d<128
-  float* stats = reinterpret_cast<float*>(smem + C::kOffMisc + 1024 + 512);  // [128][2]
+  float* pow_tab = reinterpret_cast<float*>(smem + C::kOffMisc + 256);    // gamma^d
+  float* rev_tab = reinterpret_cast<float*>(smem + C::kOffMisc + 768);    // gamma^(127-d)
+  float* wg_part = reinterpret_cast<float*>(smem);                        // [2][2][128], after bar_o
+  float* stats = reinterpret_cast<float*>(smem + 2048);                   // [128][2], after bar_o
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int part = blockIdx.x % p.parts;
@@ -431,7 +445,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     mbar_init(bar_inter, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_s[i], 1);
-      mbar_init(&bar_p[i], kEpiThreads);
+      mbar_init(&bar_p[i], 2 * kWgThreads);
     }
     mbar_init(bar_o, 1);
     mbar_init(drain, 1);
@@ -451,6 +465,10 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem = *tmem_hold;
 
+  // Unit sequence shared by producer and MMA issuer, one 32 KB stage each:
+  //   [S_hi and S_lo of d_k rows 64u..64u+63, u < DK/64 (if the chunk reads a state)],
+  //   K(0), then for kb = 0..r: [K(kb+1) if kb < r], V(kb) keys 0-63, V(kb) keys 64-127.
+  // K(kb) is DK/128 units of 128 keys x 128 d_k.
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0 && !*abort_flag) {
@@ -463,7 +481,6 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         tma_load_2d(smem + u * kTallBox, &tmQ, bar_q, h * DK + 64 * u, t0);
       int it = 0;
       bool ok = true;
-      // one stage per unit, in the MMA issue order
       auto next = [&](uint32_t bytes) -> uint8_t* {
         const int st = it % NST;
         if (!mbar_wait(&empty[st], ((it / NST) & 1) ^ 1, abort_flag, p.err)) return nullptr;
@@ -543,11 +560,9 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const uint32_t sb = stage_wait();
             if (!sb) { ok = false; break; }
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sdesc_sw128(q_base + u * kTallBox + kk * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(sb + kk * 2048, kBox, 1024);
-              mma_bf16(tmem + C::kTmemO, ad, bd, id_qs, (u | hl | kk) != 0);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(tmem + C::kTmemO, sdesc_sw128(q_base + u * kTallBox + kk * 32, 16, 1024),
+                       sdesc_sw128(sb + kk * 2048, kBox, 1024), id_qs, (u | hl | kk) != 0);
             issued = true;
             stage_free();
           }
@@ -562,9 +577,9 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const int qbox = ku * 2 + kk / 4;
-            const uint64_t ad = sdesc_sw128(q_base + qbox * kTallBox + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sb + (kk / 4) * kTallBox + (kk & 3) * 32, 16, 1024);
-            mma_bf16(dst, ad, bd, id_qk, (ku | kk) != 0);
+            mma_bf16(dst, sdesc_sw128(q_base + qbox * kTallBox + (kk & 3) * 32, 16, 1024),
+                     sdesc_sw128(sb + (kk / 4) * kTallBox + (kk & 3) * 32, 16, 1024), id_qk,
+                     (ku | kk) != 0);
           }
           issued = true;
           stage_free();
@@ -574,7 +589,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       };
       if (ok) ok = issue_qk(0);
       for (int kb = 0; kb <= r && ok; ++kb) {
-        // scores for the next key block go to the other buffer while P_kb is formed
+        // scores of the next key block go to the other buffer while P_kb is formed
         if (kb + 1 <= r && !issue_qk(kb + 1)) { ok = false; break; }
         if (!mbar_wait(&bar_p[kb & 1], (kb >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
@@ -584,7 +599,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           if (!sb) { ok = false; break; }
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const int ks = vu * 4 + kk;                      // 16 keys: 16ks .. 16ks+15
+            const int ks = vu * 4 + kk;                      // keys 16ks .. 16ks+15
             const uint32_t a_hi = pbuf + 32 * (ks >> 1) + 8 * (ks & 1);
             const uint64_t bd = sdesc_sw128(sb + kk * 2048, kBox, 1024);
             mma_bf16_ts(tmem + C::kTmemO, a_hi, bd, id_pv, need_inter || kb > 0 || ks > 0);
@@ -601,27 +616,31 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
     }
   } else {
-    // ---------------- epilogue warpgroup ----------------
+    // ---------------- epilogue: warpgroup wg owns key pieces 2wg, 2wg+1 and O columns
+    // [wg*NV/2, (wg+1)*NV/2) ----------------
+    const int wg = (warp - 2) >> 2;                   // 0 or 1
     const int quad = warp & 3;
     const int row = quad * 32 + lane;                 // query row within the block
     const int i = r * kRowsPerTile + row;              // row within the chunk
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const int et = threadIdx.x - 64;                  // 0..127
-    pow_tab[et] = dec.pow(et);
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const int et = threadIdx.x - 64;                  // 0..255
+    if (et < 128) pow_tab[et] = dec.pow(et);
+    else rev_tab[et - 128] = dec.pow(255 - et);
+    wg2_sync();
     bool ok = !*abort_flag;
+    const uint32_t o_cols = tmem + lane_off + C::kTmemO + wg * kHalf;
     if (ok && need_inter) {
       ok = mbar_wait(bar_inter, 0, abort_flag, p.err);
       if (ok) {
         tc_fence_after();
         const float sc = dec.pow(i + 1);
-        for (int j = 0; j < NV / 32; ++j) {
+        for (int j = 0; j < kHalf / 32; ++j) {
           float x[32];
-          tmem_ld32(tmem + lane_off + C::kTmemO + 32 * j, x);
+          tmem_ld32(o_cols + 32 * j, x);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) x[e] *= sc;
-          tmem_st32(tmem + lane_off + C::kTmemO + 32 * j, x);
+          tmem_st32(o_cols + 32 * j, x);
         }
         tmem_wait_st();
       }
@@ -636,57 +655,78 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const int key_lim = si.len - kKeysPerBlock * kb;   // keys j' >= key_lim are past the chunk
       const uint32_t buf = tmem + lane_off + (sb ? C::kTmemS1 : C::kTmemS0);
 #pragma unroll 1
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 2 * wg; j < 2 * wg + 2; ++j) {
         float x[32];
         tmem_ld32(buf + 32 * j, x);
+        float wv[32];
+        if (diag) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int jp = 32 * j + e;
+            wv[e] = jp <= row ? pow_tab[row - jp] : 0.f;
+          }
+        } else {
+          const float4* rt = reinterpret_cast<const float4*>(rev_tab + 32 * j);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 t4 = rt[e];
+            wv[4 * e] = arow * t4.x; wv[4 * e + 1] = arow * t4.y;
+            wv[4 * e + 2] = arow * t4.z; wv[4 * e + 3] = arow * t4.w;
+          }
+        }
+        if (key_lim < 32 * j + 32) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (32 * j + e >= key_lim) wv[e] = 0.f;
+        }
         tmem_wait_ld();
-        uint32_t w[32];
+        float pw[32];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          float pv[2];
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const int jp = 32 * j + e + t;
-            float wgt;
-            if (diag) wgt = (jp <= row) ? pow_tab[row - jp] : 0.f;
-            else wgt = arow * pow_tab[127 - jp];
-            if (jp >= key_lim) wgt = 0.f;
-            pv[t] = x[e + t] * wgt;
-          }
-          // columns 32j .. 32j+15: P_hi of keys 32j .. 32j+31, two per column;
-          // columns 32j+16 .. 32j+31: P_lo of the same keys
-          pack_split(pv[0], pv[1], w[e >> 1], w[16 + (e >> 1)]);
+          uint32_t hi, lo;
+          pack_split(x[e] * wv[e], x[e + 1] * wv[e + 1], hi, lo);
+          pw[e >> 1] = __uint_as_float(hi);
+          pw[16 + (e >> 1)] = __uint_as_float(lo);
         }
-        tmem_st32(buf + 32 * j, *reinterpret_cast<float(*)[32]>(w));
+        tmem_st32(buf + 32 * j, pw);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_p[sb]);
     }
-    // final O
-    float mean = 0.f, m2 = 0.f;
     if (ok) ok = mbar_wait(bar_o, 0, abort_flag, p.err);
-    if (ok) {
-      tc_fence_after();
-      if (p.gated) {
-        float sum = 0.f;
-        for (int j = 0; j < NV / 32; ++j) {
+    if (ok) tc_fence_after();
+    // GroupNorm statistics of this part: mean, then centred sum of squares,
+    // each summed over the two warpgroups' column halves (barriers unconditional)
+    if (p.gated) {
+      float sum = 0.f;
+      if (ok) {
+        for (int j = 0; j < kHalf / 32; ++j) {
           float x[32];
-          tmem_ld32(tmem + lane_off + C::kTmemO + 32 * j, x);
+          tmem_ld32(o_cols + 32 * j, x);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) sum += x[e];
         }
-        mean = sum / NV;
-        for (int j = 0; j < NV / 32; ++j) {
+      }
+      wg_part[wg * 128 + row] = sum;
+      wg2_sync();
+      const float mean = (wg_part[row] + wg_part[128 + row]) * (1.0f / NV);
+      float m2 = 0.f;
+      if (ok) {
+        for (int j = 0; j < kHalf / 32; ++j) {
           float x[32];
-          tmem_ld32(tmem + lane_off + C::kTmemO + 32 * j, x);
+          tmem_ld32(o_cols + 32 * j, x);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) m2 += (x[e] - mean) * (x[e] - mean);
+          for (int e = 0; e < 32; ++e) m2 = fmaf(x[e] - mean, x[e] - mean, m2);
         }
+      }
+      wg_part[256 + wg * 128 + row] = m2;
+      wg2_sync();
+      if (wg == 0) {
         stats[2 * row] = mean;
-        stats[2 * row + 1] = m2;
+        stats[2 * row + 1] = wg_part[256 + row] + wg_part[384 + row];
       }
     }
   }
@@ -694,8 +734,8 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   tc_fence_before();
   __syncthreads();
   const bool ok_all = !*abort_flag;
-  float mean_all = 0.f, rstd = 0.f;
   if (p.parts > 1 && p.gated) cluster_sync();      // partner's stats are written
+  float mean_all = 0.f, rstd = 0.f;
   if (warp >= 2 && ok_all && p.gated) {
     const int row = (warp & 3) * 32 + lane;
     float mean = stats[2 * row], m2 = stats[2 * row + 1];
@@ -715,38 +755,62 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   if (p.parts > 1 && p.gated) cluster_sync();      // partner has finished reading ours
   if (warp >= 2 && ok_all) {
     tc_fence_after();
+    const int wg = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t o_cols = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::kTmemO + wg * kHalf;
     const bool live = row < nrows;
-    const size_t obase = (static_cast<size_t>(t0 + row) * p.H + h) * p.dv + NV * part;
-    for (int j = 0; j < NV / 32; ++j) {
+    const int col0 = NV * part + wg * kHalf;          // first d_v column of this warpgroup
+    const size_t obase = (static_cast<size_t>(t0 + row) * p.H + h) * p.dv + col0;
+    const float shift = -mean_all * rstd;
+    for (int j = 0; j < kHalf / 32; ++j) {
       float x[32];
-      tmem_ld32(tmem + lane_off + C::kTmemO + 32 * j, x);
+      tmem_ld32(o_cols + 32 * j, x);
       tmem_wait_ld();
       if (!live) continue;
       if (p.gated) {
-        const int c0 = h * p.dv + NV * part + 32 * j;
+        float gv[32];
+        if (p.g_bf16) {
+          const uint4* gp = reinterpret_cast<const uint4*>(
+              static_cast<const __nv_bfloat16*>(p.g) + obase + 32 * j);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float y = (x[e] - mean_all) * rstd;
-          if (p.gn_w) y *= p.gn_w[c0 + e];
-          if (p.gn_b) y += p.gn_b[c0 + e];
-          const float gv = ld_gate(p.g, p.g_bf16, obase + 32 * j + e);
-          x[e] = y * (gv / (1.0f + expf(-gv)));
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const uint4 u = gp[c4];
+            const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[q2]));
+              gv[8 * c4 + 2 * q2] = f.x;
+              gv[8 * c4 + 2 * q2 + 1] = f.y;
+            }
+          }
+        } else {
+          const float4* gp = reinterpret_cast<const float4*>(static_cast<const float*>(p.g) + obase + 32 * j);
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 f = gp[c4];
+            gv[4 * c4] = f.x; gv[4 * c4 + 1] = f.y; gv[4 * c4 + 2] = f.z; gv[4 * c4 + 3] = f.w;
+          }
         }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = fmaf(x[e], rstd, shift);
+        if (p.gn_w || p.gn_b) {
+          const int c0 = h * p.dv + col0 + 32 * j;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (p.gn_w) x[e] *= p.gn_w[c0 + e];
+            if (p.gn_b) x[e] += p.gn_b[c0 + e];
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] *= swish_fast(gv[e]);
       }
       if (p.out_bf16) {
         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + obase + 32 * j);
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint4 u;
-          u.x = pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]);
-          u.y = pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]);
-          u.z = pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]);
-          u.w = pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]);
-          dst[c4] = u;
-        }
+        for (int c4 = 0; c4 < 4; ++c4)
+          dst[c4] = make_uint4(pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]), pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]),
+                               pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]), pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]));
       } else {
         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + 32 * j);
 #pragma unroll
@@ -846,44 +910,46 @@ bool chunkwise_tc_supported(int dk, int dv, int chunk) {
 
 int chunkwise_tc_chunk(int chunk) { return chunk < 128 ? 128 : chunk; }
 
-cudaError_t launch_chunkwise_tc(const void* q, const void* k, const void* v,
-                                const SeqLayout& L, const float* state_in, float* state_out,
-                                void* out, DType out_t, const void* g, DType g_t,
-                                const float* gn_w, const float* gn_b, float eps, bool gated,
-                                ChunkWorkspace ws, int H, int dk, int dv,
+cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const void* v,
+                                const SeqLayout& L, const float* state_in, bool has_state_in,
+                                float* state_out, void* out, DType out_t, const void* g,
+                                DType g_t, const float* gn_w, const float* gn_b, float eps,
+                                bool gated, ChunkWorkspace ws, int H, int dk, int dv,
                                 const HeadDecay& dec, unsigned* err, cudaStream_t s) {
   if (!chunkwise_tc_supported(dk, dv, L.chunk)) return cudaErrorNotSupported;
-  // ---- state pass ----
-  const int NS = dv >= 256 ? 256 : dv;
-  StateParams sp;
-  sp.L = L;
-  sp.chunk_base = ws.chunk_base;
-  sp.state_in = state_in;
-  sp.state_out = state_out;
-  sp.ws = static_cast<__nv_bfloat16*>(ws.states);
-  sp.H = H;
-  sp.dk = dk;
-  sp.dv = dv;
-  sp.dec = dec;
-  sp.err = err;
   const uint64_t Ttot = static_cast<uint64_t>(L.Ttot > 0 ? L.Ttot : 1);
-  CUtensorMap mk_st, mv_st, mq, mk, mv, ms;
-  if (!make_map(&mk_st, k, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 64) ||
-      !make_map(&mv_st, v, static_cast<uint64_t>(H) * dv, Ttot, static_cast<uint64_t>(H) * dv, 64))
-    return cudaErrorInvalidValue;
-  cudaError_t e;
-  switch (NS) {
-    case 64: e = launch_state<64>(mk_st, mv_st, sp, s); break;
-    case 128: e = launch_state<128>(mk_st, mv_st, sp, s); break;
-    default: e = launch_state<256>(mk_st, mv_st, sp, s); break;
+  cudaError_t e = cudaSuccess;
+  if (phases & 1) {
+    // ---- state pass ----
+    const int NS = dv >= 256 ? 256 : dv;
+    StateParams sp;
+    sp.L = L;
+    sp.chunk_base = ws.chunk_base;
+    sp.state_in = state_in;
+    sp.state_out = state_out;
+    sp.ws = static_cast<__nv_bfloat16*>(ws.states);
+    sp.H = H;
+    sp.dk = dk;
+    sp.dv = dv;
+    sp.dec = dec;
+    sp.err = err;
+    CUtensorMap mk_st, mv_st;
+    if (!make_map(&mk_st, k, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 64) ||
+        !make_map(&mv_st, v, static_cast<uint64_t>(H) * dv, Ttot, static_cast<uint64_t>(H) * dv, 64))
+      return cudaErrorInvalidValue;
+    switch (NS) {
+      case 64: e = launch_state<64>(mk_st, mv_st, sp, s); break;
+      case 128: e = launch_state<128>(mk_st, mv_st, sp, s); break;
+      default: e = launch_state<256>(mk_st, mv_st, sp, s); break;
+    }
   }
-  if (e != cudaSuccess || L.Ttot == 0) return e;
+  if (e != cudaSuccess || L.Ttot == 0 || !(phases & 2)) return e;
   // ---- output pass ----
   const int NV = dv > 256 ? 256 : dv;
   OutParams op;
   op.L = L;
   op.chunk_base = ws.chunk_base;
-  op.has_state_in = state_in != nullptr;
+  op.has_state_in = has_state_in;
   op.out = out;
   op.out_bf16 = out_t == DType::BF16;
   op.g = g;
@@ -900,6 +966,7 @@ cudaError_t launch_chunkwise_tc(const void* q, const void* k, const void* v,
   op.dec = dec;
   op.err = err;
   const uint64_t srows = static_cast<uint64_t>(ws.nslots) * H * 2 * dk;   // hi and lo planes
+  CUtensorMap mq, mk, mv, ms;
   if (!make_map(&mq, q, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 128) ||
       !make_map(&mk, k, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 128) ||
       !make_map(&mv, v, static_cast<uint64_t>(H) * dv, Ttot, static_cast<uint64_t>(H) * dv, 64) ||

@@ -15,8 +15,8 @@ enum class DType { F32 = 0, BF16 = 1 };
 // Workspace layout of the chunkwise forward:
 //   [meta: chunk_base int32[nseq+1], rounded up to 256 B][states]
 // states hold the state entering every chunk, one slot per chunk:
-//   [slot][H][dk][dv] float32 on the CUDA-core path; [slot][H][2][dk][dv]
-//   bfloat16 on the tensor-core path (the state as hi + lo bf16 parts).
+//   [slot][H][dk][dv], float32 on the CUDA-core path and float16 (the MMA
+//   operand of the cross-chunk read) on the tensor-core path.
 struct ChunkWorkspace {
   int32_t* chunk_base;   // device, nseq+1 entries (varlen only; else unused)
   void* states;          // device
@@ -33,7 +33,10 @@ cudaError_t launch_parallel_simt(const void* q, const void* k, const void* v, DT
 cudaError_t launch_chunk_prep(const SeqLayout& L, ChunkWorkspace ws, unsigned* err,
                               cudaStream_t s);
 
-cudaError_t launch_chunkwise_simt(const void* q, const void* k, const void* v, DType in_t,
+// phases: bit 0 = state pass (per-chunk states into the workspace, state_out),
+//         bit 1 = output pass (reads the workspace written by a state pass).
+cudaError_t launch_chunkwise_simt(int phases, const void* q, const void* k, const void* v,
+                                  DType in_t,
                                   const SeqLayout& L, const float* state_in, float* state_out,
                                   void* out, DType out_t, const void* g, DType g_t,
                                   const float* gn_w, const float* gn_b, float eps, bool gated,
@@ -51,8 +54,9 @@ cudaError_t launch_norm_gate(const void* o, DType o_t, const void* g, DType g_t,
 // Tensor-core (tcgen05) chunkwise forward for bf16 inputs.
 bool chunkwise_tc_supported(int dk, int dv, int chunk);
 int chunkwise_tc_chunk(int chunk);  // chunk length the kernels evaluate
-cudaError_t launch_chunkwise_tc(const void* q, const void* k, const void* v,
-                                const SeqLayout& L, const float* state_in, float* state_out,
+cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const void* v,
+                                const SeqLayout& L, const float* state_in, bool has_state_in,
+                                float* state_out,
                                 void* out, DType out_t, const void* g, DType g_t,
                                 const float* gn_w, const float* gn_b, float eps, bool gated,
                                 ChunkWorkspace ws, int H, int dk, int dv,

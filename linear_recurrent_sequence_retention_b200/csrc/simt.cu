@@ -387,12 +387,13 @@ cudaError_t parallel_typed(const void* q, const void* k, const void* v, void* o,
 }
 
 template <typename Tin, typename To, typename Tg>
-cudaError_t chunkwise_typed(const void* q, const void* k, const void* v, const SeqLayout& L,
+cudaError_t chunkwise_typed(int phases, const void* q, const void* k, const void* v,
+                            const SeqLayout& L,
                             const float* state_in, float* state_out, void* out, const void* g,
                             const float* gn_w, const float* gn_b, float eps, bool gated,
                             ChunkWorkspace ws, int H, int dk, int dv, const HeadDecay& dec,
                             cudaStream_t s) {
-  {
+  if (phases & 1) {
     size_t smem = sizeof(float) * (kStateTok * dk + kStateTok * 32);
     auto kern = chunk_state_simt_kernel<Tin>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -405,7 +406,7 @@ cudaError_t chunkwise_typed(const void* q, const void* k, const void* v, const S
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (L.Ttot == 0) return cudaSuccess;
+  if (L.Ttot == 0 || !(phases & 2)) return cudaSuccess;
   size_t smem = sizeof(float) * (2 * kRows * (dk + 1) + kKeys * dv + kRows * (kKeys + 1) +
                                  kRows * 8);
   auto kern = chunk_out_simt_kernel<Tin, To, Tg>;
@@ -446,7 +447,8 @@ cudaError_t launch_chunk_prep(const SeqLayout& L, ChunkWorkspace ws, unsigned* e
   return cudaGetLastError();
 }
 
-cudaError_t launch_chunkwise_simt(const void* q, const void* k, const void* v, DType in_t,
+cudaError_t launch_chunkwise_simt(int phases, const void* q, const void* k, const void* v,
+                                  DType in_t,
                                   const SeqLayout& L, const float* state_in, float* state_out,
                                   void* out, DType out_t, const void* g, DType g_t,
                                   const float* gn_w, const float* gn_b, float eps, bool gated,
@@ -457,16 +459,16 @@ cudaError_t launch_chunkwise_simt(const void* q, const void* k, const void* v, D
   using bf = __nv_bfloat16;
   if (out_t == DType::F32)
     return g_t == DType::F32
-               ? chunkwise_typed<float, float, float>(q, k, v, L, state_in, state_out, out, g,
+               ? chunkwise_typed<float, float, float>(phases, q, k, v, L, state_in, state_out, out, g,
                                                       gn_w, gn_b, eps, gated, ws, H, dk, dv,
                                                       dec, s)
-               : chunkwise_typed<float, float, bf>(q, k, v, L, state_in, state_out, out, g,
+               : chunkwise_typed<float, float, bf>(phases, q, k, v, L, state_in, state_out, out, g,
                                                    gn_w, gn_b, eps, gated, ws, H, dk, dv, dec,
                                                    s);
   return g_t == DType::F32
-             ? chunkwise_typed<float, bf, float>(q, k, v, L, state_in, state_out, out, g, gn_w,
+             ? chunkwise_typed<float, bf, float>(phases, q, k, v, L, state_in, state_out, out, g, gn_w,
                                                  gn_b, eps, gated, ws, H, dk, dv, dec, s)
-             : chunkwise_typed<float, bf, bf>(q, k, v, L, state_in, state_out, out, g, gn_w,
+             : chunkwise_typed<float, bf, bf>(phases, q, k, v, L, state_in, state_out, out, g, gn_w,
                                               gn_b, eps, gated, ws, H, dk, dv, dec, s);
 }
 

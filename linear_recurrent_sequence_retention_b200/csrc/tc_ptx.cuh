@@ -183,6 +183,18 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&r)[32]) 
       : "memory");
 }
 
+// 32 lanes x 16 columns store (same lane rule as tmem_ld32).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&u)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32"
+      " [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(
+          taddr),
+      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]),
+      "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]),
+      "r"(u[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -223,7 +235,7 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
-// D[tmem] (+)= A[smem] * B[smem]; issued by one thread.
+// D[tmem] (+)= A[smem] * B[smem] (16-bit operands, type given by idesc); one thread.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                          uint32_t idesc, bool accumulate) {
   asm volatile(
@@ -234,7 +246,7 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]; A is 128 lanes (rows) x 16 bf16 (K), two
+// D[tmem] (+)= A[tmem] * B[smem]; A is 128 lanes (rows) x 16 16-bit values (K), two
 // consecutive K elements packed per 32-bit column (element 2c in the low half),
 // so one K-step of A spans 8 columns starting at a_tmem.
 __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
@@ -285,9 +297,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&p);
 }
 
+// ---- hi/lo bf16 pairs ------------------------------------------------------------
+//
 // x = hi + lo with hi = bf16(x) and lo = bf16(x - hi): the pair carries about
 // 16 significant bits, so a product accumulated as hi*y + lo*y in f32 is exact
-// to ~2^-17 relative instead of bf16's 2^-9.
+// to ~2^-17 relative instead of bf16's 2^-9.  The kernels round the three
+// intermediates that feed an MMA (decayed scores, the carried state, zeta * K)
+// this way; the inputs q, k, v enter as the exact bf16 values they are.
 __device__ __forceinline__ void split_bf16(float x, float& hi, float& lo) {
   hi = __bfloat162float(__float2bfloat16_rn(x));
   lo = x - hi;
@@ -300,6 +316,13 @@ __device__ __forceinline__ void pack_split(float x0, float x1, uint32_t& hi, uin
   split_bf16(x1, h1, l1);
   hi = pack_bf16(h0, h1);
   lo = pack_bf16(l0, l1);
+}
+
+// swish(g) = g * sigmoid(g) with the fast exponential and division intrinsics
+// (relative error ~1e-6, far below the bf16/f32 output rounding).  For g ->
+// -inf the denominator overflows to inf and the result is the correct 0.
+__device__ __forceinline__ float swish_fast(float g) {
+  return __fdividef(g, 1.0f + __expf(-g));
 }
 
 }  // namespace tc

@@ -33,6 +33,8 @@ EXPORTED = (
     "retention_parallel_fwd",
     "retention_chunkwise_workspace_size",
     "retention_chunkwise_fwd",
+    "retention_chunkwise_states",
+    "retention_chunkwise_outputs",
     "retention_recurrent_step",
     "msr_norm_gate",
     "retention_check_device_error",
@@ -77,6 +79,13 @@ def lib():
     L.retention_chunkwise_fwd.argtypes = [vp, vp, vp, ci, cd, ci, vp, ci, vp, vp, vp, ci,
                                           ctypes.POINTER(NormGate), vp, ctypes.c_size_t,
                                           ci, ci, ci, ci, ci, vp]
+    L.retention_chunkwise_states.restype = ci
+    L.retention_chunkwise_states.argtypes = [vp, vp, ci, cd, ci, vp, ci, vp, vp, vp,
+                                             ctypes.c_size_t, ci, ci, ci, ci, ci, vp]
+    L.retention_chunkwise_outputs.restype = ci
+    L.retention_chunkwise_outputs.argtypes = [vp, vp, vp, ci, cd, ci, vp, ci, ci, vp, ci,
+                                              ctypes.POINTER(NormGate), vp, ctypes.c_size_t,
+                                              ci, ci, ci, ci, ci, vp]
     L.retention_recurrent_step.restype = ci
     L.retention_recurrent_step.argtypes = [vp, vp, vp, ci, cd, vp, vp, ci, ci, ci, ci, ci, vp]
     L.msr_norm_gate.restype = ci
@@ -227,6 +236,59 @@ def chunkwise_fwd(q, k, v, gamma, chunk, cu_seqlens=None, state_in=None, return_
         workspace.numel() * workspace.element_size(), B, T, H, dk, dv, _stream(stream))
     _check(st, "retention_chunkwise_fwd")
     return (out, state_out) if return_state else out
+
+
+def chunkwise_states(k, v, gamma, chunk, cu_seqlens=None, state_in=None, state_out=None,
+                     workspace=None, stream=None):
+    """State phase only: per-chunk states into ``workspace`` (returned) and the
+    final states into ``state_out`` (optional, float32 [nseq|B,H,dk,dv])."""
+    for t, n in ((k, "k"), (v, "v")):
+        _dev(t, n)
+    B, T, H, dk = k.shape
+    dv = v.shape[3]
+    nseq = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None:
+        _dev(cu_seqlens, "cu_seqlens")
+    need = lib().retention_chunkwise_workspace_size(_dt(k), chunk, B, T, H, dk, dv, nseq)
+    if need == 0:
+        raise RetentionError(RET_ERR_UNSUPPORTED if _dt(k) == RET_BF16 else RET_ERR_INVALID_ARG,
+                             "retention_chunkwise_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, k.device)
+    for t, n in ((state_in, "state_in"), (state_out, "state_out")):
+        if t is not None:
+            _dev(t, n)
+    st = lib().retention_chunkwise_states(
+        _ptr(k), _ptr(v), _dt(k), _gammas(gamma, H), int(chunk), _ptr(cu_seqlens), nseq,
+        _ptr(state_in), _ptr(state_out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), B, T, H, dk, dv, _stream(stream))
+    _check(st, "retention_chunkwise_states")
+    return workspace
+
+
+def chunkwise_outputs(q, k, v, gamma, chunk, workspace, cu_seqlens=None, has_state_in=False,
+                      g=None, gn_weight=None, gn_bias=None, eps=1e-5, out_dtype=None, out=None,
+                      stream=None):
+    """Output phase only: reads the workspace of a preceding chunkwise_states call."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (workspace, "workspace")):
+        _dev(t, n)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    nseq = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty(B, T, H, dv, device=q.device, dtype=out_dtype or q.dtype)
+    ng = None
+    if g is not None:
+        _dev(g, "g")
+        ng = NormGate(g.data_ptr(), _dt(g), gn_weight.data_ptr() if gn_weight is not None else None,
+                      gn_bias.data_ptr() if gn_bias is not None else None, float(eps))
+    st = lib().retention_chunkwise_outputs(
+        _ptr(q), _ptr(k), _ptr(v), _dt(q), _gammas(gamma, H), int(chunk), _ptr(cu_seqlens), nseq,
+        1 if has_state_in else 0, _ptr(out), _dt(out),
+        ctypes.byref(ng) if ng is not None else None, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), B, T, H, dk, dv, _stream(stream))
+    _check(st, "retention_chunkwise_outputs")
+    return out
 
 
 def recurrent_step(q, k, v, gamma, state, out_dtype=torch.float32, out=None, stream=None):

@@ -129,3 +129,28 @@ def test_repeat_calls_identical():
     ws.fill_(7)
     y2 = ops.chunkwise_fwd(*args, g=g.cuda(), workspace=ws)
     assert torch.equal(y1, y2)
+
+
+@pytest.mark.parametrize("varlen", [False, True])
+def test_phase_calls_equal_fused_call(varlen):
+    """retention_chunkwise_states + retention_chunkwise_outputs == retention_chunkwise_fwd."""
+    H, dk, dv, chunk = 2, 128, 256, 128
+    if varlen:
+        cu = torch.from_numpy(W.cu_seqlens_of([200, 0, 333])).cuda()
+        B, T = 1, 533
+    else:
+        cu, B, T = None, 2, 400
+    q, k, v, g = W.make_qkvg(B, T, H, dk, dv, "bf16", seed=17)
+    q, k, v, g = q.cuda(), k.cuda(), v.cuda(), g.cuda()
+    nst = 3 if varlen else B
+    s0 = W.make_state(nst, H, dk, dv, seed=1, scale=0.05).cuda()
+    gam = W.head_gammas(H)
+    y1, S1 = ops.chunkwise_fwd(q, k, v, gam, chunk, cu_seqlens=cu, state_in=s0, g=g,
+                               return_state=True)
+    S2 = torch.empty_like(S1)
+    ws = ops.chunkwise_states(k, v, gam, chunk, cu_seqlens=cu, state_in=s0, state_out=S2)
+    y2 = ops.chunkwise_outputs(q, k, v, gam, chunk, ws, cu_seqlens=cu, has_state_in=True, g=g)
+    ops.check_device_error()
+    assert torch.equal(y1, y2)
+    assert torch.equal(S1, S2)
+
