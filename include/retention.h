@@ -213,6 +213,42 @@ RET_API ret_status retention_chunkwise_outputs(const void* q, const void* k, con
                                                int dk, int dv, ret_stream_t stream);
 
 /*
+ * retention_chunkwise_fwd for callers that cannot allocate device memory.
+ * The paper has no counterpart: this is a deployment convenience.  Some
+ * callers have no allocator to hand: code that runs where cudaMalloc is not
+ * allowed or would stall (inside a memory pool's own bookkeeping, in embedded
+ * runtimes with a fixed device budget, or wherever the process must not grow
+ * its device footprint after start-up).  This entry point takes the same
+ * arguments as retention_chunkwise_fwd except the workspace: it uses a
+ * scratch array compiled into the library instead, and it allocates nothing
+ * (no cudaMalloc, no cudaFree, no allocating library call).
+ *   - The scratch array holds RETENTION_STATIC_WORKSPACE_BYTES on every GPU
+ *     that loads this library, for as long as the library stays loaded.
+ *   - A request whose retention_chunkwise_workspace_size() exceeds that
+ *     capacity returns RET_ERR_WORKSPACE and enqueues nothing; other
+ *     validation errors are those of retention_chunkwise_fwd.
+ *   - The first call on a device looks up the array's device address (one
+ *     cudaGetSymbolAddress per device, cached); make that first call before
+ *     any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; nothing in it needs to start at zero.  Calls that overlap on the
+ *     GPU (different streams, or several host threads) race on the array and
+ *     must be serialised by the caller.
+ * Outputs equal those of retention_chunkwise_fwd on the same arguments.
+ */
+#define RETENTION_STATIC_WORKSPACE_BYTES ((size_t)32 << 20)
+
+RET_API ret_status retention_chunkwise_fwd_static_ws(const void* q, const void* k,
+                                                     const void* v, ret_dtype in_dtype,
+                                                     const double* gamma, int chunk,
+                                                     const int32_t* cu_seqlens, int nseq,
+                                                     const float* state_in, float* state_out,
+                                                     void* out, ret_dtype out_dtype,
+                                                     const ret_norm_gate* ng,
+                                                     int B, int T, int H, int dk, int dv,
+                                                     ret_stream_t stream);
+
+/*
  * One recurrent decode step for N independent sequences (abeam.tech summary,
  * 「学習は並列、生成は状態更新」): for every (n, h), in this order,
  *     S <- gamma_h S + k^T v      (state updated in place)

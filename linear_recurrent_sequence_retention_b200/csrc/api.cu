@@ -341,3 +341,60 @@ ret_status retention_check_device_error(ret_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Chunkwise forward that allocates nothing: its scratch is a file-scope
+// device array of RETENTION_STATIC_WORKSPACE_BYTES, present on every device
+// that loads this library for as long as the library stays loaded.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticWorkspaceBytes = RETENTION_STATIC_WORKSPACE_BYTES;
+static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+std::mutex g_static_mu;
+void* g_static_addr[kMaxDevices] = {};
+
+// The host-side name g_static_workspace is only a stand-in for the device
+// array: its device address is resolved here, once per device, with that
+// device current, and cached for later calls.
+void* static_workspace() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr)
+      return nullptr;
+    g_static_addr[dev] = p;
+  }
+  return g_static_addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+ret_status retention_chunkwise_fwd_static_ws(const void* q, const void* k, const void* v,
+                                             ret_dtype in_dtype, const double* gamma, int chunk,
+                                             const int32_t* cu_seqlens, int nseq,
+                                             const float* state_in, float* state_out,
+                                             void* out, ret_dtype out_dtype,
+                                             const ret_norm_gate* ng,
+                                             int B, int T, int H, int dk, int dv,
+                                             ret_stream_t stream) {
+  const size_t need = retention_chunkwise_workspace_size(in_dtype, chunk, B, T, H, dk, dv,
+                                                         cu_seqlens ? nseq : 0);
+  if (need == 0)   // invalid or unsupported: let the regular validation name the reason
+    return retention_chunkwise_fwd(q, k, v, in_dtype, gamma, chunk, cu_seqlens, nseq, state_in,
+                                   state_out, out, out_dtype, ng, nullptr, 0, B, T, H, dk, dv,
+                                   stream);
+  if (need > kStaticWorkspaceBytes) return RET_ERR_WORKSPACE;
+  void* ws = static_workspace();
+  if (ws == nullptr) return RET_ERR_CUDA;
+  return retention_chunkwise_fwd(q, k, v, in_dtype, gamma, chunk, cu_seqlens, nseq, state_in,
+                                 state_out, out, out_dtype, ng, ws, kStaticWorkspaceBytes, B, T,
+                                 H, dk, dv, stream);
+}
+
+}  // extern "C"

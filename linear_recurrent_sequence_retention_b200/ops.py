@@ -27,6 +27,9 @@ RET_ERR_DEVICE_DATA = 6
 RET_F32 = 0
 RET_BF16 = 1
 
+# Capacity of the library's built-in scratch (RETENTION_STATIC_WORKSPACE_BYTES).
+STATIC_WORKSPACE_BYTES = 32 << 20
+
 EXPORTED = (
     "retention_abi_version",
     "retention_status_string",
@@ -35,6 +38,7 @@ EXPORTED = (
     "retention_chunkwise_fwd",
     "retention_chunkwise_states",
     "retention_chunkwise_outputs",
+    "retention_chunkwise_fwd_static_ws",
     "retention_recurrent_step",
     "msr_norm_gate",
     "retention_check_device_error",
@@ -86,6 +90,10 @@ def lib():
     L.retention_chunkwise_outputs.argtypes = [vp, vp, vp, ci, cd, ci, vp, ci, ci, vp, ci,
                                               ctypes.POINTER(NormGate), vp, ctypes.c_size_t,
                                               ci, ci, ci, ci, ci, vp]
+    L.retention_chunkwise_fwd_static_ws.restype = ci
+    L.retention_chunkwise_fwd_static_ws.argtypes = [vp, vp, vp, ci, cd, ci, vp, ci, vp, vp, vp,
+                                                    ci, ctypes.POINTER(NormGate),
+                                                    ci, ci, ci, ci, ci, vp]
     L.retention_recurrent_step.restype = ci
     L.retention_recurrent_step.argtypes = [vp, vp, vp, ci, cd, vp, vp, ci, ci, ci, ci, ci, vp]
     L.msr_norm_gate.restype = ci
@@ -288,6 +296,33 @@ def chunkwise_outputs(q, k, v, gamma, chunk, workspace, cu_seqlens=None, has_sta
         ctypes.byref(ng) if ng is not None else None, _ptr(workspace),
         workspace.numel() * workspace.element_size(), B, T, H, dk, dv, _stream(stream))
     _check(st, "retention_chunkwise_outputs")
+    return out
+
+
+def chunkwise_fwd_static_ws(q, k, v, gamma, chunk, cu_seqlens=None, state_in=None,
+                            state_out=None, g=None, gn_weight=None, gn_bias=None, eps=1e-5,
+                            out=None, out_dtype=None, stream=None):
+    """chunkwise_fwd without a workspace argument: the library uses its built-in
+    device scratch (STATIC_WORKSPACE_BYTES) and allocates nothing itself.
+    Outputs (and ``state_out``, if given) must be preallocated by the caller
+    only if they are passed; here they are created with torch for convenience."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    nseq = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty(B, T, H, dv, device=q.device, dtype=out_dtype or q.dtype)
+    ng = None
+    if g is not None:
+        _dev(g, "g")
+        ng = NormGate(g.data_ptr(), _dt(g), gn_weight.data_ptr() if gn_weight is not None else None,
+                      gn_bias.data_ptr() if gn_bias is not None else None, float(eps))
+    st = lib().retention_chunkwise_fwd_static_ws(
+        _ptr(q), _ptr(k), _ptr(v), _dt(q), _gammas(gamma, H), int(chunk), _ptr(cu_seqlens), nseq,
+        _ptr(state_in), _ptr(state_out), _ptr(out), _dt(out),
+        ctypes.byref(ng) if ng is not None else None, B, T, H, dk, dv, _stream(stream))
+    _check(st, "retention_chunkwise_fwd_static_ws")
     return out
 
 
