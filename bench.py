@@ -381,7 +381,7 @@ def run_decode(args, world, rank, pk, pk_kind):
     gam = W.head_gammas(H)
     S = torch.empty(N, H, dk, dv, device=dev, dtype=torch.float32)
     # prefill: state-only chunkwise pass over 8192 tokens, in groups of sequences
-    grp = 16
+    grp = min(16, N)
     gen = torch.Generator(device=dev)
     gen.manual_seed(1000 + rank)
     sc = 1.0 / math.sqrt(dk)
@@ -443,12 +443,21 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--B", type=int, default=None, help="override the headline batch (profiling)")
     ap.add_argument("--T", type=int, default=None, help="override the headline length (profiling)")
+    ap.add_argument("--no-headline", action="store_true", help="decode only (profiling)")
+    ap.add_argument("--decode-N", type=int, default=None, help="override the decode batch (profiling)")
+    ap.add_argument("--decode-steps", type=int, default=None, help="override the decode steps")
     args = ap.parse_args()
     if args.warmup < 3:
         log("warm-up below 3 steps is not allowed; using 3")
         args.warmup = 3
     world, rank, local = dist_setup()
     pk, pk_kind = peaks()
+    if args.decode_N or args.decode_steps:
+        import dataclasses
+        base = W.WORKLOADS[DECODE]
+        N, st = args.decode_N or base.B, args.decode_steps or base.decode_steps
+        W.WORKLOADS[DECODE] = dataclasses.replace(base, B=N, decode_steps=st,
+                                                  name=f"{base.name}@N{N}_steps{st}")
     if args.B or args.T:
         import dataclasses
         base = W.WORKLOADS[HEADLINE]
@@ -484,6 +493,13 @@ def main():
         return
 
     assert torch.cuda.is_available(), "bench.py needs a CUDA device (use --impl reference for the CPU arm)"
+    if args.no_headline:
+        dec = run_decode(args, world, rank, pk, pk_kind)
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "decode": dec, "n_gpus": world}), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     head = run_headline(args, world, rank, pk, pk_kind)
     dec = None if args.no_decode else run_decode(args, world, rank, pk, pk_kind)
     cpu = None

@@ -87,6 +87,21 @@ __device__ __forceinline__ bool slot_to_chunk(const SeqLayout& L, const int32_t*
 // Named barrier over the 256 threads of warps 2..9.
 __device__ __forceinline__ void wg2_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
+// AND of `v` over the 128 threads of warps 2..5 (named barrier 2); every one of
+// them gets the same answer, so loops that contain barrier 2 stay uniform.
+__device__ __forceinline__ bool wga_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u)
+      : "memory");
+  return r != 0;
+}
+
 // ===========================================================================
 // State kernel
 // ===========================================================================
@@ -108,20 +123,26 @@ struct StCfg {
   static constexpr uint32_t kKBytes = 2 * kBox;              // 64 tokens x 128 rows of d_k
   static constexpr uint32_t kVBytes = (NS / 64) * kBox;      // 64 tokens x NS
   static constexpr uint32_t kStage = 2 * kKBytes + kVBytes;  // K hi | K lo | V
-  static constexpr int kStages = (200704 / kStage) < 6 ? (200704 / kStage) : 6;
-  static constexpr uint32_t kSmem = kStages * kStage + 256;
+  // staging for the TMA store of the state entering a chunk: one 128 x 64
+  // box of the hi plane and one of the lo plane
+  static constexpr uint32_t kStaging = 2 * kTallBox;
+  static constexpr int kStagesFit = static_cast<int>((232448 - kStaging - 1024) / kStage);
+  static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
+  static constexpr uint32_t kOffStaging = kStages * kStage;
+  static constexpr uint32_t kSmem = kOffStaging + kStaging + 256;
 };
 
 template <int NS>
 __global__ void __launch_bounds__(kThreads, 1)
 state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-             const StateParams p) {
+             const __grid_constant__ CUtensorMap tmW, const StateParams p) {
   using SC = StCfg<NS>;
   constexpr int NSTG = SC::kStages;
   constexpr uint32_t kStage = SC::kStage;
   constexpr uint32_t kKBytes = SC::kKBytes;
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NSTG * kStage);
+  uint8_t* staging = smem + SC::kOffStaging;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SC::kOffStaging + SC::kStaging);
   uint64_t* full = bars;
   uint64_t* empty = full + NSTG;
   uint64_t* kready = empty + NSTG;
@@ -235,62 +256,87 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     const int i = 128 * m + row;                 // d_k index
     const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const size_t st_off = ((static_cast<size_t>(s) * p.H + h) * p.dk + i) * p.dv + NS * part;
-    bool ok = !*abort_flag;
+    const bool leader = threadIdx.x == 64;
+    if (leader) tma_prefetch_desc(&tmW);
+    bool ok = wga_all(!*abort_flag);
     for (int c = 0; c < nch && ok; ++c) {
       const int Lc = min(L.chunk, b - (a + c * L.chunk));
       const long long slot = L.cu == nullptr
                                  ? static_cast<long long>(s) * ceil_div(L.T, L.chunk) + c
                                  : static_cast<long long>(p.chunk_base[s]) + c;
       const bool slot_ok = slot >= 0 && slot < L.nslots;
-      const size_t hrow = ((static_cast<size_t>(slot_ok ? slot : 0) * p.H + h) * 2) * p.dk + i;
-      __nv_bfloat16* whi = p.ws + hrow * p.dv + NS * part;
-      __nv_bfloat16* wlo = p.ws + (hrow + p.dk) * p.dv + NS * part;
+      // workspace rows of this CTA's 128 d_k rows in the hi plane; lo follows dk rows later
+      const int wrow = static_cast<int>(((slot_ok ? slot : 0) * p.H + h) * 2 * p.dk) + 128 * m;
       if (c > 0) {
-        if (!mbar_wait(acc_full, (c - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+        ok = wga_all(mbar_wait(acc_full, (c - 1) & 1, abort_flag, p.err));
+        if (!ok) break;
         tc_fence_after();
       }
       const float gL = dec.pow(Lc);
+      const uint64_t gL2 = f2_make(gL, gL);
 #pragma unroll 1
-      for (int j = 0; j < NS / 32; ++j) {
-        float r[32];
+      for (int j = 0; j < NS / 32; j += 2) {       // 64 columns per TMA store box
+        float r[2][32];
         if (c == 0) {
-          if (p.state_in) {
-            const float4* src = reinterpret_cast<const float4*>(p.state_in + st_off + 32 * j);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              float4 x = src[e];
-              r[4 * e] = x.x; r[4 * e + 1] = x.y; r[4 * e + 2] = x.z; r[4 * e + 3] = x.w;
+          for (int hp = 0; hp < 2; ++hp) {
+            if (p.state_in) {
+              const float4* src = reinterpret_cast<const float4*>(p.state_in + st_off + 32 * (j + hp));
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float4 x = src[e];
+                r[hp][4 * e] = x.x; r[hp][4 * e + 1] = x.y; r[hp][4 * e + 2] = x.z; r[hp][4 * e + 3] = x.w;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) r[hp][e] = 0.f;
             }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = 0.f;
           }
         } else {
-          tmem_ld32(trow + 32 * j, r);
+          tmem_ld32(trow + 32 * j, r[0]);
+          tmem_ld32(trow + 32 * (j + 1), r[1]);
           tmem_wait_ld();
         }
-        if (slot_ok) {   // the state entering chunk c, as a hi/lo bf16 pair
-          uint4* dh = reinterpret_cast<uint4*>(whi + 32 * j);
-          uint4* dl = reinterpret_cast<uint4*>(wlo + 32 * j);
+        // the staging boxes are free once the previous store stopped reading them
+        if (leader) tma_store_wait_read();
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+        // row `row` of two 128 x 64 swizzled boxes (hi, lo): 16-byte piece cc of
+        // the row goes to piece cc ^ (row & 7)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint4 uh, ul;
-            pack_split(r[8 * e + 0], r[8 * e + 1], uh.x, ul.x);
-            pack_split(r[8 * e + 2], r[8 * e + 3], uh.y, ul.y);
-            pack_split(r[8 * e + 4], r[8 * e + 5], uh.z, ul.z);
-            pack_split(r[8 * e + 6], r[8 * e + 7], uh.w, ul.w);
-            dh[e] = uh;
-            dl[e] = ul;
-          }
+        for (int cc = 0; cc < 8; ++cc) {
+          const float* x = &r[cc >> 2][(cc & 3) * 8];
+          uint4 uh, ul;
+          pack_split(x[0], x[1], uh.x, ul.x);
+          pack_split(x[2], x[3], uh.y, ul.y);
+          pack_split(x[4], x[5], uh.z, ul.z);
+          pack_split(x[6], x[7], uh.w, ul.w);
+          const int off = row * 128 + ((cc ^ (row & 7)) << 4);
+          *reinterpret_cast<uint4*>(staging + off) = uh;
+          *reinterpret_cast<uint4*>(staging + kTallBox + off) = ul;
+        }
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+        if (leader && slot_ok) {
+          tma_store_2d(&tmW, staging, NS * part + 32 * j, wrow);
+          tma_store_2d(&tmW, staging + kTallBox, NS * part + 32 * j, wrow + p.dk);
+          tma_store_commit();
         }
 #pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] *= gL;
-        tmem_st32(trow + 32 * j, r);
+        for (int hp = 0; hp < 2; ++hp) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const uint64_t v2 = f2_mul(f2_make(r[hp][e], r[hp][e + 1]), gL2);
+            r[hp][e] = f2_lo(v2);
+            r[hp][e + 1] = f2_hi(v2);
+          }
+          tmem_st32(trow + 32 * (j + hp), r[hp]);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(acc_ready);
     }
+    if (leader) tma_store_wait_all();
     // final state
     if (ok && nch > 0) {
       if (mbar_wait(acc_full, (nch - 1) & 1, abort_flag, p.err)) {
@@ -329,18 +375,25 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         uint8_t* rowb = smem + st * kStage + (t >> 6) * kBox + (t & 63) * 128;
         uint4* hp = reinterpret_cast<uint4*>(rowb);
         uint4* lp = reinterpret_cast<uint4*>(rowb + kKBytes);
+        // every piece of the row gets the same factor, so visit the row's eight
+        // 16-byte pieces in the order e ^ (row & 7): lanes of 8 consecutive rows then
+        // touch 8 different bank groups instead of the same one
+        const int sw = t & 7;
+        uint4 u[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) u[e] = hp[e ^ sw];
+        const uint64_t z2 = f2_make(z, z);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          uint4 u = hp[e];
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          const uint32_t w[4] = {u[e].x, u[e].y, u[e].z, u[e].w};
           uint32_t wh[4], wl[4];
 #pragma unroll
           for (int q2 = 0; q2 < 4; ++q2) {
-            float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[q2]));
-            pack_split(f.x * z, f.y * z, wh[q2], wl[q2]);
+            const uint64_t p2 = f2_mul(f2_make(bf16_lo(w[q2]), bf16_hi(w[q2])), z2);
+            pack_split(f2_lo(p2), f2_hi(p2), wh[q2], wl[q2]);
           }
-          hp[e] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-          lp[e] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+          hp[e ^ sw] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          lp[e ^ sw] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
         }
         fence_proxy_async_smem();
         mbar_arrive(&kready[st]);
@@ -667,11 +720,14 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           }
         } else {
           const float4* rt = reinterpret_cast<const float4*>(rev_tab + 32 * j);
+          const uint64_t a2 = f2_make(arow, arow);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const float4 t4 = rt[e];
-            wv[4 * e] = arow * t4.x; wv[4 * e + 1] = arow * t4.y;
-            wv[4 * e + 2] = arow * t4.z; wv[4 * e + 3] = arow * t4.w;
+            const uint64_t w0 = f2_mul(f2_make(t4.x, t4.y), a2);
+            const uint64_t w1 = f2_mul(f2_make(t4.z, t4.w), a2);
+            wv[4 * e] = f2_lo(w0); wv[4 * e + 1] = f2_hi(w0);
+            wv[4 * e + 2] = f2_lo(w1); wv[4 * e + 3] = f2_hi(w1);
           }
         }
         if (key_lim < 32 * j + 32) {
@@ -684,7 +740,8 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           uint32_t hi, lo;
-          pack_split(x[e] * wv[e], x[e + 1] * wv[e + 1], hi, lo);
+          const uint64_t p2 = f2_mul(f2_make(x[e], x[e + 1]), f2_make(wv[e], wv[e + 1]));
+          pack_split(f2_lo(p2), f2_hi(p2), hi, lo);
           pw[e >> 1] = __uint_as_float(hi);
           pw[16 + (e >> 1)] = __uint_as_float(lo);
         }
@@ -696,37 +753,40 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
     if (ok) ok = mbar_wait(bar_o, 0, abort_flag, p.err);
     if (ok) tc_fence_after();
-    // GroupNorm statistics of this part: mean, then centred sum of squares,
-    // each summed over the two warpgroups' column halves (barriers unconditional)
+    // GroupNorm statistics of this part in one pass: sums of (x - x0) and
+    // (x - x0)^2 with x0 the row's first value in this warpgroup's half (a
+    // shift that keeps the sums well conditioned); the two halves combine as
+    // (mean, M2) pairs.  Barriers are unconditional.
     if (p.gated) {
-      float sum = 0.f;
+      float mean_w = 0.f, m2_w = 0.f;
       if (ok) {
+        uint64_t s1 = 0, s2 = 0;
+        float x0 = 0.f;
         for (int j = 0; j < kHalf / 32; ++j) {
           float x[32];
           tmem_ld32(o_cols + 32 * j, x);
           tmem_wait_ld();
+          if (j == 0) x0 = x[0];
+          const uint64_t nx0 = f2_make(-x0, -x0);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) sum += x[e];
+          for (int e = 0; e < 32; e += 2) {
+            const uint64_t d = f2_add(f2_make(x[e], x[e + 1]), nx0);
+            s1 = f2_add(s1, d);
+            s2 = f2_fma(d, d, s2);
+          }
         }
+        const float S1 = f2_lo(s1) + f2_hi(s1), S2 = f2_lo(s2) + f2_hi(s2);
+        mean_w = x0 + S1 * (1.0f / kHalf);
+        m2_w = fmaxf(S2 - S1 * S1 * (1.0f / kHalf), 0.f);
       }
-      wg_part[wg * 128 + row] = sum;
-      wg2_sync();
-      const float mean = (wg_part[row] + wg_part[128 + row]) * (1.0f / NV);
-      float m2 = 0.f;
-      if (ok) {
-        for (int j = 0; j < kHalf / 32; ++j) {
-          float x[32];
-          tmem_ld32(o_cols + 32 * j, x);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) m2 = fmaf(x[e] - mean, x[e] - mean, m2);
-        }
-      }
-      wg_part[256 + wg * 128 + row] = m2;
+      wg_part[wg * 128 + row] = mean_w;
+      wg_part[256 + wg * 128 + row] = m2_w;
       wg2_sync();
       if (wg == 0) {
-        stats[2 * row] = mean;
-        stats[2 * row + 1] = wg_part[256 + row] + wg_part[384 + row];
+        const float m0 = wg_part[row], m1 = wg_part[128 + row];
+        const float d = m1 - m0;
+        stats[2 * row] = 0.5f * (m0 + m1);
+        stats[2 * row + 1] = wg_part[256 + row] + wg_part[384 + row] + d * d * (0.5f * kHalf);
       }
     }
   }
@@ -792,8 +852,13 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             gv[4 * c4] = f.x; gv[4 * c4 + 1] = f.y; gv[4 * c4 + 2] = f.z; gv[4 * c4 + 3] = f.w;
           }
         }
+        const uint64_t rs2 = f2_make(rstd, rstd), sh2 = f2_make(shift, shift);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = fmaf(x[e], rstd, shift);
+        for (int e = 0; e < 32; e += 2) {
+          const uint64_t y2 = f2_fma(f2_make(x[e], x[e + 1]), rs2, sh2);
+          x[e] = f2_lo(y2);
+          x[e + 1] = f2_hi(y2);
+        }
         if (p.gn_w || p.gn_b) {
           const int c0 = h * p.dv + col0 + 32 * j;
 #pragma unroll
@@ -802,8 +867,19 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (p.gn_b) x[e] += p.gn_b[c0 + e];
           }
         }
+        // swish(g) = g / (1 + 2^(-g log2 e)); paired where the math allows
+        const uint64_t nl2e = f2_make(-1.4426950408889634f, -1.4426950408889634f);
+        const uint64_t one2 = f2_make(1.f, 1.f);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] *= swish_fast(gv[e]);
+        for (int e = 0; e < 32; e += 2) {
+          const uint64_t g2 = f2_make(gv[e], gv[e + 1]);
+          const uint64_t t2 = f2_mul(g2, nl2e);
+          const uint64_t d2 = f2_add(f2_make(exp2f_fast(f2_lo(t2)), exp2f_fast(f2_hi(t2))), one2);
+          const uint64_t s2 = f2_mul(g2, f2_make(rcp_fast(f2_lo(d2)), rcp_fast(f2_hi(d2))));
+          const uint64_t o2 = f2_mul(f2_make(x[e], x[e + 1]), s2);
+          x[e] = f2_lo(o2);
+          x[e + 1] = f2_hi(o2);
+        }
       }
       if (p.out_bf16) {
         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + obase + 32 * j);
@@ -862,15 +938,15 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
 }
 
 template <int NS>
-cudaError_t launch_state(const CUtensorMap& mk, const CUtensorMap& mv, const StateParams& sp,
-                         cudaStream_t s) {
+cudaError_t launch_state(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mw,
+                         const StateParams& sp, cudaStream_t s) {
   const size_t smem = StCfg<NS>::kSmem;
   auto kern = state_kernel<NS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(sp.L.nseq, sp.H, (sp.dk / 128) * (sp.dv / NS));
-  kern<<<grid, kThreads, smem, s>>>(mk, mv, sp);
+  kern<<<grid, kThreads, smem, s>>>(mk, mv, mw, sp);
   return cudaGetLastError();
 }
 
@@ -933,14 +1009,16 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
     sp.dv = dv;
     sp.dec = dec;
     sp.err = err;
-    CUtensorMap mk_st, mv_st;
+    CUtensorMap mk_st, mv_st, mw_st;
+    const uint64_t wrows = static_cast<uint64_t>(ws.nslots) * H * 2 * dk;   // hi and lo planes
     if (!make_map(&mk_st, k, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 64) ||
-        !make_map(&mv_st, v, static_cast<uint64_t>(H) * dv, Ttot, static_cast<uint64_t>(H) * dv, 64))
+        !make_map(&mv_st, v, static_cast<uint64_t>(H) * dv, Ttot, static_cast<uint64_t>(H) * dv, 64) ||
+        !make_map(&mw_st, ws.states, dv, wrows, dv, 128))
       return cudaErrorInvalidValue;
     switch (NS) {
-      case 64: e = launch_state<64>(mk_st, mv_st, sp, s); break;
-      case 128: e = launch_state<128>(mk_st, mv_st, sp, s); break;
-      default: e = launch_state<256>(mk_st, mv_st, sp, s); break;
+      case 64: e = launch_state<64>(mk_st, mv_st, mw_st, sp, s); break;
+      case 128: e = launch_state<128>(mk_st, mv_st, mw_st, sp, s); break;
+      default: e = launch_state<256>(mk_st, mv_st, mw_st, sp, s); break;
     }
   }
   if (e != cudaSuccess || L.Ttot == 0 || !(phases & 2)) return e;
