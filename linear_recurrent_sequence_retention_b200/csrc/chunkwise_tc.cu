@@ -41,6 +41,8 @@
 // returns.
 #include <cudaTypedefs.h>
 
+#include <cstring>
+
 #include "launch.h"
 #include "tc_ptx.cuh"
 
@@ -425,6 +427,8 @@ struct OutParams {
   const float* gn_b;
   float eps;
   int gated;
+  int g_tma;                   // gate tile streamed by TMA (bf16 gate)
+  int y_tma;                   // full output tiles written by TMA (bf16 output)
   int H, dk, dv;
   int rb;                      // 128-row blocks per chunk
   int parts;                   // d_v parts (cluster size)
@@ -452,6 +456,7 @@ template <int DK, int NV>
 __global__ void __launch_bounds__(kThreads, 1)
 output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
+              const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmY,
               const OutParams p) {
   using C = OutCfg<DK, NV>;
   constexpr int NST = C::kStages;
@@ -488,6 +493,15 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int nrows = min(kRowsPerTile, si.len - r * kRowsPerTile);
   const bool need_inter = si.c > 0 || p.has_state_in;
   const Decay1 dec(p.dec, h);
+  // stages used by the MMA operands; the gate/output tile (NV/64 boxes of
+  // 128 rows x 64 columns, two per stage) follows them in ring order
+  const int n_mma_units = (need_inter ? 2 * (DK / 64) : 0) + (r + 1) * (DK / 128 + 2);
+  constexpr int kIoBoxes = NV / 64;
+  constexpr int kIoUnits = (kIoBoxes + 1) / 2;
+  auto io_box = [&](int bx) -> uint8_t* {
+    const int unit = n_mma_units + bx / 2;
+    return smem + C::kOffStages + (unit % NST) * kOutStage + (bx & 1) * kTallBox;
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NST; ++i) {
@@ -576,6 +590,18 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       for (int kb = 0; kb <= r && ok; ++kb) {
         if (kb + 1 <= r) load_k(kb + 1);
         load_v(kb);
+      }
+      if (p.gated && p.g_tma) {      // the gate rows of this tile, for the epilogue
+        tma_prefetch_desc(&tmG);
+        for (int u = 0; u < kIoUnits && ok; ++u) {
+          const int nb = (kIoBoxes - 2 * u) >= 2 ? 2 : 1;
+          uint8_t* dst = next(nb * kTallBox);
+          if (!dst) { ok = false; break; }
+          for (int bb = 0; bb < nb; ++bb)
+            tma_load_2d(dst + bb * kTallBox, &tmG, &full[it % NST],
+                        h * p.dv + NV * part + 64 * (2 * u + bb), t0);
+          ++it;
+        }
       }
       if (!ok) {
         mbar_wait_drain(bar_q, 0);
@@ -813,8 +839,11 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     rstd = 1.0f / sqrtf(m2 / cnt + p.eps);
   }
   if (p.parts > 1 && p.gated) cluster_sync();      // partner has finished reading ours
-  if (warp >= 2 && ok_all) {
-    tc_fence_after();
+  // Full tiles with a bf16 output go through shared memory (in place of the
+  // gate tile, same swizzled layout) and TMA stores; partial tiles are
+  // written directly so that no row past the chunk is touched.
+  const bool out_tma = p.y_tma && nrows == kRowsPerTile;
+  if (warp >= 2) {
     const int wg = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
@@ -823,28 +852,35 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int col0 = NV * part + wg * kHalf;          // first d_v column of this warpgroup
     const size_t obase = (static_cast<size_t>(t0 + row) * p.H + h) * p.dv + col0;
     const float shift = -mean_all * rstd;
-    for (int j = 0; j < kHalf / 32; ++j) {
+    bool go = ok_all;
+    if (go && p.gated && p.g_tma) {
+      for (int u = 0; u < kIoUnits && go; ++u) {
+        const int unit = n_mma_units + u;
+        go = mbar_wait(&full[unit % NST], (unit / NST) & 1, abort_flag, p.err);
+      }
+    }
+    if (go) tc_fence_after();
+    for (int j = 0; j < kHalf / 32 && go; ++j) {
       float x[32];
       tmem_ld32(o_cols + 32 * j, x);
-      tmem_wait_ld();
-      if (!live) continue;
+      // this piece's 32 columns in the staged gate/output box: box, first 16-byte piece
+      const int cpart = wg * kHalf + 32 * j;
+      uint8_t* brow = io_box(cpart >> 6) + row * 128;
+      const int pc0 = (cpart & 63) >> 3;
       if (p.gated) {
         float gv[32];
-        if (p.g_bf16) {
-          const uint4* gp = reinterpret_cast<const uint4*>(
-              static_cast<const __nv_bfloat16*>(p.g) + obase + 32 * j);
+        if (p.g_tma) {
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
-            const uint4 u = gp[c4];
+            const uint4 u = *reinterpret_cast<const uint4*>(brow + (((pc0 + c4) ^ (row & 7)) << 4));
             const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
             for (int q2 = 0; q2 < 4; ++q2) {
-              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[q2]));
-              gv[8 * c4 + 2 * q2] = f.x;
-              gv[8 * c4 + 2 * q2 + 1] = f.y;
+              gv[8 * c4 + 2 * q2] = bf16_lo(wv[q2]);
+              gv[8 * c4 + 2 * q2 + 1] = bf16_hi(wv[q2]);
             }
           }
-        } else {
+        } else if (live) {
           const float4* gp = reinterpret_cast<const float4*>(static_cast<const float*>(p.g) + obase + 32 * j);
 #pragma unroll
           for (int c4 = 0; c4 < 8; ++c4) {
@@ -852,6 +888,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             gv[4 * c4] = f.x; gv[4 * c4 + 1] = f.y; gv[4 * c4 + 2] = f.z; gv[4 * c4 + 3] = f.w;
           }
         }
+        tmem_wait_ld();
         const uint64_t rs2 = f2_make(rstd, rstd), sh2 = f2_make(shift, shift);
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
@@ -880,8 +917,18 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           x[e] = f2_lo(o2);
           x[e + 1] = f2_hi(o2);
         }
+      } else {
+        tmem_wait_ld();
       }
-      if (p.out_bf16) {
+      if (out_tma) {
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+          *reinterpret_cast<uint4*>(brow + (((pc0 + c4) ^ (row & 7)) << 4)) =
+              make_uint4(pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]), pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]),
+                         pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]), pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]));
+      } else if (!live) {
+        continue;
+      } else if (p.out_bf16) {
         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + obase + 32 * j);
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4)
@@ -892,6 +939,17 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4)
           dst[c4] = make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
+      }
+    }
+    if (out_tma) {                    // uniform: every epilogue thread reaches the barrier
+      fence_proxy_async_smem();
+      wg2_sync();
+      if (threadIdx.x == 64 && go) {
+        tma_prefetch_desc(&tmY);
+        for (int bx = 0; bx < kIoBoxes; ++bx)
+          tma_store_2d(&tmY, io_box(bx), h * p.dv + NV * part + 64 * bx, t0);
+        tma_store_commit();
+        tma_store_wait_all();
       }
     }
   }
@@ -952,8 +1010,8 @@ cudaError_t launch_state(const CUtensorMap& mk, const CUtensorMap& mv, const CUt
 
 template <int DK, int NV>
 cudaError_t launch_out(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const CUtensorMap& ms, const OutParams& op, long long units,
-                       cudaStream_t s) {
+                       const CUtensorMap& ms, const CUtensorMap& mg, const CUtensorMap& my,
+                       const OutParams& op, long long units, cudaStream_t s) {
   using C = OutCfg<DK, NV>;
   static_assert(C::kSmem <= 232448, "shared memory budget");
   auto kern = output_kernel<DK, NV>;
@@ -972,7 +1030,7 @@ cudaError_t launch_out(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ms, op);
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ms, mg, my, op);
 }
 
 }  // namespace
@@ -1043,25 +1101,34 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
   op.parts = dv / NV;
   op.dec = dec;
   op.err = err;
+  op.g_tma = (gated && g_t == DType::BF16) ? 1 : 0;
+  op.y_tma = out_t == DType::BF16 ? 1 : 0;
   const uint64_t srows = static_cast<uint64_t>(ws.nslots) * H * 2 * dk;   // hi and lo planes
-  CUtensorMap mq, mk, mv, ms;
+  const uint64_t hdv = static_cast<uint64_t>(H) * dv;
+  CUtensorMap mq, mk, mv, ms, mg, my;
   if (!make_map(&mq, q, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 128) ||
       !make_map(&mk, k, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 128) ||
-      !make_map(&mv, v, static_cast<uint64_t>(H) * dv, Ttot, static_cast<uint64_t>(H) * dv, 64) ||
+      !make_map(&mv, v, hdv, Ttot, hdv, 64) ||
       !make_map(&ms, ws.states, dv, srows, dv, 64))
+    return cudaErrorInvalidValue;
+  // gate and output tiles: [Ttot rows][H*dv] bf16 (maps only built when used)
+  std::memset(&mg, 0, sizeof(mg));
+  std::memset(&my, 0, sizeof(my));
+  if ((op.g_tma && !make_map(&mg, g, hdv, Ttot, hdv, 128)) ||
+      (op.y_tma && !make_map(&my, out, hdv, Ttot, hdv, 128)))
     return cudaErrorInvalidValue;
   const long long units = ws.nslots * op.rb;
   if (dk == 128) {
     switch (NV) {
-      case 64: return launch_out<128, 64>(mq, mk, mv, ms, op, units, s);
-      case 128: return launch_out<128, 128>(mq, mk, mv, ms, op, units, s);
-      default: return launch_out<128, 256>(mq, mk, mv, ms, op, units, s);
+      case 64: return launch_out<128, 64>(mq, mk, mv, ms, mg, my, op, units, s);
+      case 128: return launch_out<128, 128>(mq, mk, mv, ms, mg, my, op, units, s);
+      default: return launch_out<128, 256>(mq, mk, mv, ms, mg, my, op, units, s);
     }
   }
   switch (NV) {
-    case 64: return launch_out<256, 64>(mq, mk, mv, ms, op, units, s);
-    case 128: return launch_out<256, 128>(mq, mk, mv, ms, op, units, s);
-    default: return launch_out<256, 256>(mq, mk, mv, ms, op, units, s);
+    case 64: return launch_out<256, 64>(mq, mk, mv, ms, mg, my, op, units, s);
+    case 128: return launch_out<256, 128>(mq, mk, mv, ms, mg, my, op, units, s);
+    default: return launch_out<256, 256>(mq, mk, mv, ms, mg, my, op, units, s);
   }
 }
 
