@@ -89,6 +89,12 @@ __device__ __forceinline__ bool slot_to_chunk(const SeqLayout& L, const int32_t*
 // Named barrier over the 256 threads of warps 2..9.
 __device__ __forceinline__ void wg2_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
+// Named barrier over the 128 threads of epilogue warpgroup wg (warps 2+4wg .. 5+4wg).
+__device__ __forceinline__ void wg_sync(int wg) {
+  if (wg == 0) asm volatile("bar.sync 2, 128;" ::: "memory");
+  else asm volatile("bar.sync 3, 128;" ::: "memory");
+}
+
 // AND of `v` over the 128 threads of warps 2..5 (named barrier 2); every one of
 // them gets the same answer, so loops that contain barrier 2 stay uniform.
 __device__ __forceinline__ bool wga_all(bool v) {
@@ -439,9 +445,10 @@ struct OutParams {
 template <int DK, int NV>
 struct OutCfg {
   static constexpr uint32_t kQBytes = (DK / 64) * kTallBox;
-  // barriers | gamma^d table | gamma^(127-d) table; the GroupNorm partials live
-  // in the Q region, which is free once every MMA has completed
-  static constexpr uint32_t kMiscBytes = 256 + 512 + 512;
+  // barriers | gamma^d table | gamma^(127-d) table | the partner CTA's
+  // GroupNorm (mean, M2) per row; this CTA's own partials live in the Q
+  // region, which is free once every MMA has completed
+  static constexpr uint32_t kMiscBytes = 256 + 512 + 512 + 1024;
   static constexpr int kStages = static_cast<int>((232448 - kQBytes - kMiscBytes) / kOutStage);
   static constexpr uint32_t kOffStages = kQBytes;
   static constexpr uint32_t kOffMisc = kOffStages + kStages * kOutStage;
@@ -471,12 +478,13 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   uint64_t* bar_p = bar_s + 2;           // [2] P written over the scores
   uint64_t* bar_o = bar_p + 2;           // all MMAs done
   uint64_t* drain = bar_o + 1;
-  uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* bar_x = drain + 1;           // the partner's statistics have arrived
+  uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(bar_x + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_hold + 1);
   float* pow_tab = reinterpret_cast<float*>(smem + C::kOffMisc + 256);    // gamma^d
   float* rev_tab = reinterpret_cast<float*>(smem + C::kOffMisc + 768);    // gamma^(127-d)
+  float* xrecv = reinterpret_cast<float*>(smem + C::kOffMisc + 1280);    // [128][2]
   float* wg_part = reinterpret_cast<float*>(smem);                        // [2][2][128], after bar_o
-  float* stats = reinterpret_cast<float*>(smem + 2048);                   // [128][2], after bar_o
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int part = blockIdx.x % p.parts;
@@ -492,6 +500,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int t0 = si.cs + r * kRowsPerTile;                  // first token of the row block
   const int nrows = min(kRowsPerTile, si.len - r * kRowsPerTile);
   const bool need_inter = si.c > 0 || p.has_state_in;
+  const bool xchg = p.parts > 1 && p.gated;           // GroupNorm spans both CTAs of the cluster
   const Decay1 dec(p.dec, h);
   // stages used by the MMA operands; the gate/output tile (NV/64 boxes of
   // 128 rows x 64 columns, two per stage) follows them in ring order
@@ -516,6 +525,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
     mbar_init(bar_o, 1);
     mbar_init(drain, 1);
+    mbar_init(bar_x, kWgThreads);
     *abort_flag = 0;
     if ((smem_u32(smem) & 1023u) != 0) {
       *abort_flag = 1;
@@ -531,6 +541,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_hold;
+  if (xchg) cluster_arrive_relaxed();    // barrier initialisation done (waited on before first use)
 
   // Unit sequence shared by producer and MMA issuer, one 32 KB stage each:
   //   [S_hi and S_lo of d_k rows 64u..64u+63, u < DK/64 (if the chunk reads a state)],
@@ -779,10 +790,12 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
     if (ok) ok = mbar_wait(bar_o, 0, abort_flag, p.err);
     if (ok) tc_fence_after();
-    // GroupNorm statistics of this part in one pass: sums of (x - x0) and
-    // (x - x0)^2 with x0 the row's first value in this warpgroup's half (a
-    // shift that keeps the sums well conditioned); the two halves combine as
-    // (mean, M2) pairs.  Barriers are unconditional.
+    // GroupNorm statistics in one pass: sums of (x - x0) and (x - x0)^2 with
+    // x0 the row's first value in this warpgroup's half (a shift that keeps
+    // the sums well conditioned); halves and parts combine as (mean, M2)
+    // pairs.  Barriers and the exchange with the partner CTA are
+    // unconditional, so an aborted CTA still meets its partner.
+    float mean_all = 0.f, rstd = 0.f;
     if (p.gated) {
       float mean_w = 0.f, m2_w = 0.f;
       if (ok) {
@@ -808,51 +821,49 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       wg_part[wg * 128 + row] = mean_w;
       wg_part[256 + wg * 128 + row] = m2_w;
       wg2_sync();
-      if (wg == 0) {
-        const float m0 = wg_part[row], m1 = wg_part[128 + row];
-        const float d = m1 - m0;
-        stats[2 * row] = 0.5f * (m0 + m1);
-        stats[2 * row + 1] = wg_part[256 + row] + wg_part[384 + row] + d * d * (0.5f * kHalf);
+      const float m0 = wg_part[row], m1 = wg_part[128 + row];
+      const float dd = m1 - m0;
+      float mean = 0.5f * (m0 + m1);
+      float m2 = wg_part[256 + row] + wg_part[384 + row] + dd * dd * (0.5f * kHalf);
+      float cnt = static_cast<float>(NV);
+      if (xchg) {
+        // the other d_v part: warpgroup 0 writes this part's (mean, M2) into
+        // the partner's receive buffer and arrives on its barrier
+        cluster_wait();                              // partner's barriers are initialised
+        if (wg == 0) {
+          const uint32_t other = cluster_ctarank() ^ 1u;
+          st_cluster_f32(cluster_addr(&xrecv[2 * row], other), mean);
+          st_cluster_f32(cluster_addr(&xrecv[2 * row + 1], other), m2);
+          mbar_arrive_cluster(cluster_addr(bar_x, other));
+        }
+        cluster_arrive();                            // this CTA's remote accesses are done
+        if (mbar_wait_cluster(bar_x, 0, abort_flag, p.err)) {
+          const float mo = xrecv[2 * row], m2o = xrecv[2 * row + 1];
+          const float d = mo - mean;
+          m2 = m2 + m2o + d * d * (cnt * 0.5f);
+          mean = 0.5f * (mean + mo);
+          cnt *= 2.f;
+        } else {
+          ok = false;
+        }
       }
+      mean_all = mean;
+      rstd = 1.0f / sqrtf(m2 / cnt + p.eps);
     }
-  }
-  // ---------------- join: GroupNorm statistics across the d_v parts ----------------
-  tc_fence_before();
-  __syncthreads();
-  const bool ok_all = !*abort_flag;
-  if (p.parts > 1 && p.gated) cluster_sync();      // partner's stats are written
-  float mean_all = 0.f, rstd = 0.f;
-  if (warp >= 2 && ok_all && p.gated) {
-    const int row = (warp & 3) * 32 + lane;
-    float mean = stats[2 * row], m2 = stats[2 * row + 1];
-    float cnt = static_cast<float>(NV);
-    if (p.parts > 1) {
-      const uint32_t other = cluster_ctarank() ^ 1u;
-      const float mo = ld_cluster_f32(&stats[2 * row], other);
-      const float m2o = ld_cluster_f32(&stats[2 * row + 1], other);
-      const float d = mo - mean;
-      m2 = m2 + m2o + d * d * (cnt * 0.5f);
-      mean = 0.5f * (mean + mo);
-      cnt *= 2.f;
-    }
-    mean_all = mean;
-    rstd = 1.0f / sqrtf(m2 / cnt + p.eps);
-  }
-  if (p.parts > 1 && p.gated) cluster_sync();      // partner has finished reading ours
-  // Full tiles with a bf16 output go through shared memory (in place of the
-  // gate tile, same swizzled layout) and TMA stores; partial tiles are
-  // written directly so that no row past the chunk is touched.
-  const bool out_tma = p.y_tma && nrows == kRowsPerTile;
-  if (warp >= 2) {
-    const int wg = (warp - 2) >> 2;
-    const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    const uint32_t o_cols = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::kTmemO + wg * kHalf;
+
+    // ---------------- GroupNorm, gate, store ----------------
+    // Full tiles with a bf16 output go through shared memory (in place of the
+    // gate tile, same swizzled layout) and TMA stores, one per 64-column box
+    // as soon as its warpgroup has written it; partial tiles are written
+    // directly so that no row past the chunk is touched.
+    const bool out_tma = p.y_tma && nrows == kRowsPerTile;
+    constexpr bool kBoxPerWg = kHalf >= 64;          // each warpgroup owns whole boxes
+    const bool wg_leader = ((threadIdx.x - 64) & 127) == 0;   // first thread of the warpgroup
     const bool live = row < nrows;
     const int col0 = NV * part + wg * kHalf;          // first d_v column of this warpgroup
     const size_t obase = (static_cast<size_t>(t0 + row) * p.H + h) * p.dv + col0;
     const float shift = -mean_all * rstd;
-    bool go = ok_all;
+    bool go = ok && !*abort_flag;
     if (go && p.gated && p.g_tma) {
       for (int u = 0; u < kIoUnits && go; ++u) {
         const int unit = n_mma_units + u;
@@ -860,98 +871,117 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
     }
     if (go) tc_fence_after();
-    for (int j = 0; j < kHalf / 32 && go; ++j) {
-      float x[32];
-      tmem_ld32(o_cols + 32 * j, x);
+    if (out_tma && wg_leader) tma_prefetch_desc(&tmY);
+    for (int j = 0; j < kHalf / 32; ++j) {
       // this piece's 32 columns in the staged gate/output box: box, first 16-byte piece
       const int cpart = wg * kHalf + 32 * j;
       uint8_t* brow = io_box(cpart >> 6) + row * 128;
       const int pc0 = (cpart & 63) >> 3;
-      if (p.gated) {
-        float gv[32];
-        if (p.g_tma) {
+      if (go) {
+        float x[32];
+        tmem_ld32(o_cols + 32 * j, x);
+        if (p.gated) {
+          float gv[32];
+          if (p.g_tma) {
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const uint4 u = *reinterpret_cast<const uint4*>(brow + (((pc0 + c4) ^ (row & 7)) << 4));
-            const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const uint4 u = *reinterpret_cast<const uint4*>(brow + (((pc0 + c4) ^ (row & 7)) << 4));
+              const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2) {
-              gv[8 * c4 + 2 * q2] = bf16_lo(wv[q2]);
-              gv[8 * c4 + 2 * q2 + 1] = bf16_hi(wv[q2]);
+              for (int q2 = 0; q2 < 4; ++q2) {
+                gv[8 * c4 + 2 * q2] = bf16_lo(wv[q2]);
+                gv[8 * c4 + 2 * q2 + 1] = bf16_hi(wv[q2]);
+              }
+            }
+          } else if (live) {
+            const float4* gp = reinterpret_cast<const float4*>(static_cast<const float*>(p.g) + obase + 32 * j);
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4) {
+              const float4 f = gp[c4];
+              gv[4 * c4] = f.x; gv[4 * c4 + 1] = f.y; gv[4 * c4 + 2] = f.z; gv[4 * c4 + 3] = f.w;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) gv[e] = 0.f;
+          }
+          tmem_wait_ld();
+          const uint64_t rs2 = f2_make(rstd, rstd), sh2 = f2_make(shift, shift);
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const uint64_t y2 = f2_fma(f2_make(x[e], x[e + 1]), rs2, sh2);
+            x[e] = f2_lo(y2);
+            x[e + 1] = f2_hi(y2);
+          }
+          if (p.gn_w || p.gn_b) {
+            const int c0 = h * p.dv + col0 + 32 * j;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (p.gn_w) x[e] *= p.gn_w[c0 + e];
+              if (p.gn_b) x[e] += p.gn_b[c0 + e];
             }
           }
+          // swish(g) = g sigmoid(g) = u + u tanh(u) with u = g/2 (sigmoid(g) =
+          // (1 + tanh(g/2))/2): one special-function op per element
+          const uint64_t half2 = f2_make(0.5f, 0.5f);
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const uint64_t u2 = f2_mul(f2_make(gv[e], gv[e + 1]), half2);
+            const uint64_t s2 = f2_fma(u2, f2_make(tanh_fast(f2_lo(u2)), tanh_fast(f2_hi(u2))), u2);
+            const uint64_t o2 = f2_mul(f2_make(x[e], x[e + 1]), s2);
+            x[e] = f2_lo(o2);
+            x[e + 1] = f2_hi(o2);
+          }
+        } else {
+          tmem_wait_ld();
+        }
+        if (out_tma) {
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+            *reinterpret_cast<uint4*>(brow + (((pc0 + c4) ^ (row & 7)) << 4)) =
+                make_uint4(pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]), pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]),
+                           pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]), pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]));
+        } else if (live && p.out_bf16) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + obase + 32 * j);
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+            dst[c4] = make_uint4(pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]), pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]),
+                                 pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]), pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]));
         } else if (live) {
-          const float4* gp = reinterpret_cast<const float4*>(static_cast<const float*>(p.g) + obase + 32 * j);
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + 32 * j);
 #pragma unroll
-          for (int c4 = 0; c4 < 8; ++c4) {
-            const float4 f = gp[c4];
-            gv[4 * c4] = f.x; gv[4 * c4 + 1] = f.y; gv[4 * c4 + 2] = f.z; gv[4 * c4 + 3] = f.w;
-          }
+          for (int c4 = 0; c4 < 8; ++c4)
+            dst[c4] = make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
         }
-        tmem_wait_ld();
-        const uint64_t rs2 = f2_make(rstd, rstd), sh2 = f2_make(shift, shift);
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const uint64_t y2 = f2_fma(f2_make(x[e], x[e + 1]), rs2, sh2);
-          x[e] = f2_lo(y2);
-          x[e + 1] = f2_hi(y2);
-        }
-        if (p.gn_w || p.gn_b) {
-          const int c0 = h * p.dv + col0 + 32 * j;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (p.gn_w) x[e] *= p.gn_w[c0 + e];
-            if (p.gn_b) x[e] += p.gn_b[c0 + e];
-          }
-        }
-        // swish(g) = g / (1 + 2^(-g log2 e)); paired where the math allows
-        const uint64_t nl2e = f2_make(-1.4426950408889634f, -1.4426950408889634f);
-        const uint64_t one2 = f2_make(1.f, 1.f);
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const uint64_t g2 = f2_make(gv[e], gv[e + 1]);
-          const uint64_t t2 = f2_mul(g2, nl2e);
-          const uint64_t d2 = f2_add(f2_make(exp2f_fast(f2_lo(t2)), exp2f_fast(f2_hi(t2))), one2);
-          const uint64_t s2 = f2_mul(g2, f2_make(rcp_fast(f2_lo(d2)), rcp_fast(f2_hi(d2))));
-          const uint64_t o2 = f2_mul(f2_make(x[e], x[e + 1]), s2);
-          x[e] = f2_lo(o2);
-          x[e + 1] = f2_hi(o2);
-        }
-      } else {
-        tmem_wait_ld();
       }
-      if (out_tma) {
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
-          *reinterpret_cast<uint4*>(brow + (((pc0 + c4) ^ (row & 7)) << 4)) =
-              make_uint4(pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]), pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]),
-                         pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]), pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]));
-      } else if (!live) {
-        continue;
-      } else if (p.out_bf16) {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + obase + 32 * j);
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
-          dst[c4] = make_uint4(pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]), pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]),
-                               pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]), pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]));
-      } else {
-        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + 32 * j);
-#pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4)
-          dst[c4] = make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
+      if (kBoxPerWg && out_tma && (j & 1)) {       // uniform over the warpgroup
+        // box cpart/64 is complete: hand it to the TMA engine
+        fence_proxy_async_smem();
+        wg_sync(wg);
+        if (wg_leader && go) {
+          tma_store_2d(&tmY, io_box(cpart >> 6), h * p.dv + NV * part + 64 * (cpart >> 6), t0);
+          tma_store_commit();
+        }
       }
     }
-    if (out_tma) {                    // uniform: every epilogue thread reaches the barrier
+    if (!kBoxPerWg && out_tma) {                   // boxes shared by both warpgroups
       fence_proxy_async_smem();
       wg2_sync();
       if (threadIdx.x == 64 && go) {
-        tma_prefetch_desc(&tmY);
         for (int bx = 0; bx < kIoBoxes; ++bx)
           tma_store_2d(&tmY, io_box(bx), h * p.dv + NV * part + 64 * bx, t0);
         tma_store_commit();
-        tma_store_wait_all();
       }
     }
+    // shared memory may be released once the stores have read it; the
+    // global writes complete on their own
+    if (out_tma && go && (kBoxPerWg ? wg_leader : threadIdx.x == 64)) tma_store_wait_read();
+  }
+  if (xchg) {
+    if (warp < 2) {
+      cluster_wait();
+      cluster_arrive();
+    }
+    cluster_wait();        // the partner has written its statistics: no more remote access here
   }
   tc_fence_before();
   __syncthreads();
