@@ -86,6 +86,10 @@ __device__ __forceinline__ bool slot_to_chunk(const SeqLayout& L, const int32_t*
   return si.len > 0;
 }
 
+// AND of `v` over the 32 lanes of the warp (tcgen05.ld/st are warp-collective,
+// so every guard around them must be warp-uniform).
+__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v) != 0; }
+
 // Named barrier over the 256 threads of warps 2..9.
 __device__ __forceinline__ void wg2_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
@@ -347,7 +351,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     if (leader) tma_store_wait_all();
     // final state
     if (ok && nch > 0) {
-      if (mbar_wait(acc_full, (nch - 1) & 1, abort_flag, p.err)) {
+      if (warp_all(mbar_wait(acc_full, (nch - 1) & 1, abort_flag, p.err))) {
         tc_fence_after();
         if (p.state_out) {
           for (int j = 0; j < NS / 32; ++j) {
@@ -720,7 +724,8 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     bool ok = !*abort_flag;
     const uint32_t o_cols = tmem + lane_off + C::kTmemO + wg * kHalf;
     if (ok && need_inter) {
-      ok = mbar_wait(bar_inter, 0, abort_flag, p.err);
+      // tcgen05.ld/st are warp-collective: every guard around them is warp-uniform
+      ok = warp_all(mbar_wait(bar_inter, 0, abort_flag, p.err));
       if (ok) {
         tc_fence_after();
         const float sc = dec.pow(i + 1);
@@ -737,7 +742,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
     for (int kb = 0; kb <= r && ok; ++kb) {
       const int sb = kb & 1;
-      if (!mbar_wait(&bar_s[sb], (kb >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+      if (!warp_all(mbar_wait(&bar_s[sb], (kb >> 1) & 1, abort_flag, p.err))) { ok = false; break; }
       tc_fence_after();
       const bool diag = kb == r;
       // off-diagonal: gamma^(i-j) = gamma^(i - 128kb - 127) * gamma^(127 - j')
@@ -789,6 +794,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mbar_arrive(&bar_p[sb]);
     }
     if (ok) ok = mbar_wait(bar_o, 0, abort_flag, p.err);
+    ok = warp_all(ok);
     if (ok) tc_fence_after();
     // GroupNorm statistics in one pass: sums of (x - x0) and (x - x0)^2 with
     // x0 the row's first value in this warpgroup's half (a shift that keeps
@@ -863,12 +869,13 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int col0 = NV * part + wg * kHalf;          // first d_v column of this warpgroup
     const size_t obase = (static_cast<size_t>(t0 + row) * p.H + h) * p.dv + col0;
     const float shift = -mean_all * rstd;
-    bool go = ok && !*abort_flag;
+    bool go = warp_all(ok && !*abort_flag);
     if (go && p.gated && p.g_tma) {
       for (int u = 0; u < kIoUnits && go; ++u) {
         const int unit = n_mma_units + u;
         go = mbar_wait(&full[unit % NST], (unit / NST) & 1, abort_flag, p.err);
       }
+      go = warp_all(go);
     }
     if (go) tc_fence_after();
     if (out_tma && wg_leader) tma_prefetch_desc(&tmY);
