@@ -13,13 +13,16 @@
 //
 //  state_kernel   one CTA per (sequence, head, 128 rows of d_k, NS columns of
 //                 d_v).  The state block lives in TMEM (f32) for the whole
-//                 sequence.  Warpgroup A, before each chunk, stores the state
-//                 entering it in the chunk's workspace slot (as a hi/lo bf16
-//                 pair), scales TMEM by gamma^L and releases the MMA; warpgroup
-//                 B turns every staged K tile into zeta*K hi/lo tiles
-//                 (zeta_j = gamma^(L-1-j)) ahead of the MMA, which accumulates
-//                 S += (zeta K)_hi^T V + (zeta K)_lo^T V.  The final f32 state
-//                 goes to state_out.
+//                 sequence, in two accumulators used in turn: the MMA
+//                 accumulates a chunk's contribution dS = (zeta K)_hi^T V +
+//                 (zeta K)_lo^T V into one (zeta_j = gamma^(L-1-j); warpgroup
+//                 B turns every staged K tile into zeta*K hi/lo tiles ahead of
+//                 it) while the other holds the state entering the chunk;
+//                 warpgroup A then forms S = gamma^L S_prev + dS in place,
+//                 releases the older accumulator to the next chunk and stores
+//                 S in the next chunk's workspace slot (as a hi/lo bf16 pair)
+//                 while that chunk runs.  The final f32 state goes to
+//                 state_out.
 //
 //  output_kernel  one CTA per (chunk, 128-row block r of the chunk, head,
 //                 NV-wide part of d_v); the halves of d_v = 512 form a 2-CTA
@@ -158,8 +161,8 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
   uint64_t* full = bars;
   uint64_t* empty = full + NSTG;
   uint64_t* kready = empty + NSTG;
-  uint64_t* acc_ready = kready + NSTG;
-  uint64_t* acc_full = acc_ready + 1;
+  uint64_t* acc_free = kready + NSTG;    // warpgroup A has read the older accumulator
+  uint64_t* acc_full = acc_free + 1;     // the chunk's contribution is complete
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_hold + 1);
@@ -179,7 +182,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       mbar_init(&empty[i], 1);
       mbar_init(&kready[i], kWgThreads);
     }
-    mbar_init(acc_ready, kWgThreads);
+    mbar_init(acc_free, kWgThreads);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -190,7 +193,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_hold, NS);
+    tmem_alloc(tmem_hold, 2 * NS);       // two accumulators of NS columns
     tmem_relinquish();
   }
   tc_fence_before();
@@ -229,14 +232,17 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer: S += (zeta K)_hi^T V + (zeta K)_lo^T V ----------------
+    // ---------------- MMA issuer: dS_c = (zeta K)_hi^T V + (zeta K)_lo^T V ----------------
+    // into accumulator c & 1 (the other one holds the state entering the chunk)
     if (lane == 0 && !*abort_flag) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, NS, true, true);
       int it = 0;
       bool ok = true, issued = false;
       for (int c = 0; c < nch && ok; ++c) {
         const int Lc = min(L.chunk, b - (a + c * L.chunk));
-        if (!mbar_wait(acc_ready, c & 1, abort_flag, p.err)) { ok = false; break; }
+        const uint32_t acc = tmem + (c & 1) * NS;
+        // this accumulator last held S_(c-2), which warpgroup A has read by now
+        if (c > 0 && !mbar_wait(acc_free, (c - 1) & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         for (int sb = 0; sb * kStTok < Lc; ++sb, ++it) {
           const int st = it % NSTG;
@@ -248,8 +254,8 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
 #pragma unroll
           for (int ks = 0; ks < kStTok / 16; ++ks) {
             const uint64_t bd = sdesc_sw128(vb + ks * 2048, kBox, 1024);
-            mma_bf16(tmem, sdesc_sw128(khi + ks * 2048, kBox, 1024), bd, idesc, true);
-            mma_bf16(tmem, sdesc_sw128(klo + ks * 2048, kBox, 1024), bd, idesc, true);
+            mma_bf16(acc, sdesc_sw128(khi + ks * 2048, kBox, 1024), bd, idesc, (sb | ks) != 0);
+            mma_bf16(acc, sdesc_sw128(klo + ks * 2048, kBox, 1024), bd, idesc, true);
           }
           issued = true;
           mma_commit(&empty[st]);
@@ -262,7 +268,12 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       }
     }
   } else if (warp < 6) {
-    // ---------------- warpgroup A: the state block in TMEM ----------------
+    // ---------------- warpgroup A: the carried state ----------------
+    // S_(c-1) sits in accumulator (c+1) & 1 while the MMA accumulates the
+    // chunk's contribution dS_c into accumulator c & 1; then
+    //     S_c = gamma^L S_(c-1) + dS_c   (written over dS_c)
+    // releases the older accumulator for chunk c+1, and S_c (the state entering
+    // chunk c+1) goes to that chunk's workspace slot while chunk c+1 runs.
     const int quad = warp & 3;
     const int row = quad * 32 + lane;            // TMEM lane = row of the state block
     const int i = 128 * m + row;                 // d_k index
@@ -270,45 +281,23 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     const size_t st_off = ((static_cast<size_t>(s) * p.H + h) * p.dk + i) * p.dv + NS * part;
     const bool leader = threadIdx.x == 64;
     if (leader) tma_prefetch_desc(&tmW);
-    bool ok = wga_all(!*abort_flag);
-    for (int c = 0; c < nch && ok; ++c) {
-      const int Lc = min(L.chunk, b - (a + c * L.chunk));
-      const long long slot = L.cu == nullptr
-                                 ? static_cast<long long>(s) * ceil_div(L.T, L.chunk) + c
-                                 : static_cast<long long>(p.chunk_base[s]) + c;
+    auto slot_of = [&](int c) -> long long {
+      return L.cu == nullptr ? static_cast<long long>(s) * ceil_div(L.T, L.chunk) + c
+                             : static_cast<long long>(p.chunk_base[s]) + c;
+    };
+    // The state in accumulator column `col` -> workspace slot `slot` as a hi/lo
+    // bf16 pair, one 128 x 64 box of each plane per TMA store.  Barrier 2 is
+    // reached by all 128 threads the same number of times.
+    auto stage_state = [&](uint32_t col, long long slot) {
       const bool slot_ok = slot >= 0 && slot < L.nslots;
       // workspace rows of this CTA's 128 d_k rows in the hi plane; lo follows dk rows later
       const int wrow = static_cast<int>(((slot_ok ? slot : 0) * p.H + h) * 2 * p.dk) + 128 * m;
-      if (c > 0) {
-        ok = wga_all(mbar_wait(acc_full, (c - 1) & 1, abort_flag, p.err));
-        if (!ok) break;
-        tc_fence_after();
-      }
-      const float gL = dec.pow(Lc);
-      const uint64_t gL2 = f2_make(gL, gL);
 #pragma unroll 1
-      for (int j = 0; j < NS / 32; j += 2) {       // 64 columns per TMA store box
+      for (int j = 0; j < NS / 32; j += 2) {
         float r[2][32];
-        if (c == 0) {
-#pragma unroll
-          for (int hp = 0; hp < 2; ++hp) {
-            if (p.state_in) {
-              const float4* src = reinterpret_cast<const float4*>(p.state_in + st_off + 32 * (j + hp));
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float4 x = src[e];
-                r[hp][4 * e] = x.x; r[hp][4 * e + 1] = x.y; r[hp][4 * e + 2] = x.z; r[hp][4 * e + 3] = x.w;
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) r[hp][e] = 0.f;
-            }
-          }
-        } else {
-          tmem_ld32(trow + 32 * j, r[0]);
-          tmem_ld32(trow + 32 * (j + 1), r[1]);
-          tmem_wait_ld();
-        }
+        tmem_ld32(trow + col + 32 * j, r[0]);
+        tmem_ld32(trow + col + 32 * (j + 1), r[1]);
+        tmem_wait_ld();
         // the staging boxes are free once the previous store stopped reading them
         if (leader) tma_store_wait_read();
         asm volatile("bar.sync 2, 128;" ::: "memory");
@@ -333,36 +322,70 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
           tma_store_2d(&tmW, staging + kTallBox, NS * part + 32 * j, wrow + p.dk);
           tma_store_commit();
         }
+      }
+    };
+    bool ok = wga_all(!*abort_flag);
+    if (ok && nch > 0) {
+      // the state entering chunk 0 (state_in, or zero) into accumulator 1
+#pragma unroll 1
+      for (int j = 0; j < NS / 32; ++j) {
+        float r[32];
+        if (p.state_in) {
+          const float4* src = reinterpret_cast<const float4*>(p.state_in + st_off + 32 * j);
 #pragma unroll
-        for (int hp = 0; hp < 2; ++hp) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const uint64_t v2 = f2_mul(f2_make(r[hp][e], r[hp][e + 1]), gL2);
-            r[hp][e] = f2_lo(v2);
-            r[hp][e + 1] = f2_hi(v2);
+          for (int e = 0; e < 8; ++e) {
+            const float4 x = src[e];
+            r[4 * e] = x.x; r[4 * e + 1] = x.y; r[4 * e + 2] = x.z; r[4 * e + 3] = x.w;
           }
-          tmem_st32(trow + 32 * (j + hp), r[hp]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = 0.f;
         }
+        tmem_st32(trow + NS + 32 * j, r);
+      }
+      tmem_wait_st();
+      stage_state(NS, slot_of(0));
+    }
+    for (int c = 0; c < nch && ok; ++c) {
+      const int Lc = min(L.chunk, b - (a + c * L.chunk));
+      ok = wga_all(mbar_wait(acc_full, c & 1, abort_flag, p.err));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t dcol = (c & 1) * NS, pcol = ((c + 1) & 1) * NS;
+      const float gL = dec.pow(Lc);
+      const uint64_t gL2 = f2_make(gL, gL);
+#pragma unroll 1
+      for (int j = 0; j < NS / 32; ++j) {
+        float sp[32], sd[32];
+        tmem_ld32(trow + pcol + 32 * j, sp);
+        tmem_ld32(trow + dcol + 32 * j, sd);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const uint64_t v2 = f2_fma(f2_make(sp[e], sp[e + 1]), gL2, f2_make(sd[e], sd[e + 1]));
+          sd[e] = f2_lo(v2);
+          sd[e + 1] = f2_hi(v2);
+        }
+        tmem_st32(trow + dcol + 32 * j, sd);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(acc_ready);
+      mbar_arrive(acc_free);                     // accumulator pcol may take chunk c+1
+      if (c + 1 < nch) stage_state(dcol, slot_of(c + 1));
     }
     if (leader) tma_store_wait_all();
-    // final state
+    // final state: S_(nch-1), in accumulator (nch-1) & 1
     if (ok && nch > 0) {
-      if (warp_all(mbar_wait(acc_full, (nch - 1) & 1, abort_flag, p.err))) {
-        tc_fence_after();
-        if (p.state_out) {
-          for (int j = 0; j < NS / 32; ++j) {
-            float r[32];
-            tmem_ld32(trow + 32 * j, r);
-            tmem_wait_ld();
-            float4* dst = reinterpret_cast<float4*>(p.state_out + st_off + 32 * j);
+      if (p.state_out) {
+        const uint32_t fcol = ((nch - 1) & 1) * NS;
+        for (int j = 0; j < NS / 32; ++j) {
+          float r[32];
+          tmem_ld32(trow + fcol + 32 * j, r);
+          tmem_wait_ld();
+          float4* dst = reinterpret_cast<float4*>(p.state_out + st_off + 32 * j);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              dst[e] = make_float4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]);
-          }
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]);
         }
       }
     } else if (ok && p.state_out) {   // empty sequence: the state passes through
@@ -416,7 +439,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, NS);
+    tmem_dealloc(tmem, 2 * NS);
   }
 }
 
