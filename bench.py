@@ -188,11 +188,24 @@ def sum_over_ranks(x, world):
 # CPU baseline: the fp64 oracle, as it stands, on a bounded sample
 # ---------------------------------------------------------------------------
 
+def sample_len(wl, i):
+    """Token count of the i-th sampled (sequence, head) pair of a workload."""
+    if wl.varlen:
+        nseq, lo, hi = wl.varlen
+        return int(W.varlen_lengths(nseq, lo, hi, seed=0)[i % nseq])
+    return wl.T
+
+
+def n_pairs(wl):
+    return (wl.varlen[0] if wl.varlen else wl.B) * wl.H
+
+
 def oracle_sample_step(wl, seed, chunk):
     """One (sequence, head) of the workload through the oracle: the chunkwise
     form over all its tokens, then GroupNorm + gate when the workload has it."""
     import oracle
-    q, k, v, g = W.make_qkvg(1, wl.T, 1, wl.dk, wl.dv, "bf16", seed=seed, gate=wl.norm_gate)
+    q, k, v, g = W.make_qkvg(1, sample_len(wl, seed), 1, wl.dk, wl.dv, "bf16", seed=seed,
+                             gate=wl.norm_gate)
     f = W.to_f64
     gam = W.head_gammas(wl.H)[seed % wl.H]
     t0 = time.perf_counter()
@@ -214,17 +227,18 @@ def blas_threads():
 def cpu_baseline(wl, budget_s=15.0):
     """Oracle throughput in tokens/s (one token = all H heads), timed on a
     sample of whole (sequence, head) pairs for about ``budget_s`` seconds."""
-    done, elapsed = 0, 0.0
+    done, elapsed, token_heads = 0, 0.0, 0
     while elapsed < budget_s or done == 0:
         elapsed += oracle_sample_step(wl, done, wl.chunk)
+        token_heads += sample_len(wl, done)
         done += 1
-        if done >= wl.B * wl.H:
+        if done >= n_pairs(wl):
             break
-    token_heads = done * wl.T
+    what = "chunkwise form + GroupNorm/gate" if wl.norm_gate else "chunkwise form"
     return {"value": token_heads / wl.H / elapsed, "unit": "tokens/s",
             "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{done} of {wl.B * wl.H} (sequence, head) pairs of {wl.name}, "
-                      f"{wl.T} tokens each, chunkwise form + GroupNorm/gate in numpy float64; "
+            "sample": f"{done} of {n_pairs(wl)} (sequence, head) pairs of {wl.name}, "
+                      f"{token_heads} token-heads, {what} in numpy float64; "
                       f"tokens/s counts a token once all {wl.H} heads are done"}
 
 
@@ -248,27 +262,62 @@ def traffic_from_profile():
     return float(m2.group(1))
 
 
+def config_of(wl, world):
+    Bx, Tx, nst, cu = shape_of(wl)
+    in_mb = Bx * Tx * wl.H * (2 * wl.dk + wl.dv + (wl.dv if wl.norm_gate else 0)) * 2 / 1e6
+    cfg = {"workload": wl.name, "B_per_gpu": Bx, "T": Tx, "H": wl.H, "d_k": wl.dk, "d_v": wl.dv,
+           "chunk": wl.chunk,
+           "epilogue": ("per-head GroupNorm (eps 1e-5) + swish gate, y bf16" if wl.norm_gate
+                        else "none, o bf16"),
+           "state_out": "f32 final state" if wl.state_out else "none",
+           "parallelism": f"dp{world}",
+           "l2": (f"inputs ({in_mb:.0f} MB per step) larger than L2; no flush" if in_mb >= 264
+                  else f"inputs ({in_mb:.0f} MB per step) near or below L2 size: L2 flushed "
+                       "(256 MB write) between timed steps, outside the per-step events")}
+    if cu is not None:
+        cfg["packed"] = f"{nst} sequences, {Tx} tokens, cu_seqlens"
+    return cfg
+
+
+def shape_of(wl):
+    """(B, T, number of sequences, cu_seqlens or None) of a chunkwise workload; a
+    packed variable-length batch is one row of all its tokens."""
+    if wl.varlen:
+        nseq, lo, hi = wl.varlen
+        cu = W.cu_seqlens_of(W.varlen_lengths(nseq, lo, hi, seed=0))
+        return 1, int(cu[-1]), nseq, cu
+    return wl.B, wl.T, wl.B, None
+
+
 def run_headline(args, world, rank, pk, pk_kind):
     from linear_recurrent_sequence_retention_b200 import ops
     wl = W.WORKLOADS[HEADLINE]
     dev = torch.device("cuda")
-    q, k, v, g = W.make_qkvg(wl.B, wl.T, wl.H, wl.dk, wl.dv, "bf16", seed=rank, device=dev)
+    Bx, Tx, nst, cu = shape_of(wl)
+    q, k, v, g = W.make_qkvg(Bx, Tx, wl.H, wl.dk, wl.dv, "bf16", seed=rank, gate=wl.norm_gate,
+                             device=dev)
+    cu = None if cu is None else torch.from_numpy(cu).to(dev)
     gam = W.head_gammas(wl.H)
-    y = torch.empty(wl.B, wl.T, wl.H, wl.dv, device=dev, dtype=torch.bfloat16)
-    S = torch.empty(wl.B, wl.H, wl.dk, wl.dv, device=dev, dtype=torch.float32)
-    ws = ops.alloc_workspace(ops.chunkwise_workspace_size(torch.bfloat16, wl.chunk, wl.B, wl.T,
-                                                          wl.H, wl.dk, wl.dv), dev)
+    y = torch.empty(Bx, Tx, wl.H, wl.dv, device=dev, dtype=torch.bfloat16)
+    S = torch.empty(nst, wl.H, wl.dk, wl.dv, device=dev, dtype=torch.float32) if wl.state_out else None
+    ws = ops.alloc_workspace(ops.chunkwise_workspace_size(torch.bfloat16, wl.chunk, Bx, Tx, wl.H,
+                                                          wl.dk, wl.dv, nst if cu is not None else 0),
+                             dev)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record()
-        ops.chunkwise_states(k, v, gam, wl.chunk, state_out=S, workspace=ws)
+        ops.chunkwise_states(k, v, gam, wl.chunk, cu_seqlens=cu, state_out=S, workspace=ws)
         if ev is not None:
             ev[1].record()
-        ops.chunkwise_outputs(q, k, v, gam, wl.chunk, ws, g=g, out=y)
+        ops.chunkwise_outputs(q, k, v, gam, wl.chunk, ws, cu_seqlens=cu, g=g, out=y)
         if ev is not None:
             ev[2].record()
 
+    # inputs that fit in L2 are flushed between timed steps (a 256 MB write,
+    # outside the per-step events), so every step reads them from HBM
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, g) if t is not None)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if in_bytes < (252 << 20) else None
     for _ in range(args.warmup):
         step()
     ops.check_device_error()
@@ -282,6 +331,8 @@ def run_headline(args, world, rank, pk, pk_kind):
     torch.cuda.synchronize()
     start.record()
     for i in range(K):
+        if flush is not None:
+            flush.fill_(i & 0xff)
         step(evs[i])
     end.record()
     torch.cuda.synchronize()
@@ -291,14 +342,16 @@ def run_headline(args, world, rank, pk, pk_kind):
     ms_total = start.elapsed_time(end)
     ms_state = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     ms_out = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    if flush is not None:     # the step time is the sum of the two kernels' events
+        ms_total = float(np.sum([e[0].elapsed_time(e[2]) for e in evs]))
     ms_step = max_over_ranks(ms_total / K, world)
-    tokens = sum_over_ranks(wl.B * wl.T, world)
+    tokens = sum_over_ranks(Bx * Tx, world)
     value = tokens / (ms_step / 1e3)
 
     # roofline of the dominant (output) kernel, algorithmic counts
     chunk_exec = max(wl.chunk, 128)
     f_out, f_state, b_in, b_out = alg_counts(wl, chunk_exec)
-    units = wl.B * wl.T * wl.H                      # token-heads per launch
+    units = Bx * Tx * wl.H                          # token-heads per launch
     flops_launch = f_out * units
     bytes_launch = (b_in + b_out) * units
     t_out = ms_out / 1e3
@@ -325,7 +378,7 @@ def run_headline(args, world, rank, pk, pk_kind):
               "frac_of_spec": step_flops / (ms_step / 1e3) / 1e12 / 2250.0,
               "algorithmic_flops_per_step": step_flops,
               "counting": f"per token-head (C+1)(dk+dv) + 4 dk dv, C={chunk_exec}"}
-    step_bytes = (b_in + b_out) * units + wl.B * wl.H * wl.dk * wl.dv * 4
+    step_bytes = (b_in + b_out) * units + (nst * wl.H * wl.dk * wl.dv * 4 if wl.state_out else 0)
     hbm = {"achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9, "peak_gbs": peak_bw,
            "frac": step_bytes / (ms_step / 1e3) / 1e9 / peak_bw,
            "algorithmic_bytes_per_step": step_bytes}
@@ -334,18 +387,21 @@ def run_headline(args, world, rank, pk, pk_kind):
     # end to end through the public API with pinned host buffers
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv, hg = (t.to("cpu").pin_memory() for t in (q, k, v, g))
+        ins = [t for t in (q, k, v, g) if t is not None]
+        hins = [t.to("cpu").pin_memory() for t in ins]
+        dins = [torch.empty_like(t) for t in ins]
         hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-        hS = torch.empty(S.shape, dtype=S.dtype).pin_memory()
-        dq, dk_, dv_, dg = (torch.empty_like(t) for t in (q, k, v, g))
+        hS = None if S is None else torch.empty(S.shape, dtype=S.dtype).pin_memory()
 
         def e2e_step():
-            for d, hsrc in ((dq, hq), (dk_, hk), (dv_, hv), (dg, hg)):
+            for d, hsrc in zip(dins, hins):
                 d.copy_(hsrc, non_blocking=True)
-            ops.chunkwise_fwd(dq, dk_, dv_, gam, wl.chunk, g=dg, out=y, state_out=S,
-                              workspace=ws)
+            dg = dins[3] if g is not None else None
+            ops.chunkwise_fwd(dins[0], dins[1], dins[2], gam, wl.chunk, cu_seqlens=cu, g=dg, out=y,
+                              state_out=S, workspace=ws)
             hy.copy_(y, non_blocking=True)
-            hS.copy_(S, non_blocking=True)
+            if hS is not None:
+                hS.copy_(S, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
@@ -360,17 +416,17 @@ def run_headline(args, world, rank, pk, pk_kind):
         torch.cuda.synchronize()
         barrier(world)
         ms_e2e = max_over_ranks(e0.elapsed_time(e1) / Ke, world)
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg))
-        d2h = hy.numel() * hy.element_size() + hS.numel() * hS.element_size()
+        h2d = sum(t.numel() * t.element_size() for t in hins)
+        d2h = hy.numel() * hy.element_size() + (0 if hS is None else hS.numel() * hS.element_size())
         e2e = {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "ms_per_step": ms_e2e,
                "steps": Ke, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "api": "ops.chunkwise_fwd (C ABI retention_chunkwise_fwd) from pinned host memory"}
-        del hq, hk, hv, hg, dq, dk_, dv_, dg
+        del hins, dins
     del q, k, v, g, y, ws
     torch.cuda.empty_cache()
     return {"value": value, "ms_per_step": ms_step, "roofline": roof, "tensor": tensor,
             "hbm": hbm, "kernels": kernels, "e2e": e2e, "clocks": clocks,
-            "gpu_launches": 2 * K, "wl": wl}
+            "gpu_launches": (3 if cu is not None else 2) * K, "wl": wl}
 
 
 def run_decode(args, world, rank, pk, pk_kind):
@@ -432,6 +488,7 @@ def run_decode(args, world, rank, pk, pk_kind):
 
 
 def main():
+    global HEADLINE
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
@@ -441,6 +498,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--workload", default=HEADLINE,
+                    choices=[n for n, w in W.WORKLOADS.items() if w.dtype == "bf16" and not w.decode_steps],
+                    help="chunkwise workload to time (default: the 6.7B-shaped headline)")
     ap.add_argument("--B", type=int, default=None, help="override the headline batch (profiling)")
     ap.add_argument("--T", type=int, default=None, help="override the headline length (profiling)")
     ap.add_argument("--no-headline", action="store_true", help="decode only (profiling)")
@@ -458,6 +518,7 @@ def main():
         N, st = args.decode_N or base.B, args.decode_steps or base.decode_steps
         W.WORKLOADS[DECODE] = dataclasses.replace(base, B=N, decode_steps=st,
                                                   name=f"{base.name}@N{N}_steps{st}")
+    HEADLINE = args.workload
     if args.B or args.T:
         import dataclasses
         base = W.WORKLOADS[HEADLINE]
@@ -473,7 +534,8 @@ def main():
                 oracle_sample_step(wl, i, wl.chunk)
             times = [oracle_sample_step(wl, i, wl.chunk) for i in range(args.steps)]
             ms = 1e3 * float(np.sum(times)) / args.steps
-            val = wl.T / wl.H / (ms / 1e3)
+            toks = float(np.mean([sample_len(wl, i) for i in range(args.steps)]))
+            val = toks / wl.H / (ms / 1e3)
             line = {"metric": METRIC, "value": val, "unit": "tokens/s", "impl": "reference",
                     "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                     "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -483,8 +545,9 @@ def main():
                                "step": "one (sequence, head) pair of the workload"},
                     "cpu_baseline": {"value": val, "unit": "tokens/s", "kind": "oracle",
                                      "cores": blas_threads(),
-                                     "sample": f"each step: one of the {wl.B * wl.H} (sequence, "
-                                               f"head) pairs, {wl.T} tokens, numpy float64"},
+                                     "sample": f"each step: one of the {n_pairs(wl)} (sequence, "
+                                               f"head) pairs ({toks:.0f} tokens on average), "
+                                               "numpy float64"},
                     "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                             "d2h_bytes_per_step": 0}}
             print(json.dumps(line), flush=True)
@@ -519,12 +582,7 @@ def main():
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": wl.name, "B_per_gpu": wl.B, "T": wl.T, "H": wl.H,
-                       "d_k": wl.dk, "d_v": wl.dv, "chunk": wl.chunk,
-                       "epilogue": "per-head GroupNorm (eps 1e-5) + swish gate, y bf16",
-                       "state_out": "f32 final state", "parallelism": f"dp{world}",
-                       "l2": f"inputs ({wl.B * wl.T * wl.H * (2 * wl.dk + 2 * wl.dv) * 2 / 1e6:.0f} MB "
-                             "per step) larger than L2; no flush"},
+            "config": config_of(wl, world),
             "roofline": head["roofline"],
             "tensor": head["tensor"],
             "hbm": head["hbm"],

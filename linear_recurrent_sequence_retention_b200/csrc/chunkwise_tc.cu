@@ -1024,6 +1024,21 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 // ===========================================================================
 // Host side
 // ===========================================================================
+// Streaming multiprocessors of the current device (queried once per device).
+int sm_count() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = 148;
+  }
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static bool tried = false;
@@ -1115,7 +1130,13 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
   cudaError_t e = cudaSuccess;
   if (phases & 1) {
     // ---- state pass ----
-    const int NS = dv >= 256 ? 256 : dv;
+    // d_v columns per CTA: the widest of 256/128/64 whose grid still covers
+    // most of the SMs (every CTA walks its sequence serially, so a small
+    // batch needs narrower blocks to fill the machine)
+    int NS = dv >= 256 ? 256 : dv;
+    const long long blocks = static_cast<long long>(L.nseq) * H * (dk / 128);
+    const int sms = sm_count();
+    while (NS > 64 && blocks * (dv / NS) * 5 < static_cast<long long>(sms) * 3) NS /= 2;
     StateParams sp;
     sp.L = L;
     sp.chunk_base = ws.chunk_base;
