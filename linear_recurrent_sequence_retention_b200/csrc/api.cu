@@ -203,6 +203,7 @@ ret_status prepare_chunk_call(int phases, const void* q, const void* k, const vo
       workspace_bytes < c->p.bytes)
     return RET_ERR_WORKSPACE;
   c->ws.chunk_base = static_cast<int32_t*>(const_cast<void*>(workspace));
+  c->ws.order = c->ws.chunk_base + c->p.L.nseq + 1;
   c->ws.states = static_cast<char*>(const_cast<void*>(workspace)) + c->p.meta;
   c->ws.nslots = c->p.slots;
   c->err = error_word();

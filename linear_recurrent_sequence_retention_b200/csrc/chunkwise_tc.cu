@@ -125,6 +125,7 @@ constexpr int kStTok = 64;           // tokens per pipeline stage
 struct StateParams {
   SeqLayout L;
   const int32_t* chunk_base;
+  const int32_t* order;              // varlen: sequences longest first (else nullptr)
   const float* state_in;
   float* state_out;
   __nv_bfloat16* ws;                 // [nslots][H][2 (hi, lo)][dk][dv] bf16
@@ -168,8 +169,14 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_hold + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int s = blockIdx.x, h = blockIdx.y;
-  const int m = blockIdx.z % (p.dk / 128), part = blockIdx.z / (p.dk / 128);
+  // 1-D grid, sequence-major: all (head, d_k block, d_v part) CTAs of a
+  // sequence are adjacent, and packed sequences go longest first
+  const int zn = (p.dk / 128) * (p.dv / NS);
+  const int rank = static_cast<int>(blockIdx.x / (p.H * zn));
+  const int rem = static_cast<int>(blockIdx.x % (p.H * zn));
+  const int h = rem / zn, zz = rem % zn;
+  const int s = p.order ? p.order[rank] : rank;
+  const int m = zz % (p.dk / 128), part = zz / (p.dk / 128);
   const SeqLayout& L = p.L;
   int a, b;
   seq_bounds(L, s, a, b);
@@ -1078,7 +1085,7 @@ cudaError_t launch_state(const CUtensorMap& mk, const CUtensorMap& mv, const CUt
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid(sp.L.nseq, sp.H, (sp.dk / 128) * (sp.dv / NS));
+  dim3 grid(static_cast<unsigned>(sp.L.nseq) * sp.H * (sp.dk / 128) * (sp.dv / NS));
   kern<<<grid, kThreads, smem, s>>>(mk, mv, mw, sp);
   return cudaGetLastError();
 }
@@ -1140,6 +1147,7 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
     StateParams sp;
     sp.L = L;
     sp.chunk_base = ws.chunk_base;
+    sp.order = L.cu ? ws.order : nullptr;
     sp.state_in = state_in;
     sp.state_out = state_out;
     sp.ws = static_cast<__nv_bfloat16*>(ws.states);

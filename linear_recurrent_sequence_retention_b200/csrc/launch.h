@@ -19,6 +19,7 @@ enum class DType { F32 = 0, BF16 = 1 };
 //   operand of the cross-chunk read) on the tensor-core path.
 struct ChunkWorkspace {
   int32_t* chunk_base;   // device, nseq+1 entries (varlen only; else unused)
+  int32_t* order;        // device, nseq entries: sequences longest first (varlen only)
   void* states;          // device
   long long nslots;      // slots available
 };

@@ -87,10 +87,18 @@ parallel_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
 // Chunk bookkeeping for packed sequences: chunk_base[s] = number of chunks of
 // all sequences before s.  One block; also checks cu_seqlens.
 // ---------------------------------------------------------------------------
-__global__ void chunk_prep_kernel(SeqLayout L, int32_t* chunk_base, unsigned* err) {
+//
+// order[0..nseq) lists the sequences by chunk count, longest first (ties in any
+// order; counts of kOrderBins-1 chunks or more share the top bin), so that a
+// grid walking sequences in that order starts the longest serial chains first.
+constexpr int kOrderBins = 2048;
+
+__global__ void chunk_prep_kernel(SeqLayout L, int32_t* chunk_base, int32_t* order, unsigned* err) {
   __shared__ int carry;
   __shared__ int bad;
+  __shared__ int bins[kOrderBins];
   if (threadIdx.x == 0) { carry = 0; bad = 0; }
+  for (int i = threadIdx.x; i < kOrderBins; i += blockDim.x) bins[i] = 0;
   __syncthreads();
   if (threadIdx.x == 0) {
     if (L.cu[0] != 0 || L.cu[L.nseq] != L.Ttot) bad = 1;
@@ -115,7 +123,10 @@ __global__ void chunk_prep_kernel(SeqLayout L, int32_t* chunk_base, unsigned* er
       sc[threadIdx.x] += x;
       __syncthreads();
     }
-    if (s < L.nseq) chunk_base[s] = carry + sc[threadIdx.x] - n;
+    if (s < L.nseq) {
+      chunk_base[s] = carry + sc[threadIdx.x] - n;
+      atomicAdd(&bins[min(n, kOrderBins - 1)], 1);
+    }
     __syncthreads();
     if (threadIdx.x == blockDim.x - 1) carry += sc[threadIdx.x];
     __syncthreads();
@@ -123,6 +134,32 @@ __global__ void chunk_prep_kernel(SeqLayout L, int32_t* chunk_base, unsigned* er
   if (threadIdx.x == 0) {
     chunk_base[L.nseq] = carry;
     if (bad) raise_error(err, kErrDeviceData);
+  }
+  // bins -> first position of each chunk count in the longest-first order:
+  // exclusive scan from the top bin down (two bins per thread)
+  __shared__ int pos[kOrderBins];
+  {
+    const int hi = kOrderBins - 1 - 2 * threadIdx.x;      // this thread's bins: hi, hi-1
+    const int c0 = hi >= 0 ? bins[hi] : 0, c1 = hi >= 1 ? bins[hi - 1] : 0;
+    __shared__ int ps[1024];
+    ps[threadIdx.x] = c0 + c1;
+    __syncthreads();
+    for (int off = 1; off < blockDim.x; off <<= 1) {
+      int x = threadIdx.x >= off ? ps[threadIdx.x - off] : 0;
+      __syncthreads();
+      ps[threadIdx.x] += x;
+      __syncthreads();
+    }
+    const int before = ps[threadIdx.x] - (c0 + c1);          // sequences in higher bins
+    if (hi >= 0) pos[hi] = before;
+    if (hi >= 1) pos[hi - 1] = before + c0;
+  }
+  __syncthreads();
+  for (int s = threadIdx.x; s < L.nseq; s += blockDim.x) {
+    int a, b;
+    seq_bounds(L, s, a, b);
+    const int n = ceil_div(b - a, L.chunk);
+    order[atomicAdd(&pos[min(n, kOrderBins - 1)], 1)] = s;
   }
 }
 
@@ -425,7 +462,8 @@ cudaError_t chunkwise_typed(int phases, const void* q, const void* k, const void
 }  // namespace
 
 size_t chunkwise_meta_bytes(int nseq) {
-  size_t b = sizeof(int32_t) * (static_cast<size_t>(nseq) + 1);
+  // chunk_base [nseq+1] | longest-first sequence order [nseq]
+  size_t b = sizeof(int32_t) * (2 * static_cast<size_t>(nseq) + 1);
   return (b + 255) / 256 * 256;
 }
 
@@ -443,7 +481,7 @@ cudaError_t launch_parallel_simt(const void* q, const void* k, const void* v, DT
 cudaError_t launch_chunk_prep(const SeqLayout& L, ChunkWorkspace ws, unsigned* err,
                               cudaStream_t s) {
   if (L.cu == nullptr) return cudaSuccess;
-  chunk_prep_kernel<<<1, 1024, 0, s>>>(L, ws.chunk_base, err);
+  chunk_prep_kernel<<<1, 1024, 0, s>>>(L, ws.chunk_base, ws.order, err);
   return cudaGetLastError();
 }
 
