@@ -165,8 +165,9 @@ RET_API size_t retention_chunkwise_workspace_size(ret_dtype in_dtype, int chunk,
  * Supported:
  *   in_dtype RET_F32: dk, dv in 1..256, any chunk >= 1 (CUDA-core float32).
  *   in_dtype RET_BF16: tensor-core kernels (tcgen05, TMEM accumulators), dk in
- *          {64, 128, 256}, dv in {64, 128, 256, 512}, chunk in
- *          {64, 128, 256, 512}.  Chunks shorter than 128 tokens are
+ *          {128, 256}, dv in {64, 128, 256, 512}, chunk in
+ *          {64, 128, 256, 512}; other bf16 shapes (dk = 64 among them)
+ *          return RET_ERR_UNSUPPORTED.  Chunks shorter than 128 tokens are
  *          evaluated as 128-token chunks, which yields the same result.
  *   out dtype RET_F32 or RET_BF16; H <= 64; T*H*max(dk,dv) < 2^31.
  */
@@ -285,6 +286,17 @@ RET_API ret_status msr_norm_gate(const void* o, ret_dtype o_dtype, const ret_nor
  * call, RET_ERR_CUDA if the synchronisation itself failed.
  */
 RET_API ret_status retention_check_device_error(ret_stream_t stream);
+
+/*
+ * Failure-detection self-test (no counterpart on the pages: it exercises this
+ * library's own time-out path).  Enqueues on `stream` one single-warp kernel
+ * that waits on a shared-memory barrier nothing ever arrives on, through the
+ * same bounded wait every tensor-core kernel uses (about 2 s of SM clock).
+ * When the bound expires the kernel sets the device error word and returns,
+ * so a following retention_check_device_error() returns RET_ERR_TIMEOUT and
+ * the context stays usable.  Returns RET_ERR_CUDA if the launch failed.
+ */
+RET_API ret_status retention_selftest_wait_timeout(ret_stream_t stream);
 
 #ifdef __cplusplus
 }

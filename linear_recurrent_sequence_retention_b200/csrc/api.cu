@@ -323,6 +323,12 @@ ret_status msr_norm_gate(const void* o, ret_dtype o_dtype, const ret_norm_gate* 
                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 
+ret_status retention_selftest_wait_timeout(ret_stream_t stream) {
+  unsigned* err = error_word();
+  if (!err) return RET_ERR_CUDA;
+  return cuda_status(ret::launch_wait_timeout_selftest(err, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 ret_status retention_check_device_error(ret_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return RET_ERR_CUDA;

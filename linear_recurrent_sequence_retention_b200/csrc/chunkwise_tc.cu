@@ -1115,7 +1115,29 @@ cudaError_t launch_out(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ms, mg, my, op);
 }
 
+// One warp waits on an mbarrier that nothing arrives on, through the bounded
+// wait of the kernels above; on expiry that wait raises the time-out error.
+__global__ void wait_timeout_selftest_kernel(unsigned* err) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) {
+    volatile int* af = &abort_flag;
+    (void)mbar_wait(&bar, 0, af, err);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t s) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, s>>>(err);
+  return cudaGetLastError();
+}
 
 bool chunkwise_tc_supported(int dk, int dv, int chunk) {
   const bool dk_ok = dk == 128 || dk == 256;

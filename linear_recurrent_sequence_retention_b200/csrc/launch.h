@@ -54,6 +54,9 @@ cudaError_t launch_norm_gate(const void* o, DType o_t, const void* g, DType g_t,
 
 // Tensor-core (tcgen05) chunkwise forward for bf16 inputs.
 bool chunkwise_tc_supported(int dk, int dv, int chunk);
+
+// One bounded wait that is never satisfied (failure-detection self-test).
+cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t s);
 int chunkwise_tc_chunk(int chunk);  // chunk length the kernels evaluate
 cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const void* v,
                                 const SeqLayout& L, const float* state_in, bool has_state_in,

@@ -42,6 +42,7 @@ EXPORTED = (
     "retention_recurrent_step",
     "msr_norm_gate",
     "retention_check_device_error",
+    "retention_selftest_wait_timeout",
 )
 
 
@@ -100,6 +101,8 @@ def lib():
     L.msr_norm_gate.argtypes = [vp, ci, ctypes.POINTER(NormGate), vp, ci, ci, ci, ci, vp]
     L.retention_check_device_error.restype = ci
     L.retention_check_device_error.argtypes = [vp]
+    L.retention_selftest_wait_timeout.restype = ci
+    L.retention_selftest_wait_timeout.argtypes = [vp]
     _lib = L
     return L
 
@@ -343,15 +346,22 @@ def recurrent_step(q, k, v, gamma, state, out_dtype=torch.float32, out=None, str
     return out
 
 
-def norm_gate(o, g, weight=None, bias=None, eps=1e-5, out_dtype=None, stream=None):
-    """Per-head GroupNorm + swish gate; o: [ntok,H,dv] (any leading dims), g same size."""
+def norm_gate(o, g, weight=None, bias=None, eps=1e-5, out_dtype=None, out=None, stream=None):
+    """Per-head GroupNorm + swish gate; o: [ntok,H,dv] (any leading dims), g same size.
+    ``out`` (optional) is a preallocated contiguous output of o's size."""
     _dev(o, "o")
     _dev(g, "g")
     H, dv = o.shape[-2], o.shape[-1]
     ntok = o.numel() // (H * dv)
     if g.numel() != o.numel():
         raise ValueError("g must have as many elements as o")
-    y = torch.empty(o.shape, device=o.device, dtype=out_dtype or o.dtype)
+    if out is None:
+        y = torch.empty(o.shape, device=o.device, dtype=out_dtype or o.dtype)
+    else:
+        _dev(out, "out")
+        if out.numel() != o.numel():
+            raise ValueError("out must have as many elements as o")
+        y = out
     ng = NormGate(g.data_ptr(), _dt(g), weight.data_ptr() if weight is not None else None,
                   bias.data_ptr() if bias is not None else None, float(eps))
     st = lib().msr_norm_gate(_ptr(o), _dt(o), ctypes.byref(ng), _ptr(y), _dt(y), ntok, H, dv,
@@ -363,3 +373,9 @@ def norm_gate(o, g, weight=None, bias=None, eps=1e-5, out_dtype=None, stream=Non
 def check_device_error(stream=None):
     """Synchronise the stream and raise if a kernel reported a device-side error."""
     _check(lib().retention_check_device_error(_stream(stream)), "retention_check_device_error")
+
+
+def selftest_wait_timeout(stream=None):
+    """Enqueue the failure-detection self-test: one bounded wait that is never
+    satisfied.  A following check_device_error() raises RET_ERR_TIMEOUT."""
+    _check(lib().retention_selftest_wait_timeout(_stream(stream)), "retention_selftest_wait_timeout")
