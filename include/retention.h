@@ -165,9 +165,9 @@ RET_API size_t retention_chunkwise_workspace_size(ret_dtype in_dtype, int chunk,
  * Supported:
  *   in_dtype RET_F32: dk, dv in 1..256, any chunk >= 1 (CUDA-core float32).
  *   in_dtype RET_BF16: tensor-core kernels (tcgen05, TMEM accumulators), dk in
- *          {128, 256}, dv in {64, 128, 256, 512}, chunk in
- *          {64, 128, 256, 512}; other bf16 shapes (dk = 64 among them)
- *          return RET_ERR_UNSUPPORTED.  Chunks shorter than 128 tokens are
+ *          {64, 128, 256}, dv in {64, 128, 256, 512}, chunk in
+ *          {64, 128, 256, 512}; other bf16 shapes return
+ *          RET_ERR_UNSUPPORTED.  Chunks shorter than 128 tokens are
  *          evaluated as 128-token chunks, which yields the same result.
  *   out dtype RET_F32 or RET_BF16; H <= 64; T*H*max(dk,dv) < 2^31.
  */

@@ -171,12 +171,14 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // 1-D grid, sequence-major: all (head, d_k block, d_v part) CTAs of a
   // sequence are adjacent, and packed sequences go longest first
-  const int zn = (p.dk / 128) * (p.dv / NS);
+  const int mblocks = (p.dk + 127) / 128;        // 128-row blocks of d_k (d_k = 64: one, half used)
+  const int zn = mblocks * (p.dv / NS);
   const int rank = static_cast<int>(blockIdx.x / (p.H * zn));
   const int rem = static_cast<int>(blockIdx.x % (p.H * zn));
   const int h = rem / zn, zz = rem % zn;
   const int s = p.order ? p.order[rank] : rank;
-  const int m = zz % (p.dk / 128), part = zz / (p.dk / 128);
+  const int m = zz % mblocks, part = zz / mblocks;
+  const int kboxes = p.dk >= 128 ? 2 : 1;        // 64-column K boxes loaded per stage
   const SeqLayout& L = p.L;
   int a, b;
   seq_bounds(L, s, a, b);
@@ -203,6 +205,15 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     tmem_alloc(tmem_hold, 2 * NS);       // two accumulators of NS columns
     tmem_relinquish();
   }
+  if (kboxes == 1) {
+    // d_k = 64: the second 64-row half of every zeta*K tile (hi and lo) stays
+    // zero, so the 128-row MMA adds nothing to TMEM rows 64..127
+    for (int st = 0; st < NSTG; ++st)
+      for (int o = threadIdx.x * 16; o < static_cast<int>(kBox); o += kThreads * 16)
+        for (int hl = 0; hl < 2; ++hl)
+          *reinterpret_cast<uint4*>(smem + st * kStage + hl * kKBytes + kBox + o) = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -222,9 +233,9 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
           const int st = it % NSTG;
           if (!mbar_wait(&empty[st], ((it / NSTG) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
           uint8_t* base = smem + st * kStage;
-          mbar_arrive_expect_tx(&full[st], kKBytes + SC::kVBytes);
+          mbar_arrive_expect_tx(&full[st], kboxes * kBox + SC::kVBytes);
           const int y = tok0 + sb * kStTok;
-          for (int bx = 0; bx < 2; ++bx)
+          for (int bx = 0; bx < kboxes; ++bx)
             tma_load_2d(base + bx * kBox, &tmK, &full[st], h * p.dk + 128 * m + 64 * bx, y);
           for (int bx = 0; bx < NS / 64; ++bx)
             tma_load_2d(base + 2 * kKBytes + bx * kBox, &tmV, &full[st],
@@ -284,8 +295,9 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     const int quad = warp & 3;
     const int row = quad * 32 + lane;            // TMEM lane = row of the state block
     const int i = 128 * m + row;                 // d_k index
+    const bool row_ok = i < p.dk;                // d_k = 64: TMEM rows 64..127 hold zeros
     const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    const size_t st_off = ((static_cast<size_t>(s) * p.H + h) * p.dk + i) * p.dv + NS * part;
+    const size_t st_off = ((static_cast<size_t>(s) * p.H + h) * p.dk + (row_ok ? i : 0)) * p.dv + NS * part;
     const bool leader = threadIdx.x == 64;
     if (leader) tma_prefetch_desc(&tmW);
     auto slot_of = [&](int c) -> long long {
@@ -325,6 +337,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         fence_proxy_async_smem();
         asm volatile("bar.sync 2, 128;" ::: "memory");
         if (leader && slot_ok) {
+          // boxes of min(d_k, 128) rows: the first rows of the staged boxes
           tma_store_2d(&tmW, staging, NS * part + 32 * j, wrow);
           tma_store_2d(&tmW, staging + kTallBox, NS * part + 32 * j, wrow + p.dk);
           tma_store_commit();
@@ -337,7 +350,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
 #pragma unroll 1
       for (int j = 0; j < NS / 32; ++j) {
         float r[32];
-        if (p.state_in) {
+        if (p.state_in && row_ok) {
           const float4* src = reinterpret_cast<const float4*>(p.state_in + st_off + 32 * j);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -389,13 +402,14 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
           float r[32];
           tmem_ld32(trow + fcol + 32 * j, r);
           tmem_wait_ld();
+          if (!row_ok) continue;
           float4* dst = reinterpret_cast<float4*>(p.state_out + st_off + 32 * j);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             dst[e] = make_float4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]);
         }
       }
-    } else if (ok && p.state_out) {   // empty sequence: the state passes through
+    } else if (ok && p.state_out && row_ok) {   // empty sequence: the state passes through
       for (int j = 0; j < NS; j += 4) {
         float4 x = p.state_in ? *reinterpret_cast<const float4*>(p.state_in + st_off + j)
                               : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -538,7 +552,10 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const Decay1 dec(p.dec, h);
   // stages used by the MMA operands; the gate/output tile (NV/64 boxes of
   // 128 rows x 64 columns, two per stage) follows them in ring order
-  const int n_mma_units = (need_inter ? 2 * (DK / 64) : 0) + (r + 1) * (DK / 128 + 2);
+  // K(kb) is kKU units of kKB 64-column boxes (128 keys each)
+  constexpr int kKU = DK >= 128 ? DK / 128 : 1;
+  constexpr int kKB = DK >= 128 ? 2 : 1;
+  const int n_mma_units = (need_inter ? 2 * (DK / 64) : 0) + (r + 1) * (kKU + 2);
   constexpr int kIoBoxes = NV / 64;
   constexpr int kIoUnits = (kIoBoxes + 1) / 2;
   auto io_box = [&](int bx) -> uint8_t* {
@@ -612,10 +629,10 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       }
       auto load_k = [&](int kb) {
-        for (int ku = 0; ku < DK / 128 && ok; ++ku) {
-          uint8_t* dst = next(2 * kTallBox);
+        for (int ku = 0; ku < kKU && ok; ++ku) {
+          uint8_t* dst = next(kKB * kTallBox);
           if (!dst) { ok = false; break; }
-          for (int bx = 0; bx < 2; ++bx)
+          for (int bx = 0; bx < kKB; ++bx)
             tma_load_2d(dst + bx * kTallBox, &tmK, &full[it % NST], h * DK + 128 * ku + 64 * bx,
                         si.cs + kKeysPerBlock * kb);
           ++it;
@@ -695,11 +712,11 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
       auto issue_qk = [&](int kb) -> bool {
         const uint32_t dst = tmem + ((kb & 1) ? C::kTmemS1 : C::kTmemS0);
-        for (int ku = 0; ku < DK / 128; ++ku) {
+        for (int ku = 0; ku < kKU; ++ku) {
           const uint32_t sb = stage_wait();
           if (!sb) return false;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
+          for (int kk = 0; kk < 4 * kKB; ++kk) {
             const int qbox = ku * 2 + kk / 4;
             mma_bf16(dst, sdesc_sw128(q_base + qbox * kTallBox + (kk & 3) * 32, 16, 1024),
                      sdesc_sw128(sb + (kk / 4) * kTallBox + (kk & 3) * 32, 16, 1024), id_qk,
@@ -1085,7 +1102,7 @@ cudaError_t launch_state(const CUtensorMap& mk, const CUtensorMap& mv, const CUt
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(sp.L.nseq) * sp.H * (sp.dk / 128) * (sp.dv / NS));
+  dim3 grid(static_cast<unsigned>(sp.L.nseq) * sp.H * ((sp.dk + 127) / 128) * (sp.dv / NS));
   kern<<<grid, kThreads, smem, s>>>(mk, mv, mw, sp);
   return cudaGetLastError();
 }
@@ -1140,7 +1157,7 @@ cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t s) {
 }
 
 bool chunkwise_tc_supported(int dk, int dv, int chunk) {
-  const bool dk_ok = dk == 128 || dk == 256;
+  const bool dk_ok = dk == 64 || dk == 128 || dk == 256;
   const bool dv_ok = dv == 64 || dv == 128 || dv == 256 || dv == 512;
   const bool c_ok = chunk == 64 || chunk == 128 || chunk == 256 || chunk == 512;
   return dk_ok && dv_ok && c_ok;
@@ -1163,7 +1180,7 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
     // most of the SMs (every CTA walks its sequence serially, so a small
     // batch needs narrower blocks to fill the machine)
     int NS = dv >= 256 ? 256 : dv;
-    const long long blocks = static_cast<long long>(L.nseq) * H * (dk / 128);
+    const long long blocks = static_cast<long long>(L.nseq) * H * ((dk + 127) / 128);
     const int sms = sm_count();
     while (NS > 64 && blocks * (dv / NS) * 5 < static_cast<long long>(sms) * 3) NS /= 2;
     StateParams sp;
@@ -1182,7 +1199,7 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
     const uint64_t wrows = static_cast<uint64_t>(ws.nslots) * H * 2 * dk;   // hi and lo planes
     if (!make_map(&mk_st, k, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 64) ||
         !make_map(&mv_st, v, static_cast<uint64_t>(H) * dv, Ttot, static_cast<uint64_t>(H) * dv, 64) ||
-        !make_map(&mw_st, ws.states, dv, wrows, dv, 128))
+        !make_map(&mw_st, ws.states, dv, wrows, dv, dk < 128 ? dk : 128))
       return cudaErrorInvalidValue;
     switch (NS) {
       case 64: e = launch_state<64>(mk_st, mv_st, mw_st, sp, s); break;
@@ -1229,6 +1246,13 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
       (op.y_tma && !make_map(&my, out, hdv, Ttot, hdv, 128)))
     return cudaErrorInvalidValue;
   const long long units = ws.nslots * op.rb;
+  if (dk == 64) {
+    switch (NV) {
+      case 64: return launch_out<64, 64>(mq, mk, mv, ms, mg, my, op, units, s);
+      case 128: return launch_out<64, 128>(mq, mk, mv, ms, mg, my, op, units, s);
+      default: return launch_out<64, 256>(mq, mk, mv, ms, mg, my, op, units, s);
+    }
+  }
   if (dk == 128) {
     switch (NV) {
       case 64: return launch_out<128, 64>(mq, mk, mv, ms, mg, my, op, units, s);

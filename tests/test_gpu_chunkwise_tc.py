@@ -48,6 +48,7 @@ def _run(B, T, H, dk, dv, chunk, gated, out_dtype, state_in=False, seed=0, gam=N
 @pytest.mark.parametrize("dk,dv,chunk", [
     (128, 64, 128), (128, 128, 128), (128, 256, 128), (128, 256, 256),
     (256, 256, 512), (256, 512, 512), (256, 512, 128), (128, 512, 256), (256, 64, 256),
+    (64, 128, 128), (64, 512, 256), (64, 64, 512),
 ])
 @pytest.mark.parametrize("gated", [False, True])
 def test_shapes_f32_out(dk, dv, chunk, gated):
@@ -98,10 +99,11 @@ def test_chunk_length_invariance_bf16():
         assert_close(f64(o), ref, "bf16", 2, f"chunk={chunk}")
 
 
-def test_varlen_packed():
+@pytest.mark.parametrize("dk", [128, 64])
+def test_varlen_packed(dk):
     lens = [300, 0, 1, 77, 128, 129, 513, 64]
     cu = W.cu_seqlens_of(lens)
-    H, dk, dv, chunk = 2, 128, 128, 128
+    H, dv, chunk = 2, 128, 128
     Tt = int(cu[-1])
     q, k, v, g = W.make_qkvg(1, Tt, H, dk, dv, "bf16", seed=13)
     gam = W.head_gammas(H)

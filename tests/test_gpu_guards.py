@@ -35,7 +35,7 @@ def assert_guards(buf, what):
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("gated", [False, True])
 @pytest.mark.parametrize("dk,dv,chunk,T", [(128, 128, 128, 333), (256, 512, 512, 700),
-                                           (128, 256, 256, 129)])
+                                           (128, 256, 256, 129), (64, 256, 128, 200)])
 def test_chunkwise_tc_writes_only_its_outputs(out_dtype, gated, dk, dv, chunk, T):
     B, H = 2, 2
     q, k, v, g = W.make_qkvg(B, T, H, dk, dv, "bf16", seed=dk + T, gate=gated, device="cuda")
