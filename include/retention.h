@@ -56,7 +56,7 @@
  *             arguments are valid but this build has no kernel for the shape
  *             or dtype combination; there is no fallback path.
  *   Aliasing: outputs must not overlap inputs, except that
- *             retention_recurrent_step updates `state` in place by design.
+ *             retention_recurrent_step(s) update `state` in place by design.
  */
 #ifndef RETENTION_H_
 #define RETENTION_H_
@@ -265,6 +265,28 @@ RET_API ret_status retention_recurrent_step(const void* q, const void* k, const 
                                     float* state, void* o, ret_dtype o_dtype,
                                     int N, int H, int dk, int dv,
                                     ret_stream_t stream);
+
+/*
+ * Tn consecutive recurrent decode steps for N independent sequences in one
+ * pass over the state (the recurrence of retention_recurrent_step applied Tn
+ * times; abeam.tech summary, 「学習は並列、生成は状態更新」, with the sum
+ * unrolled as in the chunkwise form of 「長文の学習にはチャンク再帰を使う」):
+ *     o_t = gamma^(t+1) q_t S + sum_{j<=t} gamma^(t-j) (q_t . k_j) v_j
+ *     S  <- gamma^Tn S + sum_j gamma^(Tn-1-j) k_j^T v_j
+ * for t = 0..Tn-1, with S the state entering the call.  The state is read and
+ * written once for all Tn tokens (speculative or prompt-continuation steps).
+ *   q, k: [N,Tn,H,dk] in_dtype   v: [N,Tn,H,dv] in_dtype   (token-major)
+ *   state: [N,H,dk,dv] float32, read and overwritten
+ *   o: [N,Tn,H,dv] o_dtype
+ * Supported: 1 <= Tn <= 16, dk and dv multiples of 4 with dk <= 512 and
+ * dv <= 4096 (float32 FMAs on CUDA cores; the call is bound by the state's
+ * HBM traffic); otherwise RET_ERR_UNSUPPORTED.
+ */
+RET_API ret_status retention_recurrent_steps(const void* q, const void* k, const void* v,
+                                             ret_dtype in_dtype, const double* gamma,
+                                             float* state, void* o, ret_dtype o_dtype,
+                                             int N, int Tn, int H, int dk, int dv,
+                                             ret_stream_t stream);
 
 /*
  * Standalone per-head GroupNorm + Swish gate (the epilogue that

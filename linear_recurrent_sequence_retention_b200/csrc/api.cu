@@ -308,6 +308,24 @@ ret_status retention_recurrent_step(const void* q, const void* k, const void* v,
                                              dk, dv, dec, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+ret_status retention_recurrent_steps(const void* q, const void* k, const void* v,
+                                     ret_dtype in_dtype, const double* gamma, float* state,
+                                     void* o, ret_dtype o_dtype, int N, int Tn, int H, int dk,
+                                     int dv, ret_stream_t stream) {
+  if (!q || !k || !v || !state || !o || !dtype_ok(in_dtype) || !dtype_ok(o_dtype))
+    return RET_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(o))
+    return RET_ERR_INVALID_ARG;
+  if (N < 1 || Tn < 1 || H < 1 || dk < 1 || dv < 1) return RET_ERR_INVALID_ARG;
+  ret::HeadDecay dec;
+  if (!make_decay(gamma, H, &dec)) return RET_ERR_INVALID_ARG;
+  if (Tn > 16 || dk > 512 || dv > 4096 || dk % 4 != 0 || dv % 4 != 0) return RET_ERR_UNSUPPORTED;
+  if (N > 65535 || H > 65535) return RET_ERR_UNSUPPORTED;
+  return cuda_status(ret::launch_decode_steps(q, k, v, dt(in_dtype), state, o, dt(o_dtype), N, Tn,
+                                              H, dk, dv, dec,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
 ret_status msr_norm_gate(const void* o, ret_dtype o_dtype, const ret_norm_gate* ng, void* y,
                          ret_dtype y_dtype, int ntok, int H, int dv, ret_stream_t stream) {
   if (!o || !ng || !ng->g || !y || !dtype_ok(o_dtype) || !dtype_ok(y_dtype) ||

@@ -44,6 +44,10 @@ cudaError_t launch_chunkwise_simt(int phases, const void* q, const void* k, cons
                                   ChunkWorkspace ws, int H, int dk, int dv,
                                   const HeadDecay& dec, unsigned* err, cudaStream_t s);
 
+// Tn (1..16) tokens per sequence in one pass over the state.
+cudaError_t launch_decode_steps(const void* q, const void* k, const void* v, DType in_t,
+                                float* state, void* o, DType o_t, int N, int Tn, int H, int dk,
+                                int dv, const HeadDecay& dec, cudaStream_t s);
 cudaError_t launch_decode_step(const void* q, const void* k, const void* v, DType in_t,
                                float* state, void* o, DType o_t, int N, int H, int dk, int dv,
                                const HeadDecay& dec, cudaStream_t s);

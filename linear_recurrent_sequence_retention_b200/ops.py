@@ -40,6 +40,7 @@ EXPORTED = (
     "retention_chunkwise_outputs",
     "retention_chunkwise_fwd_static_ws",
     "retention_recurrent_step",
+    "retention_recurrent_steps",
     "msr_norm_gate",
     "retention_check_device_error",
     "retention_selftest_wait_timeout",
@@ -97,6 +98,8 @@ def lib():
                                                     ci, ci, ci, ci, ci, vp]
     L.retention_recurrent_step.restype = ci
     L.retention_recurrent_step.argtypes = [vp, vp, vp, ci, cd, vp, vp, ci, ci, ci, ci, ci, vp]
+    L.retention_recurrent_steps.restype = ci
+    L.retention_recurrent_steps.argtypes = [vp, vp, vp, ci, cd, vp, vp, ci, ci, ci, ci, ci, ci, vp]
     L.msr_norm_gate.restype = ci
     L.msr_norm_gate.argtypes = [vp, ci, ctypes.POINTER(NormGate), vp, ci, ci, ci, ci, vp]
     L.retention_check_device_error.restype = ci
@@ -343,6 +346,26 @@ def recurrent_step(q, k, v, gamma, state, out_dtype=torch.float32, out=None, str
                                         _ptr(state), _ptr(out), _dt(out), N, H, dk, dv,
                                         _stream(stream))
     _check(st, "retention_recurrent_step")
+    return out
+
+
+def recurrent_steps(q, k, v, gamma, state, out_dtype=torch.float32, out=None, stream=None):
+    """Tn decode steps in one pass over the state; q,k: [N,Tn,H,dk], v: [N,Tn,H,dv];
+    updates ``state`` [N,H,dk,dv] in place and returns o [N,Tn,H,dv]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (state, "state")):
+        _dev(t, n)
+    N, Tn, H, dk = q.shape
+    dv = v.shape[3]
+    if state.dtype != torch.float32 or tuple(state.shape) != (N, H, dk, dv):
+        raise ValueError(f"state must be float32 [{N},{H},{dk},{dv}]")
+    if out is None:
+        out = torch.empty(N, Tn, H, dv, device=q.device, dtype=out_dtype)
+    else:
+        _dev(out, "out")
+    g = _gammas(gamma, H)
+    st = lib().retention_recurrent_steps(_ptr(q), _ptr(k), _ptr(v), _dt(q), g, _ptr(state),
+                                         _ptr(out), _dt(out), N, Tn, H, dk, dv, _stream(stream))
+    _check(st, "retention_recurrent_steps")
     return out
 
 

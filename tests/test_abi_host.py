@@ -121,6 +121,18 @@ def test_decode_and_norm_gate_reject_bad_arguments():
     assert L.msr_norm_gate(FAKE, 1, ctypes.byref(ng), FAKE, 1, 0, 2, 8, None) == ops.RET_ERR_INVALID_ARG
 
 
+def test_recurrent_steps_reject_bad_arguments():
+    ops, L = _lib()
+    f = L.retention_recurrent_steps
+    # (q, k, v, in_dtype, gamma, state, o, o_dtype, N, Tn, H, dk, dv, stream)
+    assert f(FAKE, FAKE, FAKE, 1, _g(0.5), None, FAKE, 0, 1, 4, 1, 8, 8, None) == ops.RET_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, _g(0.5), FAKE, FAKE, 0, 1, 0, 1, 8, 8, None) == ops.RET_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, _g(1.5), FAKE, FAKE, 0, 1, 4, 1, 8, 8, None) == ops.RET_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, _g(0.5), FAKE, FAKE, 0, 1, 17, 1, 8, 8, None) == ops.RET_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 1, _g(0.5), FAKE, FAKE, 0, 1, 4, 1, 6, 8, None) == ops.RET_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 1, _g(0.5), FAKE, FAKE, 0, 1, 4, 1, 1024, 8, None) == ops.RET_ERR_UNSUPPORTED
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     from linear_recurrent_sequence_retention_b200 import ops
     monkeypatch.setattr(ops, "_lib", None)
