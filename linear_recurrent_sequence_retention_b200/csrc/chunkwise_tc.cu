@@ -1046,6 +1046,479 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 }
 
 // ===========================================================================
+// Output kernel for one-block chunks (compact: two CTAs per SM)
+// ===========================================================================
+// When every chunk is a single 128-row block (chunk <= 128) a tile has one
+// key block: a handful of MMAs against fixed costs (the Q and state loads, the
+// GroupNorm/gate pass).  This variant holds half an SM: 6 warps (producer, MMA
+// issuer, one epilogue warpgroup that forms P over all 128 keys and owns all
+// output columns), 256 TMEM columns (O, then the score tile) and 16 KB ring
+// stages in about 100 KB of shared memory, so two tiles share every SM and one
+// tile's epilogue overlaps the other's loads and MMAs.  Same arithmetic as
+// output_kernel (hi/lo P and state, one-pass GroupNorm statistics, one-op
+// swish), for d_k <= 128 and d_v parts of <= 128 columns.
+constexpr int kThreadsC = 192;
+constexpr uint32_t kStageC = 16384;
+
+template <int DK, int NV>
+struct OutCfgC {
+  static constexpr uint32_t kQBytes = (DK / 64) * kTallBox;
+  // barriers | gamma^d table | the partner CTA's GroupNorm (mean, M2) per row
+  static constexpr uint32_t kMiscBytes = 256 + 512 + 1024;
+  static constexpr uint32_t kBudget = 113 * 1024;                 // two CTAs per SM
+  static constexpr int kStages = static_cast<int>((kBudget - kQBytes - kMiscBytes) / kStageC);
+  static constexpr uint32_t kOffStages = kQBytes;
+  static constexpr uint32_t kOffMisc = kOffStages + kStages * kStageC;
+  static constexpr uint32_t kSmem = kOffMisc + kMiscBytes;
+  static constexpr uint32_t kTmemO = 0, kTmemS = 128;
+};
+
+// Named barrier over the 128 threads of the compact kernel's epilogue warpgroup.
+__device__ __forceinline__ void epi_sync_c() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int DK, int NV>
+__global__ void __launch_bounds__(256, 2)   // 6 warps, registers sized as for 8 (allocation granularity)
+output_kernel_c(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
+                const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmY,
+                const OutParams p) {
+  using C = OutCfgC<DK, NV>;
+  constexpr int NST = C::kStages;
+  static_assert(DK <= 128 && NV <= 128, "compact tiles: d_k <= 128, d_v part <= 128");
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffMisc);
+  uint64_t* full = bars;                 // [NST]
+  uint64_t* empty = full + NST;          // [NST]
+  uint64_t* bar_q = empty + NST;
+  uint64_t* bar_inter = bar_q + 1;
+  uint64_t* bar_s = bar_inter + 1;       // scores ready in TMEM
+  uint64_t* bar_p = bar_s + 1;           // P written over the scores
+  uint64_t* bar_o = bar_p + 1;           // all MMAs done
+  uint64_t* drain = bar_o + 1;
+  uint64_t* bar_x = drain + 1;           // the partner's statistics have arrived
+  uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(bar_x + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_hold + 1);
+  float* pow_tab = reinterpret_cast<float*>(smem + C::kOffMisc + 256);    // gamma^d
+  float* xrecv = reinterpret_cast<float*>(smem + C::kOffMisc + 768);     // [128][2]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int part = blockIdx.x % p.parts;
+  const long long slot = blockIdx.x / p.parts;
+  const int h = blockIdx.y;
+  SeqInfo si;
+  // Identical for both CTAs of a cluster, so a skipped slot skips together.
+  if (slot >= p.L.nslots) return;
+  if (!slot_to_chunk(p.L, p.chunk_base, slot, si)) return;
+  const int t0 = si.cs;                                   // first token of the chunk
+  const int nrows = min(kRowsPerTile, si.len);
+  const bool need_inter = si.c > 0 || p.has_state_in;
+  const bool xchg = p.parts > 1 && p.gated;
+  const Decay1 dec(p.dec, h);
+  // ring units (16 KB): [S_hi, S_lo of d_k rows 64u..64u+63], K (DK/64 boxes of
+  // 128 keys x 64 d_k), V (keys 0-63, 64-127), then the gate/output tile, one
+  // 128 x 64 box per unit
+  const int n_mma_units = (need_inter ? 2 * (DK / 64) : 0) + DK / 64 + 2;
+  auto io_box = [&](int bx) -> uint8_t* {
+    return smem + C::kOffStages + ((n_mma_units + bx) % NST) * kStageC;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(bar_q, 1);
+    mbar_init(bar_inter, 1);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_p, kWgThreads);
+    mbar_init(bar_o, 1);
+    mbar_init(drain, 1);
+    mbar_init(bar_x, kWgThreads);
+    *abort_flag = 0;
+    if ((smem_u32(smem) & 1023u) != 0) {
+      *abort_flag = 1;
+      raise_error(p.err, kErrTimeout);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_hold, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_hold;
+  if (xchg) cluster_arrive_relaxed();    // barrier initialisation done (waited on before first use)
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && !*abort_flag) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmS);
+      mbar_arrive_expect_tx(bar_q, C::kQBytes);
+      for (int u = 0; u < DK / 64; ++u)
+        tma_load_2d(smem + u * kTallBox, &tmQ, bar_q, h * DK + 64 * u, t0);
+      int it = 0;
+      bool ok = true;
+      auto next = [&](uint32_t bytes) -> uint8_t* {
+        const int st = it % NST;
+        if (!mbar_wait(&empty[st], ((it / NST) & 1) ^ 1, abort_flag, p.err)) return nullptr;
+        mbar_arrive_expect_tx(&full[st], bytes);
+        return smem + C::kOffStages + st * kStageC;
+      };
+      if (need_inter) {
+        for (int u = 0; u < DK / 64 && ok; ++u) {
+          for (int hl = 0; hl < 2 && ok; ++hl) {
+            const int srow = static_cast<int>(((slot * p.H + h) * 2 + hl) * DK) + 64 * u;
+            uint8_t* dst = next((NV / 64) * kBox);
+            if (!dst) { ok = false; break; }
+            for (int bx = 0; bx < NV / 64; ++bx)
+              tma_load_2d(dst + bx * kBox, &tmS, &full[it % NST], NV * part + 64 * bx, srow);
+            ++it;
+          }
+        }
+      }
+      for (int ku = 0; ku < DK / 64 && ok; ++ku) {
+        uint8_t* dst = next(kTallBox);
+        if (!dst) { ok = false; break; }
+        tma_load_2d(dst, &tmK, &full[it % NST], h * DK + 64 * ku, si.cs);
+        ++it;
+      }
+      for (int vu = 0; vu < 2 && ok; ++vu) {
+        uint8_t* dst = next((NV / 64) * kBox);
+        if (!dst) { ok = false; break; }
+        for (int bx = 0; bx < NV / 64; ++bx)
+          tma_load_2d(dst + bx * kBox, &tmV, &full[it % NST], h * p.dv + NV * part + 64 * bx,
+                      si.cs + 64 * vu);
+        ++it;
+      }
+      if (p.gated && p.g_tma) {      // the gate rows of this tile, for the epilogue
+        tma_prefetch_desc(&tmG);
+        for (int u = 0; u < NV / 64 && ok; ++u) {
+          uint8_t* dst = next(kTallBox);
+          if (!dst) { ok = false; break; }
+          tma_load_2d(dst, &tmG, &full[it % NST], h * p.dv + NV * part + 64 * u, t0);
+          ++it;
+        }
+      }
+      if (!ok) {
+        mbar_wait_drain(bar_q, 0);
+        for (int j = 1; j <= NST && it - j >= 0; ++j) {
+          const int i2 = it - j;
+          mbar_wait_drain(&full[i2 % NST], (i2 / NST) & 1);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0 && !*abort_flag) {
+      constexpr uint32_t id_qs = idesc_bf16_f32(128, NV, false, true);
+      constexpr uint32_t id_qk = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t id_pv = idesc_bf16_f32(128, NV, false, true);
+      const uint32_t q_base = smem_u32(smem);
+      const uint32_t st_base = smem_u32(smem + C::kOffStages);
+      int it = 0;
+      bool ok = true, issued = false;
+      auto stage_wait = [&]() -> uint32_t {
+        const int st = it % NST;
+        if (!mbar_wait(&full[st], (it / NST) & 1, abort_flag, p.err)) return 0;
+        tc_fence_after();
+        return st_base + st * kStageC;
+      };
+      auto stage_free = [&]() {
+        mma_commit(&empty[it % NST]);
+        ++it;
+      };
+      ok = mbar_wait(bar_q, 0, abort_flag, p.err);
+      if (ok && need_inter) {
+        // O = Q S_hi + Q S_lo  (the state entering the chunk, split in two bf16 parts)
+        for (int u = 0; u < DK / 64 && ok; ++u) {
+          for (int hl = 0; hl < 2; ++hl) {
+            const uint32_t sb = stage_wait();
+            if (!sb) { ok = false; break; }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(tmem + C::kTmemO, sdesc_sw128(q_base + u * kTallBox + kk * 32, 16, 1024),
+                       sdesc_sw128(sb + kk * 2048, kBox, 1024), id_qs, (u | hl | kk) != 0);
+            issued = true;
+            stage_free();
+          }
+        }
+        if (ok) mma_commit(bar_inter);
+      }
+      // scores Q K^T of the chunk's keys
+      for (int ku = 0; ku < DK / 64 && ok; ++ku) {
+        const uint32_t sb = stage_wait();
+        if (!sb) { ok = false; break; }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + C::kTmemS, sdesc_sw128(q_base + ku * kTallBox + kk * 32, 16, 1024),
+                   sdesc_sw128(sb + kk * 32, 16, 1024), id_qk, (ku | kk) != 0);
+        issued = true;
+        stage_free();
+      }
+      if (ok) mma_commit(bar_s);
+      if (ok && !mbar_wait(bar_p, 0, abort_flag, p.err)) ok = false;
+      if (ok) {
+        tc_fence_after();
+        const uint32_t pbuf = tmem + C::kTmemS;
+        for (int vu = 0; vu < 2 && ok; ++vu) {
+          const uint32_t sb = stage_wait();
+          if (!sb) { ok = false; break; }
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int ks = vu * 4 + kk;                      // keys 16ks .. 16ks+15
+            const uint32_t a_hi = pbuf + 32 * (ks >> 1) + 8 * (ks & 1);
+            const uint64_t bd = sdesc_sw128(sb + kk * 2048, kBox, 1024);
+            mma_bf16_ts(tmem + C::kTmemO, a_hi, bd, id_pv, need_inter || ks > 0);
+            mma_bf16_ts(tmem + C::kTmemO, a_hi + 16, bd, id_pv, true);
+          }
+          stage_free();
+        }
+      }
+      if (ok) {
+        mma_commit(bar_o);
+      } else if (issued) {
+        mma_commit(drain);
+        mbar_wait_drain(drain, 0);
+      }
+    }
+  } else {
+    // ---------------- epilogue: one warpgroup, one thread per query row ----------------
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;                 // query row of the chunk
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t o_cols = tmem + lane_off + C::kTmemO;
+    const int et = threadIdx.x - 64;                  // 0..127
+    pow_tab[et] = dec.pow(et);
+    epi_sync_c();
+    bool ok = !*abort_flag;
+    if (ok && need_inter) {
+      // tcgen05.ld/st are warp-collective: every guard around them is warp-uniform
+      ok = warp_all(mbar_wait(bar_inter, 0, abort_flag, p.err));
+      if (ok) {
+        tc_fence_after();
+        const float sc = dec.pow(row + 1);
+        for (int j = 0; j < NV / 32; ++j) {
+          float x[32];
+          tmem_ld32(o_cols + 32 * j, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] *= sc;
+          tmem_st32(o_cols + 32 * j, x);
+        }
+        tmem_wait_st();
+      }
+    }
+    if (ok) ok = warp_all(mbar_wait(bar_s, 0, abort_flag, p.err));
+    if (ok) {
+      tc_fence_after();
+      const uint32_t buf = tmem + lane_off + C::kTmemS;
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {                   // keys 32j .. 32j+31
+        float x[32];
+        tmem_ld32(buf + 32 * j, x);
+        float wv[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int jp = 32 * j + e;
+          wv[e] = (jp <= row && jp < si.len) ? pow_tab[row - jp] : 0.f;
+        }
+        tmem_wait_ld();
+        float pw[32];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          uint32_t hi, lo;
+          const uint64_t p2 = f2_mul(f2_make(x[e], x[e + 1]), f2_make(wv[e], wv[e + 1]));
+          pack_split(f2_lo(p2), f2_hi(p2), hi, lo);
+          pw[e >> 1] = __uint_as_float(hi);
+          pw[16 + (e >> 1)] = __uint_as_float(lo);
+        }
+        tmem_st32(buf + 32 * j, pw);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p);
+    }
+    if (ok) ok = mbar_wait(bar_o, 0, abort_flag, p.err);
+    ok = warp_all(ok);
+    if (ok) tc_fence_after();
+    // GroupNorm statistics in one pass (shifted by the row's first value); the
+    // two d_v parts of a cluster combine as (mean, M2) pairs through the
+    // partner's receive buffer.  The exchange is unconditional, so an aborted
+    // CTA still meets its partner.
+    float mean_all = 0.f, rstd = 0.f;
+    if (p.gated) {
+      float mean = 0.f, m2 = 0.f;
+      if (ok) {
+        uint64_t s1 = 0, s2 = 0;
+        float x0 = 0.f;
+        for (int j = 0; j < NV / 32; ++j) {
+          float x[32];
+          tmem_ld32(o_cols + 32 * j, x);
+          tmem_wait_ld();
+          if (j == 0) x0 = x[0];
+          const uint64_t nx0 = f2_make(-x0, -x0);
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const uint64_t d = f2_add(f2_make(x[e], x[e + 1]), nx0);
+            s1 = f2_add(s1, d);
+            s2 = f2_fma(d, d, s2);
+          }
+        }
+        const float S1 = f2_lo(s1) + f2_hi(s1), S2 = f2_lo(s2) + f2_hi(s2);
+        mean = x0 + S1 * (1.0f / NV);
+        m2 = fmaxf(S2 - S1 * S1 * (1.0f / NV), 0.f);
+      }
+      float cnt = static_cast<float>(NV);
+      if (xchg) {
+        cluster_wait();                              // partner's barriers are initialised
+        const uint32_t other = cluster_ctarank() ^ 1u;
+        st_cluster_f32(cluster_addr(&xrecv[2 * row], other), mean);
+        st_cluster_f32(cluster_addr(&xrecv[2 * row + 1], other), m2);
+        mbar_arrive_cluster(cluster_addr(bar_x, other));
+        cluster_arrive();                            // this CTA's remote accesses are done
+        if (mbar_wait_cluster(bar_x, 0, abort_flag, p.err)) {
+          const float mo = xrecv[2 * row], m2o = xrecv[2 * row + 1];
+          const float d = mo - mean;
+          m2 = m2 + m2o + d * d * (cnt * 0.5f);
+          mean = 0.5f * (mean + mo);
+          cnt *= 2.f;
+        } else {
+          ok = false;
+        }
+      }
+      mean_all = mean;
+      rstd = 1.0f / sqrtf(m2 / cnt + p.eps);
+    }
+
+    // ---------------- GroupNorm, gate, store ----------------
+    const bool out_tma = p.y_tma && nrows == kRowsPerTile;
+    const bool leader = threadIdx.x == 64;
+    const bool live = row < nrows;
+    const int col0 = NV * part;
+    const size_t obase = (static_cast<size_t>(t0 + row) * p.H + h) * p.dv + col0;
+    const float shift = -mean_all * rstd;
+    bool go = warp_all(ok && !*abort_flag);
+    if (go && p.gated && p.g_tma) {
+      for (int u = 0; u < NV / 64 && go; ++u) {
+        const int unit = n_mma_units + u;
+        go = mbar_wait(&full[unit % NST], (unit / NST) & 1, abort_flag, p.err);
+      }
+      go = warp_all(go);
+    }
+    if (go) tc_fence_after();
+    if (out_tma && leader) tma_prefetch_desc(&tmY);
+    for (int j = 0; j < NV / 32; ++j) {
+      uint8_t* brow = io_box(j >> 1) + row * 128;      // 64-column box j/2
+      const int pc0 = (j & 1) * 4;
+      if (go) {
+        float x[32];
+        tmem_ld32(o_cols + 32 * j, x);
+        if (p.gated) {
+          float gv[32];
+          if (p.g_tma) {
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const uint4 u = *reinterpret_cast<const uint4*>(brow + (((pc0 + c4) ^ (row & 7)) << 4));
+              const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int q2 = 0; q2 < 4; ++q2) {
+                gv[8 * c4 + 2 * q2] = bf16_lo(wv[q2]);
+                gv[8 * c4 + 2 * q2 + 1] = bf16_hi(wv[q2]);
+              }
+            }
+          } else if (live) {
+            const float4* gp = reinterpret_cast<const float4*>(static_cast<const float*>(p.g) + obase + 32 * j);
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4) {
+              const float4 f = gp[c4];
+              gv[4 * c4] = f.x; gv[4 * c4 + 1] = f.y; gv[4 * c4 + 2] = f.z; gv[4 * c4 + 3] = f.w;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) gv[e] = 0.f;
+          }
+          tmem_wait_ld();
+          const uint64_t rs2 = f2_make(rstd, rstd), sh2 = f2_make(shift, shift);
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const uint64_t y2 = f2_fma(f2_make(x[e], x[e + 1]), rs2, sh2);
+            x[e] = f2_lo(y2);
+            x[e + 1] = f2_hi(y2);
+          }
+          if (p.gn_w || p.gn_b) {
+            const int c0 = h * p.dv + col0 + 32 * j;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (p.gn_w) x[e] *= p.gn_w[c0 + e];
+              if (p.gn_b) x[e] += p.gn_b[c0 + e];
+            }
+          }
+          // swish(g) = g sigmoid(g) = u + u tanh(u) with u = g/2: one
+          // special-function op per element
+          const uint64_t half2 = f2_make(0.5f, 0.5f);
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const uint64_t u2 = f2_mul(f2_make(gv[e], gv[e + 1]), half2);
+            const uint64_t s2 = f2_fma(u2, f2_make(tanh_fast(f2_lo(u2)), tanh_fast(f2_hi(u2))), u2);
+            const uint64_t o2 = f2_mul(f2_make(x[e], x[e + 1]), s2);
+            x[e] = f2_lo(o2);
+            x[e + 1] = f2_hi(o2);
+          }
+        } else {
+          tmem_wait_ld();
+        }
+        if (out_tma) {
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+            *reinterpret_cast<uint4*>(brow + (((pc0 + c4) ^ (row & 7)) << 4)) =
+                make_uint4(pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]), pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]),
+                           pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]), pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]));
+        } else if (live && p.out_bf16) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + obase + 32 * j);
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+            dst[c4] = make_uint4(pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]), pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]),
+                                 pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]), pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]));
+        } else if (live) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + 32 * j);
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4)
+            dst[c4] = make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
+        }
+      }
+      if (out_tma && (j & 1)) {                       // uniform over the warpgroup
+        // box j/2 is complete: hand it to the TMA engine
+        fence_proxy_async_smem();
+        epi_sync_c();
+        if (leader && go) {
+          tma_store_2d(&tmY, io_box(j >> 1), h * p.dv + NV * part + 64 * (j >> 1), t0);
+          tma_store_commit();
+        }
+      }
+    }
+    if (out_tma && go && leader) tma_store_wait_read();
+  }
+  if (xchg) {
+    if (warp < 2) {
+      cluster_wait();
+      cluster_arrive();
+    }
+    cluster_wait();        // the partner has written its statistics: no more remote access here
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// ===========================================================================
 // Host side
 // ===========================================================================
 // Streaming multiprocessors of the current device (queried once per device).
@@ -1149,6 +1622,30 @@ __global__ void wait_timeout_selftest_kernel(unsigned* err) {
   }
 }
 
+template <int DK, int NV>
+cudaError_t launch_out_c(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const CUtensorMap& ms, const CUtensorMap& mg, const CUtensorMap& my,
+                         const OutParams& op, long long slots, cudaStream_t s) {
+  using C = OutCfgC<DK, NV>;
+  auto kern = output_kernel_c<DK, NV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(C::kSmem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(slots * op.parts), op.H, 1);
+  cfg.blockDim = dim3(kThreadsC, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = op.parts;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ms, mg, my, op);
+}
+
 }  // namespace
 
 cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t s) {
@@ -1246,6 +1743,21 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
       (op.y_tma && !make_map(&my, out, hdv, Ttot, hdv, 128)))
     return cudaErrorInvalidValue;
   const long long units = ws.nslots * op.rb;
+  if (op.rb == 1 && dk <= 128 && dv <= 256) {
+    // one-block chunks: the compact kernel, two CTAs per SM, d_v in parts of <= 128
+    op.parts = dv > 128 ? 2 : 1;
+    const int NVc = dv / op.parts;
+    if (dk == 64) {
+      switch (NVc) {
+        case 64: return launch_out_c<64, 64>(mq, mk, mv, ms, mg, my, op, ws.nslots, s);
+        default: return launch_out_c<64, 128>(mq, mk, mv, ms, mg, my, op, ws.nslots, s);
+      }
+    }
+    switch (NVc) {
+      case 64: return launch_out_c<128, 64>(mq, mk, mv, ms, mg, my, op, ws.nslots, s);
+      default: return launch_out_c<128, 128>(mq, mk, mv, ms, mg, my, op, ws.nslots, s);
+    }
+  }
   if (dk == 64) {
     switch (NV) {
       case 64: return launch_out<64, 64>(mq, mk, mv, ms, mg, my, op, units, s);
