@@ -24,16 +24,19 @@
 //                 while that chunk runs.  The final f32 state goes to
 //                 state_out.
 //
-//  output_kernel  one CTA per (chunk, 128-row block r of the chunk, head,
-//                 NV-wide part of d_v); the halves of d_v = 512 form a 2-CTA
-//                 cluster that exchanges the GroupNorm statistics through
-//                 distributed shared memory.  MMA order:
+//  output_kernel  persistent, one CTA per SM, each CTA owning an NV-wide part
+//                 of d_v (the halves of d_v = 512 form a 2-CTA cluster that
+//                 exchanges the GroupNorm statistics through distributed
+//                 shared memory) and walking output tiles (chunk, 128-row
+//                 block r of the chunk, head).  MMA order per tile:
 //                   O  = Q S_hi + Q S_lo           (then O *= gamma^(i+1) in TMEM)
 //                   Sc = Q K_kb^T  for kb = 0..r   (double-buffered in TMEM)
-//                   O += P_hi V_kb + P_lo V_kb     (P = decayed, masked Sc, kept
+//                   O  += P_hi V_kb + P_lo V_kb    (P = decayed, masked Sc, kept
 //                                                   in TMEM as the MMA's A operand)
-//                 Each epilogue warpgroup forms P for half of the keys and owns
-//                 half of the output columns in the GroupNorm + gate epilogue.
+//                 O and the score buffers swap TMEM halves from tile to tile,
+//                 so the next tile's Q S MMAs run during this tile's
+//                 GroupNorm + gate epilogue.  Each epilogue warpgroup forms P
+//                 for half of the keys and owns half of the output columns.
 //
 // Precision: q, k, v enter the MMAs as the exact bf16 values they are; the
 // three rounded intermediates (decayed scores, carried state, zeta*K) enter as
@@ -465,7 +468,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
 }
 
 // ===========================================================================
-// Output kernel
+// Output kernel (persistent)
 // ===========================================================================
 constexpr uint32_t kOutStage = 32768;
 
@@ -486,6 +489,10 @@ struct OutParams {
   int H, dk, dv;
   int rb;                      // 128-row blocks per chunk
   int parts;                   // d_v parts (cluster size)
+  int ntiles;                  // chunk slots x heads x row blocks (persistent kernel)
+  int nch;                     // chunks per sequence (equal-length layout)
+  int nclusters;               // clusters in the persistent grid
+  int shift;                   // per-round rotation of the tile order (persistent kernel)
   HeadDecay dec;
   unsigned* err;
 };
@@ -493,19 +500,90 @@ struct OutParams {
 template <int DK, int NV>
 struct OutCfg {
   static constexpr uint32_t kQBytes = (DK / 64) * kTallBox;
-  // barriers | gamma^d table | gamma^(127-d) table | the partner CTA's
-  // GroupNorm (mean, M2) per row; this CTA's own partials live in the Q
-  // region, which is free once every MMA has completed
-  static constexpr uint32_t kMiscBytes = 256 + 512 + 512 + 1024;
+  // barriers | gamma^d table | GroupNorm pairs passed between the two
+  // warpgroups | GroupNorm pairs received from the partner CTA
+  static constexpr uint32_t kMiscBytes = 256 + 512 + 1024 + 1024;
   static constexpr int kStages = static_cast<int>((232448 - kQBytes - kMiscBytes) / kOutStage);
   static constexpr uint32_t kOffStages = kQBytes;
   static constexpr uint32_t kOffMisc = kOffStages + kStages * kOutStage;
   static constexpr uint32_t kSmem = kOffMisc + kMiscBytes;
-  // TMEM columns: O, then two score buffers of 128 columns.  P of key piece j
-  // (keys 32j..32j+31) is written over that piece's own columns: 32j..32j+15
-  // hold P_hi (two keys per column), 32j+16..32j+31 hold P_lo.
-  static constexpr uint32_t kTmemO = 0, kTmemS0 = 256, kTmemS1 = 384;
+  // TMEM: two halves of 256 columns used in turn.  Tile number n of a CTA
+  // keeps O in half (n & 1) and its two 128-column score buffers in the other
+  // half, so the next tile's Q S MMAs run while this tile's epilogue still
+  // reads O.  P of key piece j (keys 32j..32j+31) is written over that piece's
+  // own score columns: 32j..32j+15 hold P_hi (two keys per column),
+  // 32j+16..32j+31 hold P_lo.
+  static constexpr uint32_t kHalfCols = 256;
 };
+
+// One 128-row output tile: rows 128r..128r+127 of a chunk, one head, all d_v
+// columns of this CTA's part.
+struct OutTile {
+  SeqInfo si;
+  long long slot;
+  int h, r, t0, nrows;
+  bool inter;                  // reads the state carried into the chunk
+};
+
+// The tiles of one cluster.  Tile u = ((slot * H + h) * rb + (rb - 1 - r)):
+// the row blocks of a (chunk, head) are adjacent, heaviest first.  In round k
+// cluster c takes tile k * nclusters + (c + k * shift) mod nclusters, so each
+// round covers a contiguous range of tiles (the row blocks of a chunk run at
+// the same time and share its K, V and state tiles in L2) while the row block,
+// and with it the tile's cost, rotates from round to round for every cluster.
+// Every role of both CTAs of the cluster walks the same sequence.
+struct TileWalk {
+  int k = 0;
+  __device__ __forceinline__ bool next(const OutParams& p, int cid, OutTile& t) {
+    while (true) {
+      const int base = k * p.nclusters;
+      if (base >= p.ntiles) return false;
+      const int u = base + static_cast<int>(static_cast<unsigned>(cid + k * p.shift) %
+                                            static_cast<unsigned>(p.nclusters));
+      ++k;
+      if (u >= p.ntiles) continue;
+      // 32-bit index arithmetic: the host keeps the tile count below 2^31
+      const unsigned gh = static_cast<unsigned>(u) / static_cast<unsigned>(p.rb);
+      const unsigned slot = gh / static_cast<unsigned>(p.H);
+      t.h = static_cast<int>(gh - slot * static_cast<unsigned>(p.H));
+      t.r = p.rb - 1 - static_cast<int>(static_cast<unsigned>(u) - gh * static_cast<unsigned>(p.rb));
+      t.slot = slot;
+      if (p.L.cu == nullptr) {
+        const unsigned sq = slot / static_cast<unsigned>(p.nch);
+        if (static_cast<int>(sq) >= p.L.nseq) continue;
+        t.si.s = static_cast<int>(sq);
+        t.si.c = static_cast<int>(slot - sq * static_cast<unsigned>(p.nch));
+        t.si.a = t.si.s * p.L.T;
+        t.si.b = t.si.a + p.L.T;
+        t.si.cs = t.si.a + t.si.c * p.L.chunk;
+        t.si.len = min(p.L.chunk, t.si.b - t.si.cs);
+        if (t.si.len <= 0) continue;
+      } else if (!slot_to_chunk(p.L, p.chunk_base, slot, t.si)) {
+        continue;
+      }
+      if (t.r * kRowsPerTile >= t.si.len) continue;
+      t.t0 = t.si.cs + t.r * kRowsPerTile;
+      t.nrows = min(kRowsPerTile, t.si.len - t.r * kRowsPerTile);
+      t.inter = t.si.c > 0 || p.has_state_in;
+      return true;
+    }
+  }
+};
+
+// AND of `v` over the 256 epilogue threads (named barrier 4); every one of them
+// gets the same answer.
+__device__ __forceinline__ bool epi_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 4, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u)
+      : "memory");
+  return r != 0;
+}
 
 template <int DK, int NV>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -518,49 +596,38 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   constexpr int kHalf = NV / 2;                       // O columns per epilogue warpgroup
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffMisc);
-  uint64_t* full = bars;                 // [NST]
-  uint64_t* empty = full + NST;          // [NST]
-  uint64_t* bar_q = empty + NST;
-  uint64_t* bar_inter = bar_q + 1;
+  uint64_t* full = bars;                 // [NST] stage loaded
+  uint64_t* empty = full + NST;          // [NST] stage consumed
+  uint64_t* bar_q = empty + NST;         // Q tile loaded
+  uint64_t* q_free = bar_q + 1;          // every MMA reading Q has completed
+  uint64_t* bar_inter = q_free + 1;      // O = Q S done
   uint64_t* bar_s = bar_inter + 1;       // [2] scores ready in TMEM
   uint64_t* bar_p = bar_s + 2;           // [2] P written over the scores
-  uint64_t* bar_o = bar_p + 2;           // all MMAs done
-  uint64_t* drain = bar_o + 1;
+  uint64_t* bar_o = bar_p + 2;           // all MMAs of the tile done
+  uint64_t* o_free = bar_o + 1;          // the epilogue has read the tile's O
+  uint64_t* drain = o_free + 1;
   uint64_t* bar_x = drain + 1;           // the partner's statistics have arrived
-  uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(bar_x + 1);
+  uint64_t* bar_xack = bar_x + 1;        // the partner has read this CTA's statistics
+  uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(bar_xack + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_hold + 1);
-  float* pow_tab = reinterpret_cast<float*>(smem + C::kOffMisc + 256);    // gamma^d
-  float* rev_tab = reinterpret_cast<float*>(smem + C::kOffMisc + 768);    // gamma^(127-d)
-  float* xrecv = reinterpret_cast<float*>(smem + C::kOffMisc + 1280);    // [128][2]
-  float* wg_part = reinterpret_cast<float*>(smem);                        // [2][2][128], after bar_o
+  float* pow_tab = reinterpret_cast<float*>(smem + C::kOffMisc + 256);    // gamma^d, d < 128
+  float* wgx = reinterpret_cast<float*>(smem + C::kOffMisc + 768);        // [128][2]
+  float* xrecv = reinterpret_cast<float*>(smem + C::kOffMisc + 1792);     // [128][2]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int part = blockIdx.x % p.parts;
-  const long long unit = blockIdx.x / p.parts;
-  const int h = blockIdx.y;
-  const long long slot = unit / p.rb;
-  const int r = p.rb - 1 - static_cast<int>(unit % p.rb);   // heaviest row blocks first
-  SeqInfo si;
-  // Identical for both CTAs of a cluster, so a skipped unit skips together.
-  if (slot >= p.L.nslots) return;
-  if (!slot_to_chunk(p.L, p.chunk_base, slot, si)) return;
-  if (r * kRowsPerTile >= si.len) return;
-  const int t0 = si.cs + r * kRowsPerTile;                  // first token of the row block
-  const int nrows = min(kRowsPerTile, si.len - r * kRowsPerTile);
-  const bool need_inter = si.c > 0 || p.has_state_in;
+  const int cid = blockIdx.x / p.parts;
   const bool xchg = p.parts > 1 && p.gated;           // GroupNorm spans both CTAs of the cluster
-  const Decay1 dec(p.dec, h);
-  // stages used by the MMA operands; the gate/output tile (NV/64 boxes of
-  // 128 rows x 64 columns, two per stage) follows them in ring order
   // K(kb) is kKU units of kKB 64-column boxes (128 keys each)
   constexpr int kKU = DK >= 128 ? DK / 128 : 1;
   constexpr int kKB = DK >= 128 ? 2 : 1;
-  const int n_mma_units = (need_inter ? 2 * (DK / 64) : 0) + (r + 1) * (kKU + 2);
+  // the gate/output tile: NV/64 boxes of 128 rows x 64 columns, two per stage
   constexpr int kIoBoxes = NV / 64;
   constexpr int kIoUnits = (kIoBoxes + 1) / 2;
-  auto io_box = [&](int bx) -> uint8_t* {
-    const int unit = n_mma_units + bx / 2;
-    return smem + C::kOffStages + (unit % NST) * kOutStage + (bx & 1) * kTallBox;
+  // ring units of a tile: its MMA operands, then (when staged) the gate/output tile
+  auto mma_units = [&](const OutTile& t) { return (t.inter ? 2 * (DK / 64) : 0) + (t.r + 1) * (kKU + 2); };
+  auto io_staged = [&](const OutTile& t) {
+    return (p.gated && p.g_tma) || (p.y_tma && t.nrows == kRowsPerTile);
   };
 
   if (threadIdx.x == 0) {
@@ -569,14 +636,17 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mbar_init(&empty[i], 1);
     }
     mbar_init(bar_q, 1);
+    mbar_init(q_free, 1);
     mbar_init(bar_inter, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_s[i], 1);
       mbar_init(&bar_p[i], 2 * kWgThreads);
     }
     mbar_init(bar_o, 1);
+    mbar_init(o_free, 2 * kWgThreads);
     mbar_init(drain, 1);
     mbar_init(bar_x, kWgThreads);
+    mbar_init(bar_xack, kWgThreads);
     *abort_flag = 0;
     if ((smem_u32(smem) & 1023u) != 0) {
       *abort_flag = 1;
@@ -593,11 +663,18 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem = *tmem_hold;
   if (xchg) cluster_arrive_relaxed();    // barrier initialisation done (waited on before first use)
+  bool cluster_waited = false;           // this thread has passed that first cluster barrier phase
 
-  // Unit sequence shared by producer and MMA issuer, one 32 KB stage each:
+  TileWalk walk;
+  OutTile t;
+
+  // Per tile, the ring units in the order the MMA consumes them (32 KB each):
   //   [S_hi and S_lo of d_k rows 64u..64u+63, u < DK/64 (if the chunk reads a state)],
-  //   K(0), then for kb = 0..r: [K(kb+1) if kb < r], V(kb) keys 0-63, V(kb) keys 64-127.
-  // K(kb) is DK/128 units of 128 keys x 128 d_k.
+  //   K(0), then for kb = 0..r: [K(kb+1) if kb < r], V(kb) keys 0-63, V(kb) keys 64-127,
+  //   then the gate tile (or, with a bf16 output and no TMA gate, the same
+  //   number of empty units reserved as output staging).
+  // The ring runs on across tiles, so the next tile's Q, state and first key
+  // block stream in during this tile's epilogue.
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0 && !*abort_flag) {
@@ -605,10 +682,8 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmS);
-      mbar_arrive_expect_tx(bar_q, C::kQBytes);
-      for (int u = 0; u < DK / 64; ++u)
-        tma_load_2d(smem + u * kTallBox, &tmQ, bar_q, h * DK + 64 * u, t0);
-      int it = 0;
+      if (p.gated && p.g_tma) tma_prefetch_desc(&tmG);
+      int it = 0, tq = 0;
       bool ok = true;
       auto next = [&](uint32_t bytes) -> uint8_t* {
         const int st = it % NST;
@@ -616,57 +691,68 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_arrive_expect_tx(&full[st], bytes);
         return smem + C::kOffStages + st * kOutStage;
       };
-      if (need_inter) {
-        for (int u = 0; u < DK / 64 && ok; ++u) {
-          for (int hl = 0; hl < 2 && ok; ++hl) {
-            const int srow = static_cast<int>(((slot * p.H + h) * 2 + hl) * DK) + 64 * u;
+      while (ok && walk.next(p, cid, t)) {
+        const int r = t.r;
+        // Q of this tile, once every MMA of the previous tile that reads Q is done
+        if (tq > 0 && !mbar_wait(q_free, (tq - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+        mbar_arrive_expect_tx(bar_q, C::kQBytes);
+        for (int u = 0; u < DK / 64; ++u)
+          tma_load_2d(smem + u * kTallBox, &tmQ, bar_q, t.h * DK + 64 * u, t.t0);
+        ++tq;
+        if (t.inter) {
+          for (int u = 0; u < DK / 64 && ok; ++u) {
+            for (int hl = 0; hl < 2 && ok; ++hl) {
+              const int srow = static_cast<int>(((t.slot * p.H + t.h) * 2 + hl) * DK) + 64 * u;
+              uint8_t* dst = next((NV / 64) * kBox);
+              if (!dst) { ok = false; break; }
+              for (int bx = 0; bx < NV / 64; ++bx)
+                tma_load_2d(dst + bx * kBox, &tmS, &full[it % NST], NV * part + 64 * bx, srow);
+              ++it;
+            }
+          }
+        }
+        auto load_k = [&](int kb) {
+          for (int ku = 0; ku < kKU && ok; ++ku) {
+            uint8_t* dst = next(kKB * kTallBox);
+            if (!dst) { ok = false; break; }
+            for (int bx = 0; bx < kKB; ++bx)
+              tma_load_2d(dst + bx * kTallBox, &tmK, &full[it % NST], t.h * DK + 128 * ku + 64 * bx,
+                          t.si.cs + kKeysPerBlock * kb);
+            ++it;
+          }
+        };
+        auto load_v = [&](int kb) {
+          for (int vu = 0; vu < 2 && ok; ++vu) {
             uint8_t* dst = next((NV / 64) * kBox);
             if (!dst) { ok = false; break; }
             for (int bx = 0; bx < NV / 64; ++bx)
-              tma_load_2d(dst + bx * kBox, &tmS, &full[it % NST], NV * part + 64 * bx, srow);
+              tma_load_2d(dst + bx * kBox, &tmV, &full[it % NST], t.h * p.dv + NV * part + 64 * bx,
+                          t.si.cs + kKeysPerBlock * kb + 64 * vu);
+            ++it;
+          }
+        };
+        load_k(0);
+        for (int kb = 0; kb <= r && ok; ++kb) {
+          if (kb + 1 <= r) load_k(kb + 1);
+          load_v(kb);
+        }
+        if (ok && io_staged(t)) {
+          const bool load_g = p.gated && p.g_tma;
+          for (int u = 0; u < kIoUnits && ok; ++u) {
+            const int nb = (kIoBoxes - 2 * u) >= 2 ? 2 : 1;
+            uint8_t* dst = next(load_g ? nb * kTallBox : 0);
+            if (!dst) { ok = false; break; }
+            if (load_g)
+              for (int bb = 0; bb < nb; ++bb)
+                tma_load_2d(dst + bb * kTallBox, &tmG, &full[it % NST],
+                            t.h * p.dv + NV * part + 64 * (2 * u + bb), t.t0);
             ++it;
           }
         }
       }
-      auto load_k = [&](int kb) {
-        for (int ku = 0; ku < kKU && ok; ++ku) {
-          uint8_t* dst = next(kKB * kTallBox);
-          if (!dst) { ok = false; break; }
-          for (int bx = 0; bx < kKB; ++bx)
-            tma_load_2d(dst + bx * kTallBox, &tmK, &full[it % NST], h * DK + 128 * ku + 64 * bx,
-                        si.cs + kKeysPerBlock * kb);
-          ++it;
-        }
-      };
-      auto load_v = [&](int kb) {
-        for (int vu = 0; vu < 2 && ok; ++vu) {
-          uint8_t* dst = next((NV / 64) * kBox);
-          if (!dst) { ok = false; break; }
-          for (int bx = 0; bx < NV / 64; ++bx)
-            tma_load_2d(dst + bx * kBox, &tmV, &full[it % NST], h * p.dv + NV * part + 64 * bx,
-                        si.cs + kKeysPerBlock * kb + 64 * vu);
-          ++it;
-        }
-      };
-      load_k(0);
-      for (int kb = 0; kb <= r && ok; ++kb) {
-        if (kb + 1 <= r) load_k(kb + 1);
-        load_v(kb);
-      }
-      if (p.gated && p.g_tma) {      // the gate rows of this tile, for the epilogue
-        tma_prefetch_desc(&tmG);
-        for (int u = 0; u < kIoUnits && ok; ++u) {
-          const int nb = (kIoBoxes - 2 * u) >= 2 ? 2 : 1;
-          uint8_t* dst = next(nb * kTallBox);
-          if (!dst) { ok = false; break; }
-          for (int bb = 0; bb < nb; ++bb)
-            tma_load_2d(dst + bb * kTallBox, &tmG, &full[it % NST],
-                        h * p.dv + NV * part + 64 * (2 * u + bb), t0);
-          ++it;
-        }
-      }
       if (!ok) {
-        mbar_wait_drain(bar_q, 0);
+        // let the copies already issued land before the CTA can exit
+        if (tq > 0) mbar_wait_drain(bar_q, (tq - 1) & 1);
         for (int j = 1; j <= NST && it - j >= 0; ++j) {
           const int i2 = it - j;
           mbar_wait_drain(&full[i2 % NST], (i2 / NST) & 1);
@@ -681,7 +767,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       constexpr uint32_t id_pv = idesc_bf16_f32(128, NV, false, true);
       const uint32_t q_base = smem_u32(smem);
       const uint32_t st_base = smem_u32(smem + C::kOffStages);
-      int it = 0;
+      int it = 0, tq = 0, sblk = 0;
       bool ok = true, issued = false;
       auto stage_wait = [&]() -> uint32_t {
         const int st = it % NST;
@@ -693,65 +779,81 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mma_commit(&empty[it % NST]);
         ++it;
       };
-      ok = mbar_wait(bar_q, 0, abort_flag, p.err);
-      if (ok && need_inter) {
-        // O = Q S_hi + Q S_lo  (the state entering the chunk, split in two bf16 parts)
-        for (int u = 0; u < DK / 64 && ok; ++u) {
-          for (int hl = 0; hl < 2; ++hl) {
-            const uint32_t sb = stage_wait();
-            if (!sb) { ok = false; break; }
+      while (ok && walk.next(p, cid, t)) {
+        const int r = t.r;
+        const uint32_t o_t = tmem + (tq & 1) * C::kHalfCols;          // this tile's O
+        const uint32_t s_t = tmem + ((tq & 1) ^ 1) * C::kHalfCols;    // its score buffers
+        if (!mbar_wait(bar_q, tq & 1, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        if (t.inter) {
+          // O = Q S_hi + Q S_lo  (the state entering the chunk, split in two bf16 parts),
+          // into the half that held the previous tile's scores
+          for (int u = 0; u < DK / 64 && ok; ++u) {
+            for (int hl = 0; hl < 2; ++hl) {
+              const uint32_t sb = stage_wait();
+              if (!sb) { ok = false; break; }
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(tmem + C::kTmemO, sdesc_sw128(q_base + u * kTallBox + kk * 32, 16, 1024),
-                       sdesc_sw128(sb + kk * 2048, kBox, 1024), id_qs, (u | hl | kk) != 0);
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(o_t, sdesc_sw128(q_base + u * kTallBox + kk * 32, 16, 1024),
+                         sdesc_sw128(sb + kk * 2048, kBox, 1024), id_qs, (u | hl | kk) != 0);
+              issued = true;
+              stage_free();
+            }
+          }
+          if (!ok) break;
+          mma_commit(bar_inter);
+        }
+        // the scores go over the previous tile's O: wait until its epilogue has read it
+        if (tq > 0 && !mbar_wait(o_free, (tq - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        auto issue_qk = [&](int kb) -> bool {
+          const uint32_t dst = s_t + 128 * (kb & 1);
+          for (int ku = 0; ku < kKU; ++ku) {
+            const uint32_t sb = stage_wait();
+            if (!sb) return false;
+#pragma unroll
+            for (int kk = 0; kk < 4 * kKB; ++kk) {
+              const int qbox = ku * 2 + kk / 4;
+              mma_bf16(dst, sdesc_sw128(q_base + qbox * kTallBox + (kk & 3) * 32, 16, 1024),
+                       sdesc_sw128(sb + (kk / 4) * kTallBox + (kk & 3) * 32, 16, 1024), id_qk,
+                       (ku | kk) != 0);
+            }
             issued = true;
             stage_free();
           }
-        }
-        if (ok) mma_commit(bar_inter);
-      }
-      auto issue_qk = [&](int kb) -> bool {
-        const uint32_t dst = tmem + ((kb & 1) ? C::kTmemS1 : C::kTmemS0);
-        for (int ku = 0; ku < kKU; ++ku) {
-          const uint32_t sb = stage_wait();
-          if (!sb) return false;
+          mma_commit(&bar_s[(sblk + kb) & 1]);
+          if (kb == r) mma_commit(q_free);     // Q may be replaced by the next tile's
+          return true;
+        };
+        if (!issue_qk(0)) { ok = false; break; }
+        for (int kb = 0; kb <= r && ok; ++kb) {
+          // scores of the next key block go to the other buffer while P_kb is formed
+          if (kb + 1 <= r && !issue_qk(kb + 1)) { ok = false; break; }
+          const int sg = sblk + kb;
+          if (!mbar_wait(&bar_p[sg & 1], (sg >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t pbuf = s_t + 128 * (kb & 1);
+          for (int vu = 0; vu < 2; ++vu) {
+            const uint32_t sb = stage_wait();
+            if (!sb) { ok = false; break; }
 #pragma unroll
-          for (int kk = 0; kk < 4 * kKB; ++kk) {
-            const int qbox = ku * 2 + kk / 4;
-            mma_bf16(dst, sdesc_sw128(q_base + qbox * kTallBox + (kk & 3) * 32, 16, 1024),
-                     sdesc_sw128(sb + (kk / 4) * kTallBox + (kk & 3) * 32, 16, 1024), id_qk,
-                     (ku | kk) != 0);
+            for (int kk = 0; kk < 4; ++kk) {
+              const int ks = vu * 4 + kk;                      // keys 16ks .. 16ks+15
+              const uint32_t a_hi = pbuf + 32 * (ks >> 1) + 8 * (ks & 1);
+              const uint64_t bd = sdesc_sw128(sb + kk * 2048, kBox, 1024);
+              mma_bf16_ts(o_t, a_hi, bd, id_pv, t.inter || kb > 0 || ks > 0);
+              mma_bf16_ts(o_t, a_hi + 16, bd, id_pv, true);
+            }
+            stage_free();
           }
-          issued = true;
-          stage_free();
         }
-        mma_commit(&bar_s[kb & 1]);
-        return true;
-      };
-      if (ok) ok = issue_qk(0);
-      for (int kb = 0; kb <= r && ok; ++kb) {
-        // scores of the next key block go to the other buffer while P_kb is formed
-        if (kb + 1 <= r && !issue_qk(kb + 1)) { ok = false; break; }
-        if (!mbar_wait(&bar_p[kb & 1], (kb >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t pbuf = tmem + ((kb & 1) ? C::kTmemS1 : C::kTmemS0);
-        for (int vu = 0; vu < 2; ++vu) {
-          const uint32_t sb = stage_wait();
-          if (!sb) { ok = false; break; }
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const int ks = vu * 4 + kk;                      // keys 16ks .. 16ks+15
-            const uint32_t a_hi = pbuf + 32 * (ks >> 1) + 8 * (ks & 1);
-            const uint64_t bd = sdesc_sw128(sb + kk * 2048, kBox, 1024);
-            mma_bf16_ts(tmem + C::kTmemO, a_hi, bd, id_pv, need_inter || kb > 0 || ks > 0);
-            mma_bf16_ts(tmem + C::kTmemO, a_hi + 16, bd, id_pv, true);
-          }
-          stage_free();
-        }
-      }
-      if (ok) {
+        if (!ok) break;
         mma_commit(bar_o);
-      } else if (issued) {
+        sblk += r + 1;
+        ++tq;
+        if (io_staged(t)) it += kIoUnits;      // gate/output staging: released by the epilogue
+      }
+      if (!ok && issued) {
         mma_commit(drain);
         mbar_wait_drain(drain, 0);
       }
@@ -762,280 +864,324 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int wg = (warp - 2) >> 2;                   // 0 or 1
     const int quad = warp & 3;
     const int row = quad * 32 + lane;                 // query row within the block
-    const int i = r * kRowsPerTile + row;              // row within the chunk
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const int et = threadIdx.x - 64;                  // 0..255
-    if (et < 128) pow_tab[et] = dec.pow(et);
-    else rev_tab[et - 128] = dec.pow(255 - et);
-    wg2_sync();
-    bool ok = !*abort_flag;
-    const uint32_t o_cols = tmem + lane_off + C::kTmemO + wg * kHalf;
-    if (ok && need_inter) {
-      // tcgen05.ld/st are warp-collective: every guard around them is warp-uniform
-      ok = warp_all(mbar_wait(bar_inter, 0, abort_flag, p.err));
-      if (ok) {
-        tc_fence_after();
-        const float sc = dec.pow(i + 1);
-        for (int j = 0; j < kHalf / 32; ++j) {
-          float x[32];
-          tmem_ld32(o_cols + 32 * j, x);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] *= sc;
-          tmem_st32(o_cols + 32 * j, x);
-        }
-        tmem_wait_st();
-      }
-    }
-    for (int kb = 0; kb <= r && ok; ++kb) {
-      const int sb = kb & 1;
-      if (!warp_all(mbar_wait(&bar_s[sb], (kb >> 1) & 1, abort_flag, p.err))) { ok = false; break; }
-      tc_fence_after();
-      const bool diag = kb == r;
-      // off-diagonal: gamma^(i-j) = gamma^(i - 128kb - 127) * gamma^(127 - j')
-      const float arow = diag ? 0.f : dec.pow(i - kKeysPerBlock * kb - 127);
-      const int key_lim = si.len - kKeysPerBlock * kb;   // keys j' >= key_lim are past the chunk
-      const uint32_t buf = tmem + lane_off + (sb ? C::kTmemS1 : C::kTmemS0);
-#pragma unroll 1
-      for (int j = 2 * wg; j < 2 * wg + 2; ++j) {
-        float x[32];
-        tmem_ld32(buf + 32 * j, x);
-        float wv[32];
-        if (diag) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int jp = 32 * j + e;
-            wv[e] = jp <= row ? pow_tab[row - jp] : 0.f;
-          }
-        } else {
-          const float4* rt = reinterpret_cast<const float4*>(rev_tab + 32 * j);
-          const uint64_t a2 = f2_make(arow, arow);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 t4 = rt[e];
-            const uint64_t w0 = f2_mul(f2_make(t4.x, t4.y), a2);
-            const uint64_t w1 = f2_mul(f2_make(t4.z, t4.w), a2);
-            wv[4 * e] = f2_lo(w0); wv[4 * e + 1] = f2_hi(w0);
-            wv[4 * e + 2] = f2_lo(w1); wv[4 * e + 3] = f2_hi(w1);
-          }
-        }
-        if (key_lim < 32 * j + 32) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (32 * j + e >= key_lim) wv[e] = 0.f;
-        }
-        tmem_wait_ld();
-        float pw[32];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          uint32_t hi, lo;
-          const uint64_t p2 = f2_mul(f2_make(x[e], x[e + 1]), f2_make(wv[e], wv[e + 1]));
-          pack_split(f2_lo(p2), f2_hi(p2), hi, lo);
-          pw[e >> 1] = __uint_as_float(hi);
-          pw[16 + (e >> 1)] = __uint_as_float(lo);
-        }
-        tmem_st32(buf + 32 * j, pw);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bar_p[sb]);
-    }
-    if (ok) ok = mbar_wait(bar_o, 0, abort_flag, p.err);
-    ok = warp_all(ok);
-    if (ok) tc_fence_after();
-    // GroupNorm statistics in one pass: sums of (x - x0) and (x - x0)^2 with
-    // x0 the row's first value in this warpgroup's half (a shift that keeps
-    // the sums well conditioned); halves and parts combine as (mean, M2)
-    // pairs.  Barriers and the exchange with the partner CTA are
-    // unconditional, so an aborted CTA still meets its partner.
-    float mean_all = 0.f, rstd = 0.f;
-    if (p.gated) {
-      float mean_w = 0.f, m2_w = 0.f;
-      if (ok) {
-        uint64_t s1 = 0, s2 = 0;
-        float x0 = 0.f;
-        for (int j = 0; j < kHalf / 32; ++j) {
-          float x[32];
-          tmem_ld32(o_cols + 32 * j, x);
-          tmem_wait_ld();
-          if (j == 0) x0 = x[0];
-          const uint64_t nx0 = f2_make(-x0, -x0);
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const uint64_t d = f2_add(f2_make(x[e], x[e + 1]), nx0);
-            s1 = f2_add(s1, d);
-            s2 = f2_fma(d, d, s2);
-          }
-        }
-        const float S1 = f2_lo(s1) + f2_hi(s1), S2 = f2_lo(s2) + f2_hi(s2);
-        mean_w = x0 + S1 * (1.0f / kHalf);
-        m2_w = fmaxf(S2 - S1 * S1 * (1.0f / kHalf), 0.f);
-      }
-      wg_part[wg * 128 + row] = mean_w;
-      wg_part[256 + wg * 128 + row] = m2_w;
+    const bool wg_leader = (et & 127) == 0;           // first thread of the warpgroup
+    constexpr bool kBoxPerWg = kHalf >= 64;           // each warpgroup owns whole boxes
+    const uint32_t other = xchg ? (cluster_ctarank() ^ 1u) : 0u;
+    int tq = 0, sblk = 0, ninter = 0, eit = 0;
+    bool ok = true;
+    while (walk.next(p, cid, t)) {
+      // uniform over the 256 epilogue threads: the named barriers below stay matched
+      if (!epi_all(ok && !*abort_flag)) break;
+      const int r = t.r;
+      const int i = r * kRowsPerTile + row;            // row within the chunk
+      const uint32_t o_cols = tmem + lane_off + (tq & 1) * C::kHalfCols + wg * kHalf;
+      const uint32_t s_t = tmem + lane_off + ((tq & 1) ^ 1) * C::kHalfCols;
+      const int n_mma = mma_units(t);
+      const bool staged = io_staged(t);
+      auto io_box = [&](int bx) -> uint8_t* {
+        const int unit = eit + n_mma + bx / 2;
+        return smem + C::kOffStages + (unit % NST) * kOutStage + (bx & 1) * kTallBox;
+      };
+      const Decay1 dec(p.dec, t.h);
+      // gamma^d for this tile's head (the previous tile's P is complete: every
+      // epilogue thread passed the barrier in epi_all above after forming it)
+      if (et < 128) pow_tab[et] = dec.pow(et);
       wg2_sync();
-      const float m0 = wg_part[row], m1 = wg_part[128 + row];
-      const float dd = m1 - m0;
-      float mean = 0.5f * (m0 + m1);
-      float m2 = wg_part[256 + row] + wg_part[384 + row] + dd * dd * (0.5f * kHalf);
-      float cnt = static_cast<float>(NV);
-      if (xchg) {
-        // the other d_v part: warpgroup 0 writes this part's (mean, M2) into
-        // the partner's receive buffer and arrives on its barrier
-        cluster_wait();                              // partner's barriers are initialised
-        if (wg == 0) {
-          const uint32_t other = cluster_ctarank() ^ 1u;
-          st_cluster_f32(cluster_addr(&xrecv[2 * row], other), mean);
-          st_cluster_f32(cluster_addr(&xrecv[2 * row + 1], other), m2);
-          mbar_arrive_cluster(cluster_addr(bar_x, other));
-        }
-        cluster_arrive();                            // this CTA's remote accesses are done
-        if (mbar_wait_cluster(bar_x, 0, abort_flag, p.err)) {
-          const float mo = xrecv[2 * row], m2o = xrecv[2 * row + 1];
-          const float d = mo - mean;
-          m2 = m2 + m2o + d * d * (cnt * 0.5f);
-          mean = 0.5f * (mean + mo);
-          cnt *= 2.f;
-        } else {
-          ok = false;
+      if (t.inter) {
+        // tcgen05.ld/st are warp-collective: every guard around them is warp-uniform
+        ok = warp_all(ok && mbar_wait(bar_inter, ninter & 1, abort_flag, p.err));
+        ++ninter;
+        if (ok) {
+          tc_fence_after();
+          const float sc = dec.pow(i + 1);
+          for (int j = 0; j < kHalf / 32; ++j) {
+            float x[32];
+            tmem_ld32(o_cols + 32 * j, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] *= sc;
+            tmem_st32(o_cols + 32 * j, x);
+          }
+          tmem_wait_st();
         }
       }
-      mean_all = mean;
-      rstd = 1.0f / sqrtf(m2 / cnt + p.eps);
-    }
-
-    // ---------------- GroupNorm, gate, store ----------------
-    // Full tiles with a bf16 output go through shared memory (in place of the
-    // gate tile, same swizzled layout) and TMA stores, one per 64-column box
-    // as soon as its warpgroup has written it; partial tiles are written
-    // directly so that no row past the chunk is touched.
-    const bool out_tma = p.y_tma && nrows == kRowsPerTile;
-    constexpr bool kBoxPerWg = kHalf >= 64;          // each warpgroup owns whole boxes
-    const bool wg_leader = ((threadIdx.x - 64) & 127) == 0;   // first thread of the warpgroup
-    const bool live = row < nrows;
-    const int col0 = NV * part + wg * kHalf;          // first d_v column of this warpgroup
-    const size_t obase = (static_cast<size_t>(t0 + row) * p.H + h) * p.dv + col0;
-    const float shift = -mean_all * rstd;
-    bool go = warp_all(ok && !*abort_flag);
-    if (go && p.gated && p.g_tma) {
-      for (int u = 0; u < kIoUnits && go; ++u) {
-        const int unit = n_mma_units + u;
-        go = mbar_wait(&full[unit % NST], (unit / NST) & 1, abort_flag, p.err);
-      }
-      go = warp_all(go);
-    }
-    if (go) tc_fence_after();
-    if (out_tma && wg_leader) tma_prefetch_desc(&tmY);
-    for (int j = 0; j < kHalf / 32; ++j) {
-      // this piece's 32 columns in the staged gate/output box: box, first 16-byte piece
-      const int cpart = wg * kHalf + 32 * j;
-      uint8_t* brow = io_box(cpart >> 6) + row * 128;
-      const int pc0 = (cpart & 63) >> 3;
-      if (go) {
-        float x[32];
-        tmem_ld32(o_cols + 32 * j, x);
-        if (p.gated) {
-          float gv[32];
-          if (p.g_tma) {
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              const uint4 u = *reinterpret_cast<const uint4*>(brow + (((pc0 + c4) ^ (row & 7)) << 4));
-              const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-              for (int q2 = 0; q2 < 4; ++q2) {
-                gv[8 * c4 + 2 * q2] = bf16_lo(wv[q2]);
-                gv[8 * c4 + 2 * q2 + 1] = bf16_hi(wv[q2]);
-              }
-            }
-          } else if (live) {
-            const float4* gp = reinterpret_cast<const float4*>(static_cast<const float*>(p.g) + obase + 32 * j);
-#pragma unroll
-            for (int c4 = 0; c4 < 8; ++c4) {
-              const float4 f = gp[c4];
-              gv[4 * c4] = f.x; gv[4 * c4 + 1] = f.y; gv[4 * c4 + 2] = f.z; gv[4 * c4 + 3] = f.w;
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) gv[e] = 0.f;
-          }
-          tmem_wait_ld();
-          const uint64_t rs2 = f2_make(rstd, rstd), sh2 = f2_make(shift, shift);
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const uint64_t y2 = f2_fma(f2_make(x[e], x[e + 1]), rs2, sh2);
-            x[e] = f2_lo(y2);
-            x[e + 1] = f2_hi(y2);
-          }
-          if (p.gn_w || p.gn_b) {
-            const int c0 = h * p.dv + col0 + 32 * j;
+      for (int kb = 0; kb <= r && ok; ++kb) {
+        const int sg = sblk + kb;
+        if (!warp_all(mbar_wait(&bar_s[sg & 1], (sg >> 1) & 1, abort_flag, p.err))) { ok = false; break; }
+        tc_fence_after();
+        const bool diag = kb == r;
+        // off-diagonal: gamma^(i-j) = gamma^(i - 128kb - 127) * gamma^(127 - j')
+        const float arow = diag ? 0.f : dec.pow(i - kKeysPerBlock * kb - 127);
+        const int key_lim = t.si.len - kKeysPerBlock * kb;   // keys j' >= key_lim are past the chunk
+        const uint32_t buf = s_t + 128 * (kb & 1);
+#pragma unroll 1
+        for (int j = 2 * wg; j < 2 * wg + 2; ++j) {
+          float x[32];
+          tmem_ld32(buf + 32 * j, x);
+          float wv[32];
+          if (diag) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              if (p.gn_w) x[e] *= p.gn_w[c0 + e];
-              if (p.gn_b) x[e] += p.gn_b[c0 + e];
+              const int jp = 32 * j + e;
+              wv[e] = jp <= row ? pow_tab[row - jp] : 0.f;
+            }
+          } else {
+            // gamma^(127 - 32j - e), read as float4 from the table in descending order
+            const uint64_t a2 = f2_make(arow, arow);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+              const float4 t4 = *reinterpret_cast<const float4*>(pow_tab + 124 - 32 * j - 4 * m);
+              const uint64_t w0 = f2_mul(f2_make(t4.w, t4.z), a2);
+              const uint64_t w1 = f2_mul(f2_make(t4.y, t4.x), a2);
+              wv[4 * m] = f2_lo(w0); wv[4 * m + 1] = f2_hi(w0);
+              wv[4 * m + 2] = f2_lo(w1); wv[4 * m + 3] = f2_hi(w1);
             }
           }
-          // swish(g) = g sigmoid(g) = u + u tanh(u) with u = g/2 (sigmoid(g) =
-          // (1 + tanh(g/2))/2): one special-function op per element
-          const uint64_t half2 = f2_make(0.5f, 0.5f);
+          if (key_lim < 32 * j + 32) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (32 * j + e >= key_lim) wv[e] = 0.f;
+          }
+          tmem_wait_ld();
+          float pw[32];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const uint64_t u2 = f2_mul(f2_make(gv[e], gv[e + 1]), half2);
-            const uint64_t s2 = f2_fma(u2, f2_make(tanh_fast(f2_lo(u2)), tanh_fast(f2_hi(u2))), u2);
-            const uint64_t o2 = f2_mul(f2_make(x[e], x[e + 1]), s2);
-            x[e] = f2_lo(o2);
-            x[e + 1] = f2_hi(o2);
+            uint32_t hi, lo;
+            const uint64_t p2 = f2_mul(f2_make(x[e], x[e + 1]), f2_make(wv[e], wv[e + 1]));
+            pack_split(f2_lo(p2), f2_hi(p2), hi, lo);
+            pw[e >> 1] = __uint_as_float(hi);
+            pw[16 + (e >> 1)] = __uint_as_float(lo);
           }
-        } else {
-          tmem_wait_ld();
+          tmem_st32(buf + 32 * j, pw);
         }
-        if (out_tma) {
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar_p[sg & 1]);
+      }
+      sblk += r + 1;
+      ok = warp_all(ok && mbar_wait(bar_o, tq & 1, abort_flag, p.err));
+      if (ok) tc_fence_after();
+      // GroupNorm statistics in one pass: sums of (x - x0) and (x - x0)^2 with
+      // x0 the row's first value in this warpgroup's half (a shift that keeps
+      // the sums well conditioned).  Warpgroup 1 hands its (mean, M2) to
+      // warpgroup 0, which combines the halves, exchanges with the partner
+      // CTA (the other d_v part) and hands back (mean, 1/std).  Barriers and
+      // the exchange are unconditional, so an aborted CTA still meets its
+      // partner.
+      float mean_all = 0.f, rstd = 0.f;
+      if (p.gated) {
+        float mean_w = 0.f, m2_w = 0.f;
+        if (ok) {
+          uint64_t s1 = 0, s2 = 0;
+          float x0 = 0.f;
+          for (int j = 0; j < kHalf / 32; ++j) {
+            float x[32];
+            tmem_ld32(o_cols + 32 * j, x);
+            tmem_wait_ld();
+            if (j == 0) x0 = x[0];
+            const uint64_t nx0 = f2_make(-x0, -x0);
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4)
-            *reinterpret_cast<uint4*>(brow + (((pc0 + c4) ^ (row & 7)) << 4)) =
-                make_uint4(pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]), pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]),
-                           pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]), pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]));
-        } else if (live && p.out_bf16) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + obase + 32 * j);
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4)
-            dst[c4] = make_uint4(pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]), pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]),
-                                 pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]), pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]));
-        } else if (live) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + 32 * j);
-#pragma unroll
-          for (int c4 = 0; c4 < 8; ++c4)
-            dst[c4] = make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
+            for (int e = 0; e < 32; e += 2) {
+              const uint64_t d = f2_add(f2_make(x[e], x[e + 1]), nx0);
+              s1 = f2_add(s1, d);
+              s2 = f2_fma(d, d, s2);
+            }
+          }
+          const float S1 = f2_lo(s1) + f2_hi(s1), S2 = f2_lo(s2) + f2_hi(s2);
+          mean_w = x0 + S1 * (1.0f / kHalf);
+          m2_w = fmaxf(S2 - S1 * S1 * (1.0f / kHalf), 0.f);
+        }
+        if (wg == 1) {
+          wgx[2 * row] = mean_w;
+          wgx[2 * row + 1] = m2_w;
+        }
+        wg2_sync();
+        if (wg == 0) {
+          const float m1 = wgx[2 * row], m21 = wgx[2 * row + 1];
+          const float dd = m1 - mean_w;
+          float mean = 0.5f * (mean_w + m1);
+          float m2 = m2_w + m21 + dd * dd * (0.5f * kHalf);
+          float cnt = static_cast<float>(NV);
+          if (xchg) {
+            // the other d_v part: write this part's (mean, M2) into the
+            // partner's receive buffer once it has read the previous pair,
+            // arrive on its barrier, then read the partner's pair and release
+            // this CTA's receive buffer
+            if (!cluster_waited) {
+              cluster_wait();                        // partner's barriers are initialised
+              cluster_waited = true;
+            }
+            bool xok = tq == 0 || mbar_wait_cluster(bar_xack, (tq - 1) & 1, abort_flag, p.err);
+            if (xok) {
+              st_cluster_f32(cluster_addr(&xrecv[2 * row], other), mean);
+              st_cluster_f32(cluster_addr(&xrecv[2 * row + 1], other), m2);
+            }
+            mbar_arrive_cluster(cluster_addr(bar_x, other));
+            xok = mbar_wait_cluster(bar_x, tq & 1, abort_flag, p.err) && xok;
+            if (xok) {
+              const float mo = xrecv[2 * row], m2o = xrecv[2 * row + 1];
+              const float d = mo - mean;
+              m2 = m2 + m2o + d * d * (cnt * 0.5f);
+              mean = 0.5f * (mean + mo);
+              cnt *= 2.f;
+            } else {
+              ok = false;
+            }
+            mbar_arrive_cluster(cluster_addr(bar_xack, other));
+          }
+          mean_all = mean;
+          rstd = 1.0f / sqrtf(m2 / cnt + p.eps);
+          wgx[2 * row] = mean_all;
+          wgx[2 * row + 1] = rstd;
+        }
+        wg2_sync();
+        if (wg == 1) {
+          mean_all = wgx[2 * row];
+          rstd = wgx[2 * row + 1];
         }
       }
-      if (kBoxPerWg && out_tma && (j & 1)) {       // uniform over the warpgroup
-        // box cpart/64 is complete: hand it to the TMA engine
+
+      // ---------------- GroupNorm, gate, store ----------------
+      // Full tiles with a bf16 output go through shared memory (in place of the
+      // gate tile, same swizzled layout) and TMA stores, one per 64-column box
+      // as soon as its warpgroup has written it; partial tiles are written
+      // directly so that no row past the chunk is touched.
+      const bool out_tma = p.y_tma && t.nrows == kRowsPerTile;
+      const bool live = row < t.nrows;
+      const int col0 = NV * part + wg * kHalf;          // first d_v column of this warpgroup
+      const size_t obase = (static_cast<size_t>(t.t0 + row) * p.H + t.h) * p.dv + col0;
+      const float shift = -mean_all * rstd;
+      bool go = warp_all(ok && !*abort_flag);
+      if (go && staged) {
+        for (int u = 0; u < kIoUnits && go; ++u) {
+          const int unit = eit + n_mma + u;
+          go = mbar_wait(&full[unit % NST], (unit / NST) & 1, abort_flag, p.err);
+        }
+        go = warp_all(go);
+      }
+      if (go) tc_fence_after();
+      for (int j = 0; j < kHalf / 32; ++j) {
+        // this piece's 32 columns in the staged gate/output box: box, first 16-byte piece
+        const int cpart = wg * kHalf + 32 * j;
+        uint8_t* brow = io_box(cpart >> 6) + row * 128;
+        const int pc0 = (cpart & 63) >> 3;
+        if (go) {
+          float x[32];
+          tmem_ld32(o_cols + 32 * j, x);
+          if (p.gated) {
+            float gv[32];
+            if (p.g_tma) {
+#pragma unroll
+              for (int c4 = 0; c4 < 4; ++c4) {
+                const uint4 u = *reinterpret_cast<const uint4*>(brow + (((pc0 + c4) ^ (row & 7)) << 4));
+                const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) {
+                  gv[8 * c4 + 2 * q2] = bf16_lo(wv[q2]);
+                  gv[8 * c4 + 2 * q2 + 1] = bf16_hi(wv[q2]);
+                }
+              }
+            } else if (live) {
+              const float4* gp = reinterpret_cast<const float4*>(static_cast<const float*>(p.g) + obase + 32 * j);
+#pragma unroll
+              for (int c4 = 0; c4 < 8; ++c4) {
+                const float4 f = gp[c4];
+                gv[4 * c4] = f.x; gv[4 * c4 + 1] = f.y; gv[4 * c4 + 2] = f.z; gv[4 * c4 + 3] = f.w;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) gv[e] = 0.f;
+            }
+            tmem_wait_ld();
+            const uint64_t rs2 = f2_make(rstd, rstd), sh2 = f2_make(shift, shift);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const uint64_t y2 = f2_fma(f2_make(x[e], x[e + 1]), rs2, sh2);
+              x[e] = f2_lo(y2);
+              x[e + 1] = f2_hi(y2);
+            }
+            if (p.gn_w || p.gn_b) {
+              const int c0 = t.h * p.dv + col0 + 32 * j;
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                if (p.gn_w) x[e] *= p.gn_w[c0 + e];
+                if (p.gn_b) x[e] += p.gn_b[c0 + e];
+              }
+            }
+            // swish(g) = g sigmoid(g) = u + u tanh(u) with u = g/2 (sigmoid(g) =
+            // (1 + tanh(g/2))/2): one special-function op per element
+            const uint64_t half2 = f2_make(0.5f, 0.5f);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const uint64_t u2 = f2_mul(f2_make(gv[e], gv[e + 1]), half2);
+              const uint64_t s2 = f2_fma(u2, f2_make(tanh_fast(f2_lo(u2)), tanh_fast(f2_hi(u2))), u2);
+              const uint64_t o2 = f2_mul(f2_make(x[e], x[e + 1]), s2);
+              x[e] = f2_lo(o2);
+              x[e + 1] = f2_hi(o2);
+            }
+          } else {
+            tmem_wait_ld();
+          }
+          if (out_tma) {
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+              *reinterpret_cast<uint4*>(brow + (((pc0 + c4) ^ (row & 7)) << 4)) =
+                  make_uint4(pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]), pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]),
+                             pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]), pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]));
+          } else if (live && p.out_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + obase + 32 * j);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+              dst[c4] = make_uint4(pack_bf16(x[8 * c4 + 0], x[8 * c4 + 1]), pack_bf16(x[8 * c4 + 2], x[8 * c4 + 3]),
+                                   pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]), pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]));
+          } else if (live) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + 32 * j);
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4)
+              dst[c4] = make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
+          }
+        }
+        if (kBoxPerWg && out_tma && (j & 1)) {       // uniform over the warpgroup
+          // box cpart/64 is complete: hand it to the TMA engine
+          fence_proxy_async_smem();
+          wg_sync(wg);
+          if (wg_leader && go) {
+            tma_store_2d(&tmY, io_box(cpart >> 6), t.h * p.dv + NV * part + 64 * (cpart >> 6), t.t0);
+            tma_store_commit();
+          }
+        }
+      }
+      // every read of this tile's O is complete: its TMEM half may take the
+      // next tile's scores
+      tc_fence_before();
+      mbar_arrive(o_free);
+      if (!kBoxPerWg && out_tma) {                   // boxes shared by both warpgroups
         fence_proxy_async_smem();
-        wg_sync(wg);
-        if (wg_leader && go) {
-          tma_store_2d(&tmY, io_box(cpart >> 6), h * p.dv + NV * part + 64 * (cpart >> 6), t0);
+        wg2_sync();
+        if (et == 0 && go) {
+          for (int bx = 0; bx < kIoBoxes; ++bx)
+            tma_store_2d(&tmY, io_box(bx), t.h * p.dv + NV * part + 64 * bx, t.t0);
           tma_store_commit();
         }
       }
-    }
-    if (!kBoxPerWg && out_tma) {                   // boxes shared by both warpgroups
-      fence_proxy_async_smem();
-      wg2_sync();
-      if (threadIdx.x == 64 && go) {
-        for (int bx = 0; bx < kIoBoxes; ++bx)
-          tma_store_2d(&tmY, io_box(bx), h * p.dv + NV * part + 64 * bx, t0);
-        tma_store_commit();
+      // the staging units go back to the producer once the stores have read
+      // them (the global writes complete on their own)
+      if (out_tma && go && (kBoxPerWg ? wg_leader : et == 0)) tma_store_wait_read();
+      if (staged) {
+        wg2_sync();
+        if (et == 0)
+          for (int u = 0; u < kIoUnits; ++u) mbar_arrive(&empty[(eit + n_mma + u) % NST]);
       }
+      eit += n_mma + (staged ? kIoUnits : 0);
+      ++tq;
     }
-    // shared memory may be released once the stores have read it; the
-    // global writes complete on their own
-    if (out_tma && go && (kBoxPerWg ? wg_leader : threadIdx.x == 64)) tma_store_wait_read();
   }
   if (xchg) {
-    if (warp < 2) {
-      cluster_wait();
-      cluster_arrive();
-    }
-    cluster_wait();        // the partner has written its statistics: no more remote access here
+    if (!cluster_waited) cluster_wait();
+    cluster_arrive();
+    cluster_wait();        // the partner has made its last remote access here
   }
   tc_fence_before();
   __syncthreads();
@@ -1583,7 +1729,7 @@ cudaError_t launch_state(const CUtensorMap& mk, const CUtensorMap& mv, const CUt
 template <int DK, int NV>
 cudaError_t launch_out(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const CUtensorMap& ms, const CUtensorMap& mg, const CUtensorMap& my,
-                       const OutParams& op, long long units, cudaStream_t s) {
+                       OutParams op, cudaStream_t s) {
   using C = OutCfg<DK, NV>;
   static_assert(C::kSmem <= 232448, "shared memory budget");
   auto kern = output_kernel<DK, NV>;
@@ -1591,7 +1737,6 @@ cudaError_t launch_out(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(units * op.parts), op.H, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = s;
@@ -1602,6 +1747,26 @@ cudaError_t launch_out(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // persistent grid: as many clusters as can be resident at once (one CTA
+  // per SM), queried once per device and cluster size
+  static int resident[64][3] = {};
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int& ncl = resident[dev & 63][op.parts];
+  if (ncl == 0) {
+    cfg.gridDim = dim3(static_cast<unsigned>(op.parts), 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+      (void)cudaGetLastError();
+      n = sm_count() / op.parts;
+    }
+    ncl = n > 0 ? n : 1;
+  }
+  op.nclusters = op.ntiles < ncl ? op.ntiles : ncl;
+  // rotate the row block every round (an odd stride through the rb row blocks)
+  op.shift = (op.nclusters % 2 == 0) ? 1 : 2;
+  cfg.gridDim = dim3(static_cast<unsigned>(op.nclusters * op.parts), 1, 1);
   return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ms, mg, my, op);
 }
 
@@ -1742,7 +1907,12 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
   if ((op.g_tma && !make_map(&mg, g, hdv, Ttot, hdv, 128)) ||
       (op.y_tma && !make_map(&my, out, hdv, Ttot, hdv, 128)))
     return cudaErrorInvalidValue;
-  const long long units = ws.nslots * op.rb;
+  const long long ntiles = static_cast<long long>(ws.nslots) * H * op.rb;
+  if (ntiles >= (1ll << 31)) return cudaErrorInvalidValue;
+  op.ntiles = static_cast<int>(ntiles);
+  op.nch = (L.T + L.chunk - 1) / L.chunk;
+  op.nclusters = 1;
+  op.shift = 1;
   if (op.rb == 1 && dk <= 128 && dv <= 256) {
     // one-block chunks: the compact kernel, two CTAs per SM, d_v in parts of <= 128
     op.parts = dv > 128 ? 2 : 1;
@@ -1760,22 +1930,22 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
   }
   if (dk == 64) {
     switch (NV) {
-      case 64: return launch_out<64, 64>(mq, mk, mv, ms, mg, my, op, units, s);
-      case 128: return launch_out<64, 128>(mq, mk, mv, ms, mg, my, op, units, s);
-      default: return launch_out<64, 256>(mq, mk, mv, ms, mg, my, op, units, s);
+      case 64: return launch_out<64, 64>(mq, mk, mv, ms, mg, my, op, s);
+      case 128: return launch_out<64, 128>(mq, mk, mv, ms, mg, my, op, s);
+      default: return launch_out<64, 256>(mq, mk, mv, ms, mg, my, op, s);
     }
   }
   if (dk == 128) {
     switch (NV) {
-      case 64: return launch_out<128, 64>(mq, mk, mv, ms, mg, my, op, units, s);
-      case 128: return launch_out<128, 128>(mq, mk, mv, ms, mg, my, op, units, s);
-      default: return launch_out<128, 256>(mq, mk, mv, ms, mg, my, op, units, s);
+      case 64: return launch_out<128, 64>(mq, mk, mv, ms, mg, my, op, s);
+      case 128: return launch_out<128, 128>(mq, mk, mv, ms, mg, my, op, s);
+      default: return launch_out<128, 256>(mq, mk, mv, ms, mg, my, op, s);
     }
   }
   switch (NV) {
-    case 64: return launch_out<256, 64>(mq, mk, mv, ms, mg, my, op, units, s);
-    case 128: return launch_out<256, 128>(mq, mk, mv, ms, mg, my, op, units, s);
-    default: return launch_out<256, 256>(mq, mk, mv, ms, mg, my, op, units, s);
+    case 64: return launch_out<256, 64>(mq, mk, mv, ms, mg, my, op, s);
+    case 128: return launch_out<256, 128>(mq, mk, mv, ms, mg, my, op, s);
+    default: return launch_out<256, 256>(mq, mk, mv, ms, mg, my, op, s);
   }
 }
 
