@@ -167,8 +167,9 @@ RET_API size_t retention_chunkwise_workspace_size(ret_dtype in_dtype, int chunk,
  *   in_dtype RET_BF16: tensor-core kernels (tcgen05, TMEM accumulators), dk in
  *          {64, 128, 256}, dv in {64, 128, 256, 512}, chunk in
  *          {64, 128, 256, 512}; other bf16 shapes return
- *          RET_ERR_UNSUPPORTED.  Chunks shorter than 128 tokens are
- *          evaluated as 128-token chunks, which yields the same result.
+ *          RET_ERR_UNSUPPORTED.  Chunks shorter than 128 tokens (256
+ *          when dv >= 256) are evaluated as chunks of that length, which
+ *          yields the same result.
  *   out dtype RET_F32 or RET_BF16; H <= 64; T*H*max(dk,dv) < 2^31.
  */
 RET_API ret_status retention_chunkwise_fwd(const void* q, const void* k, const void* v,

@@ -87,7 +87,7 @@ ret_status plan_chunkwise(ret_dtype in_dtype, int chunk, int B, int T, int H, in
   int ce = chunk;
   if (in_dtype == RET_BF16) {
     if (!ret::chunkwise_tc_supported(dk, dv, chunk)) return RET_ERR_UNSUPPORTED;
-    ce = ret::chunkwise_tc_chunk(chunk);
+    ce = ret::chunkwise_tc_chunk(chunk, dv);
     p->tc = true;
     p->elem = 4;   // two bf16 planes per state element (hi and lo parts)
   } else {

@@ -1825,7 +1825,15 @@ bool chunkwise_tc_supported(int dk, int dv, int chunk) {
   return dk_ok && dv_ok && c_ok;
 }
 
-int chunkwise_tc_chunk(int chunk) { return chunk < 128 ? 128 : chunk; }
+// Chunk length the tensor-core kernels evaluate.  Every chunk length gives the
+// same result (the chunkwise form splits the same sum at different points), so
+// short chunks run as longer ones: at least one 128-row block, and at least 256
+// tokens when d_v >= 256, where the per-chunk state (d_k x d_v) would otherwise
+// cost as much workspace traffic as the chunk's own inputs.
+int chunkwise_tc_chunk(int chunk, int dv) {
+  const int lo = dv >= 256 ? 256 : 128;
+  return chunk < lo ? lo : chunk;
+}
 
 cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const void* v,
                                 const SeqLayout& L, const float* state_in, bool has_state_in,

@@ -61,7 +61,7 @@ bool chunkwise_tc_supported(int dk, int dv, int chunk);
 
 // One bounded wait that is never satisfied (failure-detection self-test).
 cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t s);
-int chunkwise_tc_chunk(int chunk);  // chunk length the kernels evaluate
+int chunkwise_tc_chunk(int chunk, int dv);  // chunk length the kernels evaluate
 cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const void* v,
                                 const SeqLayout& L, const float* state_in, bool has_state_in,
                                 float* state_out,
