@@ -78,6 +78,9 @@ __all__ = [
     "msr_chunkwise",
     "msr_chunkwise_varlen",
     "msr_recurrent_step",
+    "retention_backward",
+    "msr_backward",
+    "msr_backward_varlen",
 ]
 
 
@@ -318,3 +321,94 @@ def msr_recurrent_step(q, k, v, gamma, state):
         for h in range(H):
             o[n, h], S_new[n, h] = recurrent_step(q[n, h], k[n, h], v[n, h], gamma[h], S[n, h])
     return o, S_new
+
+
+# ---------------------------------------------------------------------------
+# Backward: gradients of the definition (what training in the parallel form
+# needs; the pages give the forward only)
+# ---------------------------------------------------------------------------
+
+def retention_backward(q, k, v, gamma, d_out, state=None, d_state=None):
+    """Gradients of one head with respect to q, k, v and the initial state.
+
+    The forward is the definition started from an initial state S0 (the
+    recurrent form of [RetNet-JA] 「学習は並列、生成は状態更新」 run from S0):
+        o_n = sum_{m<=n} gamma^(n-m) (q_n . k_m) v_m + gamma^(n+1) q_n S0
+        S_T = gamma^T S0 + sum_m gamma^(T-1-m) k_m^T v_m
+    For L = <d_out, o> + <d_state, S_T> the gradients, written with the decay
+    mask D of the parallel form, are
+        dQ  = ((dO V^T) * D) K         + diag(gamma^(n+1)) dO S0^T
+        dK  = ((dO V^T) * D)^T Q       + diag(gamma^(T-1-m)) V dS_T^T
+        dV  = ((Q K^T) * D)^T dO       + diag(gamma^(T-1-m)) K dS_T
+        dS0 = Q^T diag(gamma^(n+1)) dO + gamma^T dS_T
+    ``state`` / ``d_state`` of None mean zero.  Returns
+    ``(dq [T,dk], dk [T,dk], dv [T,dv], d_state_in [dk,dv])``.
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(d_out)
+    T, dk, dv = q.shape[0], q.shape[1], v.shape[1]
+    gamma = float(gamma)
+    D = decay_mask(gamma, T)
+    A = (do @ v.T) * D                                  # gamma^(n-m) (do_n . v_m)
+    P = (q @ k.T) * D                                   # gamma^(n-m) (q_n . k_m)
+    dq = A @ k
+    dk_ = A.T @ q
+    dv_ = P.T @ do
+    g_in = np.power(gamma, np.arange(1, T + 1))         # gamma^(n+1)
+    g_out = np.power(gamma, np.arange(T - 1, -1, -1))   # gamma^(T-1-m)
+    dS0 = q.T @ (g_in[:, None] * do)
+    if state is not None:
+        dq = dq + g_in[:, None] * (do @ _f64(state).T)
+    if d_state is not None:
+        dS = _f64(d_state)
+        dk_ = dk_ + g_out[:, None] * (v @ dS.T)
+        dv_ = dv_ + g_out[:, None] * (k @ dS)
+        dS0 = dS0 + (gamma ** T) * dS
+    return dq, dk_, dv_, dS0
+
+
+def msr_backward(q, k, v, gamma, d_out, state=None, d_state=None):
+    """``retention_backward`` for every (batch, head) in the boundary layout
+    ``[B, T, H, d]``; ``state``, ``d_state``: ``[B, H, dk, dv]`` or None.
+    Returns ``(dq, dk, dv, d_state_in [B, H, dk, dv])``."""
+    q, k, v, gamma = _heads(q, k, v, gamma)
+    do = _f64(d_out)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    dq, dkk, dvv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
+    dS0 = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            dq[b, :, h], dkk[b, :, h], dvv[b, :, h], dS0[b, h] = retention_backward(
+                q[b, :, h], k[b, :, h], v[b, :, h], gamma[h], do[b, :, h],
+                None if state is None else state[b, h],
+                None if d_state is None else d_state[b, h])
+    return dq, dkk, dvv, dS0
+
+
+def msr_backward_varlen(q, k, v, gamma, d_out, cu_seqlens, state=None, d_state=None,
+                        heads=None):
+    """Packed variable-length batch (``B = 1``, sequences at ``cu_seqlens``):
+    every sequence is differentiated on its own (reading 9).  ``state``,
+    ``d_state``: ``[nseq, H, dk, dv]`` or None; an empty sequence passes
+    ``d_state`` straight to its ``d_state_in``.  ``heads`` optionally restricts
+    the work to a list of heads."""
+    q, k, v, gamma = _heads(q, k, v, gamma)
+    do = _f64(d_out)
+    cu = [int(x) for x in cu_seqlens]
+    nseq = len(cu) - 1
+    _, T, H, dk = q.shape
+    dv = v.shape[3]
+    dq, dkk, dvv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
+    dS0 = np.zeros((nseq, H, dk, dv))
+    hs = range(H) if heads is None else heads
+    for i in range(nseq):
+        a, b = cu[i], cu[i + 1]
+        for h in hs:
+            s0 = None if state is None else state[i, h]
+            dS = None if d_state is None else d_state[i, h]
+            if b > a:
+                dq[0, a:b, h], dkk[0, a:b, h], dvv[0, a:b, h], dS0[i, h] = retention_backward(
+                    q[0, a:b, h], k[0, a:b, h], v[0, a:b, h], gamma[h], do[0, a:b, h], s0, dS)
+            else:
+                dS0[i, h] = 0.0 if dS is None else _f64(dS)
+    return dq, dkk, dvv, dS0
