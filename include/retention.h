@@ -290,6 +290,47 @@ RET_API ret_status retention_recurrent_steps(const void* q, const void* k, const
                                              ret_stream_t stream);
 
 /*
+ * Backward of the chunkwise form: the gradients for training in the parallel
+ * form (eulerwa.com tutorial "3. RetNet 상세", section "장점"; the pages state
+ * the forward only, these are its derivatives).  For each sequence and head,
+ * with the forward started from S0 = state_in (zero if NULL),
+ *     o_n = sum_{m<=n} gamma^(n-m) (q_n . k_m) v_m + gamma^(n+1) q_n S0
+ *     S_T = gamma^T S0 + sum_m gamma^(T-1-m) k_m^T v_m
+ * and upstream gradients dO = d_out and dS_T = d_state_out (zero if NULL):
+ *     dq_n = sum_{m<=n} gamma^(n-m) (dO_n . v_m) k_m + gamma^(n+1) dO_n S0^T
+ *     dk_m = sum_{n>=m} gamma^(n-m) (dO_n . v_m) q_n + gamma^(T-1-m) v_m dS_T^T
+ *     dv_m = sum_{n>=m} gamma^(n-m) (q_n . k_m) dO_n + gamma^(T-1-m) k_m dS_T
+ *     dS0  = sum_n gamma^(n+1) q_n^T dO_n + gamma^T dS_T      (-> d_state_in)
+ * evaluated chunk by chunk (`chunk` tokens; any length gives the same values):
+ * a forward pass over the chunks carries S, a backward pass carries the state
+ * of everything after each chunk.  This is the gradient of the raw retention
+ * output o; the GroupNorm and gate, when used, are differentiated by the caller.
+ *   q, k: [B,T,H,dk] in_dtype   v, d_out: [B,T,H,dv] in_dtype (same layout and
+ *   packing as retention_chunkwise_fwd, incl. cu_seqlens/nseq)
+ *   state_in, d_state_out: [nseq|B,H,dk,dv] float32 or NULL
+ *   dq, dk: [B,T,H,dk] float32   dv: [B,T,H,dv] float32   (written in full)
+ *   d_state_in: [nseq|B,H,dk,dv] float32 or NULL (not emitted)
+ *   workspace: caller-owned device buffer, 256-byte aligned, at least
+ *     retention_chunkwise_bwd_workspace_size(...) bytes (chunk offsets and two
+ *     float32 states per chunk); RET_ERR_WORKSPACE otherwise.
+ * Supported: in_dtype RET_F32 or RET_BF16, dk and dv in 1..256, any chunk >= 1;
+ * every product and sum is float32 on CUDA cores (bf16 inputs are widened
+ * exactly).  Larger heads return RET_ERR_UNSUPPORTED.  The workspace size query
+ * returns 0 for arguments the call would reject.
+ */
+RET_API size_t retention_chunkwise_bwd_workspace_size(ret_dtype in_dtype, int chunk, int B,
+                                                      int T, int H, int dk, int dv, int nseq);
+RET_API ret_status retention_chunkwise_bwd(const void* q, const void* k, const void* v,
+                                           const void* d_out, ret_dtype in_dtype,
+                                           const double* gamma, int chunk,
+                                           const int32_t* cu_seqlens, int nseq,
+                                           const float* state_in, const float* d_state_out,
+                                           float* dq, float* dk, float* dv, float* d_state_in,
+                                           void* workspace, size_t workspace_bytes,
+                                           int B, int T, int H, int dk_, int dv_,
+                                           ret_stream_t stream);
+
+/*
  * Standalone per-head GroupNorm + Swish gate (the epilogue that
  * retention_chunkwise_fwd fuses when given `ng`).
  *   o: [ntok, H, dv] o_dtype     y: [ntok, H, dv] y_dtype (may not alias o)

@@ -341,6 +341,104 @@ ret_status msr_norm_gate(const void* o, ret_dtype o_dtype, const ret_norm_gate* 
                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 
+}  // extern "C"
+
+namespace {
+
+struct BwdPlan {
+  ret::SeqLayout L;
+  size_t meta;
+  long long slots;
+  size_t state_bytes;   // one set of per-chunk states
+  size_t bytes;
+};
+
+// Shared by the backward's size query and call: every supported shape runs on
+// CUDA cores in float32 (bf16 inputs are read exactly and widened).
+ret_status plan_chunkwise_bwd(ret_dtype in_dtype, int chunk, int B, int T, int H, int dk, int dv,
+                              int nseq, const int32_t* cu, BwdPlan* p) {
+  if (!dtype_ok(in_dtype) || chunk < 1 || H < 1 || H > ret::kMaxHeads || dk < 1 || dv < 1 ||
+      nseq < 0)
+    return RET_ERR_INVALID_ARG;
+  const bool varlen = nseq > 0;
+  if (varlen) {
+    if (B != 1 || T < 0) return RET_ERR_INVALID_ARG;
+  } else if (B < 1 || T < 1) {
+    return RET_ERR_INVALID_ARG;
+  }
+  const long long Ttot = varlen ? T : static_cast<long long>(B) * T;
+  const int dmax = dk > dv ? dk : dv;
+  if (!fits_int(Ttot * H * static_cast<long long>(dmax)) || !fits_int(Ttot + chunk))
+    return RET_ERR_INVALID_ARG;
+  if (dk > 256 || dv > 256) return RET_ERR_UNSUPPORTED;
+  p->L.cu = varlen ? cu : nullptr;
+  p->L.nseq = varlen ? nseq : B;
+  p->L.T = varlen ? 0 : T;
+  p->L.Ttot = static_cast<int>(Ttot);
+  p->L.chunk = chunk;
+  p->meta = ret::chunkwise_meta_bytes(p->L.nseq);
+  p->slots = varlen ? (Ttot + chunk - 1) / chunk + nseq
+                    : static_cast<long long>(B) * ((T + chunk - 1) / chunk);
+  p->L.nslots = p->slots;
+  p->state_bytes = static_cast<size_t>(p->slots) * H * dk * dv * sizeof(float);
+  p->bytes = p->meta + 2 * p->state_bytes;
+  return RET_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t retention_chunkwise_bwd_workspace_size(ret_dtype in_dtype, int chunk, int B, int T,
+                                              int H, int dk, int dv, int nseq) {
+  BwdPlan p;
+  if (plan_chunkwise_bwd(in_dtype, chunk, B, T, H, dk, dv, nseq, nullptr, &p) != RET_OK) return 0;
+  return p.bytes;
+}
+
+ret_status retention_chunkwise_bwd(const void* q, const void* k, const void* v, const void* d_out,
+                                   ret_dtype in_dtype, const double* gamma, int chunk,
+                                   const int32_t* cu_seqlens, int nseq, const float* state_in,
+                                   const float* d_state_out, float* dq, float* dk, float* dv,
+                                   float* d_state_in, void* workspace, size_t workspace_bytes,
+                                   int B, int T, int H, int dk_, int dv_, ret_stream_t stream) {
+  const bool varlen = cu_seqlens != nullptr;
+  if (varlen != (nseq > 0)) return RET_ERR_INVALID_ARG;
+  BwdPlan p;
+  ret_status st = plan_chunkwise_bwd(in_dtype, chunk, B, T, H, dk_, dv_, varlen ? nseq : 0,
+                                     cu_seqlens, &p);
+  if (st != RET_OK) return st;
+  if (p.L.Ttot > 0 && (!q || !k || !v || !d_out || !dq || !dk || !dv)) return RET_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, d_out, dq, dk, dv, state_in, d_state_out, d_state_in, cu_seqlens};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return RET_ERR_INVALID_ARG;
+  ret::HeadDecay dec;
+  if (!make_decay(gamma, H, &dec)) return RET_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < p.bytes)
+    return RET_ERR_WORKSPACE;
+  unsigned* err = error_word();
+  if (!err) return RET_ERR_CUDA;
+  char* base = static_cast<char*>(workspace);
+  ret::ChunkWorkspace fw;
+  fw.chunk_base = reinterpret_cast<int32_t*>(base);
+  fw.order = fw.chunk_base + p.L.nseq + 1;
+  fw.states = base + p.meta;
+  fw.nslots = p.slots;
+  ret::ChunkBwdWorkspace ws;
+  ws.chunk_base = fw.chunk_base;
+  ws.order = fw.order;
+  ws.fwd_states = reinterpret_cast<float*>(base + p.meta);
+  ws.bwd_states = reinterpret_cast<float*>(base + p.meta + p.state_bytes);
+  ws.nslots = p.slots;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = ret::launch_chunk_prep(p.L, fw, err, s);
+  if (e == cudaSuccess)
+    e = ret::launch_chunkwise_bwd_simt(q, k, v, d_out, dt(in_dtype), p.L, state_in, d_state_out,
+                                       dq, dk, dv, d_state_in, ws, H, dk_, dv_, dec, s);
+  return cuda_status(e);
+}
+
 ret_status retention_selftest_wait_timeout(ret_stream_t stream) {
   unsigned* err = error_word();
   if (!err) return RET_ERR_CUDA;

@@ -15,8 +15,9 @@ enum class DType { F32 = 0, BF16 = 1 };
 // Workspace layout of the chunkwise forward:
 //   [meta: chunk_base int32[nseq+1], rounded up to 256 B][states]
 // states hold the state entering every chunk, one slot per chunk:
-//   [slot][H][dk][dv], float32 on the CUDA-core path and float16 (the MMA
-//   operand of the cross-chunk read) on the tensor-core path.
+//   [slot][H][dk][dv], float32 on the CUDA-core path; on the tensor-core path
+//   [slot][H][2][dk][dv] bf16, the hi and lo parts of the state (the MMA
+//   operands of the cross-chunk read).
 struct ChunkWorkspace {
   int32_t* chunk_base;   // device, nseq+1 entries (varlen only; else unused)
   int32_t* order;        // device, nseq entries: sequences longest first (varlen only)
@@ -43,6 +44,24 @@ cudaError_t launch_chunkwise_simt(int phases, const void* q, const void* k, cons
                                   const float* gn_w, const float* gn_b, float eps, bool gated,
                                   ChunkWorkspace ws, int H, int dk, int dv,
                                   const HeadDecay& dec, unsigned* err, cudaStream_t s);
+
+// Workspace of the chunkwise backward: [meta as above][forward states][backward
+// states], both [slot][H][dk][dv] float32.
+struct ChunkBwdWorkspace {
+  int32_t* chunk_base;   // device, nseq+1 entries (varlen only)
+  int32_t* order;        // device, nseq entries (varlen only)
+  float* fwd_states;     // state entering each chunk
+  float* bwd_states;     // gradient state of everything after each chunk
+  long long nslots;
+};
+
+// CUDA-core backward of the chunkwise form (f32 or bf16 inputs, f32 gradients).
+cudaError_t launch_chunkwise_bwd_simt(const void* q, const void* k, const void* v,
+                                      const void* d_out, DType in_t, const SeqLayout& L,
+                                      const float* state_in, const float* d_state_out, float* dq,
+                                      float* dk, float* dv, float* d_state_in,
+                                      const ChunkBwdWorkspace& ws, int H, int dk_, int dv_,
+                                      const HeadDecay& dec, cudaStream_t s);
 
 // Tn (1..16) tokens per sequence in one pass over the state.
 cudaError_t launch_decode_steps(const void* q, const void* k, const void* v, DType in_t,

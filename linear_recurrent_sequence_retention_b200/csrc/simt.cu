@@ -174,11 +174,15 @@ __device__ __forceinline__ long long slot_of(const SeqLayout& L, const int32_t* 
 // Walks the sequence's chunks in order; before each chunk it stores the state
 // entering it (S_prev) in the workspace, then applies
 //     S <- gamma^L S + sum_j gamma^(L-1-j) k_j^T v_j.
+// With kRev the chunks are walked from the last to the first and the update is
+//     F <- gamma^L F + sum_j gamma^(j+1) k_j^T v_j
+// (the backward's state of the future, called with k = q and v = dO): the
+// value stored for chunk c is then the state of everything after it.
 // Lane = column, warp w owns state rows w, w+8, ... (dk <= 256 -> 32 rows).
 // ---------------------------------------------------------------------------
 constexpr int kStateTok = 32;
 
-template <typename Tin>
+template <typename Tin, bool kRev>
 __global__ void __launch_bounds__(kThreads)
 chunk_state_simt_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, SeqLayout L,
                         const int32_t* __restrict__ chunk_base,
@@ -203,7 +207,8 @@ chunk_state_simt_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, Se
                ? state_in[((static_cast<size_t>(s) * H + h) * dk + i) * dv + col] : 0.f;
   }
   const int nch = ceil_div(len, L.chunk);
-  for (int c = 0; c < nch; ++c) {
+  for (int cc = 0; cc < nch; ++cc) {
+    const int c = kRev ? nch - 1 - cc : cc;
     const long long slot = slot_of(L, chunk_base, s, c);
     if (slot >= 0 && slot < L.nslots) {
       float* dst = ws_states + (static_cast<size_t>(slot) * H + h) * dk * dv;
@@ -227,7 +232,7 @@ chunk_state_simt_kernel(const Tin* __restrict__ k, const Tin* __restrict__ v, Se
       for (int e = threadIdx.x; e < kStateTok * 32; e += kThreads) {
         int jj = e / 32, cc = e % 32, j = j0 + jj, cl = blockIdx.x * 32 + cc;
         vt[e] = (j < Lc && cl < dv)
-                    ? gpow(dec, h, Lc - 1 - j) *
+                    ? gpow(dec, h, kRev ? j + 1 : Lc - 1 - j) *
                           Io<Tin>::ld(v, (static_cast<size_t>(c0 + j) * H + h) * dv + cl)
                     : 0.f;
       }
@@ -408,6 +413,189 @@ chunk_out_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   }
 }
 
+// ---------------------------------------------------------------------------
+// Gradient pass of the backward: block = (16 flat token rows, head h).  Row n
+// at position i of its chunk [cs, ce) gets
+//   causal (kAnti = false):      out_n = sum_{cs <= m <= n} gamma^(n-m) (a_n.b_m) c_m
+//                                        + gamma^(i+1) a_n M
+//   anti-causal (kAnti = true):  out_n = sum_{n <= m < ce} gamma^(m-n) (a_n.b_m) c_m
+//                                        + gamma^(ce-1-n) a_n M
+// where M is the state stored in the workspace slot of the row's chunk: a
+// [da][dc] matrix, or with kTrans the transpose of a stored [dc][da] one.
+// a, b: [Ttot][H][da]; c, out: [Ttot][H][dc].  Thread t owns column t
+// (dc <= 256).
+// ---------------------------------------------------------------------------
+template <typename Tin, bool kAnti, bool kTrans>
+__global__ void __launch_bounds__(kThreads)
+chunk_grad_simt_kernel(const Tin* __restrict__ a, const Tin* __restrict__ b,
+                       const Tin* __restrict__ c, SeqLayout L,
+                       const int32_t* __restrict__ chunk_base,
+                       const float* __restrict__ ws_states, float* __restrict__ out, int H,
+                       int da, int dc, HeadDecay dec) {
+  extern __shared__ float smem[];
+  const int lda = da + 1;
+  float* as = smem;                        // [kRows][da+1]
+  float* bs = as + kRows * lda;            // [kKeys][da+1]
+  float* cv = bs + kKeys * lda;            // [kKeys][dc]
+  float* ss = cv + kKeys * dc;             // [kRows][kKeys+1]
+  __shared__ int row_lo[kRows], row_hi[kRows], row_w[kRows];
+  __shared__ long long row_slot[kRows];
+
+  const int n0 = blockIdx.x * kRows, h = blockIdx.y;
+  const int tid = threadIdx.x;
+  if (tid < kRows) {
+    // key range [lo, hi] of the row inside its chunk and the exponent of its
+    // state weight; lo > hi marks a row outside every sequence
+    const int n = n0 + tid;
+    int lo = 1, hi = 0, w = 0;
+    long long slot = -1;
+    if (n < L.Ttot) {
+      const int sq = seq_of_token(L, n);
+      int sa, sb;
+      seq_bounds(L, sq, sa, sb);
+      if (n >= sa && n < sb) {
+        const int ch = (n - sa) / L.chunk;
+        const int cs = sa + ch * L.chunk;
+        const int ce = min(cs + L.chunk, sb);
+        if (kAnti) {
+          lo = n; hi = ce - 1; w = ce - 1 - n;
+        } else {
+          lo = cs; hi = n; w = n - cs + 1;
+        }
+        slot = slot_of(L, chunk_base, sq, ch);
+      }
+    }
+    row_lo[tid] = lo;
+    row_hi[tid] = hi;
+    row_w[tid] = w;
+    row_slot[tid] = slot;
+  }
+  for (int e = tid; e < kRows * da; e += kThreads) {
+    const int r = e / da, d = e % da, n = n0 + r;
+    as[r * lda + d] = n < L.Ttot ? Io<Tin>::ld(a, (static_cast<size_t>(n) * H + h) * da + d) : 0.f;
+  }
+  __syncthreads();
+
+  float acc[kRows];
+#pragma unroll
+  for (int r = 0; r < kRows; ++r) acc[r] = 0.f;
+  int kbeg = 0x7fffffff, kend = -1;
+  for (int r = 0; r < kRows; ++r) {
+    if (row_lo[r] <= row_hi[r]) {
+      kbeg = min(kbeg, row_lo[r]);
+      kend = max(kend, row_hi[r]);
+    }
+  }
+  for (int m0 = kbeg; m0 <= kend; m0 += kKeys) {
+    __syncthreads();
+    for (int e = tid; e < kKeys * da; e += kThreads) {
+      const int j = e / da, d = e % da, m = m0 + j;
+      bs[j * lda + d] = m <= kend ? Io<Tin>::ld(b, (static_cast<size_t>(m) * H + h) * da + d) : 0.f;
+    }
+    for (int e = tid; e < kKeys * dc; e += kThreads) {
+      const int j = e / dc, d = e % dc, m = m0 + j;
+      cv[j * dc + d] = m <= kend ? Io<Tin>::ld(c, (static_cast<size_t>(m) * H + h) * dc + d) : 0.f;
+    }
+    __syncthreads();
+    {
+      const int r = tid / kKeys, j = tid % kKeys;
+      const int n = n0 + r, m = m0 + j;
+      float sc = 0.f;
+      if (m >= row_lo[r] && m <= row_hi[r]) {
+        for (int d = 0; d < da; ++d) sc = fmaf(as[r * lda + d], bs[j * lda + d], sc);
+        sc *= gpow(dec, h, kAnti ? m - n : n - m);
+      }
+      ss[r * (kKeys + 1) + j] = sc;
+    }
+    __syncthreads();
+    if (tid < dc) {
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) {
+        float x = acc[r];
+        for (int j = 0; j < kKeys; ++j) x = fmaf(ss[r * (kKeys + 1) + j], cv[j * dc + tid], x);
+        acc[r] = x;
+      }
+    }
+  }
+  if (tid < dc) {
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      const int n = n0 + r;
+      if (row_lo[r] > row_hi[r]) continue;
+      float x = acc[r];
+      if (row_slot[r] >= 0 && row_slot[r] < L.nslots) {
+        const float* M = ws_states + (static_cast<size_t>(row_slot[r]) * H + h) * da * dc;
+        float t = 0.f;
+        for (int d = 0; d < da; ++d)
+          t = fmaf(as[r * lda + d], kTrans ? M[static_cast<size_t>(tid) * da + d]
+                                           : M[static_cast<size_t>(d) * dc + tid], t);
+        x = fmaf(gpow(dec, h, row_w[r]), t, x);
+      }
+      out[(static_cast<size_t>(n) * H + h) * dc + tid] = x;
+    }
+  }
+}
+
+template <typename Tin>
+cudaError_t launch_state_pass(bool rev, const void* k, const void* v, const SeqLayout& L,
+                              const int32_t* chunk_base, const float* state_in, float* state_out,
+                              float* states, int H, int dk, int dv, const HeadDecay& dec,
+                              cudaStream_t s) {
+  const size_t smem = sizeof(float) * (kStateTok * dk + kStateTok * 32);
+  auto kern = rev ? chunk_state_simt_kernel<Tin, true> : chunk_state_simt_kernel<Tin, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid((dv + 31) / 32, H, L.nseq);
+  kern<<<grid, kThreads, smem, s>>>(static_cast<const Tin*>(k), static_cast<const Tin*>(v), L,
+                                    chunk_base, state_in, state_out, states, H, dk, dv, dec);
+  return cudaGetLastError();
+}
+
+template <typename Tin, bool kAnti, bool kTrans>
+cudaError_t launch_grad_pass(const void* a, const void* b, const void* c, const SeqLayout& L,
+                             const int32_t* chunk_base, const float* states, float* out, int H,
+                             int da, int dc, const HeadDecay& dec, cudaStream_t s) {
+  const size_t smem =
+      sizeof(float) * ((kRows + kKeys) * (da + 1) + kKeys * dc + kRows * (kKeys + 1));
+  auto kern = chunk_grad_simt_kernel<Tin, kAnti, kTrans>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid((L.Ttot + kRows - 1) / kRows, H);
+  kern<<<grid, kThreads, smem, s>>>(static_cast<const Tin*>(a), static_cast<const Tin*>(b),
+                                    static_cast<const Tin*>(c), L, chunk_base, states, out, H, da,
+                                    dc, dec);
+  return cudaGetLastError();
+}
+
+// The backward in five launches: the forward states S (entering each chunk),
+// the states of the future F (after each chunk, walked backwards, ending in
+// d_state_in), then dQ (causal, reads S^T), dV (anti-causal, reads F) and dK
+// (anti-causal, reads F^T).
+template <typename Tin>
+cudaError_t chunkwise_bwd_typed(const void* q, const void* k, const void* v, const void* d_out,
+                                const SeqLayout& L, const float* state_in,
+                                const float* d_state_out, float* dq, float* dk, float* dv,
+                                float* d_state_in, const ChunkBwdWorkspace& ws, int H, int dk_,
+                                int dv_, const HeadDecay& dec, cudaStream_t s) {
+  cudaError_t e = launch_state_pass<Tin>(false, k, v, L, ws.chunk_base, state_in, nullptr,
+                                         ws.fwd_states, H, dk_, dv_, dec, s);
+  if (e == cudaSuccess)
+    e = launch_state_pass<Tin>(true, q, d_out, L, ws.chunk_base, d_state_out, d_state_in,
+                               ws.bwd_states, H, dk_, dv_, dec, s);
+  if (e != cudaSuccess || L.Ttot == 0) return e;
+  e = launch_grad_pass<Tin, false, true>(d_out, v, k, L, ws.chunk_base, ws.fwd_states, dq, H,
+                                         dv_, dk_, dec, s);
+  if (e == cudaSuccess)
+    e = launch_grad_pass<Tin, true, false>(k, q, d_out, L, ws.chunk_base, ws.bwd_states, dv, H,
+                                           dk_, dv_, dec, s);
+  if (e == cudaSuccess)
+    e = launch_grad_pass<Tin, true, true>(v, d_out, q, L, ws.chunk_base, ws.bwd_states, dk, H,
+                                          dv_, dk_, dec, s);
+  return e;
+}
+
 template <typename Tin, typename To>
 cudaError_t parallel_typed(const void* q, const void* k, const void* v, void* o, int B, int T,
                            int H, int dk, int dv, const HeadDecay& dec, cudaStream_t s) {
@@ -432,7 +620,7 @@ cudaError_t chunkwise_typed(int phases, const void* q, const void* k, const void
                             cudaStream_t s) {
   if (phases & 1) {
     size_t smem = sizeof(float) * (kStateTok * dk + kStateTok * 32);
-    auto kern = chunk_state_simt_kernel<Tin>;
+    auto kern = chunk_state_simt_kernel<Tin, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -508,6 +696,19 @@ cudaError_t launch_chunkwise_simt(int phases, const void* q, const void* k, cons
                                                  gn_b, eps, gated, ws, H, dk, dv, dec, s)
              : chunkwise_typed<float, bf, bf>(phases, q, k, v, L, state_in, state_out, out, g, gn_w,
                                               gn_b, eps, gated, ws, H, dk, dv, dec, s);
+}
+
+cudaError_t launch_chunkwise_bwd_simt(const void* q, const void* k, const void* v,
+                                      const void* d_out, DType in_t, const SeqLayout& L,
+                                      const float* state_in, const float* d_state_out, float* dq,
+                                      float* dk, float* dv, float* d_state_in,
+                                      const ChunkBwdWorkspace& ws, int H, int dk_, int dv_,
+                                      const HeadDecay& dec, cudaStream_t s) {
+  if (in_t == DType::F32)
+    return chunkwise_bwd_typed<float>(q, k, v, d_out, L, state_in, d_state_out, dq, dk, dv,
+                                      d_state_in, ws, H, dk_, dv_, dec, s);
+  return chunkwise_bwd_typed<__nv_bfloat16>(q, k, v, d_out, L, state_in, d_state_out, dq, dk, dv,
+                                            d_state_in, ws, H, dk_, dv_, dec, s);
 }
 
 }  // namespace ret

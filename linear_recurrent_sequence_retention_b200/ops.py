@@ -39,6 +39,8 @@ EXPORTED = (
     "retention_chunkwise_states",
     "retention_chunkwise_outputs",
     "retention_chunkwise_fwd_static_ws",
+    "retention_chunkwise_bwd_workspace_size",
+    "retention_chunkwise_bwd",
     "retention_recurrent_step",
     "retention_recurrent_steps",
     "msr_norm_gate",
@@ -96,6 +98,12 @@ def lib():
     L.retention_chunkwise_fwd_static_ws.argtypes = [vp, vp, vp, ci, cd, ci, vp, ci, vp, vp, vp,
                                                     ci, ctypes.POINTER(NormGate),
                                                     ci, ci, ci, ci, ci, vp]
+    L.retention_chunkwise_bwd_workspace_size.restype = ctypes.c_size_t
+    L.retention_chunkwise_bwd_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci]
+    L.retention_chunkwise_bwd.restype = ci
+    L.retention_chunkwise_bwd.argtypes = [vp, vp, vp, vp, ci, cd, ci, vp, ci, vp, vp,
+                                          vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                          ci, ci, ci, ci, ci, vp]
     L.retention_recurrent_step.restype = ci
     L.retention_recurrent_step.argtypes = [vp, vp, vp, ci, cd, vp, vp, ci, ci, ci, ci, ci, vp]
     L.retention_recurrent_steps.restype = ci
@@ -330,6 +338,60 @@ def chunkwise_fwd_static_ws(q, k, v, gamma, chunk, cu_seqlens=None, state_in=Non
         ctypes.byref(ng) if ng is not None else None, B, T, H, dk, dv, _stream(stream))
     _check(st, "retention_chunkwise_fwd_static_ws")
     return out
+
+
+def chunkwise_bwd_workspace_size(dtype, chunk, B, T, H, dk, dv, nseq=0):
+    code = RET_F32 if dtype == torch.float32 else RET_BF16
+    return int(lib().retention_chunkwise_bwd_workspace_size(code, chunk, B, T, H, dk, dv, nseq))
+
+
+def chunkwise_bwd(q, k, v, d_out, gamma, chunk, cu_seqlens=None, state_in=None,
+                  d_state_out=None, return_d_state=False, workspace=None, stream=None):
+    """Gradients of the chunkwise form (retention_chunkwise_bwd).
+
+    q, k: [B,T,H,dk]; v, d_out: [B,T,H,dv], one dtype; packed sequences as in
+    :func:`chunkwise_fwd`.  ``state_in`` is the forward's initial state and
+    ``d_state_out`` the gradient of its final state (float32 [nseq|B,H,dk,dv],
+    optional).  Returns float32 ``(dq, dk, dv)`` and, with ``return_d_state``,
+    the gradient of the initial state.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_out, "d_out")):
+        _dev(t, n)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    if (k.shape != q.shape or v.shape[:3] != q.shape[:3] or d_out.shape != v.shape
+            or len({q.dtype, k.dtype, v.dtype, d_out.dtype}) != 1):
+        raise ValueError("q, k, v, d_out shapes/dtypes disagree")
+    nseq = 0
+    if cu_seqlens is not None:
+        _dev(cu_seqlens, "cu_seqlens")
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise ValueError("cu_seqlens must be a 1-D int32 tensor with at least two entries")
+        nseq = cu_seqlens.numel() - 1
+    nstate = nseq if nseq else B
+    for t, n in ((state_in, "state_in"), (d_state_out, "d_state_out")):
+        if t is not None:
+            _dev(t, n)
+            if t.dtype != torch.float32 or tuple(t.shape) != (nstate, H, dk, dv):
+                raise ValueError(f"{n} must be float32 [{nstate},{H},{dk},{dv}]")
+    dq = torch.empty(B, T, H, dk, device=q.device, dtype=torch.float32)
+    dkk = torch.empty(B, T, H, dk, device=q.device, dtype=torch.float32)
+    dvv = torch.empty(B, T, H, dv, device=q.device, dtype=torch.float32)
+    dS0 = (torch.empty(nstate, H, dk, dv, device=q.device, dtype=torch.float32)
+           if return_d_state else None)
+    need = lib().retention_chunkwise_bwd_workspace_size(_dt(q), chunk, B, T, H, dk, dv, nseq)
+    if need == 0:
+        raise RetentionError(RET_ERR_UNSUPPORTED if max(dk, dv) > 256 else RET_ERR_INVALID_ARG,
+                             "retention_chunkwise_bwd_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    st = lib().retention_chunkwise_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(d_out), _dt(q), _gammas(gamma, H), int(chunk),
+        _ptr(cu_seqlens), nseq, _ptr(state_in), _ptr(d_state_out), _ptr(dq), _ptr(dkk),
+        _ptr(dvv), _ptr(dS0), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        B, T, H, dk, dv, _stream(stream))
+    _check(st, "retention_chunkwise_bwd")
+    return (dq, dkk, dvv, dS0) if return_d_state else (dq, dkk, dvv)
 
 
 def recurrent_step(q, k, v, gamma, state, out_dtype=torch.float32, out=None, stream=None):

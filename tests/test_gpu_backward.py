@@ -1,0 +1,122 @@
+"""GPU parity of the chunkwise backward (retention_chunkwise_bwd) against the
+fp64 oracle's gradients, through the C ABI.
+
+The kernels compute every product and sum in float32 from inputs that are
+exact (float32, or bfloat16 widened exactly), so both input dtypes are held
+to the float32 tolerance: relative L2 <= 1e-5 over each gradient, whole and
+per head.  Cases span several chunks with ragged tails, chunk lengths of one
+token and longer than the sequence, the largest supported heads, gamma = 0
+and gamma = 1, an initial state and an upstream state gradient, and packed
+sequences including empty ones.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_recurrent_sequence_retention_b200 import ops, workloads as W
+from tests._util import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    torch.cuda.init()
+    yield
+    ops.check_device_error()
+
+
+def _inputs(B, T, H, dk, dv, dtype, seed, with_state):
+    q, k, v, _ = W.make_qkvg(B, T, H, dk, dv, dtype, seed=seed, gate=False)
+    g = torch.Generator().manual_seed(seed + 7)
+    do = torch.randn(B, T, H, dv, generator=g).to(W.torch_dtype(dtype))
+    S0 = torch.randn(B, H, dk, dv, generator=g) if with_state else None
+    dS = torch.randn(B, H, dk, dv, generator=g) if with_state else None
+    return q, k, v, do, S0, dS
+
+
+def _check(got, ref, H, what):
+    names = ("dq", "dk", "dv")
+    for x, y, n in zip(got[:3], ref[:3], names):
+        assert_close(W.to_f64(x), y, "f32", 2, f"{what} {n}")
+    if len(got) > 3 and got[3] is not None:
+        assert_close(W.to_f64(got[3]), ref[3], "f32", 1, f"{what} d_state_in")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("B,T,H,dk,dv,chunk,with_state", [
+    (2, 77, 2, 16, 24, 16, True),      # several chunks, ragged tail, dk != dv
+    (1, 37, 2, 8, 8, 1, False),        # one-token chunks
+    (1, 9, 1, 16, 16, 64, True),       # chunk longer than the sequence
+    (1, 300, 3, 64, 128, 64, True),    # wider heads, several tiles
+    (1, 130, 1, 256, 256, 128, True),  # largest supported heads
+])
+def test_backward_matches_oracle(dtype, B, T, H, dk, dv, chunk, with_state):
+    q, k, v, do, S0, dS = _inputs(B, T, H, dk, dv, dtype, seed=T + dk, with_state=with_state)
+    gam = W.head_gammas(H)
+    ref = oracle.msr_backward(W.to_f64(q), W.to_f64(k), W.to_f64(v), gam, W.to_f64(do),
+                              None if S0 is None else S0.double().numpy(),
+                              None if dS is None else dS.double().numpy())
+    got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, chunk,
+                            state_in=None if S0 is None else S0.cuda(),
+                            d_state_out=None if dS is None else dS.cuda(), return_d_state=True)
+    _check(got, ref, H, f"{dtype} B{B} T{T} dk{dk} dv{dv} C{chunk}")
+
+
+@pytest.mark.parametrize("gammas", [[0.0, 1.0], [1.0, 0.5]])
+def test_backward_extreme_decays(gammas):
+    """gamma = 0 (diagonal only) and gamma = 1 (no decay) through several chunks."""
+    B, T, H, dk, dv, chunk = 1, 70, 2, 16, 32, 16
+    q, k, v, do, S0, dS = _inputs(B, T, H, dk, dv, "f32", seed=5, with_state=True)
+    ref = oracle.msr_backward(W.to_f64(q), W.to_f64(k), W.to_f64(v), gammas, W.to_f64(do),
+                              S0.double().numpy(), dS.double().numpy())
+    got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gammas, chunk,
+                            state_in=S0.cuda(), d_state_out=dS.cuda(), return_d_state=True)
+    _check(got, ref, H, f"gammas {gammas}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_packed_sequences(dtype):
+    """Packed batch with an empty sequence, one-token and ragged sequences."""
+    lens = [40, 0, 1, 77, 33]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    Tt = int(cu[-1])
+    H, dk, dv, chunk = 2, 32, 16, 16
+    q, k, v, do, _, _ = _inputs(1, Tt, H, dk, dv, dtype, seed=11, with_state=False)
+    g = torch.Generator().manual_seed(12)
+    S0 = torch.randn(len(lens), H, dk, dv, generator=g)
+    dS = torch.randn(len(lens), H, dk, dv, generator=g)
+    gam = W.head_gammas(H)
+    ref = oracle.msr_backward_varlen(W.to_f64(q), W.to_f64(k), W.to_f64(v), gam, W.to_f64(do),
+                                     cu, S0.double().numpy(), dS.double().numpy())
+    got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, chunk,
+                            cu_seqlens=torch.from_numpy(cu).cuda(), state_in=S0.cuda(),
+                            d_state_out=dS.cuda(), return_d_state=True)
+    _check(got, ref, H, f"packed {dtype}")
+
+
+def test_backward_chunk_length_does_not_matter():
+    """Every chunk length evaluates the same gradients (to float32 rounding)."""
+    B, T, H, dk, dv = 1, 100, 1, 32, 32
+    q, k, v, do, S0, dS = _inputs(B, T, H, dk, dv, "f32", seed=9, with_state=True)
+    args = [t.cuda() for t in (q, k, v, do)]
+    base = ops.chunkwise_bwd(*args, W.head_gammas(H), 100, state_in=S0.cuda(),
+                             d_state_out=dS.cuda(), return_d_state=True)
+    for chunk in (1, 7, 32):
+        got = ops.chunkwise_bwd(*args, W.head_gammas(H), chunk, state_in=S0.cuda(),
+                                d_state_out=dS.cuda(), return_d_state=True)
+        for x, y in zip(got, base):
+            assert_close(W.to_f64(x), W.to_f64(y), "f32", None, f"chunk {chunk}")
+
+
+def test_backward_rejects_unsupported_and_bad_arguments():
+    q = torch.zeros(1, 8, 1, 512, device="cuda")
+    v = torch.zeros(1, 8, 1, 16, device="cuda")
+    with pytest.raises(ops.RetentionError):
+        ops.chunkwise_bwd(q, q, v, v, [0.9], 4)
+    assert ops.chunkwise_bwd_workspace_size(torch.float32, 4, 1, 8, 1, 512, 16) == 0
+    assert ops.chunkwise_bwd_workspace_size(torch.float32, 0, 1, 8, 1, 16, 16) == 0
+    assert ops.chunkwise_bwd_workspace_size(torch.float32, 4, 1, 8, 1, 16, 16) > 0
