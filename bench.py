@@ -537,6 +537,66 @@ def run_decode(args, world, rank, pk, pk_kind):
             "gpu_launches": steps + calls}
 
 
+BACKWARD = "msr_b4_h8_t2048_dk128_dv256_c128"
+
+
+def fp32_fma_peak_tflops(pk):
+    """float32 FMA roofline of the CUDA cores: SMs x 128 lanes x 2 flops x the
+    maximum SM clock (MEASURED_PEAKS' sm_max_mhz, else the part's 1965 MHz)."""
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    mhz = float(pk.get("sm_max_mhz", 1965.0))
+    return sms * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def run_backward(args, world, rank, pk, pk_kind):
+    """The chunkwise backward (dQ, dK, dV and the initial-state gradient from
+    dO and the final-state gradient) on the B=4, T=2048, H=8, d_k=128,
+    d_v=256, chunk-128 workload with bf16 inputs; float32 arithmetic on CUDA
+    cores, so the roofline is the float32 FMA peak."""
+    from linear_recurrent_sequence_retention_b200 import ops
+    wl = W.WORKLOADS[BACKWARD]
+    dev = torch.device("cuda")
+    B, T, H, dk, dv, C = wl.B, wl.T, wl.H, wl.dk, wl.dv, wl.chunk
+    q, k, v, _ = W.make_qkvg(B, T, H, dk, dv, "bf16", seed=rank, gate=False, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(2000 + rank)
+    do = torch.randn(B, T, H, dv, generator=gen, device=dev).to(torch.bfloat16)
+    dS = torch.randn(B, H, dk, dv, generator=gen, device=dev)
+    gam = W.head_gammas(H)
+    ws = ops.alloc_workspace(ops.chunkwise_bwd_workspace_size(torch.bfloat16, C, B, T, H, dk, dv), dev)
+    for _ in range(max(3, args.warmup)):
+        ops.chunkwise_bwd(q, k, v, do, gam, C, d_state_out=dS, return_d_state=True, workspace=ws)
+    ops.check_device_error()
+    reps = 10
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        ops.chunkwise_bwd(q, k, v, do, gam, C, d_state_out=dS, return_d_state=True, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ops.check_device_error()
+    ms = max_over_ranks(e0.elapsed_time(e1) / reps, world)
+    # per token-head: three intra-chunk causal products (C+1)(dk+dv) each, three
+    # state reads 2 dk dv each, two state recurrences 2 dk dv each
+    flops = (3 * (C + 1) * (dk + dv) + 10 * dk * dv) * B * T * H
+    ach = flops / (ms / 1e3) / 1e12
+    peak = fp32_fma_peak_tflops(pk)
+    del q, k, v, do, dS, ws
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "input_dtype": "bf16", "ms_per_call": ms,
+            "tokens_per_s": sum_over_ranks(B * T, world) / (ms / 1e3),
+            "roofline": {"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                         "frac": ach / peak,
+                         "peak_source": "derived: SMs x 128 FP32 lanes x 2 flops x max SM clock",
+                         "algorithmic_flops_per_call": flops,
+                         "counting": f"per token-head 3 (C+1)(dk+dv) + 10 dk dv, C={C}",
+                         "kernel": "chunk_grad_simt_kernel + chunk_state_simt_kernel"},
+            "gpu_launches": 5 * reps}
+
+
 def main():
     global HEADLINE
     ap = argparse.ArgumentParser()
@@ -546,6 +606,8 @@ def main():
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--backward-only", action="store_true", help="backward only (profiling)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--workload", default=HEADLINE,
@@ -606,6 +668,13 @@ def main():
         return
 
     assert torch.cuda.is_available(), "bench.py needs a CUDA device (use --impl reference for the CPU arm)"
+    if args.backward_only:
+        bwd = run_backward(args, world, rank, pk, pk_kind)
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "backward": bwd, "n_gpus": world}), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     if args.no_headline:
         dec = run_decode(args, world, rank, pk, pk_kind)
         if rank == 0:
@@ -615,6 +684,7 @@ def main():
         return
     head = run_headline(args, world, rank, pk, pk_kind)
     dec = None if args.no_decode else run_decode(args, world, rank, pk, pk_kind)
+    bwd = None if args.no_backward else run_backward(args, world, rank, pk, pk_kind)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(wl, args.cpu_seconds)
@@ -638,10 +708,12 @@ def main():
             "hbm": head["hbm"],
             "kernels": head["kernels"],
             "decode": dec,
+            "backward": bwd,
             "e2e": head["e2e"],
             "cpu_baseline": cpu,
             "clocks": head["clocks"],
-            "gpu_launches": head["gpu_launches"] + (dec["gpu_launches"] if dec else 0),
+            "gpu_launches": (head["gpu_launches"] + (dec["gpu_launches"] if dec else 0)
+                             + (bwd["gpu_launches"] if bwd else 0)),
             "arithmetic": "bf16 tensor-core MMAs (tcgen05) with f32 accumulation; the "
                           "carried state, decayed scores and zeta*K enter the MMAs as "
                           "hi+lo bf16 pairs",

@@ -421,9 +421,10 @@ chunk_out_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
 //   anti-causal (kAnti = true):  out_n = sum_{n <= m < ce} gamma^(m-n) (a_n.b_m) c_m
 //                                        + gamma^(ce-1-n) a_n M
 // where M is the state stored in the workspace slot of the row's chunk: a
-// [da][dc] matrix, or with kTrans the transpose of a stored [dc][da] one.
-// a, b: [Ttot][H][da]; c, out: [Ttot][H][dc].  Thread t owns column t
-// (dc <= 256).
+// [da][dc] matrix, or with kTrans the transpose of a stored [dc][da] one
+// (read through shared memory 32 of its columns at a time, so that the global
+// loads stay coalesced).  a, b: [Ttot][H][da]; c, out: [Ttot][H][dc].  Thread
+// t owns column t (dc <= 256).
 // ---------------------------------------------------------------------------
 template <typename Tin, bool kAnti, bool kTrans>
 __global__ void __launch_bounds__(kThreads)
@@ -438,6 +439,7 @@ chunk_grad_simt_kernel(const Tin* __restrict__ a, const Tin* __restrict__ b,
   float* bs = as + kRows * lda;            // [kKeys][da+1]
   float* cv = bs + kKeys * lda;            // [kKeys][dc]
   float* ss = cv + kKeys * dc;             // [kRows][kKeys+1]
+  float* mt = ss + kRows * (kKeys + 1);    // kTrans: [32][dc+1], 32 columns of M^T
   __shared__ int row_lo[kRows], row_hi[kRows], row_w[kRows];
   __shared__ long long row_slot[kRows];
 
@@ -517,6 +519,49 @@ chunk_grad_simt_kernel(const Tin* __restrict__ a, const Tin* __restrict__ b,
       }
     }
   }
+  // decayed read of the state of each row's chunk
+  if (kTrans) {
+    // rows of the block share at most a few slots: walk the distinct ones
+    float t[kRows];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) t[r] = 0.f;
+    for (int r0 = 0; r0 < kRows; ++r0) {
+      const long long slot = row_slot[r0];
+      bool first = row_lo[r0] <= row_hi[r0] && slot >= 0 && slot < L.nslots;
+      for (int r = 0; r < r0 && first; ++r)
+        if (row_slot[r] == slot && row_lo[r] <= row_hi[r]) first = false;
+      if (!first) continue;                      // uniform over the block
+      const float* M = ws_states + (static_cast<size_t>(slot) * H + h) * da * dc;
+      for (int d0 = 0; d0 < da; d0 += 32) {
+        __syncthreads();
+        for (int e = tid; e < 32 * dc; e += kThreads) {
+          const int tt = e >> 5, j = e & 31;       // 32 consecutive d of column tt
+          mt[j * (dc + 1) + tt] = d0 + j < da ? M[static_cast<size_t>(tt) * da + d0 + j] : 0.f;
+        }
+        __syncthreads();
+        if (tid < dc) {
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            if (row_slot[r] != slot) continue;
+            float x = t[r];
+            const int jn = min(32, da - d0);
+            for (int j = 0; j < jn; ++j) x = fmaf(as[r * lda + d0 + j], mt[j * (dc + 1) + tid], x);
+            t[r] = x;
+          }
+        }
+      }
+    }
+    if (tid < dc) {
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) {
+        if (row_lo[r] > row_hi[r]) continue;
+        float x = acc[r];
+        if (row_slot[r] >= 0 && row_slot[r] < L.nslots) x = fmaf(gpow(dec, h, row_w[r]), t[r], x);
+        out[(static_cast<size_t>(n0 + r) * H + h) * dc + tid] = x;
+      }
+    }
+    return;
+  }
   if (tid < dc) {
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
@@ -526,9 +571,7 @@ chunk_grad_simt_kernel(const Tin* __restrict__ a, const Tin* __restrict__ b,
       if (row_slot[r] >= 0 && row_slot[r] < L.nslots) {
         const float* M = ws_states + (static_cast<size_t>(row_slot[r]) * H + h) * da * dc;
         float t = 0.f;
-        for (int d = 0; d < da; ++d)
-          t = fmaf(as[r * lda + d], kTrans ? M[static_cast<size_t>(tid) * da + d]
-                                           : M[static_cast<size_t>(d) * dc + tid], t);
+        for (int d = 0; d < da; ++d) t = fmaf(as[r * lda + d], M[static_cast<size_t>(d) * dc + tid], t);
         x = fmaf(gpow(dec, h, row_w[r]), t, x);
       }
       out[(static_cast<size_t>(n) * H + h) * dc + tid] = x;
@@ -557,7 +600,8 @@ cudaError_t launch_grad_pass(const void* a, const void* b, const void* c, const 
                              const int32_t* chunk_base, const float* states, float* out, int H,
                              int da, int dc, const HeadDecay& dec, cudaStream_t s) {
   const size_t smem =
-      sizeof(float) * ((kRows + kKeys) * (da + 1) + kKeys * dc + kRows * (kKeys + 1));
+      sizeof(float) * ((kRows + kKeys) * (da + 1) + kKeys * dc + kRows * (kKeys + 1) +
+                       (kTrans ? 32 * (dc + 1) : 0));
   auto kern = chunk_grad_simt_kernel<Tin, kAnti, kTrans>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
