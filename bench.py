@@ -550,9 +550,11 @@ def fp32_fma_peak_tflops(pk):
 
 def run_backward(args, world, rank, pk, pk_kind):
     """The chunkwise backward (dQ, dK, dV and the initial-state gradient from
-    dO and the final-state gradient) on the B=4, T=2048, H=8, d_k=128,
-    d_v=256, chunk-128 workload with bf16 inputs; float32 arithmetic on CUDA
-    cores, so the roofline is the float32 FMA peak."""
+    dO) on the B=4, T=2048, H=8, d_k=128, d_v=256, chunk-128 workload with
+    bf16 inputs.  Without a final-state gradient it runs on the tensor-core
+    forward kernels (three retentions, bf16 MMAs, roofline: the bf16 tensor
+    peak); with one (`cuda_core` below) on CUDA cores in float32 (roofline: the
+    float32 FMA peak)."""
     from linear_recurrent_sequence_retention_b200 import ops
     wl = W.WORKLOADS[BACKWARD]
     dev = torch.device("cuda")
@@ -564,37 +566,56 @@ def run_backward(args, world, rank, pk, pk_kind):
     dS = torch.randn(B, H, dk, dv, generator=gen, device=dev)
     gam = W.head_gammas(H)
     ws = ops.alloc_workspace(ops.chunkwise_bwd_workspace_size(torch.bfloat16, C, B, T, H, dk, dv), dev)
-    for _ in range(max(3, args.warmup)):
-        ops.chunkwise_bwd(q, k, v, do, gam, C, d_state_out=dS, return_d_state=True, workspace=ws)
-    ops.check_device_error()
-    reps = 10
-    barrier(world)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(reps):
-        ops.chunkwise_bwd(q, k, v, do, gam, C, d_state_out=dS, return_d_state=True, workspace=ws)
-    e1.record()
-    torch.cuda.synchronize()
-    barrier(world)
-    ops.check_device_error()
-    ms = max_over_ranks(e0.elapsed_time(e1) / reps, world)
     # per token-head: three intra-chunk causal products (C+1)(dk+dv) each, three
     # state reads 2 dk dv each, two state recurrences 2 dk dv each
     flops = (3 * (C + 1) * (dk + dv) + 10 * dk * dv) * B * T * H
-    ach = flops / (ms / 1e3) / 1e12
-    peak = fp32_fma_peak_tflops(pk)
+    tokens = sum_over_ranks(B * T, world)
+
+    def timed(dstate, reps):
+        for _ in range(max(3, args.warmup)):
+            ops.chunkwise_bwd(q, k, v, do, gam, C, d_state_out=dstate, return_d_state=True,
+                              workspace=ws)
+        ops.check_device_error()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            ops.chunkwise_bwd(q, k, v, do, gam, C, d_state_out=dstate, return_d_state=True,
+                              workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        ops.check_device_error()
+        return max_over_ranks(e0.elapsed_time(e1) / reps, world)
+
+    reps_tc, reps_cc = 20, 5
+    ms_tc = timed(None, reps_tc)
+    ms_cc = timed(dS, reps_cc)
+    ach_tc = flops / (ms_tc / 1e3) / 1e12
+    ach_cc = flops / (ms_cc / 1e3) / 1e12
+    peak_tc = pk["bf16_tflops"]
+    peak_cc = fp32_fma_peak_tflops(pk)
     del q, k, v, do, dS, ws
     torch.cuda.empty_cache()
-    return {"workload": wl.name, "input_dtype": "bf16", "ms_per_call": ms,
-            "tokens_per_s": sum_over_ranks(B * T, world) / (ms / 1e3),
-            "roofline": {"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                         "frac": ach / peak,
-                         "peak_source": "derived: SMs x 128 FP32 lanes x 2 flops x max SM clock",
+    return {"workload": wl.name, "input_dtype": "bf16", "ms_per_call": ms_tc,
+            "tokens_per_s": tokens / (ms_tc / 1e3),
+            "path": "tensor cores: three forward retentions (dQ; dV and dK on the sequences "
+                    "read backwards) plus token-reversal copies",
+            "roofline": {"bound": "tensor", "achieved": ach_tc, "peak": peak_tc,
+                         "unit": "TFLOP/s", "frac": ach_tc / peak_tc,
+                         "peak_source": f"{pk_kind} bf16 (burst)",
                          "algorithmic_flops_per_call": flops,
                          "counting": f"per token-head 3 (C+1)(dk+dv) + 10 dk dv, C={C}",
-                         "kernel": "chunk_grad_simt_kernel + chunk_state_simt_kernel"},
-            "gpu_launches": 5 * reps}
+                         "kernel": "state_kernel + output_kernel (x3), flip_tokens_kernel"},
+            "cuda_core": {"with": "a final-state gradient (d_state_out)", "ms_per_call": ms_cc,
+                          "tokens_per_s": tokens / (ms_cc / 1e3),
+                          "roofline": {"bound": "alu", "achieved": ach_cc, "peak": peak_cc,
+                                       "unit": "TFLOP/s", "frac": ach_cc / peak_cc,
+                                       "peak_source": "derived: SMs x 128 FP32 lanes x 2 flops "
+                                                      "x max SM clock",
+                                       "kernel": "chunk_grad_simt_kernel + chunk_state_simt_kernel"}},
+            "gpu_launches": 13 * reps_tc + 5 * reps_cc}
 
 
 def main():

@@ -346,15 +346,24 @@ ret_status msr_norm_gate(const void* o, ret_dtype o_dtype, const ret_norm_gate* 
 namespace {
 
 struct BwdPlan {
-  ret::SeqLayout L;
+  ret::SeqLayout L;     // CUDA-core path: the caller's chunk
   size_t meta;
   long long slots;
-  size_t state_bytes;   // one set of per-chunk states
-  size_t bytes;
+  size_t state_bytes;   // one set of per-chunk float32 states
+  size_t bytes;         // CUDA-core path
+  bool tc_ok;           // the tensor-core path is possible (bf16, heads 64/128/256)
+  ret::SeqLayout Ltc;   // tensor-core path: the executed chunk
+  size_t tc_states;     // one set of hi/lo bf16 states at that chunk
+  size_t tc_bytes;      // tensor-core path: meta + states + scratch
 };
 
-// Shared by the backward's size query and call: every supported shape runs on
-// CUDA cores in float32 (bf16 inputs are read exactly and widened).
+bool tc_head(int d) { return d == 64 || d == 128 || d == 256; }
+
+// Shared by the backward's size query and call.  The CUDA-core path (float32
+// arithmetic, f32 or bf16 inputs, heads up to 256) takes any arguments; bf16
+// inputs with heads of 64, 128 or 256 and a chunk of 64..512 may also run on
+// the tensor-core forward kernels (see launch_chunkwise_bwd_tc), and the
+// workspace is sized for whichever path needs more.
 ret_status plan_chunkwise_bwd(ret_dtype in_dtype, int chunk, int B, int T, int H, int dk, int dv,
                               int nseq, const int32_t* cu, BwdPlan* p) {
   if (!dtype_ok(in_dtype) || chunk < 1 || H < 1 || H > ret::kMaxHeads || dk < 1 || dv < 1 ||
@@ -382,6 +391,19 @@ ret_status plan_chunkwise_bwd(ret_dtype in_dtype, int chunk, int B, int T, int H
   p->L.nslots = p->slots;
   p->state_bytes = static_cast<size_t>(p->slots) * H * dk * dv * sizeof(float);
   p->bytes = p->meta + 2 * p->state_bytes;
+  p->tc_ok = in_dtype == RET_BF16 && tc_head(dk) && tc_head(dv) &&
+             ret::chunkwise_tc_supported(dk, dv, chunk) && ret::chunkwise_tc_supported(dv, dk, chunk);
+  p->tc_bytes = 0;
+  if (p->tc_ok) {
+    // one executed chunk for the three passes (d_k and d_v exchange roles)
+    const int ce = ret::chunkwise_tc_chunk(chunk, dk > dv ? dk : dv);
+    p->Ltc = p->L;
+    p->Ltc.chunk = ce;
+    p->Ltc.nslots = varlen ? (Ttot + ce - 1) / ce + nseq
+                           : static_cast<long long>(B) * ((T + ce - 1) / ce);
+    p->tc_states = static_cast<size_t>(p->Ltc.nslots) * H * dk * dv * 4;   // hi + lo bf16
+    p->tc_bytes = p->meta + p->tc_states + ret::chunkwise_bwd_tc_scratch_bytes(p->Ltc, H, dk, dv);
+  }
   return RET_OK;
 }
 
@@ -393,7 +415,7 @@ size_t retention_chunkwise_bwd_workspace_size(ret_dtype in_dtype, int chunk, int
                                               int H, int dk, int dv, int nseq) {
   BwdPlan p;
   if (plan_chunkwise_bwd(in_dtype, chunk, B, T, H, dk, dv, nseq, nullptr, &p) != RET_OK) return 0;
-  return p.bytes;
+  return p.bytes > p.tc_bytes ? p.bytes : p.tc_bytes;
 }
 
 ret_status retention_chunkwise_bwd(const void* q, const void* k, const void* v, const void* d_out,
@@ -414,12 +436,26 @@ ret_status retention_chunkwise_bwd(const void* q, const void* k, const void* v, 
     if (ptr && !aligned16(ptr)) return RET_ERR_INVALID_ARG;
   ret::HeadDecay dec;
   if (!make_decay(gamma, H, &dec)) return RET_ERR_INVALID_ARG;
+  const bool use_tc = p.tc_ok && d_state_out == nullptr;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
-      workspace_bytes < p.bytes)
+      workspace_bytes < (use_tc ? p.tc_bytes : p.bytes))
     return RET_ERR_WORKSPACE;
   unsigned* err = error_word();
   if (!err) return RET_ERR_CUDA;
   char* base = static_cast<char*>(workspace);
+  if (use_tc) {
+    ret::ChunkWorkspace tw;
+    tw.chunk_base = reinterpret_cast<int32_t*>(base);
+    tw.order = tw.chunk_base + p.Ltc.nseq + 1;
+    tw.states = base + p.meta;
+    tw.nslots = p.Ltc.nslots;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = ret::launch_chunk_prep(p.Ltc, tw, err, s);
+    if (e == cudaSuccess)
+      e = ret::launch_chunkwise_bwd_tc(q, k, v, d_out, p.Ltc, state_in, dq, dk, dv, d_state_in, tw,
+                                       base + p.meta + p.tc_states, H, dk_, dv_, dec, err, s);
+    return cuda_status(e);
+  }
   ret::ChunkWorkspace fw;
   fw.chunk_base = reinterpret_cast<int32_t*>(base);
   fw.order = fw.chunk_base + p.L.nseq + 1;

@@ -1,0 +1,140 @@
+// Backward of the chunkwise form on the tensor-core forward kernels (bf16
+// inputs).  The gradients of the pages' retention (abeam.tech summary of Sun et
+// al. 2023, 「学習は並列、生成は状態更新」 and 「長文の学習にはチャンク再帰を使う」)
+// are three retentions of the same kind as the forward, with the operand roles
+// exchanged:
+//     dq_n = sum_{m<=n} gamma^(n-m) (dO_n . v_m) k_m + gamma^(n+1) dO_n S0^T
+//          = forward(q = dO, k = V, v = K, state_in = S0^T)
+//     dv_m = sum_{n>=m} gamma^(n-m) (k_m . q_n) dO_n
+//          = forward(q = K, k = Q, v = dO) on every sequence read backwards
+//     dk_m = sum_{n>=m} gamma^(n-m) (v_m . dO_n) q_n
+//          = forward(q = V, k = dO, v = Q) on every sequence read backwards
+//     dS0  = sum_n gamma^(n+1) q_n^T dO_n
+//          = gamma * (final state of the backwards (k = Q, v = dO) pass)
+// (reading a sequence backwards turns "n >= m" into "n' <= m'" with the same
+// distance).  This file holds the three small streaming kernels the
+// composition needs (reverse the tokens of every sequence, transpose the
+// initial state, scale the state gradient per head) and the host sequence of
+// launches; the retentions themselves run in chunkwise_tc.cu.
+#include "launch.h"
+
+namespace ret {
+namespace {
+
+constexpr int kFlipThreads = 256;
+
+// dst[a + j] = src[b - 1 - j] for every sequence [a, b) of the flat token
+// axis; a token row is `row_bytes` bytes (a multiple of 16).  One block per
+// token, 16-byte copies.
+__global__ void __launch_bounds__(kFlipThreads)
+flip_tokens_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, SeqLayout L,
+                   int row_vec) {
+  const int n = blockIdx.x;
+  if (n >= L.Ttot) return;
+  const int s = seq_of_token(L, n);
+  int a, b;
+  seq_bounds(L, s, a, b);
+  if (n < a || n >= b) return;
+  const int m = a + b - 1 - n;
+  const uint4* sr = src + static_cast<size_t>(m) * row_vec;
+  uint4* dr = dst + static_cast<size_t>(n) * row_vec;
+  for (int i = threadIdx.x; i < row_vec; i += kFlipThreads) dr[i] = sr[i];
+}
+
+// out[s][h] = in[s][h]^T  (in: [dk][dv] -> out: [dv][dk]), 32 x 32 tiles.
+__global__ void transpose_states_kernel(const float* __restrict__ in, float* __restrict__ out,
+                                        int dk, int dv) {
+  __shared__ float tile[32][33];
+  const size_t mat = static_cast<size_t>(blockIdx.z) * dk * dv;
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    tile[i][threadIdx.x] = (r < dk && c < dv) ? in[mat + static_cast<size_t>(r) * dv + c] : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (c < dv && r < dk) out[mat + static_cast<size_t>(c) * dk + r] = tile[threadIdx.x][i];
+  }
+}
+
+// x[s][h] *= gamma_h over [nmat = nseq*H][dk*dv].
+__global__ void scale_states_kernel(float* __restrict__ x, int H, size_t per, HeadDecay dec) {
+  const int mat = blockIdx.y;
+  const float gm = dec.gamma[mat % H];
+  float* p = x + static_cast<size_t>(mat) * per;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < per;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    p[i] *= gm;
+}
+
+cudaError_t flip(const void* src, void* dst, const SeqLayout& L, size_t row_bytes, cudaStream_t s) {
+  if (L.Ttot == 0) return cudaSuccess;
+  flip_tokens_kernel<<<L.Ttot, kFlipThreads, 0, s>>>(static_cast<const uint4*>(src),
+                                                     static_cast<uint4*>(dst), L,
+                                                     static_cast<int>(row_bytes / 16));
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t chunkwise_bwd_tc_scratch_bytes(const SeqLayout& L, int H, int dk, int dv) {
+  const size_t T = static_cast<size_t>(L.Ttot);
+  auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
+  return 2 * r256(T * H * dk * 2) + 2 * r256(T * H * dv * 2)      // q, k, v, dO read backwards
+         + r256(T * H * dk * 4) + r256(T * H * dv * 4)             // dK, dV of the backwards passes
+         + r256(static_cast<size_t>(L.nseq) * H * dk * dv * 4);    // S0^T
+}
+
+cudaError_t launch_chunkwise_bwd_tc(const void* q, const void* k, const void* v,
+                                    const void* d_out, const SeqLayout& L, const float* state_in,
+                                    float* dq, float* dk, float* dv, float* d_state_in,
+                                    ChunkWorkspace ws, void* scratch, int H, int dk_, int dv_,
+                                    const HeadDecay& dec, unsigned* err, cudaStream_t s) {
+  const size_t T = static_cast<size_t>(L.Ttot);
+  auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
+  char* p = static_cast<char*>(scratch);
+  void* q_r = p;  p += r256(T * H * dk_ * 2);
+  void* k_r = p;  p += r256(T * H * dk_ * 2);
+  void* v_r = p;  p += r256(T * H * dv_ * 2);
+  void* do_r = p; p += r256(T * H * dv_ * 2);
+  float* dk_r = reinterpret_cast<float*>(p); p += r256(T * H * dk_ * 4);
+  float* dv_r = reinterpret_cast<float*>(p); p += r256(T * H * dv_ * 4);
+  float* s0t = reinterpret_cast<float*>(p);
+  const size_t rq = static_cast<size_t>(H) * dk_ * 2, rv = static_cast<size_t>(H) * dv_ * 2;
+  cudaError_t e = flip(q, q_r, L, rq, s);
+  if (e == cudaSuccess) e = flip(k, k_r, L, rq, s);
+  if (e == cudaSuccess) e = flip(v, v_r, L, rv, s);
+  if (e == cudaSuccess) e = flip(d_out, do_r, L, rv, s);
+  if (e == cudaSuccess && state_in) {
+    dim3 grid((dv_ + 31) / 32, (dk_ + 31) / 32, static_cast<unsigned>(L.nseq) * H);
+    transpose_states_kernel<<<grid, dim3(32, 8), 0, s>>>(state_in, s0t, dk_, dv_);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) return e;
+  const DType F = DType::F32;
+  // dQ: forward(q = dO, k = V, v = K) from S0^T
+  e = launch_chunkwise_tc(3, d_out, v, k, L, state_in ? s0t : nullptr, state_in != nullptr,
+                          nullptr, dq, F, nullptr, F, nullptr, nullptr, 0.f, false, ws, H, dv_, dk_,
+                          dec, err, s);
+  // dV on the sequences read backwards: forward(q = K, k = Q, v = dO); its final
+  // state is sum_n gamma^n q_n^T dO_n, the initial-state gradient before one gamma
+  if (e == cudaSuccess)
+    e = launch_chunkwise_tc(3, k_r, q_r, do_r, L, nullptr, false, d_state_in, dv_r, F, nullptr, F,
+                            nullptr, nullptr, 0.f, false, ws, H, dk_, dv_, dec, err, s);
+  // dK on the sequences read backwards: forward(q = V, k = dO, v = Q)
+  if (e == cudaSuccess)
+    e = launch_chunkwise_tc(3, v_r, do_r, q_r, L, nullptr, false, nullptr, dk_r, F, nullptr, F,
+                            nullptr, nullptr, 0.f, false, ws, H, dv_, dk_, dec, err, s);
+  if (e == cudaSuccess) e = flip(dv_r, dv, L, static_cast<size_t>(H) * dv_ * 4, s);
+  if (e == cudaSuccess) e = flip(dk_r, dk, L, static_cast<size_t>(H) * dk_ * 4, s);
+  if (e == cudaSuccess && d_state_in) {
+    const size_t per = static_cast<size_t>(dk_) * dv_;
+    dim3 grid(static_cast<unsigned>((per + 1023) / 1024), static_cast<unsigned>(L.nseq) * H);
+    scale_states_kernel<<<grid, 256, 0, s>>>(d_state_in, H, per, dec);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace ret

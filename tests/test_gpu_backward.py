@@ -1,13 +1,16 @@
 """GPU parity of the chunkwise backward (retention_chunkwise_bwd) against the
 fp64 oracle's gradients, through the C ABI.
 
-The kernels compute every product and sum in float32 from inputs that are
-exact (float32, or bfloat16 widened exactly), so both input dtypes are held
-to the float32 tolerance: relative L2 <= 1e-5 over each gradient, whole and
-per head.  Cases span several chunks with ragged tails, chunk lengths of one
-token and longer than the sequence, the largest supported heads, gamma = 0
-and gamma = 1, an initial state and an upstream state gradient, and packed
-sequences including empty ones.
+On the CUDA-core path the kernels compute every product and sum in float32
+from inputs that are exact (float32, or bfloat16 widened exactly), so both
+input dtypes are held to the float32 tolerance: relative L2 <= 1e-5 over each
+gradient, whole and per head.  bf16 inputs with heads of 64/128/256 and no
+final-state gradient run on the tensor-core kernels instead and are held to
+the bf16-input tolerance (plus rel-L2 <= 1e-4 as a precision check).  Cases
+span several chunks with ragged tails, chunk lengths of one token and longer
+than the sequence, the largest supported heads, gamma = 0 and gamma = 1, an
+initial state and an upstream state gradient, and packed sequences including
+empty ones.
 """
 
 import numpy as np
@@ -16,7 +19,7 @@ import torch
 
 import oracle
 from linear_recurrent_sequence_retention_b200 import ops, workloads as W
-from tests._util import assert_close
+from tests._util import assert_close, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -64,6 +67,46 @@ def test_backward_matches_oracle(dtype, B, T, H, dk, dv, chunk, with_state):
                             state_in=None if S0 is None else S0.cuda(),
                             d_state_out=None if dS is None else dS.cuda(), return_d_state=True)
     _check(got, ref, H, f"{dtype} B{B} T{T} dk{dk} dv{dv} C{chunk}")
+
+
+@pytest.mark.parametrize("B,T,H,dk,dv,chunk,with_state", [
+    (2, 300, 2, 64, 128, 128, True),     # several chunks and tiles, initial state
+    (1, 700, 1, 128, 256, 64, False),    # 64-token chunks executed as 256
+    (1, 200, 2, 256, 64, 256, True),     # d_k > d_v
+    (1, 1030, 2, 128, 128, 512, False),  # 512-token chunks, ragged last chunk
+])
+def test_backward_tensor_core_path(B, T, H, dk, dv, chunk, with_state):
+    """bf16 inputs with heads of 64/128/256 and no final-state gradient run on the
+    tensor-core forward kernels (three retentions, two on reversed sequences);
+    held to the bf16-input tolerance and, as a precision check, rel-L2 <= 1e-4."""
+    q, k, v, do, S0, _ = _inputs(B, T, H, dk, dv, "bf16", seed=T + 3 * dk, with_state=with_state)
+    gam = W.head_gammas(H)
+    ref = oracle.msr_backward(W.to_f64(q), W.to_f64(k), W.to_f64(v), gam, W.to_f64(do),
+                              None if S0 is None else S0.double().numpy())
+    got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, chunk,
+                            state_in=None if S0 is None else S0.cuda(), return_d_state=True)
+    for x, y, n in zip(got, ref, ("dq", "dk", "dv", "d_state_in")):
+        assert_close(W.to_f64(x), y, "bf16", 2 if n != "d_state_in" else 1, f"tc {n}")
+        assert rel_l2(W.to_f64(x), y) <= 1e-4, (n, rel_l2(W.to_f64(x), y))
+
+
+def test_backward_tensor_core_packed():
+    """The tensor-core path on packed sequences (reversal inside each sequence)."""
+    lens = [300, 0, 1, 129, 64]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    Tt = int(cu[-1])
+    H, dk, dv, chunk = 2, 64, 64, 64
+    q, k, v, do, _, _ = _inputs(1, Tt, H, dk, dv, "bf16", seed=21, with_state=False)
+    S0 = torch.randn(len(lens), H, dk, dv, generator=torch.Generator().manual_seed(22))
+    gam = W.head_gammas(H)
+    ref = oracle.msr_backward_varlen(W.to_f64(q), W.to_f64(k), W.to_f64(v), gam, W.to_f64(do),
+                                     cu, S0.double().numpy())
+    got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, chunk,
+                            cu_seqlens=torch.from_numpy(cu).cuda(), state_in=S0.cuda(),
+                            return_d_state=True)
+    for x, y, n in zip(got, ref, ("dq", "dk", "dv", "d_state_in")):
+        assert_close(W.to_f64(x), y, "bf16", 2 if n != "d_state_in" else 1, f"tc packed {n}")
+        assert rel_l2(W.to_f64(x), y) <= 1e-4, (n, rel_l2(W.to_f64(x), y))
 
 
 @pytest.mark.parametrize("gammas", [[0.0, 1.0], [1.0, 0.5]])
