@@ -81,6 +81,7 @@ __all__ = [
     "retention_backward",
     "msr_backward",
     "msr_backward_varlen",
+    "rope",
 ]
 
 
@@ -412,3 +413,42 @@ def msr_backward_varlen(q, k, v, gamma, d_out, cu_seqlens, state=None, d_state=N
             else:
                 dS0[i, h] = 0.0 if dS is None else _f64(dS)
     return dq, dkk, dvv, dS0
+
+
+# ---------------------------------------------------------------------------
+# Rotary position encoding of q and k
+# ---------------------------------------------------------------------------
+
+def rope(x, base=10000.0, cu_seqlens=None):
+    """Rotary position encoding of ``x: [B, T, H, d]`` (d even), in float64.
+
+    [RetNet-JA] 「Retentionは「内容に応じた参照」と「距離による忘却」を掛け合わせる」:
+    Q and K receive a position rotation after the projections; [EulerStack]
+    "장점": RoPE-compatible.  The pages give no formula; the reading taken is
+    the standard rotary form: the pair (x[2i], x[2i+1]) of a token at position
+    p (its index within its own sequence) is rotated by the angle p * theta_i,
+    theta_i = base^(-2i/d):
+        x'[2i]   = x[2i] cos(p theta_i) - x[2i+1] sin(p theta_i)
+        x'[2i+1] = x[2i] sin(p theta_i) + x[2i+1] cos(p theta_i)
+    Packed sequences (``B = 1`` and ``cu_seqlens``) count positions from each
+    sequence's first token.
+    """
+    x = _f64(x)
+    B, T, H, d = x.shape
+    if d % 2:
+        raise ValueError("rope needs an even head dimension")
+    pos = np.zeros((B, T))
+    if cu_seqlens is None:
+        pos[:] = np.arange(T)[None, :]
+    else:
+        cu = [int(c) for c in cu_seqlens]
+        for a, b in zip(cu[:-1], cu[1:]):
+            pos[0, a:b] = np.arange(b - a)
+    theta = np.power(float(base), -np.arange(0, d, 2) / d)          # [d/2]
+    ang = pos[:, :, None, None] * theta[None, None, None, :]         # [B, T, 1, d/2]
+    c, s = np.cos(ang), np.sin(ang)
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = x0 * c - x1 * s
+    out[..., 1::2] = x0 * s + x1 * c
+    return out
