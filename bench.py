@@ -618,6 +618,41 @@ def run_backward(args, world, rank, pk, pk_kind):
             "gpu_launches": 13 * reps_tc + 5 * reps_cc}
 
 
+def run_rope(args, world, rank, pk, pk_kind):
+    """Rotary position encoding of q and k of the 6.7B-shaped workload (B=2,
+    T=8192, H=16, d_k=256, bf16): one streaming pass, HBM-bound (reads q and
+    k, writes the rotated copies)."""
+    from linear_recurrent_sequence_retention_b200 import ops
+    wl = W.WORKLOADS[HEADLINE]
+    dev = torch.device("cuda")
+    q, k, _, _ = W.make_qkvg(wl.B, wl.T, wl.H, wl.dk, 8, "bf16", seed=rank, gate=False, device=dev)
+    qo, ko = torch.empty_like(q), torch.empty_like(k)
+    for _ in range(max(3, args.warmup)):
+        ops.rope(q, k, q_out=qo, k_out=ko)
+    reps = 20
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        ops.rope(q, k, q_out=qo, k_out=ko)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ops.check_device_error()
+    ms = max_over_ranks(e0.elapsed_time(e1) / reps, world)
+    nbytes = 4 * q.numel() * q.element_size()             # q, k read; rotated q, k written
+    ach = nbytes / (ms / 1e3) / 1e9
+    del q, k, qo, ko
+    torch.cuda.empty_cache()
+    return {"workload": f"{wl.name} q,k", "ms_per_call": ms,
+            "tokens_per_s": sum_over_ranks(wl.B * wl.T, world) / (ms / 1e3),
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / pk["hbm_gbs"], "peak_source": pk_kind,
+                         "algorithmic_bytes_per_launch": nbytes, "kernel": "rope_kernel"},
+            "gpu_launches": reps}
+
+
 def main():
     global HEADLINE
     ap = argparse.ArgumentParser()
@@ -629,6 +664,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--backward-only", action="store_true", help="backward only (profiling)")
+    ap.add_argument("--no-rope", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--workload", default=HEADLINE,
@@ -706,6 +742,7 @@ def main():
     head = run_headline(args, world, rank, pk, pk_kind)
     dec = None if args.no_decode else run_decode(args, world, rank, pk, pk_kind)
     bwd = None if args.no_backward else run_backward(args, world, rank, pk, pk_kind)
+    rope = None if args.no_rope else run_rope(args, world, rank, pk, pk_kind)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(wl, args.cpu_seconds)
@@ -730,11 +767,13 @@ def main():
             "kernels": head["kernels"],
             "decode": dec,
             "backward": bwd,
+            "rope": rope,
             "e2e": head["e2e"],
             "cpu_baseline": cpu,
             "clocks": head["clocks"],
             "gpu_launches": (head["gpu_launches"] + (dec["gpu_launches"] if dec else 0)
-                             + (bwd["gpu_launches"] if bwd else 0)),
+                             + (bwd["gpu_launches"] if bwd else 0)
+                             + (rope["gpu_launches"] if rope else 0)),
             "arithmetic": "bf16 tensor-core MMAs (tcgen05) with f32 accumulation; the "
                           "carried state, decayed scores and zeta*K enter the MMAs as "
                           "hi+lo bf16 pairs",

@@ -27,7 +27,7 @@
  *
  * No 1/sqrt(d_k) factor is applied inside retention (the pages' formula has
  * none); callers fold any scale into q or k.  Rotary position encoding, if
- * used, is applied by the caller to q and k before these calls.
+ * used, is applied to q and k before these calls (retention_rope).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -56,7 +56,8 @@
  *             arguments are valid but this build has no kernel for the shape
  *             or dtype combination; there is no fallback path.
  *   Aliasing: outputs must not overlap inputs, except that
- *             retention_recurrent_step(s) update `state` in place by design.
+ *             retention_recurrent_step(s) update `state` in place by design
+ *             and retention_rope may rotate q and k in place.
  */
 #ifndef RETENTION_H_
 #define RETENTION_H_
@@ -329,6 +330,27 @@ RET_API ret_status retention_chunkwise_bwd(const void* q, const void* k, const v
                                            void* workspace, size_t workspace_bytes,
                                            int B, int T, int H, int dk_, int dv_,
                                            ret_stream_t stream);
+
+/*
+ * Rotary position encoding of q and k, applied before the retention calls.
+ * The abeam.tech summary (section 「Retentionは「内容に応じた参照」と「距離による
+ * 忘却」を掛け合わせる」) rotates Q and K by position after the projections and
+ * eulerwa.com "3. RetNet 상세" ("장점") calls retention RoPE-compatible; the
+ * pages give no formula, and this is the standard rotary form: for a token at
+ * position p (its index within its own sequence) and pair i < d/2,
+ *     x'[2i]   = x[2i] cos(p theta_i) - x[2i+1] sin(p theta_i)
+ *     x'[2i+1] = x[2i] sin(p theta_i) + x[2i+1] cos(p theta_i),
+ *     theta_i  = base^(-2i/d)                                   (base > 1)
+ *   q, k: [B,T,H,d] dtype (packed: B = 1 with cu_seqlens/nseq as for
+ *   retention_chunkwise_fwd; positions restart at every sequence)
+ *   q_out, k_out: [B,T,H,d] dtype, written in full; q_out may equal q and
+ *   k_out may equal k (in place), no other overlap.
+ * The angle is reduced modulo 2 pi in double precision, the rotation is
+ * float32 and a bf16 output is rounded to nearest once.  d even, any H.
+ */
+RET_API ret_status retention_rope(const void* q, const void* k, ret_dtype dtype, void* q_out,
+                                  void* k_out, double base, const int32_t* cu_seqlens, int nseq,
+                                  int B, int T, int H, int d, ret_stream_t stream);
 
 /*
  * Standalone per-head GroupNorm + Swish gate (the epilogue that

@@ -475,6 +475,32 @@ ret_status retention_chunkwise_bwd(const void* q, const void* k, const void* v, 
   return cuda_status(e);
 }
 
+ret_status retention_rope(const void* q, const void* k, ret_dtype dtype, void* q_out, void* k_out,
+                          double base, const int32_t* cu_seqlens, int nseq, int B, int T, int H,
+                          int d, ret_stream_t stream) {
+  if (!dtype_ok(dtype) || H < 1 || d < 2 || (d & 1) || d > 65536 || nseq < 0 ||
+      !std::isfinite(base) || base <= 1.0)
+    return RET_ERR_INVALID_ARG;
+  const bool varlen = cu_seqlens != nullptr;
+  if (varlen != (nseq > 0)) return RET_ERR_INVALID_ARG;
+  if (varlen ? (B != 1 || T < 0) : (B < 1 || T < 1)) return RET_ERR_INVALID_ARG;
+  const long long Ttot = varlen ? T : static_cast<long long>(B) * T;
+  if (!fits_int(Ttot * H * static_cast<long long>(d))) return RET_ERR_INVALID_ARG;
+  if (Ttot > 0 && (!q || !k || !q_out || !k_out)) return RET_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, q_out, k_out, cu_seqlens};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return RET_ERR_INVALID_ARG;
+  ret::SeqLayout L;
+  L.cu = varlen ? cu_seqlens : nullptr;
+  L.nseq = varlen ? nseq : B;
+  L.T = varlen ? 0 : T;
+  L.Ttot = static_cast<int>(Ttot);
+  L.chunk = 1;
+  L.nslots = 0;
+  return cuda_status(ret::launch_rope(q, k, dt(dtype), q_out, k_out, L, H, d, base,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 ret_status retention_selftest_wait_timeout(ret_stream_t stream) {
   unsigned* err = error_word();
   if (!err) return RET_ERR_CUDA;

@@ -76,6 +76,11 @@ cudaError_t launch_chunkwise_bwd_tc(const void* q, const void* k, const void* v,
                                     ChunkWorkspace ws, void* scratch, int H, int dk_, int dv_,
                                     const HeadDecay& dec, unsigned* err, cudaStream_t s);
 
+// Rotary position encoding of q and k: [Ttot][H][d], positions counted from
+// each sequence's first token; qo/ko may alias q/k.
+cudaError_t launch_rope(const void* q, const void* k, DType t, void* qo, void* ko,
+                        const SeqLayout& L, int H, int d, double base, cudaStream_t s);
+
 // Tn (1..16) tokens per sequence in one pass over the state.
 cudaError_t launch_decode_steps(const void* q, const void* k, const void* v, DType in_t,
                                 float* state, void* o, DType o_t, int N, int Tn, int H, int dk,

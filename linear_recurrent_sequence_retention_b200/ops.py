@@ -41,6 +41,7 @@ EXPORTED = (
     "retention_chunkwise_fwd_static_ws",
     "retention_chunkwise_bwd_workspace_size",
     "retention_chunkwise_bwd",
+    "retention_rope",
     "retention_recurrent_step",
     "retention_recurrent_steps",
     "msr_norm_gate",
@@ -104,6 +105,8 @@ def lib():
     L.retention_chunkwise_bwd.argtypes = [vp, vp, vp, vp, ci, cd, ci, vp, ci, vp, vp,
                                           vp, vp, vp, vp, vp, ctypes.c_size_t,
                                           ci, ci, ci, ci, ci, vp]
+    L.retention_rope.restype = ci
+    L.retention_rope.argtypes = [vp, vp, ci, vp, vp, ctypes.c_double, vp, ci, ci, ci, ci, ci, vp]
     L.retention_recurrent_step.restype = ci
     L.retention_recurrent_step.argtypes = [vp, vp, vp, ci, cd, vp, vp, ci, ci, ci, ci, ci, vp]
     L.retention_recurrent_steps.restype = ci
@@ -392,6 +395,33 @@ def chunkwise_bwd(q, k, v, d_out, gamma, chunk, cu_seqlens=None, state_in=None,
         B, T, H, dk, dv, _stream(stream))
     _check(st, "retention_chunkwise_bwd")
     return (dq, dkk, dvv, dS0) if return_d_state else (dq, dkk, dvv)
+
+
+def rope(q, k, base=10000.0, cu_seqlens=None, q_out=None, k_out=None, stream=None):
+    """Rotary position encoding of q and k ([B,T,H,d], one dtype; packed
+    sequences as in :func:`chunkwise_fwd`).  Returns ``(q_out, k_out)``; pass
+    ``q_out=q, k_out=k`` to rotate in place."""
+    _dev(q, "q")
+    _dev(k, "k")
+    if k.shape != q.shape or k.dtype != q.dtype or q.dim() != 4:
+        raise ValueError("q and k must have one [B,T,H,d] shape and one dtype")
+    B, T, H, d = q.shape
+    nseq = 0
+    if cu_seqlens is not None:
+        _dev(cu_seqlens, "cu_seqlens")
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise ValueError("cu_seqlens must be a 1-D int32 tensor with at least two entries")
+        nseq = cu_seqlens.numel() - 1
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    for t, n in ((q_out, "q_out"), (k_out, "k_out")):
+        _dev(t, n)
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError(f"{n} must match q")
+    st = lib().retention_rope(_ptr(q), _ptr(k), _dt(q), _ptr(q_out), _ptr(k_out), float(base),
+                              _ptr(cu_seqlens), nseq, B, T, H, d, _stream(stream))
+    _check(st, "retention_rope")
+    return q_out, k_out
 
 
 def recurrent_step(q, k, v, gamma, state, out_dtype=torch.float32, out=None, stream=None):
