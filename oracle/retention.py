@@ -82,6 +82,8 @@ __all__ = [
     "msr_backward",
     "msr_backward_varlen",
     "rope",
+    "softmax_features",
+    "rla",
 ]
 
 
@@ -452,3 +454,55 @@ def rope(x, base=10000.0, cu_seqlens=None):
     out[..., 0::2] = x0 * c - x1 * s
     out[..., 1::2] = x0 * s + x1 * c
     return out
+
+
+# ---------------------------------------------------------------------------
+# Residual linear attention (RLA): the linear-attention state read w tokens late
+# ---------------------------------------------------------------------------
+
+def softmax_features(x):
+    """Feature map phi(x) = softmax over the last axis (the head dimension).
+
+    The RAttention page (section "Residual Linear Attention (RLA) 수식") names a
+    feature map phi and calls a softmax-based one the best choice, without a
+    formula; the reading taken is the row softmax of each (token, head) vector.
+    """
+    x = _f64(x)
+    e = np.exp(x - x.max(axis=-1, keepdims=True))
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def rla(q, k, v, window, cu_seqlens=None, features_dtype=None):
+    """Residual linear attention of ``q, k: [B,T,H,dk]``, ``v: [B,T,H,dv]``.
+
+    RAttention page, section "Residual Linear Attention (RLA) 수식": a state
+    without decay, S_t = S_(t-1) + phi(k_t)^T v_t, read w tokens late,
+    o_t = phi(q_t) S_(t-w-1), with S of a position before the sequence = 0
+    (reading: the window w >= 0 counts the tokens the read skips, so o_t sees
+    tokens m <= t - w - 1).  Run per (sequence, head) as the recurrence written
+    on the page.  ``features_dtype`` (e.g. torch.bfloat16) rounds phi(q) and
+    phi(k) to that type first, as a library that stores the mapped tensors in
+    the input dtype does.  Returns ``o [B,T,H,dv]``.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    fq, fk = softmax_features(q), softmax_features(k)
+    if features_dtype is not None:
+        import torch
+        fq = torch.from_numpy(fq).to(features_dtype).double().numpy()
+        fk = torch.from_numpy(fk).to(features_dtype).double().numpy()
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    o = np.zeros((B, T, H, dv))
+    segs = ([(b, 0, T) for b in range(B)] if cu_seqlens is None
+            else [(0, int(a), int(e)) for a, e in zip(cu_seqlens[:-1], cu_seqlens[1:])])
+    for b, a, e in segs:
+        for h in range(H):
+            S = np.zeros((dk, dv))
+            hist = []                                  # S_t for t = a .. e-1
+            for t in range(a, e):
+                S = S + np.outer(fk[b, t, h], v[b, t, h])
+                hist.append(S.copy())
+                src = (t - a) - window - 1             # index of S_(t-w-1) in hist
+                if src >= 0:
+                    o[b, t, h] = fq[b, t, h] @ hist[src]
+    return o
