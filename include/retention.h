@@ -353,6 +353,33 @@ RET_API ret_status retention_rope(const void* q, const void* k, ret_dtype dtype,
                                   int B, int T, int H, int d, ret_stream_t stream);
 
 /*
+ * Residual linear attention (RLA), the variant on the RAttention page (section
+ * "Residual Linear Attention (RLA) 수식"): per sequence and head, a state
+ * without decay read w = `window` tokens late,
+ *     S_t = S_(t-1) + phi(k_t)^T v_t,      o_t = phi(q_t) S_(t-w-1)
+ * (S of a position before the sequence is zero, so o_t = 0 for the first w+1
+ * tokens).  phi is the softmax over the head dimension (the page names a
+ * softmax-based feature map the best choice and gives no formula).  This is
+ * the retention (R) at gamma = 1 on phi(q), phi(k_(t-w-1)), v_(t-w-1), and it
+ * runs on the same kernels: one pass maps and shifts the inputs into the
+ * workspace (stored in in_dtype), then the chunkwise forward.  The local
+ * sliding-window attention the page pairs it with is not part of this call.
+ *   q, k: [B,T,H,dk] in_dtype   v: [B,T,H,dv] in_dtype (packed sequences as
+ *   for retention_chunkwise_fwd)     o: [B,T,H,dv] o_dtype, written in full
+ *   window >= 0; workspace: >= retention_rla_workspace_size(...) bytes,
+ *   256-byte aligned (RET_ERR_WORKSPACE otherwise).
+ * Supported: the shapes of retention_chunkwise_fwd (bf16 on tensor cores, f32
+ * on CUDA cores).
+ */
+RET_API size_t retention_rla_workspace_size(ret_dtype in_dtype, int B, int T, int H, int dk,
+                                            int dv, int nseq);
+RET_API ret_status retention_rla_fwd(const void* q, const void* k, const void* v,
+                                     ret_dtype in_dtype, int window, const int32_t* cu_seqlens,
+                                     int nseq, void* o, ret_dtype o_dtype, void* workspace,
+                                     size_t workspace_bytes, int B, int T, int H, int dk, int dv,
+                                     ret_stream_t stream);
+
+/*
  * Standalone per-head GroupNorm + Swish gate (the epilogue that
  * retention_chunkwise_fwd fuses when given `ng`).
  *   o: [ntok, H, dv] o_dtype     y: [ntok, H, dv] y_dtype (may not alias o)

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "retention.h"
 #include "launch.h"
@@ -499,6 +500,93 @@ ret_status retention_rope(const void* q, const void* k, ret_dtype dtype, void* q
   L.nslots = 0;
   return cuda_status(ret::launch_rope(q, k, dt(dtype), q_out, k_out, L, H, d, base,
                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
+
+namespace {
+
+// The retention inside RLA runs with 256-token chunks on either path (every
+// chunk length gives the same result); the mapped inputs follow its workspace.
+constexpr int kRlaChunk = 256;
+
+struct RlaPlan {
+  ChunkPlan cp;
+  size_t ws_bytes;    // chunk workspace, rounded to 256 B
+  size_t bytes;       // + phi(q), shifted phi(k) and v
+};
+
+ret_status plan_rla(ret_dtype in_dtype, int B, int T, int H, int dk, int dv, int nseq,
+                    const int32_t* cu, RlaPlan* r) {
+  ret_status st = plan_chunkwise(in_dtype, kRlaChunk, B, T, H, dk, dv, nseq, cu, &r->cp);
+  if (st != RET_OK) return st;
+  auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
+  const size_t el = in_dtype == RET_F32 ? 4 : 2;
+  const size_t rows = static_cast<size_t>(r->cp.L.Ttot) * H;
+  r->ws_bytes = r256(r->cp.bytes);
+  r->bytes = r->ws_bytes + 2 * r256(rows * dk * el) + r256(rows * dv * el);
+  return RET_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t retention_rla_workspace_size(ret_dtype in_dtype, int B, int T, int H, int dk, int dv,
+                                    int nseq) {
+  RlaPlan r;
+  if (nseq < 0 || plan_rla(in_dtype, B, T, H, dk, dv, nseq, nullptr, &r) != RET_OK) return 0;
+  return r.bytes;
+}
+
+ret_status retention_rla_fwd(const void* q, const void* k, const void* v, ret_dtype in_dtype,
+                             int window, const int32_t* cu_seqlens, int nseq, void* o,
+                             ret_dtype o_dtype, void* workspace, size_t workspace_bytes, int B,
+                             int T, int H, int dk, int dv, ret_stream_t stream) {
+  const bool varlen = cu_seqlens != nullptr;
+  if (varlen != (nseq > 0) || window < 0 || !dtype_ok(o_dtype)) return RET_ERR_INVALID_ARG;
+  RlaPlan r;
+  ret_status st = plan_rla(in_dtype, B, T, H, dk, dv, varlen ? nseq : 0, cu_seqlens, &r);
+  if (st != RET_OK) return st;
+  if (r.cp.L.Ttot > 0 && (!q || !k || !v || !o)) return RET_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, cu_seqlens};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return RET_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < r.bytes)
+    return RET_ERR_WORKSPACE;
+  std::vector<double> ones(H, 1.0);
+  ret::HeadDecay dec;
+  if (!make_decay(ones.data(), H, &dec)) return RET_ERR_INVALID_ARG;
+  unsigned* err = error_word();
+  if (!err) return RET_ERR_CUDA;
+  char* base = static_cast<char*>(workspace);
+  ret::ChunkWorkspace ws;
+  ws.chunk_base = reinterpret_cast<int32_t*>(base);
+  ws.order = ws.chunk_base + r.cp.L.nseq + 1;
+  ws.states = base + r.cp.meta;
+  ws.nslots = r.cp.slots;
+  auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
+  const size_t el = in_dtype == RET_F32 ? 4 : 2;
+  const size_t rows = static_cast<size_t>(r.cp.L.Ttot) * H;
+  char* qf = base + r.ws_bytes;
+  char* ks = qf + r256(rows * dk * el);
+  char* vs = ks + r256(rows * dk * el);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = ret::launch_chunk_prep(r.cp.L, ws, err, s);
+  if (e == cudaSuccess)
+    e = ret::launch_rla_inputs(q, k, v, dt(in_dtype), qf, ks, vs, r.cp.L, H, dk, dv, window, s);
+  if (e == cudaSuccess) {
+    if (r.cp.tc)
+      e = ret::launch_chunkwise_tc(3, qf, ks, vs, r.cp.L, nullptr, false, nullptr, o, dt(o_dtype),
+                                   nullptr, DType::F32, nullptr, nullptr, 0.f, false, ws, H, dk,
+                                   dv, dec, err, s);
+    else
+      e = ret::launch_chunkwise_simt(3, qf, ks, vs, dt(in_dtype), r.cp.L, nullptr, nullptr, o,
+                                     dt(o_dtype), nullptr, DType::F32, nullptr, nullptr, 0.f,
+                                     false, ws, H, dk, dv, dec, err, s);
+  }
+  return cuda_status(e);
 }
 
 ret_status retention_selftest_wait_timeout(ret_stream_t stream) {

@@ -81,6 +81,12 @@ cudaError_t launch_chunkwise_bwd_tc(const void* q, const void* k, const void* v,
 cudaError_t launch_rope(const void* q, const void* k, DType t, void* qo, void* ko,
                         const SeqLayout& L, int H, int d, double base, cudaStream_t s);
 
+// Inputs of the residual linear attention: qf = phi(q), ks[n] = phi(k[n-w-1]),
+// vs[n] = v[n-w-1] (zero before each sequence), phi = softmax over the head dim.
+cudaError_t launch_rla_inputs(const void* q, const void* k, const void* v, DType t, void* qf,
+                              void* ks, void* vs, const SeqLayout& L, int H, int dk, int dv,
+                              int window, cudaStream_t s);
+
 // Tn (1..16) tokens per sequence in one pass over the state.
 cudaError_t launch_decode_steps(const void* q, const void* k, const void* v, DType in_t,
                                 float* state, void* o, DType o_t, int N, int Tn, int H, int dk,

@@ -42,6 +42,8 @@ EXPORTED = (
     "retention_chunkwise_bwd_workspace_size",
     "retention_chunkwise_bwd",
     "retention_rope",
+    "retention_rla_workspace_size",
+    "retention_rla_fwd",
     "retention_recurrent_step",
     "retention_recurrent_steps",
     "msr_norm_gate",
@@ -107,6 +109,11 @@ def lib():
                                           ci, ci, ci, ci, ci, vp]
     L.retention_rope.restype = ci
     L.retention_rope.argtypes = [vp, vp, ci, vp, vp, ctypes.c_double, vp, ci, ci, ci, ci, ci, vp]
+    L.retention_rla_workspace_size.restype = ctypes.c_size_t
+    L.retention_rla_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, ci]
+    L.retention_rla_fwd.restype = ci
+    L.retention_rla_fwd.argtypes = [vp, vp, vp, ci, ci, vp, ci, vp, ci, vp, ctypes.c_size_t,
+                                    ci, ci, ci, ci, ci, vp]
     L.retention_recurrent_step.restype = ci
     L.retention_recurrent_step.argtypes = [vp, vp, vp, ci, cd, vp, vp, ci, ci, ci, ci, ci, vp]
     L.retention_recurrent_steps.restype = ci
@@ -422,6 +429,39 @@ def rope(q, k, base=10000.0, cu_seqlens=None, q_out=None, k_out=None, stream=Non
                               _ptr(cu_seqlens), nseq, B, T, H, d, _stream(stream))
     _check(st, "retention_rope")
     return q_out, k_out
+
+
+def rla_fwd(q, k, v, window, cu_seqlens=None, out_dtype=None, out=None, workspace=None,
+            stream=None):
+    """Residual linear attention (retention_rla_fwd): o_t = softmax(q_t) S_(t-w-1)
+    with S_t = S_(t-1) + softmax(k_t)^T v_t.  q, k: [B,T,H,dk]; v: [B,T,H,dv];
+    packed sequences as in :func:`chunkwise_fwd`.  Returns o [B,T,H,dv]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    if k.shape != q.shape or v.shape[:3] != q.shape[:3] or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v shapes/dtypes disagree")
+    nseq = 0
+    if cu_seqlens is not None:
+        _dev(cu_seqlens, "cu_seqlens")
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise ValueError("cu_seqlens must be a 1-D int32 tensor with at least two entries")
+        nseq = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty(B, T, H, dv, device=q.device, dtype=out_dtype or q.dtype)
+    _dev(out, "out")
+    need = lib().retention_rla_workspace_size(_dt(q), B, T, H, dk, dv, nseq)
+    if need == 0:
+        raise RetentionError(RET_ERR_UNSUPPORTED, "retention_rla_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    st = lib().retention_rla_fwd(_ptr(q), _ptr(k), _ptr(v), _dt(q), int(window), _ptr(cu_seqlens),
+                                 nseq, _ptr(out), _dt(out), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), B, T, H, dk, dv,
+                                 _stream(stream))
+    _check(st, "retention_rla_fwd")
+    return out
 
 
 def recurrent_step(q, k, v, gamma, state, out_dtype=torch.float32, out=None, stream=None):
