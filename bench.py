@@ -653,6 +653,48 @@ def run_rope(args, world, rank, pk, pk_kind):
             "gpu_launches": reps}
 
 
+def run_rla(args, world, rank, pk, pk_kind):
+    """Residual linear attention, window 512 (the RAttention page's setting), on
+    the B=4, T=2048, H=8, d_k=128, d_v=256 shape with bf16 inputs: one pass
+    mapping and shifting the inputs, then the chunkwise retention at gamma = 1
+    on the tensor-core kernels (256-token chunks)."""
+    from linear_recurrent_sequence_retention_b200 import ops
+    wl = W.WORKLOADS[BACKWARD]
+    dev = torch.device("cuda")
+    B, T, H, dk, dv, w, C = wl.B, wl.T, wl.H, wl.dk, wl.dv, 512, 256
+    q, k, v, _ = W.make_qkvg(B, T, H, dk, dv, "bf16", seed=rank, gate=False, device=dev)
+    out = torch.empty(B, T, H, dv, device=dev, dtype=torch.bfloat16)
+    ws = ops.alloc_workspace(ops.lib().retention_rla_workspace_size(ops.RET_BF16, B, T, H, dk, dv, 0), dev)
+    for _ in range(max(3, args.warmup)):
+        ops.rla_fwd(q, k, v, w, out=out, workspace=ws)
+    reps = 20
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        ops.rla_fwd(q, k, v, w, out=out, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ops.check_device_error()
+    ms = max_over_ranks(e0.elapsed_time(e1) / reps, world)
+    flops = ((C + 1) * (dk + dv) + 4 * dk * dv) * B * T * H
+    ach = flops / (ms / 1e3) / 1e12
+    del q, k, v, out, ws
+    torch.cuda.empty_cache()
+    return {"workload": f"{wl.name} rla window {w}", "ms_per_call": ms,
+            "tokens_per_s": sum_over_ranks(B * T, world) / (ms / 1e3),
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
+                         "peak_source": f"{pk_kind} bf16 (burst)",
+                         "algorithmic_flops_per_call": flops,
+                         "counting": f"per token-head (C+1)(dk+dv) + 4 dk dv, C={C} (the retention "
+                                     "inside; the feature pass is HBM traffic)",
+                         "kernel": "rla_inputs_kernel + state_kernel + output_kernel"},
+            "gpu_launches": 3 * reps}
+
+
 def main():
     global HEADLINE
     ap = argparse.ArgumentParser()
@@ -665,6 +707,7 @@ def main():
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--backward-only", action="store_true", help="backward only (profiling)")
     ap.add_argument("--no-rope", action="store_true")
+    ap.add_argument("--no-rla", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--workload", default=HEADLINE,
@@ -743,6 +786,7 @@ def main():
     dec = None if args.no_decode else run_decode(args, world, rank, pk, pk_kind)
     bwd = None if args.no_backward else run_backward(args, world, rank, pk, pk_kind)
     rope = None if args.no_rope else run_rope(args, world, rank, pk, pk_kind)
+    rla = None if args.no_rla else run_rla(args, world, rank, pk, pk_kind)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(wl, args.cpu_seconds)
@@ -768,12 +812,14 @@ def main():
             "decode": dec,
             "backward": bwd,
             "rope": rope,
+            "rla": rla,
             "e2e": head["e2e"],
             "cpu_baseline": cpu,
             "clocks": head["clocks"],
             "gpu_launches": (head["gpu_launches"] + (dec["gpu_launches"] if dec else 0)
                              + (bwd["gpu_launches"] if bwd else 0)
-                             + (rope["gpu_launches"] if rope else 0)),
+                             + (rope["gpu_launches"] if rope else 0)
+                             + (rla["gpu_launches"] if rla else 0)),
             "arithmetic": "bf16 tensor-core MMAs (tcgen05) with f32 accumulation; the "
                           "carried state, decayed scores and zeta*K enter the MMAs as "
                           "hi+lo bf16 pairs",
