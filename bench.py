@@ -623,7 +623,7 @@ def run_rope(args, world, rank, pk, pk_kind):
     T=8192, H=16, d_k=256, bf16): one streaming pass, HBM-bound (reads q and
     k, writes the rotated copies)."""
     from linear_recurrent_sequence_retention_b200 import ops
-    wl = W.WORKLOADS[HEADLINE]
+    wl = W.WORKLOADS["msr_6p7b_b2_h16_t8192_dk256_dv512_c512"]
     dev = torch.device("cuda")
     q, k, _, _ = W.make_qkvg(wl.B, wl.T, wl.H, wl.dk, 8, "bf16", seed=rank, gate=False, device=dev)
     qo, ko = torch.empty_like(q), torch.empty_like(k)
