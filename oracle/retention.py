@@ -497,12 +497,11 @@ def rla(q, k, v, window, cu_seqlens=None, features_dtype=None):
             else [(0, int(a), int(e)) for a, e in zip(cu_seqlens[:-1], cu_seqlens[1:])])
     for b, a, e in segs:
         for h in range(H):
+            # S_(t-w-1), built by the same recurrence running w+1 tokens behind t
             S = np.zeros((dk, dv))
-            hist = []                                  # S_t for t = a .. e-1
             for t in range(a, e):
-                S = S + np.outer(fk[b, t, h], v[b, t, h])
-                hist.append(S.copy())
-                src = (t - a) - window - 1             # index of S_(t-w-1) in hist
-                if src >= 0:
-                    o[b, t, h] = fq[b, t, h] @ hist[src]
+                m = t - window - 1
+                if m >= a:
+                    S = S + np.outer(fk[b, m, h], v[b, m, h])
+                    o[b, t, h] = fq[b, t, h] @ S
     return o

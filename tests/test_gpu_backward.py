@@ -163,3 +163,24 @@ def test_backward_rejects_unsupported_and_bad_arguments():
     assert ops.chunkwise_bwd_workspace_size(torch.float32, 4, 1, 8, 1, 512, 16) == 0
     assert ops.chunkwise_bwd_workspace_size(torch.float32, 0, 1, 8, 1, 16, 16) == 0
     assert ops.chunkwise_bwd_workspace_size(torch.float32, 4, 1, 8, 1, 16, 16) > 0
+
+
+@pytest.mark.parametrize("path", ["tensor_core", "cuda_core"])
+def test_backward_bench_workload_sampled(path):
+    """The backward at the size bench.py times (B=4, T=2048, H=8, d_k=128, d_v=256,
+    chunk 128, bf16 inputs), checked on two sampled (sequence, head) pairs; the
+    CUDA-core path is taken by passing a final-state gradient."""
+    B, T, H, dk, dv, C = 4, 2048, 8, 128, 256, 128
+    q, k, v, do, _, dS = _inputs(B, T, H, dk, dv, "bf16", seed=77, with_state=True)
+    gam = W.head_gammas(H)
+    use_dS = path == "cuda_core"
+    got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, C,
+                            d_state_out=dS.cuda() if use_dS else None, return_d_state=True)
+    for b, h in ((0, 0), (3, 7)):
+        ref = oracle.retention_backward(W.to_f64(q[b, :, h]), W.to_f64(k[b, :, h]),
+                                        W.to_f64(v[b, :, h]), gam[h], W.to_f64(do[b, :, h]),
+                                        None, dS[b, h].double().numpy() if use_dS else None)
+        for x, y, n in zip((got[0][b, :, h], got[1][b, :, h], got[2][b, :, h], got[3][b, h]),
+                           ref, ("dq", "dk", "dv", "d_state_in")):
+            kind = "bf16" if path == "tensor_core" else "f32"
+            assert_close(W.to_f64(x), y, kind, None, f"{path} b{b} h{h} {n}")

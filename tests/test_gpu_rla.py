@@ -54,3 +54,16 @@ def test_rla_rejects_negative_window():
     q = torch.zeros(1, 8, 1, 64, device="cuda", dtype=torch.bfloat16)
     with pytest.raises(ops.RetentionError):
         ops.rla_fwd(q, q, q, -1)
+
+
+def test_rla_bench_workload_sampled():
+    """RLA at the size bench.py times (B=4, T=2048, H=8, d_k=128, d_v=256, bf16,
+    window 512), checked on two sampled (sequence, head) pairs."""
+    B, T, H, dk, dv, w = 4, 2048, 8, 128, 256, 512
+    q, k, v, _ = W.make_qkvg(B, T, H, dk, dv, "bf16", seed=0, gate=False)
+    out = ops.rla_fwd(q.cuda(), k.cuda(), v.cuda(), w, out_dtype=torch.float32)
+    for b, h in ((0, 0), (3, 7)):
+        sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
+        ref = oracle.rla(W.to_f64(q[sl]), W.to_f64(k[sl]), W.to_f64(v[sl]), w,
+                         features_dtype=torch.bfloat16)
+        assert_close(W.to_f64(out[sl]), ref, "bf16", None, f"rla bench b{b} h{h}")

@@ -76,3 +76,11 @@ def test_rope_rejects_bad_arguments():
     q = torch.zeros(1, 4, 1, 8, device="cuda")
     with pytest.raises(ops.RetentionError):
         ops.rope(q, q.clone(), base=1.0)
+
+
+def test_rope_bench_workload():
+    """The rotary encoding at the size bench.py times: q, k [2, 8192, 16, 256] bf16."""
+    q, k, _, _ = W.make_qkvg(2, 8192, 16, 256, 8, "bf16", seed=0, gate=False)
+    rq, rk = ops.rope(q.cuda(), k.cuda())
+    _check(rq, oracle.rope(W.to_f64(q)), "bf16", "q full size")
+    _check(rk, oracle.rope(W.to_f64(k)), "bf16", "k full size")
