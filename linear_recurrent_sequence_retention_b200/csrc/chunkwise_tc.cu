@@ -500,11 +500,17 @@ struct OutParams {
 template <int DK, int NV>
 struct OutCfg {
   static constexpr uint32_t kQBytes = (DK / 64) * kTallBox;
+  // The gate/output tile (NV/64 boxes of 128 rows x 64 columns) has a buffer of
+  // its own: held through the epilogue tail, it would otherwise pin ring stages
+  // that the next tile's state and key loads are waiting for.
+  static constexpr uint32_t kGateBytes = (NV / 64) * kTallBox;
   // barriers | gamma^d table | GroupNorm pairs passed between the two
   // warpgroups | GroupNorm pairs received from the partner CTA
   static constexpr uint32_t kMiscBytes = 256 + 512 + 1024 + 1024;
-  static constexpr int kStages = static_cast<int>((232448 - kQBytes - kMiscBytes) / kOutStage);
-  static constexpr uint32_t kOffStages = kQBytes;
+  static constexpr int kStages =
+      static_cast<int>((232448 - kQBytes - kGateBytes - kMiscBytes) / kOutStage);
+  static constexpr uint32_t kOffGate = kQBytes;
+  static constexpr uint32_t kOffStages = kOffGate + kGateBytes;
   static constexpr uint32_t kOffMisc = kOffStages + kStages * kOutStage;
   static constexpr uint32_t kSmem = kOffMisc + kMiscBytes;
   // TMEM: two halves of 256 columns used in turn.  Tile number n of a CTA
@@ -608,7 +614,9 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   uint64_t* drain = o_free + 1;
   uint64_t* bar_x = drain + 1;           // the partner's statistics have arrived
   uint64_t* bar_xack = bar_x + 1;        // the partner has read this CTA's statistics
-  uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(bar_xack + 1);
+  uint64_t* g_full = bar_xack + 1;       // the gate tile has landed in the gate buffer
+  uint64_t* g_empty = g_full + 1;        // the epilogue is done with the gate/output buffer
+  uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(g_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_hold + 1);
   float* pow_tab = reinterpret_cast<float*>(smem + C::kOffMisc + 256);    // gamma^d, d < 128
   float* wgx = reinterpret_cast<float*>(smem + C::kOffMisc + 768);        // [128][2]
@@ -621,10 +629,10 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   // K(kb) is kKU units of kKB 64-column boxes (128 keys each)
   constexpr int kKU = DK >= 128 ? DK / 128 : 1;
   constexpr int kKB = DK >= 128 ? 2 : 1;
-  // the gate/output tile: NV/64 boxes of 128 rows x 64 columns, two per stage
+  // the gate/output tile: NV/64 boxes of 128 rows x 64 columns in the gate buffer
   constexpr int kIoBoxes = NV / 64;
-  constexpr int kIoUnits = (kIoBoxes + 1) / 2;
-  // ring units of a tile: its MMA operands, then (when staged) the gate/output tile
+  uint8_t* const gate_buf = smem + C::kOffGate;
+  // ring units of a tile: its MMA operands
   auto mma_units = [&](const OutTile& t) { return (t.inter ? 2 * (DK / 64) : 0) + (t.r + 1) * (kKU + 2); };
   auto io_staged = [&](const OutTile& t) {
     return (p.gated && p.g_tma) || (p.y_tma && t.nrows == kRowsPerTile);
@@ -647,6 +655,8 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     mbar_init(drain, 1);
     mbar_init(bar_x, kWgThreads);
     mbar_init(bar_xack, kWgThreads);
+    mbar_init(g_full, 1);
+    mbar_init(g_empty, 1);
     *abort_flag = 0;
     if ((smem_u32(smem) & 1023u) != 0) {
       *abort_flag = 1;
@@ -683,7 +693,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmS);
       if (p.gated && p.g_tma) tma_prefetch_desc(&tmG);
-      int it = 0, tq = 0;
+      int it = 0, tq = 0, ng = 0;      // ng: staged gate/output tiles so far
       bool ok = true;
       auto next = [&](uint32_t bytes) -> uint8_t* {
         const int st = it % NST;
@@ -737,22 +747,21 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           load_v(kb);
         }
         if (ok && io_staged(t)) {
+          // the gate/output buffer, once the previous staged tile's stores have read it
+          if (!mbar_wait(g_empty, (ng & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
           const bool load_g = p.gated && p.g_tma;
-          for (int u = 0; u < kIoUnits && ok; ++u) {
-            const int nb = (kIoBoxes - 2 * u) >= 2 ? 2 : 1;
-            uint8_t* dst = next(load_g ? nb * kTallBox : 0);
-            if (!dst) { ok = false; break; }
-            if (load_g)
-              for (int bb = 0; bb < nb; ++bb)
-                tma_load_2d(dst + bb * kTallBox, &tmG, &full[it % NST],
-                            t.h * p.dv + NV * part + 64 * (2 * u + bb), t.t0);
-            ++it;
-          }
+          mbar_arrive_expect_tx(g_full, load_g ? kIoBoxes * kTallBox : 0);
+          if (load_g)
+            for (int bb = 0; bb < kIoBoxes; ++bb)
+              tma_load_2d(gate_buf + bb * kTallBox, &tmG, g_full, t.h * p.dv + NV * part + 64 * bb,
+                          t.t0);
+          ++ng;
         }
       }
       if (!ok) {
         // let the copies already issued land before the CTA can exit
         if (tq > 0) mbar_wait_drain(bar_q, (tq - 1) & 1);
+        if (ng > 0) mbar_wait_drain(g_full, (ng - 1) & 1);
         for (int j = 1; j <= NST && it - j >= 0; ++j) {
           const int i2 = it - j;
           mbar_wait_drain(&full[i2 % NST], (i2 / NST) & 1);
@@ -851,7 +860,6 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mma_commit(bar_o);
         sblk += r + 1;
         ++tq;
-        if (io_staged(t)) it += kIoUnits;      // gate/output staging: released by the epilogue
       }
       if (!ok && issued) {
         mma_commit(drain);
@@ -869,7 +877,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const bool wg_leader = (et & 127) == 0;           // first thread of the warpgroup
     constexpr bool kBoxPerWg = kHalf >= 64;           // each warpgroup owns whole boxes
     const uint32_t other = xchg ? (cluster_ctarank() ^ 1u) : 0u;
-    int tq = 0, sblk = 0, ninter = 0, eit = 0;
+    int tq = 0, sblk = 0, ninter = 0, ng = 0;
     bool ok = true;
     while (walk.next(p, cid, t)) {
       // uniform over the 256 epilogue threads: the named barriers below stay matched
@@ -878,12 +886,8 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const int i = r * kRowsPerTile + row;            // row within the chunk
       const uint32_t o_cols = tmem + lane_off + (tq & 1) * C::kHalfCols + wg * kHalf;
       const uint32_t s_t = tmem + lane_off + ((tq & 1) ^ 1) * C::kHalfCols;
-      const int n_mma = mma_units(t);
       const bool staged = io_staged(t);
-      auto io_box = [&](int bx) -> uint8_t* {
-        const int unit = eit + n_mma + bx / 2;
-        return smem + C::kOffStages + (unit % NST) * kOutStage + (bx & 1) * kTallBox;
-      };
+      auto io_box = [&](int bx) -> uint8_t* { return gate_buf + bx * kTallBox; };
       const Decay1 dec(p.dec, t.h);
       // gamma^d for this tile's head (the previous tile's P is complete: every
       // epilogue thread passed the barrier in epi_all above after forming it)
@@ -1054,13 +1058,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const size_t obase = (static_cast<size_t>(t.t0 + row) * p.H + t.h) * p.dv + col0;
       const float shift = -mean_all * rstd;
       bool go = warp_all(ok && !*abort_flag);
-      if (go && staged) {
-        for (int u = 0; u < kIoUnits && go; ++u) {
-          const int unit = eit + n_mma + u;
-          go = mbar_wait(&full[unit % NST], (unit / NST) & 1, abort_flag, p.err);
-        }
-        go = warp_all(go);
-      }
+      if (go && staged) go = warp_all(mbar_wait(g_full, ng & 1, abort_flag, p.err));
       if (go) tc_fence_after();
       for (int j = 0; j < kHalf / 32; ++j) {
         // this piece's 32 columns in the staged gate/output box: box, first 16-byte piece
@@ -1171,10 +1169,9 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       if (out_tma && go && (kBoxPerWg ? wg_leader : et == 0)) tma_store_wait_read();
       if (staged) {
         wg2_sync();
-        if (et == 0)
-          for (int u = 0; u < kIoUnits; ++u) mbar_arrive(&empty[(eit + n_mma + u) % NST]);
+        if (et == 0) mbar_arrive(g_empty);
+        ++ng;
       }
-      eit += n_mma + (staged ? kIoUnits : 0);
       ++tq;
     }
   }
