@@ -131,13 +131,16 @@ cudaError_t decode_vec(const void* q, const void* k, const void* v, float* state
 // t = 0..Tn-1 entering with state S (the recurrence above, unrolled):
 //     o_t = gamma^(t+1) q_t S + sum_{j<=t} gamma^(t-j) (q_t . k_j) v_j
 //     S'  = gamma^Tn S + sum_j gamma^(Tn-1-j) k_j^T v_j
-// so the state is read and written once for all Tn tokens.  A block owns 128
-// columns (32 lanes x float4) of one (n, h) state; every thread walks groups
-// of 4 consecutive rows (warps take groups w, w+8, ...), folding each row into
-// the Tn output partial sums and updating it in place.  The small Tn x Tn
-// score block and the per-token factors live in shared memory.
+// so the state is read and written once for all Tn tokens.  A block owns up to
+// 512 columns of one (n, h) state: warp w the 64 columns 64w.., two per lane,
+// over all dk rows, so a warp's output sums need no other warp.  Every thread
+// walks groups of 4 rows (the next group's loads in flight while this one is
+// folded in), folds each row into its Tn output partial sums and updates it in
+// place.  q_t, k_j (with their decay factors), the block's v columns and the
+// small Tn x Tn score block live in shared memory.
 // ---------------------------------------------------------------------------
-constexpr int kMultiCols = 128;
+constexpr int kMultiCols = 512;                 // columns per block
+constexpr int kMultiWarpCols = 64;              // columns per warp (2 per lane)
 
 // Four consecutive elements as floats (8-byte aligned bf16, 16-byte aligned f32).
 __device__ __forceinline__ float4 ld4(const __nv_bfloat16* p) {
@@ -155,56 +158,33 @@ decode_multi_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   extern __shared__ __align__(16) float sm[];
   float* qf = sm;                          // [MAXT][dk]  q_t, then q_t gamma^(t+1)
   float* kw = qf + MAXT * dk;              // [MAXT][dk]  k_j, then k_j gamma^(Tn-1-j)
-  float* vs = kw + MAXT * dk;              // [MAXT][128] v_j of this block's columns
+  float* vs = kw + MAXT * dk;              // [MAXT][512] v_j of this block's columns
   float* A = vs + MAXT * kMultiCols;       // [MAXT][MAXT] (q_t . k_j) gamma^(t-j), j <= t
-  float* red = A + MAXT * MAXT;            // [kWarps][MAXT][128] partial sums of q_t S
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int h = blockIdx.y, n = blockIdx.z;
   const int cblk = blockIdx.x * kMultiCols;
-  const int col0 = cblk + lane * 4;
-  const bool colok = col0 < dv;            // 4 divides dv
+  const int ncols = min(kMultiCols, dv - cblk);
+  const int wc = warp * kMultiWarpCols + lane * 2;     // this thread's first column in the block
+  const bool colok = wc < ncols;                       // 4 divides dv, so both columns are in
   const Decay1 dg(dec, h);
 
-  // q, k of all tokens and v of this block's columns, four elements per load
-  // (dk and dv are multiples of 4), every load of a thread issued before any
-  // is used
-  {
-    constexpr int kPer = (MAXT * 512 / 4 + kWarps * 32 - 1) / (kWarps * 32);   // dk <= 512
-    float4 aq[kPer], ak[kPer];
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int idx4 = (threadIdx.x + u * kWarps * 32) * 4;
-      const int t = idx4 / dk, i = idx4 % dk;
-      aq[u] = ak[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (idx4 < MAXT * dk && t < Tn) {
-        const size_t row = (static_cast<size_t>(n) * Tn + t) * H + h;
-        aq[u] = ld4(q + row * dk + i);
-        ak[u] = ld4(k + row * dk + i);
-      }
+  // q, k of all tokens and v of this block's columns into shared memory
+  for (int idx4 = threadIdx.x * 4; idx4 < MAXT * dk; idx4 += kWarps * 32 * 4) {
+    const int t = idx4 / dk, i = idx4 % dk;
+    float4 aq = make_float4(0.f, 0.f, 0.f, 0.f), ak = aq;
+    if (t < Tn) {
+      const size_t row = (static_cast<size_t>(n) * Tn + t) * H + h;
+      aq = ld4(q + row * dk + i);
+      ak = ld4(k + row * dk + i);
     }
-    constexpr int kPerV = (MAXT * kMultiCols / 4 + kWarps * 32 - 1) / (kWarps * 32);
-    float4 av[kPerV];
-#pragma unroll
-    for (int u = 0; u < kPerV; ++u) {
-      const int idx4 = (threadIdx.x + u * kWarps * 32) * 4;
-      const int t = idx4 / kMultiCols, c = cblk + idx4 % kMultiCols;
-      av[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (idx4 < MAXT * kMultiCols && t < Tn && c < dv)
-        av[u] = ld4(v + ((static_cast<size_t>(n) * Tn + t) * H + h) * dv + c);
-    }
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int idx4 = (threadIdx.x + u * kWarps * 32) * 4;
-      if (idx4 < MAXT * dk) {
-        *reinterpret_cast<float4*>(qf + idx4) = aq[u];
-        *reinterpret_cast<float4*>(kw + idx4) = ak[u];
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kPerV; ++u) {
-      const int idx4 = (threadIdx.x + u * kWarps * 32) * 4;
-      if (idx4 < MAXT * kMultiCols) *reinterpret_cast<float4*>(vs + idx4) = av[u];
-    }
+    *reinterpret_cast<float4*>(qf + idx4) = aq;
+    *reinterpret_cast<float4*>(kw + idx4) = ak;
+  }
+  for (int idx4 = threadIdx.x * 4; idx4 < MAXT * kMultiCols; idx4 += kWarps * 32 * 4) {
+    const int t = idx4 / kMultiCols, c = idx4 % kMultiCols;
+    float4 av = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t < Tn && c < ncols) av = ld4(v + ((static_cast<size_t>(n) * Tn + t) * H + h) * dv + cblk + c);
+    *reinterpret_cast<float4*>(vs + idx4) = av;
   }
   __syncthreads();
   for (int idx = warp; idx < MAXT * MAXT; idx += kWarps) {   // one (t, j) per warp
@@ -225,79 +205,68 @@ decode_multi_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     kw[idx] *= t < Tn ? dg.pow(Tn - 1 - t) : 0.f;
   }
   __syncthreads();
+  if (!colok) return;
 
-  float acc[MAXT][4];
+  float acc[MAXT][2];
 #pragma unroll
-  for (int t = 0; t < MAXT; ++t)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+  for (int t = 0; t < MAXT; ++t) acc[t][0] = acc[t][1] = 0.f;
   const float gT = dg.pow(Tn);
-  float* S = state + (static_cast<size_t>(n) * H + h) * dk * dv;
-  if (colok) {
-    // rows g0..g0+3 per iteration; the next group's rows are already in flight
-    // while this group is folded in
-    float4 xn[4];
-    if (warp * 4 < dk) {
+  float* S = state + (static_cast<size_t>(n) * H + h) * dk * dv + cblk + wc;
+  // rows g0..g0+3 per iteration; the next group's rows are already in flight
+  // while this group is folded in
+  float2 xn[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) xn[r] = __ldcs(reinterpret_cast<const float2*>(S + static_cast<size_t>(r) * dv));
+  for (int g0 = 0; g0 < dk; g0 += 4) {
+    float2 x[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) x[r] = xn[r];
+    if (g0 + 4 < dk) {
 #pragma unroll
       for (int r = 0; r < 4; ++r)
-        xn[r] = __ldcs(reinterpret_cast<const float4*>(S + static_cast<size_t>(warp * 4 + r) * dv + col0));
+        xn[r] = __ldcs(reinterpret_cast<const float2*>(S + static_cast<size_t>(g0 + 4 + r) * dv));
     }
-    for (int g0 = warp * 4; g0 < dk; g0 += kWarps * 4) {
-      float4 x[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) x[r] = xn[r];
-      if (g0 + kWarps * 4 < dk) {
+    for (int t = 0; t < MAXT; ++t) {
+      const float4 qa = *reinterpret_cast<const float4*>(qf + t * dk + g0);
+      const float qr[4] = {qa.x, qa.y, qa.z, qa.w};
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
-          xn[r] = __ldcs(reinterpret_cast<const float4*>(S + static_cast<size_t>(g0 + kWarps * 4 + r) * dv + col0));
+      for (int r = 0; r < 4; ++r) {
+        acc[t][0] = fmaf(qr[r], x[r].x, acc[t][0]);
+        acc[t][1] = fmaf(qr[r], x[r].y, acc[t][1]);
       }
-#pragma unroll
-      for (int t = 0; t < MAXT; ++t) {
-        const float4 qa = *reinterpret_cast<const float4*>(qf + t * dk + g0);
-        const float qr[4] = {qa.x, qa.y, qa.z, qa.w};
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          acc[t][0] = fmaf(qr[r], x[r].x, acc[t][0]);
-          acc[t][1] = fmaf(qr[r], x[r].y, acc[t][1]);
-          acc[t][2] = fmaf(qr[r], x[r].z, acc[t][2]);
-          acc[t][3] = fmaf(qr[r], x[r].w, acc[t][3]);
-        }
-      }
-      float4 y[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-        y[r] = make_float4(gT * x[r].x, gT * x[r].y, gT * x[r].z, gT * x[r].w);
-#pragma unroll
-      for (int j = 0; j < MAXT; ++j) {
-        const float4 ka = *reinterpret_cast<const float4*>(kw + j * dk + g0);
-        const float4 vj = *reinterpret_cast<const float4*>(vs + j * kMultiCols + lane * 4);
-        const float kr[4] = {ka.x, ka.y, ka.z, ka.w};
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          y[r].x = fmaf(kr[r], vj.x, y[r].x);
-          y[r].y = fmaf(kr[r], vj.y, y[r].y);
-          y[r].z = fmaf(kr[r], vj.z, y[r].z);
-          y[r].w = fmaf(kr[r], vj.w, y[r].w);
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-        __stcs(reinterpret_cast<float4*>(S + static_cast<size_t>(g0 + r) * dv + col0), y[r]);
     }
+    float2 y[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) y[r] = make_float2(gT * x[r].x, gT * x[r].y);
+#pragma unroll
+    for (int j = 0; j < MAXT; ++j) {
+      const float4 ka = *reinterpret_cast<const float4*>(kw + j * dk + g0);
+      const float2 vj = *reinterpret_cast<const float2*>(vs + j * kMultiCols + wc);
+      const float kr[4] = {ka.x, ka.y, ka.z, ka.w};
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        y[r].x = fmaf(kr[r], vj.x, y[r].x);
+        y[r].y = fmaf(kr[r], vj.y, y[r].y);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+      __stcs(reinterpret_cast<float2*>(S + static_cast<size_t>(g0 + r) * dv), y[r]);
   }
+  // o_t = (gamma^(t+1) q_t S) + sum_{j<=t} A[t][j] v_j for this thread's two columns
 #pragma unroll
-  for (int t = 0; t < MAXT; ++t)
-    *reinterpret_cast<float4*>(red + (warp * MAXT + t) * kMultiCols + lane * 4) =
-        make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < MAXT * kMultiCols; idx += kWarps * 32) {
-    const int t = idx / kMultiCols, c = idx % kMultiCols;
-    if (t >= Tn || cblk + c >= dv) continue;
-    float sum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) sum += red[(w * MAXT + t) * kMultiCols + c];
-    for (int j = 0; j <= t; ++j) sum = fmaf(A[t * MAXT + j], vs[j * kMultiCols + c], sum);
-    Io<To>::st(o, ((static_cast<size_t>(n) * Tn + t) * H + h) * dv + cblk + c, sum);
+  for (int t = 0; t < MAXT; ++t) {
+    if (t >= Tn) break;
+    float s0 = acc[t][0], s1 = acc[t][1];
+    for (int j = 0; j <= t; ++j) {
+      const float2 vj = *reinterpret_cast<const float2*>(vs + j * kMultiCols + wc);
+      s0 = fmaf(A[t * MAXT + j], vj.x, s0);
+      s1 = fmaf(A[t * MAXT + j], vj.y, s1);
+    }
+    const size_t ob = ((static_cast<size_t>(n) * Tn + t) * H + h) * dv + cblk + wc;
+    Io<To>::st(o, ob, s0);
+    Io<To>::st(o, ob + 1, s1);
   }
 }
 
@@ -305,8 +274,7 @@ template <typename Tin, typename To, int MAXT>
 cudaError_t decode_multi_typed(const void* q, const void* k, const void* v, float* state,
                                void* o, int N, int Tn, int H, int dk, int dv,
                                const HeadDecay& dec, cudaStream_t s) {
-  const size_t smem = sizeof(float) * (2 * MAXT * dk + MAXT * kMultiCols + MAXT * MAXT +
-                                       kWarps * MAXT * kMultiCols);
+  const size_t smem = sizeof(float) * (2 * MAXT * dk + MAXT * kMultiCols + MAXT * MAXT);
   auto kern = decode_multi_kernel<Tin, To, MAXT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
