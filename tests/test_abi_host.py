@@ -139,3 +139,60 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ops, "LIBRARY_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         ops.lib()
+
+
+def test_backward_workspace_size_and_bad_arguments():
+    ops, L = _lib()
+    ws = L.retention_chunkwise_bwd_workspace_size
+    # CUDA-core path: meta (256 B) + two fp32 states per chunk
+    assert ws(0, 16, 1, 64, 2, 16, 16, 0) == 256 + 2 * 4 * 2 * 16 * 16 * 4
+    # bf16 with heads 64/128/256 may take the tensor-core path: at least as large
+    assert ws(1, 128, 1, 256, 2, 64, 64, 0) >= 256 + 2 * 2 * 2 * 64 * 64 * 4
+    assert ws(0, 0, 1, 64, 2, 16, 16, 0) == 0            # chunk < 1
+    assert ws(0, 16, 1, 64, 2, 300, 16, 0) == 0          # heads beyond 256
+    assert ws(0, 16, 1, 64, 65, 16, 16, 0) == 0          # H > 64
+    f = L.retention_chunkwise_bwd
+
+    def call(q=FAKE, gamma=None, ws_ptr=FAKE, ws_bytes=1 << 24, cu=None, nseq=0, dq=FAKE):
+        gamma = gamma or _g(0.5, 0.9)
+        return f(q, FAKE, FAKE, FAKE, 0, gamma, 16, cu, nseq, None, None, dq, FAKE, FAKE, None,
+                 ws_ptr, ws_bytes, 1, 64, 2, 16, 16, None)
+    assert call(q=None) == ops.RET_ERR_INVALID_ARG
+    assert call(dq=None) == ops.RET_ERR_INVALID_ARG
+    assert call(q=MISALIGNED) == ops.RET_ERR_INVALID_ARG
+    assert call(gamma=_g(0.5, 1.01)) == ops.RET_ERR_INVALID_ARG
+    assert call(cu=FAKE, nseq=0) == ops.RET_ERR_INVALID_ARG
+    assert call(ws_bytes=100) == ops.RET_ERR_WORKSPACE
+    assert call(ws_ptr=ctypes.c_void_p(0x10010)) == ops.RET_ERR_WORKSPACE
+
+
+def test_rope_rejects_bad_arguments():
+    ops, L = _lib()
+    f = L.retention_rope
+
+    def call(q=FAKE, d=16, base=10000.0, cu=None, nseq=0, dtype=1):
+        return f(q, FAKE, dtype, FAKE, FAKE, base, cu, nseq, 1, 8, 2, d, None)
+    assert call(d=7) == ops.RET_ERR_INVALID_ARG          # odd head dimension
+    assert call(base=1.0) == ops.RET_ERR_INVALID_ARG
+    assert call(base=float("inf")) == ops.RET_ERR_INVALID_ARG
+    assert call(q=None) == ops.RET_ERR_INVALID_ARG
+    assert call(q=MISALIGNED) == ops.RET_ERR_INVALID_ARG
+    assert call(cu=None, nseq=2) == ops.RET_ERR_INVALID_ARG
+    assert call(dtype=5) == ops.RET_ERR_INVALID_ARG
+
+
+def test_rla_workspace_size_and_bad_arguments():
+    ops, L = _lib()
+    ws = L.retention_rla_workspace_size
+    assert ws(0, 1, 64, 2, 16, 16, 0) > 0
+    assert ws(0, 1, 64, 2, 300, 16, 0) == 0              # f32 path: heads up to 256
+    assert ws(1, 1, 64, 2, 100, 128, 0) == 0             # bf16 path: d_k in {64, 128, 256}
+    f = L.retention_rla_fwd
+
+    def call(window=4, ws_ptr=FAKE, ws_bytes=1 << 24, q=FAKE):
+        return f(q, FAKE, FAKE, 0, window, None, 0, FAKE, 0, ws_ptr, ws_bytes, 1, 64, 2, 16, 16,
+                 None)
+    assert call(window=-1) == ops.RET_ERR_INVALID_ARG
+    assert call(q=None) == ops.RET_ERR_INVALID_ARG
+    assert call(ws_bytes=100) == ops.RET_ERR_WORKSPACE
+    assert call(ws_ptr=None) == ops.RET_ERR_WORKSPACE
