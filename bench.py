@@ -550,11 +550,11 @@ def fp32_fma_peak_tflops(pk):
 
 def run_backward(args, world, rank, pk, pk_kind):
     """The chunkwise backward (dQ, dK, dV and the initial-state gradient from
-    dO) on the B=4, T=2048, H=8, d_k=128, d_v=256, chunk-128 workload with
-    bf16 inputs.  Without a final-state gradient it runs on the tensor-core
-    forward kernels (three retentions, bf16 MMAs, roofline: the bf16 tensor
-    peak); with one (`cuda_core` below) on CUDA cores in float32 (roofline: the
-    float32 FMA peak)."""
+    dO) on the B=4, T=2048, H=8, d_k=128, d_v=256, chunk-128 workload.  bf16
+    inputs run on the tensor-core forward kernels (three retentions, bf16 MMAs,
+    roofline: the bf16 tensor peak), timed without and with a final-state
+    gradient; the same values as float32 inputs (`cuda_core` below) run on CUDA
+    cores in float32 (roofline: the float32 FMA peak)."""
     from linear_recurrent_sequence_retention_b200 import ops
     wl = W.WORKLOADS[BACKWARD]
     dev = torch.device("cuda")
@@ -565,24 +565,23 @@ def run_backward(args, world, rank, pk, pk_kind):
     do = torch.randn(B, T, H, dv, generator=gen, device=dev).to(torch.bfloat16)
     dS = torch.randn(B, H, dk, dv, generator=gen, device=dev)
     gam = W.head_gammas(H)
-    ws = ops.alloc_workspace(ops.chunkwise_bwd_workspace_size(torch.bfloat16, C, B, T, H, dk, dv), dev)
+    ws = ops.alloc_workspace(max(ops.chunkwise_bwd_workspace_size(dt, C, B, T, H, dk, dv)
+                                 for dt in (torch.bfloat16, torch.float32)), dev)
     # per token-head: three intra-chunk causal products (C+1)(dk+dv) each, three
     # state reads 2 dk dv each, two state recurrences 2 dk dv each
     flops = (3 * (C + 1) * (dk + dv) + 10 * dk * dv) * B * T * H
     tokens = sum_over_ranks(B * T, world)
 
-    def timed(dstate, reps):
+    def timed(dstate, reps, x=(q, k, v, do)):
         for _ in range(max(3, args.warmup)):
-            ops.chunkwise_bwd(q, k, v, do, gam, C, d_state_out=dstate, return_d_state=True,
-                              workspace=ws)
+            ops.chunkwise_bwd(*x, gam, C, d_state_out=dstate, return_d_state=True, workspace=ws)
         ops.check_device_error()
         barrier(world)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(reps):
-            ops.chunkwise_bwd(q, k, v, do, gam, C, d_state_out=dstate, return_d_state=True,
-                              workspace=ws)
+            ops.chunkwise_bwd(*x, gam, C, d_state_out=dstate, return_d_state=True, workspace=ws)
         e1.record()
         torch.cuda.synchronize()
         barrier(world)
@@ -591,7 +590,10 @@ def run_backward(args, world, rank, pk, pk_kind):
 
     reps_tc, reps_cc = 20, 5
     ms_tc = timed(None, reps_tc)
-    ms_cc = timed(dS, reps_cc)
+    ms_tc_ds = timed(dS, reps_tc)
+    x32 = tuple(t.float() for t in (q, k, v, do))
+    ms_cc = timed(dS, reps_cc, x32)
+    del x32
     ach_tc = flops / (ms_tc / 1e3) / 1e12
     ach_cc = flops / (ms_cc / 1e3) / 1e12
     peak_tc = pk["bf16_tflops"]
@@ -600,6 +602,7 @@ def run_backward(args, world, rank, pk, pk_kind):
     torch.cuda.empty_cache()
     return {"workload": wl.name, "input_dtype": "bf16", "ms_per_call": ms_tc,
             "tokens_per_s": tokens / (ms_tc / 1e3),
+            "ms_per_call_with_d_state_out": ms_tc_ds,
             "path": "tensor cores: three forward retentions (dQ; dV and dK on the sequences "
                     "read backwards) plus token-reversal copies",
             "roofline": {"bound": "tensor", "achieved": ach_tc, "peak": peak_tc,
@@ -608,14 +611,15 @@ def run_backward(args, world, rank, pk, pk_kind):
                          "algorithmic_flops_per_call": flops,
                          "counting": f"per token-head 3 (C+1)(dk+dv) + 10 dk dv, C={C}",
                          "kernel": "state_kernel + output_kernel (x3), flip_tokens_kernel"},
-            "cuda_core": {"with": "a final-state gradient (d_state_out)", "ms_per_call": ms_cc,
+            "cuda_core": {"with": "float32 inputs (the same values) and a final-state gradient",
+                          "ms_per_call": ms_cc,
                           "tokens_per_s": tokens / (ms_cc / 1e3),
                           "roofline": {"bound": "alu", "achieved": ach_cc, "peak": peak_cc,
                                        "unit": "TFLOP/s", "frac": ach_cc / peak_cc,
                                        "peak_source": "derived: SMs x 128 FP32 lanes x 2 flops "
                                                       "x max SM clock",
                                        "kernel": "chunk_grad_simt_kernel + chunk_state_simt_kernel"}},
-            "gpu_launches": 13 * reps_tc + 5 * reps_cc}
+            "gpu_launches": 13 * reps_tc + 15 * reps_tc + 5 * reps_cc}
 
 
 def run_rope(args, world, rank, pk, pk_kind):

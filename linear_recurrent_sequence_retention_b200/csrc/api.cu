@@ -437,7 +437,12 @@ ret_status retention_chunkwise_bwd(const void* q, const void* k, const void* v, 
     if (ptr && !aligned16(ptr)) return RET_ERR_INVALID_ARG;
   ret::HeadDecay dec;
   if (!make_decay(gamma, H, &dec)) return RET_ERR_INVALID_ARG;
-  const bool use_tc = p.tc_ok && d_state_out == nullptr;
+  // a final-state gradient enters the tensor-core path as dS_T / gamma: every
+  // gamma must be 0 (handled apart) or not so small that the quotient overflows
+  bool gam_ok = true;
+  for (int h = 0; h < H; ++h)
+    if (gamma[h] != 0.0 && gamma[h] < 1e-6) gam_ok = false;
+  const bool use_tc = p.tc_ok && (d_state_out == nullptr || gam_ok);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
       workspace_bytes < (use_tc ? p.tc_bytes : p.bytes))
     return RET_ERR_WORKSPACE;
@@ -453,8 +458,9 @@ ret_status retention_chunkwise_bwd(const void* q, const void* k, const void* v, 
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = ret::launch_chunk_prep(p.Ltc, tw, err, s);
     if (e == cudaSuccess)
-      e = ret::launch_chunkwise_bwd_tc(q, k, v, d_out, p.Ltc, state_in, dq, dk, dv, d_state_in, tw,
-                                       base + p.meta + p.tc_states, H, dk_, dv_, dec, err, s);
+      e = ret::launch_chunkwise_bwd_tc(q, k, v, d_out, p.Ltc, state_in, d_state_out, dq, dk, dv,
+                                       d_state_in, tw, base + p.meta + p.tc_states, H, dk_, dv_,
+                                       dec, err, s);
     return cuda_status(e);
   }
   ret::ChunkWorkspace fw;

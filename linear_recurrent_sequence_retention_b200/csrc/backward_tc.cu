@@ -11,6 +11,13 @@
 //          = forward(q = V, k = dO, v = Q) on every sequence read backwards
 //     dS0  = sum_n gamma^(n+1) q_n^T dO_n
 //          = gamma * (final state of the backwards (k = Q, v = dO) pass)
+// A final-state gradient dS_T adds gamma^(T-1-m) k_m dS_T to dv_m and
+// gamma^(T-1-m) v_m dS_T^T to dk_m: at the backwards position m' = T-1-m that
+// is gamma^(m') k dS_T, which the forward's read of an initial state,
+// gamma^(m'+1) q S_in, gives with S_in = dS_T / gamma (and its transpose for
+// dK); the backwards pass's final state then also carries gamma^(T-1) dS_T, so
+// dS0 = gamma * final still holds.  Heads with gamma = 0 take S_in = 0 and a
+// fix-up of the last token of each sequence (the only term left, gamma^0).
 // (reading a sequence backwards turns "n >= m" into "n' <= m'" with the same
 // distance).  This file holds the three small streaming kernels the
 // composition needs (reverse the tokens of every sequence, transpose the
@@ -58,6 +65,52 @@ __global__ void transpose_states_kernel(const float* __restrict__ in, float* __r
   }
 }
 
+// out[s][h] = x[s][h] / gamma_h (zero where gamma_h = 0) over [nseq*H][dk*dv].
+__global__ void state_over_gamma_kernel(const float* __restrict__ x, float* __restrict__ out, int H,
+                                        size_t per, HeadDecay dec) {
+  const int mat = blockIdx.y;
+  const float gm = dec.gamma[mat % H];
+  const float inv = gm > 0.f ? 1.0f / gm : 0.f;
+  const float* a = x + static_cast<size_t>(mat) * per;
+  float* b = out + static_cast<size_t>(mat) * per;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < per;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    b[i] = a[i] * inv;
+}
+
+// Heads with gamma = 0: the final-state gradient reaches only the last token of
+// each sequence, dv += k dS_T and dk += dS_T v (and an empty sequence passes it
+// to d_state_in).  One block per (sequence, head).
+__global__ void zero_gamma_fixup_kernel(const __nv_bfloat16* __restrict__ k,
+                                        const __nv_bfloat16* __restrict__ v,
+                                        const float* __restrict__ dS, float* __restrict__ dk,
+                                        float* __restrict__ dv, float* __restrict__ d_state_in,
+                                        SeqLayout L, int H, int dk_, int dv_, HeadDecay dec) {
+  const int s = blockIdx.x, h = blockIdx.y;
+  if (!((dec.zero_mask >> h) & 1ull)) return;
+  int a, b;
+  seq_bounds(L, s, a, b);
+  const float* M = dS + (static_cast<size_t>(s) * H + h) * dk_ * dv_;
+  if (b == a) {
+    if (d_state_in) {
+      float* out = d_state_in + (static_cast<size_t>(s) * H + h) * dk_ * dv_;
+      for (int i = threadIdx.x; i < dk_ * dv_; i += blockDim.x) out[i] = M[i];
+    }
+    return;
+  }
+  const size_t last = static_cast<size_t>(b - 1) * H + h;
+  for (int c = threadIdx.x; c < dv_; c += blockDim.x) {
+    float x = 0.f;
+    for (int i = 0; i < dk_; ++i) x = fmaf(__bfloat162float(k[last * dk_ + i]), M[static_cast<size_t>(i) * dv_ + c], x);
+    dv[last * dv_ + c] += x;
+  }
+  for (int i = threadIdx.x; i < dk_; i += blockDim.x) {
+    float x = 0.f;
+    for (int c = 0; c < dv_; ++c) x = fmaf(M[static_cast<size_t>(i) * dv_ + c], __bfloat162float(v[last * dv_ + c]), x);
+    dk[last * dk_ + i] += x;
+  }
+}
+
 // x[s][h] *= gamma_h over [nmat = nseq*H][dk*dv].
 __global__ void scale_states_kernel(float* __restrict__ x, int H, size_t per, HeadDecay dec) {
   const int mat = blockIdx.y;
@@ -81,16 +134,18 @@ cudaError_t flip(const void* src, void* dst, const SeqLayout& L, size_t row_byte
 size_t chunkwise_bwd_tc_scratch_bytes(const SeqLayout& L, int H, int dk, int dv) {
   const size_t T = static_cast<size_t>(L.Ttot);
   auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
+  const size_t st = r256(static_cast<size_t>(L.nseq) * H * dk * dv * 4);
   return 2 * r256(T * H * dk * 2) + 2 * r256(T * H * dv * 2)      // q, k, v, dO read backwards
          + r256(T * H * dk * 4) + r256(T * H * dv * 4)             // dK, dV of the backwards passes
-         + r256(static_cast<size_t>(L.nseq) * H * dk * dv * 4);    // S0^T
+         + 3 * st;                                                 // S0^T, dS_T / gamma and its transpose
 }
 
 cudaError_t launch_chunkwise_bwd_tc(const void* q, const void* k, const void* v,
                                     const void* d_out, const SeqLayout& L, const float* state_in,
-                                    float* dq, float* dk, float* dv, float* d_state_in,
-                                    ChunkWorkspace ws, void* scratch, int H, int dk_, int dv_,
-                                    const HeadDecay& dec, unsigned* err, cudaStream_t s) {
+                                    const float* d_state_out, float* dq, float* dk, float* dv,
+                                    float* d_state_in, ChunkWorkspace ws, void* scratch, int H,
+                                    int dk_, int dv_, const HeadDecay& dec, unsigned* err,
+                                    cudaStream_t s) {
   const size_t T = static_cast<size_t>(L.Ttot);
   auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
   char* p = static_cast<char*>(scratch);
@@ -100,7 +155,10 @@ cudaError_t launch_chunkwise_bwd_tc(const void* q, const void* k, const void* v,
   void* do_r = p; p += r256(T * H * dv_ * 2);
   float* dk_r = reinterpret_cast<float*>(p); p += r256(T * H * dk_ * 4);
   float* dv_r = reinterpret_cast<float*>(p); p += r256(T * H * dv_ * 4);
-  float* s0t = reinterpret_cast<float*>(p);
+  const size_t st_bytes = r256(static_cast<size_t>(L.nseq) * H * dk_ * dv_ * 4);
+  float* s0t = reinterpret_cast<float*>(p); p += st_bytes;
+  float* sv = reinterpret_cast<float*>(p);  p += st_bytes;     // dS_T / gamma      [dk][dv]
+  float* svt = reinterpret_cast<float*>(p);                     // its transpose     [dv][dk]
   const size_t rq = static_cast<size_t>(H) * dk_ * 2, rv = static_cast<size_t>(H) * dv_ * 2;
   cudaError_t e = flip(q, q_r, L, rq, s);
   if (e == cudaSuccess) e = flip(k, k_r, L, rq, s);
@@ -111,8 +169,20 @@ cudaError_t launch_chunkwise_bwd_tc(const void* q, const void* k, const void* v,
     transpose_states_kernel<<<grid, dim3(32, 8), 0, s>>>(state_in, s0t, dk_, dv_);
     e = cudaGetLastError();
   }
+  const size_t per = static_cast<size_t>(dk_) * dv_;
+  if (e == cudaSuccess && d_state_out) {
+    dim3 grid(static_cast<unsigned>((per + 1023) / 1024), static_cast<unsigned>(L.nseq) * H);
+    state_over_gamma_kernel<<<grid, 256, 0, s>>>(d_state_out, sv, H, per, dec);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) {
+      dim3 tg((dv_ + 31) / 32, (dk_ + 31) / 32, static_cast<unsigned>(L.nseq) * H);
+      transpose_states_kernel<<<tg, dim3(32, 8), 0, s>>>(sv, svt, dk_, dv_);
+      e = cudaGetLastError();
+    }
+  }
   if (e != cudaSuccess) return e;
   const DType F = DType::F32;
+  const bool ds = d_state_out != nullptr;
   // dQ: forward(q = dO, k = V, v = K) from S0^T
   e = launch_chunkwise_tc(3, d_out, v, k, L, state_in ? s0t : nullptr, state_in != nullptr,
                           nullptr, dq, F, nullptr, F, nullptr, nullptr, 0.f, false, ws, H, dv_, dk_,
@@ -120,18 +190,23 @@ cudaError_t launch_chunkwise_bwd_tc(const void* q, const void* k, const void* v,
   // dV on the sequences read backwards: forward(q = K, k = Q, v = dO); its final
   // state is sum_n gamma^n q_n^T dO_n, the initial-state gradient before one gamma
   if (e == cudaSuccess)
-    e = launch_chunkwise_tc(3, k_r, q_r, do_r, L, nullptr, false, d_state_in, dv_r, F, nullptr, F,
-                            nullptr, nullptr, 0.f, false, ws, H, dk_, dv_, dec, err, s);
+    e = launch_chunkwise_tc(3, k_r, q_r, do_r, L, ds ? sv : nullptr, ds, d_state_in, dv_r, F,
+                            nullptr, F, nullptr, nullptr, 0.f, false, ws, H, dk_, dv_, dec, err, s);
   // dK on the sequences read backwards: forward(q = V, k = dO, v = Q)
   if (e == cudaSuccess)
-    e = launch_chunkwise_tc(3, v_r, do_r, q_r, L, nullptr, false, nullptr, dk_r, F, nullptr, F,
-                            nullptr, nullptr, 0.f, false, ws, H, dv_, dk_, dec, err, s);
+    e = launch_chunkwise_tc(3, v_r, do_r, q_r, L, ds ? svt : nullptr, ds, nullptr, dk_r, F,
+                            nullptr, F, nullptr, nullptr, 0.f, false, ws, H, dv_, dk_, dec, err, s);
   if (e == cudaSuccess) e = flip(dv_r, dv, L, static_cast<size_t>(H) * dv_ * 4, s);
   if (e == cudaSuccess) e = flip(dk_r, dk, L, static_cast<size_t>(H) * dk_ * 4, s);
   if (e == cudaSuccess && d_state_in) {
-    const size_t per = static_cast<size_t>(dk_) * dv_;
     dim3 grid(static_cast<unsigned>((per + 1023) / 1024), static_cast<unsigned>(L.nseq) * H);
     scale_states_kernel<<<grid, 256, 0, s>>>(d_state_in, H, per, dec);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess && ds && dec.zero_mask) {
+    zero_gamma_fixup_kernel<<<dim3(static_cast<unsigned>(L.nseq), H), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), d_state_out,
+        dk, dv, d_state_in, L, H, dk_, dv_, dec);
     e = cudaGetLastError();
   }
   return e;

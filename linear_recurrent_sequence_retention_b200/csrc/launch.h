@@ -64,17 +64,19 @@ cudaError_t launch_chunkwise_bwd_simt(const void* q, const void* k, const void* 
                                       const HeadDecay& dec, cudaStream_t s);
 
 // Backward on the tensor-core forward kernels (bf16 inputs, d_k and d_v in
-// {64, 128, 256}, no final-state gradient): three forward retentions with the
-// operand roles exchanged, two of them on the sequences read backwards.  `ws`
+// {64, 128, 256}; with a final-state gradient, every gamma 0 or >= 1e-6): three
+// forward retentions with the operand roles exchanged, two of them on the
+// sequences read backwards.  `ws`
 // holds the chunk offsets and one set of hi/lo states (reused by the three
 // passes); `scratch` (chunkwise_bwd_tc_scratch_bytes) the reversed inputs and
 // outputs and S0^T.
 size_t chunkwise_bwd_tc_scratch_bytes(const SeqLayout& L, int H, int dk, int dv);
 cudaError_t launch_chunkwise_bwd_tc(const void* q, const void* k, const void* v,
                                     const void* d_out, const SeqLayout& L, const float* state_in,
-                                    float* dq, float* dk, float* dv, float* d_state_in,
-                                    ChunkWorkspace ws, void* scratch, int H, int dk_, int dv_,
-                                    const HeadDecay& dec, unsigned* err, cudaStream_t s);
+                                    const float* d_state_out, float* dq, float* dk, float* dv,
+                                    float* d_state_in, ChunkWorkspace ws, void* scratch, int H,
+                                    int dk_, int dv_, const HeadDecay& dec, unsigned* err,
+                                    cudaStream_t s);
 
 // Rotary position encoding of q and k: [Ttot][H][d], positions counted from
 // each sequence's first token; qo/ko may alias q/k.

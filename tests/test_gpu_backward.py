@@ -4,9 +4,10 @@ fp64 oracle's gradients, through the C ABI.
 On the CUDA-core path the kernels compute every product and sum in float32
 from inputs that are exact (float32, or bfloat16 widened exactly), so both
 input dtypes are held to the float32 tolerance: relative L2 <= 1e-5 over each
-gradient, whole and per head.  bf16 inputs with heads of 64/128/256 and no
-final-state gradient run on the tensor-core kernels instead and are held to
-the bf16-input tolerance (plus rel-L2 <= 1e-4 as a precision check).  Cases
+gradient, whole and per head.  bf16 inputs with heads of 64/128/256 (and, with
+a final-state gradient, every gamma 0 or >= 1e-6) run on the tensor-core
+kernels instead and are held to the bf16-input tolerance (plus rel-L2 <= 1e-4
+as a precision check).  Cases
 span several chunks with ragged tails, chunk lengths of one token and longer
 than the sequence, the largest supported heads, gamma = 0 and gamma = 1, an
 initial state and an upstream state gradient, and packed sequences including
@@ -41,12 +42,26 @@ def _inputs(B, T, H, dk, dv, dtype, seed, with_state):
     return q, k, v, do, S0, dS
 
 
-def _check(got, ref, H, what):
-    names = ("dq", "dk", "dv")
-    for x, y, n in zip(got[:3], ref[:3], names):
-        assert_close(W.to_f64(x), y, "f32", 2, f"{what} {n}")
-    if len(got) > 3 and got[3] is not None:
-        assert_close(W.to_f64(got[3]), ref[3], "f32", 1, f"{what} d_state_in")
+def _tensor_core(dtype, dk, dv, gammas, with_dS):
+    """Whether the call runs on the tensor-core path (the rule of the C ABI)."""
+    heads = (64, 128, 256)
+    ok = dtype == "bf16" and dk in heads and dv in heads
+    if with_dS:
+        ok = ok and all(g == 0.0 or g >= 1e-6 for g in gammas)
+    return ok
+
+
+def _check(got, ref, H, what, tc=False):
+    names = ("dq", "dk", "dv", "d_state_in")
+    for x, y, n in zip(got, ref, names):
+        if x is None:
+            continue
+        axis = 2 if n != "d_state_in" else 1
+        if tc:
+            assert_close(W.to_f64(x), y, "bf16", axis, f"{what} {n}")
+            assert rel_l2(W.to_f64(x), y) <= 1e-4, (what, n, rel_l2(W.to_f64(x), y))
+        else:
+            assert_close(W.to_f64(x), y, "f32", axis, f"{what} {n}")
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -66,7 +81,8 @@ def test_backward_matches_oracle(dtype, B, T, H, dk, dv, chunk, with_state):
     got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, chunk,
                             state_in=None if S0 is None else S0.cuda(),
                             d_state_out=None if dS is None else dS.cuda(), return_d_state=True)
-    _check(got, ref, H, f"{dtype} B{B} T{T} dk{dk} dv{dv} C{chunk}")
+    _check(got, ref, H, f"{dtype} B{B} T{T} dk{dk} dv{dv} C{chunk}",
+           _tensor_core(dtype, dk, dv, gam, dS is not None))
 
 
 @pytest.mark.parametrize("B,T,H,dk,dv,chunk,with_state", [
@@ -75,38 +91,82 @@ def test_backward_matches_oracle(dtype, B, T, H, dk, dv, chunk, with_state):
     (1, 200, 2, 256, 64, 256, True),     # d_k > d_v
     (1, 1030, 2, 128, 128, 512, False),  # 512-token chunks, ragged last chunk
 ])
-def test_backward_tensor_core_path(B, T, H, dk, dv, chunk, with_state):
-    """bf16 inputs with heads of 64/128/256 and no final-state gradient run on the
-    tensor-core forward kernels (three retentions, two on reversed sequences);
-    held to the bf16-input tolerance and, as a precision check, rel-L2 <= 1e-4."""
-    q, k, v, do, S0, _ = _inputs(B, T, H, dk, dv, "bf16", seed=T + 3 * dk, with_state=with_state)
+@pytest.mark.parametrize("use_dS", [False, True])
+def test_backward_tensor_core_path(B, T, H, dk, dv, chunk, with_state, use_dS):
+    """bf16 inputs with heads of 64/128/256 run on the tensor-core forward kernels
+    (three retentions, two on reversed sequences; a final-state gradient enters
+    them as the initial state dS_T / gamma); held to the bf16-input tolerance
+    and, as a precision check, rel-L2 <= 1e-4."""
+    q, k, v, do, S0, dS = _inputs(B, T, H, dk, dv, "bf16", seed=T + 3 * dk, with_state=True)
+    S0 = S0 if with_state else None
+    dS = dS if use_dS else None
     gam = W.head_gammas(H)
+    assert _tensor_core("bf16", dk, dv, gam, use_dS)
     ref = oracle.msr_backward(W.to_f64(q), W.to_f64(k), W.to_f64(v), gam, W.to_f64(do),
-                              None if S0 is None else S0.double().numpy())
+                              None if S0 is None else S0.double().numpy(),
+                              None if dS is None else dS.double().numpy())
     got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, chunk,
-                            state_in=None if S0 is None else S0.cuda(), return_d_state=True)
-    for x, y, n in zip(got, ref, ("dq", "dk", "dv", "d_state_in")):
-        assert_close(W.to_f64(x), y, "bf16", 2 if n != "d_state_in" else 1, f"tc {n}")
-        assert rel_l2(W.to_f64(x), y) <= 1e-4, (n, rel_l2(W.to_f64(x), y))
+                            state_in=None if S0 is None else S0.cuda(),
+                            d_state_out=None if dS is None else dS.cuda(), return_d_state=True)
+    _check(got, ref, H, f"tc T{T} dk{dk} dv{dv} dS={use_dS}", tc=True)
 
 
-def test_backward_tensor_core_packed():
-    """The tensor-core path on packed sequences (reversal inside each sequence)."""
+@pytest.mark.parametrize("use_dS", [False, True])
+def test_backward_tensor_core_packed(use_dS):
+    """The tensor-core path on packed sequences (reversal inside each sequence;
+    an empty sequence passes dS_T straight to its initial-state gradient)."""
     lens = [300, 0, 1, 129, 64]
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     Tt = int(cu[-1])
     H, dk, dv, chunk = 2, 64, 64, 64
     q, k, v, do, _, _ = _inputs(1, Tt, H, dk, dv, "bf16", seed=21, with_state=False)
-    S0 = torch.randn(len(lens), H, dk, dv, generator=torch.Generator().manual_seed(22))
+    g = torch.Generator().manual_seed(22)
+    S0 = torch.randn(len(lens), H, dk, dv, generator=g)
+    dS = torch.randn(len(lens), H, dk, dv, generator=g) if use_dS else None
     gam = W.head_gammas(H)
     ref = oracle.msr_backward_varlen(W.to_f64(q), W.to_f64(k), W.to_f64(v), gam, W.to_f64(do),
-                                     cu, S0.double().numpy())
+                                     cu, S0.double().numpy(),
+                                     None if dS is None else dS.double().numpy())
     got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, chunk,
                             cu_seqlens=torch.from_numpy(cu).cuda(), state_in=S0.cuda(),
-                            return_d_state=True)
-    for x, y, n in zip(got, ref, ("dq", "dk", "dv", "d_state_in")):
-        assert_close(W.to_f64(x), y, "bf16", 2 if n != "d_state_in" else 1, f"tc packed {n}")
-        assert rel_l2(W.to_f64(x), y) <= 1e-4, (n, rel_l2(W.to_f64(x), y))
+                            d_state_out=None if dS is None else dS.cuda(), return_d_state=True)
+    _check(got, ref, H, f"tc packed dS={use_dS}", tc=True)
+
+
+@pytest.mark.parametrize("gammas", [[0.0, 0.96875], [1.0, 0.0]])
+def test_backward_tensor_core_zero_and_unit_decay(gammas):
+    """gamma = 0 heads on the tensor-core path with a final-state gradient: the
+    state gradient reaches only the last token of each sequence (and, for an
+    empty sequence, the initial-state gradient); gamma = 1 carries it to every
+    token undecayed."""
+    lens = [130, 0, 1, 65]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    Tt = int(cu[-1])
+    H, dk, dv, chunk = 2, 64, 128, 64
+    q, k, v, do, _, _ = _inputs(1, Tt, H, dk, dv, "bf16", seed=31, with_state=False)
+    g = torch.Generator().manual_seed(32)
+    S0 = torch.randn(len(lens), H, dk, dv, generator=g)
+    dS = torch.randn(len(lens), H, dk, dv, generator=g)
+    ref = oracle.msr_backward_varlen(W.to_f64(q), W.to_f64(k), W.to_f64(v), gammas, W.to_f64(do),
+                                     cu, S0.double().numpy(), dS.double().numpy())
+    got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gammas, chunk,
+                            cu_seqlens=torch.from_numpy(cu).cuda(), state_in=S0.cuda(),
+                            d_state_out=dS.cuda(), return_d_state=True)
+    _check(got, ref, H, f"tc gammas {gammas}", tc=True)
+
+
+def test_backward_tiny_decay_with_state_gradient_uses_cuda_cores():
+    """A gamma in (0, 1e-6) with a final-state gradient would overflow dS_T / gamma
+    on the tensor-core path; such calls run on CUDA cores (float32 tolerance)."""
+    B, T, H, dk, dv, chunk = 1, 150, 2, 64, 64, 64
+    q, k, v, do, S0, dS = _inputs(B, T, H, dk, dv, "bf16", seed=41, with_state=True)
+    gam = [1e-7, 0.9]
+    assert not _tensor_core("bf16", dk, dv, gam, True)
+    ref = oracle.msr_backward(W.to_f64(q), W.to_f64(k), W.to_f64(v), gam, W.to_f64(do),
+                              S0.double().numpy(), dS.double().numpy())
+    got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, chunk,
+                            state_in=S0.cuda(), d_state_out=dS.cuda(), return_d_state=True)
+    _check(got, ref, H, "tiny gamma")
 
 
 @pytest.mark.parametrize("gammas", [[0.0, 1.0], [1.0, 0.5]])
@@ -118,7 +178,7 @@ def test_backward_extreme_decays(gammas):
                               S0.double().numpy(), dS.double().numpy())
     got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gammas, chunk,
                             state_in=S0.cuda(), d_state_out=dS.cuda(), return_d_state=True)
-    _check(got, ref, H, f"gammas {gammas}")
+    _check(got, ref, H, f"gammas {gammas}")  # float32 inputs: CUDA cores
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -138,7 +198,7 @@ def test_backward_packed_sequences(dtype):
     got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, chunk,
                             cu_seqlens=torch.from_numpy(cu).cuda(), state_in=S0.cuda(),
                             d_state_out=dS.cuda(), return_d_state=True)
-    _check(got, ref, H, f"packed {dtype}")
+    _check(got, ref, H, f"packed {dtype}")  # heads of 32/16: CUDA cores
 
 
 def test_backward_chunk_length_does_not_matter():
@@ -165,22 +225,26 @@ def test_backward_rejects_unsupported_and_bad_arguments():
     assert ops.chunkwise_bwd_workspace_size(torch.float32, 4, 1, 8, 1, 16, 16) > 0
 
 
-@pytest.mark.parametrize("path", ["tensor_core", "cuda_core"])
+@pytest.mark.parametrize("path", ["tensor_core", "tensor_core_dS", "cuda_core"])
 def test_backward_bench_workload_sampled(path):
     """The backward at the size bench.py times (B=4, T=2048, H=8, d_k=128, d_v=256,
-    chunk 128, bf16 inputs), checked on two sampled (sequence, head) pairs; the
-    CUDA-core path is taken by passing a final-state gradient."""
+    chunk 128), checked on two sampled (sequence, head) pairs: bf16 inputs on
+    the tensor-core path without and with a final-state gradient, and the same
+    values as float32 inputs (with one) on the CUDA-core path."""
     B, T, H, dk, dv, C = 4, 2048, 8, 128, 256, 128
     q, k, v, do, _, dS = _inputs(B, T, H, dk, dv, "bf16", seed=77, with_state=True)
     gam = W.head_gammas(H)
-    use_dS = path == "cuda_core"
-    got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, C,
-                            d_state_out=dS.cuda() if use_dS else None, return_d_state=True)
+    use_dS = path != "tensor_core"
+    x = [t.cuda() for t in (q, k, v, do)]
+    if path == "cuda_core":
+        x = [t.float() for t in x]
+    got = ops.chunkwise_bwd(*x, gam, C, d_state_out=dS.cuda() if use_dS else None,
+                            return_d_state=True)
     for b, h in ((0, 0), (3, 7)):
         ref = oracle.retention_backward(W.to_f64(q[b, :, h]), W.to_f64(k[b, :, h]),
                                         W.to_f64(v[b, :, h]), gam[h], W.to_f64(do[b, :, h]),
                                         None, dS[b, h].double().numpy() if use_dS else None)
         for x, y, n in zip((got[0][b, :, h], got[1][b, :, h], got[2][b, :, h], got[3][b, h]),
                            ref, ("dq", "dk", "dv", "d_state_in")):
-            kind = "bf16" if path == "tensor_core" else "f32"
+            kind = "f32" if path == "cuda_core" else "bf16"
             assert_close(W.to_f64(x), y, kind, None, f"{path} b{b} h{h} {n}")
