@@ -5,7 +5,8 @@ The kernel computes in float32 on CUDA cores from exact bf16 or fp32 inputs,
 so both the Tn outputs and the updated state are held to the float32 bound
 (relative L2 <= 1e-5) per head and overall.  The tests span one to sixteen
 tokens, d_v not a multiple of the 128-column block, gamma = 0 and gamma = 1
-heads, and agreement with Tn single-step calls.
+heads, agreement with Tn single-step calls, several 512-column blocks with a
+ragged last one over hundreds of blocks, and the largest supported d_k.
 """
 
 import numpy as np
@@ -95,3 +96,30 @@ def test_bf16_output_and_rejects():
     with pytest.raises(ops.RetentionError) as info:
         ops.recurrent_steps(q17.cuda(), k17.cuda(), v17.cuda(), gam, S[:1].clone())
     assert info.value.status == ops.RET_ERR_UNSUPPORTED
+
+
+def test_many_items_ragged_blocks_and_rows():
+    """592 blocks (37 sequences x 8 heads x 2 column blocks); d_v = 644 (a
+    132-column last block), d_k = 68 (17 groups of 4 rows)."""
+    N, Tn, H, dk, dv = 37, 7, 8, 68, 644
+    q, k, v, S0 = _inputs(N, Tn, H, dk, dv, "bf16", seed=41)
+    gam = W.head_gammas(H)
+    S = S0.clone().cuda()
+    o = ops.recurrent_steps(q.cuda(), k.cuda(), v.cuda(), gam, S)
+    ops.check_device_error()
+    o_ref, S_ref = _oracle(q, k, v, S0, gam)
+    assert_close(f64(o), o_ref, "f32", 2, "o")
+    assert_close(f64(S), S_ref, "f32", 1, "state")
+
+
+def test_largest_dk():
+    """d_k = 512, the largest the call accepts, float32 inputs."""
+    N, Tn, H, dk, dv = 2, 16, 2, 512, 256
+    q, k, v, S0 = _inputs(N, Tn, H, dk, dv, "f32", seed=43)
+    gam = W.head_gammas(H)
+    S = S0.clone().cuda()
+    o = ops.recurrent_steps(q.cuda(), k.cuda(), v.cuda(), gam, S)
+    ops.check_device_error()
+    o_ref, S_ref = _oracle(q, k, v, S0, gam)
+    assert_close(f64(o), o_ref, "f32", 2, "o")
+    assert_close(f64(S), S_ref, "f32", 1, "state")
