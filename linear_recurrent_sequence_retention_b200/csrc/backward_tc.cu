@@ -29,23 +29,44 @@ namespace ret {
 namespace {
 
 constexpr int kFlipThreads = 256;
+constexpr int kFlipTok = 8;          // tokens per block
+constexpr int kFlipIlp = 4;          // 16-byte loads in flight per thread
 
 // dst[a + j] = src[b - 1 - j] for every sequence [a, b) of the flat token
-// axis; a token row is `row_bytes` bytes (a multiple of 16).  One block per
-// token, 16-byte copies.
+// axis; a token row is `row_vec` 16-byte vectors.  A block moves kFlipTok
+// consecutive destination rows; each thread issues kFlipIlp loads before its
+// stores, so enough bytes are in flight to keep HBM busy.  Rows outside every
+// sequence are left as they are.
 __global__ void __launch_bounds__(kFlipThreads)
 flip_tokens_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, SeqLayout L,
                    int row_vec) {
-  const int n = blockIdx.x;
-  if (n >= L.Ttot) return;
-  const int s = seq_of_token(L, n);
-  int a, b;
-  seq_bounds(L, s, a, b);
-  if (n < a || n >= b) return;
-  const int m = a + b - 1 - n;
-  const uint4* sr = src + static_cast<size_t>(m) * row_vec;
-  uint4* dr = dst + static_cast<size_t>(n) * row_vec;
-  for (int i = threadIdx.x; i < row_vec; i += kFlipThreads) dr[i] = sr[i];
+  __shared__ int srow[kFlipTok];
+  const int n0 = blockIdx.x * kFlipTok;
+  if (threadIdx.x < kFlipTok) {
+    const int n = n0 + static_cast<int>(threadIdx.x);
+    int m = -1;
+    if (n < L.Ttot) {
+      int a, b;
+      seq_bounds(L, seq_of_token(L, n), a, b);
+      if (n >= a && n < b) m = a + b - 1 - n;
+    }
+    srow[threadIdx.x] = m;
+  }
+  __syncthreads();
+  const int total = kFlipTok * row_vec;
+  for (int base = threadIdx.x; base < total; base += kFlipIlp * kFlipThreads) {
+    uint4 v[kFlipIlp];
+    int m[kFlipIlp], e[kFlipIlp];
+#pragma unroll
+    for (int u = 0; u < kFlipIlp; ++u) {
+      e[u] = base + u * kFlipThreads;
+      m[u] = e[u] < total ? srow[e[u] / row_vec] : -1;
+      if (m[u] >= 0) v[u] = src[static_cast<size_t>(m[u]) * row_vec + e[u] % row_vec];
+    }
+#pragma unroll
+    for (int u = 0; u < kFlipIlp; ++u)
+      if (m[u] >= 0) dst[static_cast<size_t>(n0) * row_vec + e[u]] = v[u];
+  }
 }
 
 // out[s][h] = in[s][h]^T  (in: [dk][dv] -> out: [dv][dk]), 32 x 32 tiles.
@@ -123,9 +144,8 @@ __global__ void scale_states_kernel(float* __restrict__ x, int H, size_t per, He
 
 cudaError_t flip(const void* src, void* dst, const SeqLayout& L, size_t row_bytes, cudaStream_t s) {
   if (L.Ttot == 0) return cudaSuccess;
-  flip_tokens_kernel<<<L.Ttot, kFlipThreads, 0, s>>>(static_cast<const uint4*>(src),
-                                                     static_cast<uint4*>(dst), L,
-                                                     static_cast<int>(row_bytes / 16));
+  flip_tokens_kernel<<<(L.Ttot + kFlipTok - 1) / kFlipTok, kFlipThreads, 0, s>>>(
+      static_cast<const uint4*>(src), static_cast<uint4*>(dst), L, static_cast<int>(row_bytes / 16));
   return cudaGetLastError();
 }
 
