@@ -43,8 +43,112 @@ __device__ __forceinline__ void softmax_row(const T* in, T* out, int d, bool zer
   for (int j = lane; j < d; j += 32) stf<T>(out, j, expf(ldf<T>(in, j) - m) * inv);
 }
 
+// VPL consecutive elements per lane as floats (one vector load / store).
+template <typename T, int VPL> struct RowVec;
+template <int VPL> struct RowVec<__nv_bfloat16, VPL> {
+  static_assert(VPL == 2 || VPL == 4 || VPL == 8, "2, 4 or 8 bf16 per lane");
+  static __device__ __forceinline__ void ld(const __nv_bfloat16* p, float (&x)[VPL]) {
+    uint32_t w[VPL / 2];
+    if constexpr (VPL == 2) {
+      w[0] = *reinterpret_cast<const uint32_t*>(p);
+    } else if constexpr (VPL == 4) {
+      const uint2 u = *reinterpret_cast<const uint2*>(p);
+      w[0] = u.x; w[1] = u.y;
+    } else {
+      const uint4 u = *reinterpret_cast<const uint4*>(p);
+      w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+    }
+#pragma unroll
+    for (int i = 0; i < VPL / 2; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  static __device__ __forceinline__ void st(__nv_bfloat16* p, const float (&x)[VPL]) {
+    uint32_t w[VPL / 2];
+#pragma unroll
+    for (int i = 0; i < VPL / 2; ++i) {
+      const __nv_bfloat162 b = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+      w[i] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    if constexpr (VPL == 2) {
+      *reinterpret_cast<uint32_t*>(p) = w[0];
+    } else if constexpr (VPL == 4) {
+      *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
+    } else {
+      *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+};
+template <int VPL> struct RowVec<float, VPL> {
+  static_assert(VPL == 2 || VPL == 4 || VPL == 8, "2, 4 or 8 floats per lane");
+  static __device__ __forceinline__ void ld(const float* p, float (&x)[VPL]) {
+    if constexpr (VPL == 2) {
+      const float2 u = *reinterpret_cast<const float2*>(p);
+      x[0] = u.x; x[1] = u.y;
+    } else {
+#pragma unroll
+      for (int i = 0; i < VPL / 4; ++i) {
+        const float4 u = reinterpret_cast<const float4*>(p)[i];
+        x[4 * i] = u.x; x[4 * i + 1] = u.y; x[4 * i + 2] = u.z; x[4 * i + 3] = u.w;
+      }
+    }
+  }
+  static __device__ __forceinline__ void st(float* p, const float (&x)[VPL]) {
+    if constexpr (VPL == 2) {
+      *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < VPL / 4; ++i)
+        reinterpret_cast<float4*>(p)[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+    }
+  }
+};
+
+// Softmax of one row of 32 * VPL elements held in registers (one warp, one
+// load and one store per lane).
+template <typename T, int VPL>
+__device__ __forceinline__ void softmax_row_reg(const T* in, T* out, bool zero) {
+  const int lane = threadIdx.x & 31;
+  float x[VPL];
+  if (zero) {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) x[i] = 0.f;
+    RowVec<T, VPL>::st(out + lane * VPL, x);
+    return;
+  }
+  RowVec<T, VPL>::ld(in + lane * VPL, x);
+  float m = x[0];
+#pragma unroll
+  for (int i = 1; i < VPL; ++i) m = fmaxf(m, x[i]);
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    x[i] = expf(x[i] - m);
+    s += x[i];
+  }
+  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float inv = 1.0f / s;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) x[i] *= inv;
+  RowVec<T, VPL>::st(out + lane * VPL, x);
+}
+
+template <typename T>
+__device__ __forceinline__ void softmax_any(const T* in, T* out, int d, bool zero) {
+  switch (d) {
+    case 64: softmax_row_reg<T, 2>(in, out, zero); break;
+    case 128: softmax_row_reg<T, 4>(in, out, zero); break;
+    case 256: softmax_row_reg<T, 8>(in, out, zero); break;
+    default: softmax_row<T>(in, out, d, zero); break;
+  }
+}
+
 // One warp per (token n, head h): q'[n] = phi(q[n]); k''[n] = phi(k[n-w-1]) and
-// v''[n] = v[n-w-1] inside n's sequence, zero before it.
+// v''[n] = v[n-w-1] inside n's sequence, zero before it.  Rows of 64, 128 or
+// 256 elements are held in registers (one vector load and store per lane);
+// other widths take the strided loops.
 template <typename T>
 __global__ void __launch_bounds__(kRlaWarps * 32)
 rla_inputs_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
@@ -64,13 +168,21 @@ rla_inputs_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
   const long long src = static_cast<long long>(n) - window - 1;
   const bool has = src >= a;
   const size_t qo = (static_cast<size_t>(n) * H + h) * dk;
-  softmax_row<T>(q + qo, qf + qo, dk, false);
+  softmax_any<T>(q + qo, qf + qo, dk, false);
   const size_t ko = has ? (static_cast<size_t>(src) * H + h) * dk : 0;
-  softmax_row<T>(k + ko, ks + qo, dk, !has);
+  softmax_any<T>(k + ko, ks + qo, dk, !has);
   const int lane = threadIdx.x & 31;
   const size_t vo = (static_cast<size_t>(n) * H + h) * dv;
   const size_t vi = has ? (static_cast<size_t>(src) * H + h) * dv : 0;
-  for (int j = lane; j < dv; j += 32) stf<T>(vs, vo + j, has ? ldf<T>(v, vi + j) : 0.f);
+  if ((dv * sizeof(T)) % 16 == 0) {
+    // 16-byte copies: rows start 16-byte aligned when their byte length is a multiple of 16
+    const int nvec = static_cast<int>(dv * sizeof(T) / 16);
+    const uint4* sv = reinterpret_cast<const uint4*>(v + vi);
+    uint4* dvp = reinterpret_cast<uint4*>(vs + vo);
+    for (int j = lane; j < nvec; j += 32) dvp[j] = has ? sv[j] : make_uint4(0, 0, 0, 0);
+  } else {
+    for (int j = lane; j < dv; j += 32) stf<T>(vs, vo + j, has ? ldf<T>(v, vi + j) : 0.f);
+  }
 }
 
 }  // namespace
