@@ -581,7 +581,7 @@ def run_decode(args, world, rank, pk, pk_kind):
              "roofline": {"bound": "hbm", "achieved": ach_m, "peak": pk["hbm_gbs"], "unit": "GB/s",
                           "frac": ach_m / pk["hbm_gbs"], "peak_source": pk_kind,
                           "algorithmic_bytes_per_launch": call_bytes,
-                          "kernel": "decode_multi_kernel"}}
+                          "kernel": "decode_multi_tc_kernel"}}
     del qs, ks, vs, qm, km, vm, S, o, om
     torch.cuda.empty_cache()
     return {"workload": wl.name, "steps": steps, "ms_per_step": ms,

@@ -323,7 +323,7 @@ ret_status retention_recurrent_steps(const void* q, const void* k, const void* v
   if (Tn > 16 || dk > 512 || dv > 4096 || dk % 4 != 0 || dv % 4 != 0) return RET_ERR_UNSUPPORTED;
   if (N > 65535 || H > 65535) return RET_ERR_UNSUPPORTED;
   return cuda_status(ret::launch_decode_steps(q, k, v, dt(in_dtype), state, o, dt(o_dtype), N, Tn,
-                                              H, dk, dv, dec,
+                                              H, dk, dv, dec, error_word(),
                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -92,7 +92,14 @@ cudaError_t launch_rla_inputs(const void* q, const void* k, const void* v, DType
 // Tn (1..16) tokens per sequence in one pass over the state.
 cudaError_t launch_decode_steps(const void* q, const void* k, const void* v, DType in_t,
                                 float* state, void* o, DType o_t, int N, int Tn, int H, int dk,
-                                int dv, const HeadDecay& dec, cudaStream_t s);
+                                int dv, const HeadDecay& dec, unsigned* err, cudaStream_t s);
+// Tn decode steps on the tensor cores (bf16 q, k, v; tf32 MMAs on the float32
+// state; d_k in {128, 256}, d_v a multiple of 128 whose operand tiles fit).
+bool decode_steps_tc_supported(int Tn, int dk, int dv);
+bool decode_steps_tc_preferred(int Tn, int dk, int dv);
+cudaError_t launch_decode_steps_tc(const void* q, const void* k, const void* v, float* state,
+                                   void* o, DType o_t, int N, int Tn, int H, int dk, int dv,
+                                   const HeadDecay& dec, unsigned* err, cudaStream_t s);
 cudaError_t launch_decode_step(const void* q, const void* k, const void* v, DType in_t,
                                float* state, void* o, DType o_t, int N, int H, int dk, int dv,
                                const HeadDecay& dec, cudaStream_t s);
