@@ -53,8 +53,8 @@ struct DtLayout {
     qs = kDtStages * kDtStage;                          // [dk/32 chunks][16 rows][128 B]
     zk = qs + (dk / 32) * kDtChunk;                     // same shape
     vb = zk + (dk / 32) * kDtChunk;                     // [dv/32 chunks][16 rows][128 B]
-    att = vb + (dv / 32) * kDtChunk;                    // [16][16] float
-    bars = att + kDtMaxT * kDtMaxT * 4;
+    att = vb + (dv / 32) * kDtChunk;                    // [16][16] float, then [2][16] decay factors
+    bars = att + kDtMaxT * kDtMaxT * 4 + 2 * kDtMaxT * 4;
     smem = bars + 256;
   }
 };
@@ -147,6 +147,18 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParam
       int it = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < p.nitems && ok; item += gridDim.x) {
+        // the next item's q, k, v rows into L2 while this item streams, so that the
+        // workers' operand tiles for it are formed from L2
+        const int nxt = item + gridDim.x;
+        if (nxt < p.nitems) {
+          const int hn = nxt % p.H, nn = nxt / p.H;
+          for (int t = 0; t < p.Tn; ++t) {
+            const size_t row = (static_cast<size_t>(nn) * p.Tn + t) * p.H + hn;
+            bulk_prefetch_l2(p.q + row * p.dk, static_cast<uint32_t>(p.dk * 2));
+            bulk_prefetch_l2(p.k + row * p.dk, static_cast<uint32_t>(p.dk * 2));
+            bulk_prefetch_l2(p.v + row * p.dv, static_cast<uint32_t>(p.dv * 2));
+          }
+        }
         for (int b = 0; b < nb && ok; ++b) {
           for (int q = 0; q < nq; ++q, ++it) {
             const int st = it % kDtStages;
@@ -243,13 +255,15 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParam
       if (!r) break;
       const int h = item % p.H, n = item / p.H;
       const Decay1 dg(p.dec, h);
-      // (a) q and k of the Tn tokens, unscaled, as plain [16][dk] float32 rows in
-      // the qs and zk regions (zero rows from Tn on); v straight into its tile
-      // (MN-major, 32-byte atoms).  16-byte loads of 8 bf16.
+      // (a) q and k of the Tn tokens, unscaled, as [16][dk] float32 rows in the
+      // qs and zk regions (k's float4 columns XOR-swizzled by row, so that the
+      // score pass below reads 16 rows without bank conflicts; zero rows from Tn
+      // on); v straight into its MN-major tile; the per-token decay factors.
+      // Every 16-byte global load is issued before the first store.
       float* qraw = reinterpret_cast<float*>(qs);
       float* kraw = reinterpret_cast<float*>(zk);
-      auto ld8 = [](const __nv_bfloat16* src, float (&x)[8]) {
-        const uint4 u = *reinterpret_cast<const uint4*>(src);
+      float* fac = att + kDtMaxT * kDtMaxT;            // [2][16]: gamma^(t+1), zeta_t
+      auto cvt8 = [](uint4 u, float (&x)[8]) {
         const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -257,72 +271,107 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParam
           x[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
         }
       };
-      for (int e8 = wt * 8; e8 < kDtMaxT * p.dk; e8 += 256 * 8) {
-        const int t = e8 / p.dk, i = e8 % p.dk;
-        float xq[8], xk[8];
-        if (t < p.Tn) {
-          const size_t row = ((static_cast<size_t>(n) * p.Tn + t) * p.H + h) * p.dk + i;
-          ld8(p.q + row, xq);
-          ld8(p.k + row, xk);
-        } else {
+      {
+        constexpr int kQK = kDtMaxT * 256 / 8 / 256;     // 16-byte vectors of q (and of k) per thread at d_k = 256
+        constexpr int kV = kDtMaxT * 512 / 8 / 256;      // of v at d_v = 512
+        const int nqk = kDtMaxT * p.dk / 8, nv = kDtMaxT * p.dv / 8;
+        uint4 uq[kQK], uk[kQK], uv[kV];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) xq[e] = xk[e] = 0.f;
+        for (int m = 0; m < kQK; ++m) {
+          const int e8 = (wt + 256 * m) * 8, t = e8 / p.dk, i = e8 % p.dk;
+          uq[m] = uk[m] = make_uint4(0, 0, 0, 0);
+          if (e8 < kDtMaxT * p.dk && t < p.Tn) {
+            const size_t row = ((static_cast<size_t>(n) * p.Tn + t) * p.H + h) * p.dk + i;
+            uq[m] = *reinterpret_cast<const uint4*>(p.q + row);
+            uk[m] = *reinterpret_cast<const uint4*>(p.k + row);
+          }
         }
-        float4* dq = reinterpret_cast<float4*>(qraw + e8);
-        float4* dk4 = reinterpret_cast<float4*>(kraw + e8);
-        dq[0] = make_float4(xq[0], xq[1], xq[2], xq[3]);
-        dq[1] = make_float4(xq[4], xq[5], xq[6], xq[7]);
-        dk4[0] = make_float4(xk[0], xk[1], xk[2], xk[3]);
-        dk4[1] = make_float4(xk[4], xk[5], xk[6], xk[7]);
-      }
-      for (int e8 = wt * 8; e8 < kDtMaxT * p.dv; e8 += 256 * 8) {
-        const int t = e8 / p.dv, cc = e8 % p.dv;
-        float xv[8];
-        if (t < p.Tn) {
-          ld8(p.v + ((static_cast<size_t>(n) * p.Tn + t) * p.H + h) * p.dv + cc, xv);
-        } else {
+        for (int m0 = 0; m0 < nv; m0 += kV * 256) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) xv[e] = 0.f;
+          for (int m = 0; m < kV; ++m) {
+            const int e8 = (m0 + wt + 256 * m) * 8, t = e8 / p.dv, cc = e8 % p.dv;
+            uv[m] = make_uint4(0, 0, 0, 0);
+            if (e8 < kDtMaxT * p.dv && t < p.Tn)
+              uv[m] = *reinterpret_cast<const uint4*>(p.v + ((static_cast<size_t>(n) * p.Tn + t) * p.H + h) * p.dv + cc);
+          }
+#pragma unroll
+          for (int m = 0; m < kV; ++m) {
+            const int e8 = (m0 + wt + 256 * m) * 8, t = e8 / p.dv, cc = e8 % p.dv;
+            if (e8 >= kDtMaxT * p.dv) continue;
+            float xv[8];
+            cvt8(uv[m], xv);
+            // 8 consecutive columns (cc mod 8 == 0) are one 32-byte atom
+            float4* dv4 = reinterpret_cast<float4*>(vb + (cc >> 5) * kDtChunk + sw32_off(t, cc));
+            dv4[0] = make_float4(xv[0], xv[1], xv[2], xv[3]);
+            dv4[1] = make_float4(xv[4], xv[5], xv[6], xv[7]);
+          }
         }
-        // 8 consecutive columns (cc mod 8 == 0) are one 32-byte atom
-        float4* dv4 = reinterpret_cast<float4*>(vb + (cc >> 5) * kDtChunk + sw32_off(t, cc));
-        dv4[0] = make_float4(xv[0], xv[1], xv[2], xv[3]);
-        dv4[1] = make_float4(xv[4], xv[5], xv[6], xv[7]);
+        (void)nqk;
+#pragma unroll
+        for (int m = 0; m < kQK; ++m) {
+          const int e8 = (wt + 256 * m) * 8, t = e8 / p.dk, i = e8 % p.dk;
+          if (e8 >= kDtMaxT * p.dk) continue;
+          float xq[8], xk[8];
+          cvt8(uq[m], xq);
+          cvt8(uk[m], xk);
+          float4* dq = reinterpret_cast<float4*>(qraw + t * p.dk + i);
+          dq[0] = make_float4(xq[0], xq[1], xq[2], xq[3]);
+          dq[1] = make_float4(xq[4], xq[5], xq[6], xq[7]);
+          float4* kr = reinterpret_cast<float4*>(kraw + t * p.dk);
+          const int c4 = i >> 2;                       // float4 column, swizzled by row t
+          kr[c4 ^ (t & 7)] = make_float4(xk[0], xk[1], xk[2], xk[3]);
+          kr[(c4 + 1) ^ (t & 7)] = make_float4(xk[4], xk[5], xk[6], xk[7]);
+        }
+        if (wt < kDtMaxT) {
+          fac[wt] = wt < p.Tn ? dg.pow(wt + 1) : 0.f;
+          fac[kDtMaxT + wt] = wt < p.Tn ? dg.pow(p.Tn - 1 - wt) : 0.f;
+        }
       }
       asm volatile("bar.sync 2, 256;" ::: "memory");
-      // (b) intra-step scores (q_t . k_j) gamma^(t-j), j <= t, from the staged rows
-      for (int idx = w; idx < kDtMaxT * kDtMaxT; idx += 8) {
-        const int t = idx / kDtMaxT, j = idx % kDtMaxT;
+      // (b) intra-step scores (q_t . k_j) gamma^(t-j), j <= t: thread (t, j)
+      {
+        const int t = wt >> 4, j = wt & 15;
         float a = 0.f;
         if (j <= t && t < p.Tn) {
-          for (int i = lane; i < p.dk; i += 32) a = fmaf(qraw[t * p.dk + i], kraw[j * p.dk + i], a);
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-          a *= dg.pow(t - j);
+          const float4* qr = reinterpret_cast<const float4*>(qraw + t * p.dk);
+          const float4* kr = reinterpret_cast<const float4*>(kraw + j * p.dk);
+          float a0 = 0.f, a1 = 0.f;
+          for (int c4 = 0; c4 < p.dk / 4; c4 += 2) {
+            const float4 x0 = qr[c4], y0 = kr[c4 ^ (j & 7)];
+            const float4 x1 = qr[c4 + 1], y1 = kr[(c4 + 1) ^ (j & 7)];
+            a0 = fmaf(x0.x, y0.x, fmaf(x0.y, y0.y, fmaf(x0.z, y0.z, fmaf(x0.w, y0.w, a0))));
+            a1 = fmaf(x1.x, y1.x, fmaf(x1.y, y1.y, fmaf(x1.z, y1.z, fmaf(x1.w, y1.w, a1))));
+          }
+          a = (a0 + a1) * dg.pow(t - j);
         }
-        if (lane == 0) att[idx] = a;
+        att[wt] = a;
       }
       // (c) the same elements rewritten in place as the MMA operand tiles:
       // q_t gamma^(t+1) (K-major, 16-byte atoms) and zeta_t k_t (MN-major,
-      // 32-byte atoms); every thread reads its elements before any writes
-      constexpr int kPer = kDtMaxT * 256 / 256;          // elements per thread at d_k = 256
-      float qv[kPer], kv[kPer];
+      // 32-byte atoms), four consecutive elements at a time; every thread reads
+      // its elements before any writes
+      {
+        constexpr int kF4 = kDtMaxT * 256 / 4 / 256;     // float4 per thread at d_k = 256
+        float4 qv[kF4], kv[kF4];
 #pragma unroll
-      for (int m = 0; m < kPer; ++m) {
-        const int e = wt + 256 * m;
-        qv[m] = e < kDtMaxT * p.dk ? qraw[e] : 0.f;
-        kv[m] = e < kDtMaxT * p.dk ? kraw[e] : 0.f;
-      }
-      asm volatile("bar.sync 2, 256;" ::: "memory");
+        for (int m = 0; m < kF4; ++m) {
+          const int e4 = (wt + 256 * m) * 4, t = e4 / p.dk, i = e4 % p.dk;
+          if (e4 < kDtMaxT * p.dk) {
+            qv[m] = *reinterpret_cast<const float4*>(qraw + e4);
+            kv[m] = reinterpret_cast<const float4*>(kraw + t * p.dk)[(i >> 2) ^ (t & 7)];
+          }
+        }
+        asm volatile("bar.sync 2, 256;" ::: "memory");
 #pragma unroll
-      for (int m = 0; m < kPer; ++m) {
-        const int e = wt + 256 * m;
-        if (e < kDtMaxT * p.dk) {
-          const int t = e / p.dk, i = e % p.dk;
-          const float sq = t < p.Tn ? dg.pow(t + 1) : 0.f;
-          const float sk = t < p.Tn ? dg.pow(p.Tn - 1 - t) : 0.f;
-          *reinterpret_cast<float*>(qs + (i >> 5) * kDtChunk + sw_off(t, i)) = qv[m] * sq;
-          *reinterpret_cast<float*>(zk + (i >> 5) * kDtChunk + sw32_off(t, i)) = kv[m] * sk;
+        for (int m = 0; m < kF4; ++m) {
+          const int e4 = (wt + 256 * m) * 4, t = e4 / p.dk, i = e4 % p.dk;
+          if (e4 >= kDtMaxT * p.dk) continue;
+          const float sq = fac[t], sk = fac[kDtMaxT + t];
+          float4 a = qv[m], c = kv[m];
+          a.x *= sq; a.y *= sq; a.z *= sq; a.w *= sq;
+          c.x *= sk; c.y *= sk; c.z *= sk; c.w *= sk;
+          *reinterpret_cast<float4*>(qs + (i >> 5) * kDtChunk + sw_off(t, i)) = a;
+          *reinterpret_cast<float4*>(zk + (i >> 5) * kDtChunk + sw32_off(t, i)) = c;
         }
       }
       fence_proxy_async_smem();
