@@ -281,8 +281,16 @@ RET_API ret_status retention_recurrent_step(const void* q, const void* k, const 
  *   state: [N,H,dk,dv] float32, read and overwritten
  *   o: [N,Tn,H,dv] o_dtype
  * Supported: 1 <= Tn <= 16, dk and dv multiples of 4 with dk <= 512 and
- * dv <= 4096 (float32 FMAs on CUDA cores; the call is bound by the state's
- * HBM traffic); otherwise RET_ERR_UNSUPPORTED.
+ * dv <= 4096; otherwise RET_ERR_UNSUPPORTED.  Two paths, chosen per call:
+ *   tensor cores: in_dtype RET_BF16, Tn >= 12, dk in {128, 256}, dv a
+ *     multiple of 128 whose operand tiles fit in shared memory (up to 512 at
+ *     dk = 256, 768 at dk = 128).  The two products that touch every state
+ *     element run as tcgen05 MMAs of kind::tf32 on the float32 state (operands
+ *     read at tf32 precision, relative 2^-11; the state itself stays float32):
+ *     results are within the bf16-input tolerance.  Needs a device error word
+ *     (retention_check_device_error reports a bounded wait that ran out).
+ *   CUDA cores: every other case, float32 FMAs (exact to float32 rounding).
+ * Both are bound by the state's HBM traffic.
  */
 RET_API ret_status retention_recurrent_steps(const void* q, const void* k, const void* v,
                                              ret_dtype in_dtype, const double* gamma,

@@ -168,3 +168,17 @@ def test_tensor_core_bf16_output():
     o_ref, S_ref = _oracle(q, k, v, S0, gam)
     assert_close(f64(o), o_ref, "bf16", 2, "o bf16", stored_bf16=True)
     _check(S, S_ref, "bf16", dk, dv, 1, "state", Tn=Tn)
+
+
+def test_tensor_core_widest_value_head():
+    """d_k = 128 with d_v = 768 (six 128-column blocks, the widest whose operand
+    tiles fit), 13 tokens."""
+    N, Tn, H, dk, dv = 4, 13, 3, 128, 768
+    q, k, v, S0 = _inputs(N, Tn, H, dk, dv, "bf16", seed=71)
+    gam = W.head_gammas(H)
+    S = S0.clone().cuda()
+    o = ops.recurrent_steps(q.cuda(), k.cuda(), v.cuda(), gam, S)
+    ops.check_device_error()
+    o_ref, S_ref = _oracle(q, k, v, S0, gam)
+    _check(o, o_ref, "bf16", dk, dv, 2, "o", Tn=Tn)
+    _check(S, S_ref, "bf16", dk, dv, 1, "state", Tn=Tn)
