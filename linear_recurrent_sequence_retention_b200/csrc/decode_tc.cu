@@ -147,20 +147,23 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParam
       int it = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < p.nitems && ok; item += gridDim.x) {
-        // the next item's q, k, v rows into L2 while this item streams, so that the
-        // workers' operand tiles for it are formed from L2
-        const int nxt = item + gridDim.x;
-        if (nxt < p.nitems) {
-          const int hn = nxt % p.H, nn = nxt / p.H;
-          for (int t = 0; t < p.Tn; ++t) {
-            const size_t row = (static_cast<size_t>(nn) * p.Tn + t) * p.H + hn;
-            bulk_prefetch_l2(p.q + row * p.dk, static_cast<uint32_t>(p.dk * 2));
-            bulk_prefetch_l2(p.k + row * p.dk, static_cast<uint32_t>(p.dk * 2));
-            bulk_prefetch_l2(p.v + row * p.dv, static_cast<uint32_t>(p.dv * 2));
-          }
-        }
         for (int b = 0; b < nb && ok; ++b) {
           for (int q = 0; q < nq; ++q, ++it) {
+            if (b == nb - 1 && q == nq - 1) {
+              // the next item's q, k, v rows into L2 with this item's last stage:
+              // a few stages before the workers form its operand tiles (earlier,
+              // the state streaming through L2 would evict them first)
+              const int nxt = item + gridDim.x;
+              if (nxt < p.nitems) {
+                const int hn = nxt % p.H, nn = nxt / p.H;
+                for (int t = 0; t < p.Tn; ++t) {
+                  const size_t row = (static_cast<size_t>(nn) * p.Tn + t) * p.H + hn;
+                  bulk_prefetch_l2(p.q + row * p.dk, static_cast<uint32_t>(p.dk * 2));
+                  bulk_prefetch_l2(p.k + row * p.dk, static_cast<uint32_t>(p.dk * 2));
+                  bulk_prefetch_l2(p.v + row * p.dv, static_cast<uint32_t>(p.dv * 2));
+                }
+              }
+            }
             const int st = it % kDtStages;
             if (!mbar_wait(&empty[st], ((it / kDtStages) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
             mbar_arrive_expect_tx(&full[st], kDtStage);
