@@ -301,8 +301,12 @@ cudaError_t launch_decode_steps(const void* q, const void* k, const void* v, DTy
                                 float* state, void* o, DType o_t, int N, int Tn, int H, int dk,
                                 int dv, const HeadDecay& dec, unsigned* err, cudaStream_t s) {
   using bf = __nv_bfloat16;
-  if (in_t == DType::BF16 && decode_steps_tc_preferred(Tn, dk, dv))
-    return launch_decode_steps_tc(q, k, v, state, o, o_t, N, Tn, H, dk, dv, dec, err, s);
+  if (in_t == DType::BF16 && decode_steps_tc_preferred(Tn, dk, dv)) {
+    // cudaErrorNotSupported: the tensor-core kernel declined before launching
+    // anything (sizes past its index or tensor-map range); the CUDA-core one runs
+    const cudaError_t e = launch_decode_steps_tc(q, k, v, state, o, o_t, N, Tn, H, dk, dv, dec, err, s);
+    if (e != cudaErrorNotSupported) return e;
+  }
   if (in_t == DType::F32)
     return o_t == DType::F32 ? decode_multi<float, float>(q, k, v, state, o, N, Tn, H, dk, dv, dec, s)
                              : decode_multi<float, bf>(q, k, v, state, o, N, Tn, H, dk, dv, dec, s);

@@ -511,6 +511,8 @@ cudaError_t launch_decode_steps_tc(const void* q, const void* k, const void* v, 
                                    void* o, DType o_t, int N, int Tn, int H, int dk, int dv,
                                    const HeadDecay& dec, unsigned* err, cudaStream_t s) {
   if (!decode_steps_tc_supported(Tn, dk, dv)) return cudaErrorNotSupported;
+  const long long items = static_cast<long long>(N) * H;
+  if (items * dk >= (1ll << 31)) return cudaErrorNotSupported;
   auto fn = dt_encode_fn();
   if (!fn) return cudaErrorNotSupported;
   // the state as [N*H*dk rows][dv] float32, boxes of 32 columns x 64 rows
@@ -522,15 +524,13 @@ cudaError_t launch_decode_steps_tc(const void* q, const void* k, const void* v, 
   if (fn(&mS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, state, gdim, gstride, box, estr,
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+    return cudaErrorNotSupported;
   DecTcParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k = static_cast<const __nv_bfloat16*>(k);
   p.v = static_cast<const __nv_bfloat16*>(v);
   p.o = o;
   p.o_bf16 = o_t == DType::BF16 ? 1 : 0;
-  const long long items = static_cast<long long>(N) * H;
-  if (items * dk >= (1ll << 31)) return cudaErrorNotSupported;
   p.nitems = static_cast<int>(items);
   p.Tn = Tn;
   p.H = H;
