@@ -277,7 +277,7 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParam
       {
         constexpr int kQK = kDtMaxT * 256 / 8 / 256;     // 16-byte vectors of q (and of k) per thread at d_k = 256
         constexpr int kV = kDtMaxT * 512 / 8 / 256;      // of v at d_v = 512
-        const int nqk = kDtMaxT * p.dk / 8, nv = kDtMaxT * p.dv / 8;
+        const int nv = kDtMaxT * p.dv / 8;
         uint4 uq[kQK], uk[kQK], uv[kV];
 #pragma unroll
         for (int m = 0; m < kQK; ++m) {
@@ -309,7 +309,6 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParam
             dv4[1] = make_float4(xv[4], xv[5], xv[6], xv[7]);
           }
         }
-        (void)nqk;
 #pragma unroll
         for (int m = 0; m < kQK; ++m) {
           const int e8 = (wt + 256 * m) * 8, t = e8 / p.dk, i = e8 % p.dk;
