@@ -53,8 +53,8 @@
  *             RET_ERR_WORKSPACE) means nothing was enqueued and no output was
  *             touched; RET_ERR_CUDA means a launch failed and earlier kernels
  *             of the same call may have run.  RET_ERR_UNSUPPORTED means the
- *             arguments are valid but this build has no kernel for the shape
- *             or dtype combination; there is no fallback path.
+ *             arguments are valid but the library has no kernel for the
+ *             shape or dtype combination; there is no fallback path.
  *   Aliasing: outputs must not overlap inputs, except that
  *             retention_recurrent_step(s) update `state` in place by design
  *             and retention_rope may rotate q and k in place.
@@ -82,7 +82,7 @@ typedef struct CUstream_st* ret_stream_t; /* == cudaStream_t */
 typedef enum {
   RET_OK = 0,
   RET_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, gamma out of [0,1] */
-  RET_ERR_UNSUPPORTED = 2,   /* valid request with no kernel in this build */
+  RET_ERR_UNSUPPORTED = 2,   /* valid request with no kernel in the library */
   RET_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
   RET_ERR_TIMEOUT = 4,       /* a bounded device-side wait expired (from check_device_error) */
   RET_ERR_WORKSPACE = 5,     /* workspace missing or smaller than the size query returned */
