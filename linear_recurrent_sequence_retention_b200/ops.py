@@ -482,8 +482,11 @@ def recurrent_step(q, k, v, gamma, state, out_dtype=torch.float32, out=None, str
 
 
 def recurrent_steps(q, k, v, gamma, state, out_dtype=torch.float32, out=None, stream=None):
-    """Tn decode steps in one pass over the state; q,k: [N,Tn,H,dk], v: [N,Tn,H,dv];
-    updates ``state`` [N,H,dk,dv] in place and returns o [N,Tn,H,dv]."""
+    """Tn (<= 16) decode steps in one pass over the state; q,k: [N,Tn,H,dk], v: [N,Tn,H,dv];
+    updates ``state`` [N,H,dk,dv] in place and returns o [N,Tn,H,dv].  bf16 inputs with
+    Tn >= 12, dk in {128, 256} and dv a multiple of 128 run on the tensor cores (tf32
+    products on the float32 state, within the bf16-input tolerance); everything else runs
+    in float32 on CUDA cores."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (state, "state")):
         _dev(t, n)
     N, Tn, H, dk = q.shape
