@@ -15,10 +15,12 @@
 //
 // Persistent: one CTA per SM walks the (n, h) states.  Warp 0 streams the
 // state through a ring of 32 KB stages (64 rows x 128 columns, TMA, 128-byte
-// swizzle with 32-byte atoms, the layout MN-major tf32 operands take); warp 1 issues the MMAs; warps 2..9 form q_t gamma^(t+1), zeta_j
-// k_j and v as float32 operand tiles (and the Tn x Tn intra-step scores),
-// update every stage in place after its read MMA, store it back with TMA and
-// finally add the intra-step terms to the outputs.  Every wait is bounded.
+// swizzle with 32-byte atoms, the layout MN-major tf32 operands take) and
+// prefetches the next state's q, k, v rows into L2; warp 1 issues the MMAs;
+// warps 2..9 form q_t gamma^(t+1), zeta_j k_j and v as float32 operand tiles
+// (and the Tn x Tn intra-step scores), update every stage in place after its
+// read MMA, store it back with TMA and finally add the intra-step terms to the
+// outputs.  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include "launch.h"
