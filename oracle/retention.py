@@ -472,7 +472,7 @@ def softmax_features(x):
     return e / e.sum(axis=-1, keepdims=True)
 
 
-def rla(q, k, v, window, cu_seqlens=None, features_dtype=None):
+def rla(q, k, v, window, cu_seqlens=None):
     """Residual linear attention of ``q, k: [B,T,H,dk]``, ``v: [B,T,H,dv]``.
 
     RAttention page, section "Residual Linear Attention (RLA) 수식": a state
@@ -480,16 +480,10 @@ def rla(q, k, v, window, cu_seqlens=None, features_dtype=None):
     o_t = phi(q_t) S_(t-w-1), with S of a position before the sequence = 0
     (reading: the window w >= 0 counts the tokens the read skips, so o_t sees
     tokens m <= t - w - 1).  Run per (sequence, head) as the recurrence written
-    on the page.  ``features_dtype`` (e.g. torch.bfloat16) rounds phi(q) and
-    phi(k) to that type first, as a library that stores the mapped tensors in
-    the input dtype does.  Returns ``o [B,T,H,dv]``.
+    on the page, with phi evaluated in float64.  Returns ``o [B,T,H,dv]``.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     fq, fk = softmax_features(q), softmax_features(k)
-    if features_dtype is not None:
-        import torch
-        fq = torch.from_numpy(fq).to(features_dtype).double().numpy()
-        fk = torch.from_numpy(fk).to(features_dtype).double().numpy()
     B, T, H, dk = q.shape
     dv = v.shape[3]
     o = np.zeros((B, T, H, dv))

@@ -2,9 +2,11 @@
 fp64 oracle, through the C ABI.
 
 float32 inputs run on the CUDA-core retention and are held to relative L2 <=
-1e-5.  bf16 inputs run on the tensor-core kernels; the oracle rounds phi(q)
-and phi(k) to bf16 as the library stores them, and the output is held to the
-bf16-input tolerance (rel-L2 <= 1e-2, max-abs <= 3e-2 RMS plus the bf16 store).
+1e-5.  bf16 inputs run on the tensor-core kernels and are held to the
+bf16-input tolerance (rel-L2 <= 1e-2, max-abs <= 3e-2 RMS, plus the bf16 store
+where the output is stored as bf16) against the oracle's float64 feature map:
+the library's bf16 storage of phi(q) and phi(k) is part of the error measured,
+not of the reference.
 Cases: windows 0, small and the page's 512, the window past a sequence,
 packed sequences with empty and one-token ones.
 """
@@ -29,8 +31,7 @@ pytestmark = pytest.mark.gpu
 ])
 def test_rla_matches_oracle(dtype, B, T, H, dk, dv, window):
     q, k, v, _ = W.make_qkvg(B, T, H, dk, dv, dtype, seed=T + window, gate=False)
-    fdt = torch.bfloat16 if dtype == "bf16" else None
-    ref = oracle.rla(W.to_f64(q), W.to_f64(k), W.to_f64(v), window, features_dtype=fdt)
+    ref = oracle.rla(W.to_f64(q), W.to_f64(k), W.to_f64(v), window)
     out = ops.rla_fwd(q.cuda(), k.cuda(), v.cuda(), window, out_dtype=torch.float32)
     if window >= T - 1:
         assert torch.all(out == 0)
@@ -43,8 +44,7 @@ def test_rla_packed_sequences():
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     Tt = int(cu[-1])
     q, k, v, _ = W.make_qkvg(1, Tt, 2, 64, 128, "bf16", seed=5, gate=False)
-    ref = oracle.rla(W.to_f64(q), W.to_f64(k), W.to_f64(v), 64, cu_seqlens=cu,
-                     features_dtype=torch.bfloat16)
+    ref = oracle.rla(W.to_f64(q), W.to_f64(k), W.to_f64(v), 64, cu_seqlens=cu)
     out = ops.rla_fwd(q.cuda(), k.cuda(), v.cuda(), 64, cu_seqlens=torch.from_numpy(cu).cuda(),
                       out_dtype=torch.bfloat16)
     assert_close(W.to_f64(out), ref, "bf16", 2, "rla packed", stored_bf16=True)
@@ -64,6 +64,5 @@ def test_rla_bench_workload_sampled():
     out = ops.rla_fwd(q.cuda(), k.cuda(), v.cuda(), w, out_dtype=torch.float32)
     for b, h in ((0, 0), (3, 7)):
         sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
-        ref = oracle.rla(W.to_f64(q[sl]), W.to_f64(k[sl]), W.to_f64(v[sl]), w,
-                         features_dtype=torch.bfloat16)
+        ref = oracle.rla(W.to_f64(q[sl]), W.to_f64(k[sl]), W.to_f64(v[sl]), w)
         assert_close(W.to_f64(out[sl]), ref, "bf16", None, f"rla bench b{b} h{h}")
