@@ -86,7 +86,8 @@ typedef enum {
   RET_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
   RET_ERR_TIMEOUT = 4,       /* a bounded device-side wait expired (from check_device_error) */
   RET_ERR_WORKSPACE = 5,     /* workspace missing or smaller than the size query returned */
-  RET_ERR_DEVICE_DATA = 6    /* device-resident metadata (cu_seqlens) was inconsistent */
+  RET_ERR_DEVICE_DATA = 6,   /* device-resident metadata (cu_seqlens) was inconsistent */
+  RET_ERR_RANGE = 7          /* a tensor-core operand exceeded fp16's range (from check_device_error) */
 } ret_status;
 
 typedef enum { RET_F32 = 0, RET_BF16 = 1 } ret_dtype;

@@ -60,12 +60,23 @@ ret_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RET_OK : RET_E
 
 bool fits_int(long long x) { return x >= 0 && x < (1ll << 31); }
 
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+// Bytes of the tensor-core path's fp16 per-chunk states, and of its fp16 copy
+// of v (`width` values per token and head), each rounded to 256 B.
+size_t tc_state_bytes(long long slots, int H, int dk, int dv) {
+  return round256(static_cast<size_t>(slots) * H * dk * dv * 2);
+}
+size_t tc_v16_bytes(long long Ttot, int H, int width) {
+  return round256(static_cast<size_t>(Ttot) * H * width * 2);
+}
+
 struct ChunkPlan {
   ret::SeqLayout L;
   bool tc;
-  size_t elem;
   size_t meta;
   long long slots;
+  size_t v16_off;     // tensor-core path: offset of the fp16 copy of v (else 0)
   size_t bytes;
 };
 
@@ -90,11 +101,9 @@ ret_status plan_chunkwise(ret_dtype in_dtype, int chunk, int B, int T, int H, in
     if (!ret::chunkwise_tc_supported(dk, dv, chunk)) return RET_ERR_UNSUPPORTED;
     ce = ret::chunkwise_tc_chunk(chunk, dv);
     p->tc = true;
-    p->elem = 4;   // two bf16 planes per state element (hi and lo parts)
   } else {
     if (dk > 256 || dv > 256) return RET_ERR_UNSUPPORTED;
     p->tc = false;
-    p->elem = 4;
   }
   p->L.cu = varlen ? cu : nullptr;
   p->L.nseq = varlen ? nseq : B;
@@ -106,7 +115,14 @@ ret_status plan_chunkwise(ret_dtype in_dtype, int chunk, int B, int T, int H, in
   p->slots = varlen ? (Ttot + ce - 1) / ce + nseq
                     : static_cast<long long>(B) * ((T + ce - 1) / ce);
   p->L.nslots = p->slots;
-  p->bytes = p->meta + static_cast<size_t>(p->slots) * H * dk * dv * p->elem;
+  if (p->tc) {
+    // fp16 states, then the fp16 copy of v written by the state pass
+    p->v16_off = p->meta + tc_state_bytes(p->slots, H, dk, dv);
+    p->bytes = p->v16_off + tc_v16_bytes(Ttot, H, dv);
+  } else {
+    p->v16_off = 0;
+    p->bytes = p->meta + static_cast<size_t>(p->slots) * H * dk * dv * sizeof(float);
+  }
   return RET_OK;
 }
 
@@ -125,6 +141,8 @@ const char* retention_status_string(ret_status s) {
     case RET_ERR_TIMEOUT: return "RET_ERR_TIMEOUT: a bounded device wait expired";
     case RET_ERR_WORKSPACE: return "RET_ERR_WORKSPACE: workspace missing or too small";
     case RET_ERR_DEVICE_DATA: return "RET_ERR_DEVICE_DATA: inconsistent cu_seqlens";
+    case RET_ERR_RANGE:
+      return "RET_ERR_RANGE: a value exceeded the fp16 range of the tensor-core operands";
   }
   return "unknown ret_status";
 }
@@ -206,6 +224,8 @@ ret_status prepare_chunk_call(int phases, const void* q, const void* k, const vo
   c->ws.chunk_base = static_cast<int32_t*>(const_cast<void*>(workspace));
   c->ws.order = c->ws.chunk_base + c->p.L.nseq + 1;
   c->ws.states = static_cast<char*>(const_cast<void*>(workspace)) + c->p.meta;
+  c->ws.v16 = c->p.v16_off ? static_cast<char*>(const_cast<void*>(workspace)) + c->p.v16_off
+                           : nullptr;
   c->ws.nslots = c->p.slots;
   c->err = error_word();
   if (!c->err) return RET_ERR_CUDA;
@@ -354,7 +374,8 @@ struct BwdPlan {
   size_t bytes;         // CUDA-core path
   bool tc_ok;           // the tensor-core path is possible (bf16, heads 64/128/256)
   ret::SeqLayout Ltc;   // tensor-core path: the executed chunk
-  size_t tc_states;     // one set of hi/lo bf16 states at that chunk
+  size_t tc_state;      // one set of fp16 states at that chunk
+  size_t tc_states;     // + the fp16 copy of the value operand (the wider of d_k, d_v)
   size_t tc_bytes;      // tensor-core path: meta + states + scratch
 };
 
@@ -402,7 +423,8 @@ ret_status plan_chunkwise_bwd(ret_dtype in_dtype, int chunk, int B, int T, int H
     p->Ltc.chunk = ce;
     p->Ltc.nslots = varlen ? (Ttot + ce - 1) / ce + nseq
                            : static_cast<long long>(B) * ((T + ce - 1) / ce);
-    p->tc_states = static_cast<size_t>(p->Ltc.nslots) * H * dk * dv * 4;   // hi + lo bf16
+    p->tc_state = tc_state_bytes(p->Ltc.nslots, H, dk, dv);
+    p->tc_states = p->tc_state + tc_v16_bytes(Ttot, H, dk > dv ? dk : dv);
     p->tc_bytes = p->meta + p->tc_states + ret::chunkwise_bwd_tc_scratch_bytes(p->Ltc, H, dk, dv);
   }
   return RET_OK;
@@ -454,6 +476,7 @@ ret_status retention_chunkwise_bwd(const void* q, const void* k, const void* v, 
     tw.chunk_base = reinterpret_cast<int32_t*>(base);
     tw.order = tw.chunk_base + p.Ltc.nseq + 1;
     tw.states = base + p.meta;
+    tw.v16 = base + p.meta + p.tc_state;
     tw.nslots = p.Ltc.nslots;
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = ret::launch_chunk_prep(p.Ltc, tw, err, s);
@@ -467,6 +490,7 @@ ret_status retention_chunkwise_bwd(const void* q, const void* k, const void* v, 
   fw.chunk_base = reinterpret_cast<int32_t*>(base);
   fw.order = fw.chunk_base + p.L.nseq + 1;
   fw.states = base + p.meta;
+  fw.v16 = nullptr;
   fw.nslots = p.slots;
   ret::ChunkBwdWorkspace ws;
   ws.chunk_base = fw.chunk_base;
@@ -571,6 +595,7 @@ ret_status retention_rla_fwd(const void* q, const void* k, const void* v, ret_dt
   ws.chunk_base = reinterpret_cast<int32_t*>(base);
   ws.order = ws.chunk_base + r.cp.L.nseq + 1;
   ws.states = base + r.cp.meta;
+  ws.v16 = r.cp.v16_off ? base + r.cp.v16_off : nullptr;
   ws.nslots = r.cp.slots;
   auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
   const size_t el = in_dtype == RET_F32 ? 4 : 2;
@@ -616,6 +641,7 @@ ret_status retention_check_device_error(ret_stream_t stream) {
   }
   if (word & ret::kErrTimeout) return RET_ERR_TIMEOUT;
   if (word & ret::kErrDeviceData) return RET_ERR_DEVICE_DATA;
+  if (word & ret::kErrRange) return RET_ERR_RANGE;
   return RET_OK;
 }
 

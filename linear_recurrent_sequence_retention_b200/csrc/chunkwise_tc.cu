@@ -120,6 +120,21 @@ __device__ __forceinline__ bool wga_all(bool v) {
   return r != 0;
 }
 
+// AND of `v` over the 128 threads of warps 6..9 (named barrier 3); same
+// contract as wga_all.
+__device__ __forceinline__ bool wgb_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 3, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u)
+      : "memory");
+  return r != 0;
+}
+
 // ===========================================================================
 // State kernel
 // ===========================================================================
@@ -131,8 +146,8 @@ struct StateParams {
   const int32_t* order;              // varlen: sequences longest first (else nullptr)
   const float* state_in;
   float* state_out;
-  __nv_bfloat16* ws;                 // [nslots][H][2 (hi, lo)][dk][dv] bf16
   int H, dk, dv;
+  int write_v16;                     // the CTAs of the first d_k block store the fp16 copy of v
   HeadDecay dec;
   unsigned* err;
 };
@@ -141,10 +156,9 @@ template <int NS>
 struct StCfg {
   static constexpr uint32_t kKBytes = 2 * kBox;              // 64 tokens x 128 rows of d_k
   static constexpr uint32_t kVBytes = (NS / 64) * kBox;      // 64 tokens x NS
-  static constexpr uint32_t kStage = 2 * kKBytes + kVBytes;  // K hi | K lo | V
-  // staging for the TMA store of the state entering a chunk: one 128 x 64
-  // box of the hi plane and one of the lo plane
-  static constexpr uint32_t kStaging = 2 * kTallBox;
+  static constexpr uint32_t kStage = kKBytes + kVBytes;      // zeta*K | V, both fp16 in place
+  // staging for the TMA store of the state entering a chunk: one 128 x 64 fp16 box
+  static constexpr uint32_t kStaging = kTallBox;
   static constexpr int kStagesFit = static_cast<int>((232448 - kStaging - 1024) / kStage);
   static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
   static constexpr uint32_t kOffStaging = kStages * kStage;
@@ -154,7 +168,8 @@ struct StCfg {
 template <int NS>
 __global__ void __launch_bounds__(kThreads, 1)
 state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-             const __grid_constant__ CUtensorMap tmW, const StateParams p) {
+             const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmV16,
+             const StateParams p) {
   using SC = StCfg<NS>;
   constexpr int NSTG = SC::kStages;
   constexpr uint32_t kStage = SC::kStage;
@@ -182,6 +197,8 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
   const int s = p.order ? p.order[rank] : rank;
   const int m = zz % mblocks, part = zz / mblocks;
   const int kboxes = p.dk >= 128 ? 2 : 1;        // 64-column K boxes loaded per stage
+  // the fp16 copy of this CTA's value columns leaves from the V stages (first d_k block only)
+  const bool v16_out = p.write_v16 && m == 0;
   const SeqLayout& L = p.L;
   int a, b;
   seq_bounds(L, s, a, b);
@@ -191,7 +208,8 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
   if (threadIdx.x == 0) {
     for (int i = 0; i < NSTG; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      // released by the MMA, and by the copy store once it has read the stage
+      mbar_init(&empty[i], v16_out ? 2 : 1);
       mbar_init(&kready[i], kWgThreads);
     }
     mbar_init(acc_free, kWgThreads);
@@ -209,12 +227,11 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     tmem_relinquish();
   }
   if (kboxes == 1) {
-    // d_k = 64: the second 64-row half of every zeta*K tile (hi and lo) stays
-    // zero, so the 128-row MMA adds nothing to TMEM rows 64..127
+    // d_k = 64: the second 64-row half of every zeta*K tile stays zero, so the
+    // 128-row MMA adds nothing to TMEM rows 64..127
     for (int st = 0; st < NSTG; ++st)
       for (int o = threadIdx.x * 16; o < static_cast<int>(kBox); o += kThreads * 16)
-        for (int hl = 0; hl < 2; ++hl)
-          *reinterpret_cast<uint4*>(smem + st * kStage + hl * kKBytes + kBox + o) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(smem + st * kStage + kBox + o) = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
   tc_fence_before();
@@ -223,7 +240,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
   const uint32_t tmem = *tmem_hold;
 
   if (warp == 0) {
-    // ---------------- TMA producer: K rows (into the hi slot) and V ----------------
+    // ---------------- TMA producer: K rows and V rows (bf16) ----------------
     if (lane == 0 && !*abort_flag) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -241,7 +258,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
           for (int bx = 0; bx < kboxes; ++bx)
             tma_load_2d(base + bx * kBox, &tmK, &full[st], h * p.dk + 128 * m + 64 * bx, y);
           for (int bx = 0; bx < NS / 64; ++bx)
-            tma_load_2d(base + 2 * kKBytes + bx * kBox, &tmV, &full[st],
+            tma_load_2d(base + kKBytes + bx * kBox, &tmV, &full[st],
                         h * p.dv + NS * part + 64 * bx, y);
         }
       }
@@ -253,10 +270,10 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer: dS_c = (zeta K)_hi^T V + (zeta K)_lo^T V ----------------
+    // ---------------- MMA issuer: dS_c = (zeta K)^T V, fp16 operands ----------------
     // into accumulator c & 1 (the other one holds the state entering the chunk)
     if (lane == 0 && !*abort_flag) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, NS, true, true);
+      constexpr uint32_t idesc = idesc_f16_f32(128, NS, true, true);
       int it = 0;
       bool ok = true, issued = false;
       for (int c = 0; c < nch && ok; ++c) {
@@ -269,15 +286,12 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
           const int st = it % NSTG;
           if (!mbar_wait(&kready[st], (it / NSTG) & 1, abort_flag, p.err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t khi = smem_u32(smem + st * kStage);
-          const uint32_t klo = khi + kKBytes;
-          const uint32_t vb = khi + 2 * kKBytes;
+          const uint32_t zk = smem_u32(smem + st * kStage);
+          const uint32_t vb = zk + kKBytes;
 #pragma unroll
-          for (int ks = 0; ks < kStTok / 16; ++ks) {
-            const uint64_t bd = sdesc_sw128(vb + ks * 2048, kBox, 1024);
-            mma_bf16(acc, sdesc_sw128(khi + ks * 2048, kBox, 1024), bd, idesc, (sb | ks) != 0);
-            mma_bf16(acc, sdesc_sw128(klo + ks * 2048, kBox, 1024), bd, idesc, true);
-          }
+          for (int ks = 0; ks < kStTok / 16; ++ks)
+            mma_bf16(acc, sdesc_sw128(zk + ks * 2048, kBox, 1024), sdesc_sw128(vb + ks * 2048, kBox, 1024),
+                     idesc, (sb | ks) != 0);
           issued = true;
           mma_commit(&empty[st]);
         }
@@ -294,7 +308,8 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     // chunk's contribution dS_c into accumulator c & 1; then
     //     S_c = gamma^L S_(c-1) + dS_c   (written over dS_c)
     // releases the older accumulator for chunk c+1, and S_c (the state entering
-    // chunk c+1) goes to that chunk's workspace slot while chunk c+1 runs.
+    // chunk c+1) goes to that chunk's workspace slot, as fp16, while chunk c+1
+    // runs.
     const int quad = warp & 3;
     const int row = quad * 32 + lane;            // TMEM lane = row of the state block
     const int i = 128 * m + row;                 // d_k index
@@ -303,46 +318,45 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     const size_t st_off = ((static_cast<size_t>(s) * p.H + h) * p.dk + (row_ok ? i : 0)) * p.dv + NS * part;
     const bool leader = threadIdx.x == 64;
     if (leader) tma_prefetch_desc(&tmW);
+    bool range_ok = true;
     auto slot_of = [&](int c) -> long long {
       return L.cu == nullptr ? static_cast<long long>(s) * ceil_div(L.T, L.chunk) + c
                              : static_cast<long long>(p.chunk_base[s]) + c;
     };
-    // The state in accumulator column `col` -> workspace slot `slot` as a hi/lo
-    // bf16 pair, one 128 x 64 box of each plane per TMA store.  Barrier 2 is
-    // reached by all 128 threads the same number of times.
+    // The state in accumulator column `col` -> workspace slot `slot` as fp16,
+    // one 128 x 64 box per TMA store.  Barrier 2 is reached by all 128 threads
+    // the same number of times.
     auto stage_state = [&](uint32_t col, long long slot) {
       const bool slot_ok = slot >= 0 && slot < L.nslots;
-      // workspace rows of this CTA's 128 d_k rows in the hi plane; lo follows dk rows later
-      const int wrow = static_cast<int>(((slot_ok ? slot : 0) * p.H + h) * 2 * p.dk) + 128 * m;
+      // workspace rows of this CTA's 128 d_k rows
+      const int wrow = static_cast<int>(((slot_ok ? slot : 0) * p.H + h) * p.dk) + 128 * m;
 #pragma unroll 1
       for (int j = 0; j < NS / 32; j += 2) {
         float r[2][32];
         tmem_ld32(trow + col + 32 * j, r[0]);
         tmem_ld32(trow + col + 32 * (j + 1), r[1]);
         tmem_wait_ld();
-        // the staging boxes are free once the previous store stopped reading them
+        // the staging box is free once the previous store stopped reading it
         if (leader) tma_store_wait_read();
         asm volatile("bar.sync 2, 128;" ::: "memory");
-        // row `row` of two 128 x 64 swizzled boxes (hi, lo): 16-byte piece cc of
-        // the row goes to piece cc ^ (row & 7)
+        // row `row` of a 128 x 64 swizzled box: 16-byte piece cc of the row
+        // goes to piece cc ^ (row & 7)
+        float amax = 0.f;
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
           const float* x = &r[cc >> 2][(cc & 3) * 8];
-          uint4 uh, ul;
-          pack_split(x[0], x[1], uh.x, ul.x);
-          pack_split(x[2], x[3], uh.y, ul.y);
-          pack_split(x[4], x[5], uh.z, ul.z);
-          pack_split(x[6], x[7], uh.w, ul.w);
-          const int off = row * 128 + ((cc ^ (row & 7)) << 4);
-          *reinterpret_cast<uint4*>(staging + off) = uh;
-          *reinterpret_cast<uint4*>(staging + kTallBox + off) = ul;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
+          const uint4 u = make_uint4(pack_f16(x[0], x[1]), pack_f16(x[2], x[3]),
+                                     pack_f16(x[4], x[5]), pack_f16(x[6], x[7]));
+          *reinterpret_cast<uint4*>(staging + row * 128 + ((cc ^ (row & 7)) << 4)) = u;
         }
+        range_ok = range_ok && !(amax > kF16Max);    // NaN passes here; it is not a range event
         fence_proxy_async_smem();
         asm volatile("bar.sync 2, 128;" ::: "memory");
         if (leader && slot_ok) {
-          // boxes of min(d_k, 128) rows: the first rows of the staged boxes
+          // a box of min(d_k, 128) rows: the first rows of the staged box
           tma_store_2d(&tmW, staging, NS * part + 32 * j, wrow);
-          tma_store_2d(&tmW, staging + kTallBox, NS * part + 32 * j, wrow + p.dk);
           tma_store_commit();
         }
       }
@@ -397,6 +411,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       if (c + 1 < nch) stage_state(dcol, slot_of(c + 1));
     }
     if (leader) tma_store_wait_all();
+    if (!range_ok) raise_error(p.err, kErrRange);
     // final state: S_(nch-1), in accumulator (nch-1) & 1
     if (ok && nch > 0) {
       if (p.state_out) {
@@ -420,44 +435,104 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       }
     }
   } else {
-    // ---------------- warpgroup B: zeta*K as hi/lo tiles, ahead of the MMA ----------------
-    const int t = threadIdx.x - 192;              // 0..127: box t/64, token row t%64
+    // ---------------- warpgroup B: the fp16 MMA operands, ahead of the MMA ----------------
+    // K rows -> zeta*K (fp16, in place), V rows -> fp16 (in place); the first
+    // d_k block's CTAs also store the converted V rows as the fp16 copy of v
+    // that the output pass reads.
+    const int t = threadIdx.x - 192;              // 0..127
+    const bool leader = t == 0;
+    if (leader && v16_out) tma_prefetch_desc(&tmV16);
     int it = 0;
-    bool ok = !*abort_flag;
+    bool ok = !*abort_flag, range_ok = true;
+    int pending_st = -1;                          // stage whose copy store may still be reading it
     for (int c = 0; c < nch && ok; ++c) {
-      const int Lc = min(L.chunk, b - (a + c * L.chunk));
+      const int tok0 = a + c * L.chunk;
+      const int Lc = min(L.chunk, b - tok0);
       for (int sb = 0; sb * kStTok < Lc; ++sb, ++it) {
         const int st = it % NSTG;
-        if (!mbar_wait(&full[st], (it / NSTG) & 1, abort_flag, p.err)) { ok = false; break; }
-        const int jtok = sb * kStTok + (t & 63);
-        const float z = jtok < Lc ? dec.pow(Lc - 1 - jtok) : 0.f;
-        uint8_t* rowb = smem + st * kStage + (t >> 6) * kBox + (t & 63) * 128;
-        uint4* hp = reinterpret_cast<uint4*>(rowb);
-        uint4* lp = reinterpret_cast<uint4*>(rowb + kKBytes);
-        // every piece of the row gets the same factor, so visit the row's eight
-        // 16-byte pieces in the order e ^ (row & 7): lanes of 8 consecutive rows then
-        // touch 8 different bank groups instead of the same one
-        const int sw = t & 7;
-        uint4 u[8];
+        // uniform over the warpgroup: the named barrier below stays matched
+        if (!wgb_all(mbar_wait(&full[st], (it / NSTG) & 1, abort_flag, p.err))) { ok = false; break; }
+        uint8_t* stage = smem + st * kStage;
+        {
+          // zeta*K: thread t owns box t/64, token row t%64 (one 128-byte row)
+          const int jtok = sb * kStTok + (t & 63);
+          const float z = jtok < Lc ? dec.pow(Lc - 1 - jtok) : 0.f;
+          uint4* rp = reinterpret_cast<uint4*>(stage + (t >> 6) * kBox + (t & 63) * 128);
+          // every piece of the row gets the same factor, so visit the row's eight
+          // 16-byte pieces in the order e ^ (row & 7): lanes of 8 consecutive rows then
+          // touch 8 different bank groups instead of the same one
+          const int sw = t & 7;
+          if (t < 64 * kboxes) {
+            uint4 u[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) u[e] = hp[e ^ sw];
-        const uint64_t z2 = f2_make(z, z);
+            for (int e = 0; e < 8; ++e) u[e] = rp[e ^ sw];
+            const uint64_t z2 = f2_make(z, z);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint32_t w[4] = {u[e].x, u[e].y, u[e].z, u[e].w};
-          uint32_t wh[4], wl[4];
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t w[4] = {u[e].x, u[e].y, u[e].z, u[e].w};
+              uint32_t wh[4];
 #pragma unroll
-          for (int q2 = 0; q2 < 4; ++q2) {
-            const uint64_t p2 = f2_mul(f2_make(bf16_lo(w[q2]), bf16_hi(w[q2])), z2);
-            pack_split(f2_lo(p2), f2_hi(p2), wh[q2], wl[q2]);
+              for (int q2 = 0; q2 < 4; ++q2) {
+                const uint64_t p2 = f2_mul(f2_make(bf16_lo(w[q2]), bf16_hi(w[q2])), z2);
+                wh[q2] = pack_f16(f2_lo(p2), f2_hi(p2));
+              }
+              rp[e ^ sw] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            }
           }
-          hp[e ^ sw] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-          lp[e ^ sw] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        }
+        {
+          // V: (NS/64) boxes x 64 rows of 128 bytes, converted bf16 -> fp16
+          uint8_t* vbase = stage + kKBytes;
+          constexpr int kVRows = (NS / 64) * 64;
+          for (int rr = t; rr < kVRows; rr += kWgThreads) {
+            uint4* rp = reinterpret_cast<uint4*>(vbase + rr * 128);
+            const int sw = rr & 7;
+            uint4 u[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) u[e] = rp[e ^ sw];
+            uint32_t bad = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const uint4 f = make_uint4(bf16x2_to_f16x2(u[e].x), bf16x2_to_f16x2(u[e].y),
+                                         bf16x2_to_f16x2(u[e].z), bf16x2_to_f16x2(u[e].w));
+              // an fp16 infinity from a finite bf16 value: |v| > 65504
+              const uint32_t wv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+              for (int q2 = 0; q2 < 4; ++q2) {
+                const uint32_t lo = wv[q2] & 0x7fffu, hi = (wv[q2] >> 16) & 0x7fffu;
+                bad |= (lo == 0x7c00u) | (hi == 0x7c00u);
+              }
+              rp[e ^ sw] = f;
+            }
+            // rows past the sequence's end hold other tokens (or the zero fill)
+            // and may overflow without concerning this sequence
+            const int jtok = sb * kStTok + (rr & 63);
+            if (bad && jtok < Lc) range_ok = false;
+          }
         }
         fence_proxy_async_smem();
         mbar_arrive(&kready[st]);
+        if (v16_out) {
+          // all 128 threads' V rows are written: store them as the fp16 copy
+          asm volatile("bar.sync 3, 128;" ::: "memory");
+          if (leader) {
+            const int y = tok0 + sb * kStTok;
+            for (int bx = 0; bx < NS / 64; ++bx)
+              tma_store_2d(&tmV16, stage + kKBytes + bx * kBox, h * p.dv + NS * part + 64 * bx, y);
+            tma_store_commit();
+            // the previous stage's copy has been read out of shared memory
+            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+            if (pending_st >= 0) mbar_arrive(&empty[pending_st]);
+            pending_st = st;
+          }
+        }
       }
     }
+    if (v16_out && leader) {
+      tma_store_wait_all();
+      if (pending_st >= 0) mbar_arrive(&empty[pending_st]);
+    }
+    if (!range_ok) raise_error(p.err, kErrRange);
   }
   tc_fence_before();
   __syncthreads();
@@ -502,7 +577,7 @@ struct OutCfg {
   static constexpr uint32_t kQBytes = (DK / 64) * kTallBox;
   // The gate/output tile (NV/64 boxes of 128 rows x 64 columns) has a buffer of
   // its own: held through the epilogue tail, it would otherwise pin ring stages
-  // that the next tile's state and key loads are waiting for.
+  // that the next tile's key loads are waiting for.
   static constexpr uint32_t kGateBytes = (NV / 64) * kTallBox;
   // barriers | gamma^d table | GroupNorm pairs passed between the two
   // warpgroups | GroupNorm pairs received from the partner CTA
@@ -513,14 +588,14 @@ struct OutCfg {
   static constexpr uint32_t kOffStages = kOffGate + kGateBytes;
   static constexpr uint32_t kOffMisc = kOffStages + kStages * kOutStage;
   static constexpr uint32_t kSmem = kOffMisc + kMiscBytes;
-  // TMEM: two halves of 256 columns used in turn.  Tile number n of a CTA
-  // keeps O in half (n & 1) and its two 128-column score buffers in the other
-  // half, so the next tile's Q S MMAs run while this tile's epilogue still
-  // reads O.  P of key piece j (keys 32j..32j+31) is written over that piece's
-  // own score columns: 32j..32j+15 hold P_hi (two keys per column),
-  // 32j+16..32j+31 hold P_lo.
-  static constexpr uint32_t kHalfCols = 256;
+  // TMEM (fixed): O in columns [0, NV), score buffers 0 and 1 in [256, 384)
+  // and [384, 512).  P of key piece j (keys 32j..32j+31) is written as fp16
+  // over the first 16 of that piece's own 32 score columns (two keys per
+  // column); the decayed query rows that read the carried state (d_k values,
+  // two per column) take a whole score buffer.
+  static constexpr uint32_t kColSB = 256;
 };
+
 
 // One 128-row output tile: rows 128r..128r+127 of a chunk, one head, all d_v
 // columns of this CTA's part.
@@ -605,13 +680,13 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   uint64_t* full = bars;                 // [NST] stage loaded
   uint64_t* empty = full + NST;          // [NST] stage consumed
   uint64_t* bar_q = empty + NST;         // Q tile loaded
-  uint64_t* q_free = bar_q + 1;          // every MMA reading Q has completed
-  uint64_t* bar_inter = q_free + 1;      // O = Q S done
-  uint64_t* bar_s = bar_inter + 1;       // [2] scores ready in TMEM
+  uint64_t* q_free = bar_q + 1;          // every MMA and every epilogue read of Q is done
+  uint64_t* bar_s = q_free + 1;          // [2] scores ready in TMEM
   uint64_t* bar_p = bar_s + 2;           // [2] P written over the scores
-  uint64_t* bar_o = bar_p + 2;           // all MMAs of the tile done
-  uint64_t* o_free = bar_o + 1;          // the epilogue has read the tile's O
-  uint64_t* drain = o_free + 1;
+  uint64_t* pv_done = bar_p + 2;         // [2] the P V MMAs of a score buffer are done
+  uint64_t* bar_pp = pv_done + 2;        // decayed query rows written (state read operand)
+  uint64_t* bar_o = bar_pp + 1;          // all MMAs of the tile done
+  uint64_t* drain = bar_o + 1;
   uint64_t* bar_x = drain + 1;           // the partner's statistics have arrived
   uint64_t* bar_xack = bar_x + 1;        // the partner has read this CTA's statistics
   uint64_t* g_full = bar_xack + 1;       // the gate tile has landed in the gate buffer
@@ -632,8 +707,6 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   // the gate/output tile: NV/64 boxes of 128 rows x 64 columns in the gate buffer
   constexpr int kIoBoxes = NV / 64;
   uint8_t* const gate_buf = smem + C::kOffGate;
-  // ring units of a tile: its MMA operands
-  auto mma_units = [&](const OutTile& t) { return (t.inter ? 2 * (DK / 64) : 0) + (t.r + 1) * (kKU + 2); };
   auto io_staged = [&](const OutTile& t) {
     return (p.gated && p.g_tma) || (p.y_tma && t.nrows == kRowsPerTile);
   };
@@ -644,14 +717,14 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mbar_init(&empty[i], 1);
     }
     mbar_init(bar_q, 1);
-    mbar_init(q_free, 1);
-    mbar_init(bar_inter, 1);
+    mbar_init(q_free, 1 + 2 * kWgThreads);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_s[i], 1);
       mbar_init(&bar_p[i], 2 * kWgThreads);
+      mbar_init(&pv_done[i], 1);
     }
+    mbar_init(bar_pp, 2 * kWgThreads);
     mbar_init(bar_o, 1);
-    mbar_init(o_free, 2 * kWgThreads);
     mbar_init(drain, 1);
     mbar_init(bar_x, kWgThreads);
     mbar_init(bar_xack, kWgThreads);
@@ -679,12 +752,11 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   OutTile t;
 
   // Per tile, the ring units in the order the MMA consumes them (32 KB each):
-  //   [S_hi and S_lo of d_k rows 64u..64u+63, u < DK/64 (if the chunk reads a state)],
-  //   K(0), then for kb = 0..r: [K(kb+1) if kb < r], V(kb) keys 0-63, V(kb) keys 64-127,
-  //   then the gate tile (or, with a bf16 output and no TMA gate, the same
-  //   number of empty units reserved as output staging).
-  // The ring runs on across tiles, so the next tile's Q, state and first key
-  // block stream in during this tile's epilogue.
+  //   K(0), then for kb = 0..r: [K(kb+1) if kb < r], V(kb) keys 0-63, V(kb) keys 64-127
+  //   (fp16 copy of v), then [S of d_k rows 64u..64u+63, u < DK/64 (fp16), if
+  //   the chunk reads a state].  The gate tile goes to its own buffer.
+  // The ring runs on across tiles, so the next tile's first key blocks stream
+  // in during this tile's epilogue.
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0 && !*abort_flag) {
@@ -703,24 +775,12 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       };
       while (ok && walk.next(p, cid, t)) {
         const int r = t.r;
-        // Q of this tile, once every MMA of the previous tile that reads Q is done
+        // Q of this tile, once the previous tile's MMAs and epilogue are done with Q
         if (tq > 0 && !mbar_wait(q_free, (tq - 1) & 1, abort_flag, p.err)) { ok = false; break; }
         mbar_arrive_expect_tx(bar_q, C::kQBytes);
         for (int u = 0; u < DK / 64; ++u)
           tma_load_2d(smem + u * kTallBox, &tmQ, bar_q, t.h * DK + 64 * u, t.t0);
         ++tq;
-        if (t.inter) {
-          for (int u = 0; u < DK / 64 && ok; ++u) {
-            for (int hl = 0; hl < 2 && ok; ++hl) {
-              const int srow = static_cast<int>(((t.slot * p.H + t.h) * 2 + hl) * DK) + 64 * u;
-              uint8_t* dst = next((NV / 64) * kBox);
-              if (!dst) { ok = false; break; }
-              for (int bx = 0; bx < NV / 64; ++bx)
-                tma_load_2d(dst + bx * kBox, &tmS, &full[it % NST], NV * part + 64 * bx, srow);
-              ++it;
-            }
-          }
-        }
         auto load_k = [&](int kb) {
           for (int ku = 0; ku < kKU && ok; ++ku) {
             uint8_t* dst = next(kKB * kTallBox);
@@ -746,6 +806,16 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           if (kb + 1 <= r) load_k(kb + 1);
           load_v(kb);
         }
+        if (ok && t.inter) {
+          for (int u = 0; u < DK / 64 && ok; ++u) {
+            const int srow = static_cast<int>((t.slot * p.H + t.h) * DK) + 64 * u;
+            uint8_t* dst = next((NV / 64) * kBox);
+            if (!dst) { ok = false; break; }
+            for (int bx = 0; bx < NV / 64; ++bx)
+              tma_load_2d(dst + bx * kBox, &tmS, &full[it % NST], NV * part + 64 * bx, srow);
+            ++it;
+          }
+        }
         if (ok && io_staged(t)) {
           // the gate/output buffer, once the previous staged tile's stores have read it
           if (!mbar_wait(g_empty, (ng & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
@@ -770,13 +840,17 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    // Per tile:  Sc(0), Sc(1);  for kb: [P(kb)] O (+)= P(kb) V(kb), Sc(kb+2);
+    // then [decayed Q rows] O += Qd S.  The first P V of a tile overwrites O:
+    // its P is formed only after the epilogue has finished with the previous
+    // tile's O.
     if (lane == 0 && !*abort_flag) {
-      constexpr uint32_t id_qs = idesc_bf16_f32(128, NV, false, true);
       constexpr uint32_t id_qk = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t id_pv = idesc_bf16_f32(128, NV, false, true);
+      constexpr uint32_t id_pv = idesc_f16_f32(128, NV, false, true);
       const uint32_t q_base = smem_u32(smem);
       const uint32_t st_base = smem_u32(smem + C::kOffStages);
-      int it = 0, tq = 0, sblk = 0;
+      const uint32_t sbuf0 = tmem + C::kColSB;
+      int it = 0, tq = 0, sblk = 0, npp = 0;   // npp: tiles that read a carried state
       bool ok = true, issued = false;
       auto stage_wait = [&]() -> uint32_t {
         const int st = it % NST;
@@ -790,33 +864,10 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       };
       while (ok && walk.next(p, cid, t)) {
         const int r = t.r;
-        const uint32_t o_t = tmem + (tq & 1) * C::kHalfCols;          // this tile's O
-        const uint32_t s_t = tmem + ((tq & 1) ^ 1) * C::kHalfCols;    // its score buffers
         if (!mbar_wait(bar_q, tq & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
-        if (t.inter) {
-          // O = Q S_hi + Q S_lo  (the state entering the chunk, split in two bf16 parts),
-          // into the half that held the previous tile's scores
-          for (int u = 0; u < DK / 64 && ok; ++u) {
-            for (int hl = 0; hl < 2; ++hl) {
-              const uint32_t sb = stage_wait();
-              if (!sb) { ok = false; break; }
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(o_t, sdesc_sw128(q_base + u * kTallBox + kk * 32, 16, 1024),
-                         sdesc_sw128(sb + kk * 2048, kBox, 1024), id_qs, (u | hl | kk) != 0);
-              issued = true;
-              stage_free();
-            }
-          }
-          if (!ok) break;
-          mma_commit(bar_inter);
-        }
-        // the scores go over the previous tile's O: wait until its epilogue has read it
-        if (tq > 0 && !mbar_wait(o_free, (tq - 1) & 1, abort_flag, p.err)) { ok = false; break; }
-        tc_fence_after();
         auto issue_qk = [&](int kb) -> bool {
-          const uint32_t dst = s_t + 128 * (kb & 1);
+          const uint32_t dst = sbuf0 + 128 * (kb & 1);
           for (int ku = 0; ku < kKU; ++ku) {
             const uint32_t sb = stage_wait();
             if (!sb) return false;
@@ -831,32 +882,52 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             stage_free();
           }
           mma_commit(&bar_s[(sblk + kb) & 1]);
-          if (kb == r) mma_commit(q_free);     // Q may be replaced by the next tile's
+          if (kb == r) mma_commit(q_free);     // the MMAs are done with Q
           return true;
         };
         if (!issue_qk(0)) { ok = false; break; }
+        if (r >= 1 && !issue_qk(1)) { ok = false; break; }
         for (int kb = 0; kb <= r && ok; ++kb) {
-          // scores of the next key block go to the other buffer while P_kb is formed
-          if (kb + 1 <= r && !issue_qk(kb + 1)) { ok = false; break; }
           const int sg = sblk + kb;
           if (!mbar_wait(&bar_p[sg & 1], (sg >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t pbuf = s_t + 128 * (kb & 1);
+          const uint32_t pbuf = sbuf0 + 128 * (kb & 1);
           for (int vu = 0; vu < 2; ++vu) {
             const uint32_t sb = stage_wait();
             if (!sb) { ok = false; break; }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const int ks = vu * 4 + kk;                      // keys 16ks .. 16ks+15
-              const uint32_t a_hi = pbuf + 32 * (ks >> 1) + 8 * (ks & 1);
-              const uint64_t bd = sdesc_sw128(sb + kk * 2048, kBox, 1024);
-              mma_bf16_ts(o_t, a_hi, bd, id_pv, t.inter || kb > 0 || ks > 0);
-              mma_bf16_ts(o_t, a_hi + 16, bd, id_pv, true);
+              mma_bf16_ts(tmem, pbuf + 32 * (ks >> 1) + 8 * (ks & 1),
+                          sdesc_sw128(sb + kk * 2048, kBox, 1024), id_pv, kb > 0 || ks > 0);
             }
             stage_free();
           }
+          if (!ok) break;
+          mma_commit(&pv_done[sg & 1]);
+          // the next scores go to the buffer this P V has just been issued from
+          // (tcgen05 MMAs of one thread execute in issue order)
+          if (kb + 2 <= r && !issue_qk(kb + 2)) { ok = false; break; }
         }
         if (!ok) break;
+        if (t.inter) {
+          // O += (gamma^(i+1) q_i) S: the decayed query rows (fp16, in the score
+          // buffer after the last one used) times the carried state (fp16)
+          if (!mbar_wait(bar_pp, npp & 1, abort_flag, p.err)) { ok = false; break; }
+          ++npp;
+          tc_fence_after();
+          const uint32_t abuf = sbuf0 + 128 * ((r + 1) & 1);
+          for (int u = 0; u < DK / 64 && ok; ++u) {
+            const uint32_t sb = stage_wait();
+            if (!sb) { ok = false; break; }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ts(tmem, abuf + 32 * u + 8 * kk, sdesc_sw128(sb + kk * 2048, kBox, 1024),
+                          id_pv, true);
+            stage_free();
+          }
+          if (!ok) break;
+        }
         mma_commit(bar_o);
         sblk += r + 1;
         ++tq;
@@ -867,25 +938,27 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
     }
   } else {
-    // ---------------- epilogue: warpgroup wg owns key pieces 2wg, 2wg+1 and O columns
+    // ---------------- epilogue: warpgroup wg owns key pieces 2wg, 2wg+1, d_k
+    // columns [wg*DK/2, (wg+1)*DK/2) of the decayed query rows, and O columns
     // [wg*NV/2, (wg+1)*NV/2) ----------------
     const int wg = (warp - 2) >> 2;                   // 0 or 1
     const int quad = warp & 3;
     const int row = quad * 32 + lane;                 // query row within the block
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t o_cols = tmem + lane_off + wg * kHalf;
+    const uint32_t sbuf0 = tmem + lane_off + C::kColSB;
     const int et = threadIdx.x - 64;                  // 0..255
     const bool wg_leader = (et & 127) == 0;           // first thread of the warpgroup
     constexpr bool kBoxPerWg = kHalf >= 64;           // each warpgroup owns whole boxes
     const uint32_t other = xchg ? (cluster_ctarank() ^ 1u) : 0u;
-    int tq = 0, sblk = 0, ninter = 0, ng = 0;
+    int tq = 0, sblk = 0, ng = 0;
     bool ok = true;
+    float pmax = 0.f;                                 // largest |P| and |decayed q| formed
     while (walk.next(p, cid, t)) {
       // uniform over the 256 epilogue threads: the named barriers below stay matched
       if (!epi_all(ok && !*abort_flag)) break;
       const int r = t.r;
       const int i = r * kRowsPerTile + row;            // row within the chunk
-      const uint32_t o_cols = tmem + lane_off + (tq & 1) * C::kHalfCols + wg * kHalf;
-      const uint32_t s_t = tmem + lane_off + ((tq & 1) ^ 1) * C::kHalfCols;
       const bool staged = io_staged(t);
       auto io_box = [&](int bx) -> uint8_t* { return gate_buf + bx * kTallBox; };
       const Decay1 dec(p.dec, t.h);
@@ -893,24 +966,6 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       // epilogue thread passed the barrier in epi_all above after forming it)
       if (et < 128) pow_tab[et] = dec.pow(et);
       wg2_sync();
-      if (t.inter) {
-        // tcgen05.ld/st are warp-collective: every guard around them is warp-uniform
-        ok = warp_all(ok && mbar_wait(bar_inter, ninter & 1, abort_flag, p.err));
-        ++ninter;
-        if (ok) {
-          tc_fence_after();
-          const float sc = dec.pow(i + 1);
-          for (int j = 0; j < kHalf / 32; ++j) {
-            float x[32];
-            tmem_ld32(o_cols + 32 * j, x);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] *= sc;
-            tmem_st32(o_cols + 32 * j, x);
-          }
-          tmem_wait_st();
-        }
-      }
       for (int kb = 0; kb <= r && ok; ++kb) {
         const int sg = sblk + kb;
         if (!warp_all(mbar_wait(&bar_s[sg & 1], (sg >> 1) & 1, abort_flag, p.err))) { ok = false; break; }
@@ -919,7 +974,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         // off-diagonal: gamma^(i-j) = gamma^(i - 128kb - 127) * gamma^(127 - j')
         const float arow = diag ? 0.f : dec.pow(i - kKeysPerBlock * kb - 127);
         const int key_lim = t.si.len - kKeysPerBlock * kb;   // keys j' >= key_lim are past the chunk
-        const uint32_t buf = s_t + 128 * (kb & 1);
+        const uint32_t buf = sbuf0 + 128 * (kb & 1);
 #pragma unroll 1
         for (int j = 2 * wg; j < 2 * wg + 2; ++j) {
           float x[32];
@@ -949,21 +1004,59 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               if (32 * j + e >= key_lim) wv[e] = 0.f;
           }
           tmem_wait_ld();
-          float pw[32];
+          uint32_t pw[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            uint32_t hi, lo;
             const uint64_t p2 = f2_mul(f2_make(x[e], x[e + 1]), f2_make(wv[e], wv[e + 1]));
-            pack_split(f2_lo(p2), f2_hi(p2), hi, lo);
-            pw[e >> 1] = __uint_as_float(hi);
-            pw[16 + (e >> 1)] = __uint_as_float(lo);
+            pmax = fmaxf(pmax, fmaxf(fabsf(f2_lo(p2)), fabsf(f2_hi(p2))));
+            pw[e >> 1] = pack_f16(f2_lo(p2), f2_hi(p2));
           }
-          tmem_st32(buf + 32 * j, pw);
+          tmem_st16(buf + 32 * j, pw);
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bar_p[sg & 1]);
       }
+      if (t.inter && ok) {
+        // the decayed query rows gamma^(i+1) q_i (fp16) into the score buffer
+        // after the last one used, once the P V MMAs that read it are done
+        if (r >= 1) {
+          const int sg = sblk + r - 1;
+          ok = warp_all(mbar_wait(&pv_done[sg & 1], (sg >> 1) & 1, abort_flag, p.err));
+          if (ok) tc_fence_after();
+        }
+        // the Q tile's TMA writes are visible to this thread's loads (Q is not
+        // reloaded before this thread releases it through q_free)
+        if (ok) ok = warp_all(mbar_wait(bar_q, tq & 1, abort_flag, p.err));
+        if (ok) {
+          const float sc = dec.pow(i + 1);
+          const uint64_t sc2 = f2_make(sc, sc);
+          const uint32_t abuf = sbuf0 + 128 * ((r + 1) & 1);
+          // this warpgroup's d_k columns: half-box pieces of 32 values
+#pragma unroll 1
+          for (int c0 = wg * (DK / 2); c0 < (wg + 1) * (DK / 2); c0 += 32) {
+            const uint8_t* qrow = smem + (c0 >> 6) * kTallBox + row * 128;
+            const int pc0 = (c0 & 63) >> 3;            // first 16-byte piece of the 32 values
+            uint32_t pw[16];
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const uint4 u = *reinterpret_cast<const uint4*>(qrow + (((pc0 + c4) ^ (row & 7)) << 4));
+              const uint32_t wq[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int q2 = 0; q2 < 4; ++q2) {
+                const uint64_t d2 = f2_mul(f2_make(bf16_lo(wq[q2]), bf16_hi(wq[q2])), sc2);
+                pmax = fmaxf(pmax, fmaxf(fabsf(f2_lo(d2)), fabsf(f2_hi(d2))));
+                pw[4 * c4 + q2] = pack_f16(f2_lo(d2), f2_hi(d2));
+              }
+            }
+            tmem_st16(abuf + (c0 >> 1), pw);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+        }
+        mbar_arrive(bar_pp);
+      }
+      mbar_arrive(q_free);                             // this thread is done reading Q
       sblk += r + 1;
       ok = warp_all(ok && mbar_wait(bar_o, tq & 1, abort_flag, p.err));
       if (ok) tc_fence_after();
@@ -1151,10 +1244,9 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           }
         }
       }
-      // every read of this tile's O is complete: its TMEM half may take the
-      // next tile's scores
+      // every read of this tile's O is complete before this thread forms the
+      // next tile's first P (which lets the MMA overwrite O)
       tc_fence_before();
-      mbar_arrive(o_free);
       if (!kBoxPerWg && out_tma) {                   // boxes shared by both warpgroups
         fence_proxy_async_smem();
         wg2_sync();
@@ -1174,6 +1266,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
       ++tq;
     }
+    if (pmax > kF16Max) raise_error(p.err, kErrRange);
   }
   if (xchg) {
     if (!cluster_waited) cluster_wait();
@@ -1233,10 +1326,11 @@ output_kernel_c(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   uint64_t* full = bars;                 // [NST]
   uint64_t* empty = full + NST;          // [NST]
   uint64_t* bar_q = empty + NST;
-  uint64_t* bar_inter = bar_q + 1;
-  uint64_t* bar_s = bar_inter + 1;       // scores ready in TMEM
+  uint64_t* bar_pv = bar_q + 1;          // the P V MMAs are done (the score tile is free)
+  uint64_t* bar_s = bar_pv + 1;          // scores ready in TMEM
   uint64_t* bar_p = bar_s + 1;           // P written over the scores
-  uint64_t* bar_o = bar_p + 1;           // all MMAs done
+  uint64_t* bar_pp = bar_p + 1;          // decayed query rows written over the score tile
+  uint64_t* bar_o = bar_pp + 1;          // all MMAs done
   uint64_t* drain = bar_o + 1;
   uint64_t* bar_x = drain + 1;           // the partner's statistics have arrived
   uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(bar_x + 1);
@@ -1257,10 +1351,10 @@ output_kernel_c(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const bool need_inter = si.c > 0 || p.has_state_in;
   const bool xchg = p.parts > 1 && p.gated;
   const Decay1 dec(p.dec, h);
-  // ring units (16 KB): [S_hi, S_lo of d_k rows 64u..64u+63], K (DK/64 boxes of
-  // 128 keys x 64 d_k), V (keys 0-63, 64-127), then the gate/output tile, one
-  // 128 x 64 box per unit
-  const int n_mma_units = (need_inter ? 2 * (DK / 64) : 0) + DK / 64 + 2;
+  // ring units (16 KB): K (DK/64 boxes of 128 keys x 64 d_k), V (keys 0-63,
+  // 64-127; fp16 copy), [S of d_k rows 64u..64u+63 (fp16)], then the
+  // gate/output tile, one 128 x 64 box per unit
+  const int n_mma_units = DK / 64 + 2 + (need_inter ? DK / 64 : 0);
   auto io_box = [&](int bx) -> uint8_t* {
     return smem + C::kOffStages + ((n_mma_units + bx) % NST) * kStageC;
   };
@@ -1271,9 +1365,10 @@ output_kernel_c(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(&empty[i], 1);
     }
     mbar_init(bar_q, 1);
-    mbar_init(bar_inter, 1);
+    mbar_init(bar_pv, 1);
     mbar_init(bar_s, 1);
     mbar_init(bar_p, kWgThreads);
+    mbar_init(bar_pp, kWgThreads);
     mbar_init(bar_o, 1);
     mbar_init(drain, 1);
     mbar_init(bar_x, kWgThreads);
@@ -1312,18 +1407,6 @@ output_kernel_c(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_arrive_expect_tx(&full[st], bytes);
         return smem + C::kOffStages + st * kStageC;
       };
-      if (need_inter) {
-        for (int u = 0; u < DK / 64 && ok; ++u) {
-          for (int hl = 0; hl < 2 && ok; ++hl) {
-            const int srow = static_cast<int>(((slot * p.H + h) * 2 + hl) * DK) + 64 * u;
-            uint8_t* dst = next((NV / 64) * kBox);
-            if (!dst) { ok = false; break; }
-            for (int bx = 0; bx < NV / 64; ++bx)
-              tma_load_2d(dst + bx * kBox, &tmS, &full[it % NST], NV * part + 64 * bx, srow);
-            ++it;
-          }
-        }
-      }
       for (int ku = 0; ku < DK / 64 && ok; ++ku) {
         uint8_t* dst = next(kTallBox);
         if (!dst) { ok = false; break; }
@@ -1337,6 +1420,16 @@ output_kernel_c(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tma_load_2d(dst + bx * kBox, &tmV, &full[it % NST], h * p.dv + NV * part + 64 * bx,
                       si.cs + 64 * vu);
         ++it;
+      }
+      if (need_inter) {
+        for (int u = 0; u < DK / 64 && ok; ++u) {
+          const int srow = static_cast<int>((slot * p.H + h) * DK) + 64 * u;
+          uint8_t* dst = next((NV / 64) * kBox);
+          if (!dst) { ok = false; break; }
+          for (int bx = 0; bx < NV / 64; ++bx)
+            tma_load_2d(dst + bx * kBox, &tmS, &full[it % NST], NV * part + 64 * bx, srow);
+          ++it;
+        }
       }
       if (p.gated && p.g_tma) {      // the gate rows of this tile, for the epilogue
         tma_prefetch_desc(&tmG);
@@ -1357,10 +1450,11 @@ output_kernel_c(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    // Sc = Q K^T; [P] O = P V; [decayed Q rows, written over the score tile
+    // once P V is done] O += Qd S.
     if (lane == 0 && !*abort_flag) {
-      constexpr uint32_t id_qs = idesc_bf16_f32(128, NV, false, true);
       constexpr uint32_t id_qk = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t id_pv = idesc_bf16_f32(128, NV, false, true);
+      constexpr uint32_t id_pv = idesc_f16_f32(128, NV, false, true);
       const uint32_t q_base = smem_u32(smem);
       const uint32_t st_base = smem_u32(smem + C::kOffStages);
       int it = 0;
@@ -1376,22 +1470,7 @@ output_kernel_c(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         ++it;
       };
       ok = mbar_wait(bar_q, 0, abort_flag, p.err);
-      if (ok && need_inter) {
-        // O = Q S_hi + Q S_lo  (the state entering the chunk, split in two bf16 parts)
-        for (int u = 0; u < DK / 64 && ok; ++u) {
-          for (int hl = 0; hl < 2; ++hl) {
-            const uint32_t sb = stage_wait();
-            if (!sb) { ok = false; break; }
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(tmem + C::kTmemO, sdesc_sw128(q_base + u * kTallBox + kk * 32, 16, 1024),
-                       sdesc_sw128(sb + kk * 2048, kBox, 1024), id_qs, (u | hl | kk) != 0);
-            issued = true;
-            stage_free();
-          }
-        }
-        if (ok) mma_commit(bar_inter);
-      }
+      if (ok) tc_fence_after();
       // scores Q K^T of the chunk's keys
       for (int ku = 0; ku < DK / 64 && ok; ++ku) {
         const uint32_t sb = stage_wait();
@@ -1414,11 +1493,24 @@ output_kernel_c(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const int ks = vu * 4 + kk;                      // keys 16ks .. 16ks+15
-            const uint32_t a_hi = pbuf + 32 * (ks >> 1) + 8 * (ks & 1);
-            const uint64_t bd = sdesc_sw128(sb + kk * 2048, kBox, 1024);
-            mma_bf16_ts(tmem + C::kTmemO, a_hi, bd, id_pv, need_inter || ks > 0);
-            mma_bf16_ts(tmem + C::kTmemO, a_hi + 16, bd, id_pv, true);
+            mma_bf16_ts(tmem + C::kTmemO, pbuf + 32 * (ks >> 1) + 8 * (ks & 1),
+                        sdesc_sw128(sb + kk * 2048, kBox, 1024), id_pv, ks > 0);
           }
+          stage_free();
+        }
+        if (ok) mma_commit(bar_pv);
+      }
+      if (ok && need_inter) {
+        // O += (gamma^(i+1) q_i) S, the decayed query rows (fp16) over the score tile
+        ok = mbar_wait(bar_pp, 0, abort_flag, p.err);
+        if (ok) tc_fence_after();
+        for (int u = 0; u < DK / 64 && ok; ++u) {
+          const uint32_t sb = stage_wait();
+          if (!sb) { ok = false; break; }
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(tmem + C::kTmemO, tmem + C::kTmemS + 32 * u + 8 * kk,
+                        sdesc_sw128(sb + kk * 2048, kBox, 1024), id_pv, true);
           stage_free();
         }
       }
@@ -1439,23 +1531,7 @@ output_kernel_c(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     pow_tab[et] = dec.pow(et);
     epi_sync_c();
     bool ok = !*abort_flag;
-    if (ok && need_inter) {
-      // tcgen05.ld/st are warp-collective: every guard around them is warp-uniform
-      ok = warp_all(mbar_wait(bar_inter, 0, abort_flag, p.err));
-      if (ok) {
-        tc_fence_after();
-        const float sc = dec.pow(row + 1);
-        for (int j = 0; j < NV / 32; ++j) {
-          float x[32];
-          tmem_ld32(o_cols + 32 * j, x);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] *= sc;
-          tmem_st32(o_cols + 32 * j, x);
-        }
-        tmem_wait_st();
-      }
-    }
+    float pmax = 0.f;                                 // largest |P| and |decayed q| formed
     if (ok) ok = warp_all(mbar_wait(bar_s, 0, abort_flag, p.err));
     if (ok) {
       tc_fence_after();
@@ -1471,21 +1547,52 @@ output_kernel_c(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           wv[e] = (jp <= row && jp < si.len) ? pow_tab[row - jp] : 0.f;
         }
         tmem_wait_ld();
-        float pw[32];
+        uint32_t pw[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          uint32_t hi, lo;
           const uint64_t p2 = f2_mul(f2_make(x[e], x[e + 1]), f2_make(wv[e], wv[e + 1]));
-          pack_split(f2_lo(p2), f2_hi(p2), hi, lo);
-          pw[e >> 1] = __uint_as_float(hi);
-          pw[16 + (e >> 1)] = __uint_as_float(lo);
+          pmax = fmaxf(pmax, fmaxf(fabsf(f2_lo(p2)), fabsf(f2_hi(p2))));
+          pw[e >> 1] = pack_f16(f2_lo(p2), f2_hi(p2));
         }
-        tmem_st32(buf + 32 * j, pw);
+        tmem_st16(buf + 32 * j, pw);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p);
     }
+    if (ok && need_inter) {
+      // the decayed query rows gamma^(row+1) q_row (fp16) over the score tile,
+      // once the P V MMAs have read it
+      ok = warp_all(mbar_wait(bar_pv, 0, abort_flag, p.err) && mbar_wait(bar_q, 0, abort_flag, p.err));
+      if (ok) {
+        tc_fence_after();
+        const float sc = dec.pow(row + 1);
+        const uint64_t sc2 = f2_make(sc, sc);
+        const uint32_t abuf = tmem + lane_off + C::kTmemS;
+#pragma unroll 1
+        for (int c0 = 0; c0 < DK; c0 += 32) {
+          const uint8_t* qrow = smem + (c0 >> 6) * kTallBox + row * 128;
+          const int pc0 = (c0 & 63) >> 3;
+          uint32_t pw[16];
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const uint4 u = *reinterpret_cast<const uint4*>(qrow + (((pc0 + c4) ^ (row & 7)) << 4));
+            const uint32_t wq[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+              const uint64_t d2 = f2_mul(f2_make(bf16_lo(wq[q2]), bf16_hi(wq[q2])), sc2);
+              pmax = fmaxf(pmax, fmaxf(fabsf(f2_lo(d2)), fabsf(f2_hi(d2))));
+              pw[4 * c4 + q2] = pack_f16(f2_lo(d2), f2_hi(d2));
+            }
+          }
+          tmem_st16(abuf + (c0 >> 1), pw);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_pp);
+      }
+    }
+    if (pmax > kF16Max) raise_error(p.err, kErrRange);
     if (ok) ok = mbar_wait(bar_o, 0, abort_flag, p.err);
     ok = warp_all(ok);
     if (ok) tc_fence_after();
@@ -1694,32 +1801,34 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor map: `rows` rows of `inner` elements, row pitch `pitch`
-// elements, box = 64 elements x box_rows rows, 128-byte swizzle.
+// 2-D tensor map of 16-bit elements (bf16, or fp16 when `f16`): `rows` rows
+// of `inner` elements, row pitch `pitch` elements, box = 64 elements x
+// box_rows rows, 128-byte swizzle.
 bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch,
-              uint32_t box_rows) {
+              uint32_t box_rows, bool f16 = false) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gdim[2] = {inner, rows};
   cuuint64_t gstride[1] = {pitch * 2};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 template <int NS>
 cudaError_t launch_state(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mw,
-                         const StateParams& sp, cudaStream_t s) {
+                         const CUtensorMap& mv16, const StateParams& sp, cudaStream_t s) {
   const size_t smem = StCfg<NS>::kSmem;
   auto kern = state_kernel<NS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(static_cast<unsigned>(sp.L.nseq) * sp.H * ((sp.dk + 127) / 128) * (sp.dv / NS));
-  kern<<<grid, kThreads, smem, s>>>(mk, mv, mw, sp);
+  kern<<<grid, kThreads, smem, s>>>(mk, mv, mw, mv16, sp);
   return cudaGetLastError();
 }
 
@@ -1856,22 +1965,25 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
     sp.order = L.cu ? ws.order : nullptr;
     sp.state_in = state_in;
     sp.state_out = state_out;
-    sp.ws = static_cast<__nv_bfloat16*>(ws.states);
+    sp.write_v16 = ws.v16 != nullptr ? 1 : 0;
     sp.H = H;
     sp.dk = dk;
     sp.dv = dv;
     sp.dec = dec;
     sp.err = err;
-    CUtensorMap mk_st, mv_st, mw_st;
-    const uint64_t wrows = static_cast<uint64_t>(ws.nslots) * H * 2 * dk;   // hi and lo planes
+    CUtensorMap mk_st, mv_st, mw_st, mv16_st;
+    const uint64_t wrows = static_cast<uint64_t>(ws.nslots) * H * dk;    // fp16 state slots
+    const uint64_t hdv = static_cast<uint64_t>(H) * dv;
+    std::memset(&mv16_st, 0, sizeof(mv16_st));
     if (!make_map(&mk_st, k, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 64) ||
-        !make_map(&mv_st, v, static_cast<uint64_t>(H) * dv, Ttot, static_cast<uint64_t>(H) * dv, 64) ||
-        !make_map(&mw_st, ws.states, dv, wrows, dv, dk < 128 ? dk : 128))
+        !make_map(&mv_st, v, hdv, Ttot, hdv, 64) ||
+        !make_map(&mw_st, ws.states, dv, wrows, dv, dk < 128 ? dk : 128, true) ||
+        (ws.v16 && !make_map(&mv16_st, ws.v16, hdv, Ttot, hdv, 64, true)))
       return cudaErrorInvalidValue;
     switch (NS) {
-      case 64: e = launch_state<64>(mk_st, mv_st, mw_st, sp, s); break;
-      case 128: e = launch_state<128>(mk_st, mv_st, mw_st, sp, s); break;
-      default: e = launch_state<256>(mk_st, mv_st, mw_st, sp, s); break;
+      case 64: e = launch_state<64>(mk_st, mv_st, mw_st, mv16_st, sp, s); break;
+      case 128: e = launch_state<128>(mk_st, mv_st, mw_st, mv16_st, sp, s); break;
+      default: e = launch_state<256>(mk_st, mv_st, mw_st, mv16_st, sp, s); break;
     }
   }
   if (e != cudaSuccess || L.Ttot == 0 || !(phases & 2)) return e;
@@ -1898,13 +2010,14 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
   op.err = err;
   op.g_tma = (gated && g_t == DType::BF16) ? 1 : 0;
   op.y_tma = out_t == DType::BF16 ? 1 : 0;
-  const uint64_t srows = static_cast<uint64_t>(ws.nslots) * H * 2 * dk;   // hi and lo planes
+  if (ws.v16 == nullptr) return cudaErrorInvalidValue;   // written by the state pass
+  const uint64_t srows = static_cast<uint64_t>(ws.nslots) * H * dk;      // fp16 state slots
   const uint64_t hdv = static_cast<uint64_t>(H) * dv;
   CUtensorMap mq, mk, mv, ms, mg, my;
   if (!make_map(&mq, q, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 128) ||
       !make_map(&mk, k, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 128) ||
-      !make_map(&mv, v, hdv, Ttot, hdv, 64) ||
-      !make_map(&ms, ws.states, dv, srows, dv, 64))
+      !make_map(&mv, ws.v16, hdv, Ttot, hdv, 64, true) ||
+      !make_map(&ms, ws.states, dv, srows, dv, 64, true))
     return cudaErrorInvalidValue;
   // gate and output tiles: [Ttot rows][H*dv] bf16 (maps only built when used)
   std::memset(&mg, 0, sizeof(mg));

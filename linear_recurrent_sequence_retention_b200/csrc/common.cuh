@@ -14,6 +14,7 @@ constexpr int kMaxHeads = 64;
 // Bits of the per-device error word (see retention_check_device_error).
 constexpr unsigned kErrTimeout = 1u;     // a bounded wait gave up
 constexpr unsigned kErrDeviceData = 2u;  // cu_seqlens inconsistent
+constexpr unsigned kErrRange = 4u;       // a value exceeded the fp16 range of the tensor-core operands
 
 // Per-head decay constants, computed on the host in double precision from the
 // caller's gamma and passed by value.  gamma^n is evaluated as

@@ -13,15 +13,17 @@ namespace ret {
 enum class DType { F32 = 0, BF16 = 1 };
 
 // Workspace layout of the chunkwise forward:
-//   [meta: chunk_base int32[nseq+1], rounded up to 256 B][states]
+//   [meta: chunk_base int32[nseq+1], rounded up to 256 B][states][v16]
 // states hold the state entering every chunk, one slot per chunk:
-//   [slot][H][dk][dv], float32 on the CUDA-core path; on the tensor-core path
-//   [slot][H][2][dk][dv] bf16, the hi and lo parts of the state (the MMA
-//   operands of the cross-chunk read).
+//   [slot][H][dk][dv], float32 on the CUDA-core path, fp16 on the tensor-core
+//   path (the MMA operand of the cross-chunk read).  v16 (tensor-core path
+//   only, at a 256-byte boundary) is the fp16 copy of v, [Ttot][H][dv], that
+//   the state pass writes for the output pass's P V products.
 struct ChunkWorkspace {
   int32_t* chunk_base;   // device, nseq+1 entries (varlen only; else unused)
   int32_t* order;        // device, nseq entries: sequences longest first (varlen only)
   void* states;          // device
+  void* v16;             // device (tensor-core path), else nullptr
   long long nslots;      // slots available
 };
 

@@ -242,6 +242,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
          ((static_cast<uint32_t>(M) >> 4) << 24);
 }
 
+// Instruction descriptor, kind::f16 with fp16 A and B (format 0) and an f32
+// accumulator; the other fields as in idesc_bf16_f32.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+         ((static_cast<uint32_t>(N) >> 3) << 17) | ((static_cast<uint32_t>(M) >> 4) << 24);
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand:
 // bits [0,14) start address >> 4, [16,30) leading byte offset >> 4,
 // [32,46) stride byte offset >> 4, [46,48) version = 1, [61,64) layout = 2
@@ -412,6 +419,31 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&p);
 }
+
+// ---- fp16 ---------------------------------------------------------------------------
+//
+// fp16 (11 significant bits) is the operand type of the MMAs whose operands
+// the kernels compute themselves: the decayed scores, the decayed query rows
+// that read the carried state, the carried state and zeta * K.  bf16 inputs
+// convert to fp16 exactly inside fp16's range (|x| <= 65504, subnormals below
+// 2^-14 keep fewer bits).
+
+// (lo, hi) -> one f16x2 word, lo in bits 0..15, round to nearest.
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// bf16x2 word -> f16x2 word (each half widened to f32, then rounded to fp16;
+// exact inside fp16's normal range).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  return pack_f16(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// Largest finite fp16 value: a magnitude above it does not fit the fp16
+// operands of the tensor-core path.
+constexpr float kF16Max = 65504.0f;
 
 // ---- hi/lo bf16 pairs ------------------------------------------------------------
 //

@@ -23,6 +23,7 @@ RET_ERR_CUDA = 3
 RET_ERR_TIMEOUT = 4
 RET_ERR_WORKSPACE = 5
 RET_ERR_DEVICE_DATA = 6
+RET_ERR_RANGE = 7
 
 RET_F32 = 0
 RET_BF16 = 1

@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol():
 def test_abi_version_and_status_strings():
     ops, L = _lib()
     assert L.retention_abi_version() == 1
-    for code in range(7):
+    for code in range(8):
         s = ops.status_string(code)
         assert s and "unknown" not in s
     assert "unknown" in ops.status_string(99)

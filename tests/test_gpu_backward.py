@@ -6,8 +6,9 @@ from inputs that are exact (float32, or bfloat16 widened exactly), so both
 input dtypes are held to the float32 tolerance: relative L2 <= 1e-5 over each
 gradient, whole and per head.  bf16 inputs with heads of 64/128/256 (and, with
 a final-state gradient, every gamma 0 or >= 1e-6) run on the tensor-core
-kernels instead and are held to the bf16-input tolerance (plus rel-L2 <= 1e-4
-as a precision check).  Cases
+kernels instead and are held to the bf16-input tolerance (plus rel-L2 <= 1e-3
+as a precision check: their computed MMA operands are fp16, unit roundoff
+2^-11, which gives ~3e-4; operands rounded to bf16 alone would give ~2e-3).  Cases
 span several chunks with ragged tails, chunk lengths of one token and longer
 than the sequence, the largest supported heads, gamma = 0 and gamma = 1, an
 initial state and an upstream state gradient, and packed sequences including
@@ -59,7 +60,7 @@ def _check(got, ref, H, what, tc=False):
         axis = 2 if n != "d_state_in" else 1
         if tc:
             assert_close(W.to_f64(x), y, "bf16", axis, f"{what} {n}")
-            assert rel_l2(W.to_f64(x), y) <= 1e-4, (what, n, rel_l2(W.to_f64(x), y))
+            assert rel_l2(W.to_f64(x), y) <= 1e-3, (what, n, rel_l2(W.to_f64(x), y))
         else:
             assert_close(W.to_f64(x), y, "f32", axis, f"{what} {n}")
 
@@ -96,7 +97,7 @@ def test_backward_tensor_core_path(B, T, H, dk, dv, chunk, with_state, use_dS):
     """bf16 inputs with heads of 64/128/256 run on the tensor-core forward kernels
     (three retentions, two on reversed sequences; a final-state gradient enters
     them as the initial state dS_T / gamma); held to the bf16-input tolerance
-    and, as a precision check, rel-L2 <= 1e-4."""
+    and, as a precision check, rel-L2 <= 1e-3."""
     q, k, v, do, S0, dS = _inputs(B, T, H, dk, dv, "bf16", seed=T + 3 * dk, with_state=True)
     S0 = S0 if with_state else None
     dS = dS if use_dS else None
