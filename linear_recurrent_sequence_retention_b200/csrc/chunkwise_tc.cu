@@ -120,25 +120,13 @@ __device__ __forceinline__ bool wga_all(bool v) {
   return r != 0;
 }
 
-// AND of `v` over the 128 threads of warps 6..9 (named barrier 3); same
-// contract as wga_all.
-__device__ __forceinline__ bool wgb_all(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 3, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(v ? 1u : 0u)
-      : "memory");
-  return r != 0;
-}
-
 // ===========================================================================
 // State kernel
 // ===========================================================================
 constexpr int kStTok = 64;           // tokens per pipeline stage
+constexpr int kStThreads = 480;      // 15 warps: producer, MMA, warpgroup A, two converter
+                                     // warpgroups, the store warp of the fp16 copy of v
+constexpr int kCvtThreads = 256;     // the converter warps 6..13
 
 struct StateParams {
   SeqLayout L;
@@ -157,8 +145,9 @@ struct StCfg {
   static constexpr uint32_t kKBytes = 2 * kBox;              // 64 tokens x 128 rows of d_k
   static constexpr uint32_t kVBytes = (NS / 64) * kBox;      // 64 tokens x NS
   static constexpr uint32_t kStage = kKBytes + kVBytes;      // zeta*K | V, both fp16 in place
-  // staging for the TMA store of the state entering a chunk: one 128 x 64 fp16 box
-  static constexpr uint32_t kStaging = kTallBox;
+  // staging for the TMA stores of the state entering a chunk: two 128 x 64
+  // fp16 boxes, filled in turn
+  static constexpr uint32_t kStaging = 2 * kTallBox;
   static constexpr int kStagesFit = static_cast<int>((232448 - kStaging - 1024) / kStage);
   static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
   static constexpr uint32_t kOffStaging = kStages * kStage;
@@ -166,7 +155,7 @@ struct StCfg {
 };
 
 template <int NS>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kStThreads, 1)
 state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
              const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmV16,
              const StateParams p) {
@@ -210,7 +199,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       mbar_init(&full[i], 1);
       // released by the MMA, and by the copy store once it has read the stage
       mbar_init(&empty[i], v16_out ? 2 : 1);
-      mbar_init(&kready[i], kWgThreads);
+      mbar_init(&kready[i], kCvtThreads);
     }
     mbar_init(acc_free, kWgThreads);
     mbar_init(acc_full, 1);
@@ -230,7 +219,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     // d_k = 64: the second 64-row half of every zeta*K tile stays zero, so the
     // 128-row MMA adds nothing to TMEM rows 64..127
     for (int st = 0; st < NSTG; ++st)
-      for (int o = threadIdx.x * 16; o < static_cast<int>(kBox); o += kThreads * 16)
+      for (int o = threadIdx.x * 16; o < static_cast<int>(kBox); o += kStThreads * 16)
         *reinterpret_cast<uint4*>(smem + st * kStage + kBox + o) = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
@@ -324,20 +313,23 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
                              : static_cast<long long>(p.chunk_base[s]) + c;
     };
     // The state in accumulator column `col` -> workspace slot `slot` as fp16,
-    // one 128 x 64 box per TMA store.  Barrier 2 is reached by all 128 threads
-    // the same number of times.
+    // one 128 x 64 box per TMA store, through the two staging boxes in turn.
+    // Barrier 2 is reached by all 128 threads the same number of times.
+    int nbox = 0;
     auto stage_state = [&](uint32_t col, long long slot) {
       const bool slot_ok = slot >= 0 && slot < L.nslots;
       // workspace rows of this CTA's 128 d_k rows
       const int wrow = static_cast<int>(((slot_ok ? slot : 0) * p.H + h) * p.dk) + 128 * m;
 #pragma unroll 1
-      for (int j = 0; j < NS / 32; j += 2) {
+      for (int j = 0; j < NS / 32; j += 2, ++nbox) {
+        uint8_t* box = staging + (nbox & 1) * kTallBox;
         float r[2][32];
         tmem_ld32(trow + col + 32 * j, r[0]);
         tmem_ld32(trow + col + 32 * (j + 1), r[1]);
         tmem_wait_ld();
-        // the staging box is free once the previous store stopped reading it
-        if (leader) tma_store_wait_read();
+        // this staging box is free once the store issued from it two boxes ago
+        // has read it (at most the other box's store is still pending)
+        if (leader) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
         asm volatile("bar.sync 2, 128;" ::: "memory");
         // row `row` of a 128 x 64 swizzled box: 16-byte piece cc of the row
         // goes to piece cc ^ (row & 7)
@@ -349,14 +341,14 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
           for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
           const uint4 u = make_uint4(pack_f16(x[0], x[1]), pack_f16(x[2], x[3]),
                                      pack_f16(x[4], x[5]), pack_f16(x[6], x[7]));
-          *reinterpret_cast<uint4*>(staging + row * 128 + ((cc ^ (row & 7)) << 4)) = u;
+          *reinterpret_cast<uint4*>(box + row * 128 + ((cc ^ (row & 7)) << 4)) = u;
         }
         range_ok = range_ok && !(amax > kF16Max);    // NaN passes here; it is not a range event
         fence_proxy_async_smem();
         asm volatile("bar.sync 2, 128;" ::: "memory");
         if (leader && slot_ok) {
           // a box of min(d_k, 128) rows: the first rows of the staged box
-          tma_store_2d(&tmW, staging, NS * part + 32 * j, wrow);
+          tma_store_2d(&tmW, box, NS * part + 32 * j, wrow);
           tma_store_commit();
         }
       }
@@ -434,105 +426,101 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         *reinterpret_cast<float4*>(p.state_out + st_off + j) = x;
       }
     }
-  } else {
-    // ---------------- warpgroup B: the fp16 MMA operands, ahead of the MMA ----------------
-    // K rows -> zeta*K (fp16, in place), V rows -> fp16 (in place); the first
-    // d_k block's CTAs also store the converted V rows as the fp16 copy of v
-    // that the output pass reads.
-    const int t = threadIdx.x - 192;              // 0..127
-    const bool leader = t == 0;
-    if (leader && v16_out) tma_prefetch_desc(&tmV16);
+  } else if (warp < 14) {
+    // ---------------- converter warps 6..13: the fp16 MMA operands, ahead of the MMA ----------------
+    // K rows -> zeta*K (fp16, in place; thread u owns half a row), V rows ->
+    // fp16 (in place; thread u owns row u).
+    const int u = threadIdx.x - 192;              // 0..255
+    constexpr int kVRows = (NS / 64) * 64;        // V rows of a stage: (NS/64) boxes x 64 tokens
+    const int krow = u >> 1, khalf = u & 1;       // this thread's K row (box krow/64) and half
+    const bool k_mine = krow < 64 * kboxes;
     int it = 0;
     bool ok = !*abort_flag, range_ok = true;
-    int pending_st = -1;                          // stage whose copy store may still be reading it
     for (int c = 0; c < nch && ok; ++c) {
       const int tok0 = a + c * L.chunk;
       const int Lc = min(L.chunk, b - tok0);
       for (int sb = 0; sb * kStTok < Lc; ++sb, ++it) {
         const int st = it % NSTG;
-        // uniform over the warpgroup: the named barrier below stays matched
-        if (!wgb_all(mbar_wait(&full[st], (it / NSTG) & 1, abort_flag, p.err))) { ok = false; break; }
+        if (!mbar_wait(&full[st], (it / NSTG) & 1, abort_flag, p.err)) { ok = false; break; }
         uint8_t* stage = smem + st * kStage;
-        {
-          // zeta*K: thread t owns box t/64, token row t%64 (one 128-byte row)
-          const int jtok = sb * kStTok + (t & 63);
+        if (k_mine) {
+          // zeta*K, pieces 4*khalf .. 4*khalf+3 of row krow%64 of box krow/64
+          const int jtok = sb * kStTok + (krow & 63);
           const float z = jtok < Lc ? dec.pow(Lc - 1 - jtok) : 0.f;
-          uint4* rp = reinterpret_cast<uint4*>(stage + (t >> 6) * kBox + (t & 63) * 128);
-          // every piece of the row gets the same factor, so visit the row's eight
-          // 16-byte pieces in the order e ^ (row & 7): lanes of 8 consecutive rows then
-          // touch 8 different bank groups instead of the same one
-          const int sw = t & 7;
-          if (t < 64 * kboxes) {
-            uint4 u[8];
+          uint4* rp = reinterpret_cast<uint4*>(stage + (krow >> 6) * kBox + (krow & 63) * 128);
+          const int sw = krow & 7;
+          uint4 w4[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) u[e] = rp[e ^ sw];
-            const uint64_t z2 = f2_make(z, z);
+          for (int e = 0; e < 4; ++e) w4[e] = rp[(4 * khalf + e) ^ sw];
+          const uint64_t z2 = f2_make(z, z);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint32_t w[4] = {u[e].x, u[e].y, u[e].z, u[e].w};
-              uint32_t wh[4];
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t w[4] = {w4[e].x, w4[e].y, w4[e].z, w4[e].w};
+            uint32_t wh[4];
 #pragma unroll
-              for (int q2 = 0; q2 < 4; ++q2) {
-                const uint64_t p2 = f2_mul(f2_make(bf16_lo(w[q2]), bf16_hi(w[q2])), z2);
-                wh[q2] = pack_f16(f2_lo(p2), f2_hi(p2));
-              }
-              rp[e ^ sw] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            for (int q2 = 0; q2 < 4; ++q2) {
+              const uint64_t p2 = f2_mul(f2_make(bf16_lo(w[q2]), bf16_hi(w[q2])), z2);
+              wh[q2] = pack_f16(f2_lo(p2), f2_hi(p2));
             }
+            rp[(4 * khalf + e) ^ sw] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
           }
         }
-        {
-          // V: (NS/64) boxes x 64 rows of 128 bytes, converted bf16 -> fp16
-          uint8_t* vbase = stage + kKBytes;
-          constexpr int kVRows = (NS / 64) * 64;
-          for (int rr = t; rr < kVRows; rr += kWgThreads) {
-            uint4* rp = reinterpret_cast<uint4*>(vbase + rr * 128);
-            const int sw = rr & 7;
-            uint4 u[8];
+        if (u < kVRows) {
+          // V row u: box u/64, token row u%64, converted bf16 -> fp16
+          uint4* rp = reinterpret_cast<uint4*>(stage + kKBytes + u * 128);
+          // every piece converts the same way, so visit them in the order
+          // e ^ (row & 7): 8 consecutive rows then touch 8 different bank groups
+          const int sw = u & 7;
+          uint4 w4[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) u[e] = rp[e ^ sw];
-            uint32_t bad = 0;
+          for (int e = 0; e < 8; ++e) w4[e] = rp[e ^ sw];
+          uint32_t amax = 0;                              // largest |bf16| bit pattern, per half
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint4 f = make_uint4(bf16x2_to_f16x2(u[e].x), bf16x2_to_f16x2(u[e].y),
-                                         bf16x2_to_f16x2(u[e].z), bf16x2_to_f16x2(u[e].w));
-              // an fp16 infinity from a finite bf16 value: |v| > 65504
-              const uint32_t wv[4] = {f.x, f.y, f.z, f.w};
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t w[4] = {w4[e].x, w4[e].y, w4[e].z, w4[e].w};
 #pragma unroll
-              for (int q2 = 0; q2 < 4; ++q2) {
-                const uint32_t lo = wv[q2] & 0x7fffu, hi = (wv[q2] >> 16) & 0x7fffu;
-                bad |= (lo == 0x7c00u) | (hi == 0x7c00u);
-              }
-              rp[e ^ sw] = f;
-            }
-            // rows past the sequence's end hold other tokens (or the zero fill)
-            // and may overflow without concerning this sequence
-            const int jtok = sb * kStTok + (rr & 63);
-            if (bad && jtok < Lc) range_ok = false;
+            for (int q2 = 0; q2 < 4; ++q2) amax = __vmaxu2(amax, w[q2] & 0x7fff7fffu);
+            rp[e ^ sw] = make_uint4(bf16x2_to_f16x2(w[0]), bf16x2_to_f16x2(w[1]),
+                                    bf16x2_to_f16x2(w[2]), bf16x2_to_f16x2(w[3]));
           }
+          // |v| >= 2^16 (bf16 0x4780) has no fp16 value; rows past the
+          // sequence's end hold other tokens (or the zero fill) and are not
+          // this sequence's to report
+          const uint32_t big = max(amax & 0xffffu, amax >> 16);
+          const int jtok = sb * kStTok + (u & 63);
+          if (big >= 0x4780u && jtok < Lc) range_ok = false;
         }
         fence_proxy_async_smem();
         mbar_arrive(&kready[st]);
-        if (v16_out) {
-          // all 128 threads' V rows are written: store them as the fp16 copy
-          asm volatile("bar.sync 3, 128;" ::: "memory");
-          if (leader) {
-            const int y = tok0 + sb * kStTok;
-            for (int bx = 0; bx < NS / 64; ++bx)
-              tma_store_2d(&tmV16, stage + kKBytes + bx * kBox, h * p.dv + NS * part + 64 * bx, y);
-            tma_store_commit();
-            // the previous stage's copy has been read out of shared memory
-            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-            if (pending_st >= 0) mbar_arrive(&empty[pending_st]);
-            pending_st = st;
-          }
-        }
       }
     }
-    if (v16_out && leader) {
-      tma_store_wait_all();
-      if (pending_st >= 0) mbar_arrive(&empty[pending_st]);
-    }
     if (!range_ok) raise_error(p.err, kErrRange);
+  } else if (warp == 14) {
+    // ---------------- store warp: the fp16 copy of v ----------------
+    // Each stage's converted V rows go out by TMA store as soon as the
+    // converters are done; the stage returns to the producer once the store
+    // has read it (its second arrival on `empty`, beside the MMA's).
+    if (v16_out && lane == 0 && !*abort_flag) {
+      tma_prefetch_desc(&tmV16);
+      int it = 0;
+      bool ok = true;
+      for (int c = 0; c < nch && ok; ++c) {
+        const int tok0 = a + c * L.chunk;
+        const int Lc = min(L.chunk, b - tok0);
+        for (int sb = 0; sb * kStTok < Lc; ++sb, ++it) {
+          const int st = it % NSTG;
+          if (!mbar_wait(&kready[st], (it / NSTG) & 1, abort_flag, p.err)) { ok = false; break; }
+          const int y = tok0 + sb * kStTok;
+          uint8_t* stage = smem + st * kStage;
+          for (int bx = 0; bx < NS / 64; ++bx)
+            tma_store_2d(&tmV16, stage + kKBytes + bx * kBox, h * p.dv + NS * part + 64 * bx, y);
+          tma_store_commit();
+          tma_store_wait_read();
+          mbar_arrive(&empty[st]);
+        }
+      }
+      tma_store_wait_all();
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -1828,7 +1816,7 @@ cudaError_t launch_state(const CUtensorMap& mk, const CUtensorMap& mv, const CUt
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(static_cast<unsigned>(sp.L.nseq) * sp.H * ((sp.dk + 127) / 128) * (sp.dv / NS));
-  kern<<<grid, kThreads, smem, s>>>(mk, mv, mw, mv16, sp);
+  kern<<<grid, kStThreads, smem, s>>>(mk, mv, mw, mv16, sp);
   return cudaGetLastError();
 }
 
