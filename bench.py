@@ -31,7 +31,6 @@ import hashlib
 import json
 import math
 import os
-import re
 import subprocess
 import sys
 import threading
@@ -51,7 +50,7 @@ HEADLINE = "msr_6p7b_b2_h16_t8192_dk256_dv512_c512"
 DECODE = "decode_6p7b_n128_h16_dk256_dv512"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TC_SOURCE = os.path.join(ROOT, "linear_recurrent_sequence_retention_b200", "csrc", "chunkwise_tc.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "chunkwise_output_kernel_6p7b_t8192_traffic.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "chunkwise_output_kernel_6p7b_t8192_traffic.json")
 
 
 def log(*a):
@@ -247,19 +246,20 @@ def cpu_baseline(wl, budget_s=15.0):
 # ---------------------------------------------------------------------------
 
 def traffic_from_profile():
-    """DRAM bytes per launch of the output kernel from the committed ncu summary,
-    only if it was taken on the current kernel source."""
+    """DRAM bytes per launch of the output kernel at the workload's full size,
+    from the committed ncu figures (a small JSON file), only if they were taken
+    on the current kernel source."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
-    text = open(TRAFFIC_FILE).read()
-    m1 = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
-    m2 = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
-    if not (m1 and m2):
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+        sha = hashlib.sha256(open(TC_SOURCE, "rb").read()).hexdigest()
+        if d.get("source_sha256") != sha:
+            return None
+        return float(d["dram_bytes_per_launch_full_size"])
+    except (OSError, ValueError, KeyError, TypeError):
         return None
-    sha = hashlib.sha256(open(TC_SOURCE, "rb").read()).hexdigest()
-    if sha != m1.group(1):
-        return None
-    return float(m2.group(1))
 
 
 def config_of(wl, world):
@@ -365,29 +365,32 @@ def run_headline(args, world, rank, pk, pk_kind):
     tokens = sum_over_ranks(Bx * Tx, world)
     value = tokens / (ms_step / 1e3)
 
-    # roofline of the dominant (output) kernel, algorithmic counts at the
-    # workload's own chunk length (the kernels may evaluate short chunks as
-    # longer ones, which executes more intra-chunk work, never less)
+    # roofline of the dominant (output) kernel.  The chunkwise path is a dense
+    # contraction judged on the tensor pipe: algorithmic flops at the
+    # workload's own chunk length over the kernel's event time against the
+    # bf16 peak; its HBM fraction is reported beside it.  The kernels may
+    # evaluate short chunks as longer ones (same result, more intra-chunk
+    # work), so the flops at the executed chunk are given too.
     f_out, f_state, b_in, b_out = alg_counts(wl, wl.chunk)
+    c_exec = ops.chunkwise_executed_chunk(torch.bfloat16, wl.chunk, wl.dk, wl.dv)
+    f_out_x, f_state_x, _, _ = alg_counts(wl, c_exec)
     units = Bx * Tx * wl.H                          # token-heads per launch
     flops_launch = f_out * units
     bytes_launch = (b_in + b_out) * units
     t_out = ms_out / 1e3
     peak_bw = pk["hbm_gbs"]
     peak_tf = pk["bf16_tflops"]
-    t_mem, t_tc = bytes_launch / (peak_bw * 1e9), flops_launch / (peak_tf * 1e12)
     traffic = traffic_from_profile()
-    if t_mem >= t_tc:
-        ach = bytes_launch / t_out / 1e9
-        roof = {"bound": "hbm", "achieved": ach, "peak": peak_bw, "unit": "GB/s",
-                "frac": ach / peak_bw, "traffic": traffic}
-    else:
-        ach = flops_launch / t_out / 1e12
-        roof = {"bound": "tensor", "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s",
-                "frac": ach / peak_tf, "traffic": traffic}
-    roof.update({"kernel": "output_kernel (tcgen05)", "peak_source": f"{pk_kind} (burst)",
-                 "algorithmic_flops_per_launch": flops_launch,
-                 "algorithmic_bytes_per_launch": bytes_launch, "launch_ms": ms_out})
+    ach = flops_launch / t_out / 1e12
+    roof = {"bound": "tensor", "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s",
+            "frac": ach / peak_tf, "traffic": traffic,
+            "kernel": "output_kernel (tcgen05)", "peak_source": f"{pk_kind} bf16 (burst)",
+            "algorithmic_flops_per_launch": flops_launch, "launch_ms": ms_out,
+            "executed_chunk": c_exec,
+            "flops_per_launch_at_executed_chunk": f_out_x * units,
+            "hbm": {"achieved_gbs": bytes_launch / t_out / 1e9, "peak_gbs": peak_bw,
+                    "frac": bytes_launch / t_out / 1e9 / peak_bw,
+                    "algorithmic_bytes_per_launch": bytes_launch}}
     step_flops = (f_out + f_state) * units
     tensor = {"achieved_tflops": step_flops / (ms_step / 1e3) / 1e12,
               "peak_tflops": peak_tf, "frac": step_flops / (ms_step / 1e3) / 1e12 / peak_tf,
@@ -395,6 +398,8 @@ def run_headline(args, world, rank, pk, pk_kind):
               "spec_peak_tflops": 2250.0,
               "frac_of_spec": step_flops / (ms_step / 1e3) / 1e12 / 2250.0,
               "algorithmic_flops_per_step": step_flops,
+              "executed_chunk": c_exec,
+              "flops_per_step_at_executed_chunk": (f_out_x + f_state_x) * units,
               "counting": f"per token-head (C+1)(dk+dv) + 4 dk dv, C={wl.chunk}"}
     step_bytes = (b_in + b_out) * units + (nst * wl.H * wl.dk * wl.dv * 4 if wl.state_out else 0)
     hbm = {"achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9, "peak_gbs": peak_bw,
@@ -871,7 +876,6 @@ def main():
             "tensor": head["tensor"],
             "hbm": head["hbm"],
             "kernels": head["kernels"],
-            "decode": dec,
             "backward": bwd,
             "rope": rope,
             "rla": rla,
@@ -882,9 +886,11 @@ def main():
                              + (bwd["gpu_launches"] if bwd else 0)
                              + (rope["gpu_launches"] if rope else 0)
                              + (rla["gpu_launches"] if rla else 0)),
-            "arithmetic": "bf16 tensor-core MMAs (tcgen05) with f32 accumulation; the "
-                          "carried state, decayed scores and zeta*K enter the MMAs as "
-                          "hi+lo bf16 pairs",
+            "arithmetic": "tensor-core MMAs (tcgen05) with f32 accumulation: q, k as bf16; "
+                          "v, the decayed scores, the decayed query rows, zeta*K and the "
+                          "carried state as fp16",
+            # last, so that a reader keeping only the line's tail still has it
+            "decode": dec,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -69,7 +69,7 @@
 extern "C" {
 #endif
 
-#define RETENTION_ABI_VERSION 1
+#define RETENTION_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define RET_API __attribute__((visibility("default")))
@@ -133,13 +133,24 @@ RET_API ret_status retention_parallel_fwd(const void* q, const void* k, const vo
 /*
  * Bytes of device workspace retention_chunkwise_fwd needs for these sizes
  * (0 if the arguments are invalid).  The workspace holds the state entering
- * every chunk; its contents need no initialisation and are scratch after the
- * call.  `nseq` = 0 for the padded layout, else the number of packed
- * sequences (then B must be 1 and T is the total token count).
+ * every chunk (float32 for float32 inputs; fp16 for bf16 inputs, which also
+ * keep an fp16 copy of v there, T*H*dv values); its contents need no
+ * initialisation and are scratch after the call.  `nseq` = 0 for the padded
+ * layout, else the number of packed sequences (then B must be 1 and T is the
+ * total token count).
  */
 RET_API size_t retention_chunkwise_workspace_size(ret_dtype in_dtype, int chunk,
                                           int B, int T, int H, int dk, int dv,
                                           int nseq);
+
+/*
+ * The chunk length the chunkwise kernels evaluate for a requested `chunk`
+ * (every chunk length gives the same result, see retention_chunkwise_fwd):
+ * `chunk` itself for float32 inputs; for bf16 inputs at least 128 tokens, and
+ * at least 256 when dv >= 256.  Returns 0 for unsupported arguments.  No
+ * counterpart on the pages: it lets a caller count the work the kernels do.
+ */
+RET_API int retention_chunkwise_executed_chunk(ret_dtype in_dtype, int chunk, int dk, int dv);
 
 /*
  * Chunkwise recurrent form (abeam.tech summary, 「長文の学習にはチャンク再帰を
@@ -173,6 +184,13 @@ RET_API size_t retention_chunkwise_workspace_size(ret_dtype in_dtype, int chunk,
  *          when dv >= 256) are evaluated as chunks of that length, which
  *          yields the same result.
  *   out dtype RET_F32 or RET_BF16; H <= 64; T*H*max(dk,dv) < 2^31.
+ * Precision of the bf16 path: q and k enter the MMAs as they are, v as its
+ *   fp16 value (exact inside fp16's range); the decayed scores, the decayed
+ *   query rows gamma^(i+1) q_i, zeta*K and the carried state are rounded to
+ *   fp16 (11 significant bits) before their MMAs; every product accumulates
+ *   in float32 and the state is carried in float32 between chunks.  A value
+ *   outside fp16's range (|v| >= 2^16, a decayed score or state entry beyond
+ *   65504) is reported as RET_ERR_RANGE by retention_check_device_error().
  */
 RET_API ret_status retention_chunkwise_fwd(const void* q, const void* k, const void* v,
                                    ret_dtype in_dtype, const double* gamma,
@@ -414,7 +432,8 @@ RET_API ret_status msr_norm_gate(const void* o, ret_dtype o_dtype, const ret_nor
  * the kernels set instead of trapping: RET_ERR_TIMEOUT when a bounded
  * wait inside a kernel gave up (the kernel then skipped its remaining work
  * and released what it held), RET_ERR_DEVICE_DATA when cu_seqlens was
- * inconsistent.  Returns RET_OK when no such event happened since the last
+ * inconsistent, RET_ERR_RANGE when a tensor-core operand left fp16's range
+ * (the outputs of that call are then not reliable).  Returns RET_OK when no such event happened since the last
  * call, RET_ERR_CUDA if the synchronisation itself failed.
  */
 RET_API ret_status retention_check_device_error(ret_stream_t stream);

@@ -170,6 +170,12 @@ size_t retention_chunkwise_workspace_size(ret_dtype in_dtype, int chunk, int B, 
   return p.bytes;
 }
 
+int retention_chunkwise_executed_chunk(ret_dtype in_dtype, int chunk, int dk, int dv) {
+  ChunkPlan p;
+  if (plan_chunkwise(in_dtype, chunk, 1, chunk, 1, dk, dv, 0, nullptr, &p) != RET_OK) return 0;
+  return p.L.chunk;
+}
+
 }  // extern "C"
 
 namespace {

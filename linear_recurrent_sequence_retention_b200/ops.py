@@ -36,6 +36,7 @@ EXPORTED = (
     "retention_status_string",
     "retention_parallel_fwd",
     "retention_chunkwise_workspace_size",
+    "retention_chunkwise_executed_chunk",
     "retention_chunkwise_fwd",
     "retention_chunkwise_states",
     "retention_chunkwise_outputs",
@@ -87,6 +88,8 @@ def lib():
     L.retention_parallel_fwd.argtypes = [vp, vp, vp, ci, cd, vp, ci, ci, ci, ci, ci, ci, vp]
     L.retention_chunkwise_workspace_size.restype = ctypes.c_size_t
     L.retention_chunkwise_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci]
+    L.retention_chunkwise_executed_chunk.restype = ci
+    L.retention_chunkwise_executed_chunk.argtypes = [ci, ci, ci, ci]
     L.retention_chunkwise_fwd.restype = ci
     L.retention_chunkwise_fwd.argtypes = [vp, vp, vp, ci, cd, ci, vp, ci, vp, vp, vp, ci,
                                           ctypes.POINTER(NormGate), vp, ctypes.c_size_t,
@@ -195,6 +198,13 @@ def parallel_fwd(q, k, v, gamma, out_dtype=None, stream=None):
 def chunkwise_workspace_size(dtype, chunk, B, T, H, dk, dv, nseq=0):
     code = RET_F32 if dtype == torch.float32 else RET_BF16
     return int(lib().retention_chunkwise_workspace_size(code, chunk, B, T, H, dk, dv, nseq))
+
+
+def chunkwise_executed_chunk(dtype, chunk, dk, dv):
+    """The chunk length the chunkwise kernels evaluate for ``chunk`` (0 if
+    unsupported); every chunk length gives the same result."""
+    code = RET_F32 if dtype == torch.float32 else RET_BF16
+    return int(lib().retention_chunkwise_executed_chunk(code, chunk, dk, dv))
 
 
 def alloc_workspace(nbytes, device):

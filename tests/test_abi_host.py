@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     ops, L = _lib()
-    assert L.retention_abi_version() == 1
+    assert L.retention_abi_version() == 2
     for code in range(8):
         s = ops.status_string(code)
         assert s and "unknown" not in s
@@ -196,3 +196,16 @@ def test_rla_workspace_size_and_bad_arguments():
     assert call(q=None) == ops.RET_ERR_INVALID_ARG
     assert call(ws_bytes=100) == ops.RET_ERR_WORKSPACE
     assert call(ws_ptr=None) == ops.RET_ERR_WORKSPACE
+
+
+def test_chunkwise_executed_chunk():
+    """The chunk the kernels evaluate: the caller's for float32 inputs; for bf16
+    at least 128 tokens, and at least 256 when d_v >= 256; 0 if unsupported."""
+    ops, L = _lib()
+    assert L.retention_chunkwise_executed_chunk(ops.RET_F32, 16, 16, 16) == 16
+    assert L.retention_chunkwise_executed_chunk(ops.RET_F32, 1, 256, 256) == 1
+    assert L.retention_chunkwise_executed_chunk(ops.RET_BF16, 64, 128, 128) == 128
+    assert L.retention_chunkwise_executed_chunk(ops.RET_BF16, 128, 128, 256) == 256
+    assert L.retention_chunkwise_executed_chunk(ops.RET_BF16, 512, 256, 512) == 512
+    assert L.retention_chunkwise_executed_chunk(ops.RET_BF16, 96, 128, 128) == 0     # unsupported chunk
+    assert L.retention_chunkwise_executed_chunk(ops.RET_F32, 0, 16, 16) == 0        # invalid chunk
