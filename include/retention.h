@@ -417,6 +417,33 @@ RET_API ret_status retention_rla_fwd(const void* q, const void* k, const void* v
                                      ret_stream_t stream);
 
 /*
+ * Chunkwise forward with the rotary position encoding of q and k fused in:
+ * the result of retention_rope(q, k, base) followed by retention_chunkwise_fwd
+ * on the rotated q and k (abeam.tech summary, 「Retentionは「内容に応じた参照」と
+ * 「距離による忘却」を掛け合わせる」: Q and K are rotated by position after the
+ * projections; the standard rotary form, see retention_rope), without a
+ * separate pass over k: the state pass rotates k as it loads it (and keeps the
+ * rotated rows for the output pass); q is rotated by one streaming pass.  The
+ * rotated values are those retention_rope stores, bit for bit.
+ * Arguments as retention_chunkwise_fwd, plus rope_base (> 1, finite); bf16
+ * inputs only (RET_ERR_UNSUPPORTED otherwise), dk even.  q and k are not
+ * modified.  workspace: at least retention_chunkwise_fwd_rope_workspace_size()
+ * bytes, 256-byte aligned (it holds the chunkwise workspace, then the rotated
+ * q and k).
+ */
+RET_API size_t retention_chunkwise_fwd_rope_workspace_size(int chunk, int B, int T, int H,
+                                                            int dk, int dv, int nseq);
+RET_API ret_status retention_chunkwise_fwd_rope(const void* q, const void* k, const void* v,
+                                                ret_dtype in_dtype, const double* gamma,
+                                                int chunk, const int32_t* cu_seqlens, int nseq,
+                                                const float* state_in, float* state_out,
+                                                void* out, ret_dtype out_dtype,
+                                                const ret_norm_gate* ng, double rope_base,
+                                                void* workspace, size_t workspace_bytes,
+                                                int B, int T, int H, int dk, int dv,
+                                                ret_stream_t stream);
+
+/*
  * Standalone per-head GroupNorm + Swish gate (the epilogue that
  * retention_chunkwise_fwd fuses when given `ng`).
  *   o: [ntok, H, dv] o_dtype     y: [ntok, H, dv] y_dtype (may not alias o)

@@ -281,6 +281,62 @@ ret_status retention_chunkwise_fwd(const void* q, const void* k, const void* v,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t retention_chunkwise_fwd_rope_workspace_size(int chunk, int B, int T, int H, int dk,
+                                                    int dv, int nseq) {
+  ChunkPlan p;
+  if (plan_chunkwise(RET_BF16, chunk, B, T, H, dk, dv, nseq, nullptr, &p) != RET_OK) return 0;
+  const size_t rows = static_cast<size_t>(p.L.Ttot) * H * dk * 2;
+  return round256(p.bytes) + 2 * round256(rows);
+}
+
+ret_status retention_chunkwise_fwd_rope(const void* q, const void* k, const void* v,
+                                        ret_dtype in_dtype, const double* gamma, int chunk,
+                                        const int32_t* cu_seqlens, int nseq,
+                                        const float* state_in, float* state_out, void* out,
+                                        ret_dtype out_dtype, const ret_norm_gate* ng,
+                                        double rope_base, void* workspace,
+                                        size_t workspace_bytes, int B, int T, int H, int dk,
+                                        int dv, ret_stream_t stream) {
+  if (in_dtype != RET_BF16) return RET_ERR_UNSUPPORTED;
+  if (!std::isfinite(rope_base) || rope_base <= 1.0 || (dk & 1)) return RET_ERR_INVALID_ARG;
+  const int ph = kPhaseStates | kPhaseOutputs;
+  const size_t need = retention_chunkwise_fwd_rope_workspace_size(chunk, B, T, H, dk, dv,
+                                                                  cu_seqlens ? nseq : 0);
+  ChunkCall c;
+  // the chunkwise part of the workspace comes first; the rotated q and k follow it
+  ret_status st = prepare_chunk_call(ph, q, k, v, in_dtype, gamma, chunk, cu_seqlens, nseq,
+                                     state_in, state_out, out, out_dtype, ng, workspace,
+                                     workspace_bytes, B, T, H, dk, dv, &c);
+  if (st != RET_OK) return st;
+  if (workspace_bytes < need) return RET_ERR_WORKSPACE;
+  char* rot = static_cast<char*>(workspace) + round256(c.p.bytes);
+  void* q_rot = rot;
+  void* k_rot = rot + round256(static_cast<size_t>(c.p.L.Ttot) * H * dk * 2);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = ret::launch_chunk_prep(c.p.L, c.ws, c.err, s);
+  // q is rotated by one streaming pass; k inside the state pass, which stores
+  // the rotated rows for the output pass
+  if (e == cudaSuccess)
+    e = ret::launch_rope(q, nullptr, DType::BF16, q_rot, nullptr, c.p.L, H, dk, rope_base, s);
+  if (e == cudaSuccess) {
+    // state pass on the caller's k (rotated in the kernel, stored to k_rot) ...
+    ret::RopeInState rope;
+    rope.base = rope_base;
+    rope.k_rot = k_rot;
+    e = ret::launch_chunkwise_tc(kPhaseStates, nullptr, k, v, c.p.L, state_in,
+                                 state_in != nullptr, state_out, nullptr, dt(out_dtype), c.g,
+                                 c.g_t, c.gw, c.gb, c.eps, ng != nullptr, c.ws, H, dk, dv, c.dec,
+                                 c.err, s, rope);
+  }
+  // ... output pass on the rotated q and k
+  if (e == cudaSuccess)
+    e = ret::launch_chunkwise_tc(kPhaseOutputs, q_rot, k_rot, v, c.p.L, state_in,
+                                 state_in != nullptr, nullptr, out, dt(out_dtype), c.g, c.g_t,
+                                 c.gw, c.gb, c.eps, ng != nullptr, c.ws, H, dk, dv, c.dec, c.err,
+                                 s);
+  return cuda_status(e);
+}
+
 ret_status retention_chunkwise_states(const void* k, const void* v, ret_dtype in_dtype,
                                       const double* gamma, int chunk,
                                       const int32_t* cu_seqlens, int nseq,

@@ -66,6 +66,32 @@ __device__ __forceinline__ void raise_error(unsigned* err, unsigned bits) {
   if (err) atomicOr(err, bits);
 }
 
+// ---- rotary position encoding ------------------------------------------------
+//
+// The standard rotary form (the pages name a position rotation of Q and K but
+// give no formula): the pair (x[2i], x[2i+1]) of a token at position p turns
+// by p * theta_i, theta_i = base^(-2i/d).  theta_i is passed in double; the
+// angle is formed and reduced modulo 2 pi in double precision and its sine and
+// cosine are taken in float on an argument in [-pi, pi], so that large
+// positions keep float accuracy.  Every kernel that rotates uses this helper
+// and rotate_pair, so the rotated values agree bit for bit between them.
+__device__ __forceinline__ double rope_theta(int i, int d, double log2_base) {
+  return exp2(-(2.0 * i / d) * log2_base);
+}
+__device__ __forceinline__ void rope_sincos(int pos, double theta, float& sn, float& cs) {
+  constexpr double kTwoPi = 6.283185307179586476925286766559;
+  const double r = static_cast<double>(pos) * theta;
+  const double turns = rint(r * (1.0 / kTwoPi));
+  const float ang = static_cast<float>(fma(-turns, kTwoPi, r));
+  sincosf(ang, &sn, &cs);
+}
+// (x0, x1) rotated by the angle whose sine and cosine are sn, cs (float32).
+__device__ __forceinline__ void rotate_pair(float x0, float x1, float sn, float cs, float& y0,
+                                            float& y1) {
+  y0 = fmaf(x0, cs, -x1 * sn);
+  y1 = fmaf(x0, sn, x1 * cs);
+}
+
 // ---- sequences and chunks -------------------------------------------------
 //
 // Both layouts are handled as packed sequences over a flat token axis of

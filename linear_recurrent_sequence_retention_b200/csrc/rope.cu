@@ -6,19 +6,15 @@
 // index within its own sequence) turns by the angle p * theta_i with
 // theta_i = base^(-2i/d).
 //
-// One streaming pass over q and k (HBM-bound).  One block per token; thread i
-// owns pair i of every head of q and k, so the angle is computed once per
-// (token, pair) and applied to 2H pairs.  The angle is formed and reduced
-// modulo 2 pi in double precision and its sine and cosine are taken in float
-// (sincosf on an argument in [-pi, pi]), so that large positions keep float
-// accuracy; the rotation itself is float32, and bf16 outputs are rounded to
-// nearest once.
+// One streaming pass over q and k (HBM-bound; k may be absent).  One block per
+// token; thread i owns pair i of every head, so the angle is computed once per
+// (token, pair) and applied to 2H pairs.  The angle and the rotation come from
+// the helpers in common.cuh (double-precision angle reduction, float32
+// rotation); bf16 outputs are rounded to nearest once.
 #include "launch.h"
 
 namespace ret {
 namespace {
-
-constexpr double kTwoPi = 6.283185307179586476925286766559;
 
 template <typename T> struct Pair;
 template <> struct Pair<float> {
@@ -59,20 +55,19 @@ rope_kernel(const T* __restrict__ q, const T* __restrict__ k, T* qo, T* ko, SeqL
   }
   const int half = d >> 1;
   for (int i = threadIdx.x; i < half; i += blockDim.x) {
-    const double theta = exp2(-(2.0 * i / d) * log2_base);
-    const double r = static_cast<double>(pos) * theta;
-    const double turns = rint(r * (1.0 / kTwoPi));
-    const float ang = static_cast<float>(fma(-turns, kTwoPi, r));
     float sn, cs;
-    sincosf(ang, &sn, &cs);
+    rope_sincos(pos, rope_theta(i, d, log2_base), sn, cs);
     for (int h = 0; h < H; ++h) {
       const size_t off = (static_cast<size_t>(n) * H + h) * d + 2 * i;
+      float y0, y1;
       const auto vq = Pair<T>::ld(q + off);
-      const auto vk = Pair<T>::ld(k + off);
-      const float q0 = Pair<T>::lo(vq), q1 = Pair<T>::hi(vq);
-      const float k0 = Pair<T>::lo(vk), k1 = Pair<T>::hi(vk);
-      Pair<T>::st(qo + off, fmaf(q0, cs, -q1 * sn), fmaf(q0, sn, q1 * cs));
-      Pair<T>::st(ko + off, fmaf(k0, cs, -k1 * sn), fmaf(k0, sn, k1 * cs));
+      rotate_pair(Pair<T>::lo(vq), Pair<T>::hi(vq), sn, cs, y0, y1);
+      Pair<T>::st(qo + off, y0, y1);
+      if (k != nullptr) {                  // k == nullptr: q alone
+        const auto vk = Pair<T>::ld(k + off);
+        rotate_pair(Pair<T>::lo(vk), Pair<T>::hi(vk), sn, cs, y0, y1);
+        Pair<T>::st(ko + off, y0, y1);
+      }
     }
   }
 }

@@ -41,6 +41,8 @@ EXPORTED = (
     "retention_chunkwise_states",
     "retention_chunkwise_outputs",
     "retention_chunkwise_fwd_static_ws",
+    "retention_chunkwise_fwd_rope_workspace_size",
+    "retention_chunkwise_fwd_rope",
     "retention_chunkwise_bwd_workspace_size",
     "retention_chunkwise_bwd",
     "retention_rope",
@@ -105,6 +107,12 @@ def lib():
     L.retention_chunkwise_fwd_static_ws.argtypes = [vp, vp, vp, ci, cd, ci, vp, ci, vp, vp, vp,
                                                     ci, ctypes.POINTER(NormGate),
                                                     ci, ci, ci, ci, ci, vp]
+    L.retention_chunkwise_fwd_rope_workspace_size.restype = ctypes.c_size_t
+    L.retention_chunkwise_fwd_rope_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, ci]
+    L.retention_chunkwise_fwd_rope.restype = ci
+    L.retention_chunkwise_fwd_rope.argtypes = [vp, vp, vp, ci, cd, ci, vp, ci, vp, vp, vp, ci,
+                                               ctypes.POINTER(NormGate), ctypes.c_double, vp,
+                                               ctypes.c_size_t, ci, ci, ci, ci, ci, vp]
     L.retention_chunkwise_bwd_workspace_size.restype = ctypes.c_size_t
     L.retention_chunkwise_bwd_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci]
     L.retention_chunkwise_bwd.restype = ci
@@ -212,14 +220,21 @@ def alloc_workspace(nbytes, device):
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
+def chunkwise_fwd_rope_workspace_size(chunk, B, T, H, dk, dv, nseq=0):
+    return lib().retention_chunkwise_fwd_rope_workspace_size(chunk, B, T, H, dk, dv, nseq)
+
+
 def chunkwise_fwd(q, k, v, gamma, chunk, cu_seqlens=None, state_in=None, return_state=False,
                   g=None, gn_weight=None, gn_bias=None, eps=1e-5, out_dtype=None, out=None,
-                  state_out=None, workspace=None, stream=None):
+                  state_out=None, workspace=None, stream=None, rope_base=None):
     """Chunkwise form (+ optional fused GroupNorm and swish gate when ``g`` is given).
 
     q,k: [B,T,H,dk]; v: [B,T,H,dv]; packed sequences: B = 1 and ``cu_seqlens``
     an int32 CUDA tensor [nseq+1].  Returns ``out`` ([B,T,H,dv]: o, or y when
-    gated) and, with ``return_state``, the final fp32 states.
+    gated) and, with ``return_state``, the final fp32 states.  With
+    ``rope_base`` (bf16 inputs only) q and k are first given the rotary
+    position encoding of :func:`rope` inside the same call
+    (``retention_chunkwise_fwd_rope``); q and k themselves are not modified.
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _dev(t, n)
@@ -266,18 +281,30 @@ def chunkwise_fwd(q, k, v, gamma, chunk, cu_seqlens=None, state_in=None, return_
         ng = NormGate(g.data_ptr(), _dt(g), gn_weight.data_ptr() if gn_weight is not None else None,
                       gn_bias.data_ptr() if gn_bias is not None else None, float(eps))
         keep.append(ng)
-    need = lib().retention_chunkwise_workspace_size(_dt(q), chunk, B, T, H, dk, dv, nseq)
+    if rope_base is not None:
+        if _dt(q) != RET_BF16:
+            raise RetentionError(RET_ERR_UNSUPPORTED, "retention_chunkwise_fwd_rope")
+        need = lib().retention_chunkwise_fwd_rope_workspace_size(chunk, B, T, H, dk, dv, nseq)
+        where = "retention_chunkwise_fwd_rope_workspace_size"
+    else:
+        need = lib().retention_chunkwise_workspace_size(_dt(q), chunk, B, T, H, dk, dv, nseq)
+        where = "retention_chunkwise_workspace_size"
     if need == 0:
         st = RET_ERR_UNSUPPORTED if _dt(q) == RET_BF16 else RET_ERR_INVALID_ARG
-        raise RetentionError(st, "retention_chunkwise_workspace_size")
+        raise RetentionError(st, where)
     if workspace is None:
         workspace = alloc_workspace(need, q.device)
-    st = lib().retention_chunkwise_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _dt(q), _gammas(gamma, H), int(chunk),
-        _ptr(cu_seqlens), nseq, _ptr(state_in), _ptr(state_out), _ptr(out), _dt(out),
-        ctypes.byref(ng) if ng is not None else None, _ptr(workspace),
-        workspace.numel() * workspace.element_size(), B, T, H, dk, dv, _stream(stream))
-    _check(st, "retention_chunkwise_fwd")
+    head = (_ptr(q), _ptr(k), _ptr(v), _dt(q), _gammas(gamma, H), int(chunk),
+            _ptr(cu_seqlens), nseq, _ptr(state_in), _ptr(state_out), _ptr(out), _dt(out),
+            ctypes.byref(ng) if ng is not None else None)
+    tail = (_ptr(workspace), workspace.numel() * workspace.element_size(), B, T, H, dk, dv,
+            _stream(stream))
+    if rope_base is not None:
+        st = lib().retention_chunkwise_fwd_rope(*head, float(rope_base), *tail)
+        _check(st, "retention_chunkwise_fwd_rope")
+    else:
+        st = lib().retention_chunkwise_fwd(*head, *tail)
+        _check(st, "retention_chunkwise_fwd")
     return (out, state_out) if return_state else out
 
 
