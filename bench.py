@@ -724,9 +724,9 @@ def run_rope(args, world, rank, pk, pk_kind):
 
 def rope_forward_ab(args, world, rank):
     """The 6.7B-shaped forward (GroupNorm + gate, y bf16, final state) on
-    rotated q and k, two ways: the rotary kernel followed by the chunkwise
-    forward, and the fused call (k rotated inside the state pass, q by one
-    q-only pass).  Same inputs, same outputs bit for bit."""
+    rotated q and k through the one-call entry (retention_chunkwise_fwd_rope:
+    the rotary pass over q and k, then the two chunkwise passes), and the
+    share of the rotary pass in it."""
     from linear_recurrent_sequence_retention_b200 import ops
     wl = W.WORKLOADS[HEADLINE]
     dev = torch.device("cuda")
@@ -735,40 +735,32 @@ def rope_forward_ab(args, world, rank):
     gam = W.head_gammas(H)
     y = torch.empty(B, T, H, dv, device=dev, dtype=torch.bfloat16)
     S = torch.empty(B, H, dk, dv, device=dev, dtype=torch.float32)
-    qo, ko = torch.empty_like(q), torch.empty_like(k)
-    ws_sep = ops.alloc_workspace(ops.chunkwise_workspace_size(torch.bfloat16, C, B, T, H, dk, dv), dev)
-    ws_fused = ops.alloc_workspace(ops.chunkwise_fwd_rope_workspace_size(C, B, T, H, dk, dv), dev)
+    ws = ops.alloc_workspace(ops.chunkwise_fwd_rope_workspace_size(C, B, T, H, dk, dv), dev)
 
-    def separate():
-        ops.rope(q, k, q_out=qo, k_out=ko)
-        ops.chunkwise_fwd(qo, ko, v, gam, C, g=g, out=y, state_out=S, workspace=ws_sep)
-
-    def fused():
-        ops.chunkwise_fwd(q, k, v, gam, C, g=g, out=y, state_out=S, workspace=ws_fused,
+    def call():
+        ops.chunkwise_fwd(q, k, v, gam, C, g=g, out=y, state_out=S, workspace=ws,
                           rope_base=10000.0)
 
-    reps, res = 20, {}
-    for name, fn in (("rope_kernel_then_forward", separate), ("fused", fused)):
-        for _ in range(max(3, args.warmup)):
-            fn()
-        barrier(world)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(reps):
-            fn()
-        e1.record()
-        torch.cuda.synchronize()
-        barrier(world)
-        res[name] = max_over_ranks(e0.elapsed_time(e1) / reps, world)
+    reps = 20
+    for _ in range(max(3, args.warmup)):
+        call()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
     ops.check_device_error()
-    del q, k, v, g, y, S, qo, ko, ws_sep, ws_fused
+    ms = max_over_ranks(e0.elapsed_time(e1) / reps, world)
+    del q, k, v, g, y, S, ws
     torch.cuda.empty_cache()
-    return {"workload": wl.name, "ms_per_call": res,
-            "faster": min(res, key=res.get),
-            "kernels": {"rope_kernel_then_forward": "rope_kernel (q, k) + chunk_prep + state + output",
-                        "fused": "chunk_prep + rope_kernel (q only) + state (rotates k) + output"},
-            "gpu_launches": 2 * reps * 4}
+    return {"workload": wl.name, "entry": "retention_chunkwise_fwd_rope", "ms_per_call": ms,
+            "tokens_per_s": sum_over_ranks(B * T, world) / (ms / 1e3),
+            "kernels": "rope_kernel (q, k) + state + output",
+            "gpu_launches": reps * 3}
 
 
 def run_rla(args, world, rank, pk, pk_kind):

@@ -417,14 +417,17 @@ RET_API ret_status retention_rla_fwd(const void* q, const void* k, const void* v
                                      ret_stream_t stream);
 
 /*
- * Chunkwise forward with the rotary position encoding of q and k fused in:
- * the result of retention_rope(q, k, base) followed by retention_chunkwise_fwd
- * on the rotated q and k (abeam.tech summary, 「Retentionは「内容に応じた参照」と
- * 「距離による忘却」を掛け合わせる」: Q and K are rotated by position after the
- * projections; the standard rotary form, see retention_rope), without a
- * separate pass over k: the state pass rotates k as it loads it (and keeps the
- * rotated rows for the output pass); q is rotated by one streaming pass.  The
- * rotated values are those retention_rope stores, bit for bit.
+ * Chunkwise forward with the rotary position encoding of q and k in the same
+ * call: the result of retention_rope(q, k, base) followed by
+ * retention_chunkwise_fwd on the rotated q and k, bit for bit (abeam.tech
+ * summary, 「Retentionは「内容に応じた参照」と「距離による忘却」を掛け合わせる」:
+ * Q and K are rotated by position after the projections; the standard rotary
+ * form, see retention_rope).  The rotated copies live in the workspace, so
+ * the caller keeps q and k unrotated and needs no buffers of its own.
+ * Schedule: one rotary pass over q and k, then the two chunkwise passes.
+ * (Rotating k inside the state pass instead was measured slower on B200: the
+ * angle reduction lands on the converter warps that set the state pass's
+ * pace.)
  * Arguments as retention_chunkwise_fwd, plus rope_base (> 1, finite); bf16
  * inputs only (RET_ERR_UNSUPPORTED otherwise), dk even.  q and k are not
  * modified.  workspace: at least retention_chunkwise_fwd_rope_workspace_size()

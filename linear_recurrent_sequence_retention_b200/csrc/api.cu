@@ -314,26 +314,15 @@ ret_status retention_chunkwise_fwd_rope(const void* q, const void* k, const void
   void* k_rot = rot + round256(static_cast<size_t>(c.p.L.Ttot) * H * dk * 2);
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = ret::launch_chunk_prep(c.p.L, c.ws, c.err, s);
-  // q is rotated by one streaming pass; k inside the state pass, which stores
-  // the rotated rows for the output pass
+  // one streaming pass rotates q and k into the workspace; the chunkwise
+  // passes then read the rotated copies (faster on this GPU than rotating k
+  // inside the state pass, whose converter warps set that pass's pace)
   if (e == cudaSuccess)
-    e = ret::launch_rope(q, nullptr, DType::BF16, q_rot, nullptr, c.p.L, H, dk, rope_base, s);
-  if (e == cudaSuccess) {
-    // state pass on the caller's k (rotated in the kernel, stored to k_rot) ...
-    ret::RopeInState rope;
-    rope.base = rope_base;
-    rope.k_rot = k_rot;
-    e = ret::launch_chunkwise_tc(kPhaseStates, nullptr, k, v, c.p.L, state_in,
-                                 state_in != nullptr, state_out, nullptr, dt(out_dtype), c.g,
-                                 c.g_t, c.gw, c.gb, c.eps, ng != nullptr, c.ws, H, dk, dv, c.dec,
-                                 c.err, s, rope);
-  }
-  // ... output pass on the rotated q and k
+    e = ret::launch_rope(q, k, DType::BF16, q_rot, k_rot, c.p.L, H, dk, rope_base, s);
   if (e == cudaSuccess)
-    e = ret::launch_chunkwise_tc(kPhaseOutputs, q_rot, k_rot, v, c.p.L, state_in,
-                                 state_in != nullptr, nullptr, out, dt(out_dtype), c.g, c.g_t,
-                                 c.gw, c.gb, c.eps, ng != nullptr, c.ws, H, dk, dv, c.dec, c.err,
-                                 s);
+    e = ret::launch_chunkwise_tc(ph, q_rot, k_rot, v, c.p.L, state_in, state_in != nullptr,
+                                 state_out, out, dt(out_dtype), c.g, c.g_t, c.gw, c.gb, c.eps,
+                                 ng != nullptr, c.ws, H, dk, dv, c.dec, c.err, s);
   return cuda_status(e);
 }
 

@@ -136,13 +136,6 @@ struct StateParams {
   float* state_out;
   int H, dk, dv;
   int write_v16;                     // the CTAs of the first d_k block store the fp16 copy of v
-  // rotary position encoding of k inside the state pass (rope != 0): K rows are
-  // rotated before zeta (the rotation of common.cuh, rounded to bf16 as a
-  // separate rotation pass would store them) and the first d_v part's CTAs
-  // store the rotated rows to k_rot
-  int rope;
-  double rope_log2base;
-  __nv_bfloat16* k_rot;
   HeadDecay dec;
   unsigned* err;
 };
@@ -155,13 +148,10 @@ struct StCfg {
   // staging for the TMA stores of the state entering a chunk: two 128 x 64
   // fp16 boxes, filled in turn
   static constexpr uint32_t kStaging = 2 * kTallBox;
-  // barriers (256 B) and the rotary theta table (1 KB) follow the staging boxes
-  static constexpr int kStagesFit = static_cast<int>((232448 - kStaging - 256 - 1024) / kStage);
+  static constexpr int kStagesFit = static_cast<int>((232448 - kStaging - 1024) / kStage);
   static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
   static constexpr uint32_t kOffStaging = kStages * kStage;
-  static constexpr uint32_t kOffTheta = kOffStaging + kStaging + 256;   // rotary theta_i, double[128]
-  static constexpr uint32_t kSmem = kOffTheta + 1024;
-  static_assert(kSmem <= 232448, "shared memory budget");
+  static constexpr uint32_t kSmem = kOffStaging + kStaging + 256;
 };
 
 template <int NS>
@@ -184,7 +174,6 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_hold + 1);
-  double* theta_tab = reinterpret_cast<double*>(smem + SC::kOffTheta);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // 1-D grid, sequence-major: all (head, d_k block, d_v part) CTAs of a
@@ -226,8 +215,6 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     tmem_alloc(tmem_hold, 2 * NS);       // two accumulators of NS columns
     tmem_relinquish();
   }
-  if (p.rope && static_cast<int>(threadIdx.x) < p.dk / 2)
-    theta_tab[threadIdx.x] = rope_theta(threadIdx.x, p.dk, p.rope_log2base);
   if (kboxes == 1) {
     // d_k = 64: the second 64-row half of every zeta*K tile stays zero, so the
     // 128-row MMA adds nothing to TMEM rows 64..127
@@ -465,30 +452,6 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
           uint4 w4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) w4[e] = rp[(4 * khalf + e) ^ sw];
-          if (p.rope && jtok < Lc) {
-            // the rotary encoding of this half row (16 pairs) at its position in the
-            // sequence, rounded to bf16; the first d_v part stores it as k_rot
-            const int pos = c * L.chunk + jtok;
-            const int col0 = 128 * m + 64 * (krow >> 6) + 32 * khalf;   // first d_k column
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              uint32_t w[4] = {w4[e].x, w4[e].y, w4[e].z, w4[e].w};
-#pragma unroll
-              for (int q2 = 0; q2 < 4; ++q2) {
-                float sn, cs, y0, y1;
-                rope_sincos(pos, theta_tab[(col0 >> 1) + 4 * e + q2], sn, cs);
-                rotate_pair(bf16_lo(w[q2]), bf16_hi(w[q2]), sn, cs, y0, y1);
-                w[q2] = pack_bf16(y0, y1);
-              }
-              w4[e] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            if (p.k_rot && part == 0) {
-              uint4* dst = reinterpret_cast<uint4*>(
-                  p.k_rot + (static_cast<size_t>(tok0 + jtok) * p.H + h) * p.dk + col0);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) dst[e] = w4[e];
-            }
-          }
           const uint64_t z2 = f2_make(z, z);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -1971,8 +1934,7 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
                                 float* state_out, void* out, DType out_t, const void* g,
                                 DType g_t, const float* gn_w, const float* gn_b, float eps,
                                 bool gated, ChunkWorkspace ws, int H, int dk, int dv,
-                                const HeadDecay& dec, unsigned* err, cudaStream_t s,
-                                RopeInState rope) {
+                                const HeadDecay& dec, unsigned* err, cudaStream_t s) {
   if (!chunkwise_tc_supported(dk, dv, L.chunk)) return cudaErrorNotSupported;
   const uint64_t Ttot = static_cast<uint64_t>(L.Ttot > 0 ? L.Ttot : 1);
   cudaError_t e = cudaSuccess;
@@ -1992,9 +1954,6 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
     sp.state_in = state_in;
     sp.state_out = state_out;
     sp.write_v16 = ws.v16 != nullptr ? 1 : 0;
-    sp.rope = rope.k_rot != nullptr ? 1 : 0;
-    sp.rope_log2base = rope.k_rot != nullptr ? log2(rope.base) : 0.0;
-    sp.k_rot = static_cast<__nv_bfloat16*>(rope.k_rot);
     sp.H = H;
     sp.dk = dk;
     sp.dv = dv;

@@ -116,19 +116,12 @@ bool chunkwise_tc_supported(int dk, int dv, int chunk);
 // One bounded wait that is never satisfied (failure-detection self-test).
 cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t s);
 int chunkwise_tc_chunk(int chunk, int dv);  // chunk length the kernels evaluate
-// Rotary encoding of k inside the state pass: k_rot (bf16 [Ttot][H][dk]) receives
-// the rotated rows, which the state pass also uses; nullptr = no rotation.
-struct RopeInState {
-  double base = 0.0;
-  void* k_rot = nullptr;
-};
 cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const void* v,
                                 const SeqLayout& L, const float* state_in, bool has_state_in,
                                 float* state_out,
                                 void* out, DType out_t, const void* g, DType g_t,
                                 const float* gn_w, const float* gn_b, float eps, bool gated,
                                 ChunkWorkspace ws, int H, int dk, int dv,
-                                const HeadDecay& dec, unsigned* err, cudaStream_t s,
-                                RopeInState rope = RopeInState());
+                                const HeadDecay& dec, unsigned* err, cudaStream_t s);
 
 }  // namespace ret

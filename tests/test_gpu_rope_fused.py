@@ -1,11 +1,10 @@
-"""GPU parity of the chunkwise forward with the rotary position encoding fused
-in (retention_chunkwise_fwd_rope), through the C ABI.
+"""GPU parity of the chunkwise forward with the rotary position encoding in
+the same call (retention_chunkwise_fwd_rope), through the C ABI.
 
 Two checks per case:
-- bit for bit against the unfused route, retention_rope followed by
-  retention_chunkwise_fwd: the state pass rotates k with the same float32
-  arithmetic as the rotary kernel and rounds it to bf16 the same way, so both
-  routes feed identical operands to identical MMAs;
+- bit for bit against the two-call route, retention_rope followed by
+  retention_chunkwise_fwd on the caller's buffers (the one-call entry keeps
+  its rotated copies in the workspace);
 - against the fp64 oracle, rope of q and k (the standard rotary form applied
   after the projections, abeam.tech summary of the RetNet paper) rounded to
   bf16, followed by the chunkwise form and, when gated, the GroupNorm + swish
