@@ -47,6 +47,7 @@ from linear_recurrent_sequence_retention_b200 import workloads as W  # noqa: E40
 
 METRIC = "retention fwd tokens/s & % bf16 tensor peak; decode steps/s & HBM GB/s % peak"
 HEADLINE = "msr_6p7b_b2_h16_t8192_dk256_dv512_c512"
+HEADLINE_6P7B = HEADLINE                # fixed: --workload may change HEADLINE
 DECODE = "decode_6p7b_n128_h16_dk256_dv512"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TC_SOURCE = os.path.join(ROOT, "linear_recurrent_sequence_retention_b200", "csrc", "chunkwise_tc.cu")
@@ -805,6 +806,58 @@ def run_rla(args, world, rank, pk, pk_kind):
             "gpu_launches": 3 * reps}
 
 
+def run_parallel(args, world, rank, pk, pk_kind):
+    """The parallel form (Q K^T * D) V on the tensor cores, bf16 inputs, f32
+    accumulation, bf16 output, at the head shapes of the two chunkwise
+    workloads: each call is the fp16 copy of v and one output-kernel launch
+    over every causal 128 x 128 (query, key) block pair."""
+    from linear_recurrent_sequence_retention_b200 import ops
+    dev = torch.device("cuda")
+    res = {}
+    launches = 0
+    for name in (HEADLINE_6P7B, BACKWARD):
+        wl = W.WORKLOADS[name]
+        B, T, H, dk, dv = wl.B, wl.T, wl.H, wl.dk, wl.dv
+        q, k, v, _ = W.make_qkvg(B, T, H, dk, dv, "bf16", seed=rank, gate=False, device=dev)
+        gam = W.head_gammas(H)
+        o = torch.empty(B, T, H, dv, device=dev, dtype=torch.bfloat16)
+        ws = ops.alloc_workspace(ops.parallel_workspace_size(torch.bfloat16, B, T, H, dk, dv), dev)
+        for _ in range(max(3, args.warmup)):
+            ops.parallel_fwd(q, k, v, gam, out=o, workspace=ws)
+        reps = 10
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            ops.parallel_fwd(q, k, v, gam, out=o, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        ops.check_device_error()
+        ms = max_over_ranks(e0.elapsed_time(e1) / reps, world)
+        # causal pairs (n, m <= n): (q_n . k_m) and its weight times v_m
+        flops = B * H * T * (T + 1) * (dk + dv)
+        ach = flops / (ms / 1e3) / 1e12
+        rb = -(-T // 128)
+        executed = B * H * rb * (rb + 1) // 2 * 128 * 128 * 2 * (dk * (2 if dv > 256 else 1) + dv)
+        res[name] = {"ms_per_call": ms, "tokens_per_s": sum_over_ranks(B * T, world) / (ms / 1e3),
+                     "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
+                                  "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
+                                  "peak_source": f"{pk_kind} bf16 (burst)",
+                                  "algorithmic_flops_per_call": flops,
+                                  "executed_flops_per_call": executed,
+                                  "counting": "B H T (T+1) (dk + dv): the causal half of Q K^T "
+                                              "and of P V; executed adds the masked half of "
+                                              "the diagonal blocks and, for dv = 512, the "
+                                              "Q K^T repeated by the second dv half",
+                                  "kernel": "v16_kernel + output_kernel"}}
+        launches += 2 * reps
+        del q, k, v, o, ws
+        torch.cuda.empty_cache()
+    return {"workloads": res, "gpu_launches": launches}
+
+
 def main():
     global HEADLINE
     ap = argparse.ArgumentParser()
@@ -818,6 +871,7 @@ def main():
     ap.add_argument("--backward-only", action="store_true", help="backward only (profiling)")
     ap.add_argument("--no-rope", action="store_true")
     ap.add_argument("--no-rla", action="store_true")
+    ap.add_argument("--no-parallel", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--workload", default=HEADLINE,
@@ -897,6 +951,7 @@ def main():
     bwd = None if args.no_backward else run_backward(args, world, rank, pk, pk_kind)
     rope = None if args.no_rope else run_rope(args, world, rank, pk, pk_kind)
     rla = None if args.no_rla else run_rla(args, world, rank, pk, pk_kind)
+    par = None if args.no_parallel else run_parallel(args, world, rank, pk, pk_kind)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(wl, args.cpu_seconds)
@@ -922,13 +977,15 @@ def main():
             "backward": bwd,
             "rope": rope,
             "rla": rla,
+            "parallel": par,
             "e2e": head["e2e"],
             "cpu_baseline": cpu,
             "clocks": head["clocks"],
             "gpu_launches": (head["gpu_launches"] + (dec["gpu_launches"] if dec else 0)
                              + (bwd["gpu_launches"] if bwd else 0)
                              + (rope["gpu_launches"] if rope else 0)
-                             + (rla["gpu_launches"] if rla else 0)),
+                             + (rla["gpu_launches"] if rla else 0)
+                             + (par["gpu_launches"] if par else 0)),
             "arithmetic": "tensor-core MMAs (tcgen05) with f32 accumulation: q, k as bf16; "
                           "v, the decayed scores, the decayed query rows, zeta*K and the "
                           "carried state as fp16",

@@ -69,7 +69,7 @@
 extern "C" {
 #endif
 
-#define RETENTION_ABI_VERSION 2
+#define RETENTION_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define RET_API __attribute__((visibility("default")))
@@ -120,13 +120,31 @@ RET_API const char* retention_status_string(ret_status status);
  * independent causal sequence of T tokens.
  *   q, k:  [B,T,H,dk] in_dtype      v: [B,T,H,dv] in_dtype
  *   o:     [B,T,H,dv] o_dtype (fully overwritten)
- * Supported: dk, dv in 1..256; T >= 1; B*T*H*max(dk,dv) < 2^31.
+ *   workspace: device scratch of at least retention_parallel_workspace_size()
+ *          bytes, 256-byte aligned, owned by the caller; NULL when that size
+ *          is 0.  Its contents on entry do not matter.
+ * Kernels:
+ *   - bf16 inputs with dk in {64,128,256} and dv in {64,128,256,512}: tensor
+ *     cores.  An fp16 copy of v goes to the workspace (exact for |v| < 2^16;
+ *     larger values are reported as RET_ERR_RANGE by
+ *     retention_check_device_error), then 128-row query tiles run against
+ *     every causal 128-key block with the scores and decay formed in f32,
+ *     rounded once to fp16 for the P V product, f32 accumulation.  Precision
+ *     and range as the chunkwise tensor-core path.
+ *   - otherwise (float32 inputs, or bf16 with other head dims): CUDA cores,
+ *     float32 arithmetic, dk and dv up to 256.
+ * Supported: T >= 1; B*T*H*max(dk,dv) < 2^31.
  * Returns RET_ERR_INVALID_ARG for null pointers, B,T,H,dk,dv < 1, H > 64 or
- * gamma outside [0,1]; RET_ERR_UNSUPPORTED for larger head dims.
+ * gamma outside [0,1]; RET_ERR_UNSUPPORTED for head dims no kernel takes;
+ * RET_ERR_WORKSPACE when the workspace is needed and missing, too small or
+ * not 256-byte aligned.
  */
+RET_API size_t retention_parallel_workspace_size(ret_dtype in_dtype, int B, int T, int H,
+                                                 int dk, int dv);
 RET_API ret_status retention_parallel_fwd(const void* q, const void* k, const void* v,
                                   ret_dtype in_dtype, const double* gamma,
                                   void* o, ret_dtype o_dtype,
+                                  void* workspace, size_t workspace_bytes,
                                   int B, int T, int H, int dk, int dv,
                                   ret_stream_t stream);
 

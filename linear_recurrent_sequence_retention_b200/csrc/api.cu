@@ -147,10 +147,20 @@ const char* retention_status_string(ret_status s) {
   return "unknown ret_status";
 }
 
+size_t retention_parallel_workspace_size(ret_dtype in_dtype, int B, int T, int H, int dk,
+                                         int dv) {
+  if (in_dtype != RET_BF16 || !ret::parallel_tc_supported(dk, dv) || B < 1 || T < 1 || H < 1)
+    return 0;
+  const int dmax = dk > dv ? dk : dv;
+  const long long tt = static_cast<long long>(B) * (T > dk ? T : dk);
+  if (!fits_int(tt * H * dmax)) return 0;
+  return ret::parallel_tc_workspace_bytes(B, T, H, dk, dv);
+}
+
 ret_status retention_parallel_fwd(const void* q, const void* k, const void* v,
                                   ret_dtype in_dtype, const double* gamma, void* o,
-                                  ret_dtype o_dtype, int B, int T, int H, int dk, int dv,
-                                  ret_stream_t stream) {
+                                  ret_dtype o_dtype, void* workspace, size_t workspace_bytes,
+                                  int B, int T, int H, int dk, int dv, ret_stream_t stream) {
   if (!q || !k || !v || !o || !dtype_ok(in_dtype) || !dtype_ok(o_dtype)) return RET_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_ERR_INVALID_ARG;
   if (B < 1 || T < 1 || H < 1 || dk < 1 || dv < 1) return RET_ERR_INVALID_ARG;
@@ -158,9 +168,20 @@ ret_status retention_parallel_fwd(const void* q, const void* k, const void* v,
   if (!make_decay(gamma, H, &dec)) return RET_ERR_INVALID_ARG;
   const int dmax = dk > dv ? dk : dv;
   if (!fits_int(static_cast<long long>(B) * T * H * dmax)) return RET_ERR_INVALID_ARG;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t need = retention_parallel_workspace_size(in_dtype, B, T, H, dk, dv);
+  if (need > 0) {
+    if (workspace == nullptr || workspace_bytes < need ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return RET_ERR_WORKSPACE;
+    unsigned* err = error_word();
+    if (!err) return RET_ERR_CUDA;
+    return cuda_status(ret::launch_parallel_tc(q, k, v, o, dt(o_dtype), B, T, H, dk, dv, dec,
+                                               workspace, err, s));
+  }
   if (dk > 256 || dv > 256) return RET_ERR_UNSUPPORTED;
   return cuda_status(ret::launch_parallel_simt(q, k, v, dt(in_dtype), o, dt(o_dtype), B, T, H,
-                                               dk, dv, dec, reinterpret_cast<cudaStream_t>(stream)));
+                                               dk, dv, dec, s));
 }
 
 size_t retention_chunkwise_workspace_size(ret_dtype in_dtype, int chunk, int B, int T, int H,

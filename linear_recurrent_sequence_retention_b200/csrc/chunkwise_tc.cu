@@ -563,17 +563,21 @@ struct OutParams {
 template <int DK, int NV>
 struct OutCfg {
   static constexpr uint32_t kQBytes = (DK / 64) * kTallBox;
-  // The gate/output tile (NV/64 boxes of 128 rows x 64 columns) has a buffer of
-  // its own: held through the epilogue tail, it would otherwise pin ring stages
-  // that the next tile's key loads are waiting for.
-  static constexpr uint32_t kGateBytes = (NV / 64) * kTallBox;
   // barriers | gamma^d table | GroupNorm pairs passed between the two
   // warpgroups | GroupNorm pairs received from the partner CTA
   static constexpr uint32_t kMiscBytes = 256 + 512 + 1024 + 1024;
+  // Everything but Q and the small tables is ring: the loads in flight per SM
+  // set the pace of this kernel (a tile moves ~0.5 MB from L2).  The
+  // gate/output tile (NV/64 boxes of 128 rows x 64 columns, two per stage)
+  // takes ring stages too, loaded after the tile's other units and released
+  // by the epilogue once its stores have read them.
   static constexpr int kStages =
-      static_cast<int>((232448 - kQBytes - kGateBytes - kMiscBytes) / kOutStage);
-  static constexpr uint32_t kOffGate = kQBytes;
-  static constexpr uint32_t kOffStages = kOffGate + kGateBytes;
+      static_cast<int>((232448 - kQBytes - kMiscBytes) / kOutStage);
+  static constexpr int kGateStages =
+      static_cast<int>(((NV / 64) * kTallBox + kOutStage - 1) / kOutStage);
+  static_assert(kStages >= kGateStages + 2, "the ring must hold the gate tile and a key unit");
+  static_assert(2 * kStages + 14 <= 32, "barrier area");
+  static constexpr uint32_t kOffStages = kQBytes;
   static constexpr uint32_t kOffMisc = kOffStages + kStages * kOutStage;
   static constexpr uint32_t kSmem = kOffMisc + kMiscBytes;
   // TMEM (fixed): O in columns [0, NV), score buffers 0 and 1 in [256, 384)
@@ -677,9 +681,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   uint64_t* drain = bar_o + 1;
   uint64_t* bar_x = drain + 1;           // the partner's statistics have arrived
   uint64_t* bar_xack = bar_x + 1;        // the partner has read this CTA's statistics
-  uint64_t* g_full = bar_xack + 1;       // the gate tile has landed in the gate buffer
-  uint64_t* g_empty = g_full + 1;        // the epilogue is done with the gate/output buffer
-  uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(g_empty + 1);
+  uint32_t* tmem_hold = reinterpret_cast<uint32_t*>(bar_xack + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_hold + 1);
   float* pow_tab = reinterpret_cast<float*>(smem + C::kOffMisc + 256);    // gamma^d, d < 128
   float* wgx = reinterpret_cast<float*>(smem + C::kOffMisc + 768);        // [128][2]
@@ -692,9 +694,15 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   // K(kb) is kKU units of kKB 64-column boxes (128 keys each)
   constexpr int kKU = DK >= 128 ? DK / 128 : 1;
   constexpr int kKB = DK >= 128 ? 2 : 1;
-  // the gate/output tile: NV/64 boxes of 128 rows x 64 columns in the gate buffer
+  // the gate/output tile: NV/64 boxes of 128 rows x 64 columns in kGateStages
+  // ring stages (two boxes per stage)
   constexpr int kIoBoxes = NV / 64;
-  uint8_t* const gate_buf = smem + C::kOffGate;
+  constexpr int kGS = C::kGateStages;
+  constexpr int kBoxesPerStage = static_cast<int>(kOutStage / kTallBox);
+  // ring units of one tile before its gate stages
+  auto tile_units = [&](const OutTile& tt) {
+    return (tt.r + 1) * (kKU + 2) + (tt.inter ? DK / 64 : 0);
+  };
   auto io_staged = [&](const OutTile& t) {
     return (p.gated && p.g_tma) || (p.y_tma && t.nrows == kRowsPerTile);
   };
@@ -716,8 +724,6 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     mbar_init(drain, 1);
     mbar_init(bar_x, kWgThreads);
     mbar_init(bar_xack, kWgThreads);
-    mbar_init(g_full, 1);
-    mbar_init(g_empty, 1);
     *abort_flag = 0;
     if ((smem_u32(smem) & 1023u) != 0) {
       *abort_flag = 1;
@@ -753,7 +759,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmS);
       if (p.gated && p.g_tma) tma_prefetch_desc(&tmG);
-      int it = 0, tq = 0, ng = 0;      // ng: staged gate/output tiles so far
+      int it = 0, tq = 0;
       bool ok = true;
       auto next = [&](uint32_t bytes) -> uint8_t* {
         const int st = it % NST;
@@ -805,21 +811,24 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           }
         }
         if (ok && io_staged(t)) {
-          // the gate/output buffer, once the previous staged tile's stores have read it
-          if (!mbar_wait(g_empty, (ng & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
+          // the gate/output tile (or, ungated, just the stages its bf16
+          // output is staged in: an arrival with no bytes)
           const bool load_g = p.gated && p.g_tma;
-          mbar_arrive_expect_tx(g_full, load_g ? kIoBoxes * kTallBox : 0);
-          if (load_g)
-            for (int bb = 0; bb < kIoBoxes; ++bb)
-              tma_load_2d(gate_buf + bb * kTallBox, &tmG, g_full, t.h * p.dv + NV * part + 64 * bb,
-                          t.t0);
-          ++ng;
+          for (int gs = 0; gs < kGS && ok; ++gs) {
+            const int nbx = min(kIoBoxes - kBoxesPerStage * gs, kBoxesPerStage);
+            uint8_t* dst = next(load_g ? nbx * kTallBox : 0);
+            if (!dst) { ok = false; break; }
+            if (load_g)
+              for (int bb = 0; bb < nbx; ++bb)
+                tma_load_2d(dst + bb * kTallBox, &tmG, &full[it % NST],
+                            t.h * p.dv + NV * part + 64 * (kBoxesPerStage * gs + bb), t.t0);
+            ++it;
+          }
         }
       }
       if (!ok) {
         // let the copies already issued land before the CTA can exit
         if (tq > 0) mbar_wait_drain(bar_q, (tq - 1) & 1);
-        if (ng > 0) mbar_wait_drain(g_full, (ng - 1) & 1);
         for (int j = 1; j <= NST && it - j >= 0; ++j) {
           const int i2 = it - j;
           mbar_wait_drain(&full[i2 % NST], (i2 / NST) & 1);
@@ -917,6 +926,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           if (!ok) break;
         }
         mma_commit(bar_o);
+        if (io_staged(t)) it += kGS;           // the gate stages belong to the epilogue
         sblk += r + 1;
         ++tq;
       }
@@ -939,7 +949,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const bool wg_leader = (et & 127) == 0;           // first thread of the warpgroup
     constexpr bool kBoxPerWg = kHalf >= 64;           // each warpgroup owns whole boxes
     const uint32_t other = xchg ? (cluster_ctarank() ^ 1u) : 0u;
-    int tq = 0, sblk = 0, ng = 0;
+    int tq = 0, sblk = 0, git = 0;                    // git: ring position, as the producer counts
     bool ok = true;
     float pmax = 0.f;                                 // largest |P| and |decayed q| formed
     while (walk.next(p, cid, t)) {
@@ -948,7 +958,12 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const int r = t.r;
       const int i = r * kRowsPerTile + row;            // row within the chunk
       const bool staged = io_staged(t);
-      auto io_box = [&](int bx) -> uint8_t* { return gate_buf + bx * kTallBox; };
+      const int g0 = git + tile_units(t);              // this tile's first gate stage
+      git = g0 + (staged ? kGS : 0);
+      auto io_box = [&](int bx) -> uint8_t* {
+        return smem + C::kOffStages + ((g0 + bx / kBoxesPerStage) % NST) * kOutStage +
+               (bx % kBoxesPerStage) * kTallBox;
+      };
       const Decay1 dec(p.dec, t.h);
       // gamma^d for this tile's head (the previous tile's P is complete: every
       // epilogue thread passed the barrier in epi_all above after forming it)
@@ -1139,7 +1154,8 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const size_t obase = (static_cast<size_t>(t.t0 + row) * p.H + t.h) * p.dv + col0;
       const float shift = -mean_all * rstd;
       bool go = warp_all(ok && !*abort_flag);
-      if (go && staged) go = warp_all(mbar_wait(g_full, ng & 1, abort_flag, p.err));
+      for (int gs = 0; gs < kGS && go && staged; ++gs)
+        go = warp_all(mbar_wait(&full[(g0 + gs) % NST], ((g0 + gs) / NST) & 1, abort_flag, p.err));
       if (go) tc_fence_after();
       for (int j = 0; j < kHalf / 32; ++j) {
         // this piece's 32 columns in the staged gate/output box: box, first 16-byte piece
@@ -1249,8 +1265,8 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       if (out_tma && go && (kBoxPerWg ? wg_leader : et == 0)) tma_store_wait_read();
       if (staged) {
         wg2_sync();
-        if (et == 0) mbar_arrive(g_empty);
-        ++ng;
+        if (et == 0)
+          for (int gs = 0; gs < kGS; ++gs) mbar_arrive(&empty[(g0 + gs) % NST]);
       }
       ++tq;
     }
@@ -1905,6 +1921,42 @@ cudaError_t launch_out_c(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ms, mg, my, op);
 }
 
+// fp16 image of v for the P V products of the parallel form (the state pass
+// writes it for the chunkwise form).  Exact inside fp16's range; |v| >= 2^16
+// (bf16 0x4780 and above, NaN and infinity included) has no fp16 value and
+// raises kErrRange.  Eight values per 16-byte access, two accesses in flight
+// per thread.
+__global__ void __launch_bounds__(256) v16_kernel(const uint4* __restrict__ v,
+                                                   uint4* __restrict__ v16, long long n16,
+                                                   unsigned* err) {
+  uint32_t amax = 0;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  auto convert = [&](uint4 w) {
+    const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) amax = __vmaxu2(amax, a[e] & 0x7fff7fffu);
+    return make_uint4(bf16x2_to_f16x2(a[0]), bf16x2_to_f16x2(a[1]), bf16x2_to_f16x2(a[2]),
+                      bf16x2_to_f16x2(a[3]));
+  };
+  for (; i + stride < n16; i += 2 * stride) {
+    const uint4 w0 = __ldcs(v + i);
+    const uint4 w1 = __ldcs(v + i + stride);
+    v16[i] = convert(w0);
+    v16[i + stride] = convert(w1);
+  }
+  if (i < n16) v16[i] = convert(__ldcs(v + i));
+  const uint32_t big = max(amax & 0xffffu, amax >> 16);
+  if (__any_sync(0xffffffffu, big >= 0x4780u) && (threadIdx.x & 31) == 0)
+    raise_error(err, kErrRange);
+}
+
+cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
+                               bool has_state_in, void* out, DType out_t, const void* g,
+                               DType g_t, const float* gn_w, const float* gn_b, float eps,
+                               bool gated, ChunkWorkspace ws, int H, int dk, int dv,
+                               const HeadDecay& dec, unsigned* err, cudaStream_t s);
+
 }  // namespace
 
 cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t s) {
@@ -1975,7 +2027,24 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
     }
   }
   if (e != cudaSuccess || L.Ttot == 0 || !(phases & 2)) return e;
-  // ---- output pass ----
+  return launch_output_pass(q, k, L, has_state_in, out, out_t, g, g_t, gn_w, gn_b, eps, gated,
+                            ws, H, dk, dv, dec, err, s);
+}
+
+namespace {
+
+// The output pass: every 128-row tile of every chunk, on the persistent
+// output kernel (or the compact one for one-block chunks).  The chunk length
+// is L.chunk, a multiple of 128 (the parallel form runs the whole sequence as
+// one chunk).  Reads q, k, the fp16 copy of v (ws.v16) and, for tiles whose
+// chunk carries a state in, the fp16 state slots (ws.states).
+cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
+                               bool has_state_in, void* out, DType out_t, const void* g,
+                               DType g_t, const float* gn_w, const float* gn_b, float eps,
+                               bool gated, ChunkWorkspace ws, int H, int dk, int dv,
+                               const HeadDecay& dec, unsigned* err, cudaStream_t s) {
+  if (L.chunk < kRowsPerTile || L.chunk % kRowsPerTile != 0) return cudaErrorInvalidValue;
+  const uint64_t Ttot = static_cast<uint64_t>(L.Ttot > 0 ? L.Ttot : 1);
   const int NV = dv > 256 ? 256 : dv;
   OutParams op;
   op.L = L;
@@ -2053,6 +2122,52 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
     case 128: return launch_out<256, 128>(mq, mk, mv, ms, mg, my, op, s);
     default: return launch_out<256, 256>(mq, mk, mv, ms, mg, my, op, s);
   }
+}
+
+}  // namespace
+
+bool parallel_tc_supported(int dk, int dv) {
+  return (dk == 64 || dk == 128 || dk == 256) &&
+         (dv == 64 || dv == 128 || dv == 256 || dv == 512);
+}
+
+size_t parallel_tc_workspace_bytes(int B, int T, int H, int dk, int dv) {
+  // the fp16 copy of v, at least B*H*d_k rows of d_v long: the output pass
+  // also builds its (never read) state-slot map over this buffer
+  const long long rows = static_cast<long long>(B) * (T > dk ? T : dk) * H;
+  return (static_cast<size_t>(rows) * dv * 2 + 255) & ~static_cast<size_t>(255);
+}
+
+cudaError_t launch_parallel_tc(const void* q, const void* k, const void* v, void* o, DType o_t,
+                               int B, int T, int H, int dk, int dv, const HeadDecay& dec,
+                               void* workspace, unsigned* err, cudaStream_t s) {
+  if (!parallel_tc_supported(dk, dv) || B < 1 || T < 1) return cudaErrorNotSupported;
+  // every (b, h) sequence is one chunk of ceil(T/128)*128 tokens with no
+  // incoming state: the chunkwise form then reduces to the parallel form
+  // (the intra-chunk term is (Q K^T * D) V over the whole sequence)
+  SeqLayout L;
+  L.cu = nullptr;
+  L.nseq = B;
+  L.T = T;
+  L.Ttot = B * T;
+  L.chunk = (T + kRowsPerTile - 1) / kRowsPerTile * kRowsPerTile;
+  L.nslots = B;
+  ChunkWorkspace ws;
+  ws.chunk_base = nullptr;
+  ws.order = nullptr;
+  ws.states = workspace;
+  ws.v16 = workspace;
+  ws.nslots = B;
+  const long long n16 = static_cast<long long>(B) * T * H * dv / 8;
+  const long long want = (n16 + 511) / 512;
+  const long long cap = static_cast<long long>(sm_count()) * 8;
+  const int blocks = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
+  v16_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(workspace),
+                                    n16, err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_output_pass(q, k, L, false, o, o_t, nullptr, DType::BF16, nullptr, nullptr, 0.f,
+                            false, ws, H, dk, dv, dec, err, s);
 }
 
 }  // namespace ret

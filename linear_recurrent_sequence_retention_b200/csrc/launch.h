@@ -124,4 +124,12 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
                                 ChunkWorkspace ws, int H, int dk, int dv,
                                 const HeadDecay& dec, unsigned* err, cudaStream_t s);
 
+// Parallel form on the tensor cores (bf16 inputs): an fp16 copy of v, then the
+// chunkwise output kernel with each sequence as a single chunk.
+bool parallel_tc_supported(int dk, int dv);
+size_t parallel_tc_workspace_bytes(int B, int T, int H, int dk, int dv);
+cudaError_t launch_parallel_tc(const void* q, const void* k, const void* v, void* o, DType o_t,
+                               int B, int T, int H, int dk, int dv, const HeadDecay& dec,
+                               void* workspace, unsigned* err, cudaStream_t s);
+
 }  // namespace ret

@@ -34,6 +34,7 @@ STATIC_WORKSPACE_BYTES = 32 << 20
 EXPORTED = (
     "retention_abi_version",
     "retention_status_string",
+    "retention_parallel_workspace_size",
     "retention_parallel_fwd",
     "retention_chunkwise_workspace_size",
     "retention_chunkwise_executed_chunk",
@@ -86,8 +87,11 @@ def lib():
     L.retention_abi_version.argtypes = []
     L.retention_status_string.restype = ctypes.c_char_p
     L.retention_status_string.argtypes = [ci]
+    L.retention_parallel_workspace_size.restype = ctypes.c_size_t
+    L.retention_parallel_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci]
     L.retention_parallel_fwd.restype = ci
-    L.retention_parallel_fwd.argtypes = [vp, vp, vp, ci, cd, vp, ci, ci, ci, ci, ci, ci, vp]
+    L.retention_parallel_fwd.argtypes = [vp, vp, vp, ci, cd, vp, ci, vp, ctypes.c_size_t,
+                                         ci, ci, ci, ci, ci, vp]
     L.retention_chunkwise_workspace_size.restype = ctypes.c_size_t
     L.retention_chunkwise_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci]
     L.retention_chunkwise_executed_chunk.restype = ci
@@ -188,19 +192,37 @@ def abi_version():
     return lib().retention_abi_version()
 
 
-def parallel_fwd(q, k, v, gamma, out_dtype=None, stream=None):
-    """Parallel form; q,k: [B,T,H,dk], v: [B,T,H,dv] -> o [B,T,H,dv]."""
+def parallel_workspace_size(dtype, B, T, H, dk, dv):
+    """Bytes of workspace the parallel form needs (0: none, the CUDA-core kernel)."""
+    code = RET_F32 if dtype == torch.float32 else RET_BF16
+    return int(lib().retention_parallel_workspace_size(code, B, T, H, dk, dv))
+
+
+def parallel_fwd(q, k, v, gamma, out_dtype=None, out=None, workspace=None, stream=None):
+    """Parallel form; q,k: [B,T,H,dk], v: [B,T,H,dv] -> o [B,T,H,dv].  bf16
+    inputs of the tensor-core head dims use a workspace (allocated here when
+    not given)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _dev(t, n)
     B, T, H, dk = q.shape
     dv = v.shape[3]
     if k.shape != q.shape or v.shape[:3] != q.shape[:3] or k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("q, k, v shapes/dtypes disagree")
-    o = torch.empty(B, T, H, dv, device=q.device, dtype=out_dtype or q.dtype)
+    if out is None:
+        out = torch.empty(B, T, H, dv, device=q.device, dtype=out_dtype or q.dtype)
+    else:
+        _dev(out, "out")
+        if tuple(out.shape) != (B, T, H, dv):
+            raise ValueError("out has the wrong shape")
+    need = lib().retention_parallel_workspace_size(_dt(q), B, T, H, dk, dv)
+    if need and workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = lib().retention_parallel_fwd(_ptr(q), _ptr(k), _ptr(v), _dt(q), _gammas(gamma, H),
-                                      _ptr(o), _dt(o), B, T, H, dk, dv, _stream(stream))
+                                      _ptr(out), _dt(out), _ptr(workspace), nbytes,
+                                      B, T, H, dk, dv, _stream(stream))
     _check(st, "retention_parallel_fwd")
-    return o
+    return out
 
 
 def chunkwise_workspace_size(dtype, chunk, B, T, H, dk, dv, nseq=0):

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     ops, L = _lib()
-    assert L.retention_abi_version() == 2
+    assert L.retention_abi_version() == 3
     for code in range(8):
         s = ops.status_string(code)
         assert s and "unknown" not in s
@@ -51,6 +51,7 @@ def test_abi_version_and_status_strings():
 
 FAKE = ctypes.c_void_p(0x10000)          # aligned, never dereferenced on these paths
 MISALIGNED = ctypes.c_void_p(0x10004)
+FAKE_WS = 0x100000                           # 256-byte aligned, never dereferenced
 
 
 def _g(*vals):
@@ -61,8 +62,8 @@ def test_parallel_rejects_bad_arguments():
     ops, L = _lib()
     f = L.retention_parallel_fwd
     ok = dict(B=1, T=8, H=2, dk=16, dv=16)
-    args = lambda q=FAKE, gamma=_g(0.5, 0.9), dk=16, dv=16, T=8, H=2, o_dt=0: (
-        q, FAKE, FAKE, 0, gamma, FAKE, o_dt, 1, T, H, dk, dv, None)
+    args = lambda q=FAKE, gamma=_g(0.5, 0.9), dk=16, dv=16, T=8, H=2, o_dt=0, dt=0, ws=None, nb=0: (
+        q, FAKE, FAKE, dt, gamma, FAKE, o_dt, ws, nb, 1, T, H, dk, dv, None)
     assert f(*args(q=None)) == ops.RET_ERR_INVALID_ARG
     assert f(*args(q=MISALIGNED)) == ops.RET_ERR_INVALID_ARG
     assert f(*args(gamma=_g(0.5, 1.5))) == ops.RET_ERR_INVALID_ARG
@@ -71,6 +72,18 @@ def test_parallel_rejects_bad_arguments():
     assert f(*args(T=0)) == ops.RET_ERR_INVALID_ARG
     assert f(*args(o_dt=7)) == ops.RET_ERR_INVALID_ARG
     assert f(*args(dk=300)) == ops.RET_ERR_UNSUPPORTED
+    # bf16 at tensor-core head dims needs the workspace: missing, short or misaligned
+    need = L.retention_parallel_workspace_size(ops.RET_BF16, 1, 8, 2, 128, 256)
+    assert need == 1 * 128 * 2 * 256 * 2     # fp16 copy of v, max(T, d_k) rows per sequence
+    bf = dict(dt=ops.RET_BF16, dk=128, dv=256)
+    assert f(*args(**bf)) == ops.RET_ERR_WORKSPACE
+    assert f(*args(**bf, ws=FAKE_WS, nb=need - 256)) == ops.RET_ERR_WORKSPACE
+    assert f(*args(**bf, ws=FAKE_WS + 16, nb=need)) == ops.RET_ERR_WORKSPACE
+    assert f(*args(dt=ops.RET_BF16, dk=128, dv=300)) == ops.RET_ERR_UNSUPPORTED
+    # float32 and non-tensor-core bf16 shapes need none
+    assert L.retention_parallel_workspace_size(ops.RET_F32, 1, 8, 2, 128, 256) == 0
+    assert L.retention_parallel_workspace_size(ops.RET_BF16, 1, 8, 2, 16, 16) == 0
+    assert L.retention_parallel_workspace_size(ops.RET_BF16, 2, 1000, 3, 64, 512) == 2 * 1000 * 3 * 512 * 2
 
 
 def test_workspace_size_query():
