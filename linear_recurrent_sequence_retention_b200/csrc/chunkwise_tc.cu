@@ -722,7 +722,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     mbar_init(bar_pp, 2 * kWgThreads);
     mbar_init(bar_o, 1);
     mbar_init(drain, 1);
-    mbar_init(bar_x, kWgThreads);
+    mbar_init(bar_x, 1);                  // armed per tile with the partner's 1 KB
     mbar_init(bar_xack, kWgThreads);
     *abort_flag = 0;
     if ((smem_u32(smem) & 1023u) != 0) {
@@ -1105,20 +1105,18 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           float m2 = m2_w + m21 + dd * dd * (0.5f * kHalf);
           float cnt = static_cast<float>(NV);
           if (xchg) {
-            // the other d_v part: write this part's (mean, M2) into the
-            // partner's receive buffer once it has read the previous pair,
-            // arrive on its barrier, then read the partner's pair and release
-            // this CTA's receive buffer
+            // the other d_v part: once the partner has read the previous
+            // pair, send this part's (mean, M2) into its receive buffer with
+            // st.async (the store signals 8 bytes on the partner's barrier,
+            // which its first epilogue thread arms for 128 rows), then read
+            // the partner's pair and release this CTA's receive buffer
             if (!cluster_waited) {
               cluster_wait();                        // partner's barriers are initialised
               cluster_waited = true;
             }
             bool xok = tq == 0 || mbar_wait_cluster(bar_xack, (tq - 1) & 1, abort_flag, p.err);
-            if (xok) {
-              st_cluster_f32(cluster_addr(&xrecv[2 * row], other), mean);
-              st_cluster_f32(cluster_addr(&xrecv[2 * row + 1], other), m2);
-            }
-            mbar_arrive_cluster(cluster_addr(bar_x, other));
+            if (et == 0) mbar_arrive_expect_tx(bar_x, kWgThreads * 8);
+            st_async_f32x2(cluster_addr(&xrecv[2 * row], other), mean, m2, cluster_addr(bar_x, other));
             xok = mbar_wait_cluster(bar_x, tq & 1, abort_flag, p.err) && xok;
             if (xok) {
               const float mo = xrecv[2 * row], m2o = xrecv[2 * row + 1];

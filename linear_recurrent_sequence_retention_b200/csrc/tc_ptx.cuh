@@ -373,6 +373,15 @@ __device__ __forceinline__ void st_cluster_f32(uint32_t remote, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
 }
 
+// Stores two floats into another CTA's shared memory and signals 8 bytes of
+// transaction on that CTA's mbarrier (cluster addresses), in one operation.
+__device__ __forceinline__ void st_async_f32x2(uint32_t remote, float a, float b,
+                                               uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];"
+               ::"r"(remote), "f"(a), "f"(b), "r"(remote_bar)
+               : "memory");
+}
+
 // Arrives on an mbarrier of another CTA in the cluster, releasing this
 // thread's earlier writes (including remote stores) at cluster scope.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
