@@ -664,6 +664,7 @@ def run_backward(args, world, rank, pk, pk_kind):
     peak_cc = fp32_fma_peak_tflops(pk)
     del q, k, v, do, dS, ws
     torch.cuda.empty_cache()
+    big = backward_6p7b(args, world, rank, pk, pk_kind)
     return {"workload": wl.name, "input_dtype": "bf16", "ms_per_call": ms_tc,
             "tokens_per_s": tokens / (ms_tc / 1e3),
             "ms_per_call_with_d_state_out": ms_tc_ds,
@@ -683,7 +684,54 @@ def run_backward(args, world, rank, pk, pk_kind):
                                        "peak_source": "derived: SMs x 128 FP32 lanes x 2 flops "
                                                       "x max SM clock",
                                        "kernel": "chunk_grad_simt_kernel + chunk_state_simt_kernel"}},
-            "gpu_launches": 13 * reps_tc + 15 * reps_tc + 5 * reps_cc}
+            "6p7b": big,
+            "gpu_launches": 13 * reps_tc + 15 * reps_tc + 5 * reps_cc + big["gpu_launches"]}
+
+
+def backward_6p7b(args, world, rank, pk, pk_kind):
+    """The backward at the 6.7B-shaped workload (B=2, T=8192, H=16, d_k=256,
+    d_v=512, chunk 512, bf16, with a final-state gradient): tensor cores, the
+    dQ and dK retentions in two d_v halves each."""
+    from linear_recurrent_sequence_retention_b200 import ops
+    wl = W.WORKLOADS[HEADLINE_6P7B]
+    dev = torch.device("cuda")
+    B, T, H, dk, dv, C = wl.B, wl.T, wl.H, wl.dk, wl.dv, wl.chunk
+    q, k, v, _ = W.make_qkvg(B, T, H, dk, dv, "bf16", seed=rank, gate=False, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(3000 + rank)
+    do = torch.randn(B, T, H, dv, generator=gen, device=dev).to(torch.bfloat16)
+    dS = torch.randn(B, H, dk, dv, generator=gen, device=dev)
+    gam = W.head_gammas(H)
+    ws = ops.alloc_workspace(ops.chunkwise_bwd_workspace_size(torch.bfloat16, C, B, T, H, dk, dv), dev)
+    flops = (3 * (C + 1) * (dk + dv) + 10 * dk * dv) * B * T * H
+    reps = 5
+    for _ in range(max(3, args.warmup)):
+        ops.chunkwise_bwd(q, k, v, do, gam, C, d_state_out=dS, return_d_state=True, workspace=ws)
+    ops.check_device_error()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        ops.chunkwise_bwd(q, k, v, do, gam, C, d_state_out=dS, return_d_state=True, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ops.check_device_error()
+    ms = max_over_ranks(e0.elapsed_time(e1) / reps, world)
+    ach = flops / (ms / 1e3) / 1e12
+    del q, k, v, do, dS, ws
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "ms_per_call_with_d_state_out": ms,
+            "tokens_per_s": sum_over_ranks(B * T, world) / (ms / 1e3),
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
+                         "peak_source": f"{pk_kind} bf16 (burst)",
+                         "algorithmic_flops_per_call": flops,
+                         "counting": f"per token-head 3 (C+1)(dk+dv) + 10 dk dv, C={C}",
+                         "kernel": "state_kernel + output_kernel (x5: dQ and dK in two d_v "
+                                   "halves), flip_tokens_kernel, split_heads_kernel"},
+            "gpu_launches": reps * 22}
 
 
 def run_rope(args, world, rank, pk, pk_kind):

@@ -444,7 +444,8 @@ struct BwdPlan {
   long long slots;
   size_t state_bytes;   // one set of per-chunk float32 states
   size_t bytes;         // CUDA-core path
-  bool tc_ok;           // the tensor-core path is possible (bf16, heads 64/128/256)
+  bool simt_ok;         // the CUDA-core path is possible (heads up to 256)
+  bool tc_ok;           // the tensor-core path is possible (bf16, d_k 64/128/256, d_v 64..512)
   ret::SeqLayout Ltc;   // tensor-core path: the executed chunk
   size_t tc_state;      // one set of fp16 states at that chunk
   size_t tc_states;     // + the fp16 copy of the value operand (the wider of d_k, d_v)
@@ -455,9 +456,10 @@ bool tc_head(int d) { return d == 64 || d == 128 || d == 256; }
 
 // Shared by the backward's size query and call.  The CUDA-core path (float32
 // arithmetic, f32 or bf16 inputs, heads up to 256) takes any arguments; bf16
-// inputs with heads of 64, 128 or 256 and a chunk of 64..512 may also run on
-// the tensor-core forward kernels (see launch_chunkwise_bwd_tc), and the
-// workspace is sized for whichever path needs more.
+// inputs with d_k in {64, 128, 256}, d_v in {64, 128, 256, 512} and a chunk of
+// 64..512 may also run on the tensor-core forward kernels (see
+// launch_chunkwise_bwd_tc; d_v = 512 only there), and the workspace is sized
+// for whichever possible path needs more.
 ret_status plan_chunkwise_bwd(ret_dtype in_dtype, int chunk, int B, int T, int H, int dk, int dv,
                               int nseq, const int32_t* cu, BwdPlan* p) {
   if (!dtype_ok(in_dtype) || chunk < 1 || H < 1 || H > ret::kMaxHeads || dk < 1 || dv < 1 ||
@@ -473,7 +475,9 @@ ret_status plan_chunkwise_bwd(ret_dtype in_dtype, int chunk, int B, int T, int H
   const int dmax = dk > dv ? dk : dv;
   if (!fits_int(Ttot * H * static_cast<long long>(dmax)) || !fits_int(Ttot + chunk))
     return RET_ERR_INVALID_ARG;
-  if (dk > 256 || dv > 256) return RET_ERR_UNSUPPORTED;
+  const bool tc_shape = in_dtype == RET_BF16 && tc_head(dk) && (tc_head(dv) || dv == 512);
+  p->simt_ok = dk <= 256 && dv <= 256;
+  if (!p->simt_ok && !tc_shape) return RET_ERR_UNSUPPORTED;
   p->L.cu = varlen ? cu : nullptr;
   p->L.nseq = varlen ? nseq : B;
   p->L.T = varlen ? 0 : T;
@@ -485,8 +489,11 @@ ret_status plan_chunkwise_bwd(ret_dtype in_dtype, int chunk, int B, int T, int H
   p->L.nslots = p->slots;
   p->state_bytes = static_cast<size_t>(p->slots) * H * dk * dv * sizeof(float);
   p->bytes = p->meta + 2 * p->state_bytes;
-  p->tc_ok = in_dtype == RET_BF16 && tc_head(dk) && tc_head(dv) &&
-             ret::chunkwise_tc_supported(dk, dv, chunk) && ret::chunkwise_tc_supported(dv, dk, chunk);
+  // the d_v = 512 passes that contract over d_v run on 256-wide halves
+  const int dvq = dv > 256 ? dv / 2 : dv;
+  p->tc_ok = tc_shape && ret::chunkwise_tc_supported(dk, dv, chunk) &&
+             ret::chunkwise_tc_supported(dvq, dk, chunk);
+  if (!p->simt_ok && !p->tc_ok) return RET_ERR_UNSUPPORTED;
   p->tc_bytes = 0;
   if (p->tc_ok) {
     // one executed chunk for the three passes (d_k and d_v exchange roles)
@@ -510,7 +517,8 @@ size_t retention_chunkwise_bwd_workspace_size(ret_dtype in_dtype, int chunk, int
                                               int H, int dk, int dv, int nseq) {
   BwdPlan p;
   if (plan_chunkwise_bwd(in_dtype, chunk, B, T, H, dk, dv, nseq, nullptr, &p) != RET_OK) return 0;
-  return p.bytes > p.tc_bytes ? p.bytes : p.tc_bytes;
+  const size_t a = p.simt_ok ? p.bytes : 0, b = p.tc_ok ? p.tc_bytes : 0;
+  return a > b ? a : b;
 }
 
 ret_status retention_chunkwise_bwd(const void* q, const void* k, const void* v, const void* d_out,
@@ -537,6 +545,7 @@ ret_status retention_chunkwise_bwd(const void* q, const void* k, const void* v, 
   for (int h = 0; h < H; ++h)
     if (gamma[h] != 0.0 && gamma[h] < 1e-6) gam_ok = false;
   const bool use_tc = p.tc_ok && (d_state_out == nullptr || gam_ok);
+  if (!use_tc && !p.simt_ok) return RET_ERR_UNSUPPORTED;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
       workspace_bytes < (use_tc ? p.tc_bytes : p.bytes))
     return RET_ERR_WORKSPACE;

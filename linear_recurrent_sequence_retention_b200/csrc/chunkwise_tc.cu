@@ -549,6 +549,7 @@ struct OutParams {
   int gated;
   int g_tma;                   // gate tile streamed by TMA (bf16 gate)
   int y_tma;                   // full output tiles written by TMA (bf16 output)
+  int acc_out;                 // float32 output, ungated: out += o instead of out = o
   int H, dk, dv;
   int rb;                      // 128-row blocks per chunk
   int parts;                   // d_v parts (cluster size)
@@ -1231,9 +1232,18 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                    pack_bf16(x[8 * c4 + 4], x[8 * c4 + 5]), pack_bf16(x[8 * c4 + 6], x[8 * c4 + 7]));
           } else if (live) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + 32 * j);
+            if (p.acc_out) {
 #pragma unroll
-            for (int c4 = 0; c4 < 8; ++c4)
-              dst[c4] = make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
+              for (int c4 = 0; c4 < 8; ++c4) {
+                const float4 a = dst[c4];
+                dst[c4] = make_float4(x[4 * c4] + a.x, x[4 * c4 + 1] + a.y, x[4 * c4 + 2] + a.z,
+                                      x[4 * c4 + 3] + a.w);
+              }
+            } else {
+#pragma unroll
+              for (int c4 = 0; c4 < 8; ++c4)
+                dst[c4] = make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
+            }
           }
         }
         if (kBoxPerWg && out_tma && (j & 1)) {       // uniform over the warpgroup
@@ -1953,7 +1963,8 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
                                bool has_state_in, void* out, DType out_t, const void* g,
                                DType g_t, const float* gn_w, const float* gn_b, float eps,
                                bool gated, ChunkWorkspace ws, int H, int dk, int dv,
-                               const HeadDecay& dec, unsigned* err, cudaStream_t s);
+                               const HeadDecay& dec, unsigned* err, cudaStream_t s,
+                               bool acc_out);
 
 }  // namespace
 
@@ -1984,7 +1995,8 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
                                 float* state_out, void* out, DType out_t, const void* g,
                                 DType g_t, const float* gn_w, const float* gn_b, float eps,
                                 bool gated, ChunkWorkspace ws, int H, int dk, int dv,
-                                const HeadDecay& dec, unsigned* err, cudaStream_t s) {
+                                const HeadDecay& dec, unsigned* err, cudaStream_t s,
+                                bool acc_out) {
   if (!chunkwise_tc_supported(dk, dv, L.chunk)) return cudaErrorNotSupported;
   const uint64_t Ttot = static_cast<uint64_t>(L.Ttot > 0 ? L.Ttot : 1);
   cudaError_t e = cudaSuccess;
@@ -2026,7 +2038,7 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
   }
   if (e != cudaSuccess || L.Ttot == 0 || !(phases & 2)) return e;
   return launch_output_pass(q, k, L, has_state_in, out, out_t, g, g_t, gn_w, gn_b, eps, gated,
-                            ws, H, dk, dv, dec, err, s);
+                            ws, H, dk, dv, dec, err, s, acc_out);
 }
 
 namespace {
@@ -2040,8 +2052,12 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
                                bool has_state_in, void* out, DType out_t, const void* g,
                                DType g_t, const float* gn_w, const float* gn_b, float eps,
                                bool gated, ChunkWorkspace ws, int H, int dk, int dv,
-                               const HeadDecay& dec, unsigned* err, cudaStream_t s) {
+                               const HeadDecay& dec, unsigned* err, cudaStream_t s,
+                               bool acc_out) {
   if (L.chunk < kRowsPerTile || L.chunk % kRowsPerTile != 0) return cudaErrorInvalidValue;
+  // accumulation: float32, ungated, and only in the persistent kernel (multi-block chunks)
+  if (acc_out && (out_t != DType::F32 || gated || L.chunk == kRowsPerTile))
+    return cudaErrorInvalidValue;
   const uint64_t Ttot = static_cast<uint64_t>(L.Ttot > 0 ? L.Ttot : 1);
   const int NV = dv > 256 ? 256 : dv;
   OutParams op;
@@ -2065,6 +2081,7 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
   op.err = err;
   op.g_tma = (gated && g_t == DType::BF16) ? 1 : 0;
   op.y_tma = out_t == DType::BF16 ? 1 : 0;
+  op.acc_out = acc_out ? 1 : 0;
   if (ws.v16 == nullptr) return cudaErrorInvalidValue;   // written by the state pass
   const uint64_t srows = static_cast<uint64_t>(ws.nslots) * H * dk;      // fp16 state slots
   const uint64_t hdv = static_cast<uint64_t>(H) * dv;
@@ -2165,7 +2182,7 @@ cudaError_t launch_parallel_tc(const void* q, const void* k, const void* v, void
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_output_pass(q, k, L, false, o, o_t, nullptr, DType::BF16, nullptr, nullptr, 0.f,
-                            false, ws, H, dk, dv, dec, err, s);
+                            false, ws, H, dk, dv, dec, err, s, false);
 }
 
 }  // namespace ret

@@ -13,13 +13,14 @@
 // the MMA operands are read at tf32 precision, relative error 2^-11), which
 // keeps the outputs and the carried state well inside the bf16-input bound.
 //
-// Persistent: one CTA per SM walks the (n, h) states.  Warp 0 streams the
-// state through a ring of 32 KB stages (64 rows x 128 columns, TMA, 128-byte
-// swizzle with 32-byte atoms, the layout MN-major tf32 operands take) and
-// prefetches the next state's q, k, v rows into L2; warp 1 issues the MMAs;
-// warps 2..9 form q_t gamma^(t+1), zeta_j k_j and v as float32 operand tiles
-// (and the Tn x Tn intra-step scores), update every stage in place after its
-// read MMA, store it back with TMA and finally add the intra-step terms to the
+// Persistent: one CTA per SM walks the (n, h) states.  Warp 0 streams, through
+// a ring of 32 KB stages, first the item's q, k, v rows (bf16, one stage, TMA)
+// and then its state (64 rows x 128 columns per stage, TMA, 128-byte swizzle
+// with 32-byte atoms, the layout MN-major tf32 operands take); warp 1 issues
+// the MMAs; warps 2..9 form q_t gamma^(t+1), zeta_j k_j and v as float32
+// operand tiles from the q, k, v stage (and the Tn x Tn intra-step scores, by
+// mma.sync on four warps), update every state stage in place after its read
+// MMA, store it back with TMA and finally add the intra-step terms to the
 // outputs.  Every wait is bounded.
 #include <cudaTypedefs.h>
 
@@ -89,7 +90,9 @@ __device__ __forceinline__ uint64_t sdesc_sw128_atom32(uint32_t saddr, uint32_t 
 __device__ __forceinline__ bool wall(bool v) { return __all_sync(0xffffffffu, v) != 0; }
 
 __global__ void __launch_bounds__(kDtThreads, 1)
-decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParams p) {
+decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const DecTcParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const DtLayout lay(p.dk, p.dv);
   uint8_t* ring = smem;
@@ -146,26 +149,28 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParam
     // ---------------- TMA producer: the state, 64 rows x 128 columns per stage ----------------
     if (lane == 0 && !*abort_flag) {
       tma_prefetch_desc(&tmS);
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
       int it = 0;
       bool ok = true;
+      const uint32_t qkv_bytes = static_cast<uint32_t>(p.Tn * (2 * p.dk + p.dv) * 2);
       for (int item = blockIdx.x; item < p.nitems && ok; item += gridDim.x) {
+        {
+          // the item's q, k and v rows (bf16, [Tn][dk], [Tn][dk], [dv/128][Tn][128]) into one stage
+          const int st = it % kDtStages;
+          if (!mbar_wait(&empty[st], ((it / kDtStages) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[st], qkv_bytes);
+          uint8_t* dst = ring + st * kDtStage;
+          const int h = item % p.H, y0 = (item / p.H) * p.Tn;
+          tma_load_2d(dst, &tmQ, &full[st], h * p.dk, y0);
+          tma_load_2d(dst + p.Tn * p.dk * 2, &tmK, &full[st], h * p.dk, y0);
+          for (int vbx = 0; vbx < p.dv / 128; ++vbx)
+            tma_load_2d(dst + 2 * p.Tn * p.dk * 2 + vbx * p.Tn * 256, &tmV, &full[st], h * p.dv + 128 * vbx, y0);
+          ++it;
+        }
         for (int b = 0; b < nb && ok; ++b) {
           for (int q = 0; q < nq; ++q, ++it) {
-            if (b == nb - 1 && q == nq - 1) {
-              // the next item's q, k, v rows into L2 with this item's last stage:
-              // a few stages before the workers form its operand tiles (earlier,
-              // the state streaming through L2 would evict them first)
-              const int nxt = item + gridDim.x;
-              if (nxt < p.nitems) {
-                const int hn = nxt % p.H, nn = nxt / p.H;
-                for (int t = 0; t < p.Tn; ++t) {
-                  const size_t row = (static_cast<size_t>(nn) * p.Tn + t) * p.H + hn;
-                  bulk_prefetch_l2(p.q + row * p.dk, static_cast<uint32_t>(p.dk * 2));
-                  bulk_prefetch_l2(p.k + row * p.dk, static_cast<uint32_t>(p.dk * 2));
-                  bulk_prefetch_l2(p.v + row * p.dv, static_cast<uint32_t>(p.dv * 2));
-                }
-              }
-            }
             const int st = it % kDtStages;
             if (!mbar_wait(&empty[st], ((it / kDtStages) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
             mbar_arrive_expect_tx(&full[st], kDtStage);
@@ -192,6 +197,7 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParam
       int it = 0, ndu = 0, nitem = 0;
       bool ok = true, issued = false;
       for (int item = blockIdx.x; item < p.nitems && ok; item += gridDim.x, ++nitem) {
+        ++it;                                   // the item's q, k, v stage (the workers' own)
         if (!mbar_wait(pro_full, nitem & 1, abort_flag, p.err)) { ok = false; break; }
         if (nitem > 0 && !mbar_wait(do_free, (nitem - 1) & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
@@ -260,11 +266,16 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParam
       if (!r) break;
       const int h = item % p.H, n = item / p.H;
       const Decay1 dg(p.dec, h);
+      const int qkv_it = it++;
+      const uint8_t* qkv = ring + (qkv_it % kDtStages) * kDtStage;
+      const bool qkv_ok = wall(ok && mbar_wait(&full[qkv_it % kDtStages], (qkv_it / kDtStages) & 1, abort_flag, p.err));
+      if (!qkv_ok) ok = false;
       // (a) q and k of the Tn tokens, unscaled, as [16][dk] float32 rows in the
       // qs and zk regions (k's float4 columns XOR-swizzled by row, so that the
       // score pass below reads 16 rows without bank conflicts; zero rows from Tn
       // on); v straight into its MN-major tile; the per-token decay factors.
-      // Every 16-byte global load is issued before the first store.
+      // The rows come from the item's q, k, v ring stage; every 16-byte load
+      // is issued before the first store.
       float* qraw = reinterpret_cast<float*>(qs);
       float* kraw = reinterpret_cast<float*>(zk);
       float* fac = att + kDtMaxT * kDtMaxT;            // [2][16]: gamma^(t+1), zeta_t
@@ -285,10 +296,9 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParam
         for (int m = 0; m < kQK; ++m) {
           const int e8 = (wt + 256 * m) * 8, t = e8 / p.dk, i = e8 % p.dk;
           uq[m] = uk[m] = make_uint4(0, 0, 0, 0);
-          if (e8 < kDtMaxT * p.dk && t < p.Tn) {
-            const size_t row = ((static_cast<size_t>(n) * p.Tn + t) * p.H + h) * p.dk + i;
-            uq[m] = *reinterpret_cast<const uint4*>(p.q + row);
-            uk[m] = *reinterpret_cast<const uint4*>(p.k + row);
+          if (e8 < kDtMaxT * p.dk && t < p.Tn && qkv_ok) {
+            uq[m] = *reinterpret_cast<const uint4*>(qkv + (t * p.dk + i) * 2);
+            uk[m] = *reinterpret_cast<const uint4*>(qkv + ((p.Tn + t) * p.dk + i) * 2);
           }
         }
         for (int m0 = 0; m0 < nv; m0 += kV * 256) {
@@ -296,8 +306,9 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParam
           for (int m = 0; m < kV; ++m) {
             const int e8 = (m0 + wt + 256 * m) * 8, t = e8 / p.dv, cc = e8 % p.dv;
             uv[m] = make_uint4(0, 0, 0, 0);
-            if (e8 < kDtMaxT * p.dv && t < p.Tn)
-              uv[m] = *reinterpret_cast<const uint4*>(p.v + ((static_cast<size_t>(n) * p.Tn + t) * p.H + h) * p.dv + cc);
+            if (e8 < kDtMaxT * p.dv && t < p.Tn && qkv_ok)
+              uv[m] = *reinterpret_cast<const uint4*>(qkv + 2 * p.Tn * p.dk * 2 + (cc >> 7) * p.Tn * 256 +
+                                                      (t * 128 + (cc & 127)) * 2);
           }
 #pragma unroll
           for (int m = 0; m < kV; ++m) {
@@ -332,23 +343,51 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParam
         }
       }
       asm volatile("bar.sync 2, 256;" ::: "memory");
-      // (b) intra-step scores (q_t . k_j) gamma^(t-j), j <= t: thread (t, j)
-      {
-        const int t = wt >> 4, j = wt & 15;
-        float a = 0.f;
-        if (j <= t && t < p.Tn) {
-          const float4* qr = reinterpret_cast<const float4*>(qraw + t * p.dk);
-          const float4* kr = reinterpret_cast<const float4*>(kraw + j * p.dk);
-          float a0 = 0.f, a1 = 0.f;
-          for (int c4 = 0; c4 < p.dk / 4; c4 += 2) {
-            const float4 x0 = qr[c4], y0 = kr[c4 ^ (j & 7)];
-            const float4 x1 = qr[c4 + 1], y1 = kr[(c4 + 1) ^ (j & 7)];
-            a0 = fmaf(x0.x, y0.x, fmaf(x0.y, y0.y, fmaf(x0.z, y0.z, fmaf(x0.w, y0.w, a0))));
-            a1 = fmaf(x1.x, y1.x, fmaf(x1.y, y1.y, fmaf(x1.z, y1.z, fmaf(x1.w, y1.w, a1))));
-          }
-          a = (a0 + a1) * dg.pow(t - j);
+      if (wt == 0) {                                   // the q, k, v stage is read
+        mbar_arrive(&empty[qkv_it % kDtStages]);
+        mbar_arrive(&mma_done[qkv_it % kDtStages]);    // keeps that barrier's phases in step with the ring
+      }
+      // (b) intra-step scores (q_t . k_j) gamma^(t-j), j <= t, on the tensor
+      // cores (mma.sync m16n8k8, tf32: q and k are bf16 values, exact in tf32):
+      // warp w < 4 forms the 16 x 8 tile of keys 8 (w & 1).. over half of d_k
+      // (w >> 1); the second half's tile passes through att
+      if (w < 4) {
+        const int nt = w & 1, kh = w >> 1;
+        const int g = lane >> 2, tq = lane & 3;
+        const int jrow = 8 * nt + g;                    // key of this thread's B values
+        const float* qa = qraw + g * p.dk;
+        const float* qb = qraw + (g + 8) * p.dk;
+        const float* kr = kraw + jrow * p.dk;
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        const int kbeg = kh * (p.dk / 2), kend = kbeg + p.dk / 2;
+        for (int k0 = kbeg; k0 < kend; k0 += 8) {
+          const int c0 = k0 + tq, c1 = k0 + tq + 4;
+          const uint32_t a0 = __float_as_uint(qa[c0]), a1 = __float_as_uint(qb[c0]);
+          const uint32_t a2 = __float_as_uint(qa[c1]), a3 = __float_as_uint(qb[c1]);
+          const uint32_t b0 = __float_as_uint(kr[(((c0 >> 2) ^ (jrow & 7)) << 2) + (c0 & 3)]);
+          const uint32_t b1 = __float_as_uint(kr[(((c1 >> 2) ^ (jrow & 7)) << 2) + (c1 & 3)]);
+          asm volatile(
+              "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, "
+              "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+              : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+              : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
         }
-        att[wt] = a;
+        const int j0 = 8 * nt + 2 * tq;
+        if (kh == 1) {
+          att[g * kDtMaxT + j0] = c[0];
+          att[g * kDtMaxT + j0 + 1] = c[1];
+          att[(g + 8) * kDtMaxT + j0] = c[2];
+          att[(g + 8) * kDtMaxT + j0 + 1] = c[3];
+        }
+        asm volatile("bar.sync 5, 128;" ::: "memory");
+        if (kh == 0) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int t = g + 8 * (e >> 1), j = j0 + (e & 1);
+            const float x = c[e] + att[t * kDtMaxT + j];
+            att[t * kDtMaxT + j] = (j <= t && t < p.Tn) ? x * dg.pow(t - j) : 0.f;
+          }
+        }
       }
       // (c) the same elements rewritten in place as the MMA operand tiles:
       // q_t gamma^(t+1) (K-major, 16-byte atoms) and zeta_t k_t (MN-major,
@@ -450,12 +489,16 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const DecTcParam
           tmem_ld16(tmem + 256 + 16 * b + (static_cast<uint32_t>(32 * quad) << 16), ot);
           tmem_wait_ld();
           const int c = 128 * b + 32 * quad + lane;     // d_v column
+          float vj[kDtMaxT];                             // v_j[c], rows from Tn on are zero
+#pragma unroll
+          for (int j = 0; j < kDtMaxT; ++j)
+            vj[j] = *reinterpret_cast<const float*>(vb + (c >> 5) * kDtChunk + sw32_off(j, c));
 #pragma unroll
           for (int t = 0; t < kDtMaxT; ++t) {
             if (t >= p.Tn) break;
             float s = ot[t];
-            for (int j = 0; j <= t; ++j)
-              s = fmaf(att[t * kDtMaxT + j], *reinterpret_cast<const float*>(vb + (c >> 5) * kDtChunk + sw32_off(j, c)), s);
+#pragma unroll
+            for (int j = 0; j <= t; ++j) s = fmaf(att[t * kDtMaxT + j], vj[j], s);
             const size_t oi = ((static_cast<size_t>(n) * p.Tn + t) * p.H + h) * p.dv + c;
             if (p.o_bf16)
               static_cast<__nv_bfloat16*>(p.o)[oi] = __float2bfloat16_rn(s);
@@ -499,7 +542,8 @@ PFN_cuTensorMapEncodeTiled_v12000 dt_encode_fn() {
 
 bool decode_steps_tc_supported(int Tn, int dk, int dv) {
   return Tn >= 1 && Tn <= kDtMaxT && (dk == 128 || dk == 256) && dv % 128 == 0 &&
-         DtLayout(dk, dv).smem <= 232448;
+         DtLayout(dk, dv).smem <= 232448 &&
+         static_cast<uint32_t>(Tn * (2 * dk + dv) * 2) <= kDtStage;
 }
 
 // The tensor cores pay off once the 2 Tn FMAs per state element dominate the
@@ -526,6 +570,27 @@ cudaError_t launch_decode_steps_tc(const void* q, const void* k, const void* v, 
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorNotSupported;
+  // q, k: [N*Tn rows][H*dk] bf16, boxes of dk x Tn; v: [N*Tn][H*dv], boxes of 128 x Tn
+  CUtensorMap mQ, mK, mV;
+  {
+    const cuuint32_t one[2] = {1, 1};
+    cuuint64_t gq[2] = {static_cast<cuuint64_t>(H) * dk, static_cast<cuuint64_t>(N) * Tn};
+    cuuint64_t sq[1] = {static_cast<cuuint64_t>(H) * dk * 2};
+    cuuint32_t bq[2] = {static_cast<cuuint32_t>(dk), static_cast<cuuint32_t>(Tn)};
+    cuuint64_t gv[2] = {static_cast<cuuint64_t>(H) * dv, static_cast<cuuint64_t>(N) * Tn};
+    cuuint64_t sv[1] = {static_cast<cuuint64_t>(H) * dv * 2};
+    cuuint32_t bv[2] = {128, static_cast<cuuint32_t>(Tn)};
+    if (fn(&mQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), gq, sq, bq, one,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        fn(&mK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k), gq, sq, bq, one,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        fn(&mV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(v), gv, sv, bv, one,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+  }
   DecTcParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k = static_cast<const __nv_bfloat16*>(k);
@@ -548,7 +613,7 @@ cudaError_t launch_decode_steps_tc(const void* q, const void* k, const void* v, 
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const int grid = p.nitems < sms ? p.nitems : sms;
-  decode_multi_tc_kernel<<<grid, kDtThreads, smem, s>>>(mS, p);
+  decode_multi_tc_kernel<<<grid, kDtThreads, smem, s>>>(mS, mQ, mK, mV, p);
   return cudaGetLastError();
 }
 

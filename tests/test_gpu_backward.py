@@ -12,7 +12,9 @@ as a precision check: their computed MMA operands are fp16, unit roundoff
 span several chunks with ragged tails, chunk lengths of one token and longer
 than the sequence, the largest supported heads, gamma = 0 and gamma = 1, an
 initial state and an upstream state gradient, and packed sequences including
-empty ones.
+empty ones.  d_v = 512 (the 6.7B head shape) runs on the tensor cores only,
+with the two retentions that contract over d_v split into halves; it is
+checked at small sizes and on a sampled (sequence, head) pair at T = 8192.
 """
 
 import numpy as np
@@ -46,7 +48,7 @@ def _inputs(B, T, H, dk, dv, dtype, seed, with_state):
 def _tensor_core(dtype, dk, dv, gammas, with_dS):
     """Whether the call runs on the tensor-core path (the rule of the C ABI)."""
     heads = (64, 128, 256)
-    ok = dtype == "bf16" and dk in heads and dv in heads
+    ok = dtype == "bf16" and dk in heads and dv in heads + (512,)
     if with_dS:
         ok = ok and all(g == 0.0 or g >= 1e-6 for g in gammas)
     return ok
@@ -216,6 +218,64 @@ def test_backward_chunk_length_does_not_matter():
             assert_close(W.to_f64(x), W.to_f64(y), "f32", None, f"chunk {chunk}")
 
 
+@pytest.mark.parametrize("B,T,H,dk,chunk,with_state,use_dS", [
+    (2, 300, 2, 128, 256, True, True),     # several chunks and tiles, both state terms
+    (1, 700, 1, 256, 512, True, False),    # the 6.7B heads, 512-token chunks, ragged tail
+    (1, 1030, 2, 64, 128, False, True),    # 128-token chunks executed as 256
+])
+def test_backward_tensor_core_dv512(B, T, H, dk, chunk, with_state, use_dS):
+    """d_v = 512: dQ and dK run as two passes over the halves of d_v (the score
+    contracts over d_v), the second adding to the first; dV in one pass."""
+    dv = 512
+    q, k, v, do, S0, dS = _inputs(B, T, H, dk, dv, "bf16", seed=T + dk, with_state=True)
+    S0 = S0 if with_state else None
+    dS = dS if use_dS else None
+    gam = W.head_gammas(H)
+    assert _tensor_core("bf16", dk, dv, gam, use_dS)
+    ref = oracle.msr_backward(W.to_f64(q), W.to_f64(k), W.to_f64(v), gam, W.to_f64(do),
+                              None if S0 is None else S0.double().numpy(),
+                              None if dS is None else dS.double().numpy())
+    got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, chunk,
+                            state_in=None if S0 is None else S0.cuda(),
+                            d_state_out=None if dS is None else dS.cuda(), return_d_state=True)
+    _check(got, ref, H, f"tc dv512 T{T} dk{dk} C{chunk} dS={use_dS}", tc=True)
+
+
+def test_backward_tensor_core_dv512_packed():
+    lens = [300, 0, 1, 257, 64]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    Tt = int(cu[-1])
+    H, dk, dv, chunk = 2, 128, 512, 256
+    q, k, v, do, _, _ = _inputs(1, Tt, H, dk, dv, "bf16", seed=23, with_state=False)
+    g = torch.Generator().manual_seed(24)
+    S0 = torch.randn(len(lens), H, dk, dv, generator=g)
+    dS = torch.randn(len(lens), H, dk, dv, generator=g)
+    gam = W.head_gammas(H)
+    ref = oracle.msr_backward_varlen(W.to_f64(q), W.to_f64(k), W.to_f64(v), gam, W.to_f64(do),
+                                     cu, S0.double().numpy(), dS.double().numpy())
+    got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, chunk,
+                            cu_seqlens=torch.from_numpy(cu).cuda(), state_in=S0.cuda(),
+                            d_state_out=dS.cuda(), return_d_state=True)
+    _check(got, ref, H, "tc dv512 packed", tc=True)
+
+
+def test_backward_6p7b_heads_t8192_sampled():
+    """The 6.7B-shaped backward (B=2, T=8192, H=16, d_k=256, d_v=512, chunk 512)
+    in full on the GPU, against the oracle on one sampled (sequence, head)."""
+    B, T, H, dk, dv, C = 2, 8192, 16, 256, 512, 512
+    q, k, v, do, _, dS = _inputs(B, T, H, dk, dv, "bf16", seed=88, with_state=True)
+    gam = W.head_gammas(H)
+    got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, C,
+                            d_state_out=dS.cuda(), return_d_state=True)
+    b, h = 1, 15
+    ref = oracle.retention_backward(W.to_f64(q[b, :, h]), W.to_f64(k[b, :, h]),
+                                    W.to_f64(v[b, :, h]), gam[h], W.to_f64(do[b, :, h]),
+                                    None, dS[b, h].double().numpy())
+    for x, y, n in zip((got[0][b, :, h], got[1][b, :, h], got[2][b, :, h], got[3][b, h]), ref,
+                       ("dq", "dk", "dv", "d_state_in")):
+        assert_close(W.to_f64(x), y, "bf16", None, f"6.7B b{b} h{h} {n}")
+
+
 def test_backward_rejects_unsupported_and_bad_arguments():
     q = torch.zeros(1, 8, 1, 512, device="cuda")
     v = torch.zeros(1, 8, 1, 16, device="cuda")
@@ -224,6 +284,16 @@ def test_backward_rejects_unsupported_and_bad_arguments():
     assert ops.chunkwise_bwd_workspace_size(torch.float32, 4, 1, 8, 1, 512, 16) == 0
     assert ops.chunkwise_bwd_workspace_size(torch.float32, 0, 1, 8, 1, 16, 16) == 0
     assert ops.chunkwise_bwd_workspace_size(torch.float32, 4, 1, 8, 1, 16, 16) > 0
+    # d_v = 512: bf16 on the tensor cores only
+    assert ops.chunkwise_bwd_workspace_size(torch.bfloat16, 256, 1, 8, 1, 128, 512) > 0
+    assert ops.chunkwise_bwd_workspace_size(torch.float32, 256, 1, 8, 1, 128, 512) == 0
+    assert ops.chunkwise_bwd_workspace_size(torch.bfloat16, 256, 1, 8, 1, 16, 512) == 0
+    # a final-state gradient with a tiny gamma needs the CUDA cores, which d_v = 512 lacks
+    qb = torch.zeros(1, 8, 1, 128, device="cuda", dtype=torch.bfloat16)
+    vb = torch.zeros(1, 8, 1, 512, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(ops.RetentionError):
+        ops.chunkwise_bwd(qb, qb, vb, vb, [1e-7], 256,
+                          d_state_out=torch.zeros(1, 1, 128, 512, device="cuda"))
 
 
 @pytest.mark.parametrize("path", ["tensor_core", "tensor_core_dS", "cuda_core"])
