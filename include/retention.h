@@ -363,19 +363,18 @@ RET_API ret_status retention_recurrent_steps(const void* q, const void* k, const
  * and bf16 with dk in {64, 128, 256}, dv = 512 on the tensor cores.
  * Two paths, chosen per call:
  *   tensor cores: in_dtype RET_BF16 with dk in {64, 128, 256}, dv in {64, 128,
- *     256, 512}, a chunk of 64..512 and, when d_state_out is given, every
- *     gamma 0 or >= 1e-6.  The three gradients are three forward retentions
- *     with the operand roles exchanged (dK and dV on the sequences read
- *     backwards, dS_T entering as the initial state dS_T / gamma), on the
- *     forward's tcgen05 kernels with the forward's precision (fp16 operands,
- *     float32 accumulation).  With dv = 512 the dQ and dK retentions, whose
- *     scores contract over dv, each run as two passes over the halves of dv,
- *     the second adding to the first.  `chunk` only selects the layout, the
- *     kernels' own chunk is used.
+ *     256, 512} and a chunk of 64..512.  The three gradients are three
+ *     retentions with the operand roles exchanged, on the forward's tcgen05
+ *     kernels with the forward's precision (fp16 operands, float32
+ *     accumulation): dQ causal from S0^T; dV and dK anti-causal (the chunks
+ *     walked last to first, each carrying the state of everything after it),
+ *     started from dS_T and dS_T^T, the dV pass's final state being dS0.
+ *     With dv = 512 the dQ and dK retentions, whose scores contract over dv,
+ *     each run as two passes over the halves of dv, the second adding to the
+ *     first.  `chunk` only selects the layout, the kernels' own chunk is used.
  *   CUDA cores: every other supported case; every product and sum is float32
  *     (bf16 inputs are widened exactly).
- * Other heads (and dv = 512 where the tensor-core path cannot run) return
- * RET_ERR_UNSUPPORTED.  The workspace size query returns 0
+ * Other heads return RET_ERR_UNSUPPORTED.  The workspace size query returns 0
  * for arguments the call would reject, and otherwise the larger of the two
  * paths' needs.
  */

@@ -539,13 +539,7 @@ ret_status retention_chunkwise_bwd(const void* q, const void* k, const void* v, 
     if (ptr && !aligned16(ptr)) return RET_ERR_INVALID_ARG;
   ret::HeadDecay dec;
   if (!make_decay(gamma, H, &dec)) return RET_ERR_INVALID_ARG;
-  // a final-state gradient enters the tensor-core path as dS_T / gamma: every
-  // gamma must be 0 (handled apart) or not so small that the quotient overflows
-  bool gam_ok = true;
-  for (int h = 0; h < H; ++h)
-    if (gamma[h] != 0.0 && gamma[h] < 1e-6) gam_ok = false;
-  const bool use_tc = p.tc_ok && (d_state_out == nullptr || gam_ok);
-  if (!use_tc && !p.simt_ok) return RET_ERR_UNSUPPORTED;
+  const bool use_tc = p.tc_ok;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
       workspace_bytes < (use_tc ? p.tc_bytes : p.bytes))
     return RET_ERR_WORKSPACE;

@@ -136,6 +136,9 @@ struct StateParams {
   float* state_out;
   int H, dk, dv;
   int write_v16;                     // the CTAs of the first d_k block store the fp16 copy of v
+  // anti-causal mode: the chunks are walked last to first and each carries the
+  // state of everything after it, F_(c-1) = gamma^L F_c + sum_j gamma^(j+1) k_j^T v_j
+  int anti;
   HeadDecay dec;
   unsigned* err;
 };
@@ -193,6 +196,8 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
   seq_bounds(L, s, a, b);
   const int nch = ceil_div(b - a, L.chunk);
   const Decay1 dec(p.dec, h);
+  // the chunk taken c-th: chunk c, or chunk nch-1-c in the anti-causal mode
+  auto chunk_of = [&](int c) { return p.anti ? nch - 1 - c : c; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NSTG; ++i) {
@@ -236,7 +241,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       int it = 0;
       bool ok = true;
       for (int c = 0; c < nch && ok; ++c) {
-        const int tok0 = a + c * L.chunk;
+        const int tok0 = a + chunk_of(c) * L.chunk;
         const int Lc = min(L.chunk, b - tok0);
         for (int sb = 0; sb * kStTok < Lc; ++sb, ++it) {
           const int st = it % NSTG;
@@ -266,7 +271,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       int it = 0;
       bool ok = true, issued = false;
       for (int c = 0; c < nch && ok; ++c) {
-        const int Lc = min(L.chunk, b - (a + c * L.chunk));
+        const int Lc = min(L.chunk, b - (a + chunk_of(c) * L.chunk));
         const uint32_t acc = tmem + (c & 1) * NS;
         // this accumulator last held S_(c-2), which warpgroup A has read by now
         if (c > 0 && !mbar_wait(acc_free, (c - 1) & 1, abort_flag, p.err)) { ok = false; break; }
@@ -373,10 +378,10 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         tmem_st32(trow + NS + 32 * j, r);
       }
       tmem_wait_st();
-      stage_state(NS, slot_of(0));
+      stage_state(NS, slot_of(chunk_of(0)));
     }
     for (int c = 0; c < nch && ok; ++c) {
-      const int Lc = min(L.chunk, b - (a + c * L.chunk));
+      const int Lc = min(L.chunk, b - (a + chunk_of(c) * L.chunk));
       ok = wga_all(mbar_wait(acc_full, c & 1, abort_flag, p.err));
       if (!ok) break;
       tc_fence_after();
@@ -400,7 +405,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(acc_free);                     // accumulator pcol may take chunk c+1
-      if (c + 1 < nch) stage_state(dcol, slot_of(c + 1));
+      if (c + 1 < nch) stage_state(dcol, slot_of(chunk_of(c + 1)));
     }
     if (leader) tma_store_wait_all();
     if (!range_ok) raise_error(p.err, kErrRange);
@@ -437,16 +442,17 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     int it = 0;
     bool ok = !*abort_flag, range_ok = true;
     for (int c = 0; c < nch && ok; ++c) {
-      const int tok0 = a + c * L.chunk;
+      const int tok0 = a + chunk_of(c) * L.chunk;
       const int Lc = min(L.chunk, b - tok0);
       for (int sb = 0; sb * kStTok < Lc; ++sb, ++it) {
         const int st = it % NSTG;
         if (!mbar_wait(&full[st], (it / NSTG) & 1, abort_flag, p.err)) { ok = false; break; }
         uint8_t* stage = smem + st * kStage;
         if (k_mine) {
-          // zeta*K, pieces 4*khalf .. 4*khalf+3 of row krow%64 of box krow/64
+          // zeta*K, pieces 4*khalf .. 4*khalf+3 of row krow%64 of box krow/64:
+          // zeta_j = gamma^(L-1-j), or gamma^(j+1) in the anti-causal mode
           const int jtok = sb * kStTok + (krow & 63);
-          const float z = jtok < Lc ? dec.pow(Lc - 1 - jtok) : 0.f;
+          const float z = jtok < Lc ? dec.pow(p.anti ? jtok + 1 : Lc - 1 - jtok) : 0.f;
           uint4* rp = reinterpret_cast<uint4*>(stage + (krow >> 6) * kBox + (krow & 63) * 128);
           const int sw = krow & 7;
           uint4 w4[4];
@@ -505,7 +511,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       int it = 0;
       bool ok = true;
       for (int c = 0; c < nch && ok; ++c) {
-        const int tok0 = a + c * L.chunk;
+        const int tok0 = a + chunk_of(c) * L.chunk;
         const int Lc = min(L.chunk, b - tok0);
         for (int sb = 0; sb * kStTok < Lc; ++sb, ++it) {
           const int st = it % NSTG;
@@ -550,6 +556,9 @@ struct OutParams {
   int g_tma;                   // gate tile streamed by TMA (bf16 gate)
   int y_tma;                   // full output tiles written by TMA (bf16 output)
   int acc_out;                 // float32 output, ungated: out += o instead of out = o
+  // anti-causal mode: o_i = sum_{j >= i} gamma^(j-i) (q_i . k_j) v_j + gamma^(L-1-i) q_i F,
+  // F the state of everything after the chunk (the state pass's anti-causal walk)
+  int anti;
   int H, dk, dv;
   int rb;                      // 128-row blocks per chunk
   int parts;                   // d_v parts (cluster size)
@@ -596,6 +605,7 @@ struct OutTile {
   SeqInfo si;
   long long slot;
   int h, r, t0, nrows;
+  int kb0, nkb;                // key blocks kb0 .. kb0+nkb-1 (0..r causal, r..last anti-causal)
   bool inter;                  // reads the state carried into the chunk
 };
 
@@ -620,7 +630,9 @@ struct TileWalk {
       const unsigned gh = static_cast<unsigned>(u) / static_cast<unsigned>(p.rb);
       const unsigned slot = gh / static_cast<unsigned>(p.H);
       t.h = static_cast<int>(gh - slot * static_cast<unsigned>(p.H));
-      t.r = p.rb - 1 - static_cast<int>(static_cast<unsigned>(u) - gh * static_cast<unsigned>(p.rb));
+      // heaviest row block first: the last one (causal) or the first (anti-causal)
+      const int rr = static_cast<int>(static_cast<unsigned>(u) - gh * static_cast<unsigned>(p.rb));
+      t.r = p.anti ? rr : p.rb - 1 - rr;
       t.slot = slot;
       if (p.L.cu == nullptr) {
         const unsigned sq = slot / static_cast<unsigned>(p.nch);
@@ -638,7 +650,15 @@ struct TileWalk {
       if (t.r * kRowsPerTile >= t.si.len) continue;
       t.t0 = t.si.cs + t.r * kRowsPerTile;
       t.nrows = min(kRowsPerTile, t.si.len - t.r * kRowsPerTile);
-      t.inter = t.si.c > 0 || p.has_state_in;
+      if (p.anti) {
+        t.kb0 = t.r;
+        t.nkb = (t.si.len + kKeysPerBlock - 1) / kKeysPerBlock - t.r;
+        t.inter = t.si.cs + t.si.len < t.si.b || p.has_state_in;   // a later chunk, or a state in
+      } else {
+        t.kb0 = 0;
+        t.nkb = t.r + 1;
+        t.inter = t.si.c > 0 || p.has_state_in;
+      }
       return true;
     }
   }
@@ -702,7 +722,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   constexpr int kBoxesPerStage = static_cast<int>(kOutStage / kTallBox);
   // ring units of one tile before its gate stages
   auto tile_units = [&](const OutTile& tt) {
-    return (tt.r + 1) * (kKU + 2) + (tt.inter ? DK / 64 : 0);
+    return tt.nkb * (kKU + 2) + (tt.inter ? DK / 64 : 0);
   };
   auto io_staged = [&](const OutTile& t) {
     return (p.gated && p.g_tma) || (p.y_tma && t.nrows == kRowsPerTile);
@@ -769,7 +789,6 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         return smem + C::kOffStages + st * kOutStage;
       };
       while (ok && walk.next(p, cid, t)) {
-        const int r = t.r;
         // Q of this tile, once the previous tile's MMAs and epilogue are done with Q
         if (tq > 0 && !mbar_wait(q_free, (tq - 1) & 1, abort_flag, p.err)) { ok = false; break; }
         mbar_arrive_expect_tx(bar_q, C::kQBytes);
@@ -796,10 +815,10 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             ++it;
           }
         };
-        load_k(0);
-        for (int kb = 0; kb <= r && ok; ++kb) {
-          if (kb + 1 <= r) load_k(kb + 1);
-          load_v(kb);
+        load_k(t.kb0);
+        for (int kk = 0; kk < t.nkb && ok; ++kk) {
+          if (kk + 1 < t.nkb) load_k(t.kb0 + kk + 1);
+          load_v(t.kb0 + kk);
         }
         if (ok && t.inter) {
           for (int u = 0; u < DK / 64 && ok; ++u) {
@@ -861,10 +880,9 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         ++it;
       };
       while (ok && walk.next(p, cid, t)) {
-        const int r = t.r;
         if (!mbar_wait(bar_q, tq & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
-        auto issue_qk = [&](int kb) -> bool {
+        auto issue_qk = [&](int kb) -> bool {          // kb: the tile's kb-th key block
           const uint32_t dst = sbuf0 + 128 * (kb & 1);
           for (int ku = 0; ku < kKU; ++ku) {
             const uint32_t sb = stage_wait();
@@ -880,12 +898,12 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             stage_free();
           }
           mma_commit(&bar_s[(sblk + kb) & 1]);
-          if (kb == r) mma_commit(q_free);     // the MMAs are done with Q
+          if (kb == t.nkb - 1) mma_commit(q_free);     // the MMAs are done with Q
           return true;
         };
         if (!issue_qk(0)) { ok = false; break; }
-        if (r >= 1 && !issue_qk(1)) { ok = false; break; }
-        for (int kb = 0; kb <= r && ok; ++kb) {
+        if (t.nkb >= 2 && !issue_qk(1)) { ok = false; break; }
+        for (int kb = 0; kb < t.nkb && ok; ++kb) {
           const int sg = sblk + kb;
           if (!mbar_wait(&bar_p[sg & 1], (sg >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
           tc_fence_after();
@@ -905,7 +923,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           mma_commit(&pv_done[sg & 1]);
           // the next scores go to the buffer this P V has just been issued from
           // (tcgen05 MMAs of one thread execute in issue order)
-          if (kb + 2 <= r && !issue_qk(kb + 2)) { ok = false; break; }
+          if (kb + 2 < t.nkb && !issue_qk(kb + 2)) { ok = false; break; }
         }
         if (!ok) break;
         if (t.inter) {
@@ -914,7 +932,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           if (!mbar_wait(bar_pp, npp & 1, abort_flag, p.err)) { ok = false; break; }
           ++npp;
           tc_fence_after();
-          const uint32_t abuf = sbuf0 + 128 * ((r + 1) & 1);
+          const uint32_t abuf = sbuf0 + 128 * (t.nkb & 1);
           for (int u = 0; u < DK / 64 && ok; ++u) {
             const uint32_t sb = stage_wait();
             if (!sb) { ok = false; break; }
@@ -928,7 +946,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
         mma_commit(bar_o);
         if (io_staged(t)) it += kGS;           // the gate stages belong to the epilogue
-        sblk += r + 1;
+        sblk += t.nkb;
         ++tq;
       }
       if (!ok && issued) {
@@ -970,25 +988,42 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       // epilogue thread passed the barrier in epi_all above after forming it)
       if (et < 128) pow_tab[et] = dec.pow(et);
       wg2_sync();
-      for (int kb = 0; kb <= r && ok; ++kb) {
-        const int sg = sblk + kb;
+      for (int kk = 0; kk < t.nkb && ok; ++kk) {
+        const int kb = t.kb0 + kk;                       // key block within the chunk
+        const int sg = sblk + kk;
         if (!warp_all(mbar_wait(&bar_s[sg & 1], (sg >> 1) & 1, abort_flag, p.err))) { ok = false; break; }
         tc_fence_after();
         const bool diag = kb == r;
-        // off-diagonal: gamma^(i-j) = gamma^(i - 128kb - 127) * gamma^(127 - j')
-        const float arow = diag ? 0.f : dec.pow(i - kKeysPerBlock * kb - 127);
+        // off-diagonal: gamma^(i-j) = gamma^(i - 128kb - 127) * gamma^(127 - j'), or in
+        // the anti-causal mode gamma^(j-i) = gamma^(128kb - i) * gamma^(j')
+        const float arow = diag ? 0.f
+                                : dec.pow(p.anti ? kKeysPerBlock * kb - i : i - kKeysPerBlock * kb - 127);
         const int key_lim = t.si.len - kKeysPerBlock * kb;   // keys j' >= key_lim are past the chunk
-        const uint32_t buf = sbuf0 + 128 * (kb & 1);
+        const uint32_t buf = sbuf0 + 128 * (kk & 1);
 #pragma unroll 1
         for (int j = 2 * wg; j < 2 * wg + 2; ++j) {
           float x[32];
           tmem_ld32(buf + 32 * j, x);
           float wv[32];
-          if (diag) {
+          if (diag && p.anti) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int jp = 32 * j + e;
+              wv[e] = jp >= row ? pow_tab[jp - row] : 0.f;
+            }
+          } else if (diag) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const int jp = 32 * j + e;
               wv[e] = jp <= row ? pow_tab[row - jp] : 0.f;
+            }
+          } else if (p.anti) {
+            // gamma^(32j + e), read as float4 from the table in ascending order
+#pragma unroll
+            for (int m4 = 0; m4 < 8; ++m4) {
+              const float4 t4 = *reinterpret_cast<const float4*>(pow_tab + 32 * j + 4 * m4);
+              wv[4 * m4] = t4.x * arow; wv[4 * m4 + 1] = t4.y * arow;
+              wv[4 * m4 + 2] = t4.z * arow; wv[4 * m4 + 3] = t4.w * arow;
             }
           } else {
             // gamma^(127 - 32j - e), read as float4 from the table in descending order
@@ -1024,8 +1059,8 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       if (t.inter && ok) {
         // the decayed query rows gamma^(i+1) q_i (fp16) into the score buffer
         // after the last one used, once the P V MMAs that read it are done
-        if (r >= 1) {
-          const int sg = sblk + r - 1;
+        if (t.nkb >= 2) {
+          const int sg = sblk + t.nkb - 2;
           ok = warp_all(mbar_wait(&pv_done[sg & 1], (sg >> 1) & 1, abort_flag, p.err));
           if (ok) tc_fence_after();
         }
@@ -1033,9 +1068,10 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         // reloaded before this thread releases it through q_free)
         if (ok) ok = warp_all(mbar_wait(bar_q, tq & 1, abort_flag, p.err));
         if (ok) {
-          const float sc = dec.pow(i + 1);
+          // gamma^(i+1), or gamma^(L-1-i) in the anti-causal mode (rows past the chunk: 0)
+          const float sc = p.anti ? (i < t.si.len ? dec.pow(t.si.len - 1 - i) : 0.f) : dec.pow(i + 1);
           const uint64_t sc2 = f2_make(sc, sc);
-          const uint32_t abuf = sbuf0 + 128 * ((r + 1) & 1);
+          const uint32_t abuf = sbuf0 + 128 * (t.nkb & 1);
           // this warpgroup's d_k columns: half-box pieces of 32 values
 #pragma unroll 1
           for (int c0 = wg * (DK / 2); c0 < (wg + 1) * (DK / 2); c0 += 32) {
@@ -1061,7 +1097,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_arrive(bar_pp);
       }
       mbar_arrive(q_free);                             // this thread is done reading Q
-      sblk += r + 1;
+      sblk += t.nkb;
       ok = warp_all(ok && mbar_wait(bar_o, tq & 1, abort_flag, p.err));
       if (ok) tc_fence_after();
       // GroupNorm statistics in one pass: sums of (x - x0) and (x - x0)^2 with
@@ -1964,7 +2000,7 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
                                DType g_t, const float* gn_w, const float* gn_b, float eps,
                                bool gated, ChunkWorkspace ws, int H, int dk, int dv,
                                const HeadDecay& dec, unsigned* err, cudaStream_t s,
-                               bool acc_out);
+                               bool acc_out, bool anti);
 
 }  // namespace
 
@@ -1996,7 +2032,7 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
                                 DType g_t, const float* gn_w, const float* gn_b, float eps,
                                 bool gated, ChunkWorkspace ws, int H, int dk, int dv,
                                 const HeadDecay& dec, unsigned* err, cudaStream_t s,
-                                bool acc_out) {
+                                bool acc_out, bool anti) {
   if (!chunkwise_tc_supported(dk, dv, L.chunk)) return cudaErrorNotSupported;
   const uint64_t Ttot = static_cast<uint64_t>(L.Ttot > 0 ? L.Ttot : 1);
   cudaError_t e = cudaSuccess;
@@ -2016,6 +2052,7 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
     sp.state_in = state_in;
     sp.state_out = state_out;
     sp.write_v16 = ws.v16 != nullptr ? 1 : 0;
+    sp.anti = anti ? 1 : 0;
     sp.H = H;
     sp.dk = dk;
     sp.dv = dv;
@@ -2038,7 +2075,7 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
   }
   if (e != cudaSuccess || L.Ttot == 0 || !(phases & 2)) return e;
   return launch_output_pass(q, k, L, has_state_in, out, out_t, g, g_t, gn_w, gn_b, eps, gated,
-                            ws, H, dk, dv, dec, err, s, acc_out);
+                            ws, H, dk, dv, dec, err, s, acc_out, anti);
 }
 
 namespace {
@@ -2053,11 +2090,10 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
                                DType g_t, const float* gn_w, const float* gn_b, float eps,
                                bool gated, ChunkWorkspace ws, int H, int dk, int dv,
                                const HeadDecay& dec, unsigned* err, cudaStream_t s,
-                               bool acc_out) {
+                               bool acc_out, bool anti) {
   if (L.chunk < kRowsPerTile || L.chunk % kRowsPerTile != 0) return cudaErrorInvalidValue;
-  // accumulation: float32, ungated, and only in the persistent kernel (multi-block chunks)
-  if (acc_out && (out_t != DType::F32 || gated || L.chunk == kRowsPerTile))
-    return cudaErrorInvalidValue;
+  // accumulation: float32 and ungated (the persistent kernel)
+  if (acc_out && (out_t != DType::F32 || gated)) return cudaErrorInvalidValue;
   const uint64_t Ttot = static_cast<uint64_t>(L.Ttot > 0 ? L.Ttot : 1);
   const int NV = dv > 256 ? 256 : dv;
   OutParams op;
@@ -2082,6 +2118,7 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
   op.g_tma = (gated && g_t == DType::BF16) ? 1 : 0;
   op.y_tma = out_t == DType::BF16 ? 1 : 0;
   op.acc_out = acc_out ? 1 : 0;
+  op.anti = anti ? 1 : 0;
   if (ws.v16 == nullptr) return cudaErrorInvalidValue;   // written by the state pass
   const uint64_t srows = static_cast<uint64_t>(ws.nslots) * H * dk;      // fp16 state slots
   const uint64_t hdv = static_cast<uint64_t>(H) * dv;
@@ -2103,7 +2140,8 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
   op.nch = (L.T + L.chunk - 1) / L.chunk;
   op.nclusters = 1;
   op.shift = 1;
-  if (op.rb == 1 && dk <= 128 && dv <= 256) {
+  // the compact kernel has neither the anti-causal mode nor accumulation
+  if (op.rb == 1 && dk <= 128 && dv <= 256 && !anti && !acc_out) {
     // one-block chunks: the compact kernel, two CTAs per SM, d_v in parts of <= 128
     op.parts = dv > 128 ? 2 : 1;
     const int NVc = dv / op.parts;
@@ -2182,7 +2220,7 @@ cudaError_t launch_parallel_tc(const void* q, const void* k, const void* v, void
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_output_pass(q, k, L, false, o, o_t, nullptr, DType::BF16, nullptr, nullptr, 0.f,
-                            false, ws, H, dk, dv, dec, err, s, false);
+                            false, ws, H, dk, dv, dec, err, s, false, false);
 }
 
 }  // namespace ret

@@ -123,7 +123,7 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
                                 const float* gn_w, const float* gn_b, float eps, bool gated,
                                 ChunkWorkspace ws, int H, int dk, int dv,
                                 const HeadDecay& dec, unsigned* err, cudaStream_t s,
-                                bool acc_out = false);
+                                bool acc_out = false, bool anti = false);
 
 // Parallel form on the tensor cores (bf16 inputs): an fp16 copy of v, then the
 // chunkwise output kernel with each sequence as a single chunk.

@@ -4,9 +4,9 @@ fp64 oracle's gradients, through the C ABI.
 On the CUDA-core path the kernels compute every product and sum in float32
 from inputs that are exact (float32, or bfloat16 widened exactly), so both
 input dtypes are held to the float32 tolerance: relative L2 <= 1e-5 over each
-gradient, whole and per head.  bf16 inputs with heads of 64/128/256 (and, with
-a final-state gradient, every gamma 0 or >= 1e-6) run on the tensor-core
-kernels instead and are held to the bf16-input tolerance (plus rel-L2 <= 1e-3
+gradient, whole and per head.  bf16 inputs with d_k in 64/128/256 and d_v in
+64/128/256/512 run on the tensor-core kernels instead (the causal and
+anti-causal forward retentions) and are held to the bf16-input tolerance (plus rel-L2 <= 1e-3
 as a precision check: their computed MMA operands are fp16, unit roundoff
 2^-11, which gives ~3e-4; operands rounded to bf16 alone would give ~2e-3).  Cases
 span several chunks with ragged tails, chunk lengths of one token and longer
@@ -48,10 +48,7 @@ def _inputs(B, T, H, dk, dv, dtype, seed, with_state):
 def _tensor_core(dtype, dk, dv, gammas, with_dS):
     """Whether the call runs on the tensor-core path (the rule of the C ABI)."""
     heads = (64, 128, 256)
-    ok = dtype == "bf16" and dk in heads and dv in heads + (512,)
-    if with_dS:
-        ok = ok and all(g == 0.0 or g >= 1e-6 for g in gammas)
-    return ok
+    return dtype == "bf16" and dk in heads and dv in heads + (512,)
 
 
 def _check(got, ref, H, what, tc=False):
@@ -97,9 +94,9 @@ def test_backward_matches_oracle(dtype, B, T, H, dk, dv, chunk, with_state):
 @pytest.mark.parametrize("use_dS", [False, True])
 def test_backward_tensor_core_path(B, T, H, dk, dv, chunk, with_state, use_dS):
     """bf16 inputs with heads of 64/128/256 run on the tensor-core forward kernels
-    (three retentions, two on reversed sequences; a final-state gradient enters
-    them as the initial state dS_T / gamma); held to the bf16-input tolerance
-    and, as a precision check, rel-L2 <= 1e-3."""
+    (three retentions: dQ causal, dV and dK anti-causal, a final-state gradient
+    entering those two as the state after the last chunk); held to the
+    bf16-input tolerance and, as a precision check, rel-L2 <= 1e-3."""
     q, k, v, do, S0, dS = _inputs(B, T, H, dk, dv, "bf16", seed=T + 3 * dk, with_state=True)
     S0 = S0 if with_state else None
     dS = dS if use_dS else None
@@ -116,8 +113,9 @@ def test_backward_tensor_core_path(B, T, H, dk, dv, chunk, with_state, use_dS):
 
 @pytest.mark.parametrize("use_dS", [False, True])
 def test_backward_tensor_core_packed(use_dS):
-    """The tensor-core path on packed sequences (reversal inside each sequence;
-    an empty sequence passes dS_T straight to its initial-state gradient)."""
+    """The tensor-core path on packed sequences (the anti-causal walk runs inside
+    each sequence; an empty sequence passes dS_T straight to its initial-state
+    gradient)."""
     lens = [300, 0, 1, 129, 64]
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     Tt = int(cu[-1])
@@ -158,18 +156,20 @@ def test_backward_tensor_core_zero_and_unit_decay(gammas):
     _check(got, ref, H, f"tc gammas {gammas}", tc=True)
 
 
-def test_backward_tiny_decay_with_state_gradient_uses_cuda_cores():
-    """A gamma in (0, 1e-6) with a final-state gradient would overflow dS_T / gamma
-    on the tensor-core path; such calls run on CUDA cores (float32 tolerance)."""
-    B, T, H, dk, dv, chunk = 1, 150, 2, 64, 64, 64
+@pytest.mark.parametrize("dv", [64, 512])
+def test_backward_tiny_decay_with_state_gradient(dv):
+    """A gamma far below any that decays over one chunk, with a final-state
+    gradient: the anti-causal passes start from dS_T itself, so nothing is
+    divided by gamma (the state gradient reaches the last tokens only)."""
+    B, T, H, dk, chunk = 1, 150, 2, 64, 64
     q, k, v, do, S0, dS = _inputs(B, T, H, dk, dv, "bf16", seed=41, with_state=True)
     gam = [1e-7, 0.9]
-    assert not _tensor_core("bf16", dk, dv, gam, True)
+    assert _tensor_core("bf16", dk, dv, gam, True)
     ref = oracle.msr_backward(W.to_f64(q), W.to_f64(k), W.to_f64(v), gam, W.to_f64(do),
                               S0.double().numpy(), dS.double().numpy())
     got = ops.chunkwise_bwd(q.cuda(), k.cuda(), v.cuda(), do.cuda(), gam, chunk,
                             state_in=S0.cuda(), d_state_out=dS.cuda(), return_d_state=True)
-    _check(got, ref, H, "tiny gamma")
+    _check(got, ref, H, f"tiny gamma dv{dv}", tc=True)
 
 
 @pytest.mark.parametrize("gammas", [[0.0, 1.0], [1.0, 0.5]])
@@ -288,12 +288,6 @@ def test_backward_rejects_unsupported_and_bad_arguments():
     assert ops.chunkwise_bwd_workspace_size(torch.bfloat16, 256, 1, 8, 1, 128, 512) > 0
     assert ops.chunkwise_bwd_workspace_size(torch.float32, 256, 1, 8, 1, 128, 512) == 0
     assert ops.chunkwise_bwd_workspace_size(torch.bfloat16, 256, 1, 8, 1, 16, 512) == 0
-    # a final-state gradient with a tiny gamma needs the CUDA cores, which d_v = 512 lacks
-    qb = torch.zeros(1, 8, 1, 128, device="cuda", dtype=torch.bfloat16)
-    vb = torch.zeros(1, 8, 1, 512, device="cuda", dtype=torch.bfloat16)
-    with pytest.raises(ops.RetentionError):
-        ops.chunkwise_bwd(qb, qb, vb, vb, [1e-7], 256,
-                          d_state_out=torch.zeros(1, 1, 128, 512, device="cuda"))
 
 
 @pytest.mark.parametrize("path", ["tensor_core", "tensor_core_dS", "cuda_core"])
