@@ -11,6 +11,9 @@
 //          = anti-causal(q = V, k = dO, v = Q, state in = dS_T^T)
 //     dS0  = sum_n gamma^(n+1) q_n^T dO_n + gamma^T dS_T
 //          = the final state of the anti-causal (Q, dO) pass.
+// The dK pass's state, sum gamma^(j+1) dO_j^T q_j, is the transpose of the dV
+// pass's: it runs no state pass of its own and reads the dV pass's state slots
+// transposed (K-major), with an fp16 copy of Q as its value operand.
 // The anti-causal retention walks the chunks last to first carrying the state
 // of everything after each chunk, F_(c-1) = gamma^L F_c + sum_j gamma^(j+1)
 // k_j^T v_j, and reads it as gamma^(L-1-i) q_i F_c; started from dS_T it
@@ -154,7 +157,7 @@ size_t chunkwise_bwd_tc_scratch_bytes(const SeqLayout& L, int H, int dk, int dv)
   const size_t T = static_cast<size_t>(L.Ttot);
   auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
   const size_t st = r256(static_cast<size_t>(L.nseq) * H * dk * dv * 4);
-  size_t b = 2 * st;                                     // S0^T and dS_T^T (each split in d_v halves)
+  size_t b = st;                                         // S0^T (split in d_v halves)
   if (dv > 256) b += 4 * r256(T * H * (dv / 2) * 2);     // the d_v halves of dO and V
   return b;
 }
@@ -174,10 +177,8 @@ cudaError_t launch_chunkwise_bwd_tc(const void* q, const void* k, const void* v,
   char* p = static_cast<char*>(scratch);
   const size_t st_bytes = r256(static_cast<size_t>(L.nseq) * H * dk_ * dv_ * 4);
   float* s0t = reinterpret_cast<float*>(p); p += st_bytes;   // S0^T   [dv][dk] (split: 2 x [hd][dk])
-  float* dst = reinterpret_cast<float*>(p); p += st_bytes;   // dS_T^T, split the same way
   const size_t half_st = static_cast<size_t>(L.nseq) * H * hd * dk_;   // floats per half
   float* s0t_h[2] = {s0t, s0t + half_st};
-  float* dst_h[2] = {dst, dst + half_st};
   const void* doh[2] = {d_out, nullptr};
   const void* vh[2] = {v, nullptr};
   cudaError_t e = cudaSuccess;
@@ -194,8 +195,6 @@ cudaError_t launch_chunkwise_bwd_tc(const void* q, const void* k, const void* v,
   const int nmat = L.nseq * H;
   if (e == cudaSuccess && state_in)
     e = transpose_split(state_in, s0t_h[0], s0t_h[1], nmat, dk_, dv_, hd, s);
-  if (e == cudaSuccess && d_state_out)
-    e = transpose_split(d_state_out, dst_h[0], dst_h[1], nmat, dk_, dv_, hd, s);
   if (e != cudaSuccess) return e;
   const DType F = DType::F32;
   const bool ds = d_state_out != nullptr;
@@ -219,11 +218,19 @@ cudaError_t launch_chunkwise_bwd_tc(const void* q, const void* k, const void* v,
       e = cudaGetLastError();
     }
   }
-  // dK: anti-causal(q = V, k = dO, v = Q) from dS_T^T (per d_v half, summed)
-  for (int i = 0; i < nh && e == cudaSuccess; ++i)
-    e = launch_chunkwise_tc(3, vh[i], doh[i], q, L, ds ? dst_h[i] : nullptr, ds, nullptr, dk, F,
-                            nullptr, F, nullptr, nullptr, 0.f, false, ws, H, hd, dk_, dec, err, s,
-                            i > 0, true);
+  // dK: anti-causal(q = V, k = dO, v = Q) on the dV pass's states read
+  // transposed (they start from dS_T, so the last chunk reads dS_T^T), its value
+  // operand the fp16 copy of Q; per d_v half, summed
+  if (e == cudaSuccess) e = launch_to_f16(q, ws.v16, static_cast<long long>(T) * H * dk_, err, s);
+  for (int i = 0; i < nh && e == cudaSuccess; ++i) {
+    StateRead sr;
+    sr.transposed = true;
+    sr.col0 = i * hd;
+    sr.stored_dv = dv_;
+    e = launch_chunkwise_tc(2, vh[i], doh[i], q, L, nullptr, ds, nullptr, dk, F, nullptr, F,
+                            nullptr, nullptr, 0.f, false, ws, H, hd, dk_, dec, err, s, i > 0, true,
+                            sr);
+  }
   return e;
 }
 

@@ -559,6 +559,10 @@ struct OutParams {
   // anti-causal mode: o_i = sum_{j >= i} gamma^(j-i) (q_i . k_j) v_j + gamma^(L-1-i) q_i F,
   // F the state of everything after the chunk (the state pass's anti-causal walk)
   int anti;
+  // the carried state read transposed (s_kmajor): the slots hold another
+  // pass's state [dv rows][stored columns]; this pass multiplies by the
+  // columns s_col0 .. s_col0+dk-1 of it, as a K-major operand
+  int s_kmajor, s_col0;
   int H, dk, dv;
   int rb;                      // 128-row blocks per chunk
   int parts;                   // d_v parts (cluster size)
@@ -822,11 +826,17 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
         if (ok && t.inter) {
           for (int u = 0; u < DK / 64 && ok; ++u) {
-            const int srow = static_cast<int>((t.slot * p.H + t.h) * DK) + 64 * u;
             uint8_t* dst = next((NV / 64) * kBox);
             if (!dst) { ok = false; break; }
-            for (int bx = 0; bx < NV / 64; ++bx)
-              tma_load_2d(dst + bx * kBox, &tmS, &full[it % NST], NV * part + 64 * bx, srow);
+            if (p.s_kmajor) {
+              // 64 state rows of this pass = 64 columns of the stored state, all NV of its rows
+              tma_load_2d(dst, &tmS, &full[it % NST], p.s_col0 + 64 * u,
+                          static_cast<int>((t.slot * p.H + t.h) * NV));
+            } else {
+              const int srow = static_cast<int>((t.slot * p.H + t.h) * DK) + 64 * u;
+              for (int bx = 0; bx < NV / 64; ++bx)
+                tma_load_2d(dst + bx * kBox, &tmS, &full[it % NST], NV * part + 64 * bx, srow);
+            }
             ++it;
           }
         }
@@ -864,6 +874,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (lane == 0 && !*abort_flag) {
       constexpr uint32_t id_qk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t id_pv = idesc_f16_f32(128, NV, false, true);
+      constexpr uint32_t id_qs_k = idesc_f16_f32(128, NV, false, false);   // K-major state
       const uint32_t q_base = smem_u32(smem);
       const uint32_t st_base = smem_u32(smem + C::kOffStages);
       const uint32_t sbuf0 = tmem + C::kColSB;
@@ -936,10 +947,17 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           for (int u = 0; u < DK / 64 && ok; ++u) {
             const uint32_t sb = stage_wait();
             if (!sb) { ok = false; break; }
+            if (p.s_kmajor) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ts(tmem, abuf + 32 * u + 8 * kk, sdesc_sw128(sb + kk * 2048, kBox, 1024),
-                          id_pv, true);
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ts(tmem, abuf + 32 * u + 8 * kk, sdesc_sw128(sb + kk * 32, 16, 1024),
+                            id_qs_k, true);
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ts(tmem, abuf + 32 * u + 8 * kk, sdesc_sw128(sb + kk * 2048, kBox, 1024),
+                            id_pv, true);
+            }
             stage_free();
           }
           if (!ok) break;
@@ -2000,7 +2018,7 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
                                DType g_t, const float* gn_w, const float* gn_b, float eps,
                                bool gated, ChunkWorkspace ws, int H, int dk, int dv,
                                const HeadDecay& dec, unsigned* err, cudaStream_t s,
-                               bool acc_out, bool anti);
+                               bool acc_out, bool anti, StateRead sr);
 
 }  // namespace
 
@@ -2032,7 +2050,7 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
                                 DType g_t, const float* gn_w, const float* gn_b, float eps,
                                 bool gated, ChunkWorkspace ws, int H, int dk, int dv,
                                 const HeadDecay& dec, unsigned* err, cudaStream_t s,
-                                bool acc_out, bool anti) {
+                                bool acc_out, bool anti, StateRead sr) {
   if (!chunkwise_tc_supported(dk, dv, L.chunk)) return cudaErrorNotSupported;
   const uint64_t Ttot = static_cast<uint64_t>(L.Ttot > 0 ? L.Ttot : 1);
   cudaError_t e = cudaSuccess;
@@ -2075,7 +2093,7 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
   }
   if (e != cudaSuccess || L.Ttot == 0 || !(phases & 2)) return e;
   return launch_output_pass(q, k, L, has_state_in, out, out_t, g, g_t, gn_w, gn_b, eps, gated,
-                            ws, H, dk, dv, dec, err, s, acc_out, anti);
+                            ws, H, dk, dv, dec, err, s, acc_out, anti, sr);
 }
 
 namespace {
@@ -2090,7 +2108,7 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
                                DType g_t, const float* gn_w, const float* gn_b, float eps,
                                bool gated, ChunkWorkspace ws, int H, int dk, int dv,
                                const HeadDecay& dec, unsigned* err, cudaStream_t s,
-                               bool acc_out, bool anti) {
+                               bool acc_out, bool anti, StateRead sr) {
   if (L.chunk < kRowsPerTile || L.chunk % kRowsPerTile != 0) return cudaErrorInvalidValue;
   // accumulation: float32 and ungated (the persistent kernel)
   if (acc_out && (out_t != DType::F32 || gated)) return cudaErrorInvalidValue;
@@ -2119,14 +2137,21 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
   op.y_tma = out_t == DType::BF16 ? 1 : 0;
   op.acc_out = acc_out ? 1 : 0;
   op.anti = anti ? 1 : 0;
+  op.s_kmajor = sr.transposed ? 1 : 0;
+  op.s_col0 = sr.col0;
   if (ws.v16 == nullptr) return cudaErrorInvalidValue;   // written by the state pass
-  const uint64_t srows = static_cast<uint64_t>(ws.nslots) * H * dk;      // fp16 state slots
+  // a transposed read: the slots hold [dv rows][stored_dv] (dv <= 256, one part)
+  if (sr.transposed && (dv > 256 || sr.col0 < 0 || sr.col0 % 64 != 0 || sr.col0 + dk > sr.stored_dv))
+    return cudaErrorInvalidValue;
   const uint64_t hdv = static_cast<uint64_t>(H) * dv;
   CUtensorMap mq, mk, mv, ms, mg, my;
+  const bool s_ok = sr.transposed
+      ? make_map(&ms, ws.states, sr.stored_dv, static_cast<uint64_t>(ws.nslots) * H * dv,
+                 sr.stored_dv, static_cast<uint32_t>(NV), true)
+      : make_map(&ms, ws.states, dv, static_cast<uint64_t>(ws.nslots) * H * dk, dv, 64, true);
   if (!make_map(&mq, q, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 128) ||
       !make_map(&mk, k, static_cast<uint64_t>(H) * dk, Ttot, static_cast<uint64_t>(H) * dk, 128) ||
-      !make_map(&mv, ws.v16, hdv, Ttot, hdv, 64, true) ||
-      !make_map(&ms, ws.states, dv, srows, dv, 64, true))
+      !make_map(&mv, ws.v16, hdv, Ttot, hdv, 64, true) || !s_ok)
     return cudaErrorInvalidValue;
   // gate and output tiles: [Ttot rows][H*dv] bf16 (maps only built when used)
   std::memset(&mg, 0, sizeof(mg));
@@ -2140,8 +2165,8 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
   op.nch = (L.T + L.chunk - 1) / L.chunk;
   op.nclusters = 1;
   op.shift = 1;
-  // the compact kernel has neither the anti-causal mode nor accumulation
-  if (op.rb == 1 && dk <= 128 && dv <= 256 && !anti && !acc_out) {
+  // the compact kernel has neither the anti-causal mode, accumulation nor transposed reads
+  if (op.rb == 1 && dk <= 128 && dv <= 256 && !anti && !acc_out && !sr.transposed) {
     // one-block chunks: the compact kernel, two CTAs per SM, d_v in parts of <= 128
     op.parts = dv > 128 ? 2 : 1;
     const int NVc = dv / op.parts;
@@ -2178,6 +2203,17 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
 }
 
 }  // namespace
+
+cudaError_t launch_to_f16(const void* src, void* dst, long long n, unsigned* err, cudaStream_t s) {
+  if (n % 8 != 0) return cudaErrorInvalidValue;
+  const long long n16 = n / 8;
+  if (n16 == 0) return cudaSuccess;
+  const long long want = (n16 + 511) / 512;
+  const long long cap = static_cast<long long>(sm_count()) * 8;
+  const int blocks = static_cast<int>(want < cap ? want : cap);
+  v16_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16, err);
+  return cudaGetLastError();
+}
 
 bool parallel_tc_supported(int dk, int dv) {
   return (dk == 64 || dk == 128 || dk == 256) &&
@@ -2220,7 +2256,7 @@ cudaError_t launch_parallel_tc(const void* q, const void* k, const void* v, void
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_output_pass(q, k, L, false, o, o_t, nullptr, DType::BF16, nullptr, nullptr, 0.f,
-                            false, ws, H, dk, dv, dec, err, s, false, false);
+                            false, ws, H, dk, dv, dec, err, s, false, false, StateRead());
 }
 
 }  // namespace ret

@@ -116,6 +116,14 @@ bool chunkwise_tc_supported(int dk, int dv, int chunk);
 // One bounded wait that is never satisfied (failure-detection self-test).
 cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t s);
 int chunkwise_tc_chunk(int chunk, int dv);  // chunk length the kernels evaluate
+// The output pass may read the carried state transposed: the slots then hold
+// another pass's state [dv rows][stored_dv columns] (fp16) and this pass uses
+// its columns col0 .. col0+dk-1 (the backward's dK pass on the dV pass's states).
+struct StateRead {
+  bool transposed = false;
+  int col0 = 0;
+  int stored_dv = 0;
+};
 cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const void* v,
                                 const SeqLayout& L, const float* state_in, bool has_state_in,
                                 float* state_out,
@@ -123,7 +131,10 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
                                 const float* gn_w, const float* gn_b, float eps, bool gated,
                                 ChunkWorkspace ws, int H, int dk, int dv,
                                 const HeadDecay& dec, unsigned* err, cudaStream_t s,
-                                bool acc_out = false, bool anti = false);
+                                bool acc_out = false, bool anti = false,
+                                StateRead sr = StateRead());
+// bf16 -> fp16 copy of n elements (n a multiple of 8); |x| >= 2^16 raises kErrRange.
+cudaError_t launch_to_f16(const void* src, void* dst, long long n, unsigned* err, cudaStream_t s);
 
 // Parallel form on the tensor cores (bf16 inputs): an fp16 copy of v, then the
 // chunkwise output kernel with each sequence as a single chunk.
