@@ -246,17 +246,17 @@ def cpu_baseline(wl, budget_s=15.0):
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def traffic_from_profile():
+def traffic_from_profile(workload):
     """DRAM bytes per launch of the output kernel at the workload's full size,
     from the committed ncu figures (a small JSON file), only if they were taken
-    on the current kernel source."""
+    on this workload and on the current kernel source."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     try:
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
         sha = hashlib.sha256(open(TC_SOURCE, "rb").read()).hexdigest()
-        if d.get("source_sha256") != sha:
+        if d.get("source_sha256") != sha or d.get("workload") != workload:
             return None
         return float(d["dram_bytes_per_launch_full_size"])
     except (OSError, ValueError, KeyError, TypeError):
@@ -381,7 +381,7 @@ def run_headline(args, world, rank, pk, pk_kind):
     t_out = ms_out / 1e3
     peak_bw = pk["hbm_gbs"]
     peak_tf = pk["bf16_tflops"]
-    traffic = traffic_from_profile()
+    traffic = traffic_from_profile(wl.name)
     ach = flops_launch / t_out / 1e12
     roof = {"bound": "tensor", "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s",
             "frac": ach / peak_tf, "traffic": traffic,
