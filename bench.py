@@ -917,6 +917,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--backward-only", action="store_true", help="backward only (profiling)")
+    ap.add_argument("--parallel-only", action="store_true", help="parallel form only (profiling)")
     ap.add_argument("--no-rope", action="store_true")
     ap.add_argument("--no-rla", action="store_true")
     ap.add_argument("--no-parallel", action="store_true")
@@ -984,6 +985,13 @@ def main():
         bwd = run_backward(args, world, rank, pk, pk_kind)
         if rank == 0:
             print(json.dumps({"metric": METRIC, "backward": bwd, "n_gpus": world}), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    if args.parallel_only:
+        par = run_parallel(args, world, rank, pk, pk_kind)
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "parallel": par, "n_gpus": world}), flush=True)
         if world > 1:
             torch.distributed.destroy_process_group()
         return
