@@ -146,7 +146,8 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_con
   const uint32_t tmem = *tmem_hold;
 
   if (warp == 0) {
-    // ---------------- TMA producer: the state, 64 rows x 128 columns per stage ----------------
+    // ---------------- TMA producer: per item the q, k, v stage, then the state ----------------
+    // (64 rows x 128 columns per stage)
     if (lane == 0 && !*abort_flag) {
       tma_prefetch_desc(&tmS);
       tma_prefetch_desc(&tmQ);
