@@ -130,7 +130,10 @@ RET_API const char* retention_status_string(ret_status status);
  *     retention_check_device_error), then 128-row query tiles run against
  *     every causal 128-key block with the scores and decay formed in f32,
  *     rounded once to fp16 for the P V product, f32 accumulation.  Precision
- *     and range as the chunkwise tensor-core path.
+ *     and range as the chunkwise tensor-core path.  The workspace also holds
+ *     a tile counter (its last 256 bytes): tiles cost 1 to T/128 key blocks,
+ *     so the persistent kernel hands them out in a dynamic order.  Calls
+ *     that share one workspace must be ordered (one stream).
  *   - otherwise (float32 inputs, or bf16 with other head dims): CUDA cores,
  *     float32 arithmetic, dk and dv up to 256.
  * Supported: T >= 1; B*T*H*max(dk,dv) < 2^31.

@@ -563,6 +563,11 @@ struct OutParams {
   // pass's state [dv rows][stored columns]; this pass multiplies by the
   // columns s_col0 .. s_col0+dk-1 of it, as a K-major operand
   int s_kmajor, s_col0;
+  // dynamic tile order (dyn): each cluster takes its next tile from a global
+  // counter (zeroed before the launch), in the static order's sequence of
+  // tiles; the fetch is made once per cluster and handed to every role
+  int dyn;         // selects the kernel instantiation (set on the host)
+  int* tile_ctr;
   int H, dk, dv;
   int rb;                      // 128-row blocks per chunk
   int parts;                   // d_v parts (cluster size)
@@ -621,7 +626,46 @@ struct OutTile {
 // and with it the tile's cost, rotates from round to round for every cluster.
 // Every role of both CTAs of the cluster walks the same sequence.
 struct TileWalk {
-  int k = 0;
+  int k = 0;   // static order: rounds taken
+  int n = 0;   // dynamic order: tiles taken from the cluster's queue
+  // Tile u of the fixed tile sequence; false if it holds no rows.
+  __device__ __forceinline__ bool decode(const OutParams& p, int u, OutTile& t) const {
+    // 32-bit index arithmetic: the host keeps the tile count below 2^31
+    const unsigned gh = static_cast<unsigned>(u) / static_cast<unsigned>(p.rb);
+    const unsigned slot = gh / static_cast<unsigned>(p.H);
+    t.h = static_cast<int>(gh - slot * static_cast<unsigned>(p.H));
+    // heaviest row block first: the last one (causal) or the first (anti-causal)
+    const int rr = static_cast<int>(static_cast<unsigned>(u) - gh * static_cast<unsigned>(p.rb));
+    t.r = p.anti ? rr : p.rb - 1 - rr;
+    t.slot = slot;
+    if (p.L.cu == nullptr) {
+      const unsigned sq = slot / static_cast<unsigned>(p.nch);
+      if (static_cast<int>(sq) >= p.L.nseq) return false;
+      t.si.s = static_cast<int>(sq);
+      t.si.c = static_cast<int>(slot - sq * static_cast<unsigned>(p.nch));
+      t.si.a = t.si.s * p.L.T;
+      t.si.b = t.si.a + p.L.T;
+      t.si.cs = t.si.a + t.si.c * p.L.chunk;
+      t.si.len = min(p.L.chunk, t.si.b - t.si.cs);
+      if (t.si.len <= 0) return false;
+    } else if (!slot_to_chunk(p.L, p.chunk_base, slot, t.si)) {
+      return false;
+    }
+    if (t.r * kRowsPerTile >= t.si.len) return false;
+    t.t0 = t.si.cs + t.r * kRowsPerTile;
+    t.nrows = min(kRowsPerTile, t.si.len - t.r * kRowsPerTile);
+    if (p.anti) {
+      t.kb0 = t.r;
+      t.nkb = (t.si.len + kKeysPerBlock - 1) / kKeysPerBlock - t.r;
+      t.inter = t.si.cs + t.si.len < t.si.b || p.has_state_in;   // a later chunk, or a state in
+    } else {
+      t.kb0 = 0;
+      t.nkb = t.r + 1;
+      t.inter = t.si.c > 0 || p.has_state_in;
+    }
+    return true;
+  }
+  // The static order: in round k cluster c takes tile k * nclusters + (c + k * shift) mod nclusters.
   __device__ __forceinline__ bool next(const OutParams& p, int cid, OutTile& t) {
     while (true) {
       const int base = k * p.nclusters;
@@ -629,41 +673,7 @@ struct TileWalk {
       const int u = base + static_cast<int>(static_cast<unsigned>(cid + k * p.shift) %
                                             static_cast<unsigned>(p.nclusters));
       ++k;
-      if (u >= p.ntiles) continue;
-      // 32-bit index arithmetic: the host keeps the tile count below 2^31
-      const unsigned gh = static_cast<unsigned>(u) / static_cast<unsigned>(p.rb);
-      const unsigned slot = gh / static_cast<unsigned>(p.H);
-      t.h = static_cast<int>(gh - slot * static_cast<unsigned>(p.H));
-      // heaviest row block first: the last one (causal) or the first (anti-causal)
-      const int rr = static_cast<int>(static_cast<unsigned>(u) - gh * static_cast<unsigned>(p.rb));
-      t.r = p.anti ? rr : p.rb - 1 - rr;
-      t.slot = slot;
-      if (p.L.cu == nullptr) {
-        const unsigned sq = slot / static_cast<unsigned>(p.nch);
-        if (static_cast<int>(sq) >= p.L.nseq) continue;
-        t.si.s = static_cast<int>(sq);
-        t.si.c = static_cast<int>(slot - sq * static_cast<unsigned>(p.nch));
-        t.si.a = t.si.s * p.L.T;
-        t.si.b = t.si.a + p.L.T;
-        t.si.cs = t.si.a + t.si.c * p.L.chunk;
-        t.si.len = min(p.L.chunk, t.si.b - t.si.cs);
-        if (t.si.len <= 0) continue;
-      } else if (!slot_to_chunk(p.L, p.chunk_base, slot, t.si)) {
-        continue;
-      }
-      if (t.r * kRowsPerTile >= t.si.len) continue;
-      t.t0 = t.si.cs + t.r * kRowsPerTile;
-      t.nrows = min(kRowsPerTile, t.si.len - t.r * kRowsPerTile);
-      if (p.anti) {
-        t.kb0 = t.r;
-        t.nkb = (t.si.len + kKeysPerBlock - 1) / kKeysPerBlock - t.r;
-        t.inter = t.si.cs + t.si.len < t.si.b || p.has_state_in;   // a later chunk, or a state in
-      } else {
-        t.kb0 = 0;
-        t.nkb = t.r + 1;
-        t.inter = t.si.c > 0 || p.has_state_in;
-      }
-      return true;
+      if (u < p.ntiles && decode(p, u, t)) return true;
     }
   }
 };
@@ -683,7 +693,7 @@ __device__ __forceinline__ bool epi_all(bool v) {
   return r != 0;
 }
 
-template <int DK, int NV>
+template <int DK, int NV, bool DYN>
 __global__ void __launch_bounds__(kThreads, 1)
 output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
@@ -711,6 +721,13 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   float* pow_tab = reinterpret_cast<float*>(smem + C::kOffMisc + 256);    // gamma^d, d < 128
   float* wgx = reinterpret_cast<float*>(smem + C::kOffMisc + 768);        // [128][2]
   float* xrecv = reinterpret_cast<float*>(smem + C::kOffMisc + 1792);     // [128][2]
+  // dynamic tile queue (ungated launches only, in place of xrecv): kDynQ tile
+  // indices, their full barriers (arrived by the fetcher) and, in the first
+  // CTA of the cluster, their empty barriers (arrived by every other role)
+  constexpr int kDynQ = 4;
+  int* dq = reinterpret_cast<int*>(smem + C::kOffMisc + 1792);
+  uint64_t* dq_full = reinterpret_cast<uint64_t*>(smem + C::kOffMisc + 1792 + 64);
+  uint64_t* dq_empty = dq_full + kDynQ;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int part = blockIdx.x % p.parts;
@@ -749,6 +766,12 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     mbar_init(drain, 1);
     mbar_init(bar_x, 1);                  // armed per tile with the partner's 1 KB
     mbar_init(bar_xack, kWgThreads);
+    if (DYN && !p.gated) {
+      for (int i = 0; i < kDynQ; ++i) {
+        mbar_init(&dq_full[i], 1);
+        mbar_init(&dq_empty[i], 2 + 3 * (p.parts - 1));
+      }
+    }
     *abort_flag = 0;
     if ((smem_u32(smem) & 1023u) != 0) {
       *abort_flag = 1;
@@ -764,11 +787,52 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_hold;
-  if (xchg) cluster_arrive_relaxed();    // barrier initialisation done (waited on before first use)
+  const bool dynq = DYN && !p.gated;    // the dynamic queue lives where xrecv would
+  const bool cl = p.parts > 1 && (p.gated || dynq);
+  if (cl) cluster_arrive_relaxed();      // barrier initialisation done (waited on before first use)
   bool cluster_waited = false;           // this thread has passed that first cluster barrier phase
 
   TileWalk walk;
   OutTile t;
+  const bool fetcher = cluster_ctarank() == 0;   // the cluster's first CTA fetches the tiles
+  // The next tile in the dynamic order, for one thread of a role: the fetcher
+  // (the first CTA's producer) takes it from the counter and publishes it;
+  // every other role waits for it. Returns the tile index (-1 at the end);
+  // *okr = false if a wait ran out.
+  auto dyn_take = [&](bool fetch, bool* okr) -> int {
+    const int slot = walk.n % kDynQ;
+    const uint32_t ph = (walk.n / kDynQ) & 1;
+    if (cl && !cluster_waited) {
+      cluster_wait();                    // the partner's barriers are initialised
+      cluster_waited = true;
+    }
+    int u = -1;
+    if (fetch) {
+      if (!mbar_wait(&dq_empty[slot], ph ^ 1, abort_flag, p.err)) { *okr = false; return -1; }
+      OutTile tt;
+      do {
+        u = atomicAdd(p.tile_ctr, 1);
+      } while (u < p.ntiles && !walk.decode(p, u, tt));
+      if (u >= p.ntiles) u = -1;
+      dq[slot] = u;
+      if (p.parts > 1) {
+        st_cluster_f32(cluster_addr(&dq[slot], 1u), __int_as_float(u));
+        mbar_arrive_cluster(cluster_addr(&dq_full[slot], 1u));
+      }
+      mbar_arrive(&dq_full[slot]);
+    } else {
+      if (!mbar_wait_cluster(&dq_full[slot], ph, abort_flag, p.err)) { *okr = false; return -1; }
+      u = dq[slot];
+    }
+    ++walk.n;
+    return u;
+  };
+  // a consumer role is done reading the queue slot it took last
+  auto dyn_release = [&]() {
+    const int slot = (walk.n - 1) % kDynQ;
+    if (fetcher) mbar_arrive(&dq_empty[slot]);
+    else mbar_arrive_cluster(cluster_addr(&dq_empty[slot], 0u));
+  };
 
   // Per tile, the ring units in the order the MMA consumes them (32 KB each):
   //   K(0), then for kb = 0..r: [K(kb+1) if kb < r], V(kb) keys 0-63, V(kb) keys 64-127
@@ -792,7 +856,15 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_arrive_expect_tx(&full[st], bytes);
         return smem + C::kOffStages + st * kOutStage;
       };
-      while (ok && walk.next(p, cid, t)) {
+      while (ok) {
+        if (dynq) {
+          const int u = dyn_take(fetcher, &ok);
+          if (u < 0) break;
+          if (!fetcher) dyn_release();
+          walk.decode(p, u, t);
+        } else if (!walk.next(p, cid, t)) {
+          break;
+        }
         // Q of this tile, once the previous tile's MMAs and epilogue are done with Q
         if (tq > 0 && !mbar_wait(q_free, (tq - 1) & 1, abort_flag, p.err)) { ok = false; break; }
         mbar_arrive_expect_tx(bar_q, C::kQBytes);
@@ -890,7 +962,15 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mma_commit(&empty[it % NST]);
         ++it;
       };
-      while (ok && walk.next(p, cid, t)) {
+      while (ok) {
+        if (dynq) {
+          const int u = dyn_take(false, &ok);
+          if (u < 0) break;
+          dyn_release();
+          walk.decode(p, u, t);
+        } else if (!walk.next(p, cid, t)) {
+          break;
+        }
         if (!mbar_wait(bar_q, tq & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         auto issue_qk = [&](int kb) -> bool {          // kb: the tile's kb-th key block
@@ -989,9 +1069,25 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     int tq = 0, sblk = 0, git = 0;                    // git: ring position, as the producer counts
     bool ok = true;
     float pmax = 0.f;                                 // largest |P| and |decayed q| formed
-    while (walk.next(p, cid, t)) {
+    while (true) {
+      int u = 0;
+      bool got = true;
+      if (dynq) {
+        bool wok = true;
+        u = dyn_take(false, &wok);
+        got = warp_all(wok);
+      } else {
+        got = walk.next(p, cid, t);              // the same for every thread
+        u = got ? 0 : -1;
+        got = true;
+      }
       // uniform over the 256 epilogue threads: the named barriers below stay matched
-      if (!epi_all(ok && !*abort_flag)) break;
+      if (!epi_all(got && ok && !*abort_flag)) break;
+      if (u < 0) break;                          // every thread read the same index
+      if (dynq) {
+        if (et == 0) dyn_release();              // all 256 threads have read the slot
+        walk.decode(p, u, t);
+      }
       const int r = t.r;
       const int i = r * kRowsPerTile + row;            // row within the chunk
       const bool staged = io_staged(t);
@@ -1334,7 +1430,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
     if (pmax > kF16Max) raise_error(p.err, kErrRange);
   }
-  if (xchg) {
+  if (cl) {
     if (!cluster_waited) cluster_wait();
     cluster_arrive();
     cluster_wait();        // the partner has made its last remote access here
@@ -1904,7 +2000,8 @@ cudaError_t launch_out(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
                        OutParams op, cudaStream_t s) {
   using C = OutCfg<DK, NV>;
   static_assert(C::kSmem <= 232448, "shared memory budget");
-  auto kern = output_kernel<DK, NV>;
+  // the dynamic tile order is its own instantiation: the static walk keeps its code
+  auto kern = op.dyn ? output_kernel<DK, NV, true> : output_kernel<DK, NV, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
@@ -1921,11 +2018,11 @@ cudaError_t launch_out(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   cfg.numAttrs = 1;
   // persistent grid: as many clusters as can be resident at once (one CTA
   // per SM), queried once per device and cluster size
-  static int resident[64][3] = {};
+  static int resident[64][3][2] = {};
   int dev = 0;
   e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int& ncl = resident[dev & 63][op.parts];
+  int& ncl = resident[dev & 63][op.parts][op.dyn ? 1 : 0];
   if (ncl == 0) {
     cfg.gridDim = dim3(static_cast<unsigned>(op.parts), 1, 1);
     int n = 0;
@@ -1990,7 +2087,8 @@ cudaError_t launch_out_c(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
 // per thread.
 __global__ void __launch_bounds__(256) v16_kernel(const uint4* __restrict__ v,
                                                    uint4* __restrict__ v16, long long n16,
-                                                   unsigned* err) {
+                                                   unsigned* err, int* tile_ctr) {
+  if (tile_ctr && blockIdx.x == 0 && threadIdx.x == 0) *tile_ctr = 0;   // for the next kernel
   uint32_t amax = 0;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -2018,7 +2116,7 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
                                DType g_t, const float* gn_w, const float* gn_b, float eps,
                                bool gated, ChunkWorkspace ws, int H, int dk, int dv,
                                const HeadDecay& dec, unsigned* err, cudaStream_t s,
-                               bool acc_out, bool anti, StateRead sr);
+                               bool acc_out, bool anti, StateRead sr, int* tile_ctr);
 
 }  // namespace
 
@@ -2093,7 +2191,7 @@ cudaError_t launch_chunkwise_tc(int phases, const void* q, const void* k, const 
   }
   if (e != cudaSuccess || L.Ttot == 0 || !(phases & 2)) return e;
   return launch_output_pass(q, k, L, has_state_in, out, out_t, g, g_t, gn_w, gn_b, eps, gated,
-                            ws, H, dk, dv, dec, err, s, acc_out, anti, sr);
+                            ws, H, dk, dv, dec, err, s, acc_out, anti, sr, nullptr);
 }
 
 namespace {
@@ -2108,7 +2206,7 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
                                DType g_t, const float* gn_w, const float* gn_b, float eps,
                                bool gated, ChunkWorkspace ws, int H, int dk, int dv,
                                const HeadDecay& dec, unsigned* err, cudaStream_t s,
-                               bool acc_out, bool anti, StateRead sr) {
+                               bool acc_out, bool anti, StateRead sr, int* tile_ctr) {
   if (L.chunk < kRowsPerTile || L.chunk % kRowsPerTile != 0) return cudaErrorInvalidValue;
   // accumulation: float32 and ungated (the persistent kernel)
   if (acc_out && (out_t != DType::F32 || gated)) return cudaErrorInvalidValue;
@@ -2138,6 +2236,8 @@ cudaError_t launch_output_pass(const void* q, const void* k, const SeqLayout& L,
   op.acc_out = acc_out ? 1 : 0;
   op.anti = anti ? 1 : 0;
   op.s_kmajor = sr.transposed ? 1 : 0;
+  op.dyn = (tile_ctr != nullptr && !gated) ? 1 : 0;
+  op.tile_ctr = tile_ctr;
   op.s_col0 = sr.col0;
   if (ws.v16 == nullptr) return cudaErrorInvalidValue;   // written by the state pass
   // a transposed read: the slots hold [dv rows][stored_dv] (dv <= 256, one part)
@@ -2211,7 +2311,8 @@ cudaError_t launch_to_f16(const void* src, void* dst, long long n, unsigned* err
   const long long want = (n16 + 511) / 512;
   const long long cap = static_cast<long long>(sm_count()) * 8;
   const int blocks = static_cast<int>(want < cap ? want : cap);
-  v16_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16, err);
+  v16_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16, err,
+                                    nullptr);
   return cudaGetLastError();
 }
 
@@ -2224,7 +2325,8 @@ size_t parallel_tc_workspace_bytes(int B, int T, int H, int dk, int dv) {
   // the fp16 copy of v, at least B*H*d_k rows of d_v long: the output pass
   // also builds its (never read) state-slot map over this buffer
   const long long rows = static_cast<long long>(B) * (T > dk ? T : dk) * H;
-  return (static_cast<size_t>(rows) * dv * 2 + 255) & ~static_cast<size_t>(255);
+  // then 256 bytes for the tile counter of the dynamic tile order
+  return ((static_cast<size_t>(rows) * dv * 2 + 255) & ~static_cast<size_t>(255)) + 256;
 }
 
 cudaError_t launch_parallel_tc(const void* q, const void* k, const void* v, void* o, DType o_t,
@@ -2251,12 +2353,15 @@ cudaError_t launch_parallel_tc(const void* q, const void* k, const void* v, void
   const long long want = (n16 + 511) / 512;
   const long long cap = static_cast<long long>(sm_count()) * 8;
   const int blocks = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
+  int* ctr = reinterpret_cast<int*>(static_cast<char*>(workspace) +
+                                    parallel_tc_workspace_bytes(B, T, H, dk, dv) - 256);
   v16_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(workspace),
-                                    n16, err);
+                                    n16, err, ctr);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  // rows of a sequence cost 1 .. T/128 key blocks: the tiles go out in a dynamic order
   return launch_output_pass(q, k, L, false, o, o_t, nullptr, DType::BF16, nullptr, nullptr, 0.f,
-                            false, ws, H, dk, dv, dec, err, s, false, false, StateRead());
+                            false, ws, H, dk, dv, dec, err, s, false, false, StateRead(), ctr);
 }
 
 }  // namespace ret

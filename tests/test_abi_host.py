@@ -74,7 +74,8 @@ def test_parallel_rejects_bad_arguments():
     assert f(*args(dk=300)) == ops.RET_ERR_UNSUPPORTED
     # bf16 at tensor-core head dims needs the workspace: missing, short or misaligned
     need = L.retention_parallel_workspace_size(ops.RET_BF16, 1, 8, 2, 128, 256)
-    assert need == 1 * 128 * 2 * 256 * 2     # fp16 copy of v, max(T, d_k) rows per sequence
+    # fp16 copy of v, max(T, d_k) rows per sequence, then 256 bytes for the tile counter
+    assert need == 1 * 128 * 2 * 256 * 2 + 256
     bf = dict(dt=ops.RET_BF16, dk=128, dv=256)
     assert f(*args(**bf)) == ops.RET_ERR_WORKSPACE
     assert f(*args(**bf, ws=FAKE_WS, nb=need - 256)) == ops.RET_ERR_WORKSPACE
@@ -83,7 +84,7 @@ def test_parallel_rejects_bad_arguments():
     # float32 and non-tensor-core bf16 shapes need none
     assert L.retention_parallel_workspace_size(ops.RET_F32, 1, 8, 2, 128, 256) == 0
     assert L.retention_parallel_workspace_size(ops.RET_BF16, 1, 8, 2, 16, 16) == 0
-    assert L.retention_parallel_workspace_size(ops.RET_BF16, 2, 1000, 3, 64, 512) == 2 * 1000 * 3 * 512 * 2
+    assert L.retention_parallel_workspace_size(ops.RET_BF16, 2, 1000, 3, 64, 512) == 2 * 1000 * 3 * 512 * 2 + 256
 
 
 def test_workspace_size_query():
