@@ -1043,7 +1043,15 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           if (!ok) break;
         }
         mma_commit(bar_o);
-        if (io_staged(t)) it += kGS;           // the gate stages belong to the epilogue
+        if (io_staged(t)) {
+          // The gate stages belong to the epilogue, but this thread still waits
+          // for them to land: its waits then stay in ring order, so a later
+          // wait on one of these stages cannot match the parity of the phase
+          // one lap older while the gate load is still in flight.
+          for (int gs = 0; gs < kGS && ok; ++gs, ++it)
+            ok = mbar_wait(&full[it % NST], (it / NST) & 1, abort_flag, p.err);
+          if (!ok) break;
+        }
         sblk += t.nkb;
         ++tq;
       }
