@@ -189,8 +189,12 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
   const int s = p.order ? p.order[rank] : rank;
   const int m = zz % mblocks, part = zz / mblocks;
   const int kboxes = p.dk >= 128 ? 2 : 1;        // 64-column K boxes loaded per stage
-  // the fp16 copy of this CTA's value columns leaves from the V stages (first d_k block only)
-  const bool v16_out = p.write_v16 && m == 0;
+  // the fp16 copy of this CTA's value columns leaves from the V stages; the d_k
+  // blocks of a column part split its 64-column boxes, so no CTA of the pair
+  // holds its stages longer than the other
+  const int v16_per = ((NS / 64) + mblocks - 1) / mblocks;    // boxes stored per d_k block
+  const int v16_b0 = m * v16_per, v16_b1 = min((m + 1) * v16_per, NS / 64);
+  const bool v16_out = p.write_v16 && v16_b0 < v16_b1;
   const SeqLayout& L = p.L;
   int a, b;
   seq_bounds(L, s, a, b);
@@ -518,7 +522,7 @@ state_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
           if (!mbar_wait(&kready[st], (it / NSTG) & 1, abort_flag, p.err)) { ok = false; break; }
           const int y = tok0 + sb * kStTok;
           uint8_t* stage = smem + st * kStage;
-          for (int bx = 0; bx < NS / 64; ++bx)
+          for (int bx = v16_b0; bx < v16_b1; ++bx)
             tma_store_2d(&tmV16, stage + kKBytes + bx * kBox, h * p.dv + NS * part + 64 * bx, y);
           tma_store_commit();
           tma_store_wait_read();
