@@ -111,6 +111,13 @@ typedef struct {
 /* ABI version of the loaded library (RETENTION_ABI_VERSION at build time). */
 RET_API int retention_abi_version(void);
 
+/* SHA-256, as 64 hex digits, of the sources the library was built from (the
+ * kernel sources and this header), or "unknown" for a build that did not pass
+ * it.  Static string, owned by the library.  The Python binding compares it
+ * with the source tree next to it and refuses a library built from other
+ * sources. */
+RET_API const char* retention_source_sha(void);
+
 /* Static, human-readable name of a status code. */
 RET_API const char* retention_status_string(ret_status status);
 

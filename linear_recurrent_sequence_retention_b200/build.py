@@ -38,6 +38,18 @@ def nvcc():
     raise RuntimeError("nvcc not found; CUDA toolkit 12.8+ is required to build libretention")
 
 
+def source_sha():
+    """SHA-256 (hex) of the kernel sources and the public header, as the library embeds it."""
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
+                   + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")))
+    for p in files:
+        h.update(os.path.basename(p).encode() + b"\0")
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def _digest(src, extra_flags):
     h = hashlib.sha256()
     h.update(" ".join(NVCC_FLAGS + extra_flags).encode())
@@ -72,8 +84,16 @@ def build(verbose=False, extra_flags=()):
     os.makedirs(BUILD, exist_ok=True)
     extra = list(extra_flags)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    # api.cu carries the sources' hash (retention_source_sha), so a library
+    # built from other sources is refused by the binding
+    sha_flag = ["-DRET_SOURCE_SHA=" + source_sha()]
+
+    def one(src):
+        flags = extra + (sha_flag if os.path.basename(src) == "api.cu" else [])
+        return _compile(src, flags, verbose)
+
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, extra, verbose), srcs))
+        objs = list(ex.map(one, srcs))
     tmp = LIB + ".tmp"
     cmd = [nvcc()] + ARCH + ["-shared", "-o", tmp] + objs
     if verbose:

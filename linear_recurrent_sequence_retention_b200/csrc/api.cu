@@ -132,6 +132,14 @@ extern "C" {
 
 int retention_abi_version(void) { return RETENTION_ABI_VERSION; }
 
+// The build passes the SHA-256 of the sources as RET_SOURCE_SHA (a bare hex token).
+#ifndef RET_SOURCE_SHA
+#define RET_SOURCE_SHA unknown
+#endif
+#define RET_STR2(x) #x
+#define RET_STR(x) RET_STR2(x)
+const char* retention_source_sha(void) { return RET_STR(RET_SOURCE_SHA); }
+
 const char* retention_status_string(ret_status s) {
   switch (s) {
     case RET_OK: return "RET_OK";

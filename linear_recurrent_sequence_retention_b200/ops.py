@@ -15,6 +15,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIBRARY_PATH = os.path.join(_HERE, "libretention.so")
+_IN_TREE_LIBRARY = LIBRARY_PATH
 
 RET_OK = 0
 RET_ERR_INVALID_ARG = 1
@@ -33,6 +34,7 @@ STATIC_WORKSPACE_BYTES = 32 << 20
 
 EXPORTED = (
     "retention_abi_version",
+    "retention_source_sha",
     "retention_status_string",
     "retention_parallel_workspace_size",
     "retention_parallel_fwd",
@@ -72,8 +74,21 @@ class NormGate(ctypes.Structure):
 _lib = None
 
 
+def _check_sources(L):
+    """Refuse the in-tree library if it was built from sources other than the tree's."""
+    if (os.path.abspath(LIBRARY_PATH) != _IN_TREE_LIBRARY
+            or not os.path.isdir(os.path.join(_HERE, "csrc"))):
+        return
+    from . import build
+    want, got = build.source_sha(), L.retention_source_sha().decode()
+    if got != want:
+        raise RuntimeError(
+            f"{LIBRARY_PATH} was built from other sources (library {got[:12]}, tree "
+            f"{want[:12]}): rebuild it with `python -m linear_recurrent_sequence_retention_b200.build`")
+
+
 def lib():
-    """The loaded library (loads it on first use; raises if it is not built)."""
+    """The loaded library (loads it on first use; raises if it is not built or is stale)."""
     global _lib
     if _lib is not None:
         return _lib
@@ -85,6 +100,9 @@ def lib():
     vp, ci, cd = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_double)
     L.retention_abi_version.restype = ci
     L.retention_abi_version.argtypes = []
+    L.retention_source_sha.restype = ctypes.c_char_p
+    L.retention_source_sha.argtypes = []
+    _check_sources(L)
     L.retention_status_string.restype = ctypes.c_char_p
     L.retention_status_string.argtypes = [ci]
     L.retention_parallel_workspace_size.restype = ctypes.c_size_t

@@ -40,6 +40,17 @@ def test_library_exports_every_declared_symbol():
     assert set(ops.EXPORTED) <= set(declared_symbols())
 
 
+def test_library_is_built_from_this_tree(monkeypatch):
+    """The library embeds the hash of its sources; the binding refuses another tree's build."""
+    ops, L = _lib()
+    from linear_recurrent_sequence_retention_b200 import build
+    sha = L.retention_source_sha().decode()
+    assert re.fullmatch(r"[0-9a-f]{64}", sha) and sha == build.source_sha()
+    monkeypatch.setattr(build, "source_sha", lambda: "0" * 64)
+    with pytest.raises(RuntimeError, match="built from other sources"):
+        ops._check_sources(L)
+
+
 def test_abi_version_and_status_strings():
     ops, L = _lib()
     assert L.retention_abi_version() == 3
