@@ -170,8 +170,12 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_con
             tma_load_2d(dst + 2 * p.Tn * p.dk * 2 + vbx * p.Tn * 256, &tmV, &full[st], h * p.dv + 128 * vbx, y0);
           ++it;
         }
+        // row-block major: the d_v blocks of the same 128 state rows go out one
+        // after another, so every 2 KB row of the state streams whole
+        for (int mb = 0; mb < nm && ok; ++mb)
         for (int b = 0; b < nb && ok; ++b) {
-          for (int q = 0; q < nq; ++q, ++it) {
+          for (int q2 = 0; q2 < 2; ++q2, ++it) {
+            const int q = 2 * mb + q2;
             const int st = it % kDtStages;
             if (!mbar_wait(&empty[st], ((it / kDtStages) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
             mbar_arrive_expect_tx(&full[st], kDtStage);
@@ -202,8 +206,8 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_con
         if (!mbar_wait(pro_full, nitem & 1, abort_flag, p.err)) { ok = false; break; }
         if (nitem > 0 && !mbar_wait(do_free, (nitem - 1) & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
-        for (int b = 0; b < nb && ok; ++b) {
-          for (int mb = 0; mb < nm && ok; ++mb, ++ndu) {
+        for (int mb = 0; mb < nm && ok; ++mb) {
+          for (int b = 0; b < nb && ok; ++b, ++ndu) {
             const int u = ndu & 1;
             if (ndu >= 2 && !mbar_wait(&du_free[u], ((ndu >> 1) + 1) & 1, abort_flag, p.err)) { ok = false; break; }
             tc_fence_after();
@@ -252,6 +256,7 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_con
     const int wt = threadIdx.x - 64;        // 0..255
     const bool store_leader = quad == 2 * set && half == 0 && lane == 0;
     int it = 0, ndu = 0, nitem = 0;
+    int pend_st = -1;      // (store leader) the item's last stage, released after the outputs
     bool ok = true;
     for (int item = blockIdx.x; item < p.nitems; item += gridDim.x, ++nitem) {
       // uniform over the 256 workers: the named barriers below stay matched
@@ -424,8 +429,8 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_con
 
       // stages: S' = gamma^Tn S + dS in place, then back to global memory
       const float gT = dg.pow(p.Tn);
-      for (int b = 0; b < nb; ++b) {
-        for (int mb = 0; mb < nm; ++mb, ++ndu) {
+      for (int mb = 0; mb < nm; ++mb) {
+        for (int b = 0; b < nb; ++b, ++ndu) {
           const int u = ndu & 1;
           for (int q2 = 0; q2 < 2; ++q2, ++it) {
             const int q = 2 * mb + q2;
@@ -474,8 +479,12 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_con
               for (int c = 0; c < 4; ++c)
                 tma_store_2d(&tmS, stg + c * kDtBox, 128 * b + 32 * c, item * p.dk + 64 * q);
               tma_store_commit();
-              tma_store_wait_read();
-              mbar_arrive(&empty[st]);
+              if (b == nb - 1 && mb == nm - 1) {
+                pend_st = st;      // its store reads while the outputs are formed
+              } else {
+                tma_store_wait_read();
+                mbar_arrive(&empty[st]);
+              }
             }
           }
         }
@@ -509,6 +518,11 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_con
         }
       } else {
         ok = false;
+      }
+      if (pend_st >= 0) {
+        tma_store_wait_read();
+        mbar_arrive(&empty[pend_st]);
+        pend_st = -1;
       }
       tc_fence_before();
       __syncwarp();
