@@ -174,9 +174,10 @@ RET_API size_t retention_chunkwise_workspace_size(ret_dtype in_dtype, int chunk,
 /*
  * The chunk length the chunkwise kernels evaluate for a requested `chunk`
  * (every chunk length gives the same result, see retention_chunkwise_fwd):
- * `chunk` itself for float32 inputs; for bf16 inputs at least 128 tokens, and
- * at least 256 when dv >= 256.  Returns 0 for unsupported arguments.  No
- * counterpart on the pages: it lets a caller count the work the kernels do.
+ * `chunk` itself for float32 inputs; for bf16 inputs 128 tokens, or 256 when
+ * dv >= 256, whatever chunk was requested (the length the tensor-core kernels
+ * run fastest at).  Returns 0 for unsupported arguments.  No counterpart on
+ * the pages: it lets a caller count the work the kernels do.
  */
 RET_API int retention_chunkwise_executed_chunk(ret_dtype in_dtype, int chunk, int dk, int dv);
 
@@ -208,9 +209,9 @@ RET_API int retention_chunkwise_executed_chunk(ret_dtype in_dtype, int chunk, in
  *   in_dtype RET_BF16: tensor-core kernels (tcgen05, TMEM accumulators), dk in
  *          {64, 128, 256}, dv in {64, 128, 256, 512}, chunk in
  *          {64, 128, 256, 512}; other bf16 shapes return
- *          RET_ERR_UNSUPPORTED.  Chunks shorter than 128 tokens (256
- *          when dv >= 256) are evaluated as chunks of that length, which
- *          yields the same result.
+ *          RET_ERR_UNSUPPORTED.  Every requested chunk is evaluated as
+ *          chunks of 128 tokens (256 when dv >= 256), which yields the same
+ *          result up to rounding (retention_chunkwise_executed_chunk).
  *   out dtype RET_F32 or RET_BF16; H <= 64; T*H*max(dk,dv) < 2^31.
  * Precision of the bf16 path: q and k enter the MMAs as they are, v as its
  *   fp16 value (exact inside fp16's range); the decayed scores, the decayed

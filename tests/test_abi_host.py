@@ -231,6 +231,8 @@ def test_chunkwise_executed_chunk():
     assert L.retention_chunkwise_executed_chunk(ops.RET_F32, 1, 256, 256) == 1
     assert L.retention_chunkwise_executed_chunk(ops.RET_BF16, 64, 128, 128) == 128
     assert L.retention_chunkwise_executed_chunk(ops.RET_BF16, 128, 128, 256) == 256
-    assert L.retention_chunkwise_executed_chunk(ops.RET_BF16, 512, 256, 512) == 512
+    assert L.retention_chunkwise_executed_chunk(ops.RET_BF16, 512, 256, 512) == 256
+    assert L.retention_chunkwise_executed_chunk(ops.RET_BF16, 512, 128, 128) == 128
+    assert L.retention_chunkwise_executed_chunk(ops.RET_BF16, 256, 64, 128) == 128
     assert L.retention_chunkwise_executed_chunk(ops.RET_BF16, 96, 128, 128) == 0     # unsupported chunk
     assert L.retention_chunkwise_executed_chunk(ops.RET_F32, 0, 16, 16) == 0        # invalid chunk
