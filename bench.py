@@ -777,7 +777,7 @@ def rope_forward_ab(args, world, rank):
     the rotary pass over q and k, then the two chunkwise passes), and the
     share of the rotary pass in it."""
     from linear_recurrent_sequence_retention_b200 import ops
-    wl = W.WORKLOADS[HEADLINE]
+    wl = W.WORKLOADS[HEADLINE_6P7B]          # whatever --workload times
     dev = torch.device("cuda")
     B, T, H, dk, dv, C = wl.B, wl.T, wl.H, wl.dk, wl.dv, wl.chunk
     q, k, v, g = W.make_qkvg(B, T, H, dk, dv, "bf16", seed=rank, gate=True, device=dev)
