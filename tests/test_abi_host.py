@@ -113,6 +113,27 @@ def test_workspace_size_query():
     assert ws(0, 16, 1, 64, 2, 300, 16, 0) == 0          # fp32 path: dk <= 256
 
 
+def test_tensor_core_workspace_layout():
+    """bf16: meta words | fp16 state per executed chunk | fp16 copy of v, each rounded to 256 B;
+    the executed chunk is 128 tokens, or 256 when dv >= 256, whatever chunk was asked for."""
+    ops, L = _lib()
+    ws = L.retention_chunkwise_workspace_size
+    r256 = lambda b: (b + 255) // 256 * 256
+
+    def expect(B, T, H, dk, dv, nseq=0):
+        ce = 256 if dv >= 256 else 128
+        ttot = T if nseq else B * T
+        slots = (ttot + ce - 1) // ce + nseq if nseq else B * ((T + ce - 1) // ce)
+        nmeta = nseq if nseq else B
+        return (r256(4 * (2 * nmeta + 1)) + r256(slots * H * dk * dv * 2)
+                + r256(ttot * H * dv * 2))
+    for chunk in (64, 128, 256, 512):
+        assert ws(1, chunk, 2, 8192, 16, 256, 512, 0) == expect(2, 8192, 16, 256, 512)
+        assert ws(1, chunk, 4, 2048, 8, 128, 256, 0) == expect(4, 2048, 8, 128, 256)
+        assert ws(1, chunk, 3, 1000, 2, 64, 128, 0) == expect(3, 1000, 2, 64, 128)
+    assert ws(1, 64, 1, 550655, 8, 128, 128, 64) == expect(1, 550655, 8, 128, 128, nseq=64)
+
+
 def test_chunkwise_rejects_bad_arguments():
     ops, L = _lib()
     f = L.retention_chunkwise_fwd
