@@ -171,7 +171,8 @@ decode_multi_tc_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_con
           ++it;
         }
         // row-block major: the d_v blocks of the same 128 state rows go out one
-        // after another, so every 2 KB row of the state streams whole
+        // after another, so the four 512-byte pieces of each 2 KB state row are
+        // fetched two stages apart (four in column-block order)
         for (int mb = 0; mb < nm && ok; ++mb)
         for (int b = 0; b < nb && ok; ++b) {
           for (int q2 = 0; q2 < 2; ++q2, ++it) {
