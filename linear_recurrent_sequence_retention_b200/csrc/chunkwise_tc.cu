@@ -135,7 +135,7 @@ struct StateParams {
   const float* state_in;
   float* state_out;
   int H, dk, dv;
-  int write_v16;                     // the CTAs of the first d_k block store the fp16 copy of v
+  int write_v16;                     // store the fp16 copy of v (the d_k blocks split its columns)
   // anti-causal mode: the chunks are walked last to first and each carries the
   // state of everything after it, F_(c-1) = gamma^L F_c + sum_j gamma^(j+1) k_j^T v_j
   int anti;
