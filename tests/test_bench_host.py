@@ -72,3 +72,32 @@ def test_cross_rank_reductions_gloo():
     mp.start_processes(_reduce_worker, args=(2, _free_port(), out), nprocs=2, join=True,
                        start_method="spawn")
     assert out[0] == (2.0, 20.0) and out[1] == (2.0, 20.0)
+
+
+def test_traffic_figure_is_keyed_to_workload_and_kernel_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed counters only for the workload they were
+    taken on and while the kernel source still hashes to the recorded value."""
+    sys.path.insert(0, ROOT)
+    import hashlib
+    import bench
+    src = tmp_path / "kernel.cu"
+    src.write_text("// kernel source\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()
+    fig = tmp_path / "traffic.json"
+    fig.write_text(json.dumps({"workload": "wl_a", "source_sha256": sha,
+                               "dram_bytes_per_launch_full_size": 123}))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(fig))
+    monkeypatch.setattr(bench, "TC_SOURCE", str(src))
+    assert bench.traffic_from_profile("wl_a") == 123.0
+    assert bench.traffic_from_profile("wl_b") is None          # another workload
+    src.write_text("// kernel source, changed\n")
+    assert bench.traffic_from_profile("wl_a") is None          # the kernel changed since
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
+    assert bench.traffic_from_profile("wl_a") is None
+
+
+def test_committed_traffic_figure_matches_the_current_kernel():
+    """The figure under profiles/ belongs to the kernel source in the tree."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.traffic_from_profile(bench.HEADLINE_6P7B) is not None
